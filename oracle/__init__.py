@@ -1,0 +1,21 @@
+"""CPU oracle for the token-sparse decode step (test infrastructure only).
+
+Plain float64 numpy restatement of what the decode step computes.  Only the
+tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline and
+reference legs may import it; the product path never does.
+"""
+
+from .reference import (  # noqa: F401
+    rope,
+    dominant_dims,
+    tip_scores,
+    select_top,
+    attend,
+    focused_attention,
+    stream_positions,
+    dense_positions,
+    decode_row,
+    decode_step,
+    shared_index_step,
+    tie_band_check,
+)

@@ -1,0 +1,275 @@
+"""Float64 CPU oracle of one token-sparse decode step.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or
+executes this file: only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference legs do.  It shares no code with the CUDA
+path (no kernels, headers, tables or helpers); both sides only read the same
+seeded bf16 inputs, which this module upcasts exactly to float64.
+
+Sources (web-page summaries of the methods; section names as printed):
+
+* FASA: Frequency-aware Sparse Attention -- §2.A (frequency chunks: RoPE splits
+  a d-dim vector into d/2 orthogonal 2-D subspaces), §2.B.1 (Token Importance
+  Predictor: a token's importance is the sum of the q.k contributions of the
+  head's dominant chunks I_dom only; the N_fac best tokens are kept), §2.B.2
+  (Focused Attention Computation: full-dimension attention over only those
+  tokens, keeping their original absolute positions), §2.C (FASA-C keeps the
+  whole cache on the GPU and reads only part of K).
+* Resumen Técnico: Autonomía de Cabezales (AoH) -- Metodología §4 (retrieval
+  heads keep the full global cache; streaming heads keep a fixed sink and a
+  recent window; GQA scores are aggregated per group).
+* El enrutamiento compartido entre capas ... (CLSA: You Only Index Once) --
+  "Cómo funciona CLSA" (an indexer layer scores the cache once, takes the
+  top-k once and hands the same index to every cross-decoder layer sharing
+  that cache).
+* Resumen Técnico: Por qué existen los patrones de atención (TAPPA) --
+  "Mecanismos de Patrones Predictibles" (RoPE's relative-position property:
+  shifting q and k together leaves their interaction unchanged).
+
+Readings where the pages are silent (each is listed in the design notes):
+
+* rotate-half RoPE layout: chunk c is the pair of dims (c, c + d/2), rotated by
+  angle p * theta^(-2c/d);
+* the importance score is computed on the rotated q and k, without the
+  1/sqrt(d) scale, and summed over the q heads of a GQA group;
+* ties in the top-N_fac go to the lower token position; selections are
+  returned in ascending position order; N_fac >= L selects every token;
+* the selection is the TIP top-N_fac only (no sink or window tokens added);
+* a streaming head attends to positions [0, min(S, L)) U [max(0, L - W), L);
+* q head h belongs to KV group h // G (contiguous GQA groups);
+* the shared index is one top-k per (sequence, KV head) on full-dimension
+  scores summed over the group, reused by every head of the group in every
+  layer.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM = 0, 1, 2
+
+
+# --------------------------------------------------------------------------------------
+# RoPE frequency chunks (FASA §2.A)
+# --------------------------------------------------------------------------------------
+
+def rope(x: np.ndarray, positions: Sequence[float], theta: float) -> np.ndarray:
+    """Rotate each row x[i] (float64 [n, d]) to absolute position positions[i].
+
+    Chunk c = dims (c, c + d/2) is turned by angle positions[i] * theta^(-2c/d).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    n, d = x.shape
+    C = d // 2
+    out = np.empty_like(x)
+    for c in range(C):
+        w = theta ** (-2.0 * c / d)
+        for i in range(n):
+            a = float(positions[i]) * w
+            ca, sa = math.cos(a), math.sin(a)
+            u, v = x[i, c], x[i, c + C]
+            out[i, c] = ca * u - sa * v
+            out[i, c + C] = sa * u + ca * v
+    return out
+
+
+def dominant_dims(idom: Sequence[int], head_dim: int) -> List[int]:
+    """The dims that the chunks in I_dom span: c and c + d/2 for every c."""
+    C = head_dim // 2
+    return [int(c) for c in idom] + [int(c) + C for c in idom]
+
+
+# --------------------------------------------------------------------------------------
+# Token Importance Predictor (FASA §2.B.1) with GQA group aggregation (AoH §4)
+# --------------------------------------------------------------------------------------
+
+def tip_scores(q_group: np.ndarray, keys: np.ndarray, idom: Sequence[int]) -> np.ndarray:
+    """Importance of every cached token for one KV group.
+
+    s[t] = sum over q heads h of the group, over chunks c in I_dom, of
+           q_h[c] k_t[c] + q_h[c + C] k_t[c + C].
+    q_group: [G, d]; keys: [L, d]; returns float64 [L].
+    """
+    q_group = np.asarray(q_group, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    d = keys.shape[1]
+    C = d // 2
+    s = np.zeros(keys.shape[0], dtype=np.float64)
+    for h in range(q_group.shape[0]):
+        for c in idom:
+            c = int(c)
+            s += q_group[h, c] * keys[:, c] + q_group[h, c + C] * keys[:, c + C]
+    return s
+
+
+# --------------------------------------------------------------------------------------
+# top-N_fac selection (FASA §2.B.1; CLSA's single top-k)
+# --------------------------------------------------------------------------------------
+
+def select_top(scores: np.ndarray, n: int) -> np.ndarray:
+    """Positions of the n highest scores, lower position first among equals; ascending output."""
+    scores = np.asarray(scores)
+    L = scores.shape[0]
+    n = min(int(n), L)
+    if n <= 0:
+        return np.zeros(0, dtype=np.int64)
+    pos = np.arange(L)
+    order = np.lexsort((pos, -scores.astype(np.float64)))  # primary: score desc; secondary: position asc
+    return np.sort(order[:n]).astype(np.int64)
+
+
+def tie_band_check(gpu_sel: np.ndarray, ref_scores: np.ndarray, n: int, rel: float = 1e-4) -> Tuple[bool, str]:
+    """Is ``gpu_sel`` a valid top-n of ``ref_scores`` up to the score band around the n-th score?
+
+    With s_n the n-th largest oracle score and beta = rel * max(|s_n|, mean|s|):
+    every token with s > s_n + beta must be selected, none with s < s_n - beta,
+    and exactly n tokens must be selected (each at most once).
+    """
+    s = np.asarray(ref_scores, dtype=np.float64)
+    L = s.shape[0]
+    n = min(int(n), L)
+    sel = np.asarray(gpu_sel, dtype=np.int64)
+    if sel.shape[0] != n:
+        return False, f"selected {sel.shape[0]} tokens, expected {n}"
+    if n == 0:
+        return True, ""
+    if np.any(sel < 0) or np.any(sel >= L):
+        return False, "position out of range"
+    if np.unique(sel).shape[0] != n:
+        return False, "duplicate positions"
+    if n == L:
+        return True, ""
+    s_n = np.sort(s)[::-1][n - 1]
+    beta = rel * max(abs(s_n), float(np.mean(np.abs(s))))
+    chosen = np.zeros(L, dtype=bool)
+    chosen[sel] = True
+    must = s > s_n + beta
+    never = s < s_n - beta
+    if np.any(must & ~chosen):
+        return False, f"{int(np.sum(must & ~chosen))} tokens above the band missing"
+    if np.any(never & chosen):
+        return False, f"{int(np.sum(never & chosen))} tokens below the band selected"
+    return True, ""
+
+
+# --------------------------------------------------------------------------------------
+# attention (FASA §2.B.2 focused attention; AoH §4 retrieval / streaming heads)
+# --------------------------------------------------------------------------------------
+
+def attend(q: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float) -> np.ndarray:
+    """softmax(scale * keys @ q) @ values, in float64; empty key set -> zeros."""
+    keys = np.asarray(keys, dtype=np.float64)
+    values = np.asarray(values, dtype=np.float64)
+    if keys.shape[0] == 0:
+        return np.zeros(values.shape[1], dtype=np.float64)
+    z = scale * (keys @ np.asarray(q, dtype=np.float64))
+    p = np.exp(z - np.max(z))
+    p /= np.sum(p)
+    return p @ values
+
+
+def focused_attention(q_group: np.ndarray, keys: np.ndarray, values: np.ndarray,
+                      sel: np.ndarray, scale: float) -> np.ndarray:
+    """Full-dimension attention of every q head of a group over the selected positions.
+
+    The selected keys are used exactly as cached (rotated at their original
+    positions); nothing is re-rotated.  Returns [G, d].
+    """
+    ks = np.asarray(keys, dtype=np.float64)[sel]
+    vs = np.asarray(values, dtype=np.float64)[sel]
+    return np.stack([attend(q_group[h], ks, vs, scale) for h in range(q_group.shape[0])])
+
+
+def stream_positions(L: int, sink: int, window: int) -> np.ndarray:
+    """Sink tokens [0, min(S, L)) together with the recent window [max(0, L - W), L)."""
+    keep = set(range(0, min(sink, L))) | set(range(max(0, L - window), L))
+    return np.array(sorted(keep), dtype=np.int64)
+
+
+def dense_positions(L: int) -> np.ndarray:
+    return np.arange(L, dtype=np.int64)
+
+
+# --------------------------------------------------------------------------------------
+# one decode step
+# --------------------------------------------------------------------------------------
+
+def decode_row(q_group: np.ndarray, keys: np.ndarray, values: np.ndarray, role: int, scale: float,
+               idom: Optional[Sequence[int]] = None, n_fac: int = 0,
+               sink: int = 0, window: int = 0) -> Dict[str, np.ndarray]:
+    """Decode-step output of one (sequence, KV group) by head role.
+
+    SPARSE: TIP scores -> top-N_fac -> focused attention; DENSE: attention over
+    the whole cache; STREAM: attention over the sink + recent window.
+    Returns {"out": [G, d], "sel": positions used, "scores": TIP scores or None}.
+    """
+    L = keys.shape[0]
+    if role == ROLE_SPARSE:
+        s = tip_scores(q_group, keys, idom)
+        sel = select_top(s, n_fac)
+        return {"out": focused_attention(q_group, keys, values, sel, scale), "sel": sel, "scores": s}
+    if role == ROLE_DENSE:
+        sel = dense_positions(L)
+    elif role == ROLE_STREAM:
+        sel = stream_positions(L, sink, window)
+    else:
+        raise ValueError(f"unknown role {role}")
+    return {"out": focused_attention(q_group, keys, values, sel, scale), "sel": sel, "scores": None}
+
+
+def decode_step(q: np.ndarray, k: np.ndarray, v: np.ndarray, offsets: Sequence[int], roles: Sequence[int],
+                scale: float, idom: Optional[np.ndarray] = None, n_fac_per_seq: Optional[Sequence[int]] = None,
+                sink: int = 0, window: int = 0,
+                rows: Optional[Sequence[Tuple[int, int]]] = None) -> Dict[Tuple[int, int], Dict[str, np.ndarray]]:
+    """Every (b, g) row of one decode step (or only ``rows``).
+
+    q: [B, Hq, d]; k, v: [T_total, Hkv, d]; offsets: [B + 1].
+    """
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    if rows is None:
+        rows = [(b, g) for b in range(B) for g in range(Hkv)]
+    res = {}
+    for b, g in rows:
+        o0, o1 = int(offsets[b]), int(offsets[b + 1])
+        res[(b, g)] = decode_row(
+            np.asarray(q[b, g * G:(g + 1) * G], dtype=np.float64),
+            np.asarray(k[o0:o1, g], dtype=np.float64), np.asarray(v[o0:o1, g], dtype=np.float64),
+            int(roles[g]), scale,
+            None if idom is None else idom[g], 0 if n_fac_per_seq is None else int(n_fac_per_seq[b]),
+            sink, window)
+    return res
+
+
+def shared_index_step(q_index: np.ndarray, q_layers: np.ndarray, k: np.ndarray, v: np.ndarray,
+                      offsets: Sequence[int], topk: int, scale: float,
+                      rows: Optional[Sequence[Tuple[int, int]]] = None) -> Dict[Tuple[int, int], Dict[str, np.ndarray]]:
+    """Shared-index cross-decoder stack: index once, reuse in every layer.
+
+    The indexer's full-dimension scores (every chunk, summed over the group's
+    q heads) give one top-k per (sequence, KV group); each layer l then runs
+    focused attention of its own q over those positions of the shared cache.
+    q_index: [B, Hq, d]; q_layers: [n_layers, B, Hq, d].
+    Returns {(b, g): {"sel", "scores", "out": [n_layers, G, d]}}.
+    """
+    n_layers, B, Hq, d = q_layers.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    all_chunks = list(range(d // 2))
+    if rows is None:
+        rows = [(b, g) for b in range(B) for g in range(Hkv)]
+    res = {}
+    for b, g in rows:
+        o0, o1 = int(offsets[b]), int(offsets[b + 1])
+        keys = np.asarray(k[o0:o1, g], dtype=np.float64)
+        vals = np.asarray(v[o0:o1, g], dtype=np.float64)
+        s = tip_scores(np.asarray(q_index[b, g * G:(g + 1) * G], dtype=np.float64), keys, all_chunks)
+        sel = select_top(s, topk)
+        out = np.stack([focused_attention(np.asarray(q_layers[l, b, g * G:(g + 1) * G], dtype=np.float64),
+                                          keys, vals, sel, scale) for l in range(n_layers)])
+        res[(b, g)] = {"sel": sel, "scores": s, "out": out}
+    return res

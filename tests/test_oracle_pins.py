@@ -1,0 +1,334 @@
+"""Pins of the float64 oracle to facts other than itself.
+
+Each test checks the oracle against a closed form, a hand-worked example, an
+independent library routine on a special case, an invariant of the mathematics
+or brute force on tiny inputs, so that a dropped term, a wrong sign, a wrong
+pairing of RoPE dims or a transposed operand fails at least one of them.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+from oracle.reference import ROLE_DENSE, ROLE_SPARSE, ROLE_STREAM
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_example.json")
+
+
+@pytest.fixture(scope="module")
+def hand():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------- RoPE chunks
+
+def test_rope_quarter_turn_closed_form():
+    # d = 2: a single chunk with frequency theta^0 = 1; position pi/2 turns (1, 0) into (0, 1).
+    out = oracle.rope(np.array([[1.0, 0.0]]), [math.pi / 2], 1e4)
+    assert np.allclose(out, [[0.0, 1.0]], atol=1e-15)
+
+
+def test_rope_pairs_dim_c_with_c_plus_half():
+    # d = 4, theta = 100: chunk 1 (dims 1 and 3) has frequency 100^(-1/2) = 0.1;
+    # position 5*pi is a quarter turn for it, so one-hot dim 1 lands on dim 3 and nowhere else.
+    x = np.array([[0.0, 1.0, 0.0, 0.0]])
+    out = oracle.rope(x, [5 * math.pi], 100.0)
+    assert np.allclose(out, [[0.0, 0.0, 0.0, 1.0]], atol=1e-14)
+    # chunk 0 (dims 0 and 2) has frequency 1: position pi flips its sign.
+    out0 = oracle.rope(np.array([[1.0, 0.0, 0.0, 0.0]]), [math.pi], 100.0)
+    assert np.allclose(out0, [[-1.0, 0.0, 0.0, 0.0]], atol=1e-14)
+
+
+def test_rope_full_period_is_identity_and_norm_per_chunk():
+    rng = np.random.default_rng(0)
+    d, theta = 16, 1e4
+    x = rng.standard_normal((1, d))
+    C = d // 2
+    for c in range(C):
+        period = 2 * math.pi / theta ** (-2.0 * c / d)
+        y = oracle.rope(x, [period], theta)
+        # chunk c is back where it started
+        assert np.allclose(y[0, [c, c + C]], x[0, [c, c + C]], rtol=1e-9, atol=1e-9)
+    y = oracle.rope(x, [123.0], theta)
+    for c in range(C):
+        assert math.isclose(np.hypot(y[0, c], y[0, c + C]), np.hypot(x[0, c], x[0, c + C]), rel_tol=1e-13)
+
+
+def test_rope_relative_position_invariance():
+    # Shifting q and k by the same amount leaves q.k unchanged (RoPE's relative-position property).
+    rng = np.random.default_rng(1)
+    d, theta = 64, 1e4
+    q = rng.standard_normal((1, d))
+    ks = rng.standard_normal((5, d))
+    m, ns = 512.0, [0.0, 3.0, 100.0, 400.0, 511.0]
+    base = oracle.rope(ks, ns, theta) @ oracle.rope(q, [m], theta)[0]
+    for delta in [1.0, 17.0, 1000.0, 65536.0]:
+        moved = oracle.rope(ks, [n + delta for n in ns], theta) @ oracle.rope(q, [m + delta], theta)[0]
+        assert np.allclose(moved, base, rtol=1e-9, atol=1e-9)
+    # and it is not invariant to moving only one of them
+    moved_k = oracle.rope(ks, [n + 7.0 for n in ns], theta) @ oracle.rope(q, [m], theta)[0]
+    assert not np.allclose(moved_k, base, rtol=1e-3)
+
+
+def test_generator_rotation_agrees_with_oracle_rope():
+    # The input generator's float32 rotation and the oracle's float64 one are two separate
+    # implementations of the same map.
+    from workloads import rope_rotate_f32
+
+    rng = np.random.default_rng(2)
+    for d, theta in [(64, 1e4), (128, 5e5), (128, 1e6)]:
+        x = rng.standard_normal((6, d)).astype(np.float32)
+        pos = np.array([0, 1, 77, 4095, 32767, 131071])
+        a = rope_rotate_f32(x, pos, theta).astype(np.float64)
+        b = oracle.rope(x.astype(np.float64), pos, theta)
+        assert np.allclose(a, b, rtol=0, atol=1e-5 * np.abs(x).max())
+
+
+# ---------------------------------------------------------------------------- TIP scores
+
+def test_tip_hand_example(hand):
+    q = np.array(hand["q_group"], dtype=np.float64)
+    k = np.array(hand["keys"], dtype=np.float64)
+    assert np.array_equal(oracle.tip_scores(q, k, hand["idom"]), hand["tip_scores"])
+    assert np.array_equal(oracle.tip_scores(q, k, [0, 1]), hand["full_scores"])
+
+
+def test_tip_all_chunks_equals_full_dot():
+    rng = np.random.default_rng(3)
+    for G, d, L in [(1, 64, 50), (4, 128, 300), (7, 128, 33)]:
+        q = rng.standard_normal((G, d))
+        k = rng.standard_normal((L, d))
+        s = oracle.tip_scores(q, k, range(d // 2))
+        ref = np.dot(k, q.sum(axis=0))
+        assert np.allclose(s, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_tip_is_linear_in_the_group():
+    rng = np.random.default_rng(4)
+    G, d, L = 4, 128, 200
+    q = rng.standard_normal((G, d))
+    k = rng.standard_normal((L, d))
+    idom = np.sort(rng.choice(d // 2, 16, replace=False))
+    per_head = sum(oracle.tip_scores(q[h:h + 1], k, idom) for h in range(G))
+    assert np.allclose(oracle.tip_scores(q, k, idom), per_head, rtol=1e-12, atol=1e-12)
+
+
+def test_tip_one_hot_query_reads_exactly_the_dominant_dims():
+    rng = np.random.default_rng(5)
+    d, L = 16, 9
+    C = d // 2
+    k = rng.standard_normal((L, d))
+    idom = [1, 5]
+    dims = set(oracle.dominant_dims(idom, d))
+    assert dims == {1, 5, 1 + C, 5 + C}
+    for i in range(d):
+        q = np.zeros((1, d))
+        q[0, i] = 1.0
+        s = oracle.tip_scores(q, k, idom)
+        if i in dims:
+            assert np.array_equal(s, k[:, i])
+        else:
+            assert np.array_equal(s, np.zeros(L))
+
+
+# ---------------------------------------------------------------------------- selection
+
+def _brute_force_top(scores, n):
+    """The unique n-subset whose every member beats every outsider (score desc, position asc)."""
+    L = len(scores)
+    better = lambda a, b: scores[a] > scores[b] or (scores[a] == scores[b] and a < b)
+    found = []
+    for sub in itertools.combinations(range(L), n):
+        inside = set(sub)
+        if all(better(a, b) for a in inside for b in range(L) if b not in inside):
+            found.append(sub)
+    assert len(found) == 1
+    return np.array(found[0])
+
+
+def test_select_matches_brute_force_on_tiny_rows():
+    rng = np.random.default_rng(6)
+    for trial in range(60):
+        L = int(rng.integers(1, 11))
+        # small integer scores so that ties are frequent
+        s = rng.integers(-3, 4, size=L).astype(np.float64)
+        for n in range(0, L + 1):
+            got = oracle.select_top(s, n)
+            if n == 0:
+                assert got.size == 0
+                continue
+            assert np.array_equal(got, _brute_force_top(s, n)), (s, n)
+
+
+def test_select_hand_example(hand):
+    s = np.array(hand["tip_scores"], dtype=np.float64)
+    assert list(oracle.select_top(s, 2)) == hand["top2"]
+    assert list(oracle.select_top(s, 3)) == hand["top3"]
+    assert list(oracle.select_top(np.array(hand["full_scores"], float), 2)) == hand["full_top2"]
+
+
+def test_select_special_cases():
+    assert list(oracle.select_top(np.zeros(10), 4)) == [0, 1, 2, 3]          # all equal -> lowest positions
+    assert list(oracle.select_top(np.array([1.0, 2.0, 2.0, 1.0]), 1)) == [1]  # duplicate maximum -> lower
+    assert list(oracle.select_top(np.array([3.0, 1.0, 2.0]), 10)) == [0, 1, 2]  # N_fac >= L -> everything
+    assert list(oracle.select_top(np.array([-0.0, 0.0, -1.0]), 1)) == [0]     # -0 and +0 are equal scores
+
+
+def test_tie_band_check_accepts_and_rejects():
+    s = np.array([10.0, 5.0, 5.0000001, 1.0, 0.0])
+    assert oracle.tie_band_check(np.array([0, 2]), s, 2)[0]
+    assert oracle.tie_band_check(np.array([0, 1]), s, 2)[0]       # swap inside the band
+    assert not oracle.tie_band_check(np.array([0, 3]), s, 2)[0]   # token below the band
+    assert not oracle.tie_band_check(np.array([1, 2]), s, 2)[0]   # token above the band missing
+    assert not oracle.tie_band_check(np.array([0]), s, 2)[0]      # wrong count
+    assert not oracle.tie_band_check(np.array([0, 0]), s, 2)[0]   # duplicate
+
+
+# ---------------------------------------------------------------------------- attention
+
+def test_attend_hand_example(hand):
+    a = hand["attention"]
+    k = np.array(hand["keys"], dtype=np.float64)
+    v = np.array(a["values"], dtype=np.float64)
+    sel = np.array(a["selected"])
+    out = oracle.focused_attention(np.array([a["q"]], float), k, v, sel, a["scale"])
+    assert np.allclose(out[0], a["out"], rtol=1e-15, atol=1e-15)
+
+
+def test_attend_two_tokens_is_logistic():
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        q, k1, k2, v1, v2 = rng.standard_normal((5, 8))
+        z1, z2 = 0.3 * k1 @ q, 0.3 * k2 @ q
+        w1 = 1.0 / (1.0 + math.exp(-(z1 - z2)))
+        ref = w1 * v1 + (1.0 - w1) * v2
+        assert np.allclose(oracle.attend(q, np.stack([k1, k2]), np.stack([v1, v2]), 0.3), ref, rtol=1e-13, atol=1e-14)
+
+
+def test_attend_weights_match_library_softmax_and_sum_to_one():
+    rng = np.random.default_rng(8)
+    L, d = 40, 16
+    q, k = rng.standard_normal(d), rng.standard_normal((L, d))
+    # values = identity rows -> the output is the weight vector itself
+    p = oracle.attend(q, k, np.eye(L), 0.25)
+    assert np.allclose(p, scipy.special.softmax(0.25 * k @ q), rtol=1e-12, atol=1e-15)
+    assert math.isclose(oracle.attend(q, k, np.ones((L, 1)), 0.25)[0], 1.0, rel_tol=1e-14)
+
+
+def test_attend_dominant_key():
+    rng = np.random.default_rng(9)
+    L, d = 30, 16
+    q = rng.standard_normal(d)
+    k = rng.standard_normal((L, d)) * 0.1
+    v = rng.standard_normal((L, d))
+    k[17] = q * (60.0 / (q @ q))            # logit margin ~ 60 over every other key
+    assert np.allclose(oracle.attend(q, k, v, 1.0), v[17], rtol=0, atol=1e-12)
+
+
+def test_focused_with_every_token_is_dense():
+    rng = np.random.default_rng(10)
+    G, d, L = 4, 32, 57
+    q = rng.standard_normal((G, d))
+    k, v = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    idom = [0, 3, 9]
+    res = oracle.decode_row(q, k, v, ROLE_SPARSE, 0.2, idom=idom, n_fac=L + 5)
+    dense = scipy.special.softmax(0.2 * q @ k.T, axis=1) @ v
+    assert np.allclose(res["out"], dense, rtol=1e-12, atol=1e-13)
+    assert np.array_equal(res["sel"], np.arange(L))
+
+
+def test_focused_keeps_original_positions():
+    # Re-rotating the selected keys at compacted positions 0..n-1 is a different (wrong) computation.
+    rng = np.random.default_rng(11)
+    d, L, theta = 32, 64, 1e4
+    raw_k = rng.standard_normal((L, d))
+    raw_q = rng.standard_normal((1, d))
+    v = rng.standard_normal((L, d))
+    k = oracle.rope(raw_k, range(L), theta)
+    q = oracle.rope(raw_q, [L], theta)
+    sel = np.array([2, 9, 30, 31, 50, 63])
+    right = oracle.focused_attention(q, k, v, sel, 0.3)
+    k_wrong = oracle.rope(raw_k[sel], range(len(sel)), theta)
+    wrong = oracle.focused_attention(q, k_wrong, v[sel], np.arange(len(sel)), 0.3)
+    assert not np.allclose(right, wrong, atol=1e-3)
+
+
+# ---------------------------------------------------------------------------- head roles
+
+def test_stream_positions_hand_example(hand):
+    st = hand["stream"]
+    assert list(oracle.stream_positions(st["L"], st["sink"], st["window"])) == st["positions"]
+    assert list(oracle.stream_positions(10, 0, 0)) == []
+    assert list(oracle.stream_positions(10, 4, 8)) == list(range(10))   # S + W >= L -> dense
+    assert list(oracle.stream_positions(3, 128, 4096)) == [0, 1, 2]
+
+
+def test_stream_head_is_masked_dense_attention():
+    rng = np.random.default_rng(12)
+    G, d, L, S, W = 2, 16, 90, 5, 20
+    q = rng.standard_normal((G, d))
+    k, v = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    res = oracle.decode_row(q, k, v, ROLE_STREAM, 0.25, sink=S, window=W)
+    mask = np.full(L, -np.inf)
+    mask[:S] = 0.0
+    mask[L - W:] = 0.0
+    ref = scipy.special.softmax(0.25 * q @ k.T + mask[None, :], axis=1) @ v
+    assert np.allclose(res["out"], ref, rtol=1e-12, atol=1e-13)
+    dense = oracle.decode_row(q, k, v, ROLE_DENSE, 0.25)
+    wide = oracle.decode_row(q, k, v, ROLE_STREAM, 0.25, sink=50, window=40)
+    assert np.allclose(dense["out"], wide["out"], rtol=1e-13, atol=1e-14)
+
+
+def test_decode_step_gqa_groups_are_contiguous():
+    # q head h reads KV group h // G: with G = 2, heads 2 and 3 use KV group 1.
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, d, L = 1, 4, 2, 16, 12
+    q = rng.standard_normal((B, Hq, d))
+    k, v = rng.standard_normal((L, Hkv, d)), rng.standard_normal((L, Hkv, d))
+    res = oracle.decode_step(q, k, v, [0, L], [ROLE_DENSE, ROLE_DENSE], 0.25)
+    for h in range(Hq):
+        ref = scipy.special.softmax(0.25 * k[:, h // 2] @ q[0, h]) @ v[:, h // 2]
+        assert np.allclose(res[(0, h // 2)]["out"][h % 2], ref, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------- shared index
+
+def test_shared_index_with_k_equal_L_is_dense_in_every_layer():
+    rng = np.random.default_rng(14)
+    n_layers, B, Hq, Hkv, d, L = 3, 2, 4, 2, 16, 20
+    qi = rng.standard_normal((B, Hq, d))
+    ql = rng.standard_normal((n_layers, B, Hq, d))
+    k, v = rng.standard_normal((B * L, Hkv, d)), rng.standard_normal((B * L, Hkv, d))
+    res = oracle.shared_index_step(qi, ql, k, v, [0, L, 2 * L], L, 0.25)
+    for (b, g), r in res.items():
+        for l in range(n_layers):
+            for j in range(2):
+                h = g * 2 + j
+                ref = scipy.special.softmax(0.25 * k[b * L:(b + 1) * L, g] @ ql[l, b, h]) @ v[b * L:(b + 1) * L, g]
+                assert np.allclose(r["out"][l, j], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_shared_index_scores_are_full_dot_and_one_index_per_group():
+    rng = np.random.default_rng(15)
+    n_layers, B, Hq, Hkv, d, L = 2, 1, 4, 2, 16, 50
+    qi = rng.standard_normal((B, Hq, d))
+    ql = rng.standard_normal((n_layers, B, Hq, d))
+    k, v = rng.standard_normal((L, Hkv, d)), rng.standard_normal((L, Hkv, d))
+    res = oracle.shared_index_step(qi, ql, k, v, [0, L], 7, 0.25)
+    for g in range(Hkv):
+        r = res[(0, g)]
+        ref = k[:, g] @ qi[0, 2 * g:2 * g + 2].sum(axis=0)
+        assert np.allclose(r["scores"], ref, rtol=1e-12, atol=1e-12)
+        assert np.array_equal(r["sel"], np.sort(np.argsort(-ref, kind="stable")[:7]))
+        # every layer attends over that same index
+        for l in range(n_layers):
+            for j in range(2):
+                want = oracle.attend(ql[l, 0, 2 * g + j], k[r["sel"], g], v[r["sel"], g], 0.25)
+                assert np.allclose(r["out"][l, j], want, rtol=1e-14, atol=1e-15)
