@@ -1,0 +1,246 @@
+/*
+ * aoh.h -- C ABI of the token-sparse decode library (libaoh.so).
+ *
+ * One decode step of token-sparse attention over a long KV cache, on one
+ * sm_100a GPU:
+ *   1. importance scores from the dominant RoPE frequency chunks of each KV
+ *      head (FASA: Frequency-aware Sparse Attention, section 2.B.1, Token
+ *      Importance Predictor; chunks as defined in section 2.A),
+ *   2. a per-(sequence, KV head) top-N_fac selection of those scores
+ *      (same section),
+ *   3. exact full-dimension softmax attention over only the selected tokens
+ *      at their original positions (section 2.B.2, Focused Attention
+ *      Computation; the whole cache stays on the GPU and only part of K is
+ *      read, as in the FASA-C variant of section 2.C).
+ * Around it: the retrieval / streaming head-role split of the AoH summary
+ * (Resumen Tecnico: Autonomia de Cabezales, Metodologia section 4:
+ * retrieval heads attend to the whole cache, streaming heads to a sink plus
+ * a recent window), and the shared index of the CLSA article (El
+ * enrutamiento compartido entre capas..., "Como funciona CLSA": one top-k,
+ * computed once, reused by every cross-decoder layer over a shared cache).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every buffer is owned by the caller.  Pointers marked "device" must be
+ *   device memory of the current CUDA device; "host" pointers are read
+ *   during the call only.  The library allocates no memory.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *   asynchronous: they validate their arguments on the host, enqueue kernels
+ *   on `stream` and return.  No call synchronises, except aoh_device_check.
+ * - Errors come back as aoh_status; nothing is thrown across the ABI.
+ *   Argument errors are found on the host before anything is launched and
+ *   leave every output untouched.  A failed launch returns AOH_ERR_CUDA.
+ *   Conditions only the device can see (a stored position outside its
+ *   sequence, a per-sequence N_fac above the capacity, a chunk id outside
+ *   [0, d/2)) are recorded in a per-device error word, the offending access
+ *   is skipped, and aoh_device_check() reports them.
+ * - Tensors are bf16 (raw 16-bit storage) unless stated otherwise; outputs
+ *   are fp32.  Keys and queries are already rotated by RoPE at their
+ *   absolute positions (keys of sequence b at 0..L_b-1, its query at L_b);
+ *   nothing here rotates, so "original positions" hold by construction.
+ * - GQA: q head h reads KV head g = h / G with G = n_q_heads / n_kv_heads
+ *   (contiguous groups).
+ */
+#ifndef AOH_H
+#define AOH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AOH_OK = 0,
+  AOH_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent shapes          */
+  AOH_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim not 64/128) */
+  AOH_ERR_ALIGNMENT = 3,     /* a pointer or stride breaks the 16-byte row rule      */
+  AOH_ERR_WORKSPACE = 4,     /* workspace NULL, too small or not 256-byte aligned    */
+  AOH_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed                 */
+  AOH_ERR_DEVICE_CHECK = 6   /* a device-side check fired (see aoh_device_check)     */
+} aoh_status;
+
+/* Head roles, one per KV head (AoH summary, Metodologia section 4). */
+enum {
+  AOH_ROLE_SPARSE = 0, /* importance score -> top-N_fac -> focused attention      */
+  AOH_ROLE_DENSE = 1,  /* retrieval head: attention over every cached token        */
+  AOH_ROLE_STREAM = 2  /* streaming head: sink tokens plus the recent window only  */
+};
+
+/*
+ * The KV cache of one decode step (ragged batch).
+ *
+ * Element i of KV head h of global token t is at
+ *   k[t * stride_tok + h * stride_head + i]   (same for v),
+ * where sequence b owns global tokens [offsets[b], offsets[b+1]) and its
+ * local position p is global token offsets[b] + p.  head_dim elements of a
+ * row are contiguous.  k and v must be 16-byte aligned and both strides
+ * multiples of 8 elements (every row starts on a 16-byte boundary).
+ *
+ * k_dom (optional) is a packed copy of the dominant columns of K, laid out
+ * [n_kv_heads][total_tokens][k_dom_cols]: in row (h, t), column j < n_dom
+ * holds K dim I_dom[h][j], column n_dom + j holds dim I_dom[h][j] + d/2, the
+ * rest (up to k_dom_cols, a multiple of 8) are zero.  aoh_pack_dominant
+ * writes it.  With it the importance scan reads 4 * n_dom bytes per token
+ * and head instead of the sectors of K that the chunks touch.
+ */
+typedef struct aoh_kv_cache {
+  const void* k;               /* device, bf16                                         */
+  const void* v;               /* device, bf16                                         */
+  const int32_t* offsets;      /* device int32 [batch + 1], non-decreasing, offsets[0]=0 */
+  int32_t batch;               /* number of sequences B (0 is a no-op)                 */
+  int32_t n_kv_heads;          /* Hkv, 1..128                                          */
+  int32_t head_dim;            /* d: 64 or 128                                         */
+  int32_t max_len;             /* host copy of max_b L_b (an upper bound is fine)       */
+  int64_t total_tokens;        /* host copy of offsets[batch], < 2^31                  */
+  int64_t stride_tok;          /* elements between tokens t and t+1 of one head        */
+  int64_t stride_head;         /* elements between heads h and h+1 of one token        */
+  const void* k_dom;           /* device bf16 [Hkv][total_tokens][k_dom_cols], or NULL */
+  int32_t k_dom_cols;          /* row length of k_dom in elements (0 when k_dom NULL)  */
+} aoh_kv_cache;
+
+/* Human-readable name of a status code (static string). */
+const char* aoh_status_string(aoh_status s);
+
+/* Library ABI version: 1. */
+int32_t aoh_version(void);
+
+/*
+ * aoh_device_check -- synchronise `stream`, then read and clear this
+ * device's error word.  Returns AOH_OK, AOH_ERR_DEVICE_CHECK (and, if
+ * `detail` is not NULL, writes 4 host int32: check id, then three values of
+ * the first failing access), or AOH_ERR_CUDA.
+ */
+aoh_status aoh_device_check(void* stream, int32_t* detail);
+
+/*
+ * aoh_pack_dominant -- write the packed dominant-column copy of K
+ * (layout in aoh_kv_cache above).  A cache-maintenance step: run it when
+ * tokens are appended, not per decode step.  FASA section 2.C (FASA-M keeps
+ * only the dominant parts of K on the GPU; this is that layout kept beside
+ * the full cache).
+ *   idom     device int32 [n_kv_heads][n_dom], chunk ids in [0, d/2)
+ *   n_dom    1 .. d/2, and 2*n_dom <= k_dom_cols
+ *   k_dom    device bf16 [n_kv_heads][kv->total_tokens][k_dom_cols], 16-B aligned
+ *   k_dom_cols  multiple of 8
+ * kv->k_dom is ignored here.
+ */
+aoh_status aoh_pack_dominant(const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom,
+                             void* k_dom, int32_t k_dom_cols, void* stream);
+
+/*
+ * aoh_tip_score -- importance of every cached token (FASA section 2.B.1,
+ * with GQA aggregation by summing over the group, AoH section 4):
+ *   scores[g][t] = sum over q heads h of group g, over c in I_dom[g], of
+ *                  q_h[c] * k_t[c] + q_h[c + d/2] * k_t[c + d/2]
+ * computed as one fp32 dot of the fp32 group sum of q with the dominant
+ * columns of k_t.  No 1/sqrt(d) scale.
+ *   q        device bf16 [B][n_q_heads][d], contiguous
+ *   idom     device int32 [Hkv][n_dom], chunk ids in [0, d/2).  With every
+ *            chunk listed (n_dom = d/2) the score is the full q.k of the
+ *            group sum: the shared indexer's score.
+ *   scores   device fp32 [Hkv][kv->total_tokens]; entry (g, offsets[b] + p)
+ *            is token p of sequence b.
+ * If kv->k_dom is set it must have been packed with this idom / n_dom and
+ * the scan reads it; otherwise K is read in place.
+ */
+aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
+                         const int32_t* idom, int32_t n_dom, float* scores, void* stream);
+
+/*
+ * aoh_topk_select -- per (sequence b, KV head g): the n = min(N_fac_b, L_b)
+ * positions with the largest scores (FASA section 2.B.1; the shared index's
+ * single top-k).  Equal scores: the lower position wins; -0 equals +0.
+ * Output positions are ascending.
+ *   scores          device fp32 [Hkv][total_tokens] (layout of aoh_tip_score);
+ *                   finite values
+ *   n_fac           N_fac for every sequence when n_fac_per_seq is NULL
+ *   n_fac_per_seq   device int32 [B] or NULL
+ *   n_fac_cap       capacity per row; n_fac (or every n_fac_per_seq entry) <= cap
+ *   idx             device int32 [B][Hkv][n_fac_cap]; entries >= n are set to -1
+ *   count           device int32 [B][Hkv]: n
+ * Deterministic: the same input gives the same bits.
+ */
+aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
+                           const int32_t* n_fac_per_seq, int32_t n_fac_cap,
+                           int32_t* idx, int32_t* count, void* stream);
+
+/*
+ * aoh_sparse_decode -- the whole sparse step for the heads whose role is
+ * AOH_ROLE_SPARSE: importance scores, top-N_fac, then exact attention of
+ * every q head of the group over the selected tokens (FASA sections 2.B.1
+ * and 2.B.2):
+ *   out[b][h] = sum over selected t of softmax_t(scale * q_h . k_t) * v_t
+ * in fp32 (online softmax, split over the selection, then combined).
+ *   q, idom, n_dom, n_fac, n_fac_per_seq, n_fac_cap: as above
+ *   roles      host uint8 [Hkv] or NULL (= every head SPARSE); only rows of
+ *              SPARSE heads are computed and written
+ *   scale      softmax scale, usually 1/sqrt(d)
+ *   out        device fp32 [B][n_q_heads][d]
+ *   idx_out, count_out   optional device outputs of the selection (layouts of
+ *              aoh_topk_select, rows of non-SPARSE heads untouched), or NULL
+ *   workspace  device, 256-byte aligned, >= aoh_sparse_decode_workspace_size
+ *              bytes, zero-filled once before its first use (every call
+ *              leaves its counters at zero again)
+ * A sequence with L_b = 0 gives zero rows.
+ */
+aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
+                             const int32_t* idom, int32_t n_dom, int32_t n_fac,
+                             const int32_t* n_fac_per_seq, int32_t n_fac_cap,
+                             const uint8_t* roles, float scale, float* out,
+                             int32_t* idx_out, int32_t* count_out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+size_t aoh_sparse_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads,
+                                        int32_t n_fac_cap);
+
+/*
+ * aoh_stream_decode -- attention for the heads whose role is AOH_ROLE_DENSE
+ * (every position [0, L_b)) or AOH_ROLE_STREAM (positions
+ * [0, min(sink, L_b)) together with [max(0, L_b - window), L_b)); AoH
+ * summary, Metodologia section 4.  Same arithmetic as aoh_sparse_decode.
+ *   roles      host uint8 [Hkv] (required)
+ *   sink, window >= 0
+ *   out        device fp32 [B][n_q_heads][d]; only DENSE / STREAM rows written
+ *   workspace  as for aoh_sparse_decode, >= aoh_stream_decode_workspace_size
+ * Calling aoh_sparse_decode and aoh_stream_decode on the same `out` with the
+ * same roles gives the full head-role-split decode step.
+ */
+aoh_status aoh_stream_decode(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
+                             const uint8_t* roles, int32_t sink, int32_t window, float scale,
+                             float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+size_t aoh_stream_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads,
+                                        const uint8_t* roles, int32_t sink, int32_t window);
+
+/*
+ * aoh_shared_index_decode -- the cross-decoder layers of a shared-cache
+ * stack reuse one index ("Como funciona CLSA"): for every layer l, every
+ * q head h of group g and sequence b,
+ *   out[l][b][h] = sum over t in idx[b][g][0 .. count[b][g]) of
+ *                  softmax_t(scale * q_layers[l][b][h] . k_t) * v_t.
+ * The index is read once per (b, g) and the K / V rows it names are read
+ * once for all n_layers * G query rows.  Build the index with
+ * aoh_tip_score (idom = every chunk 0..d/2-1) and aoh_topk_select.
+ *   q_layers   device bf16 [n_layers][B][n_q_heads][d], contiguous
+ *   n_layers * (n_q_heads / n_kv_heads) <= 32
+ *   idx, count, n_fac_cap: layouts of aoh_topk_select; positions must lie in
+ *              [0, L_b) (checked on the device)
+ *   out        device fp32 [n_layers][B][n_q_heads][d]
+ *   workspace  as above, >= aoh_shared_index_decode_workspace_size
+ */
+aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32_t n_q_heads,
+                                   const aoh_kv_cache* kv, const int32_t* idx,
+                                   const int32_t* count, int32_t n_fac_cap, float scale,
+                                   float* out, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+size_t aoh_shared_index_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_layers,
+                                              int32_t n_q_heads, int32_t n_fac_cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AOH_H */

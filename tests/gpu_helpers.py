@@ -1,0 +1,133 @@
+"""Shared helpers of the GPU parity tests: move seeded inputs to the device, run the
+CUDA path through the C ABI, compare with the float64 oracle on the same inputs."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from token_sparse_decode_b200 import binding as B
+from token_sparse_decode_b200.step import SharedIndexStep, SparseDecodeStep
+
+OUT_ATOL = 2e-3        # outputs, absolute, unit-variance V
+SCORE_REL = 1e-4       # scores, relative to sum |q_c| |k_c| over the scored dims
+BAND_REL = 1e-4        # top-k tie band, relative to the n-th score
+
+
+class Dev:
+    """A Workload's tensors on the GPU."""
+
+    def __init__(self, w, device="cuda"):
+        self.w = w
+        self.k = w.k.to(device)
+        self.v = w.v.to(device)
+        self.q = w.q.to(device)
+        self.q_layers = None if w.q_layers is None else w.q_layers.to(device)
+        self.offsets = w.offsets.to(device)
+        self.idom = None if w.idom is None else w.idom.to(device)
+        self.n_fac_per_seq = w.n_fac_per_seq.to(device)
+        self.max_len = w.max_len
+        self.T = w.total_tokens
+
+    def kv(self, k_dom=None):
+        return B.make_kv(self.k, self.v, self.offsets, self.max_len, self.T, k_dom)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().double().numpy()
+
+
+def row_inputs(w, b, g):
+    """float64 (q_group, keys, values) of row (b, g) of a Workload (exact upcasts of its bf16)."""
+    G = w.spec.group
+    o0, o1 = int(w.offsets[b]), int(w.offsets[b + 1])
+    return (f64(w.q[b, g * G:(g + 1) * G]), f64(w.k[o0:o1, g]), f64(w.v[o0:o1, g]))
+
+
+def check_device():
+    st, detail = B.device_check()
+    assert st == 0, f"device check fired: {detail}"
+
+
+def score_bound(q_group, keys, idom):
+    """sum over the scored dims of |q_c| |k_c| (the scale of the fp32 rounding of one score)."""
+    return oracle.tip_scores(np.abs(q_group), np.abs(keys), idom)
+
+
+def band_swap_bound(q_group, keys, values, scores, n, scale):
+    """Largest change of a head's output when band members are swapped (oracle values only).
+
+    Tokens whose score lies within the band of the n-th score may be exchanged;
+    attention over the kept core C moves by at most 2 max|v| * sum_band w / sum_C w.
+    """
+    s = np.asarray(scores)
+    L = s.shape[0]
+    if n >= L or n == 0:
+        return 0.0
+    s_n = np.sort(s)[::-1][n - 1]
+    beta = BAND_REL * max(abs(s_n), float(np.mean(np.abs(s))))
+    band = np.abs(s - s_n) <= beta
+    core = s > s_n + beta
+    worst = 0.0
+    for h in range(q_group.shape[0]):
+        z = scale * (keys @ q_group[h])
+        z = z - z.max()
+        w = np.exp(z)
+        wc = w[core].sum()
+        if wc <= 0:
+            return np.inf
+        worst = max(worst, 2 * np.abs(values).max() * w[band].sum() / wc)
+    return worst
+
+
+def compare_sparse_row(w, b, g, gpu_sel, gpu_out, stats=None):
+    """Check one SPARSE row: selection within the tie band, output within 2e-3 of the oracle."""
+    q_group, keys, values = row_inputs(w, b, g)
+    idom = w.idom[g].tolist()
+    n = int(min(int(w.n_fac_per_seq[b]), keys.shape[0]))
+    s = oracle.tip_scores(q_group, keys, idom)
+    ok, msg = oracle.tie_band_check(gpu_sel, s, n, BAND_REL)
+    assert ok, f"row ({b},{g}): {msg}"
+    ref_sel = oracle.select_top(s, n)
+    ref_out = oracle.focused_attention(q_group, keys, values, ref_sel, w.scale)
+    tol = OUT_ATOL
+    same = np.array_equal(np.asarray(gpu_sel), ref_sel)
+    if not same:
+        tol += band_swap_bound(q_group, keys, values, s, n, w.scale)
+    if stats is not None:
+        stats["rows"] = stats.get("rows", 0) + 1
+        stats["swapped"] = stats.get("swapped", 0) + (0 if same else 1)
+    err = np.abs(gpu_out - ref_out).max() if ref_out.size else 0.0
+    assert err <= tol, f"row ({b},{g}): max |out - oracle| = {err:.3g} > {tol:.3g}"
+    return err
+
+
+def compare_window_row(w, b, g, gpu_out, role, sink, window):
+    q_group, keys, values = row_inputs(w, b, g)
+    ref = oracle.decode_row(q_group, keys, values, role, w.scale, sink=sink, window=window)["out"]
+    err = np.abs(gpu_out - ref).max() if ref.size else 0.0
+    assert err <= OUT_ATOL, f"row ({b},{g}) role {role}: max err {err:.3g}"
+    return err
+
+
+def run_sparse(d: Dev, pack=True):
+    w = d.w
+    step = SparseDecodeStep(d.k, d.v, d.offsets, d.max_len, d.T, w.spec.n_q_heads, w.roles.tolist(), w.scale,
+                            idom=d.idom, n_fac=int(w.n_fac_per_seq.max()) if len(w.n_fac_per_seq) else 0,
+                            n_fac_per_seq=d.n_fac_per_seq, n_fac_cap=max(1, int(w.n_fac_per_seq.max())),
+                            sink=w.spec.sink, window=w.spec.window, pack_dominant=pack)
+    out = step(d.q)
+    torch.cuda.synchronize()
+    check_device()
+    return step, out
+
+
+def run_shared(d: Dev):
+    w = d.w
+    step = SharedIndexStep(d.k, d.v, d.offsets, d.max_len, d.T, w.spec.n_layers, w.spec.n_q_heads,
+                           w.spec.topk_shared, w.scale)
+    out = step(d.q, d.q_layers)
+    torch.cuda.synchronize()
+    check_device()
+    return step, out

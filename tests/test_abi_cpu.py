@@ -1,0 +1,134 @@
+"""The C ABI on the CPU: the library loads, exports every declared symbol, its
+struct layout matches the header, and host-side validation rejects bad calls
+before anything reaches a GPU (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+import torch  # noqa: F401  (loads torch's CUDA runtime first, as in real use)
+
+from token_sparse_decode_b200 import binding as B
+from token_sparse_decode_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "aoh.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return B.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(aoh_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.aoh_version() == 1
+    assert lib.aoh_status_string(0) == b"ok"
+    assert lib.aoh_status_string(4).startswith(b"workspace")
+    assert lib.aoh_status_string(99) == b"unknown status"
+
+
+def test_struct_layout_matches_header():
+    src = r"""
+    #include <stdio.h>
+    #include <stddef.h>
+    #include "aoh.h"
+    int main(void) {
+      printf("%zu %zu %zu %zu %zu %zu\n", sizeof(aoh_kv_cache), offsetof(aoh_kv_cache, batch),
+             offsetof(aoh_kv_cache, total_tokens), offsetof(aoh_kv_cache, stride_head),
+             offsetof(aoh_kv_cache, k_dom), offsetof(aoh_kv_cache, k_dom_cols));
+      return 0;
+    }
+    """
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()]
+    K = B.KVCache
+    assert vals == [ctypes.sizeof(K), K.batch.offset, K.total_tokens.offset, K.stride_head.offset,
+                    K.k_dom.offset, K.k_dom_cols.offset]
+
+
+def fake_kv(**kw):
+    kv = B.KVCache()
+    kv.k, kv.v, kv.offsets = 0x10000, 0x20000, 0x30000
+    kv.batch, kv.n_kv_heads, kv.head_dim, kv.max_len = 2, 8, 128, 1000
+    kv.total_tokens, kv.stride_tok, kv.stride_head = 2000, 8 * 128, 128
+    for a, b in kw.items():
+        setattr(kv, a, b)
+    return kv
+
+
+def call_sparse(lib, kv, **kw):
+    a = dict(q=0x40000, hq=32, idom=0x50000, n_dom=16, n_fac=64, nfps=None, cap=64, roles=None, scale=0.088,
+             out=0x60000, idx=None, cnt=None, ws=0x70000, ws_bytes=1 << 40)
+    a.update(kw)
+    return lib.aoh_sparse_decode(a["q"], a["hq"], ctypes.byref(kv), a["idom"], a["n_dom"], a["n_fac"], a["nfps"],
+                                 a["cap"], a["roles"], a["scale"], a["out"], a["idx"], a["cnt"], a["ws"],
+                                 a["ws_bytes"], None)
+
+
+def test_host_validation_rejects_before_launch(lib):
+    INVALID, UNSUP, ALIGN, WS = 1, 2, 3, 4
+    assert lib.aoh_tip_score(0x40000, 32, None, 0x50000, 16, 0x60000, None) == INVALID
+    assert call_sparse(lib, fake_kv(head_dim=96)) == UNSUP
+    assert call_sparse(lib, fake_kv(k=0x10008)) == ALIGN            # K not 16-byte aligned
+    assert call_sparse(lib, fake_kv(stride_tok=8 * 128 + 4)) == ALIGN
+    assert call_sparse(lib, fake_kv(), hq=30) == INVALID            # Hq % Hkv != 0
+    assert call_sparse(lib, fake_kv(), n_dom=65) == INVALID         # n_dom > d/2
+    assert call_sparse(lib, fake_kv(), n_dom=0) == INVALID
+    assert call_sparse(lib, fake_kv(), n_fac=65, cap=64) == INVALID  # N_fac above capacity
+    assert call_sparse(lib, fake_kv(), ws=None) == WS
+    assert call_sparse(lib, fake_kv(), ws_bytes=100) == WS
+    assert call_sparse(lib, fake_kv(), ws=0x70010) == WS            # not 256-byte aligned
+    assert call_sparse(lib, fake_kv(), q=None) == INVALID
+    assert call_sparse(lib, fake_kv(), q=0x40004) == ALIGN
+    assert call_sparse(lib, fake_kv(), scale=float("nan")) == INVALID
+    assert call_sparse(lib, fake_kv(n_kv_heads=0)) == INVALID
+    assert call_sparse(lib, fake_kv(total_tokens=1 << 31)) == INVALID
+    bad_roles = (ctypes.c_uint8 * 8)(0, 1, 2, 3, 0, 0, 0, 0)
+    assert call_sparse(lib, fake_kv(), roles=ctypes.cast(bad_roles, ctypes.c_void_p)) == INVALID
+    assert call_sparse(lib, fake_kv(batch=0)) == 0                  # empty batch is a no-op
+    roles = (ctypes.c_uint8 * 8)(*([2] * 8))
+    r = ctypes.cast(roles, ctypes.c_void_p)
+    assert lib.aoh_stream_decode(0x40000, 32, ctypes.byref(fake_kv()), None, 4, 60, 0.1, 0x60000, 0x70000,
+                                 1 << 40, None) == INVALID          # roles required
+    assert lib.aoh_stream_decode(0x40000, 32, ctypes.byref(fake_kv()), r, -1, 60, 0.1, 0x60000, 0x70000,
+                                 1 << 40, None) == INVALID
+    # shared index: more than 32 query rows per KV head
+    assert lib.aoh_shared_index_decode(0x40000, 9, 32, ctypes.byref(fake_kv()), 0x50000, 0x58000, 64, 0.1,
+                                       0x60000, 0x70000, 1 << 40, None) == UNSUP
+    assert lib.aoh_topk_select(0x40000, ctypes.byref(fake_kv()), 10, None, 0, 0x50000, 0x58000, None) == INVALID
+    assert lib.aoh_pack_dominant(ctypes.byref(fake_kv()), 0x50000, 16, 0x60000, 36, None) == INVALID
+
+
+def test_workspace_sizes_are_host_computations(lib):
+    kv = fake_kv()
+    s = lib.aoh_sparse_decode_workspace_size(ctypes.byref(kv), 32, 2048)
+    # at least the fp32 score row of every head plus the index
+    assert s >= 4 * 8 * 2000 + 4 * 2 * 8 * 2048
+    assert s % 256 == 0
+    roles = (ctypes.c_uint8 * 8)(*([1, 2] * 4))
+    assert lib.aoh_stream_decode_workspace_size(ctypes.byref(kv), 32, ctypes.cast(roles, ctypes.c_void_p), 4, 60) > 0
+    assert lib.aoh_shared_index_decode_workspace_size(ctypes.byref(kv), 8, 32, 2048) > 0
+    assert lib.aoh_shared_index_decode_workspace_size(ctypes.byref(kv), 9, 32, 2048) == 0
+    assert lib.aoh_sparse_decode_workspace_size(ctypes.byref(fake_kv(head_dim=96)), 32, 64) == 0

@@ -1,0 +1,288 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Tolerances: selected index sets bit-exact except for swaps inside the 1e-4 score
+band around the n-th score; scores within 1e-4 of sum |q_c||k_c|; outputs within
+2e-3 absolute (unit-variance V).  On caller-given fp32 scores the selection is
+compared bit for bit.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (OUT_ATOL, SCORE_REL, Dev, check_device, compare_sparse_row, compare_window_row, f64,
+                         row_inputs, run_shared, run_sparse, score_bound, band_swap_bound)
+from token_sparse_decode_b200 import binding as B
+from workloads import ROLE_DENSE, ROLE_SPARSE, ROLE_STREAM, WorkloadSpec, make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def spec(**kw):
+    base = dict(name="medium", batch=3, n_q_heads=32, n_kv_heads=8, head_dim=128, theta=5e5,
+                len_range=(300, 6000), n_dom=16, n_fac_div=8, roles=(ROLE_SPARSE,) * 8,
+                planted_frac=0.01, seed=77)
+    base.update(kw)
+    return WorkloadSpec(**base)
+
+
+MEDIUM = {
+    "gqa4_d128": spec(),
+    "gqa7_d128": spec(n_q_heads=28, n_kv_heads=4, roles=(ROLE_SPARSE,) * 4, theta=1e6, seed=78),
+    "mha_d64": spec(n_q_heads=4, n_kv_heads=4, head_dim=64, theta=1e4, n_dom=4, roles=(ROLE_SPARSE,) * 4,
+                    len_range=(100, 2500), seed=79),
+    "gqa16_d64": spec(n_q_heads=32, n_kv_heads=2, head_dim=64, theta=1e4, n_dom=5, roles=(ROLE_SPARSE,) * 2,
+                      seed=80),
+}
+
+
+# ------------------------------------------------------------------------------ TIP scores
+
+@pytest.mark.parametrize("name", list(MEDIUM))
+@pytest.mark.parametrize("packed", [True, False])
+def test_tip_scores_match_oracle(name, packed):
+    w = make_workload(MEDIUM[name])
+    d = Dev(w)
+    k_dom = None
+    kv0 = d.kv()
+    if packed:
+        k_dom = torch.empty((w.spec.n_kv_heads, d.T, B.k_dom_cols(w.spec.n_dom)), dtype=torch.bfloat16,
+                            device="cuda")
+        B.pack_dominant(kv0, d.idom, w.spec.n_dom, k_dom)
+    scores = torch.full((w.spec.n_kv_heads, d.T), float("nan"), device="cuda")
+    B.tip_score(d.q, d.kv(k_dom), d.idom, w.spec.n_dom, scores)
+    torch.cuda.synchronize()
+    check_device()
+    got = f64(scores)
+    for b in range(w.spec.batch):
+        o0, o1 = int(w.offsets[b]), int(w.offsets[b + 1])
+        for g in range(w.spec.n_kv_heads):
+            qg, keys, _ = row_inputs(w, b, g)
+            idom = w.idom[g].tolist()
+            ref = oracle.tip_scores(qg, keys, idom)
+            bound = SCORE_REL * score_bound(qg, keys, idom)
+            assert np.all(np.abs(got[g, o0:o1] - ref) <= bound), (b, g)
+
+
+def test_tip_all_chunks_is_full_dot():
+    w = make_workload(spec(batch=2, len_range=(1000, 3000)))
+    d = Dev(w)
+    C = w.spec.head_dim // 2
+    all_chunks = torch.arange(C, dtype=torch.int32, device="cuda").repeat(w.spec.n_kv_heads, 1).contiguous()
+    scores = torch.empty((w.spec.n_kv_heads, d.T), device="cuda")
+    B.tip_score(d.q, d.kv(), all_chunks, C, scores)
+    torch.cuda.synchronize()
+    got = f64(scores)
+    for b in range(2):
+        o0, o1 = int(w.offsets[b]), int(w.offsets[b + 1])
+        for g in range(w.spec.n_kv_heads):
+            qg, keys, _ = row_inputs(w, b, g)
+            ref = keys @ qg.sum(axis=0)
+            bound = SCORE_REL * (np.abs(keys) @ np.abs(qg).sum(axis=0))
+            assert np.all(np.abs(got[g, o0:o1] - ref) <= bound)
+
+
+# ------------------------------------------------------------------------------ top-k on given scores
+
+def given_scores(rng, lengths, Hkv, kind):
+    T = int(sum(lengths))
+    if kind == "normal":
+        s = rng.standard_normal((Hkv, T)).astype(np.float32)
+    elif kind == "ties":   # few distinct values: ties everywhere, including at the threshold
+        s = (np.round(rng.standard_normal((Hkv, T)) * 2) / 2).astype(np.float32)
+    elif kind == "zeros":  # -0 and +0 mixed, all equal
+        s = np.where(rng.random((Hkv, T)) < 0.5, np.float32(-0.0), np.float32(0.0)).astype(np.float32)
+    else:                  # wide dynamic range, negative and positive
+        s = (rng.standard_normal((Hkv, T)) * np.exp(rng.uniform(-20, 20, (Hkv, T)))).astype(np.float32)
+    return s
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
+def test_topk_bit_exact_on_given_scores(kind):
+    rng = np.random.default_rng(5)
+    lengths = [0, 1, 7, 512, 3000, 20000, 65, 131]
+    Hkv = 3
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = given_scores(rng, lengths, Hkv, kind)
+    nfps = np.array([5, 1, 7, 64, 1000, 2047, 100, 130], dtype=np.int32)
+    cap = 2048
+    dev = torch.device("cuda")
+    k = torch.zeros((int(offs[-1]), Hkv, 64), dtype=torch.bfloat16, device=dev)
+    kv = B.make_kv(k, k, torch.from_numpy(offs).to(dev), max(lengths), int(offs[-1]))
+    idx = torch.full((len(lengths), Hkv, cap), 12345, dtype=torch.int32, device=dev)
+    cnt = torch.full((len(lengths), Hkv), -7, dtype=torch.int32, device=dev)
+    B.topk_select(torch.from_numpy(s).to(dev), kv, 0, torch.from_numpy(nfps).to(dev), cap, idx, cnt)
+    torch.cuda.synchronize()
+    check_device()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b, L in enumerate(lengths):
+        for g in range(Hkv):
+            row = s[g, offs[b]:offs[b + 1]]
+            ref = oracle.select_top(row, int(nfps[b]))
+            n = len(ref)
+            assert cnt_h[b, g] == n
+            assert np.array_equal(idx_h[b, g, :n], ref), (kind, b, g)
+            assert np.all(idx_h[b, g, n:] == -1)
+
+
+def test_topk_fixed_nfac_and_determinism():
+    rng = np.random.default_rng(6)
+    lengths = [131072, 4096, 777]
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = (np.round(rng.standard_normal((2, int(offs[-1]))) * 8) / 8).astype(np.float32)
+    dev = torch.device("cuda")
+    k = torch.zeros((int(offs[-1]), 2, 64), dtype=torch.bfloat16, device=dev)
+    kv = B.make_kv(k, k, torch.from_numpy(offs).to(dev), max(lengths), int(offs[-1]))
+    sd = torch.from_numpy(s).to(dev)
+    outs = []
+    for _ in range(2):
+        idx = torch.empty((3, 2, 2048), dtype=torch.int32, device=dev)
+        cnt = torch.empty((3, 2), dtype=torch.int32, device=dev)
+        B.topk_select(sd, kv, 2048, None, 2048, idx, cnt)
+        torch.cuda.synchronize()
+        outs.append((idx.cpu().numpy(), cnt.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    for b in range(3):
+        for g in range(2):
+            ref = oracle.select_top(s[g, offs[b]:offs[b + 1]], 2048)
+            assert np.array_equal(outs[0][0][b, g, :len(ref)], ref)
+
+
+# ------------------------------------------------------------------------------ sparse decode
+
+@pytest.mark.parametrize("name", list(MEDIUM))
+@pytest.mark.parametrize("pack", [True, False])
+def test_sparse_decode_matches_oracle(name, pack):
+    w = make_workload(MEDIUM[name])
+    d = Dev(w)
+    step, out = run_sparse(d, pack=pack)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = w.spec.group
+    stats = {}
+    for b in range(w.spec.batch):
+        for g in range(w.spec.n_kv_heads):
+            n = cnt_h[b, g]
+            compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G], stats)
+    assert stats["swapped"] <= max(1, stats["rows"] // 10)
+
+
+def test_sparse_decode_is_deterministic():
+    w = make_workload(MEDIUM["gqa4_d128"])
+    d = Dev(w)
+    step, out = run_sparse(d)
+    first = out.clone()
+    step(d.q)
+    torch.cuda.synchronize()
+    assert torch.equal(first, step.out)
+
+
+# ------------------------------------------------------------------------------ retrieval / streaming heads
+
+@pytest.mark.parametrize("sink,window", [(4, 60), (128, 512), (0, 100), (3000, 4000), (0, 0)])
+def test_stream_decode_matches_oracle(sink, window):
+    roles = (ROLE_DENSE, ROLE_STREAM, ROLE_STREAM, ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_STREAM, ROLE_STREAM)
+    w = make_workload(spec(roles=roles, sink=sink, window=window, len_range=(0, 7000), seed=81))
+    d = Dev(w)
+    kv = d.kv()
+    out = torch.full((w.spec.batch, w.spec.n_q_heads, w.spec.head_dim), 777.0, device="cuda")
+    ws = B.workspace(B.stream_decode_workspace_size(kv, w.spec.n_q_heads, roles, sink, window), "cuda")
+    B.stream_decode(d.q, kv, roles, sink, window, w.scale, out, ws)
+    torch.cuda.synchronize()
+    check_device()
+    out_h = f64(out)
+    G = w.spec.group
+    for b in range(w.spec.batch):
+        for g, role in enumerate(roles):
+            rows = out_h[b, g * G:(g + 1) * G]
+            if role == ROLE_SPARSE:
+                assert np.all(rows == 777.0)   # not this call's heads: untouched
+            else:
+                compare_window_row(w, b, g, rows, role, sink, window)
+
+
+def test_full_role_split_step_mixed_heads():
+    roles = (ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_SPARSE)
+    w = make_workload(spec(n_q_heads=16, n_kv_heads=4, roles=roles, sink=16, window=200, n_fac_div=4, seed=82))
+    d = Dev(w)
+    step, out = run_sparse(d)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = w.spec.group
+    for b in range(w.spec.batch):
+        for g, role in enumerate(roles):
+            rows = out_h[b, g * G:(g + 1) * G]
+            if role == ROLE_SPARSE:
+                compare_sparse_row(w, b, g, idx_h[b, g, :cnt_h[b, g]], rows)
+            else:
+                compare_window_row(w, b, g, rows, role, w.spec.sink, w.spec.window)
+
+
+# ------------------------------------------------------------------------------ shared index
+
+@pytest.mark.parametrize("n_layers,hq,hkv", [(8, 32, 8), (2, 16, 4), (3, 16, 4), (1, 8, 8)])
+def test_shared_index_decode_matches_oracle(n_layers, hq, hkv):
+    sp = WorkloadSpec(name="shared", batch=2, n_q_heads=hq, n_kv_heads=hkv, head_dim=128, theta=5e5,
+                      len_range=(500, 9000), n_layers=n_layers, topk_shared=700, seed=90 + n_layers)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_shared(d)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = sp.group
+    ref = oracle.shared_index_step(f64(w.q), f64(w.q_layers), f64(w.k), f64(w.v), w.offsets.tolist(), 700,
+                                   w.scale)
+    for (b, g), r in ref.items():
+        n = cnt_h[b, g]
+        sel = idx_h[b, g, :n]
+        ok, msg = oracle.tie_band_check(sel, r["scores"], min(700, int(w.lengths[b])))
+        assert ok, msg
+        tol = OUT_ATOL
+        if not np.array_equal(sel, r["sel"]):
+            qg, keys, values = row_inputs(w, b, g)
+            for l in range(n_layers):
+                tol = max(tol, OUT_ATOL + band_swap_bound(f64(w.q_layers[l, b, g * G:(g + 1) * G]), keys, values,
+                                                          r["scores"], n, w.scale))
+        err = np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max()
+        assert err <= tol, (b, g, err)
+
+
+def test_shared_index_reports_out_of_range_positions():
+    sp = WorkloadSpec(name="shared", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, theta=1e4,
+                      lengths=(300,), n_layers=2, topk_shared=16, seed=3)
+    w = make_workload(sp)
+    d = Dev(w)
+    kv = d.kv()
+    idx = torch.arange(16, dtype=torch.int32, device="cuda").repeat(1, 2, 1).contiguous()
+    idx[0, 1, 5] = 300            # one past the end of the sequence
+    cnt = torch.full((1, 2), 16, dtype=torch.int32, device="cuda")
+    out = torch.empty((2, 1, 8, 64), device="cuda")
+    ws = B.workspace(B.shared_index_decode_workspace_size(kv, 2, 8, 16), "cuda")
+    B.shared_index_decode(d.q_layers, kv, idx, cnt, 16, w.scale, out, ws)
+    st, detail = B.device_check()
+    assert st == 6 and detail[0] == 1 and detail[3] == 300
+    assert B.device_check()[0] == 0   # reading clears the word
+    assert torch.isfinite(out).all()
+
+
+# ------------------------------------------------------------------------------ edge cases
+
+def test_edge_cases_empty_and_short_sequences():
+    sp = spec(batch=5, lengths=(0, 1, 2, 64, 65), len_range=None, n_fac_div=0, n_fac=64, n_dom=3,
+              planted_frac=0.0, seed=84)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_sparse(d)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = sp.group
+    for b in range(sp.batch):
+        for g in range(sp.n_kv_heads):
+            n = cnt_h[b, g]
+            assert n == min(64, int(w.lengths[b]))
+            if w.lengths[b] == 0:
+                assert np.all(out_h[b, g * G:(g + 1) * G] == 0.0)
+            else:
+                compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G])
+            assert np.all(idx_h[b, g, n:] == -1)

@@ -1,0 +1,200 @@
+"""ctypes binding of libaoh.so: argument marshalling only.
+
+Every entry point takes torch CUDA tensors, turns them into raw device pointers
+and sizes, calls the C function of the same name on the current torch stream and
+raises AohError on a non-zero status.  No arithmetic of the decode step happens
+here; if the library is missing the import fails (there is no fallback).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libaoh.so")
+
+ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM = 0, 1, 2
+STATUS = {0: "AOH_OK", 1: "AOH_ERR_INVALID_ARG", 2: "AOH_ERR_UNSUPPORTED", 3: "AOH_ERR_ALIGNMENT",
+          4: "AOH_ERR_WORKSPACE", 5: "AOH_ERR_CUDA", 6: "AOH_ERR_DEVICE_CHECK"}
+
+EXPORTS = (
+    "aoh_status_string", "aoh_version", "aoh_device_check", "aoh_pack_dominant", "aoh_tip_score",
+    "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
+    "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
+)
+
+
+class AohError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {STATUS.get(status, status)}")
+
+
+class KVCache(ctypes.Structure):
+    """Mirror of ``aoh_kv_cache`` (include/aoh.h)."""
+
+    _fields_ = [
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+        ("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("max_len", ctypes.c_int32), ("total_tokens", ctypes.c_int64), ("stride_tok", ctypes.c_int64),
+        ("stride_head", ctypes.c_int64), ("k_dom", ctypes.c_void_p), ("k_dom_cols", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libaoh.so once (after torch, so that it binds to torch's CUDA runtime)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built: run `python -m token_sparse_decode_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, F32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        KVP = ctypes.POINTER(KVCache)
+        sig = {
+            "aoh_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "aoh_version": (I32, []),
+            "aoh_device_check": (ctypes.c_int, [P, P]),
+            "aoh_pack_dominant": (ctypes.c_int, [KVP, P, I32, P, I32, P]),
+            "aoh_tip_score": (ctypes.c_int, [P, I32, KVP, P, I32, P, P]),
+            "aoh_topk_select": (ctypes.c_int, [P, KVP, I32, P, I32, P, P, P]),
+            "aoh_sparse_decode": (ctypes.c_int, [P, I32, KVP, P, I32, I32, P, I32, P, F32, P, P, P, P, SZ, P]),
+            "aoh_sparse_decode_workspace_size": (SZ, [KVP, I32, I32]),
+            "aoh_stream_decode": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P, SZ, P]),
+            "aoh_stream_decode_workspace_size": (SZ, [KVP, I32, P, I32, I32]),
+            "aoh_shared_index_decode": (ctypes.c_int, [P, I32, I32, KVP, P, P, I32, F32, P, P, SZ, P]),
+            "aoh_shared_index_decode_workspace_size": (SZ, [KVP, I32, I32, I32]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise AohError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _host_u8(arr) -> Optional[ctypes.Array]:
+    if arr is None:
+        return None
+    vals = [int(x) for x in (arr.tolist() if hasattr(arr, "tolist") else arr)]
+    return (ctypes.c_uint8 * len(vals))(*vals)
+
+
+def make_kv(k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
+            k_dom: Optional[torch.Tensor] = None) -> KVCache:
+    """Describe a cache held in torch tensors k, v of shape [T, Hkv, d] (bf16, last dim contiguous)."""
+    assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16 and k.is_cuda and v.is_cuda
+    assert k.shape == v.shape and k.stride() == v.stride() and k.stride(2) == 1
+    assert offsets.dtype == torch.int32 and offsets.is_cuda
+    kv = KVCache()
+    kv.k, kv.v, kv.offsets = k.data_ptr(), v.data_ptr(), offsets.data_ptr()
+    kv.batch = offsets.numel() - 1
+    kv.n_kv_heads = k.shape[1]
+    kv.head_dim = k.shape[2]
+    kv.max_len = int(max_len)
+    kv.total_tokens = int(total_tokens)
+    kv.stride_tok = k.stride(0)
+    kv.stride_head = k.stride(1)
+    if k_dom is not None:
+        assert k_dom.dtype == torch.bfloat16 and k_dom.is_cuda and k_dom.is_contiguous()
+        kv.k_dom = k_dom.data_ptr()
+        kv.k_dom_cols = k_dom.shape[-1]
+    return kv
+
+
+def k_dom_cols(n_dom: int) -> int:
+    """Row length of the packed dominant-column copy: 2*n_dom rounded up to 8 * 2^j elements."""
+    c = 8
+    while c < 2 * n_dom:
+        c *= 2
+    return c
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled device buffer (the allocator gives >= 512-byte alignment)."""
+    return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------- entry points
+
+def device_check(stream=None):
+    detail = (ctypes.c_int32 * 4)()
+    st = lib().aoh_device_check(_stream(stream), ctypes.cast(detail, ctypes.c_void_p))
+    return st, list(detail)
+
+
+def pack_dominant(kv: KVCache, idom: torch.Tensor, n_dom: int, k_dom: torch.Tensor, stream=None) -> None:
+    _check("aoh_pack_dominant", lib().aoh_pack_dominant(ctypes.byref(kv), _ptr(idom), n_dom, _ptr(k_dom),
+                                                         k_dom.shape[-1], _stream(stream)))
+
+
+def tip_score(q: torch.Tensor, kv: KVCache, idom: torch.Tensor, n_dom: int, scores: torch.Tensor,
+              stream=None) -> None:
+    _check("aoh_tip_score", lib().aoh_tip_score(_ptr(q), q.shape[-2], ctypes.byref(kv), _ptr(idom), n_dom,
+                                                 _ptr(scores), _stream(stream)))
+
+
+def topk_select(scores: torch.Tensor, kv: KVCache, n_fac: int, n_fac_per_seq: Optional[torch.Tensor],
+                n_fac_cap: int, idx: torch.Tensor, count: torch.Tensor, stream=None) -> None:
+    _check("aoh_topk_select", lib().aoh_topk_select(_ptr(scores), ctypes.byref(kv), n_fac, _ptr(n_fac_per_seq),
+                                                     n_fac_cap, _ptr(idx), _ptr(count), _stream(stream)))
+
+
+def sparse_decode_workspace_size(kv: KVCache, n_q_heads: int, n_fac_cap: int) -> int:
+    return int(lib().aoh_sparse_decode_workspace_size(ctypes.byref(kv), n_q_heads, n_fac_cap))
+
+
+def sparse_decode(q: torch.Tensor, kv: KVCache, idom: torch.Tensor, n_dom: int, n_fac: int,
+                  n_fac_per_seq: Optional[torch.Tensor], n_fac_cap: int, roles, scale: float,
+                  out: torch.Tensor, ws: torch.Tensor, idx_out: Optional[torch.Tensor] = None,
+                  count_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    r = _host_u8(roles)
+    _check("aoh_sparse_decode", lib().aoh_sparse_decode(
+        _ptr(q), q.shape[-2], ctypes.byref(kv), _ptr(idom), n_dom, n_fac, _ptr(n_fac_per_seq), n_fac_cap,
+        None if r is None else ctypes.cast(r, ctypes.c_void_p), float(scale), _ptr(out), _ptr(idx_out),
+        _ptr(count_out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def stream_decode_workspace_size(kv: KVCache, n_q_heads: int, roles, sink: int, window: int) -> int:
+    r = _host_u8(roles)
+    return int(lib().aoh_stream_decode_workspace_size(ctypes.byref(kv), n_q_heads,
+                                                      ctypes.cast(r, ctypes.c_void_p), sink, window))
+
+
+def stream_decode(q: torch.Tensor, kv: KVCache, roles, sink: int, window: int, scale: float,
+                  out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    r = _host_u8(roles)
+    _check("aoh_stream_decode", lib().aoh_stream_decode(
+        _ptr(q), q.shape[-2], ctypes.byref(kv), ctypes.cast(r, ctypes.c_void_p), sink, window, float(scale),
+        _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def shared_index_decode_workspace_size(kv: KVCache, n_layers: int, n_q_heads: int, n_fac_cap: int) -> int:
+    return int(lib().aoh_shared_index_decode_workspace_size(ctypes.byref(kv), n_layers, n_q_heads, n_fac_cap))
+
+
+def shared_index_decode(q_layers: torch.Tensor, kv: KVCache, idx: torch.Tensor, count: torch.Tensor,
+                        n_fac_cap: int, scale: float, out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    _check("aoh_shared_index_decode", lib().aoh_shared_index_decode(
+        _ptr(q_layers), q_layers.shape[0], q_layers.shape[-2], ctypes.byref(kv), _ptr(idx), _ptr(count),
+        n_fac_cap, float(scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))

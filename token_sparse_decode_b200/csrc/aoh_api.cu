@@ -1,0 +1,524 @@
+// C ABI of the token-sparse decode step: argument checks on the host, then
+// asynchronous launches on the caller's stream.  Declarations and the contract
+// of every entry point are in include/aoh.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "aoh.h"
+#include "device_common.cuh"
+#include "flash_gather.cuh"
+#include "tip_score.cuh"
+#include "topk_select.cuh"
+
+using namespace aoh;
+
+namespace {
+
+constexpr int kSmCount = 148;        // B200
+constexpr int kMaxQRows = 32;        // query rows per KV head in one gather kernel (4 n-tiles)
+constexpr int kSelMaxCluster = 8;    // portable cluster size
+constexpr size_t kSelSmemCap = 200 * 1024;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+aoh_status check_kv(const aoh_kv_cache* kv) {
+  if (!kv) return AOH_ERR_INVALID_ARG;
+  if (kv->batch < 0 || kv->n_kv_heads < 1 || kv->n_kv_heads > kMaxHeads) return AOH_ERR_INVALID_ARG;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return AOH_ERR_UNSUPPORTED;
+  if (kv->max_len < 0 || kv->total_tokens < 0 || kv->total_tokens >= (int64_t(1) << 31))
+    return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0) return AOH_OK;
+  if (!kv->k || !kv->v || !kv->offsets) return AOH_ERR_INVALID_ARG;
+  if (kv->stride_tok < 1 || kv->stride_head < 1) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(kv->k) || !aligned16(kv->v) || (kv->stride_tok % 8) || (kv->stride_head % 8))
+    return AOH_ERR_ALIGNMENT;
+  if (kv->k_dom) {
+    if (kv->k_dom_cols < 8 || kv->k_dom_cols > 128 || (kv->k_dom_cols % 8)) return AOH_ERR_INVALID_ARG;
+    if (!aligned16(kv->k_dom)) return AOH_ERR_ALIGNMENT;
+  }
+  return AOH_OK;
+}
+
+aoh_status check_heads(const aoh_kv_cache* kv, int32_t n_q_heads) {
+  if (n_q_heads < 1 || n_q_heads % kv->n_kv_heads) return AOH_ERR_INVALID_ARG;
+  return AOH_OK;
+}
+
+aoh_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AOH_OK : AOH_ERR_CUDA; }
+
+template <typename F>
+aoh_status set_smem(F* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return AOH_OK;
+  return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+}
+
+// ------------------------------------------------------------------ gather-kernel geometry
+struct FdGeom {
+  int chunk;
+  int max_splits;
+  int nqp;
+  int rows;
+  size_t ticket_bytes, ml_bytes, acc_bytes;
+};
+
+FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
+  FdGeom g{};
+  const int64_t target = int64_t(kSmCount) * 4;
+  int64_t chunk = ceil_div(std::max<int64_t>(work_tokens, 1), target);
+  chunk = ceil_div(chunk, kFdTS) * kFdTS;
+  chunk = std::min<int64_t>(std::max<int64_t>(chunk, kFdTS), 8192);
+  g.chunk = (int)chunk;
+  g.max_splits = (int)std::max<int64_t>(1, ceil_div(std::max<int64_t>(n_max, 1), chunk));
+  g.nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
+  g.rows = rows;
+  g.ticket_bytes = align256(sizeof(int32_t) * (size_t)std::max(rows, 1));
+  g.ml_bytes = align256(sizeof(float) * (size_t)rows * g.max_splits * g.nqp * 2);
+  g.acc_bytes = align256(sizeof(float) * (size_t)rows * g.max_splits * g.nqp * d);
+  return g;
+}
+
+size_t fd_bytes(const FdGeom& g) { return g.ticket_bytes + g.ml_bytes + g.acc_bytes; }
+
+// Workspace layout: [tickets][part_ml][part_acc][extra...]; tickets first so that a
+// zero-filled workspace starts with zero tickets.
+void fd_bind(FdecParams& fp, const FdGeom& g, uint8_t* ws) {
+  fp.tickets = reinterpret_cast<int32_t*>(ws);
+  fp.part_ml = reinterpret_cast<float*>(ws + g.ticket_bytes);
+  fp.part_acc = reinterpret_cast<float*>(ws + g.ticket_bytes + g.ml_bytes);
+  fp.chunk = g.chunk;
+  fp.max_splits = g.max_splits;
+}
+
+template <int D, int NT>
+aoh_status launch_fd_t(const FdecParams& fp, int n_listed, int B, cudaStream_t st) {
+  const size_t smem = FdTile<D>::kSmem;
+  static bool configured = false;  // attribute is per function and process-wide
+  if (!configured) {
+    aoh_status s = set_smem(flash_gather_kernel<D, NT>, smem);
+    if (s != AOH_OK) return s;
+    configured = true;
+  }
+  dim3 grid(fp.max_splits, n_listed, B);
+  flash_gather_kernel<D, NT><<<grid, kFdThreads, smem, st>>>(fp);
+  return cuda_status(cudaGetLastError());
+}
+
+aoh_status launch_fd(const FdecParams& fp, int d, int nqp, int n_listed, int B, cudaStream_t st) {
+  if (d == 128) {
+    if (nqp == 8) return launch_fd_t<128, 1>(fp, n_listed, B, st);
+    if (nqp == 16) return launch_fd_t<128, 2>(fp, n_listed, B, st);
+    return launch_fd_t<128, 4>(fp, n_listed, B, st);
+  }
+  if (nqp == 8) return launch_fd_t<64, 1>(fp, n_listed, B, st);
+  if (nqp == 16) return launch_fd_t<64, 2>(fp, n_listed, B, st);
+  return launch_fd_t<64, 4>(fp, n_listed, B, st);
+}
+
+// ------------------------------------------------------------------ TIP scan
+aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom,
+                      float* scores, const uint8_t* heads, int n_listed, cudaStream_t st) {
+  TipParams tp{};
+  tp.q = static_cast<const uint16_t*>(q);
+  tp.idom = idom;
+  tp.offsets = kv->offsets;
+  tp.scores = scores;
+  tp.T = (int32_t)kv->total_tokens;
+  tp.Hq = Hq;
+  tp.Hkv = kv->n_kv_heads;
+  tp.d = kv->head_dim;
+  tp.G = Hq / kv->n_kv_heads;
+  tp.n_dom = n_dom;
+  if (kv->k_dom) {
+    if (2 * n_dom > kv->k_dom_cols) return AOH_ERR_INVALID_ARG;
+    tp.src = static_cast<const uint16_t*>(kv->k_dom);
+    tp.row_stride_tok = kv->k_dom_cols;
+    tp.row_stride_head = kv->total_tokens * kv->k_dom_cols;
+    tp.row_len = kv->k_dom_cols;
+    tp.packed = 1;
+  } else {
+    tp.src = static_cast<const uint16_t*>(kv->k);
+    tp.row_stride_tok = kv->stride_tok;
+    tp.row_stride_head = kv->stride_head;
+    tp.row_len = kv->head_dim;
+    tp.packed = 0;
+  }
+  memcpy(tp.heads, heads, n_listed);
+  const int64_t rows = int64_t(kv->batch) * n_listed;
+  int64_t tile = ceil_div(std::max<int64_t>(1, int64_t(kv->max_len) * rows), int64_t(kSmCount) * 6);
+  tile = std::min<int64_t>(std::max<int64_t>(ceil_div(tile, 256) * 256, 256), 8192);
+  tp.tile = (int32_t)tile;
+  dim3 grid((unsigned)std::max<int64_t>(1, ceil_div(kv->max_len, tile)), n_listed, kv->batch);
+  int lanes = 1;
+  while (lanes * 8 < tp.row_len) lanes <<= 1;
+  switch (lanes) {
+    case 1: tip_score_kernel<1><<<grid, kTipThreads, 0, st>>>(tp); break;
+    case 2: tip_score_kernel<2><<<grid, kTipThreads, 0, st>>>(tp); break;
+    case 4: tip_score_kernel<4><<<grid, kTipThreads, 0, st>>>(tp); break;
+    case 8: tip_score_kernel<8><<<grid, kTipThreads, 0, st>>>(tp); break;
+    default: tip_score_kernel<16><<<grid, kTipThreads, 0, st>>>(tp); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------------------ top-k select
+aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
+                         int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
+                         cudaStream_t st) {
+  SelectParams sp{};
+  sp.scores = scores;
+  sp.offsets = kv->offsets;
+  sp.n_fac_per_seq = nfps;
+  sp.idx = idx;
+  sp.count = count;
+  sp.T = (int32_t)kv->total_tokens;
+  sp.Hkv = kv->n_kv_heads;
+  sp.n_fac = n_fac;
+  sp.cap = cap;
+  memcpy(sp.heads, heads, n_listed);
+  const int CL = (int)std::min<int64_t>(kSelMaxCluster, std::max<int64_t>(1, ceil_div(kv->max_len, 256)));
+  const int64_t chunk = std::max<int64_t>(4, ceil_div(ceil_div(std::max(kv->max_len, 1), CL), 4) * 4);
+  sp.chunk = (int32_t)chunk;
+  size_t smem = (size_t)chunk * 4;
+  sp.keys_in_smem = smem <= kSelSmemCap;
+  if (!sp.keys_in_smem) smem = 0;
+  static size_t configured = 0;
+  if (smem > configured) {
+    aoh_status s = set_smem(topk_select_kernel, kSelSmemCap);
+    if (s != AOH_OK) return s;
+    configured = kSelSmemCap;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, n_listed, kv->batch);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, topk_select_kernel, sp));
+}
+
+int list_heads(const aoh_kv_cache* kv, const uint8_t* roles, bool want_sparse, uint8_t* out) {
+  int n = 0;
+  for (int g = 0; g < kv->n_kv_heads; ++g) {
+    const uint8_t r = roles ? roles[g] : (uint8_t)AOH_ROLE_SPARSE;
+    const bool sparse = (r == AOH_ROLE_SPARSE);
+    if (sparse == want_sparse) out[n++] = (uint8_t)g;
+  }
+  return n;
+}
+
+aoh_status check_roles(const aoh_kv_cache* kv, const uint8_t* roles) {
+  if (!roles) return AOH_OK;
+  for (int g = 0; g < kv->n_kv_heads; ++g)
+    if (roles[g] > AOH_ROLE_STREAM) return AOH_ERR_INVALID_ARG;
+  return AOH_OK;
+}
+
+// Geometry of the sparse step (depends only on what the size query also sees).
+FdGeom sparse_geom(const aoh_kv_cache* kv, int32_t Hq, int32_t cap) {
+  const int G = Hq / kv->n_kv_heads;
+  const int rows = kv->batch * kv->n_kv_heads;
+  return fd_geom(int64_t(rows) * cap, cap, rows, G, kv->head_dim);
+}
+
+size_t sparse_ws_bytes(const aoh_kv_cache* kv, int32_t Hq, int32_t cap, size_t* off_scores, size_t* off_idx,
+                       size_t* off_count) {
+  const FdGeom g = sparse_geom(kv, Hq, cap);
+  size_t o = fd_bytes(g);
+  *off_scores = o;
+  o += align256(sizeof(float) * (size_t)kv->n_kv_heads * (size_t)kv->total_tokens);
+  *off_idx = o;
+  o += align256(sizeof(int32_t) * (size_t)kv->batch * kv->n_kv_heads * (size_t)cap);
+  *off_count = o;
+  o += align256(sizeof(int32_t) * (size_t)kv->batch * kv->n_kv_heads);
+  return o;
+}
+
+FdGeom stream_geom(const aoh_kv_cache* kv, int32_t Hq, const uint8_t* roles, int32_t sink, int32_t window) {
+  int64_t n_max = 0, work = 0;
+  for (int g = 0; g < kv->n_kv_heads; ++g) {
+    const uint8_t r = roles[g];
+    if (r == AOH_ROLE_SPARSE) continue;
+    const int64_t L = kv->max_len;
+    const int64_t n = (r == AOH_ROLE_DENSE) ? L : std::min<int64_t>(L, int64_t(sink) + window);
+    n_max = std::max(n_max, n);
+    work += n * kv->batch;
+  }
+  const int G = Hq / kv->n_kv_heads;
+  return fd_geom(work, n_max, kv->batch * kv->n_kv_heads, G, kv->head_dim);
+}
+
+FdGeom shared_geom(const aoh_kv_cache* kv, int32_t n_layers, int32_t Hq, int32_t cap) {
+  const int G = Hq / kv->n_kv_heads;
+  const int rows = kv->batch * kv->n_kv_heads;
+  return fd_geom(int64_t(rows) * cap, cap, rows, n_layers * G, kv->head_dim);
+}
+
+bool ws_ok(const void* ws, size_t have, size_t need) {
+  if (need == 0) return true;
+  return ws && have >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0;
+}
+
+}  // namespace
+
+// ===================================================================== exported
+extern "C" {
+
+const char* aoh_status_string(aoh_status s) {
+  switch (s) {
+    case AOH_OK: return "ok";
+    case AOH_ERR_INVALID_ARG: return "invalid argument";
+    case AOH_ERR_UNSUPPORTED: return "unsupported shape";
+    case AOH_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case AOH_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case AOH_ERR_CUDA: return "CUDA error";
+    case AOH_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+int32_t aoh_version(void) { return 1; }
+
+aoh_status aoh_device_check(void* stream, int32_t* detail) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return AOH_ERR_CUDA;
+  int h[4] = {0, 0, 0, 0};
+  if (cudaMemcpyFromSymbol(h, g_device_error, sizeof(h)) != cudaSuccess) return AOH_ERR_CUDA;
+  if (detail) memcpy(detail, h, sizeof(h));
+  if (h[0] == 0) return AOH_OK;
+  const int z[4] = {0, 0, 0, 0};
+  if (cudaMemcpyToSymbol(g_device_error, z, sizeof(z)) != cudaSuccess) return AOH_ERR_CUDA;
+  return AOH_ERR_DEVICE_CHECK;
+}
+
+aoh_status aoh_pack_dominant(const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom, void* k_dom,
+                             int32_t k_dom_cols, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if (n_dom < 1 || n_dom > kv->head_dim / 2) return AOH_ERR_INVALID_ARG;
+  if (k_dom_cols < 2 * n_dom || k_dom_cols > 128 || (k_dom_cols % 8)) return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0 || kv->total_tokens == 0) return AOH_OK;
+  if (!idom || !k_dom) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(k_dom)) return AOH_ERR_ALIGNMENT;
+  PackParams pp{};
+  pp.k = static_cast<const uint16_t*>(kv->k);
+  pp.idom = idom;
+  pp.k_dom = static_cast<uint16_t*>(k_dom);
+  pp.stride_tok = kv->stride_tok;
+  pp.stride_head = kv->stride_head;
+  pp.T = (int32_t)kv->total_tokens;
+  pp.Hkv = kv->n_kv_heads;
+  pp.d = kv->head_dim;
+  pp.n_dom = n_dom;
+  pp.cols = k_dom_cols;
+  const int64_t total = int64_t(pp.Hkv) * pp.T * pp.cols;
+  const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), int64_t(kSmCount) * 16);
+  pack_dominant_kernel<<<blocks, 256, 0, as_stream(stream)>>>(pp);
+  return cuda_status(cudaGetLastError());
+}
+
+aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv, const int32_t* idom,
+                         int32_t n_dom, float* scores, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if (n_dom < 1 || n_dom > kv->head_dim / 2) return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0 || kv->total_tokens == 0) return AOH_OK;
+  if (!q || !idom || !scores) return AOH_ERR_INVALID_ARG;
+  uint8_t heads[kMaxHeads];
+  const int n = list_heads(kv, nullptr, true, heads);
+  return launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n, as_stream(stream));
+}
+
+aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
+                           const int32_t* n_fac_per_seq, int32_t n_fac_cap, int32_t* idx, int32_t* count,
+                           void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if (n_fac_cap < 1) return AOH_ERR_INVALID_ARG;
+  if (!n_fac_per_seq && (n_fac < 0 || n_fac > n_fac_cap)) return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0) return AOH_OK;
+  if (!idx || !count || (!scores && kv->total_tokens > 0)) return AOH_ERR_INVALID_ARG;
+  uint8_t heads[kMaxHeads];
+  const int n = list_heads(kv, nullptr, true, heads);
+  return launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
+}
+
+size_t aoh_sparse_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, int32_t n_fac_cap) {
+  if (check_kv(kv) != AOH_OK || check_heads(kv, n_q_heads) != AOH_OK || n_fac_cap < 1) return 0;
+  if (n_q_heads / kv->n_kv_heads > kMaxQRows) return 0;
+  size_t a, b, c;
+  return sparse_ws_bytes(kv, n_q_heads, n_fac_cap, &a, &b, &c);
+}
+
+aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv, const int32_t* idom,
+                             int32_t n_dom, int32_t n_fac, const int32_t* n_fac_per_seq, int32_t n_fac_cap,
+                             const uint8_t* roles, float scale, float* out, int32_t* idx_out,
+                             int32_t* count_out, void* workspace, size_t workspace_bytes, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if ((s = check_roles(kv, roles)) != AOH_OK) return s;
+  const int G = n_q_heads / kv->n_kv_heads;
+  if (G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (n_dom < 1 || n_dom > kv->head_dim / 2) return AOH_ERR_INVALID_ARG;
+  if (n_fac_cap < 1) return AOH_ERR_INVALID_ARG;
+  if (!n_fac_per_seq && (n_fac < 0 || n_fac > n_fac_cap)) return AOH_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  if ((idx_out == nullptr) != (count_out == nullptr)) return AOH_ERR_INVALID_ARG;
+  if (kv->k_dom && 2 * n_dom > kv->k_dom_cols) return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0) return AOH_OK;
+  if (!q || !idom || !out) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(q)) return AOH_ERR_ALIGNMENT;
+  size_t off_scores, off_idx, off_count;
+  const size_t need = sparse_ws_bytes(kv, n_q_heads, n_fac_cap, &off_scores, &off_idx, &off_count);
+  if (!ws_ok(workspace, workspace_bytes, need)) return AOH_ERR_WORKSPACE;
+  uint8_t heads[kMaxHeads];
+  const int n_listed = list_heads(kv, roles, true, heads);
+  if (n_listed == 0) return AOH_OK;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* scores = reinterpret_cast<float*>(ws + off_scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + off_idx);
+  int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + off_count);
+
+  if (kv->total_tokens > 0) {
+    if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st)) != AOH_OK) return s;
+  }
+  if ((s = launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st)) != AOH_OK)
+    return s;
+
+  const FdGeom geo = sparse_geom(kv, n_q_heads, n_fac_cap);
+  FdecParams fp{};
+  fp.q = static_cast<const uint16_t*>(q);
+  fp.k = static_cast<const uint16_t*>(kv->k);
+  fp.v = static_cast<const uint16_t*>(kv->v);
+  fp.offsets = kv->offsets;
+  fp.idx = idx;
+  fp.count = cnt;
+  fp.out = out;
+  fp.stride_tok = kv->stride_tok;
+  fp.stride_head = kv->stride_head;
+  fp.B = kv->batch;
+  fp.Hq = n_q_heads;
+  fp.Hkv = kv->n_kv_heads;
+  fp.G = G;
+  fp.NQ = G;
+  fp.cap = n_fac_cap;
+  fp.list_mode = 1;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  memcpy(fp.heads, heads, n_listed);
+  fd_bind(fp, geo, ws);
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st);
+}
+
+size_t aoh_stream_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, const uint8_t* roles,
+                                        int32_t sink, int32_t window) {
+  if (check_kv(kv) != AOH_OK || check_heads(kv, n_q_heads) != AOH_OK || !roles) return 0;
+  if (check_roles(kv, roles) != AOH_OK || sink < 0 || window < 0) return 0;
+  if (n_q_heads / kv->n_kv_heads > kMaxQRows) return 0;
+  return fd_bytes(stream_geom(kv, n_q_heads, roles, sink, window));
+}
+
+aoh_status aoh_stream_decode(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv, const uint8_t* roles,
+                             int32_t sink, int32_t window, float scale, float* out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if (!roles) return AOH_ERR_INVALID_ARG;
+  if ((s = check_roles(kv, roles)) != AOH_OK) return s;
+  const int G = n_q_heads / kv->n_kv_heads;
+  if (G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (sink < 0 || window < 0 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0) return AOH_OK;
+  if (!q || !out) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(q)) return AOH_ERR_ALIGNMENT;
+  const FdGeom geo = stream_geom(kv, n_q_heads, roles, sink, window);
+  if (!ws_ok(workspace, workspace_bytes, fd_bytes(geo))) return AOH_ERR_WORKSPACE;
+  uint8_t heads[kMaxHeads];
+  const int n_listed = list_heads(kv, roles, false, heads);
+  if (n_listed == 0) return AOH_OK;
+  FdecParams fp{};
+  fp.q = static_cast<const uint16_t*>(q);
+  fp.k = static_cast<const uint16_t*>(kv->k);
+  fp.v = static_cast<const uint16_t*>(kv->v);
+  fp.offsets = kv->offsets;
+  fp.out = out;
+  fp.stride_tok = kv->stride_tok;
+  fp.stride_head = kv->stride_head;
+  fp.B = kv->batch;
+  fp.Hq = n_q_heads;
+  fp.Hkv = kv->n_kv_heads;
+  fp.G = G;
+  fp.NQ = G;
+  fp.cap = 0;
+  fp.list_mode = 0;
+  fp.sink = sink;
+  fp.window = window;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  memcpy(fp.heads, heads, n_listed);
+  memcpy(fp.roles, roles, kv->n_kv_heads);
+  fd_bind(fp, geo, static_cast<uint8_t*>(workspace));
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream));
+}
+
+size_t aoh_shared_index_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_layers, int32_t n_q_heads,
+                                              int32_t n_fac_cap) {
+  if (check_kv(kv) != AOH_OK || check_heads(kv, n_q_heads) != AOH_OK || n_layers < 1 || n_fac_cap < 1) return 0;
+  if (int64_t(n_layers) * (n_q_heads / kv->n_kv_heads) > kMaxQRows) return 0;
+  return fd_bytes(shared_geom(kv, n_layers, n_q_heads, n_fac_cap));
+}
+
+aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32_t n_q_heads,
+                                   const aoh_kv_cache* kv, const int32_t* idx, const int32_t* count,
+                                   int32_t n_fac_cap, float scale, float* out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if (n_layers < 1 || n_fac_cap < 1 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  const int G = n_q_heads / kv->n_kv_heads;
+  if (int64_t(n_layers) * G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (kv->batch == 0) return AOH_OK;
+  if (!q_layers || !idx || !count || !out) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(q_layers)) return AOH_ERR_ALIGNMENT;
+  const FdGeom geo = shared_geom(kv, n_layers, n_q_heads, n_fac_cap);
+  if (!ws_ok(workspace, workspace_bytes, fd_bytes(geo))) return AOH_ERR_WORKSPACE;
+  uint8_t heads[kMaxHeads];
+  const int n_listed = list_heads(kv, nullptr, true, heads);
+  FdecParams fp{};
+  fp.q = static_cast<const uint16_t*>(q_layers);
+  fp.k = static_cast<const uint16_t*>(kv->k);
+  fp.v = static_cast<const uint16_t*>(kv->v);
+  fp.offsets = kv->offsets;
+  fp.idx = idx;
+  fp.count = count;
+  fp.out = out;
+  fp.stride_tok = kv->stride_tok;
+  fp.stride_head = kv->stride_head;
+  fp.B = kv->batch;
+  fp.Hq = n_q_heads;
+  fp.Hkv = kv->n_kv_heads;
+  fp.G = G;
+  fp.NQ = n_layers * G;
+  fp.cap = n_fac_cap;
+  fp.list_mode = 1;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  memcpy(fp.heads, heads, n_listed);
+  fd_bind(fp, geo, static_cast<uint8_t*>(workspace));
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,346 @@
+// Gather flash-decode: exact softmax attention of NQ query rows over a list of
+// cached token positions of one KV head.
+//
+// Serves three operations with one body:
+//   * focused attention over the selected tokens (FASA: Frequency-aware Sparse
+//     Attention, §2.B.2): positions come from the top-N_fac index, NQ = G;
+//   * retrieval / streaming heads (AoH summary, Metodología §4): positions are
+//     [0, L) or [0, min(S, L)) U [max(S, L - W), L), NQ = G;
+//   * the shared-index cross-decoder layers ("Cómo funciona CLSA"): one index,
+//     NQ = n_layers * G query rows read every gathered K/V row once.
+//
+// Work split: blockIdx = (split, listed KV head, sequence).  A CTA owns `chunk`
+// consecutive list entries, streams their K and V rows through a 3-stage
+// cp.async pipeline into 128-byte-swizzled shared tiles (the layout a TMA
+// 128B-swizzle load produces), and runs the contraction on tensor cores with the
+// tokens on the M side:
+//     S^T[16 tok x 8 q] = K[16 tok x d] . Q^T[d x 8 q]          (m16n8k16, bf16)
+//     O^T[d x 8 q]     += V^T[d x 16 tok] . P^T[16 tok x 8 q]
+// so G <= 8 query rows fill the N = 8 side of one MMA (G = 7: 7/8 useful) instead
+// of padding 16 rows.  P goes from the accumulator layout to the B-operand layout
+// with movmatrix.trans.  Softmax is online in fp32 (exp2 domain).  Each CTA
+// writes (m, l, acc) for its chunk; the last CTA of a row (atomic ticket) merges
+// the partials and writes the fp32 output, then re-arms the ticket to zero.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace aoh {
+
+constexpr int kFdThreads = 128;  // 4 warps
+constexpr int kFdTS = 64;        // tokens per pipeline stage
+constexpr int kFdStages = 3;
+
+struct FdecParams {
+  const uint16_t* q;         // row (layer l, b, h) at q + ((l * B + b) * Hq + h) * D
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* offsets;    // [B + 1]
+  const int32_t* idx;        // list mode: [B][Hkv][cap]
+  const int32_t* count;      // list mode: [B][Hkv]
+  float* out;                // row (l, b, h) at out + ((l * B + b) * Hq + h) * D
+  float* part_ml;            // [rows][max_splits][NQP][2]
+  float* part_acc;           // [rows][max_splits][NQP][D]
+  int32_t* tickets;          // [rows], zero between calls
+  int64_t stride_tok, stride_head;
+  int32_t B, Hq, Hkv, G, NQ, cap;
+  int32_t chunk;             // list entries per CTA, multiple of kFdTS
+  int32_t max_splits;
+  int32_t list_mode;         // 1: positions from idx/count; 0: role ranges
+  int32_t sink, window;
+  float scale_log2;          // softmax scale * log2(e)
+  uint8_t heads[kMaxHeads];  // listed KV heads (blockIdx.y)
+  uint8_t roles[kMaxHeads];  // role of every KV head (range mode)
+};
+
+template <int D>
+struct FdTile {
+  static constexpr int kTileBytes = kFdTS * D * 2;      // one of K or V per stage
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kSmem = kFdStages * kStageBytes;
+};
+
+// Byte offset of (row r, dim dd) in a [kFdTS x D] bf16 tile stored as D/64 column
+// halves of [kFdTS x 128 B], 16-byte chunks XOR-swizzled by (r mod 8).
+__device__ __forceinline__ uint32_t fd_tile_off(int r, int dd) {
+  const int half = dd >> 6;
+  const int cc = (dd & 63) >> 3;
+  return (uint32_t)(half * (kFdTS * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecParams p) {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
+  constexpr int KS = D / 16;         // k-steps of QK, m-tiles of PV
+  constexpr int WT = 4 / NT;         // token groups (warps sharing one n-tile)
+  constexpr int SUB = kFdTS / 16;    // 16-token sub-tiles per stage
+  constexpr int NQP = NT * 8;        // padded query rows
+  constexpr int CPR = D / 8;         // 16-byte chunks per row
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.z;
+  const int y = blockIdx.y;
+  const int g = p.heads[y];
+  const int split = blockIdx.x;
+  const int row_id = b * gridDim.y + y;
+  const int off = p.offsets[b];
+  const int L = p.offsets[b + 1] - off;
+
+  // ---- the row's list of positions
+  int n, ra = 0, rb = 0;
+  const int32_t* lst = nullptr;
+  if (p.list_mode) {
+    n = p.count[b * p.Hkv + g];
+    if (n > p.cap) {
+      if (split == 0 && tid == 0) record_error(kCheckCount, b, g, n);
+      n = p.cap;
+    }
+    n = max(n, 0);
+    lst = p.idx + ((int64_t)b * p.Hkv + g) * p.cap;
+  } else {
+    if (p.roles[g] == 1) {  // DENSE
+      ra = L;
+      rb = L;
+    } else {                // STREAM
+      ra = min(p.sink, L);
+      rb = max(ra, L - p.window);
+    }
+    n = ra + (L - rb);
+  }
+  const int nsplit = (n + p.chunk - 1) / p.chunk;
+
+  if (n == 0) {  // nothing to attend to: zero rows
+    if (split == 0) {
+      for (int e = tid; e < p.NQ * D; e += kFdThreads) {
+        const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
+        p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + e % D] = 0.f;
+      }
+    }
+    return;
+  }
+  if (split >= nsplit) return;
+  const int j0 = split * p.chunk;
+  const int ntok = min(n, j0 + p.chunk) - j0;
+  const int nstages = (ntok + kFdTS - 1) / kFdTS;
+
+  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const uint32_t sbase = smem_u32(smem);
+
+  auto issue_stage = [&](int st) {
+    if (st < nstages) {
+      const uint32_t kt = sbase + (st % kFdStages) * FdTile<D>::kStageBytes;
+      const uint32_t vt = kt + FdTile<D>::kTileBytes;
+#pragma unroll
+      for (int c = tid; c < kFdTS * CPR; c += kFdThreads) {
+        const int r = c / CPR, ch = c % CPR;
+        const int jj = st * kFdTS + r;  // entry within this CTA's chunk
+        bool ok = jj < ntok;
+        int pos = 0;
+        if (ok) {
+          const int j = j0 + jj;
+          if (p.list_mode) {
+            pos = __ldg(lst + j);
+            if (pos < 0 || pos >= L) {
+              if (ch == 0) record_error(kCheckPosition, b, g, pos);
+              ok = false;
+              pos = 0;
+            }
+          } else {
+            pos = j < ra ? j : rb + (j - ra);
+          }
+        }
+        const int64_t eo = (int64_t)pos * p.stride_tok + ch * 8;
+        const uint32_t so = fd_tile_off(r, ch * 8);
+        cp_async_16(kt + so, kbase + eo, ok);
+        cp_async_16(vt + so, vbase + eo, ok);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // ---- Q as B fragments: column n = lane/4 of the warp's n-tile
+  const int nt = warp % NT, tg = warp / NT;
+  uint32_t bq[KS][2];
+  {
+    const int qr = nt * 8 + (lane >> 2);
+    if (qr < p.NQ) {
+      const int l = qr / p.G, h = g * p.G + qr % p.G;
+      const uint16_t* qp = p.q + (((int64_t)l * p.B + b) * p.Hq + h) * D + 2 * (lane & 3);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        bq[ks][0] = *reinterpret_cast<const uint32_t*>(qp + ks * 16);
+        bq[ks][1] = *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8);
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) bq[ks][0] = bq[ks][1] = 0u;
+    }
+  }
+
+  float acc[KS][4];
+#pragma unroll
+  for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // q rows 2*(lane%4) and +1
+
+#pragma unroll
+  for (int s = 0; s < kFdStages - 1; ++s) issue_stage(s);
+
+  for (int st = 0; st < nstages; ++st) {
+    cp_async_wait<kFdStages - 2>();
+    __syncthreads();
+    issue_stage(st + kFdStages - 1);
+    const uint32_t kt = sbase + (st % kFdStages) * FdTile<D>::kStageBytes;
+    const uint32_t vt = kt + FdTile<D>::kTileBytes;
+#pragma unroll
+    for (int i = 0; i < SUB / WT; ++i) {
+      const int u = tg + WT * i;
+      const int nv = ntok - (st * kFdTS + u * 16);  // valid tokens in this sub-tile
+      if (nv <= 0) break;                           // warp-uniform
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int r = u * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int dsel = (lane >> 4) * 8;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(a, kt + fd_tile_off(r, ks * 16 + dsel));
+          mma_16816(s4, a, bq[ks][0], bq[ks][1]);
+        }
+      }
+      const int ta = lane >> 2, tb = ta + 8;
+      const float x0 = ta < nv ? s4[0] * p.scale_log2 : -INFINITY;
+      const float x1 = ta < nv ? s4[1] * p.scale_log2 : -INFINITY;
+      const float x2 = tb < nv ? s4[2] * p.scale_log2 : -INFINITY;
+      const float x3 = tb < nv ? s4[3] * p.scale_log2 : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: nv >= 1
+      const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+      const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+      const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+      l0 = l0 * al0 + p0 + p2;
+      l1 = l1 * al1 + p1 + p3;
+      m0 = mn0;
+      m1 = mn1;
+#pragma unroll
+      for (int i2 = 0; i2 < KS; ++i2) {
+        acc[i2][0] *= al0;
+        acc[i2][1] *= al1;
+        acc[i2][2] *= al0;
+        acc[i2][3] *= al1;
+      }
+      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+      {
+        const int r = u * 16 + (lane & 7) + (lane >> 4) * 8;
+        const int dsel = ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          uint32_t a[4];
+          ldsm_x4_trans(a, vt + fd_tile_off(r, mt * 16 + dsel));
+          mma_16816(acc[mt], a, pb0, pb1);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  // ---- merge the WT token groups of every n-tile, through shared memory
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  __syncthreads();  // every warp is done with the stage buffers
+  float* red_ml = reinterpret_cast<float*>(smem);             // [4 warps][8][2]
+  float* red_acc = red_ml + 4 * 8 * 2;                        // [4 warps][8][D]
+  {
+    const int c0 = 2 * (lane & 3);
+    if (lane < 4) {
+      red_ml[(warp * 8 + c0) * 2 + 0] = m0;
+      red_ml[(warp * 8 + c0) * 2 + 1] = l0;
+      red_ml[(warp * 8 + c0 + 1) * 2 + 0] = m1;
+      red_ml[(warp * 8 + c0 + 1) * 2 + 1] = l1;
+    }
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      const int d0 = mt * 16 + (lane >> 2);
+      red_acc[(warp * 8 + c0) * D + d0] = acc[mt][0];
+      red_acc[(warp * 8 + c0 + 1) * D + d0] = acc[mt][1];
+      red_acc[(warp * 8 + c0) * D + d0 + 8] = acc[mt][2];
+      red_acc[(warp * 8 + c0 + 1) * D + d0 + 8] = acc[mt][3];
+    }
+  }
+  __syncthreads();
+
+  // CTA result for padded query row qr: warps {nt + NT * t : t < WT} hold it.
+  const bool single = (nsplit == 1);
+  float* pml = p.part_ml + ((int64_t)row_id * p.max_splits + split) * NQP * 2;
+  float* pacc = p.part_acc + ((int64_t)row_id * p.max_splits + split) * NQP * D;
+  for (int e = tid; e < NQP * D; e += kFdThreads) {
+    const int qr = e / D, dd = e % D;
+    const int ntq = qr >> 3, cq = qr & 7;
+    float M = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t) * 8 + cq) * 2]);
+    float Ls = 0.f, A = 0.f;
+#pragma unroll
+    for (int t = 0; t < WT; ++t) {
+      const int w = ntq + NT * t;
+      const float mw = red_ml[(w * 8 + cq) * 2];
+      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
+      A += f * red_acc[(w * 8 + cq) * D + dd];
+    }
+    if (single) {
+      if (qr < p.NQ) {
+        const int l = qr / p.G, h = g * p.G + qr % p.G;
+        p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Ls;
+      }
+    } else {
+      pacc[qr * D + dd] = A;
+      if (dd == 0) {
+        pml[qr * 2] = M;
+        pml[qr * 2 + 1] = Ls;
+      }
+    }
+  }
+  if (single) return;
+
+  // ---- split-K combine by the last CTA of the row
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int ticket = atomicAdd(p.tickets + row_id, 1);
+    s_last = (ticket == nsplit - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
+  const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
+  for (int e = tid; e < p.NQ * D; e += kFdThreads) {
+    const int qr = e / D, dd = e % D;
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldcg(rml + ((int64_t)s * NQP + qr) * 2));
+    float Ls = 0.f, A = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+      const float f = exp2f(__ldcg(rml + ((int64_t)s * NQP + qr) * 2) - M);
+      Ls += f * __ldcg(rml + ((int64_t)s * NQP + qr) * 2 + 1);
+      A += f * __ldcg(racc + ((int64_t)s * NQP + qr) * D + dd);
+    }
+    const int l = qr / p.G, h = g * p.G + qr % p.G;
+    p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Ls;
+  }
+  if (tid == 0) p.tickets[row_id] = 0;
+}
+
+}  // namespace aoh

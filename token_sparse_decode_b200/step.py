@@ -1,0 +1,100 @@
+"""Decode steps composed from the C-ABI entry points (device buffers held by torch).
+
+``SparseDecodeStep``: the head-role-split step.  KV heads with role SPARSE run the
+importance scan over their dominant chunks, the top-N_fac select and focused
+attention (one ``aoh_sparse_decode`` call); DENSE / STREAM heads run
+``aoh_stream_decode``.  Both write into one fp32 output.
+
+``SharedIndexStep``: the shared-index cross-decoder stack.  The indexer scores
+every cached token with the full-dimension q.k (``aoh_tip_score`` with every
+chunk), takes one top-k (``aoh_topk_select``) and every layer attends over that
+index (``aoh_shared_index_decode``).
+
+Every call is asynchronous on the current torch stream; nothing is computed in
+Python.
+"""
+
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import binding as B
+
+
+class SparseDecodeStep:
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
+                 n_q_heads: int, roles: Sequence[int], scale: float, idom: Optional[torch.Tensor] = None,
+                 n_fac: int = 0, n_fac_per_seq: Optional[torch.Tensor] = None, n_fac_cap: int = 0,
+                 sink: int = 0, window: int = 0, pack_dominant: bool = True):
+        self.dev = k.device
+        self.k, self.v, self.offsets = k, v, offsets
+        self.roles = [int(r) for r in roles]
+        self.n_q_heads = n_q_heads
+        self.scale = float(scale)
+        self.sink, self.window = int(sink), int(window)
+        self.has_sparse = any(r == B.ROLE_SPARSE for r in self.roles)
+        self.has_stream = any(r != B.ROLE_SPARSE for r in self.roles)
+        self.idom = idom
+        self.n_dom = 0 if idom is None else idom.shape[1]
+        self.n_fac, self.n_fac_per_seq, self.n_fac_cap = int(n_fac), n_fac_per_seq, int(n_fac_cap)
+        batch = offsets.numel() - 1
+        d = k.shape[2]
+        self.k_dom = None
+        if self.has_sparse and pack_dominant:
+            cols = B.k_dom_cols(self.n_dom)
+            self.k_dom = torch.empty((k.shape[1], total_tokens, cols), dtype=torch.bfloat16, device=self.dev)
+            kv0 = B.make_kv(k, v, offsets, max_len, total_tokens)
+            B.pack_dominant(kv0, idom, self.n_dom, self.k_dom)
+        self.kv = B.make_kv(k, v, offsets, max_len, total_tokens, self.k_dom)
+        self.ws_sparse = self.ws_stream = None
+        if self.has_sparse:
+            self.ws_sparse = B.workspace(B.sparse_decode_workspace_size(self.kv, n_q_heads, self.n_fac_cap), self.dev)
+            self.idx = torch.empty((batch, k.shape[1], self.n_fac_cap), dtype=torch.int32, device=self.dev)
+            self.count = torch.empty((batch, k.shape[1]), dtype=torch.int32, device=self.dev)
+        if self.has_stream:
+            self.ws_stream = B.workspace(
+                B.stream_decode_workspace_size(self.kv, n_q_heads, self.roles, self.sink, self.window), self.dev)
+        self.out = torch.zeros((batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
+
+    def __call__(self, q: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        out = self.out if out is None else out
+        if self.has_sparse:
+            B.sparse_decode(q, self.kv, self.idom, self.n_dom, self.n_fac, self.n_fac_per_seq, self.n_fac_cap,
+                            self.roles, self.scale, out, self.ws_sparse, self.idx, self.count)
+        if self.has_stream:
+            B.stream_decode(q, self.kv, self.roles, self.sink, self.window, self.scale, out, self.ws_stream)
+        return out
+
+    def run_host(self, q_host: torch.Tensor, out_host: torch.Tensor, q_dev: torch.Tensor) -> None:
+        """End-to-end call with host buffers: H2D of q, the step, D2H of the output (async)."""
+        q_dev.copy_(q_host, non_blocking=True)
+        self(q_dev)
+        out_host.copy_(self.out, non_blocking=True)
+
+
+class SharedIndexStep:
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
+                 n_layers: int, n_q_heads: int, topk: int, scale: float):
+        self.dev = k.device
+        self.k, self.v, self.offsets = k, v, offsets
+        self.kv = B.make_kv(k, v, offsets, max_len, total_tokens)
+        Hkv, d = k.shape[1], k.shape[2]
+        batch = offsets.numel() - 1
+        self.n_layers, self.n_q_heads, self.topk, self.scale = n_layers, n_q_heads, int(topk), float(scale)
+        self.all_chunks = torch.arange(d // 2, dtype=torch.int32, device=self.dev).repeat(Hkv, 1).contiguous()
+        self.scores = torch.empty((Hkv, max(total_tokens, 1)), dtype=torch.float32, device=self.dev)
+        self.idx = torch.empty((batch, Hkv, self.topk), dtype=torch.int32, device=self.dev)
+        self.count = torch.empty((batch, Hkv), dtype=torch.int32, device=self.dev)
+        self.ws = B.workspace(B.shared_index_decode_workspace_size(self.kv, n_layers, n_q_heads, self.topk), self.dev)
+        self.out = torch.zeros((n_layers, batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
+
+    def index(self, q_index: torch.Tensor) -> None:
+        B.tip_score(q_index, self.kv, self.all_chunks, self.all_chunks.shape[1], self.scores)
+        B.topk_select(self.scores, self.kv, self.topk, None, self.topk, self.idx, self.count)
+
+    def __call__(self, q_index: torch.Tensor, q_layers: torch.Tensor) -> torch.Tensor:
+        self.index(q_index)
+        B.shared_index_decode(q_layers, self.kv, self.idx, self.count, self.topk, self.scale, self.out, self.ws)
+        return self.out
