@@ -106,6 +106,10 @@ const char* aoh_status_string(aoh_status s);
 /* Library ABI version: 1. */
 int32_t aoh_version(void);
 
+/* The cudaError_t code behind the last AOH_ERR_CUDA returned on the calling
+ * host thread (0 if none); cudaGetErrorString() names it. */
+int32_t aoh_last_cuda_error(void);
+
 /*
  * aoh_device_check -- synchronise `stream`, then read and clear this
  * device's error word.  Returns AOH_OK, AOH_ERR_DEVICE_CHECK (and, if

@@ -22,16 +22,18 @@ STATUS = {0: "AOH_OK", 1: "AOH_ERR_INVALID_ARG", 2: "AOH_ERR_UNSUPPORTED", 3: "A
           4: "AOH_ERR_WORKSPACE", 5: "AOH_ERR_CUDA", 6: "AOH_ERR_DEVICE_CHECK"}
 
 EXPORTS = (
-    "aoh_status_string", "aoh_version", "aoh_device_check", "aoh_pack_dominant", "aoh_tip_score",
+    "aoh_status_string", "aoh_version", "aoh_last_cuda_error", "aoh_device_check", "aoh_pack_dominant", "aoh_tip_score",
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
 )
 
 
 class AohError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, cuda_error: int = 0):
         self.status = status
-        super().__init__(f"{fn}: {STATUS.get(status, status)}")
+        self.cuda_error = cuda_error
+        extra = f" (cudaError {cuda_error})" if cuda_error else ""
+        super().__init__(f"{fn}: {STATUS.get(status, status)}{extra}")
 
 
 class KVCache(ctypes.Structure):
@@ -60,6 +62,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "aoh_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "aoh_version": (I32, []),
+            "aoh_last_cuda_error": (I32, []),
             "aoh_device_check": (ctypes.c_int, [P, P]),
             "aoh_pack_dominant": (ctypes.c_int, [KVP, P, I32, P, I32, P]),
             "aoh_tip_score": (ctypes.c_int, [P, I32, KVP, P, I32, P, P]),
@@ -81,7 +84,7 @@ def lib() -> ctypes.CDLL:
 
 def _check(fn: str, status: int) -> None:
     if status != 0:
-        raise AohError(fn, status)
+        raise AohError(fn, status, lib().aoh_last_cuda_error() if status == 5 else 0)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

@@ -51,11 +51,18 @@ aoh_status check_heads(const aoh_kv_cache* kv, int32_t n_q_heads) {
   return AOH_OK;
 }
 
-aoh_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AOH_OK : AOH_ERR_CUDA; }
+thread_local int t_last_cuda_error = 0;
 
+aoh_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return AOH_OK;
+  t_last_cuda_error = (int)e;
+  return AOH_ERR_CUDA;
+}
+
+// Opt in to `bytes` of dynamic shared memory.  Always set: static shared memory
+// counts against the 48 KB default too.
 template <typename F>
 aoh_status set_smem(F* kernel, size_t bytes) {
-  if (bytes <= 48 * 1024) return AOH_OK;
   return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
 }
 
@@ -290,6 +297,8 @@ const char* aoh_status_string(aoh_status s) {
 }
 
 int32_t aoh_version(void) { return 1; }
+
+int32_t aoh_last_cuda_error(void) { return t_last_cuda_error; }
 
 aoh_status aoh_device_check(void* stream, int32_t* detail) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return AOH_ERR_CUDA;
