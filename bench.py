@@ -1,0 +1,513 @@
+"""Benchmark of one token-sparse decode step on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole decode path over one batch: for the default
+Llama-3-8B-shaped layer (batch 4, 32 q / 8 KV heads, d 128, L 32768, 16 of 64
+dominant chunks, N_fac 2048) that is the importance scan, the top-N_fac select
+and focused attention of every KV head (``aoh_sparse_decode``), plus the
+window attention of DENSE / STREAM heads when the workload has any.  The metric
+is KV tokens scanned per second (sum over sequences of L_b per step, all ranks
+together), and the algorithmic HBM bytes per second of the step and of its
+dominant kernel against the measured copy bandwidth.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
+the launching stream; L2 is flushed (a 2 x L2 buffer is rewritten) between
+steps, outside the events.  Barrier + synchronize on both sides, max over
+ranks.  Multi-GPU: every rank decodes its own independent batch (weak scaling,
+no collective on the data path); NCCL is used only for the barrier and the
+max-reduction of the timings.
+
+``--impl reference`` times the float64 CPU oracle on the host cores instead
+(same metric and workload, each step a bounded sample of rows).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import ROLE_SPARSE, make_workload, preset  # noqa: E402
+
+METRIC = "sparse decode: KV tokens scanned/s/GPU; achieved HBM GB/s vs B200 peak"
+DEFAULT_WORKLOAD = "llama8b_gqa4_L32k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------------------ bookkeeping
+
+def algorithmic_bytes(w) -> dict:
+    """Bytes the method must move per step (inputs' K / V columns and rows; q and outputs excluded).
+
+    importance scan: 4 * n_dom bytes per (token, SPARSE KV head) with the packed dominant columns;
+    focused attention: 4 * d bytes (a K row and a V row) per selected token and KV head;
+    DENSE / STREAM heads: 4 * d bytes per attended token; shared index: the indexer's full K rows
+    (2 * d bytes per token and head) plus 4 * d per indexed token and head.
+    """
+    sp = w.spec
+    d = sp.head_dim
+    L = w.lengths.astype(np.int64)
+    roles = w.roles.numpy()
+    out = {"tip": 0, "fac": 0, "window": 0, "indexer": 0, "gather": 0}
+    if sp.n_layers > 0:
+        out["indexer"] = int(L.sum()) * sp.n_kv_heads * d * 2
+        out["gather"] = int(np.minimum(L, sp.topk_shared).sum()) * sp.n_kv_heads * 4 * d
+    else:
+        n_sparse = int((roles == ROLE_SPARSE).sum())
+        nfac = w.n_fac_per_seq.numpy().astype(np.int64)
+        out["tip"] = int(L.sum()) * n_sparse * 4 * sp.n_dom
+        out["fac"] = int(np.minimum(L, nfac).sum()) * n_sparse * 4 * d
+        for g, r in enumerate(roles):
+            if r == 1:
+                out["window"] += int(L.sum()) * 4 * d
+            elif r == 2:
+                a = np.minimum(L, sp.sink)
+                n = a + (L - np.maximum(a, L - sp.window))
+                out["window"] += int(n.sum()) * 4 * d
+    out["total"] = sum(v for k, v in out.items())
+    return out
+
+
+def measured_peak_gbs():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "token_sparse_decode_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            data = json.load(f)
+        ent = data[workload][kernel]
+        if ent.get("source_hash") != kernel_source_hash():
+            return None
+        return int(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        loaded = [x for x in sm if smax and x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ our arm
+
+def build_step(w, dev):
+    from token_sparse_decode_b200.step import SharedIndexStep, SparseDecodeStep
+
+    k, v = w.k.to(dev), w.v.to(dev)
+    offsets = w.offsets.to(dev)
+    if w.spec.n_layers > 0:
+        step = SharedIndexStep(k, v, offsets, w.max_len, w.total_tokens, w.spec.n_layers, w.spec.n_q_heads,
+                               w.spec.topk_shared, w.scale)
+        q = (w.q.to(dev), w.q_layers.to(dev))
+        return step, q
+    idom = None if w.idom is None else w.idom.to(dev)
+    step = SparseDecodeStep(k, v, offsets, w.max_len, w.total_tokens, w.spec.n_q_heads, w.roles.tolist(),
+                            w.scale, idom=idom, n_fac=int(w.n_fac_per_seq.max()),
+                            n_fac_per_seq=w.n_fac_per_seq.to(dev), n_fac_cap=int(w.n_fac_per_seq.max()),
+                            sink=w.spec.sink, window=w.spec.window)
+    return step, (w.q.to(dev),)
+
+
+def launches_per_step(w) -> int:
+    if w.spec.n_layers > 0:
+        return 3  # indexer scan, top-k, shared-index gather
+    roles = w.roles.numpy()
+    n = 0
+    if (roles == ROLE_SPARSE).any():
+        n += 3    # importance scan, top-k, focused attention
+    if (roles != ROLE_SPARSE).any():
+        n += 1    # window attention
+    return n
+
+
+def stage_timing(w, step, q, steps: int, flush) -> dict:
+    """Per-kernel device time (CUDA events on the launching stream), same inputs, L2 flushed."""
+    from token_sparse_decode_b200 import binding as B
+
+    st = torch.cuda.current_stream()
+    res = {}
+    if w.spec.n_layers > 0:
+        names = ["indexer_scan", "topk_select", "shared_gather"]
+        fns = [lambda: B.tip_score(q[0], step.kv, step.all_chunks, step.all_chunks.shape[1], step.scores),
+               lambda: B.topk_select(step.scores, step.kv, step.topk, None, step.topk, step.idx, step.count),
+               lambda: B.shared_index_decode(q[1], step.kv, step.idx, step.count, step.topk, step.scale, step.out,
+                                             step.ws)]
+    else:
+        if step.ws_sparse is None:
+            return res
+        scores = torch.empty((w.spec.n_kv_heads, max(1, w.total_tokens)), dtype=torch.float32, device=q[0].device)
+        ws1 = torch.zeros_like(step.ws_sparse)
+        kvq = q[0][None]
+        ws2 = None
+        from token_sparse_decode_b200.binding import shared_index_decode_workspace_size, workspace
+
+        ws2 = workspace(shared_index_decode_workspace_size(step.kv, 1, w.spec.n_q_heads, step.n_fac_cap),
+                        q[0].device)
+        out2 = torch.empty((1,) + tuple(step.out.shape), dtype=torch.float32, device=q[0].device)
+        names = ["tip_score", "topk_select", "focused_attention"]
+        fns = [lambda: B.tip_score(q[0], step.kv, step.idom, step.n_dom, scores),
+               lambda: B.topk_select(scores, step.kv, step.n_fac, step.n_fac_per_seq, step.n_fac_cap, step.idx,
+                                     step.count),
+               lambda: B.shared_index_decode(kvq, step.kv, step.idx, step.count, step.n_fac_cap, step.scale, out2,
+                                             ws2)]
+        del ws1
+    for fn in fns:  # warm
+        fn()
+    torch.cuda.synchronize()
+    times = {n: [] for n in names}
+    for _ in range(steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+        evs[0].record(st)
+        for i, fn in enumerate(fns):
+            fn()
+            evs[i + 1].record(st)
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            times[n].append(evs[i].elapsed_time(evs[i + 1]))
+        flush()
+    torch.cuda.synchronize()
+    for n in names:
+        res[n] = float(np.mean(times[n]))
+    return res
+
+
+def capture_graph(fn):
+    """Capture the launches of fn() (all on the current stream) into a CUDA graph."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    spec = preset(args.workload)
+    if world > 1:  # each rank decodes its own independent batch of sequences
+        from dataclasses import replace
+
+        spec = replace(spec, seed=spec.seed + 1000 * rank)
+    w = make_workload(spec)
+    step, q = build_step(w, dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    step(*q)  # first call outside capture (sets kernel attributes)
+    torch.cuda.synchronize()
+    if args.graph:
+        g_step = capture_graph(lambda: step(*q))
+        one = g_step.replay
+    else:
+        def one():
+            return step(*q)
+
+    st = torch.cuda.current_stream()
+    sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    t_wall0 = time.time()
+    for _ in range(args.warmup):
+        one()
+        flush()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs:
+        e0.record(st)
+        one()
+        e1.record(st)
+        flush()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    # keep the GPU loaded until the clock sampler has seen a few samples
+    while time.time() - t_wall0 < 1.5:
+        one()
+        flush()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+
+    # end-to-end through the public API with host buffers: H2D of q, the step, D2H of the output
+    q_host = [t.cpu().pin_memory() for t in q]
+    q_dev = [t.clone() for t in q]
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in q_host)
+    d2h = out_host.numel() * out_host.element_size()
+    def host_step():
+        for a, b_ in zip(q_dev, q_host):
+            a.copy_(b_, non_blocking=True)
+        out = step(*q_dev)
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_one = capture_graph(host_step).replay if args.graph else host_step
+    for _ in range(max(1, args.warmup)):
+        e2e_one()
+        flush()
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        e2e_one()
+        e1.record(st)
+        torch.cuda.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+        flush()
+
+    stages = stage_timing(w, step, q, args.steps if args.steps <= 200 else 200, flush)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    tokens_step = int(w.lengths.sum())
+    ms_step = ms / args.steps
+    value = tokens_step * world / (ms_step * 1e-3)
+    e2e_value = tokens_step * world / (e2e_ms / args.steps * 1e-3)
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = measured_peak_gbs()
+    if w.spec.n_layers > 0:
+        dom, dom_bytes = "indexer_scan", ab["indexer"]
+    else:
+        dom, dom_bytes = "tip_score", ab["tip"]
+        if stages and stages.get("focused_attention", 0) > stages.get("tip_score", 0):
+            dom, dom_bytes = "focused_attention", ab["fac"]
+    dom_ms = stages.get(dom)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms else None
+    step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
+    return {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; bf16 N(0,1) post-RoPE q/K, V; planted salient keys where the workload has them)",
+        "config": {
+            "workload": w.spec.name, "batch": w.spec.batch, "seq_len": int(w.max_len),
+            "tokens_per_step_per_gpu": tokens_step, "q_heads": w.spec.n_q_heads, "kv_heads": w.spec.n_kv_heads,
+            "head_dim": w.spec.head_dim, "n_dom": w.spec.n_dom, "n_fac": int(w.n_fac_per_seq.max()),
+            "n_layers": w.spec.n_layers, "parallelism": f"independent sequences per rank x{world}",
+            "l2": "flushed between timed steps (2 x L2 buffer rewritten, outside the events)",
+            "launch": "CUDA graph replay" if args.graph else "direct launches",
+            "algorithmic_bytes_per_step": ab["total"],
+        },
+        "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
+                     "bytes_per_step": ab["total"]},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": (achieved / peak) if achieved else None, "peak_source": peak_kind,
+                     "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
+                     "traffic": ncu_traffic(w.spec.name, dom)},
+        "stage_ms": stages,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step(w) * args.steps,
+        "clocks": clocks,
+        "_w": w,
+    }
+
+
+# ------------------------------------------------------------------------------ oracle (CPU) arms
+
+def oracle_rows_per_sec(w, max_seconds: float, max_rows: int = 10 ** 9):
+    """Time the float64 oracle on whole (sequence, KV head) rows of the workload, in order."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+
+    sp = w.spec
+    G = sp.group
+    rows = [(b, g) for b in range(sp.batch) for g in range(sp.n_kv_heads)]
+    done, t0 = 0, time.perf_counter()
+    tokens = 0
+    with threadpool_limits(limits=1):
+        while done < max_rows:
+            b, g = rows[done % len(rows)]
+            o0, o1 = int(w.offsets[b]), int(w.offsets[b + 1])
+            keys = w.k[o0:o1, g].double().numpy()
+            vals = w.v[o0:o1, g].double().numpy()
+            if sp.n_layers > 0:
+                qi = w.q[b:b + 1].double().numpy()
+                ql = w.q_layers[:, b:b + 1].double().numpy()
+                kk = np.ascontiguousarray(keys[:, None, :])
+                vv = np.ascontiguousarray(vals[:, None, :])
+                oracle.shared_index_step(qi[:, g * G:(g + 1) * G], ql[:, :, g * G:(g + 1) * G], kk, vv,
+                                         [0, o1 - o0], sp.topk_shared, w.scale)
+            else:
+                oracle.decode_row(w.q[b, g * G:(g + 1) * G].double().numpy(), keys, vals, int(w.roles[g]), w.scale,
+                                  None if w.idom is None else w.idom[g].tolist(), int(w.n_fac_per_seq[b]),
+                                  sp.sink, sp.window)
+            done += 1
+            tokens += o1 - o0
+            if time.perf_counter() - t0 > max_seconds:
+                break
+    dt = time.perf_counter() - t0
+    return done, tokens, dt
+
+
+def cpu_baseline(w, seconds: float = 15.0) -> dict:
+    done, tokens, dt = oracle_rows_per_sec(w, seconds)
+    rows_total = w.spec.batch * w.spec.n_kv_heads
+    step_tokens = int(w.lengths.sum())
+    # tokens/s: the fraction of a step done, times the tokens a step scans, per second
+    value = (done / rows_total) * step_tokens / dt
+    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (sequence, KV head) rows ({rows_total} make one step), float64 numpy, "
+                      f"BLAS limited to 1 thread, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = make_workload(preset(args.workload))
+    rows_total = w.spec.batch * w.spec.n_kv_heads
+    # size one step's sample so that warm-up + timed steps end within about two minutes
+    _, _, dt1 = oracle_rows_per_sec(w, 1e9, max_rows=1)
+    per_step_rows = max(1, min(rows_total, int(100.0 / max(1, args.steps + args.warmup) / max(dt1, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_rows_per_sec(w, 1e9, max_rows=per_step_rows)
+    t = 0.0
+    for _ in range(args.steps):
+        _, _, dt = oracle_rows_per_sec(w, 1e9, max_rows=per_step_rows)
+        t += dt
+    ms_step = t / args.steps * 1e3
+    value = (per_step_rows / rows_total) * int(w.lengths.sum()) / (ms_step * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same inputs)",
+        "config": {"workload": w.spec.name, "batch": w.spec.batch, "seq_len": int(w.max_len)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step_rows} of {rows_total} (sequence, KV head) rows per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", type=int, default=1, help="replay each step from a CUDA graph (1) or launch (0)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, rank, world, local_rank)
+    w = res.pop("_w")
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            res["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -110,6 +110,7 @@ def make_kv(k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: in
     assert k.shape == v.shape and k.stride() == v.stride() and k.stride(2) == 1
     assert offsets.dtype == torch.int32 and offsets.is_cuda
     kv = KVCache()
+    kv._keep = (k, v, offsets, k_dom)  # the descriptor holds raw pointers: keep the tensors alive with it
     kv.k, kv.v, kv.offsets = k.data_ptr(), v.data_ptr(), offsets.data_ptr()
     kv.batch = offsets.numel() - 1
     kv.n_kv_heads = k.shape[1]
