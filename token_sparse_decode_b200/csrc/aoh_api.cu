@@ -77,10 +77,12 @@ struct FdGeom {
 
 FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
   FdGeom g{};
-  const int64_t target = int64_t(kSmCount) * 4;
+  // about two CTAs per SM; at least two pipeline stages per CTA; at most kFdMaxSplits splits a row
+  const int64_t target = int64_t(kSmCount) * 2;
   int64_t chunk = ceil_div(std::max<int64_t>(work_tokens, 1), target);
+  chunk = std::max<int64_t>(chunk, 2 * kFdTS);
+  chunk = std::max<int64_t>(chunk, ceil_div(std::max<int64_t>(n_max, 1), kFdMaxSplits));
   chunk = ceil_div(chunk, kFdTS) * kFdTS;
-  chunk = std::min<int64_t>(std::max<int64_t>(chunk, kFdTS), 8192);
   g.chunk = (int)chunk;
   g.max_splits = (int)std::max<int64_t>(1, ceil_div(std::max<int64_t>(n_max, 1), chunk));
   g.nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);

@@ -30,6 +30,8 @@ namespace aoh {
 constexpr int kFdThreads = 128;  // 4 warps
 constexpr int kFdTS = 64;        // tokens per pipeline stage
 constexpr int kFdStages = 3;
+constexpr int kFdPosCap = 1024;  // list positions staged in shared memory per CTA
+constexpr int kFdMaxSplits = 256; // splits per row (the combine stages their weights in shared memory)
 
 struct FdecParams {
   const uint16_t* q;         // row (layer l, b, h) at q + ((l * B + b) * Hq + h) * D
@@ -79,6 +81,7 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
   constexpr int CPR = D / 8;         // 16-byte chunks per row
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ int s_last;
+  __shared__ int s_pos[kFdPosCap];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.z;
@@ -126,6 +129,20 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
   const int ntok = min(n, j0 + p.chunk) - j0;
   const int nstages = (ntok + kFdTS - 1) / kFdTS;
 
+  // list mode: stage this CTA's positions once (one round trip instead of one per stage)
+  const bool pos_in_smem = p.list_mode && ntok <= kFdPosCap;
+  if (pos_in_smem) {
+    for (int j = tid; j < ntok; j += kFdThreads) {
+      int pos = __ldg(lst + j0 + j);
+      if (pos < 0 || pos >= L) {
+        record_error(kCheckPosition, b, g, pos);
+        pos = -1;
+      }
+      s_pos[j] = pos;
+    }
+    __syncthreads();
+  }
+
   const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
   const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
   const uint32_t sbase = smem_u32(smem);
@@ -142,7 +159,13 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
         int pos = 0;
         if (ok) {
           const int j = j0 + jj;
-          if (p.list_mode) {
+          if (pos_in_smem) {
+            pos = s_pos[jj];
+            if (pos < 0) {
+              ok = false;
+              pos = 0;
+            }
+          } else if (p.list_mode) {
             pos = __ldg(lst + j);
             if (pos < 0 || pos >= L) {
               if (ch == 0) record_error(kCheckPosition, b, g, pos);
@@ -237,8 +260,13 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
         acc[i2][2] *= al0;
         acc[i2][3] *= al1;
       }
-      const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
-      const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+      // P enters the PV product as hi + lo bf16 parts (p = hi + lo to ~2^-17), so the
+      // weights are not rounded to 8 bits: with few tokens that rounding alone reaches 2e-3.
+      const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+      const uint32_t l01 = pack_bf16x2(p0 - bf16lo(h01), p1 - bf16hi(h01));
+      const uint32_t l23 = pack_bf16x2(p2 - bf16lo(h23), p3 - bf16hi(h23));
+      const uint32_t pb0 = movmatrix_trans(h01), pb1 = movmatrix_trans(h23);
+      const uint32_t pl0 = movmatrix_trans(l01), pl1 = movmatrix_trans(l23);
       {
         const int r = u * 16 + (lane & 7) + (lane >> 4) * 8;
         const int dsel = ((lane >> 3) & 1) * 8;
@@ -247,6 +275,7 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
           uint32_t a[4];
           ldsm_x4_trans(a, vt + fd_tile_off(r, mt * 16 + dsel));
           mma_16816(acc[mt], a, pb0, pb1);
+          mma_16816(acc[mt], a, pl0, pl1);
         }
       }
     }
@@ -327,18 +356,40 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
   __threadfence();
   const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
   const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
+  // weights w[s][q] = 2^(m_sq - M_q) staged in shared memory (nsplit * NQP <= kFdMaxSplits * NQP fits)
+  float* sw = reinterpret_cast<float*>(smem);        // [nsplit][NQP]
+  float* sM = sw + nsplit * NQP;                     // [NQP]
+  float* sL = sM + NQP;                              // [NQP]
+  if (tid < NQP) {
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2));
+    sM[tid] = M;
+  }
+  __syncthreads();
+  for (int e = tid; e < nsplit * NQP; e += kFdThreads) {
+    const int qr = e % NQP;
+    sw[e] = exp2f(__ldcg(rml + (int64_t)e * 2) - sM[qr]);
+  }
+  __syncthreads();
+  if (tid < NQP) {
+    float Ls = 0.f;
+    for (int s2 = 0; s2 < nsplit; ++s2) Ls += sw[s2 * NQP + tid] * __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2 + 1);
+    sL[tid] = Ls;
+  }
+  __syncthreads();
   for (int e = tid; e < p.NQ * D; e += kFdThreads) {
     const int qr = e / D, dd = e % D;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldcg(rml + ((int64_t)s * NQP + qr) * 2));
-    float Ls = 0.f, A = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-      const float f = exp2f(__ldcg(rml + ((int64_t)s * NQP + qr) * 2) - M);
-      Ls += f * __ldcg(rml + ((int64_t)s * NQP + qr) * 2 + 1);
-      A += f * __ldcg(racc + ((int64_t)s * NQP + qr) * D + dd);
+    float A0 = 0.f, A1 = 0.f, A2 = 0.f, A3 = 0.f;
+    int s2 = 0;
+    for (; s2 + 4 <= nsplit; s2 += 4) {
+      A0 += sw[(s2 + 0) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 0) * NQP + qr) * D + dd);
+      A1 += sw[(s2 + 1) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 1) * NQP + qr) * D + dd);
+      A2 += sw[(s2 + 2) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 2) * NQP + qr) * D + dd);
+      A3 += sw[(s2 + 3) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 3) * NQP + qr) * D + dd);
     }
+    for (; s2 < nsplit; ++s2) A0 += sw[s2 * NQP + qr] * __ldcg(racc + ((int64_t)s2 * NQP + qr) * D + dd);
     const int l = qr / p.G, h = g * p.G + qr % p.G;
-    p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Ls;
+    p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = ((A0 + A1) + (A2 + A3)) / sL[qr];
   }
   if (tid == 0) p.tickets[row_id] = 0;
 }

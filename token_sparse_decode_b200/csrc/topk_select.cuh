@@ -94,9 +94,17 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
     int* h = hist[pass & 1];
     if (tid < 256) h[tid] = 0;
     __syncthreads();
-    for (int i = lo + tid; i < hi; i += kSelThreads) {
-      const uint32_t k = key_at(i);
-      if ((k & pmask) == prefix) atomicAdd(&h[(k >> shift) & 255u], 1);
+    // Warp-aggregated counting: keys of one row share few leading digits (the top
+    // digit is sign + exponent), so lanes with the same bin add once per warp.
+    for (int base = lo + (tid & ~31); base < hi; base += kSelThreads) {
+      const int i = base + (tid & 31);
+      int bin = -1;
+      if (i < hi) {
+        const uint32_t k = key_at(i);
+        if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
     }
     cluster.sync();
     // cluster-wide total of the bin that this thread scans, bins taken from the top down
