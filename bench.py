@@ -177,67 +177,60 @@ def build_step(w, dev):
     return step, (w.q.to(dev),)
 
 
+KERNEL_OF_CALL = {"sparse_decode": "sparse_row_kernel", "shared_index_step": "sparse_row_kernel",
+                  "stream_decode": "flash_gather_kernel"}
+FUSED_MAX_LEN = 16 * 16384  # rows up to this length run as one cluster kernel (library rule)
+
+
 def launches_per_step(w) -> int:
     if w.spec.n_layers > 0:
-        return 3  # indexer scan, top-k, shared-index gather
+        return 1  # fused shared-index step
     roles = w.roles.numpy()
     n = 0
     if (roles == ROLE_SPARSE).any():
-        n += 3    # importance scan, top-k, focused attention
+        n += 1 if w.max_len <= FUSED_MAX_LEN else 3  # fused row kernel, or scan + select + attend
     if (roles != ROLE_SPARSE).any():
         n += 1    # window attention
     return n
 
 
 def stage_timing(w, step, q, steps: int, flush) -> dict:
-    """Per-kernel device time (CUDA events on the launching stream), same inputs, L2 flushed."""
+    """Device time of each public call of the step (CUDA events on the launching stream).
+
+    Each sample runs behind a short device-side sleep so that the host has queued
+    the calls before the first one starts: the events then time the kernels, not the
+    host's launch latency.  L2 is flushed before every sample.
+    """
     from token_sparse_decode_b200 import binding as B
 
     st = torch.cuda.current_stream()
-    res = {}
+    calls = []
     if w.spec.n_layers > 0:
-        names = ["indexer_scan", "topk_select", "shared_gather"]
-        fns = [lambda: B.tip_score(q[0], step.kv, step.all_chunks, step.all_chunks.shape[1], step.scores),
-               lambda: B.topk_select(step.scores, step.kv, step.topk, None, step.topk, step.idx, step.count),
-               lambda: B.shared_index_decode(q[1], step.kv, step.idx, step.count, step.topk, step.scale, step.out,
-                                             step.ws)]
+        calls.append(("shared_index_step", lambda: step(*q)))
     else:
-        if step.ws_sparse is None:
-            return res
-        scores = torch.empty((w.spec.n_kv_heads, max(1, w.total_tokens)), dtype=torch.float32, device=q[0].device)
-        ws1 = torch.zeros_like(step.ws_sparse)
-        kvq = q[0][None]
-        ws2 = None
-        from token_sparse_decode_b200.binding import shared_index_decode_workspace_size, workspace
-
-        ws2 = workspace(shared_index_decode_workspace_size(step.kv, 1, w.spec.n_q_heads, step.n_fac_cap),
-                        q[0].device)
-        out2 = torch.empty((1,) + tuple(step.out.shape), dtype=torch.float32, device=q[0].device)
-        names = ["tip_score", "topk_select", "focused_attention"]
-        fns = [lambda: B.tip_score(q[0], step.kv, step.idom, step.n_dom, scores),
-               lambda: B.topk_select(scores, step.kv, step.n_fac, step.n_fac_per_seq, step.n_fac_cap, step.idx,
-                                     step.count),
-               lambda: B.shared_index_decode(kvq, step.kv, step.idx, step.count, step.n_fac_cap, step.scale, out2,
-                                             ws2)]
-        del ws1
-    for fn in fns:  # warm
+        if step.has_sparse:
+            calls.append(("sparse_decode", lambda: B.sparse_decode(
+                q[0], step.kv, step.idom, step.n_dom, step.n_fac, step.n_fac_per_seq, step.n_fac_cap, step.roles,
+                step.scale, step.out, step.ws_sparse, step.idx, step.count)))
+        if step.has_stream:
+            calls.append(("stream_decode", lambda: B.stream_decode(
+                q[0], step.kv, step.roles, step.sink, step.window, step.scale, step.out, step.ws_stream)))
+    for _, fn in calls:
         fn()
     torch.cuda.synchronize()
-    times = {n: [] for n in names}
+    times = {n: [] for n, _ in calls}
     for _ in range(steps):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+        flush()
+        torch.cuda._sleep(200000)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
         evs[0].record(st)
-        for i, fn in enumerate(fns):
+        for i, (_, fn) in enumerate(calls):
             fn()
             evs[i + 1].record(st)
         torch.cuda.synchronize()
-        for i, n in enumerate(names):
+        for i, (n, _) in enumerate(calls):
             times[n].append(evs[i].elapsed_time(evs[i + 1]))
-        flush()
-    torch.cuda.synchronize()
-    for n in names:
-        res[n] = float(np.mean(times[n]))
-    return res
+    return {n: float(np.mean(t)) for n, t in times.items()}
 
 
 def capture_graph(fn):
@@ -348,12 +341,10 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = tokens_step * world / (e2e_ms / args.steps * 1e-3)
     ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_gbs()
-    if w.spec.n_layers > 0:
-        dom, dom_bytes = "indexer_scan", ab["indexer"]
-    else:
-        dom, dom_bytes = "tip_score", ab["tip"]
-        if stages and stages.get("focused_attention", 0) > stages.get("tip_score", 0):
-            dom, dom_bytes = "focused_attention", ab["fac"]
+    call_bytes = {"shared_index_step": ab["indexer"] + ab["gather"], "sparse_decode": ab["tip"] + ab["fac"],
+                  "stream_decode": ab["window"]}
+    dom = max(stages, key=lambda k: stages[k]) if stages else None
+    dom_bytes = call_bytes.get(dom, 0)
     dom_ms = stages.get(dom)
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms else None
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
@@ -381,7 +372,7 @@ def run_ours(args, rank, world, local_rank):
         },
         "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
                      "bytes_per_step": ab["total"]},
-        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        "roofline": {"kernel": KERNEL_OF_CALL.get(dom, dom), "call": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "peak_source": peak_kind,
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
                      "traffic": ncu_traffic(w.spec.name, dom)},

@@ -243,6 +243,26 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
 size_t aoh_shared_index_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_layers,
                                               int32_t n_q_heads, int32_t n_fac_cap);
 
+/*
+ * aoh_shared_index_step -- the whole shared-index stack step in one launch
+ * ("Como funciona CLSA": the indexer scores the cache once, takes one top-k
+ * and every cross-decoder layer attends over it).  Equivalent to
+ * aoh_tip_score (every chunk, q_index) + aoh_topk_select (k = topk) +
+ * aoh_shared_index_decode, without the score buffer or workspace: each
+ * (sequence, KV head) row runs in one thread-block cluster.
+ *   q_index    device bf16 [B][n_q_heads][d]: the indexer layer's queries
+ *   q_layers   device bf16 [n_layers][B][n_q_heads][d]
+ *   n_layers * (n_q_heads / n_kv_heads) <= 32
+ *   idx, count device outputs, layouts of aoh_topk_select with n_fac_cap = topk
+ *   out        device fp32 [n_layers][B][n_q_heads][d]
+ * Returns AOH_ERR_UNSUPPORTED when a row is too long for one cluster
+ * (max_len above 262144); the three-call form has no such limit.
+ */
+aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int32_t n_layers,
+                                 int32_t n_q_heads, const aoh_kv_cache* kv, int32_t topk,
+                                 int32_t* idx, int32_t* count, float scale, float* out,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif

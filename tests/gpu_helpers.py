@@ -123,10 +123,10 @@ def run_sparse(d: Dev, pack=True):
     return step, out
 
 
-def run_shared(d: Dev):
+def run_shared(d: Dev, fused: bool = True):
     w = d.w
     step = SharedIndexStep(d.k, d.v, d.offsets, d.max_len, d.T, w.spec.n_layers, w.spec.n_q_heads,
-                           w.spec.topk_shared, w.scale)
+                           w.spec.topk_shared, w.scale, fused=fused)
     out = step(d.q, d.q_layers)
     torch.cuda.synchronize()
     check_device()

@@ -221,13 +221,14 @@ def test_full_role_split_step_mixed_heads():
 
 # ------------------------------------------------------------------------------ shared index
 
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("n_layers,hq,hkv", [(8, 32, 8), (2, 16, 4), (3, 16, 4), (1, 8, 8)])
-def test_shared_index_decode_matches_oracle(n_layers, hq, hkv):
+def test_shared_index_decode_matches_oracle(n_layers, hq, hkv, fused):
     sp = WorkloadSpec(name="shared", batch=2, n_q_heads=hq, n_kv_heads=hkv, head_dim=128, theta=5e5,
                       len_range=(500, 9000), n_layers=n_layers, topk_shared=700, seed=90 + n_layers)
     w = make_workload(sp)
     d = Dev(w)
-    step, out = run_shared(d)
+    step, out = run_shared(d, fused=fused)
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
     G = sp.group
@@ -286,3 +287,29 @@ def test_edge_cases_empty_and_short_sequences():
             else:
                 compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G])
             assert np.all(idx_h[b, g, n:] == -1)
+
+
+def test_sparse_decode_long_row_uses_three_kernels():
+    # a row longer than one cluster handles (262144 positions) takes the scan / select / attend path
+    sp = WorkloadSpec(name="long", batch=1, n_q_heads=2, n_kv_heads=1, head_dim=64, theta=1e4, lengths=(300001,),
+                      n_dom=6, n_fac=3000, roles=(ROLE_SPARSE,), planted_frac=0.001, seed=85)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_sparse(d)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    compare_sparse_row(w, 0, 0, idx_h[0, 0, :cnt_h[0, 0]], out_h[0, 0:2])
+
+
+def test_sparse_decode_every_token_selected():
+    # N_fac >= L on every sequence: focused attention is dense attention
+    sp = spec(batch=2, len_range=(50, 900), n_fac_div=0, n_fac=1000, seed=86)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_sparse(d)
+    out_h = f64(out)
+    G = sp.group
+    for b in range(2):
+        for g in range(sp.n_kv_heads):
+            assert step.count[b, g].item() == w.lengths[b]
+            compare_window_row(w, b, g, out_h[b, g * G:(g + 1) * G], ROLE_DENSE, 0, 0)

@@ -25,6 +25,7 @@ EXPORTS = (
     "aoh_status_string", "aoh_version", "aoh_last_cuda_error", "aoh_device_check", "aoh_pack_dominant", "aoh_tip_score",
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
+    "aoh_shared_index_step",
 )
 
 
@@ -73,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "aoh_stream_decode_workspace_size": (SZ, [KVP, I32, P, I32, I32]),
             "aoh_shared_index_decode": (ctypes.c_int, [P, I32, I32, KVP, P, P, I32, F32, P, P, SZ, P]),
             "aoh_shared_index_decode_workspace_size": (SZ, [KVP, I32, I32, I32]),
+            "aoh_shared_index_step": (ctypes.c_int, [P, P, I32, I32, KVP, I32, P, P, F32, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -202,3 +204,10 @@ def shared_index_decode(q_layers: torch.Tensor, kv: KVCache, idx: torch.Tensor, 
     _check("aoh_shared_index_decode", lib().aoh_shared_index_decode(
         _ptr(q_layers), q_layers.shape[0], q_layers.shape[-2], ctypes.byref(kv), _ptr(idx), _ptr(count),
         n_fac_cap, float(scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def shared_index_step(q_index: torch.Tensor, q_layers: torch.Tensor, kv: KVCache, topk: int, idx: torch.Tensor,
+                      count: torch.Tensor, scale: float, out: torch.Tensor, stream=None) -> None:
+    _check("aoh_shared_index_step", lib().aoh_shared_index_step(
+        _ptr(q_index), _ptr(q_layers), q_layers.shape[0], q_layers.shape[-2], ctypes.byref(kv), topk, _ptr(idx),
+        _ptr(count), float(scale), _ptr(out), _stream(stream)))

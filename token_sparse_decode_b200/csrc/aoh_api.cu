@@ -11,6 +11,7 @@
 #include "aoh.h"
 #include "device_common.cuh"
 #include "flash_gather.cuh"
+#include "sparse_row.cuh"
 #include "tip_score.cuh"
 #include "topk_select.cuh"
 
@@ -218,6 +219,92 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
   return cuda_status(cudaLaunchKernelEx(&cfg, topk_select_kernel, sp));
 }
 
+
+// ------------------------------------------------------------------ fused row kernel
+struct FusedPlan {
+  bool ok;
+  int CL;
+  int slice_max;
+  size_t keys_bytes, smem;
+};
+
+FusedPlan fused_plan(const aoh_kv_cache* kv, int n_rows, int nq) {
+  FusedPlan f{};
+  if (nq > kMaxQRows) return f;
+  const int64_t L = std::max(kv->max_len, 1);
+  f.CL = 8;
+  if (int64_t(n_rows) * 8 < kSmCount || ceil_div(L, 8) > int64_t(kSrThreads) * kSrMaxRun) f.CL = 16;
+  const int64_t slice = (ceil_div(L, f.CL) + 3) & ~int64_t(3);
+  if (slice > int64_t(kSrThreads) * kSrMaxRun) return f;  // row too long for one cluster
+  f.slice_max = (int)slice;
+  f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
+  const size_t stage = size_t(kSrStages) * 2 * kSrTS * kv->head_dim * 2;
+  f.smem = f.keys_bytes + stage;
+  f.ok = f.smem <= 200 * 1024;
+  return f;
+}
+
+template <int D, int NT>
+aoh_status launch_rows_t(const RowParams& rp, const FusedPlan& f, int n_listed, int B, cudaStream_t st) {
+  static size_t configured = 0;
+  if (f.smem > configured) {
+    aoh_status s = set_smem(sparse_row_kernel<D, NT>, 200 * 1024);
+    if (s != AOH_OK) return s;
+    s = cuda_status(cudaFuncSetAttribute(sparse_row_kernel<D, NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    if (s != AOH_OK) return s;
+    configured = 200 * 1024;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(f.CL, n_listed, B);
+  cfg.blockDim = dim3(kSrThreads);
+  cfg.dynamicSmemBytes = f.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = f.CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_row_kernel<D, NT>, rp));
+}
+
+aoh_status launch_rows(const RowParams& rp, const FusedPlan& f, int d, int nq, int n_listed, int B,
+                       cudaStream_t st) {
+  const int nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
+  if (d == 128) {
+    if (nqp == 8) return launch_rows_t<128, 1>(rp, f, n_listed, B, st);
+    if (nqp == 16) return launch_rows_t<128, 2>(rp, f, n_listed, B, st);
+    return launch_rows_t<128, 4>(rp, f, n_listed, B, st);
+  }
+  if (nqp == 8) return launch_rows_t<64, 1>(rp, f, n_listed, B, st);
+  if (nqp == 16) return launch_rows_t<64, 2>(rp, f, n_listed, B, st);
+  return launch_rows_t<64, 4>(rp, f, n_listed, B, st);
+}
+
+// Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,
+// or (idom == nullptr) K in place with every chunk.
+void rows_score_source(RowParams& rp, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom) {
+  rp.idom = idom;
+  rp.n_dom = n_dom;
+  if (kv->k_dom && idom) {
+    rp.score_src = static_cast<const uint16_t*>(kv->k_dom);
+    rp.srow_stride_tok = kv->k_dom_cols;
+    rp.srow_stride_head = kv->total_tokens * kv->k_dom_cols;
+    rp.srow_len = kv->k_dom_cols;
+    rp.packed = 1;
+  } else {
+    rp.score_src = static_cast<const uint16_t*>(kv->k);
+    rp.srow_stride_tok = kv->stride_tok;
+    rp.srow_stride_head = kv->stride_head;
+    rp.srow_len = kv->head_dim;
+    rp.packed = 0;
+  }
+  int segs = 1;
+  while (segs * 8 < rp.srow_len) segs <<= 1;
+  rp.segs = segs;
+}
+
 int list_heads(const aoh_kv_cache* kv, const uint8_t* roles, bool want_sparse, uint8_t* out) {
   int n = 0;
   for (int g = 0; g < kv->n_kv_heads; ++g) {
@@ -404,6 +491,36 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + off_idx);
   int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + off_count);
 
+  const FusedPlan plan = fused_plan(kv, kv->batch * n_listed, G);
+  if (plan.ok) {
+    RowParams rp{};
+    rp.q_score = static_cast<const uint16_t*>(q);
+    rp.q_attn = static_cast<const uint16_t*>(q);
+    rp.k = static_cast<const uint16_t*>(kv->k);
+    rp.v = static_cast<const uint16_t*>(kv->v);
+    rp.offsets = kv->offsets;
+    rows_score_source(rp, kv, idom, n_dom);
+    rp.n_fac_per_seq = n_fac_per_seq;
+    rp.n_fac = n_fac;
+    rp.cap = n_fac_cap;
+    rp.idx_out = idx;
+    rp.count_out = cnt;
+    rp.out = out;
+    rp.stride_tok = kv->stride_tok;
+    rp.stride_head = kv->stride_head;
+    rp.T = (int32_t)kv->total_tokens;
+    rp.B = kv->batch;
+    rp.Hq = n_q_heads;
+    rp.Hkv = kv->n_kv_heads;
+    rp.G = G;
+    rp.NQ = G;
+    rp.keys_bytes = (int32_t)plan.keys_bytes;
+    rp.scale_log2 = scale * 1.4426950408889634f;
+    memcpy(rp.heads, heads, n_listed);
+    return launch_rows(rp, plan, kv->head_dim, G, n_listed, kv->batch, st);
+  }
+
+  // rows too long for one cluster: scan, select and attend as three kernels
   if (kv->total_tokens > 0) {
     if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st)) != AOH_OK) return s;
   }
@@ -530,6 +647,49 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
   memcpy(fp.heads, heads, n_listed);
   fd_bind(fp, geo, static_cast<uint8_t*>(workspace));
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream));
+}
+
+aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int32_t n_layers, int32_t n_q_heads,
+                                 const aoh_kv_cache* kv, int32_t topk, int32_t* idx, int32_t* count, float scale,
+                                 float* out, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if (n_layers < 1 || topk < 1 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  const int G = n_q_heads / kv->n_kv_heads;
+  if (int64_t(n_layers) * G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (kv->batch == 0) return AOH_OK;
+  if (!q_index || !q_layers || !idx || !count || !out) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(q_index) || !aligned16(q_layers)) return AOH_ERR_ALIGNMENT;
+  uint8_t heads[kMaxHeads];
+  const int n_listed = list_heads(kv, nullptr, true, heads);
+  const FusedPlan plan = fused_plan(kv, kv->batch * n_listed, n_layers * G);
+  if (!plan.ok) return AOH_ERR_UNSUPPORTED;
+  RowParams rp{};
+  rp.q_score = static_cast<const uint16_t*>(q_index);
+  rp.q_attn = static_cast<const uint16_t*>(q_layers);
+  rp.k = static_cast<const uint16_t*>(kv->k);
+  rp.v = static_cast<const uint16_t*>(kv->v);
+  rp.offsets = kv->offsets;
+  rows_score_source(rp, kv, nullptr, kv->head_dim / 2);
+  rp.n_fac_per_seq = nullptr;
+  rp.n_fac = topk;
+  rp.cap = topk;
+  rp.idx_out = idx;
+  rp.count_out = count;
+  rp.out = out;
+  rp.stride_tok = kv->stride_tok;
+  rp.stride_head = kv->stride_head;
+  rp.T = (int32_t)kv->total_tokens;
+  rp.B = kv->batch;
+  rp.Hq = n_q_heads;
+  rp.Hkv = kv->n_kv_heads;
+  rp.G = G;
+  rp.NQ = n_layers * G;
+  rp.keys_bytes = (int32_t)plan.keys_bytes;
+  rp.scale_log2 = scale * 1.4426950408889634f;
+  memcpy(rp.heads, heads, n_listed);
+  return launch_rows(rp, plan, kv->head_dim, n_layers * G, n_listed, kv->batch, as_stream(stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,543 @@
+// Fused decode step of one SPARSE (sequence, KV head) row in one thread-block
+// cluster: importance scan -> top-N_fac -> focused attention -> combine.
+//
+// FASA: Frequency-aware Sparse Attention, §2.B.1 (importance from the dominant
+// chunks, keep the N_fac best) and §2.B.2 (full-dimension attention over the
+// kept tokens at their original positions); the shared-index stack of "Cómo
+// funciona CLSA" is the same row with every chunk scored and NQ = n_layers * G.
+//
+// The row's L positions are cut into CL contiguous slices, one per CTA.
+//  1. scan:    each CTA streams the score rows of its slice (packed dominant
+//              columns, or K in place) with 16-byte loads, keeps the fp32 scores
+//              as order-preserving uint32 keys in shared memory and counts the
+//              first radix digit on the fly;
+//  2. select:  4-digit MSB radix select of the n-th largest key over the cluster
+//              (histograms summed through distributed shared memory, one cluster
+//              barrier per digit); ties broken toward lower positions by an ordered
+//              compaction that also writes the index (ascending) to global memory;
+//  3. attend:  every CTA gathers the K / V rows of the positions it selected from
+//              its own slice (cp.async into 128B-swizzled tiles) and runs the
+//              online-softmax contraction on tensor cores (tokens on M, query rows
+//              on N, P as hi + lo bf16 parts), 8 warps = 4 token/row groups x 2
+//              halves of the head dimension for the PV product;
+//  4. combine: the CL partial (m, l, acc) states are merged through distributed
+//              shared memory, each CTA writing 1/CL of the outputs.
+// Nothing but the index and the outputs goes to global memory; no global
+// scratch, no second launch.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "device_common.cuh"
+
+namespace aoh {
+
+namespace cgs = cooperative_groups;
+
+constexpr int kSrThreads = 256;  // 8 warps
+constexpr int kSrTS = 32;        // tokens per attention stage
+constexpr int kSrStages = 4;
+constexpr int kSrMaxRun = 64;    // keys per thread in the compaction: slice <= 256 * 64
+
+struct RowParams {
+  const uint16_t* q_score;   // [B][Hq][D]: the query that scores (group-summed)
+  const uint16_t* q_attn;    // [n_layers][B][Hq][D]: query rows of the attention
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* offsets;    // [B + 1]
+  const uint16_t* score_src; // packed k_dom or K
+  int64_t srow_stride_tok, srow_stride_head;
+  int32_t srow_len;          // elements per score row (k_dom cols, or D in place)
+  int32_t packed;            // 1: k_dom rows; 0: K rows with q masked to the dominant dims
+  int32_t segs;              // lanes per score row: srow_len / 8 rounded up to a power of two
+  const int32_t* idom;       // [Hkv][n_dom]; null = every chunk
+  int32_t n_dom;
+  const int32_t* n_fac_per_seq;
+  int32_t n_fac, cap;
+  int32_t* idx_out;          // [B][Hkv][cap]
+  int32_t* count_out;        // [B][Hkv]
+  float* out;                // [n_layers][B][Hq][D]
+  int64_t stride_tok, stride_head;
+  int32_t T, B, Hq, Hkv, G, NQ;
+  int32_t keys_bytes;        // dynamic shared memory before the attention stages
+  float scale_log2;
+  uint8_t heads[kMaxHeads];
+};
+
+// Byte offset of (row r, dim dd) in a [kSrTS x D] tile: D/64 halves of [kSrTS x 128 B],
+// 16-byte chunks XOR-swizzled by (r mod 8).
+__device__ __forceinline__ uint32_t sr_tile_off(int r, int dd) {
+  const int half = dd >> 6;
+  const int cc = (dd & 63) >> 3;
+  return (uint32_t)(half * (kSrTS * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint4 sr_ld_stream(const uint16_t* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float sr_dot8(const uint4& w, const float (&qs)[8]) {
+  float s = bf16lo(w.x) * qs[0];
+  s = fmaf(bf16hi(w.x), qs[1], s);
+  s = fmaf(bf16lo(w.y), qs[2], s);
+  s = fmaf(bf16hi(w.y), qs[3], s);
+  s = fmaf(bf16lo(w.z), qs[4], s);
+  s = fmaf(bf16hi(w.z), qs[5], s);
+  s = fmaf(bf16lo(w.w), qs[6], s);
+  s = fmaf(bf16hi(w.w), qs[7], s);
+  return s;
+}
+
+// Warp-aggregated histogram increment (bin < 0: lane does not count).
+__device__ __forceinline__ void hist_add(int* h, int bin) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams p) {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
+  constexpr int KS = D / 16;          // k-steps of QK
+  constexpr int KH = KS / 2;          // PV m-tiles per half of the head dimension
+  constexpr int WT = 4 / NT;          // token groups per (n-tile, half)
+  constexpr int SUB = kSrTS / 16;     // 16-token sub-tiles per stage
+  constexpr int NQP = NT * 8;
+  constexpr int CPR = D / 8;          // 16-byte chunks per K / V row
+  constexpr int TILE = kSrTS * D * 2;
+  constexpr int STAGE = 2 * TILE;
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ int hist[2][256];
+  __shared__ int scan_scratch[33];
+  __shared__ float qt[128];
+  __shared__ int s_bin, s_above, s_eq_before, s_sel_before;
+  __shared__ int s_cnt[2];
+
+  cgs::cluster_group cluster = cgs::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rk = (int)cluster.block_rank();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.z;
+  const int g = p.heads[blockIdx.y];
+  const int off = p.offsets[b];
+  const int L = p.offsets[b + 1] - off;
+  int nf = p.n_fac_per_seq ? p.n_fac_per_seq[b] : p.n_fac;
+  if (nf > p.cap) {
+    if (rk == 0 && tid == 0) record_error(kCheckCount, b, nf, p.cap);
+    nf = p.cap;
+  }
+  const int n = max(0, min(nf, L));
+  int32_t* idx_row = p.idx_out + ((int64_t)b * p.Hkv + g) * p.cap;
+  for (int j = n + rk * kSrThreads + tid; j < p.cap; j += CL * kSrThreads) idx_row[j] = -1;
+  if (rk == 0 && tid == 0) p.count_out[(int64_t)b * p.Hkv + g] = n;
+  if (n == 0) {  // uniform over the cluster: zero rows, no barrier taken
+    if (rk == 0) {
+      for (int e = tid; e < p.NQ * D; e += kSrThreads) {
+        const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
+        p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + e % D] = 0.f;
+      }
+    }
+    return;
+  }
+
+  const int slice = (((L + CL - 1) / CL) + 3) & ~3;
+  const int lo = min(L, rk * slice), hi = min(L, lo + slice);
+  const int m = hi - lo;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
+  int* plist = reinterpret_cast<int*>(smem);  // selected positions replace the keys
+  int nloc;
+
+  if (n < L) {
+    // =============================================================== 1. scan
+    hist[0][tid] = 0;  // kSrThreads == 256 bins
+    if (tid < p.srow_len) {
+      const int C = D / 2;
+      int dim = -1;
+      if (p.packed) {
+        if (tid < 2 * p.n_dom) {
+          const int j = tid < p.n_dom ? tid : tid - p.n_dom;
+          const int c = p.idom[g * p.n_dom + j];
+          if (c < 0 || c >= C) {
+            record_error(kCheckChunk, g, j, c);
+          } else {
+            dim = tid < p.n_dom ? c : c + C;
+          }
+        }
+      } else if (p.idom == nullptr) {
+        dim = tid;  // every chunk: the full dot
+      } else {
+        const int c = tid < C ? tid : tid - C;
+        for (int j = 0; j < p.n_dom; ++j) {
+          const int cj = p.idom[g * p.n_dom + j];
+          if (cj < 0 || cj >= C) record_error(kCheckChunk, g, j, cj);
+          if (cj == c) dim = tid;
+        }
+      }
+      float acc = 0.f;
+      if (dim >= 0) {
+        const uint16_t* qb = p.q_score + ((int64_t)b * p.Hq + (int64_t)g * p.G) * D + dim;
+        for (int h = 0; h < p.G; ++h) acc += __uint_as_float((uint32_t)qb[(int64_t)h * D] << 16);
+      }
+      qt[tid] = acc;
+    }
+    __syncthreads();
+    {
+      const int segs = p.segs;
+      const int seg = lane & (segs - 1);
+      float qs[8];
+      bool active = false;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        qs[i] = (seg * 8 + i < p.srow_len) ? qt[seg * 8 + i] : 0.f;
+        active |= (qs[i] != 0.f);
+      }
+      const int rpw = 32 / segs;               // rows per warp per load
+      const int rpi = kSrThreads / segs;       // rows per block per load
+      constexpr int U = 8;                     // loads in flight per thread
+      const uint16_t* base = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)off * p.srow_stride_tok + seg * 8;
+      const int lrow = lane / segs;
+      for (int tb = lo + warp * rpw; tb < hi; tb += U * rpi) {  // warp-uniform bounds
+        uint4 w[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int tt = tb + u * rpi + lrow;
+          w[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (tt < hi && active) w[u] = sr_ld_stream(base + (int64_t)tt * p.srow_stride_tok);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          float s = sr_dot8(w[u], qs);
+          for (int o = segs >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          const int tt = tb + u * rpi + lrow;
+          int bin = -1;
+          if (seg == 0 && tt < hi) {
+            const uint32_t key = score_key(s);
+            keys[tt - lo] = key;
+            bin = (int)(key >> 24);
+          }
+          hist_add(hist[0], bin);
+        }
+      }
+    }
+
+    // =============================================================== 2. select
+    uint32_t prefix = 0u, pmask = 0u;
+    int krem = n;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      int* h = hist[pass & 1];
+      if (pass > 0) {
+        h[tid] = 0;
+        __syncthreads();
+        for (int bs = lo + (tid & ~31); bs < hi; bs += kSrThreads) {
+          const int i = bs + lane;
+          int bin = -1;
+          if (i < hi) {
+            const uint32_t k = keys[i - lo];
+            if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
+          }
+          hist_add(h, bin);
+        }
+      }
+      cluster.sync();
+      int tot = 0;
+      {
+        const int bin = 255 - tid;  // scanned from the top bin down
+        for (int q = 0; q < CL; ++q) tot += cluster.map_shared_rank(h, q)[bin];
+      }
+      int total;
+      const int above = block_exclusive_scan(tot, scan_scratch, &total);
+      if (above < krem && krem <= above + tot) {
+        s_bin = 255 - tid;
+        s_above = above;
+      }
+      __syncthreads();
+      prefix |= (uint32_t)s_bin << shift;
+      pmask |= 255u << shift;
+      krem -= s_above;
+      __syncthreads();
+    }
+    const uint32_t KT = prefix;
+    const int need_eq = krem;
+
+    // ---- ordered compaction: positions in ascending order, lower position first among equals
+    const int run = (m + kSrThreads - 1) / kSrThreads;  // <= kSrMaxRun (host guarantees)
+    const int a0 = min(m, tid * run), a1 = min(m, (tid + 1) * run);
+    int n_eq = 0, n_gt = 0;
+    for (int i = a0; i < a1; ++i) {
+      const uint32_t k = keys[i];
+      n_gt += k > KT;
+      n_eq += k == KT;
+    }
+    int eq_cta, gt_cta;
+    const int eq_excl = block_exclusive_scan(n_eq, scan_scratch, &eq_cta);
+    block_exclusive_scan(n_gt, scan_scratch, &gt_cta);
+    if (tid == 0) {
+      s_cnt[0] = eq_cta;
+      s_cnt[1] = gt_cta;
+    }
+    cluster.sync();
+    if (tid == 0) {
+      int eq_before = 0, sel_before = 0;
+      for (int q = 0; q < rk; ++q) {
+        const int* c = cluster.map_shared_rank(s_cnt, q);
+        sel_before += c[1] + max(0, min(need_eq - eq_before, c[0]));
+        eq_before += c[0];
+      }
+      s_eq_before = eq_before;
+      s_sel_before = sel_before;
+    }
+    __syncthreads();
+    uint64_t take = 0ull;
+    int n_sel = 0;
+    {
+      const int eq_base = s_eq_before + eq_excl;
+      int seen = 0;
+      for (int i = a0; i < a1; ++i) {
+        const uint32_t k = keys[i];
+        bool t = false;
+        if (k > KT) {
+          t = true;
+        } else if (k == KT) {
+          t = (eq_base + seen < need_eq);
+          ++seen;
+        }
+        if (t) {
+          take |= 1ull << (i - a0);
+          ++n_sel;
+        }
+      }
+    }
+    int sel_cta;
+    const int my = block_exclusive_scan(n_sel, scan_scratch, &sel_cta);  // ends with a barrier
+    {
+      int o = my;
+      const int gbase = s_sel_before;
+      while (take) {
+        const int bit = __ffsll((long long)take) - 1;
+        take &= take - 1;
+        const int pos = lo + a0 + bit;
+        plist[o] = pos;
+        if (gbase + o < n) idx_row[gbase + o] = pos;
+        ++o;
+      }
+    }
+    nloc = sel_cta;
+  } else {
+    // N_fac >= L: every position of the slice, in order
+    for (int i = tid; i < m; i += kSrThreads) {
+      plist[i] = lo + i;
+      idx_row[lo + i] = lo + i;
+    }
+    nloc = m;
+  }
+  __syncthreads();
+
+  // =============================================================== 3. attend
+  const int half = warp >> 2, r4 = warp & 3;
+  const int nt = r4 % NT, tg = r4 / NT;
+  uint32_t bq[KS][2];
+  {
+    const int qr = nt * 8 + (lane >> 2);
+    if (qr < p.NQ) {
+      const int l = qr / p.G, h = g * p.G + qr % p.G;
+      const uint16_t* qp = p.q_attn + (((int64_t)l * p.B + b) * p.Hq + h) * D + 2 * (lane & 3);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        bq[ks][0] = *reinterpret_cast<const uint32_t*>(qp + ks * 16);
+        bq[ks][1] = *reinterpret_cast<const uint32_t*>(qp + ks * 16 + 8);
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) bq[ks][0] = bq[ks][1] = 0u;
+    }
+  }
+  float acc[KH][4];
+#pragma unroll
+  for (int i = 0; i < KH; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  uint8_t* stage_mem = smem + p.keys_bytes;
+  const uint32_t sbase = smem_u32(stage_mem);
+  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const int nstages = (nloc + kSrTS - 1) / kSrTS;
+  auto issue = [&](int st) {
+    if (st < nstages) {
+      const uint32_t kt = sbase + (st % kSrStages) * STAGE;
+      const uint32_t vt = kt + TILE;
+#pragma unroll
+      for (int c = tid; c < kSrTS * CPR; c += kSrThreads) {
+        const int r = c / CPR, ch = c % CPR;
+        const int jj = st * kSrTS + r;
+        const bool ok = jj < nloc;
+        const int pos = ok ? plist[jj] : 0;
+        const int64_t eo = (int64_t)pos * p.stride_tok + ch * 8;
+        const uint32_t so = sr_tile_off(r, ch * 8);
+        cp_async_16(kt + so, kbase + eo, ok);
+        cp_async_16(vt + so, vbase + eo, ok);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < kSrStages - 1; ++s) issue(s);
+  for (int st = 0; st < nstages; ++st) {
+    cp_async_wait<kSrStages - 2>();
+    __syncthreads();
+    issue(st + kSrStages - 1);
+    const uint32_t kt = sbase + (st % kSrStages) * STAGE;
+    const uint32_t vt = kt + TILE;
+#pragma unroll
+    for (int u = 0; u < SUB; ++u) {
+      if ((st * SUB + u) % WT != tg) continue;
+      const int nv = nloc - (st * kSrTS + u * 16);
+      if (nv <= 0) continue;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int r = u * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int dsel = (lane >> 4) * 8;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(a, kt + sr_tile_off(r, ks * 16 + dsel));
+          mma_16816(s4, a, bq[ks][0], bq[ks][1]);
+        }
+      }
+      const int ta = lane >> 2, tb2 = ta + 8;
+      const float x0 = ta < nv ? s4[0] * p.scale_log2 : -INFINITY;
+      const float x1 = ta < nv ? s4[1] * p.scale_log2 : -INFINITY;
+      const float x2 = tb2 < nv ? s4[2] * p.scale_log2 : -INFINITY;
+      const float x3 = tb2 < nv ? s4[3] * p.scale_log2 : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+      const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+      const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+      l0 = l0 * al0 + p0 + p2;
+      l1 = l1 * al1 + p1 + p3;
+      m0 = mn0;
+      m1 = mn1;
+#pragma unroll
+      for (int i2 = 0; i2 < KH; ++i2) {
+        acc[i2][0] *= al0;
+        acc[i2][1] *= al1;
+        acc[i2][2] *= al0;
+        acc[i2][3] *= al1;
+      }
+      const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+      const uint32_t l01 = pack_bf16x2(p0 - bf16lo(h01), p1 - bf16hi(h01));
+      const uint32_t l23 = pack_bf16x2(p2 - bf16lo(h23), p3 - bf16hi(h23));
+      const uint32_t pb0 = movmatrix_trans(h01), pb1 = movmatrix_trans(h23);
+      const uint32_t pl0 = movmatrix_trans(l01), pl1 = movmatrix_trans(l23);
+      {
+        const int r = u * 16 + (lane & 7) + (lane >> 4) * 8;
+        const int dsel = ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int mt = 0; mt < KH; ++mt) {
+          uint32_t a[4];
+          ldsm_x4_trans(a, vt + sr_tile_off(r, (half * KH + mt) * 16 + dsel));
+          mma_16816(acc[mt], a, pb0, pb1);
+          mma_16816(acc[mt], a, pl0, pl1);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  __syncthreads();  // stage buffers are free
+
+  // ---- merge the warps of this CTA: red_ml [8][8][2], red_acc [8][8][D/2]; CTA state after
+  float* red_ml = reinterpret_cast<float*>(stage_mem);
+  float* red_acc = red_ml + 8 * 8 * 2;
+  float* cst_ml = red_acc + 8 * 8 * (D / 2);   // [NQP][2]   (read by the cluster peers)
+  float* cst_acc = cst_ml + NQP * 2;           // [NQP][D]
+  {
+    const int c0 = 2 * (lane & 3);
+    if (lane < 4) {
+      red_ml[(warp * 8 + c0) * 2 + 0] = m0;
+      red_ml[(warp * 8 + c0) * 2 + 1] = l0;
+      red_ml[(warp * 8 + c0 + 1) * 2 + 0] = m1;
+      red_ml[(warp * 8 + c0 + 1) * 2 + 1] = l1;
+    }
+#pragma unroll
+    for (int mt = 0; mt < KH; ++mt) {
+      const int d0 = mt * 16 + (lane >> 2);
+      red_acc[(warp * 8 + c0) * (D / 2) + d0] = acc[mt][0];
+      red_acc[(warp * 8 + c0 + 1) * (D / 2) + d0] = acc[mt][1];
+      red_acc[(warp * 8 + c0) * (D / 2) + d0 + 8] = acc[mt][2];
+      red_acc[(warp * 8 + c0 + 1) * (D / 2) + d0 + 8] = acc[mt][3];
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < NQP * D; e += kSrThreads) {
+    const int qr = e / D, dd = e % D;
+    const int hf = dd / (D / 2), ntq = qr >> 3, cq = qr & 7;
+    float M = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t + 4 * hf) * 8 + cq) * 2]);
+    float Ls = 0.f, A = 0.f;
+#pragma unroll
+    for (int t = 0; t < WT; ++t) {
+      const int w = ntq + NT * t + 4 * hf;
+      const float mw = red_ml[(w * 8 + cq) * 2];
+      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
+      A += f * red_acc[(w * 8 + cq) * (D / 2) + (dd % (D / 2))];
+    }
+    cst_acc[qr * D + dd] = A;
+    if (dd == 0) {
+      cst_ml[qr * 2] = M;
+      cst_ml[qr * 2 + 1] = Ls;
+    }
+  }
+
+  // =============================================================== 4. combine over the cluster
+  cluster.sync();
+  float* wsm = red_ml;  // [CL][NQP] weights, then [NQP] totals (local scratch; red_* are dead)
+  float* Lsm = wsm + 16 * NQP;
+  if (tid < NQP) {
+    float M = -INFINITY;
+    for (int q = 0; q < CL; ++q) M = fmaxf(M, cluster.map_shared_rank(cst_ml, q)[tid * 2]);
+    float Ls = 0.f;
+    for (int q = 0; q < CL; ++q) {
+      const float* r_ml = cluster.map_shared_rank(cst_ml, q);
+      const float mq = r_ml[tid * 2];
+      const float f = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
+      wsm[q * NQP + tid] = f;
+      Ls += f * r_ml[tid * 2 + 1];
+    }
+    Lsm[tid] = Ls;
+  }
+  __syncthreads();
+  {
+    const int total = p.NQ * D;
+    const int per = (total + CL - 1) / CL;
+    const int e0 = rk * per, e1 = min(total, e0 + per);
+    for (int e = e0 + tid; e < e1; e += kSrThreads) {
+      const int qr = e / D, dd = e % D;
+      float A = 0.f;
+      for (int q = 0; q < CL; ++q) A += wsm[q * NQP + qr] * cluster.map_shared_rank(cst_acc, q)[qr * D + dd];
+      const int l = qr / p.G, h = g * p.G + qr % p.G;
+      p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Lsm[qr];
+    }
+  }
+  cluster.sync();  // peers may read this CTA's state until every CTA is done
+}
+
+}  // namespace aoh

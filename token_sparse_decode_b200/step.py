@@ -75,8 +75,11 @@ class SparseDecodeStep:
 
 
 class SharedIndexStep:
+    """fused=True: one ``aoh_shared_index_step`` launch; False: score, select, decode as three calls."""
+
     def __init__(self, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
-                 n_layers: int, n_q_heads: int, topk: int, scale: float):
+                 n_layers: int, n_q_heads: int, topk: int, scale: float, fused: bool = True):
+        self.fused = fused
         self.dev = k.device
         self.k, self.v, self.offsets = k, v, offsets
         self.kv = B.make_kv(k, v, offsets, max_len, total_tokens)
@@ -95,6 +98,9 @@ class SharedIndexStep:
         B.topk_select(self.scores, self.kv, self.topk, None, self.topk, self.idx, self.count)
 
     def __call__(self, q_index: torch.Tensor, q_layers: torch.Tensor) -> torch.Tensor:
+        if self.fused:
+            B.shared_index_step(q_index, q_layers, self.kv, self.topk, self.idx, self.count, self.scale, self.out)
+            return self.out
         self.index(q_index)
         B.shared_index_decode(q_layers, self.kv, self.idx, self.count, self.topk, self.scale, self.out, self.ws)
         return self.out
