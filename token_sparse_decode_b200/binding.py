@@ -129,8 +129,8 @@ def make_kv(k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: in
 
 
 def k_dom_cols(n_dom: int) -> int:
-    """Row length of the packed dominant-column copy: 2*n_dom rounded up to 8 * 2^j elements."""
-    c = 8
+    """Row length of the packed dominant-column copy: 2*n_dom rounded up to 16 * 2^j elements."""
+    c = 16
     while c < 2 * n_dom:
         c *= 2
     return c

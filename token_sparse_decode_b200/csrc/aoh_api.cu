@@ -238,7 +238,8 @@ FusedPlan fused_plan(const aoh_kv_cache* kv, int n_rows, int nq) {
   if (slice > int64_t(kSrThreads) * kSrMaxRun) return f;  // row too long for one cluster
   f.slice_max = (int)slice;
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
-  const size_t stage = size_t(kSrStages) * 2 * kSrTS * kv->head_dim * 2;
+  // the attention stages and the scan ring share one region (used one after the other)
+  const size_t stage = std::max<size_t>(size_t(kSrStages) * 2 * kSrTS * kv->head_dim * 2, 4 * kSrRingStage);
   f.smem = f.keys_bytes + stage;
   f.ok = f.smem <= 200 * 1024;
   return f;
@@ -287,7 +288,7 @@ aoh_status launch_rows(const RowParams& rp, const FusedPlan& f, int d, int nq, i
 void rows_score_source(RowParams& rp, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom) {
   rp.idom = idom;
   rp.n_dom = n_dom;
-  if (kv->k_dom && idom) {
+  if (kv->k_dom && idom && (kv->k_dom_cols % 16) == 0) {
     rp.score_src = static_cast<const uint16_t*>(kv->k_dom);
     rp.srow_stride_tok = kv->k_dom_cols;
     rp.srow_stride_head = kv->total_tokens * kv->k_dom_cols;
@@ -300,9 +301,6 @@ void rows_score_source(RowParams& rp, const aoh_kv_cache* kv, const int32_t* ido
     rp.srow_len = kv->head_dim;
     rp.packed = 0;
   }
-  int segs = 1;
-  while (segs * 8 < rp.srow_len) segs <<= 1;
-  rp.segs = segs;
 }
 
 int list_heads(const aoh_kv_cache* kv, const uint8_t* roles, bool want_sparse, uint8_t* out) {

@@ -8,9 +8,11 @@
 //
 // The row's L positions are cut into CL contiguous slices, one per CTA.
 //  1. scan:    each CTA streams the score rows of its slice (packed dominant
-//              columns, or K in place) with 16-byte loads, keeps the fp32 scores
-//              as order-preserving uint32 keys in shared memory and counts the
-//              first radix digit on the fly;
+//              columns, or K in place) through a 4-stage cp.async ring and scores
+//              16 rows per tensor-core MMA: rows on M, the group-summed query split
+//              into hi + lo bf16 parts on N (score = C[:,0] + C[:,1], fp32-exact to
+//              ~2^-17 of the query); the scores stay in shared memory as
+//              order-preserving uint32 keys;
 //  2. select:  4-digit MSB radix select of the n-th largest key over the cluster
 //              (histograms summed through distributed shared memory, one cluster
 //              barrier per digit); ties broken toward lower positions by an ordered
@@ -38,6 +40,7 @@ constexpr int kSrThreads = 256;  // 8 warps
 constexpr int kSrTS = 32;        // tokens per attention stage
 constexpr int kSrStages = 4;
 constexpr int kSrMaxRun = 64;    // keys per thread in the compaction: slice <= 256 * 64
+constexpr int kSrRingStage = 16384;  // bytes per stage of the scan ring (4 stages)
 
 struct RowParams {
   const uint16_t* q_score;   // [B][Hq][D]: the query that scores (group-summed)
@@ -47,9 +50,8 @@ struct RowParams {
   const int32_t* offsets;    // [B + 1]
   const uint16_t* score_src; // packed k_dom or K
   int64_t srow_stride_tok, srow_stride_head;
-  int32_t srow_len;          // elements per score row (k_dom cols, or D in place)
+  int32_t srow_len;          // elements per score row: 16, 32, 64 or 128 (k_dom cols, or D in place)
   int32_t packed;            // 1: k_dom rows; 0: K rows with q masked to the dominant dims
-  int32_t segs;              // lanes per score row: srow_len / 8 rounded up to a power of two
   const int32_t* idom;       // [Hkv][n_dom]; null = every chunk
   int32_t n_dom;
   const int32_t* n_fac_per_seq;
@@ -72,24 +74,14 @@ __device__ __forceinline__ uint32_t sr_tile_off(int r, int dd) {
   return (uint32_t)(half * (kSrTS * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ uint4 sr_ld_stream(const uint16_t* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ float sr_dot8(const uint4& w, const float (&qs)[8]) {
-  float s = bf16lo(w.x) * qs[0];
-  s = fmaf(bf16hi(w.x), qs[1], s);
-  s = fmaf(bf16lo(w.y), qs[2], s);
-  s = fmaf(bf16hi(w.y), qs[3], s);
-  s = fmaf(bf16lo(w.z), qs[4], s);
-  s = fmaf(bf16hi(w.z), qs[5], s);
-  s = fmaf(bf16lo(w.w), qs[6], s);
-  s = fmaf(bf16hi(w.w), qs[7], s);
-  return s;
+// Byte offset of 16-byte chunk c of row r in a ring stage of rows RB bytes long
+// (RB in {32, 64, 128, 256}): linear rows, chunk-in-128B-line XOR-swizzled by the
+// line (RB <= 128) or the row (RB = 256), so that ldmatrix reads of 8 consecutive
+// rows hit 8 distinct 16-byte bank groups.
+__device__ __forceinline__ uint32_t tip_ring_off(int r, int c, int rb_shift) {
+  const uint32_t A = ((uint32_t)r << rb_shift) + ((uint32_t)c << 4);
+  const uint32_t key = (A >> (rb_shift > 7 ? rb_shift : 7)) & 7u;
+  return (A & ~127u) | ((((A >> 4) & 7u) ^ key) << 4);
 }
 
 // Warp-aggregated histogram increment (bin < 0: lane does not count).
@@ -154,7 +146,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
 
   if (n < L) {
     // =============================================================== 1. scan
-    hist[0][tid] = 0;  // kSrThreads == 256 bins
     if (tid < p.srow_len) {
       const int C = D / 2;
       int dim = -1;
@@ -187,42 +178,74 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     }
     __syncthreads();
     {
-      const int segs = p.segs;
-      const int seg = lane & (segs - 1);
-      float qs[8];
-      bool active = false;
+      // B fragments of [hi | lo | 0 ...] (k = score dims, n = 8 columns): lanes 0-3 carry
+      // column 0 (hi), lanes 4-7 column 1 (lo), the others zeros.
+      const int ksteps = p.srow_len >> 4;   // 1 .. 8
+      uint32_t bt[8][2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        qs[i] = (seg * 8 + i < p.srow_len) ? qt[seg * 8 + i] : 0.f;
-        active |= (qs[i] != 0.f);
-      }
-      const int rpw = 32 / segs;               // rows per warp per load
-      const int rpi = kSrThreads / segs;       // rows per block per load
-      constexpr int U = 8;                     // loads in flight per thread
-      const uint16_t* base = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)off * p.srow_stride_tok + seg * 8;
-      const int lrow = lane / segs;
-      for (int tb = lo + warp * rpw; tb < hi; tb += U * rpi) {  // warp-uniform bounds
-        uint4 w[U];
+      for (int ks = 0; ks < 8; ++ks) {
+        bt[ks][0] = bt[ks][1] = 0u;
+        if (ks < ksteps && lane < 8) {
+          const int d0 = ks * 16 + 2 * (lane & 3);
+          float v[4] = {qt[d0], qt[d0 + 1], qt[d0 + 8], qt[d0 + 9]};
+          if (lane >= 4) {  // lo = value - bf16(value)
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int tt = tb + u * rpi + lrow;
-          w[u] = make_uint4(0u, 0u, 0u, 0u);
-          if (tt < hi && active) w[u] = sr_ld_stream(base + (int64_t)tt * p.srow_stride_tok);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          float s = sr_dot8(w[u], qs);
-          for (int o = segs >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          const int tt = tb + u * rpi + lrow;
-          int bin = -1;
-          if (seg == 0 && tt < hi) {
-            const uint32_t key = score_key(s);
-            keys[tt - lo] = key;
-            bin = (int)(key >> 24);
+            for (int i = 0; i < 4; ++i) v[i] -= __bfloat162float(__float2bfloat16_rn(v[i]));
           }
-          hist_add(hist[0], bin);
+          bt[ks][0] = pack_bf16x2(v[0], v[1]);
+          bt[ks][1] = pack_bf16x2(v[2], v[3]);
         }
       }
+      const int rb_shift = 31 - __clz(p.srow_len * 2);   // row bytes = 2^rb_shift
+      const int cpr = (p.srow_len * 2) >> 4;              // 16-byte chunks per row
+      const int tr = kSrRingStage >> rb_shift;            // rows per stage
+      const int nst = (m + tr - 1) / tr;
+      const uint16_t* base = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)(off + lo) * p.srow_stride_tok;
+      const uint32_t rbase = smem_u32(smem + p.keys_bytes);
+      auto issue = [&](int st) {
+        if (st < nst) {
+          const uint32_t sb = rbase + (st & 3) * kSrRingStage;
+#pragma unroll
+          for (int i = 0; i < kSrRingStage / 16 / kSrThreads; ++i) {
+            const int c = tid + i * kSrThreads;
+            const int r = c / cpr, ch = c - r * cpr;
+            const int row = st * tr + r;
+            const bool ok = row < m;
+            cp_async_16(sb + tip_ring_off(r, ch, rb_shift), base + (int64_t)(ok ? row : 0) * p.srow_stride_tok + ch * 8, ok);
+          }
+        }
+        cp_async_commit();
+      };
+      issue(0);
+      issue(1);
+      issue(2);
+      for (int st = 0; st < nst; ++st) {
+        cp_async_wait<2>();
+        __syncthreads();
+        issue(st + 3);
+        const uint32_t sb = rbase + (st & 3) * kSrRingStage;
+        for (int tile = warp; tile * 16 < tr; tile += 8) {
+          const int nv = m - (st * tr + tile * 16);
+          if (nv <= 0) break;
+          float c4[4] = {0.f, 0.f, 0.f, 0.f};
+          const int r = tile * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            if (ks < ksteps) {
+              uint32_t a[4];
+              ldsm_x4(a, sb + tip_ring_off(r, 2 * ks + (lane >> 4), rb_shift));
+              mma_16816(c4, a, bt[ks][0], bt[ks][1]);
+            }
+          }
+          if ((lane & 3) == 0) {
+            const int r0 = tile * 16 + (lane >> 2);
+            if (r0 < nv) keys[st * tr + r0] = score_key(c4[0] + c4[1]);
+            if (r0 + 8 < nv) keys[st * tr + r0 + 8] = score_key(c4[2] + c4[3]);
+          }
+        }
+      }
+      cp_async_wait<0>();
+      __syncthreads();
     }
 
     // =============================================================== 2. select
@@ -232,18 +255,16 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       int* h = hist[pass & 1];
-      if (pass > 0) {
-        h[tid] = 0;
-        __syncthreads();
-        for (int bs = lo + (tid & ~31); bs < hi; bs += kSrThreads) {
-          const int i = bs + lane;
-          int bin = -1;
-          if (i < hi) {
-            const uint32_t k = keys[i - lo];
-            if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
-          }
-          hist_add(h, bin);
+      h[tid] = 0;
+      __syncthreads();
+      for (int bs = lo + (tid & ~31); bs < hi; bs += kSrThreads) {
+        const int i = bs + lane;
+        int bin = -1;
+        if (i < hi) {
+          const uint32_t k = keys[i - lo];
+          if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
         }
+        hist_add(h, bin);
       }
       cluster.sync();
       int tot = 0;
