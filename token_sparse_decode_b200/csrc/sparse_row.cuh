@@ -238,9 +238,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
             }
           }
           if ((lane & 3) == 0) {
-            const int r0 = tile * 16 + (lane >> 2);
-            if (r0 < nv) keys[st * tr + r0] = score_key(c4[0] + c4[1]);
-            if (r0 + 8 < nv) keys[st * tr + r0 + 8] = score_key(c4[2] + c4[3]);
+            const int ri = lane >> 2;  // row within the 16-row tile; nv counts from the tile start
+            const int r0 = st * tr + tile * 16 + ri;
+            if (ri < nv) keys[r0] = score_key(c4[0] + c4[1]);
+            if (ri + 8 < nv) keys[r0 + 8] = score_key(c4[2] + c4[3]);
           }
         }
       }
