@@ -221,66 +221,121 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
 
 
 // ------------------------------------------------------------------ fused row kernel
+// Shared memory per CTA: keys of the slice, then a ring of 16 KB stages used by the
+// scan and then by the attention.  Two CTAs per SM when the keys leave room for a
+// ring of >= 64 KB in 108 KB, else one CTA per SM with up to 128 KB of ring.
+constexpr size_t kTwoPerSm = 108 * 1024;
+constexpr size_t kOnePerSm = 220 * 1024;
+constexpr size_t kRingMin = 4 * kSrRingStage;
+constexpr size_t kRingMax = kSrMaxStages * kSrRingStage;
+
 struct FusedPlan {
   bool ok;
   int CL;
-  int slice_max;
-  size_t keys_bytes, smem;
+  int slice;
+  size_t keys_bytes, ring_bytes, smem;
 };
 
-FusedPlan fused_plan(const aoh_kv_cache* kv, int n_rows, int nq) {
+FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
   FusedPlan f{};
-  if (nq > kMaxQRows) return f;
   const int64_t L = std::max(kv->max_len, 1);
-  f.CL = 8;
-  if (int64_t(n_rows) * 8 < kSmCount || ceil_div(L, 8) > int64_t(kSrThreads) * kSrMaxRun) f.CL = 16;
-  const int64_t slice = (ceil_div(L, f.CL) + 3) & ~int64_t(3);
-  if (slice > int64_t(kSrThreads) * kSrMaxRun) return f;  // row too long for one cluster
-  f.slice_max = (int)slice;
+  const int64_t slice = (ceil_div(L, CL) + 3) & ~int64_t(3);
+  if (slice > int64_t(kSrThreads) * kSrMaxRun) return f;  // row too long for CL CTAs
+  f.CL = CL;
+  f.slice = (int)slice;
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
-  // the attention stages and the scan ring share one region (used one after the other)
-  const size_t stage = std::max<size_t>(size_t(kSrStages) * 2 * kSrTS * kv->head_dim * 2, 4 * kSrRingStage);
-  f.smem = f.keys_bytes + stage;
-  f.ok = f.smem <= 200 * 1024;
+  size_t budget = kTwoPerSm;
+  if (f.keys_bytes + kRingMin > budget) budget = kOnePerSm;
+  if (f.keys_bytes + kRingMin > budget) return f;
+  f.ring_bytes = std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage);
+  f.smem = f.keys_bytes + f.ring_bytes;
+  f.ok = true;
   return f;
 }
 
+// Whether some cluster size handles these rows in one fused launch.
+bool fused_feasible(const aoh_kv_cache* kv, int nq) {
+  return nq <= kMaxQRows && fused_candidate(kv, kSrMaxCluster).ok;
+}
+
 template <int D, int NT>
-aoh_status launch_rows_t(const RowParams& rp, const FusedPlan& f, int n_listed, int B, cudaStream_t st) {
-  static size_t configured = 0;
-  if (f.smem > configured) {
-    aoh_status s = set_smem(sparse_row_kernel<D, NT>, 200 * 1024);
+aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st) {
+  auto kern = sparse_row_kernel<D, NT>;
+  static bool configured = false;
+  if (!configured) {
+    aoh_status s = set_smem(kern, kOnePerSm);
     if (s != AOH_OK) return s;
-    s = cuda_status(cudaFuncSetAttribute(sparse_row_kernel<D, NT>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    s = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     if (s != AOH_OK) return s;
-    configured = 200 * 1024;
+    configured = true;
   }
+  // cluster size: fewest waves x slice length (the per-CTA work), ties to the smaller cluster
+  static int occ_cache[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // [CL 4/8/16][two-per-SM?]
+  const int n_rows = n_listed * B;
+  FusedPlan best{};
+  int64_t best_cost = INT64_MAX;
+  const int cls[3] = {4, 8, 16};
+  for (int i = 0; i < 3; ++i) {
+    const FusedPlan f = fused_candidate(kv, cls[i]);
+    if (!f.ok) continue;
+    const int two = f.smem <= kTwoPerSm ? 1 : 0;
+    int& maxc = occ_cache[i][two];
+    if (maxc < 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(f.CL, 1, 1);
+      cfg.blockDim = dim3(kSrThreads);
+      cfg.dynamicSmemBytes = two ? kTwoPerSm : kOnePerSm;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = f.CL;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      maxc = n;
+    }
+    if (maxc <= 0) continue;
+    const int64_t waves = ceil_div(n_rows, maxc);
+    const int64_t cost = waves * f.slice;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = f;
+    }
+  }
+  if (!best.ok) return AOH_ERR_UNSUPPORTED;
+  rp.keys_bytes = (int32_t)best.keys_bytes;
+  rp.ring_bytes = (int32_t)best.ring_bytes;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(f.CL, n_listed, B);
+  cfg.gridDim = dim3(best.CL, n_listed, B);
   cfg.blockDim = dim3(kSrThreads);
-  cfg.dynamicSmemBytes = f.smem;
+  cfg.dynamicSmemBytes = best.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = f.CL;
+  attr[0].val.clusterDim.x = best.CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, sparse_row_kernel<D, NT>, rp));
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, rp));
 }
 
-aoh_status launch_rows(const RowParams& rp, const FusedPlan& f, int d, int nq, int n_listed, int B,
+aoh_status launch_rows(const RowParams& rp, const aoh_kv_cache* kv, int nq, int n_listed, int B,
                        cudaStream_t st) {
   const int nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
-  if (d == 128) {
-    if (nqp == 8) return launch_rows_t<128, 1>(rp, f, n_listed, B, st);
-    if (nqp == 16) return launch_rows_t<128, 2>(rp, f, n_listed, B, st);
-    return launch_rows_t<128, 4>(rp, f, n_listed, B, st);
+  if (kv->head_dim == 128) {
+    if (nqp == 8) return launch_rows_t<128, 1>(rp, kv, n_listed, B, st);
+    if (nqp == 16) return launch_rows_t<128, 2>(rp, kv, n_listed, B, st);
+    return launch_rows_t<128, 4>(rp, kv, n_listed, B, st);
   }
-  if (nqp == 8) return launch_rows_t<64, 1>(rp, f, n_listed, B, st);
-  if (nqp == 16) return launch_rows_t<64, 2>(rp, f, n_listed, B, st);
-  return launch_rows_t<64, 4>(rp, f, n_listed, B, st);
+  if (nqp == 8) return launch_rows_t<64, 1>(rp, kv, n_listed, B, st);
+  if (nqp == 16) return launch_rows_t<64, 2>(rp, kv, n_listed, B, st);
+  return launch_rows_t<64, 4>(rp, kv, n_listed, B, st);
 }
 
 // Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,
@@ -489,8 +544,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + off_idx);
   int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + off_count);
 
-  const FusedPlan plan = fused_plan(kv, kv->batch * n_listed, G);
-  if (plan.ok) {
+  if (fused_feasible(kv, G)) {
     RowParams rp{};
     rp.q_score = static_cast<const uint16_t*>(q);
     rp.q_attn = static_cast<const uint16_t*>(q);
@@ -512,10 +566,9 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
     rp.Hkv = kv->n_kv_heads;
     rp.G = G;
     rp.NQ = G;
-    rp.keys_bytes = (int32_t)plan.keys_bytes;
     rp.scale_log2 = scale * 1.4426950408889634f;
     memcpy(rp.heads, heads, n_listed);
-    return launch_rows(rp, plan, kv->head_dim, G, n_listed, kv->batch, st);
+    return launch_rows(rp, kv, G, n_listed, kv->batch, st);
   }
 
   // rows too long for one cluster: scan, select and attend as three kernels
@@ -661,8 +714,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   if (!aligned16(q_index) || !aligned16(q_layers)) return AOH_ERR_ALIGNMENT;
   uint8_t heads[kMaxHeads];
   const int n_listed = list_heads(kv, nullptr, true, heads);
-  const FusedPlan plan = fused_plan(kv, kv->batch * n_listed, n_layers * G);
-  if (!plan.ok) return AOH_ERR_UNSUPPORTED;
+  if (!fused_feasible(kv, n_layers * G)) return AOH_ERR_UNSUPPORTED;
   RowParams rp{};
   rp.q_score = static_cast<const uint16_t*>(q_index);
   rp.q_attn = static_cast<const uint16_t*>(q_layers);
@@ -684,10 +736,17 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   rp.Hkv = kv->n_kv_heads;
   rp.G = G;
   rp.NQ = n_layers * G;
-  rp.keys_bytes = (int32_t)plan.keys_bytes;
   rp.scale_log2 = scale * 1.4426950408889634f;
   memcpy(rp.heads, heads, n_listed);
-  return launch_rows(rp, plan, kv->head_dim, n_layers * G, n_listed, kv->batch, as_stream(stream));
+  return launch_rows(rp, kv, n_layers * G, n_listed, kv->batch, as_stream(stream));
 }
+
+#ifdef AOH_PHASE_TIMERS
+// Diagnostic build only: copy the phase stamps of the fused kernel to the host.
+int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
+  if (n_ctas > kPhaseCtas) n_ctas = kPhaseCtas;
+  return cudaMemcpyFromSymbol(host, g_phase_ns, sizeof(long long) * kPhaseSlots * n_ctas) == cudaSuccess ? 0 : 5;
+}
+#endif
 
 }  // extern "C"

@@ -38,9 +38,10 @@ namespace cgs = cooperative_groups;
 
 constexpr int kSrThreads = 256;  // 8 warps
 constexpr int kSrTS = 32;        // tokens per attention stage
-constexpr int kSrStages = 4;
+constexpr int kSrMaxStages = 8;  // ring stages (run-time count, from the shared memory left)
+constexpr int kSrMaxCluster = 16;
 constexpr int kSrMaxRun = 64;    // keys per thread in the compaction: slice <= 256 * 64
-constexpr int kSrRingStage = 16384;  // bytes per stage of the scan ring (4 stages)
+constexpr int kSrRingStage = 16384;  // bytes per stage of the scan ring
 
 struct RowParams {
   const uint16_t* q_score;   // [B][Hq][D]: the query that scores (group-summed)
@@ -61,7 +62,8 @@ struct RowParams {
   float* out;                // [n_layers][B][Hq][D]
   int64_t stride_tok, stride_head;
   int32_t T, B, Hq, Hkv, G, NQ;
-  int32_t keys_bytes;        // dynamic shared memory before the attention stages
+  int32_t keys_bytes;        // dynamic shared memory before the ring
+  int32_t ring_bytes;        // ring region (scan stages, then attention stages); >= 64 KB
   float scale_log2;
   uint8_t heads[kMaxHeads];
 };
@@ -83,6 +85,26 @@ __device__ __forceinline__ uint32_t tip_ring_off(int r, int c, int rb_shift) {
   const uint32_t key = (A >> (rb_shift > 7 ? rb_shift : 7)) & 7u;
   return (A & ~127u) | ((((A >> 4) & 7u) ^ key) << 4);
 }
+
+#ifdef AOH_PHASE_TIMERS
+// Diagnostic build only: global-timer stamps at the phase boundaries of every CTA.
+constexpr int kPhaseSlots = 8;
+constexpr int kPhaseCtas = 8192;
+__device__ long long g_phase_ns[kPhaseCtas][kPhaseSlots];
+__device__ __forceinline__ void phase_stamp(int slot) {
+  if (threadIdx.x == 0) {
+    const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    if (cta < kPhaseCtas) {
+      long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      g_phase_ns[cta][slot] = t;
+    }
+  }
+}
+#define AOH_PHASE(i) phase_stamp(i)
+#else
+#define AOH_PHASE(i)
+#endif
 
 // Warp-aggregated histogram increment (bin < 0: lane does not count).
 __device__ __forceinline__ void hist_add(int* h, int bin) {
@@ -109,7 +131,9 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   __shared__ float qt[128];
   __shared__ int s_bin, s_above, s_eq_before, s_sel_before;
   __shared__ int s_cnt[2];
+  __shared__ int s_all[kSrMaxCluster][2];
 
+  AOH_PHASE(0);
   cgs::cluster_group cluster = cgs::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int rk = (int)cluster.block_rank();
@@ -202,9 +226,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
       const int nst = (m + tr - 1) / tr;
       const uint16_t* base = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)(off + lo) * p.srow_stride_tok;
       const uint32_t rbase = smem_u32(smem + p.keys_bytes);
+      const int ns = min(kSrMaxStages, p.ring_bytes / kSrRingStage);
       auto issue = [&](int st) {
         if (st < nst) {
-          const uint32_t sb = rbase + (st & 3) * kSrRingStage;
+          const uint32_t sb = rbase + (st % ns) * kSrRingStage;
 #pragma unroll
           for (int i = 0; i < kSrRingStage / 16 / kSrThreads; ++i) {
             const int c = tid + i * kSrThreads;
@@ -216,14 +241,12 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
         }
         cp_async_commit();
       };
-      issue(0);
-      issue(1);
-      issue(2);
+      for (int s0 = 0; s0 < ns - 1; ++s0) issue(s0);
       for (int st = 0; st < nst; ++st) {
-        cp_async_wait<2>();
+        cp_async_wait_n(ns - 2);
         __syncthreads();
-        issue(st + 3);
-        const uint32_t sb = rbase + (st & 3) * kSrRingStage;
+        issue(st + ns - 1);
+        const uint32_t sb = rbase + (st % ns) * kSrRingStage;
         for (int tile = warp; tile * 16 < tr; tile += 8) {
           const int nv = m - (st * tr + tile * 16);
           if (nv <= 0) break;
@@ -249,6 +272,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
       __syncthreads();
     }
 
+    AOH_PHASE(1);
     // =============================================================== 2. select
     uint32_t prefix = 0u, pmask = 0u;
     int krem = n;
@@ -271,7 +295,11 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
       int tot = 0;
       {
         const int bin = 255 - tid;  // scanned from the top bin down
-        for (int q = 0; q < CL; ++q) tot += cluster.map_shared_rank(h, q)[bin];
+        int v[kSrMaxCluster];
+#pragma unroll
+        for (int q = 0; q < kSrMaxCluster; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
+#pragma unroll
+        for (int q = 0; q < kSrMaxCluster; ++q) tot += v[q];
       }
       int total;
       const int above = block_exclusive_scan(tot, scan_scratch, &total);
@@ -287,6 +315,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     }
     const uint32_t KT = prefix;
     const int need_eq = krem;
+    AOH_PHASE(2);
 
     // ---- ordered compaction: positions in ascending order, lower position first among equals
     const int run = (m + kSrThreads - 1) / kSrThreads;  // <= kSrMaxRun (host guarantees)
@@ -305,12 +334,17 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
       s_cnt[1] = gt_cta;
     }
     cluster.sync();
+    if (tid < CL) {
+      const int* c = cluster.map_shared_rank(s_cnt, tid);
+      s_all[tid][0] = c[0];
+      s_all[tid][1] = c[1];
+    }
+    __syncthreads();
     if (tid == 0) {
       int eq_before = 0, sel_before = 0;
       for (int q = 0; q < rk; ++q) {
-        const int* c = cluster.map_shared_rank(s_cnt, q);
-        sel_before += c[1] + max(0, min(need_eq - eq_before, c[0]));
-        eq_before += c[0];
+        sel_before += s_all[q][1] + max(0, min(need_eq - eq_before, s_all[q][0]));
+        eq_before += s_all[q][0];
       }
       s_eq_before = eq_before;
       s_sel_before = sel_before;
@@ -361,6 +395,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   }
   __syncthreads();
 
+  AOH_PHASE(3);
   // =============================================================== 3. attend
   const int half = warp >> 2, r4 = warp & 3;
   const int nt = r4 % NT, tg = r4 / NT;
@@ -390,9 +425,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
   const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
   const int nstages = (nloc + kSrTS - 1) / kSrTS;
+  const int nsa = min(kSrMaxStages, p.ring_bytes / STAGE);
   auto issue = [&](int st) {
     if (st < nstages) {
-      const uint32_t kt = sbase + (st % kSrStages) * STAGE;
+      const uint32_t kt = sbase + (st % nsa) * STAGE;
       const uint32_t vt = kt + TILE;
 #pragma unroll
       for (int c = tid; c < kSrTS * CPR; c += kSrThreads) {
@@ -408,13 +444,12 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     }
     cp_async_commit();
   };
-#pragma unroll
-  for (int s = 0; s < kSrStages - 1; ++s) issue(s);
+  for (int s = 0; s < nsa - 1; ++s) issue(s);
   for (int st = 0; st < nstages; ++st) {
-    cp_async_wait<kSrStages - 2>();
+    cp_async_wait_n(nsa - 2);
     __syncthreads();
-    issue(st + kSrStages - 1);
-    const uint32_t kt = sbase + (st % kSrStages) * STAGE;
+    issue(st + nsa - 1);
+    const uint32_t kt = sbase + (st % nsa) * STAGE;
     const uint32_t vt = kt + TILE;
 #pragma unroll
     for (int u = 0; u < SUB; ++u) {
@@ -484,6 +519,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   }
   __syncthreads();  // stage buffers are free
 
+  AOH_PHASE(4);
   // ---- merge the warps of this CTA: red_ml [8][8][2], red_acc [8][8][D/2]; CTA state after
   float* red_ml = reinterpret_cast<float*>(stage_mem);
   float* red_acc = red_ml + 8 * 8 * 2;
@@ -530,19 +566,32 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   }
 
   // =============================================================== 4. combine over the cluster
+  AOH_PHASE(5);
   cluster.sync();
+  AOH_PHASE(6);
   float* wsm = red_ml;  // [CL][NQP] weights, then [NQP] totals (local scratch; red_* are dead)
   float* Lsm = wsm + 16 * NQP;
   if (tid < NQP) {
+    float mv[kSrMaxCluster], lv[kSrMaxCluster];
+#pragma unroll
+    for (int q = 0; q < kSrMaxCluster; ++q) {
+      mv[q] = -INFINITY;
+      lv[q] = 0.f;
+      if (q < CL) {
+        const float* r_ml = cluster.map_shared_rank(cst_ml, q);
+        mv[q] = r_ml[tid * 2];
+        lv[q] = r_ml[tid * 2 + 1];
+      }
+    }
     float M = -INFINITY;
-    for (int q = 0; q < CL; ++q) M = fmaxf(M, cluster.map_shared_rank(cst_ml, q)[tid * 2]);
+#pragma unroll
+    for (int q = 0; q < kSrMaxCluster; ++q) M = fmaxf(M, mv[q]);
     float Ls = 0.f;
-    for (int q = 0; q < CL; ++q) {
-      const float* r_ml = cluster.map_shared_rank(cst_ml, q);
-      const float mq = r_ml[tid * 2];
-      const float f = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
-      wsm[q * NQP + tid] = f;
-      Ls += f * r_ml[tid * 2 + 1];
+#pragma unroll
+    for (int q = 0; q < kSrMaxCluster; ++q) {
+      const float f = (mv[q] == -INFINITY) ? 0.f : exp2f(mv[q] - M);
+      if (q < CL) wsm[q * NQP + tid] = f;
+      Ls += f * lv[q];
     }
     Lsm[tid] = Ls;
   }
@@ -553,13 +602,18 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     const int e0 = rk * per, e1 = min(total, e0 + per);
     for (int e = e0 + tid; e < e1; e += kSrThreads) {
       const int qr = e / D, dd = e % D;
+      float av[kSrMaxCluster];
+#pragma unroll
+      for (int q = 0; q < kSrMaxCluster; ++q) av[q] = (q < CL) ? cluster.map_shared_rank(cst_acc, q)[qr * D + dd] : 0.f;
       float A = 0.f;
-      for (int q = 0; q < CL; ++q) A += wsm[q * NQP + qr] * cluster.map_shared_rank(cst_acc, q)[qr * D + dd];
+#pragma unroll
+      for (int q = 0; q < kSrMaxCluster; ++q) A += (q < CL) ? wsm[q * NQP + qr] * av[q] : 0.f;
       const int l = qr / p.G, h = g * p.G + qr % p.G;
       p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Lsm[qr];
     }
   }
   cluster.sync();  // peers may read this CTA's state until every CTA is done
+  AOH_PHASE(7);
 }
 
 }  // namespace aoh
