@@ -258,6 +258,10 @@ bool fused_feasible(const aoh_kv_cache* kv, int nq) {
   return nq <= kMaxQRows && fused_candidate(kv, kSrMaxCluster).ok;
 }
 
+#ifdef AOH_PHASE_TIMERS
+int g_force_cluster = 0;  // diagnostic build: force the fused kernel's cluster size
+#endif
+
 template <int D, int NT>
 aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st) {
   auto kern = sparse_row_kernel<D, NT>;
@@ -278,6 +282,9 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   for (int i = 0; i < 3; ++i) {
     const FusedPlan f = fused_candidate(kv, cls[i]);
     if (!f.ok) continue;
+#ifdef AOH_PHASE_TIMERS
+    if (g_force_cluster && f.CL != g_force_cluster) continue;
+#endif
     const int two = f.smem <= kTwoPerSm ? 1 : 0;
     int& maxc = occ_cache[i][two];
     if (maxc < 0) {
@@ -742,6 +749,8 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
 }
 
 #ifdef AOH_PHASE_TIMERS
+void aoh_debug_force_cluster(int32_t cl) { g_force_cluster = cl; }
+
 // Diagnostic build only: copy the phase stamps of the fused kernel to the host.
 int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
   if (n_ctas > kPhaseCtas) n_ctas = kPhaseCtas;

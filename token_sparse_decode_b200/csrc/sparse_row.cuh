@@ -130,8 +130,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   __shared__ int scan_scratch[33];
   __shared__ float qt[128];
   __shared__ int s_bin, s_above, s_eq_before, s_sel_before;
-  __shared__ int s_cnt[2];
-  __shared__ int s_all[kSrMaxCluster][2];
+  __shared__ int s_gt[kSrMaxCluster], s_eq[kSrMaxCluster], s_eq_all;
 
   AOH_PHASE(0);
   cgs::cluster_group cluster = cgs::this_cluster();
@@ -274,6 +273,13 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
 
     AOH_PHASE(1);
     // =============================================================== 2. select
+    // Every CTA also learns, from the histograms it reads anyway, how many keys of
+    // each peer are above the threshold (s_gt) and equal to it (s_eq), so the
+    // compaction needs no further exchange.
+    if (tid < kSrMaxCluster) {
+      s_gt[tid] = 0;
+      s_eq[tid] = 0;
+    }
     uint32_t prefix = 0u, pmask = 0u;
     int krem = n;
 #pragma unroll 1
@@ -282,33 +288,54 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
       int* h = hist[pass & 1];
       h[tid] = 0;
       __syncthreads();
-      for (int bs = lo + (tid & ~31); bs < hi; bs += kSrThreads) {
-        const int i = bs + lane;
-        int bin = -1;
-        if (i < hi) {
-          const uint32_t k = keys[i - lo];
-          if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
+      // four keys per lane and iteration (warp-uniform trip count); the first digit
+      // (sign + exponent) is shared by most keys, so it is counted with warp
+      // aggregation, the later digits directly
+      for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
+        const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: the keys region covers it
+        const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
+        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool in = (i0 + j < m) && ((kk[j] & pmask) == prefix);
+          const int bin = in ? (int)((kk[j] >> shift) & 255u) : -1;
+          if (pass == 0) {
+            hist_add(h, bin);
+          } else if (in) {
+            atomicAdd(&h[bin], 1);
+          }
         }
-        hist_add(h, bin);
       }
       cluster.sync();
+      const int bin = 255 - tid;  // scanned from the top bin down
+      int v[kSrMaxCluster];
+#pragma unroll
+      for (int q = 0; q < kSrMaxCluster; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
       int tot = 0;
-      {
-        const int bin = 255 - tid;  // scanned from the top bin down
-        int v[kSrMaxCluster];
 #pragma unroll
-        for (int q = 0; q < kSrMaxCluster; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
-#pragma unroll
-        for (int q = 0; q < kSrMaxCluster; ++q) tot += v[q];
-      }
+      for (int q = 0; q < kSrMaxCluster; ++q) tot += v[q];
       int total;
       const int above = block_exclusive_scan(tot, scan_scratch, &total);
       if (above < krem && krem <= above + tot) {
-        s_bin = 255 - tid;
+        s_bin = bin;
         s_above = above;
       }
       __syncthreads();
-      prefix |= (uint32_t)s_bin << shift;
+      const int sb = s_bin;
+      // keys of every peer in bins above the chosen one are above the threshold
+#pragma unroll
+      for (int q = 0; q < kSrMaxCluster; ++q) {
+        if (q < CL) {
+          const int w = __reduce_add_sync(0xffffffffu, bin > sb ? v[q] : 0);
+          if (lane == 0 && w) atomicAdd(&s_gt[q], w);
+        }
+      }
+      if (pass == 3 && bin == sb) {
+#pragma unroll
+        for (int q = 0; q < kSrMaxCluster; ++q)
+          if (q < CL) s_eq[q] = v[q];
+      }
+      prefix |= (uint32_t)sb << shift;
       pmask |= 255u << shift;
       krem -= s_above;
       __syncthreads();
@@ -318,38 +345,29 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     AOH_PHASE(2);
 
     // ---- ordered compaction: positions in ascending order, lower position first among equals
-    const int run = (m + kSrThreads - 1) / kSrThreads;  // <= kSrMaxRun (host guarantees)
-    const int a0 = min(m, tid * run), a1 = min(m, (tid + 1) * run);
-    int n_eq = 0, n_gt = 0;
-    for (int i = a0; i < a1; ++i) {
-      const uint32_t k = keys[i];
-      n_gt += k > KT;
-      n_eq += k == KT;
-    }
-    int eq_cta, gt_cta;
-    const int eq_excl = block_exclusive_scan(n_eq, scan_scratch, &eq_cta);
-    block_exclusive_scan(n_gt, scan_scratch, &gt_cta);
     if (tid == 0) {
-      s_cnt[0] = eq_cta;
-      s_cnt[1] = gt_cta;
-    }
-    cluster.sync();
-    if (tid < CL) {
-      const int* c = cluster.map_shared_rank(s_cnt, tid);
-      s_all[tid][0] = c[0];
-      s_all[tid][1] = c[1];
-    }
-    __syncthreads();
-    if (tid == 0) {
-      int eq_before = 0, sel_before = 0;
-      for (int q = 0; q < rk; ++q) {
-        sel_before += s_all[q][1] + max(0, min(need_eq - eq_before, s_all[q][0]));
-        eq_before += s_all[q][0];
+      int eq_before = 0, sel_before = 0, eq_all = 0;
+      for (int q = 0; q < CL; ++q) {
+        if (q < rk) {
+          sel_before += s_gt[q] + max(0, min(need_eq - eq_before, s_eq[q]));
+          eq_before += s_eq[q];
+        }
+        eq_all += s_eq[q];
       }
       s_eq_before = eq_before;
       s_sel_before = sel_before;
+      s_eq_all = eq_all;
     }
     __syncthreads();
+    const int run = (m + kSrThreads - 1) / kSrThreads;  // <= kSrMaxRun (host guarantees)
+    const int a0 = min(m, tid * run), a1 = min(m, (tid + 1) * run);
+    int eq_excl = 0;
+    if (s_eq_all > need_eq) {  // more keys equal the threshold than are taken: rank them
+      int n_eq = 0;
+      for (int i = a0; i < a1; ++i) n_eq += keys[i] == KT;
+      int eq_cta;
+      eq_excl = block_exclusive_scan(n_eq, scan_scratch, &eq_cta);
+    }
     uint64_t take = 0ull;
     int n_sel = 0;
     {
