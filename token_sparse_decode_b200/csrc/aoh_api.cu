@@ -1,6 +1,7 @@
 // C ABI of the token-sparse decode step: argument checks on the host, then
 // asynchronous launches on the caller's stream.  Declarations and the contract
 // of every entry point are in include/aoh.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -244,18 +245,78 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
   f.CL = CL;
   f.slice = (int)slice;
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
-  size_t budget = kTwoPerSm;
-  if (f.keys_bytes + kRingMin > budget) budget = kOnePerSm;
+  // 1 KB of slack: the kernel aligns its dynamic shared memory to 1024 bytes
+  size_t budget = kTwoPerSm - 1024;
+  if (f.keys_bytes + kRingMin > budget) budget = kOnePerSm - 1024;
   if (f.keys_bytes + kRingMin > budget) return f;
   f.ring_bytes = std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage);
-  f.smem = f.keys_bytes + f.ring_bytes;
+  f.smem = f.keys_bytes + f.ring_bytes + 1024;
   f.ok = true;
   return f;
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled, resolved through the runtime (no link against the driver library)
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return (EncodeTiledFn) nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+// The scan reads its rows through a 2-D tensor map: packed rows as [Hkv * T][cols]; K in
+// place as [T][stride_tok] with the head at column g * stride_head (needs every head's
+// row inside one token stride).
+bool scan_layout_ok(const aoh_kv_cache* kv, bool packed) {
+  if (packed) return true;
+  return int64_t(kv->n_kv_heads - 1) * kv->stride_head + kv->head_dim <= kv->stride_tok;
+}
+
+aoh_status make_scan_map(RowParams& rp, const aoh_kv_cache* kv) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (!enc) return AOH_ERR_CUDA;
+  const int box = std::min(rp.srow_len, 64);
+  const int rows = std::min(256, kSrRingStage / (rp.srow_len * 2));
+  rp.scan_box = box;
+  rp.scan_rows = rows;
+  cuuint64_t dims[2], strides[1];
+  if (rp.packed) {
+    dims[0] = (cuuint64_t)kv->k_dom_cols;
+    dims[1] = (cuuint64_t)kv->n_kv_heads * (cuuint64_t)kv->total_tokens;
+    strides[0] = (cuuint64_t)kv->k_dom_cols * 2;
+  } else {
+    dims[0] = (cuuint64_t)kv->stride_tok;
+    dims[1] = (cuuint64_t)kv->total_tokens;
+    strides[0] = (cuuint64_t)kv->stride_tok * 2;
+  }
+  const cuuint32_t boxd[2] = {(cuuint32_t)box, (cuuint32_t)rows};
+  const cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box * 2 == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                : box * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUresult r = enc(&rp.tmap_scan, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(rp.score_src), dims,
+                         strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AOH_OK : AOH_ERR_CUDA;
+}
+
+bool packed_scan(const aoh_kv_cache* kv, const int32_t* idom) {
+  return kv->k_dom && idom && (kv->k_dom_cols % 16) == 0;
+}
+
 // Whether some cluster size handles these rows in one fused launch.
-bool fused_feasible(const aoh_kv_cache* kv, int nq) {
-  return nq <= kMaxQRows && fused_candidate(kv, kSrMaxCluster).ok;
+bool fused_feasible(const aoh_kv_cache* kv, int nq, bool packed) {
+  return nq <= kMaxQRows && scan_layout_ok(kv, packed) && fused_candidate(kv, kSrMaxCluster).ok;
 }
 
 #ifdef AOH_PHASE_TIMERS
@@ -285,13 +346,13 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
 #ifdef AOH_PHASE_TIMERS
     if (g_force_cluster && f.CL != g_force_cluster) continue;
 #endif
-    const int two = f.smem <= kTwoPerSm ? 1 : 0;
+    const int two = f.smem <= kTwoPerSm ? 1 : 0;  // the cache holds one entry per budget class
     int& maxc = occ_cache[i][two];
     if (maxc < 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(f.CL, 1, 1);
       cfg.blockDim = dim3(kSrThreads);
-      cfg.dynamicSmemBytes = two ? kTwoPerSm : kOnePerSm;
+      cfg.dynamicSmemBytes = f.smem;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = f.CL;
@@ -315,6 +376,10 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
     }
   }
   if (!best.ok) return AOH_ERR_UNSUPPORTED;
+  {
+    const aoh_status ms = make_scan_map(rp, kv);
+    if (ms != AOH_OK) return ms;
+  }
   rp.keys_bytes = (int32_t)best.keys_bytes;
   rp.ring_bytes = (int32_t)best.ring_bytes;
   cudaLaunchConfig_t cfg = {};
@@ -350,7 +415,7 @@ aoh_status launch_rows(const RowParams& rp, const aoh_kv_cache* kv, int nq, int 
 void rows_score_source(RowParams& rp, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom) {
   rp.idom = idom;
   rp.n_dom = n_dom;
-  if (kv->k_dom && idom && (kv->k_dom_cols % 16) == 0) {
+  if (packed_scan(kv, idom)) {
     rp.score_src = static_cast<const uint16_t*>(kv->k_dom);
     rp.srow_stride_tok = kv->k_dom_cols;
     rp.srow_stride_head = kv->total_tokens * kv->k_dom_cols;
@@ -551,7 +616,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + off_idx);
   int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + off_count);
 
-  if (fused_feasible(kv, G)) {
+  if (fused_feasible(kv, G, packed_scan(kv, idom))) {
     RowParams rp{};
     rp.q_score = static_cast<const uint16_t*>(q);
     rp.q_attn = static_cast<const uint16_t*>(q);
@@ -721,7 +786,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   if (!aligned16(q_index) || !aligned16(q_layers)) return AOH_ERR_ALIGNMENT;
   uint8_t heads[kMaxHeads];
   const int n_listed = list_heads(kv, nullptr, true, heads);
-  if (!fused_feasible(kv, n_layers * G)) return AOH_ERR_UNSUPPORTED;
+  if (!fused_feasible(kv, n_layers * G, false)) return AOH_ERR_UNSUPPORTED;
   RowParams rp{};
   rp.q_score = static_cast<const uint16_t*>(q_index);
   rp.q_attn = static_cast<const uint16_t*>(q_layers);

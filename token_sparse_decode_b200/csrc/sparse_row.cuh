@@ -29,6 +29,7 @@
 #pragma once
 
 #include <cooperative_groups.h>
+#include <cuda.h>  // CUtensorMap (the map is encoded on the host through the runtime's driver entry point)
 
 #include "device_common.cuh"
 
@@ -44,6 +45,7 @@ constexpr int kSrMaxRun = 64;    // keys per thread in the compaction: slice <= 
 constexpr int kSrRingStage = 16384;  // bytes per stage of the scan ring
 
 struct RowParams {
+  CUtensorMap tmap_scan;     // 2-D view of the score rows: packed [Hkv*T][cols] or K [T][stride_tok]
   const uint16_t* q_score;   // [B][Hq][D]: the query that scores (group-summed)
   const uint16_t* q_attn;    // [n_layers][B][Hq][D]: query rows of the attention
   const uint16_t* k;
@@ -64,26 +66,29 @@ struct RowParams {
   int32_t T, B, Hq, Hkv, G, NQ;
   int32_t keys_bytes;        // dynamic shared memory before the ring
   int32_t ring_bytes;        // ring region (scan stages, then attention stages); >= 64 KB
+  int32_t scan_box;          // scan tile: inner box (elements, <= 64) ...
+  int32_t scan_rows;         // ... and rows per stage (<= 256); halves = srow_len / scan_box
   float scale_log2;
   uint8_t heads[kMaxHeads];
 };
 
-// Byte offset of (row r, dim dd) in a [kSrTS x D] tile: D/64 halves of [kSrTS x 128 B],
-// 16-byte chunks XOR-swizzled by (r mod 8).
-__device__ __forceinline__ uint32_t sr_tile_off(int r, int dd) {
-  const int half = dd >> 6;
-  const int cc = (dd & 63) >> 3;
-  return (uint32_t)(half * (kSrTS * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
-}
+// Attention tiles: gathered K / V rows land whole (one 1-D bulk copy each) at a row
+// pitch of 2*D + 16 bytes, so the 8 rows an ldmatrix reads sit in 8 different
+// 16-byte bank groups.
+template <int D>
+struct AttTile {
+  static constexpr int kPitch = 2 * D + 16;
+  static constexpr int kTile = kSrTS * kPitch;  // one of K or V per stage
+  static constexpr int kStage = 2 * kTile;
+};
 
-// Byte offset of 16-byte chunk c of row r in a ring stage of rows RB bytes long
-// (RB in {32, 64, 128, 256}): linear rows, chunk-in-128B-line XOR-swizzled by the
-// line (RB <= 128) or the row (RB = 256), so that ldmatrix reads of 8 consecutive
-// rows hit 8 distinct 16-byte bank groups.
-__device__ __forceinline__ uint32_t tip_ring_off(int r, int c, int rb_shift) {
-  const uint32_t A = ((uint32_t)r << rb_shift) + ((uint32_t)c << 4);
-  const uint32_t key = (A >> (rb_shift > 7 ? rb_shift : 7)) & 7u;
-  return (A & ~127u) | ((((A >> 4) & 7u) ^ key) << 4);
+// Scan tiles are written by the tensor map with the span-byte swizzle (span = 2 * box,
+// 32/64/128 bytes): 16-byte chunk bits XOR address bits 7.. (span/16 - 1 mask).
+__device__ __forceinline__ uint32_t scan_tile_off(int r, int c, int span_shift, int rows) {
+  const int cpb = 1 << (span_shift - 4);     // 16-byte chunks per box row
+  const int h = c >> (span_shift - 4);
+  const uint32_t off = (uint32_t)(h * rows + r) << span_shift | (uint32_t)(c & (cpb - 1)) << 4;
+  return off ^ (((off >> 7) & (uint32_t)(cpb - 1)) << 4);
 }
 
 #ifdef AOH_PHASE_TIMERS
@@ -113,7 +118,7 @@ __device__ __forceinline__ void hist_add(int* h, int bin) {
 }
 
 template <int D, int NT>
-__global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams p) {
+__global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_constant__ RowParams p) {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
   constexpr int KS = D / 16;          // k-steps of QK
@@ -121,16 +126,15 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   constexpr int WT = 4 / NT;          // token groups per (n-tile, half)
   constexpr int SUB = kSrTS / 16;     // 16-token sub-tiles per stage
   constexpr int NQP = NT * 8;
-  constexpr int CPR = D / 8;          // 16-byte chunks per K / V row
-  constexpr int TILE = kSrTS * D * 2;
-  constexpr int STAGE = 2 * TILE;
 
-  extern __shared__ __align__(1024) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t mbar_s[kSrMaxStages], mbar_a[kSrMaxStages];
   __shared__ int hist[2][256];
   __shared__ int scan_scratch[33];
   __shared__ float qt[128];
   __shared__ int s_bin, s_above, s_eq_before, s_sel_before;
   __shared__ int s_gt[kSrMaxCluster], s_eq[kSrMaxCluster], s_eq_all;
+  __shared__ int s_gt24[8];  // per warp: this CTA's keys whose first 24 bits exceed the prefix
 
   AOH_PHASE(0);
   cgs::cluster_group cluster = cgs::this_cluster();
@@ -160,6 +164,12 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
     return;
   }
 
+  if (tid < kSrMaxCluster) {
+    s_gt[tid] = 0;
+    s_eq[tid] = 0;
+  }
+  // swizzled tensor loads need 1024-byte aligned slots: the host adds 1 KB of slack
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int slice = (((L + CL - 1) / CL) + 3) & ~3;
   const int lo = min(L, rk * slice), hi = min(L, lo + slice);
   const int m = hi - lo;
@@ -219,35 +229,43 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
           bt[ks][1] = pack_bf16x2(v[2], v[3]);
         }
       }
-      const int rb_shift = 31 - __clz(p.srow_len * 2);   // row bytes = 2^rb_shift
-      const int cpr = (p.srow_len * 2) >> 4;              // 16-byte chunks per row
-      const int tr = kSrRingStage >> rb_shift;            // rows per stage
-      const int nst = (m + tr - 1) / tr;
-      const uint16_t* base = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)(off + lo) * p.srow_stride_tok;
-      const uint32_t rbase = smem_u32(smem + p.keys_bytes);
+      // ring of tensor-map tiles: one elected thread issues halves x (box x rows) per stage
+      const int box = p.scan_box, rows = p.scan_rows;
+      const int halves = p.srow_len / box;
+      const int span_shift = 31 - __clz(box * 2);        // box row bytes = 2^span_shift
+      const int stage_bytes = halves * rows * (box * 2);
+      const int nst = (m + rows - 1) / rows;
       const int ns = min(kSrMaxStages, p.ring_bytes / kSrRingStage);
-      auto issue = [&](int st) {
-        if (st < nst) {
-          const uint32_t sb = rbase + (st % ns) * kSrRingStage;
-#pragma unroll
-          for (int i = 0; i < kSrRingStage / 16 / kSrThreads; ++i) {
-            const int c = tid + i * kSrThreads;
-            const int r = c / cpr, ch = c - r * cpr;
-            const int row = st * tr + r;
-            const bool ok = row < m;
-            cp_async_16(sb + tip_ring_off(r, ch, rb_shift), base + (int64_t)(ok ? row : 0) * p.srow_stride_tok + ch * 8, ok);
-          }
-        }
-        cp_async_commit();
-      };
-      for (int s0 = 0; s0 < ns - 1; ++s0) issue(s0);
-      for (int st = 0; st < nst; ++st) {
-        cp_async_wait_n(ns - 2);
-        __syncthreads();
-        issue(st + ns - 1);
+      const uint32_t rbase = smem_u32(smem + p.keys_bytes);
+      const int y0 = (p.packed ? g * p.T : 0) + off + lo;
+      const int x0 = p.packed ? 0 : g * (int)p.srow_stride_head;
+      if (tid == 0) {
+        for (int i = 0; i < ns; ++i) mbar_init(smem_u32(&mbar_s[i]), 1);
+        fence_mbar_init();
+        fence_proxy_async();
+      }
+      __syncthreads();
+      auto issue = [&](int st) {  // called by thread 0 only
+        const uint32_t bar = smem_u32(&mbar_s[st % ns]);
         const uint32_t sb = rbase + (st % ns) * kSrRingStage;
-        for (int tile = warp; tile * 16 < tr; tile += 8) {
-          const int nv = m - (st * tr + tile * 16);
+        mbar_expect_tx(bar, stage_bytes);
+        for (int h2 = 0; h2 < halves; ++h2)
+          tma_tile_2d(sb + h2 * rows * (box * 2), &p.tmap_scan, x0 + h2 * box, y0 + st * rows, bar);
+      };
+      if (tid == 0)
+        for (int s0 = 0; s0 < min(ns, nst); ++s0) issue(s0);
+      bool failed = false;
+      int st = 0;
+      for (; st < nst; ++st) {
+        const bool ok = mbar_wait(smem_u32(&mbar_s[st % ns]), (uint32_t)((st / ns) & 1));
+        if (__syncthreads_or(!ok)) {
+          if (tid == 0) record_error(kCheckTimeout, b, g, st);
+          failed = true;
+          break;
+        }
+        const uint32_t sb = rbase + (st % ns) * kSrRingStage;
+        for (int tile = warp; tile * 16 < rows; tile += 8) {
+          const int nv = m - (st * rows + tile * 16);
           if (nv <= 0) break;
           float c4[4] = {0.f, 0.f, 0.f, 0.f};
           const int r = tile * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -255,91 +273,121 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
           for (int ks = 0; ks < 8; ++ks) {
             if (ks < ksteps) {
               uint32_t a[4];
-              ldsm_x4(a, sb + tip_ring_off(r, 2 * ks + (lane >> 4), rb_shift));
+              ldsm_x4(a, sb + scan_tile_off(r, 2 * ks + (lane >> 4), span_shift, rows));
               mma_16816(c4, a, bt[ks][0], bt[ks][1]);
             }
           }
           if ((lane & 3) == 0) {
             const int ri = lane >> 2;  // row within the 16-row tile; nv counts from the tile start
-            const int r0 = st * tr + tile * 16 + ri;
+            const int r0 = st * rows + tile * 16 + ri;
             if (ri < nv) keys[r0] = score_key(c4[0] + c4[1]);
             if (ri + 8 < nv) keys[r0 + 8] = score_key(c4[2] + c4[3]);
           }
         }
+        __syncthreads();  // the slot is free: refill it
+        if (tid == 0 && st + ns < nst) issue(st + ns);
       }
-      cp_async_wait<0>();
+      if (failed && tid == 0) {  // drain the copies still in flight (bounded) before reuse
+        for (int s2 = st; s2 < min(nst, st + ns); ++s2) mbar_wait(smem_u32(&mbar_s[s2 % ns]), (uint32_t)((s2 / ns) & 1));
+      }
       __syncthreads();
     }
 
     AOH_PHASE(1);
     // =============================================================== 2. select
-    // Every CTA also learns, from the histograms it reads anyway, how many keys of
-    // each peer are above the threshold (s_gt) and equal to it (s_eq), so the
-    // compaction needs no further exchange.
-    if (tid < kSrMaxCluster) {
-      s_gt[tid] = 0;
-      s_eq[tid] = 0;
-    }
+    // One cluster barrier and two block barriers per digit.  In the last digit every
+    // CTA also derives, from the histograms it reads anyway, how many keys of each
+    // peer lie above the threshold (s_gt) and equal it (s_eq): the compaction then
+    // needs no further exchange.
     uint32_t prefix = 0u, pmask = 0u;
     int krem = n;
+    hist[0][tid] = 0;
+    if (tid < 8) s_gt24[tid] = 0;
+    __syncthreads();
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       int* h = hist[pass & 1];
-      h[tid] = 0;
-      __syncthreads();
-      // four keys per lane and iteration (warp-uniform trip count); the first digit
-      // (sign + exponent) is shared by most keys, so it is counted with warp
-      // aggregation, the later digits directly
+      // count (four keys per lane, warp-uniform trip count); the first digit (sign and
+      // exponent) is shared by most keys, so it is counted with warp aggregation.  In the
+      // last digit, keys whose first 24 bits exceed the prefix are counted too.
+      int above24 = 0;
       for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
-        const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: the keys region covers it
+        const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the keys region
         const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
         const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const bool in = (i0 + j < m) && ((kk[j] & pmask) == prefix);
+          const bool valid = i0 + j < m;
+          const bool in = valid && ((kk[j] & pmask) == prefix);
           const int bin = in ? (int)((kk[j] >> shift) & 255u) : -1;
           if (pass == 0) {
             hist_add(h, bin);
           } else if (in) {
             atomicAdd(&h[bin], 1);
           }
+          if (pass == 3) above24 += valid && ((kk[j] & pmask) > prefix);
         }
       }
+      if (pass == 3) {
+        above24 = __reduce_add_sync(0xffffffffu, above24);
+        if (lane == 0) s_gt24[warp] = above24;
+      }
       cluster.sync();
-      const int bin = 255 - tid;  // scanned from the top bin down
+      int* hn = hist[(pass + 1) & 1];  // peers finished reading it before this barrier
+      hn[tid] = 0;
+      const int bin = 255 - tid;       // scanned from the top bin down
       int v[kSrMaxCluster];
 #pragma unroll
       for (int q = 0; q < kSrMaxCluster; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
       int tot = 0;
 #pragma unroll
       for (int q = 0; q < kSrMaxCluster; ++q) tot += v[q];
-      int total;
-      const int above = block_exclusive_scan(tot, scan_scratch, &total);
+      // exclusive prefix over tid (bins from the top): warp scan, then the warp totals
+      int x = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) scan_scratch[warp] = x;
+      __syncthreads();
+      int above = x - tot;
+      for (int w2 = 0; w2 < warp; ++w2) above += scan_scratch[w2];
       if (above < krem && krem <= above + tot) {
         s_bin = bin;
         s_above = above;
       }
       __syncthreads();
       const int sb = s_bin;
-      // keys of every peer in bins above the chosen one are above the threshold
+      if (pass == 3) {
+        // peers' keys above the threshold: first 24 bits above the prefix, or equal
+        // there and in a higher last digit; equal to it: the chosen bin
 #pragma unroll
-      for (int q = 0; q < kSrMaxCluster; ++q) {
-        if (q < CL) {
-          const int w = __reduce_add_sync(0xffffffffu, bin > sb ? v[q] : 0);
-          if (lane == 0 && w) atomicAdd(&s_gt[q], w);
+        for (int q = 0; q < kSrMaxCluster; ++q) {
+          if (q < CL) {
+            const int w = __reduce_add_sync(0xffffffffu, bin > sb ? v[q] : 0);
+            if (lane == 0 && w) atomicAdd(&s_gt[q], w);
+          }
         }
-      }
-      if (pass == 3 && bin == sb) {
+        if (bin == sb) {
 #pragma unroll
-        for (int q = 0; q < kSrMaxCluster; ++q)
-          if (q < CL) s_eq[q] = v[q];
+          for (int q = 0; q < kSrMaxCluster; ++q)
+            if (q < CL) s_eq[q] = v[q];
+        }
+        if (tid < CL) {
+          const int* g24 = cluster.map_shared_rank(s_gt24, tid);
+          int t = 0;
+#pragma unroll
+          for (int w2 = 0; w2 < 8; ++w2) t += g24[w2];
+          atomicAdd(&s_gt[tid], t);
+        }
       }
       prefix |= (uint32_t)sb << shift;
       pmask |= 255u << shift;
       krem -= s_above;
-      __syncthreads();
     }
+    __syncthreads();
     const uint32_t KT = prefix;
     const int need_eq = krem;
     AOH_PHASE(2);
@@ -443,32 +491,39 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
   const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
   const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
   const int nstages = (nloc + kSrTS - 1) / kSrTS;
-  const int nsa = min(kSrMaxStages, p.ring_bytes / STAGE);
-  auto issue = [&](int st) {
-    if (st < nstages) {
-      const uint32_t kt = sbase + (st % nsa) * STAGE;
-      const uint32_t vt = kt + TILE;
-#pragma unroll
-      for (int c = tid; c < kSrTS * CPR; c += kSrThreads) {
-        const int r = c / CPR, ch = c % CPR;
-        const int jj = st * kSrTS + r;
-        const bool ok = jj < nloc;
-        const int pos = ok ? plist[jj] : 0;
-        const int64_t eo = (int64_t)pos * p.stride_tok + ch * 8;
-        const uint32_t so = sr_tile_off(r, ch * 8);
-        cp_async_16(kt + so, kbase + eo, ok);
-        cp_async_16(vt + so, vbase + eo, ok);
-      }
-    }
-    cp_async_commit();
+  const int nsa = min(kSrMaxStages, p.ring_bytes / AttTile<D>::kStage);
+  if (tid == 0) {
+    for (int i = 0; i < nsa; ++i) mbar_init(smem_u32(&mbar_a[i]), 1);
+    fence_mbar_init();
+    fence_proxy_async();
+  }
+  __syncthreads();
+  // warp 0 issues a stage: lane j copies the K and V rows of entry j (entries past the
+  // list repeat its first position, so every row of a tile holds finite data)
+  auto issue_att = [&](int st) {
+    const uint32_t bar = smem_u32(&mbar_a[st % nsa]);
+    const uint32_t kt = sbase + (st % nsa) * AttTile<D>::kStage;
+    const uint32_t vt = kt + AttTile<D>::kTile;
+    if (lane == 0) mbar_expect_tx(bar, kSrTS * 4 * D);
+    __syncwarp();
+    const int jj = st * kSrTS + lane;
+    const int pos = plist[jj < nloc ? jj : 0];
+    bulk_g2s(kt + lane * AttTile<D>::kPitch, kbase + (int64_t)pos * p.stride_tok, 2 * D, bar);
+    bulk_g2s(vt + lane * AttTile<D>::kPitch, vbase + (int64_t)pos * p.stride_tok, 2 * D, bar);
   };
-  for (int s = 0; s < nsa - 1; ++s) issue(s);
-  for (int st = 0; st < nstages; ++st) {
-    cp_async_wait_n(nsa - 2);
-    __syncthreads();
-    issue(st + nsa - 1);
-    const uint32_t kt = sbase + (st % nsa) * STAGE;
-    const uint32_t vt = kt + TILE;
+  if (warp == 0)
+    for (int s0 = 0; s0 < min(nsa, nstages); ++s0) issue_att(s0);
+  int st = 0;
+  bool att_failed = false;
+  for (; st < nstages; ++st) {
+    const bool ok = mbar_wait(smem_u32(&mbar_a[st % nsa]), (uint32_t)((st / nsa) & 1));
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) record_error(kCheckTimeout, b, g, 1000000 + st);
+      att_failed = true;
+      break;
+    }
+    const uint32_t kt = sbase + (st % nsa) * AttTile<D>::kStage;
+    const uint32_t vt = kt + AttTile<D>::kTile;
 #pragma unroll
     for (int u = 0; u < SUB; ++u) {
       if ((st * SUB + u) % WT != tg) continue;
@@ -481,7 +536,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t a[4];
-          ldsm_x4(a, kt + sr_tile_off(r, ks * 16 + dsel));
+          ldsm_x4(a, kt + r * AttTile<D>::kPitch + (ks * 16 + dsel) * 2);
           mma_16816(s4, a, bq[ks][0], bq[ks][1]);
         }
       }
@@ -522,14 +577,18 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const RowParams 
 #pragma unroll
         for (int mt = 0; mt < KH; ++mt) {
           uint32_t a[4];
-          ldsm_x4_trans(a, vt + sr_tile_off(r, (half * KH + mt) * 16 + dsel));
+          ldsm_x4_trans(a, vt + r * AttTile<D>::kPitch + ((half * KH + mt) * 16 + dsel) * 2);
           mma_16816(acc[mt], a, pb0, pb1);
           mma_16816(acc[mt], a, pl0, pl1);
         }
       }
     }
+    __syncthreads();  // the slot is free: refill it
+    if (warp == 0 && st + nsa < nstages) issue_att(st + nsa);
   }
-  cp_async_wait<0>();
+  if (att_failed && tid == 0) {  // drain the copies still in flight (bounded)
+    for (int s2 = st; s2 < min(nstages, st + nsa); ++s2) mbar_wait(smem_u32(&mbar_a[s2 % nsa]), (uint32_t)((s2 / nsa) & 1));
+  }
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
