@@ -93,7 +93,7 @@ __device__ __forceinline__ uint32_t scan_tile_off(int r, int c, int span_shift, 
 
 #ifdef AOH_PHASE_TIMERS
 // Diagnostic build only: global-timer stamps at the phase boundaries of every CTA.
-constexpr int kPhaseSlots = 8;
+constexpr int kPhaseSlots = 16;
 constexpr int kPhaseCtas = 8192;
 __device__ long long g_phase_ns[kPhaseCtas][kPhaseSlots];
 __device__ __forceinline__ void phase_stamp(int slot) {
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   constexpr int NQP = NT * 8;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t mbar_s[kSrMaxStages], mbar_a[kSrMaxStages];
+  __shared__ __align__(8) uint64_t mbar_s[kSrMaxStages];
   __shared__ int hist[2][256];
   __shared__ int scan_scratch[33];
   __shared__ float qt[128];
@@ -179,6 +179,32 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 
   if (n < L) {
     // =============================================================== 1. scan
+    {
+      // ring of tensor-map tiles: one elected thread issues halves x (box x rows) per stage
+      const int box = p.scan_box, rows = p.scan_rows;
+      const int halves = p.srow_len / box;
+      const int span_shift = 31 - __clz(box * 2);        // box row bytes = 2^span_shift
+      const int stage_bytes = halves * rows * (box * 2);
+      const int nst = (m + rows - 1) / rows;
+      const int ns = min(kSrMaxStages, p.ring_bytes / kSrRingStage);
+      const uint32_t rbase = smem_u32(smem + p.keys_bytes);
+      const int y0 = (p.packed ? g * p.T : 0) + off + lo;
+      const int x0 = p.packed ? 0 : g * (int)p.srow_stride_head;
+      if (tid == 0) {
+        for (int i = 0; i < ns; ++i) mbar_init(smem_u32(&mbar_s[i]), 1);
+        fence_mbar_init();
+        fence_proxy_async();
+      }
+      __syncthreads();
+      auto issue = [&](int st) {  // called by thread 0 only
+        const uint32_t bar = smem_u32(&mbar_s[st % ns]);
+        const uint32_t sb = rbase + (st % ns) * kSrRingStage;
+        mbar_expect_tx(bar, stage_bytes);
+        for (int h2 = 0; h2 < halves; ++h2)
+          tma_tile_2d(sb + h2 * rows * (box * 2), &p.tmap_scan, x0 + h2 * box, y0 + st * rows, bar);
+      };
+      if (tid == 0)
+        for (int s0 = 0; s0 < min(ns, nst); ++s0) issue(s0);
     if (tid < p.srow_len) {
       const int C = D / 2;
       int dim = -1;
@@ -205,7 +231,14 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       float acc = 0.f;
       if (dim >= 0) {
         const uint16_t* qb = p.q_score + ((int64_t)b * p.Hq + (int64_t)g * p.G) * D + dim;
-        for (int h = 0; h < p.G; ++h) acc += __uint_as_float((uint32_t)qb[(int64_t)h * D] << 16);
+        for (int h0 = 0; h0 < p.G; h0 += 8) {  // eight loads in flight, summed in head order
+          float qv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            qv[u] = (h0 + u < p.G) ? __uint_as_float((uint32_t)qb[(int64_t)(h0 + u) * D] << 16) : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc += qv[u];
+        }
       }
       qt[tid] = acc;
     }
@@ -229,31 +262,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
           bt[ks][1] = pack_bf16x2(v[2], v[3]);
         }
       }
-      // ring of tensor-map tiles: one elected thread issues halves x (box x rows) per stage
-      const int box = p.scan_box, rows = p.scan_rows;
-      const int halves = p.srow_len / box;
-      const int span_shift = 31 - __clz(box * 2);        // box row bytes = 2^span_shift
-      const int stage_bytes = halves * rows * (box * 2);
-      const int nst = (m + rows - 1) / rows;
-      const int ns = min(kSrMaxStages, p.ring_bytes / kSrRingStage);
-      const uint32_t rbase = smem_u32(smem + p.keys_bytes);
-      const int y0 = (p.packed ? g * p.T : 0) + off + lo;
-      const int x0 = p.packed ? 0 : g * (int)p.srow_stride_head;
-      if (tid == 0) {
-        for (int i = 0; i < ns; ++i) mbar_init(smem_u32(&mbar_s[i]), 1);
-        fence_mbar_init();
-        fence_proxy_async();
-      }
-      __syncthreads();
-      auto issue = [&](int st) {  // called by thread 0 only
-        const uint32_t bar = smem_u32(&mbar_s[st % ns]);
-        const uint32_t sb = rbase + (st % ns) * kSrRingStage;
-        mbar_expect_tx(bar, stage_bytes);
-        for (int h2 = 0; h2 < halves; ++h2)
-          tma_tile_2d(sb + h2 * rows * (box * 2), &p.tmap_scan, x0 + h2 * box, y0 + st * rows, bar);
-      };
-      if (tid == 0)
-        for (int s0 = 0; s0 < min(ns, nst); ++s0) issue(s0);
       bool failed = false;
       int st = 0;
       for (; st < nst; ++st) {
@@ -292,7 +300,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       }
       __syncthreads();
     }
-
+    }
     AOH_PHASE(1);
     // =============================================================== 2. select
     // One cluster barrier and two block barriers per digit.  In the last digit every
@@ -308,6 +316,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       int* h = hist[pass & 1];
+      if (pass == 1) AOH_PHASE(12);
       // count (four keys per lane, warp-uniform trip count); the first digit (sign and
       // exponent) is shared by most keys, so it is counted with warp aggregation.  In the
       // last digit, keys whose first 24 bits exceed the prefix are counted too.
@@ -333,7 +342,9 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
         above24 = __reduce_add_sync(0xffffffffu, above24);
         if (lane == 0) s_gt24[warp] = above24;
       }
+      if (pass == 1) AOH_PHASE(8);
       cluster.sync();
+      if (pass == 1) AOH_PHASE(9);
       int* hn = hist[(pass + 1) & 1];  // peers finished reading it before this barrier
       hn[tid] = 0;
       const int bin = 255 - tid;       // scanned from the top bin down
@@ -343,6 +354,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       int tot = 0;
 #pragma unroll
       for (int q = 0; q < kSrMaxCluster; ++q) tot += v[q];
+      if (pass == 1) AOH_PHASE(10);
       // exclusive prefix over tid (bins from the top): warp scan, then the warp totals
       int x = tot;
 #pragma unroll
@@ -360,6 +372,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       }
       __syncthreads();
       const int sb = s_bin;
+      if (pass == 1) AOH_PHASE(11);
       if (pass == 3) {
         // peers' keys above the threshold: first 24 bits above the prefix, or equal
         // there and in a higher last digit; equal to it: the chosen bin
@@ -465,6 +478,38 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   // =============================================================== 3. attend
   const int half = warp >> 2, r4 = warp & 3;
   const int nt = r4 % NT, tg = r4 / NT;
+  float acc[KH][4];
+#pragma unroll
+  for (int i = 0; i < KH; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  uint8_t* stage_mem = smem + p.keys_bytes;
+  const uint32_t sbase = smem_u32(stage_mem);
+  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const int nstages = (nloc + kSrTS - 1) / kSrTS;
+  const int nsa = min(kSrMaxStages, p.ring_bytes / AttTile<D>::kStage);
+  // every thread copies 16-byte chunks of the stage's K and V rows (cp.async); entries past
+  // the list repeat its first position, so every row of a tile holds finite data
+  auto issue_att = [&](int st) {
+    if (st < nstages) {
+      const uint32_t kt = sbase + (st % nsa) * AttTile<D>::kStage;
+      const uint32_t vt = kt + AttTile<D>::kTile;
+      constexpr int CPR = D / 8;
+#pragma unroll
+      for (int c = tid; c < kSrTS * CPR; c += kSrThreads) {
+        const int r = c / CPR, ch = c % CPR;
+        const int jj = st * kSrTS + r;
+        const int pos = plist[jj < nloc ? jj : 0];
+        const int64_t eo = (int64_t)pos * p.stride_tok + ch * 8;
+        const uint32_t so = r * AttTile<D>::kPitch + ch * 16;
+        cp_async_16(kt + so, kbase + eo, true);
+        cp_async_16(vt + so, vbase + eo, true);
+      }
+    }
+    cp_async_commit();
+  };
+  for (int s0 = 0; s0 < nsa - 1; ++s0) issue_att(s0);
   uint32_t bq[KS][2];
   {
     const int qr = nt * 8 + (lane >> 2);
@@ -481,47 +526,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       for (int ks = 0; ks < KS; ++ks) bq[ks][0] = bq[ks][1] = 0u;
     }
   }
-  float acc[KH][4];
-#pragma unroll
-  for (int i = 0; i < KH; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-  uint8_t* stage_mem = smem + p.keys_bytes;
-  const uint32_t sbase = smem_u32(stage_mem);
-  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
-  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
-  const int nstages = (nloc + kSrTS - 1) / kSrTS;
-  const int nsa = min(kSrMaxStages, p.ring_bytes / AttTile<D>::kStage);
-  if (tid == 0) {
-    for (int i = 0; i < nsa; ++i) mbar_init(smem_u32(&mbar_a[i]), 1);
-    fence_mbar_init();
-    fence_proxy_async();
-  }
-  __syncthreads();
-  // warp 0 issues a stage: lane j copies the K and V rows of entry j (entries past the
-  // list repeat its first position, so every row of a tile holds finite data)
-  auto issue_att = [&](int st) {
-    const uint32_t bar = smem_u32(&mbar_a[st % nsa]);
-    const uint32_t kt = sbase + (st % nsa) * AttTile<D>::kStage;
-    const uint32_t vt = kt + AttTile<D>::kTile;
-    if (lane == 0) mbar_expect_tx(bar, kSrTS * 4 * D);
-    __syncwarp();
-    const int jj = st * kSrTS + lane;
-    const int pos = plist[jj < nloc ? jj : 0];
-    bulk_g2s(kt + lane * AttTile<D>::kPitch, kbase + (int64_t)pos * p.stride_tok, 2 * D, bar);
-    bulk_g2s(vt + lane * AttTile<D>::kPitch, vbase + (int64_t)pos * p.stride_tok, 2 * D, bar);
-  };
-  if (warp == 0)
-    for (int s0 = 0; s0 < min(nsa, nstages); ++s0) issue_att(s0);
-  int st = 0;
-  bool att_failed = false;
-  for (; st < nstages; ++st) {
-    const bool ok = mbar_wait(smem_u32(&mbar_a[st % nsa]), (uint32_t)((st / nsa) & 1));
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) record_error(kCheckTimeout, b, g, 1000000 + st);
-      att_failed = true;
-      break;
-    }
+  for (int st = 0; st < nstages; ++st) {
+    cp_async_wait_n(nsa - 2);
+    __syncthreads();
+    issue_att(st + nsa - 1);
     const uint32_t kt = sbase + (st % nsa) * AttTile<D>::kStage;
     const uint32_t vt = kt + AttTile<D>::kTile;
 #pragma unroll
@@ -583,12 +591,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
         }
       }
     }
-    __syncthreads();  // the slot is free: refill it
-    if (warp == 0 && st + nsa < nstages) issue_att(st + nsa);
   }
-  if (att_failed && tid == 0) {  // drain the copies still in flight (bounded)
-    for (int s2 = st; s2 < min(nstages, st + nsa); ++s2) mbar_wait(smem_u32(&mbar_a[s2 % nsa]), (uint32_t)((s2 / nsa) & 1));
-  }
+  cp_async_wait<0>();
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
