@@ -219,6 +219,30 @@ size_t aoh_stream_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_head
                                         const uint8_t* roles, int32_t sink, int32_t window);
 
 /*
+ * aoh_stream_decode_noalloc -- aoh_stream_decode without a caller workspace.  The
+ * pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory: code that runs inside someone else's pre-reserved
+ * memory pool or a plugin host that owns every device allocation, and
+ * latency-critical paths where a cudaMalloc, with the device-wide
+ * synchronisation it may imply, is not acceptable.
+ *
+ * The split-K scratch lives in a file-scope device array of 16 MiB that every
+ * device which loads the library keeps until the process exits; the call
+ * allocates nothing.  Arguments and results are those of aoh_stream_decode.
+ *   - Returns AOH_ERR_WORKSPACE, without launching, when the step needs more
+ *     than 16 MiB of scratch (aoh_stream_decode_workspace_size gives the need).
+ *   - The first call on a device sets the array up (looks up its address with
+ *     that device current, zeroes it and synchronises the device), so make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; calls that can overlap on the GPU (different streams without
+ *     ordering) race on it.  Serialise them on one stream.
+ */
+aoh_status aoh_stream_decode_noalloc(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
+                                     const uint8_t* roles, int32_t sink, int32_t window,
+                                     float scale, float* out, void* stream);
+
+/*
  * aoh_shared_index_decode -- the cross-decoder layers of a shared-cache
  * stack reuse one index ("Como funciona CLSA"): for every layer l, every
  * q head h of group g and sequence b,

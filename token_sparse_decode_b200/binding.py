@@ -25,7 +25,7 @@ EXPORTS = (
     "aoh_status_string", "aoh_version", "aoh_last_cuda_error", "aoh_device_check", "aoh_pack_dominant", "aoh_tip_score",
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
-    "aoh_shared_index_step",
+    "aoh_shared_index_step", "aoh_stream_decode_noalloc",
 )
 
 
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "aoh_shared_index_decode": (ctypes.c_int, [P, I32, I32, KVP, P, P, I32, F32, P, P, SZ, P]),
             "aoh_shared_index_decode_workspace_size": (SZ, [KVP, I32, I32, I32]),
             "aoh_shared_index_step": (ctypes.c_int, [P, P, I32, I32, KVP, I32, P, P, F32, P, P]),
+            "aoh_stream_decode_noalloc": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -211,3 +212,12 @@ def shared_index_step(q_index: torch.Tensor, q_layers: torch.Tensor, kv: KVCache
     _check("aoh_shared_index_step", lib().aoh_shared_index_step(
         _ptr(q_index), _ptr(q_layers), q_layers.shape[0], q_layers.shape[-2], ctypes.byref(kv), topk, _ptr(idx),
         _ptr(count), float(scale), _ptr(out), _stream(stream)))
+
+
+def stream_decode_noalloc(q: torch.Tensor, kv: KVCache, roles, sink: int, window: int, scale: float,
+                          out: torch.Tensor, stream=None) -> None:
+    """aoh_stream_decode with the library's own static scratch (no workspace argument)."""
+    r = _host_u8(roles)
+    _check("aoh_stream_decode_noalloc", lib().aoh_stream_decode_noalloc(
+        _ptr(q), q.shape[-2], ctypes.byref(kv), ctypes.cast(r, ctypes.c_void_p), sink, window, float(scale),
+        _ptr(out), _stream(stream)))

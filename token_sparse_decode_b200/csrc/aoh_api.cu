@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "aoh.h"
 #include "device_common.cuh"
@@ -824,3 +825,52 @@ int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
 #endif
 
 }  // extern "C"
+
+// ===================================================================== no-allocation variant
+// Scratch for aoh_stream_decode_noalloc: a file-scope device array, so the call needs no
+// allocation.  Every device that loads the library holds it until the process exits.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_addr[256];  // device address of the array, per device ordinal (host-side)
+
+// The array's device address on the current device.  First use on a device: look the
+// address up with that device current and zero the array (the split counters at its head
+// must start at zero; every later call leaves them at zero).  This set-up synchronises
+// the device, so the first call on a device must not happen during a stream capture.
+aoh_status static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AOH_ERR_CUDA;
+  if (dev < 0 || dev >= 256) return AOH_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* ptr = nullptr;
+    aoh_status s = cuda_status(cudaGetSymbolAddress(&ptr, g_static_scratch));
+    if (s != AOH_OK) return s;
+    if ((s = cuda_status(cudaMemset(ptr, 0, kStaticScratchBytes))) != AOH_OK) return s;
+    if ((s = cuda_status(cudaDeviceSynchronize())) != AOH_OK) return s;
+    g_static_addr[dev] = ptr;
+  }
+  *out = g_static_addr[dev];
+  return AOH_OK;
+}
+}  // namespace
+
+extern "C" aoh_status aoh_stream_decode_noalloc(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
+                                                const uint8_t* roles, int32_t sink, int32_t window, float scale,
+                                                float* out, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if (!roles) return AOH_ERR_INVALID_ARG;
+  if ((s = check_roles(kv, roles)) != AOH_OK) return s;
+  if (n_q_heads / kv->n_kv_heads > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (sink < 0 || window < 0 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  if (kv->batch == 0) return AOH_OK;
+  if (fd_bytes(stream_geom(kv, n_q_heads, roles, sink, window)) > kStaticScratchBytes) return AOH_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != AOH_OK) return s;
+  return aoh_stream_decode(q, n_q_heads, kv, roles, sink, window, scale, out, scratch, kStaticScratchBytes, stream);
+}
