@@ -248,14 +248,33 @@ def capture_graph(fn):
     return g
 
 
+def shard_spec(spec, rank: int, world: int):
+    """Rank `rank`'s batch: the same shape with its own seed (independent sequences, weak scaling)."""
+    if world <= 1:
+        return spec
+    from dataclasses import replace
+
+    return replace(spec, seed=spec.seed + 1000 * rank)
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum of per-rank timings (identity on one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate_throughput(tokens_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank scans its own batch in the (max-over-ranks) step time."""
+    return tokens_per_rank_step * world / (ms_per_step * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    spec = preset(args.workload)
-    if world > 1:  # each rank decodes its own independent batch of sequences
-        from dataclasses import replace
-
-        spec = replace(spec, seed=spec.seed + 1000 * rank)
+    spec = shard_spec(preset(args.workload), rank, world)
     w = make_workload(spec)
     step, q = build_step(w, dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -330,15 +349,12 @@ def run_ours(args, rank, world, local_rank):
 
     stages = stage_timing(w, step, q, args.steps if args.steps <= 200 else 200, flush)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
     tokens_step = int(w.lengths.sum())
     ms_step = ms / args.steps
-    value = tokens_step * world / (ms_step * 1e-3)
-    e2e_value = tokens_step * world / (e2e_ms / args.steps * 1e-3)
+    value = aggregate_throughput(tokens_step, world, ms_step)
+    e2e_value = aggregate_throughput(tokens_step, world, e2e_ms / args.steps)
     ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_gbs()
     call_bytes = {"shared_index_step": ab["indexer"] + ab["gather"], "sparse_decode": ab["tip"] + ab["fac"],
