@@ -268,24 +268,29 @@ size_t aoh_shared_index_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_
                                               int32_t n_q_heads, int32_t n_fac_cap);
 
 /*
- * aoh_shared_index_step -- the whole shared-index stack step in one launch
- * ("Como funciona CLSA": the indexer scores the cache once, takes one top-k
- * and every cross-decoder layer attends over it).  Equivalent to
- * aoh_tip_score (every chunk, q_index) + aoh_topk_select (k = topk) +
- * aoh_shared_index_decode, without the score buffer or workspace: each
- * (sequence, KV head) row runs in one thread-block cluster.
+ * aoh_shared_index_step -- the whole shared-index stack step ("Como funciona
+ * CLSA": the indexer scores the cache once, takes one top-k and every
+ * cross-decoder layer attends over it).  Equivalent to aoh_tip_score (every
+ * chunk, q_index) + aoh_topk_select (k = topk) + aoh_shared_index_decode.
+ * When every (sequence, KV head) row fits one wave of thread-block clusters
+ * the step is a single launch (scan, select, attention and combine per
+ * cluster); otherwise it runs the scan over all SMs, the cluster select and
+ * the split-K gather.
  *   q_index    device bf16 [B][n_q_heads][d]: the indexer layer's queries
  *   q_layers   device bf16 [n_layers][B][n_q_heads][d]
  *   n_layers * (n_q_heads / n_kv_heads) <= 32
  *   idx, count device outputs, layouts of aoh_topk_select with n_fac_cap = topk
  *   out        device fp32 [n_layers][B][n_q_heads][d]
- * Returns AOH_ERR_UNSUPPORTED when a row is too long for one cluster
- * (max_len above 262144); the three-call form has no such limit.
+ *   workspace  device, 256-byte aligned, zero-filled once before first use,
+ *              >= aoh_shared_index_step_workspace_size bytes
  */
 aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int32_t n_layers,
                                  int32_t n_q_heads, const aoh_kv_cache* kv, int32_t topk,
                                  int32_t* idx, int32_t* count, float scale, float* out,
-                                 void* stream);
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+size_t aoh_shared_index_step_workspace_size(const aoh_kv_cache* kv, int32_t n_layers,
+                                            int32_t n_q_heads, int32_t topk);
 
 #ifdef __cplusplus
 }

@@ -313,3 +313,45 @@ def test_sparse_decode_every_token_selected():
         for g in range(sp.n_kv_heads):
             assert step.count[b, g].item() == w.lengths[b]
             compare_window_row(w, b, g, out_h[b, g * G:(g + 1) * G], ROLE_DENSE, 0, 0)
+
+
+def test_sparse_decode_many_rows_runs_three_stages():
+    # 40 sequences x 8 KV heads = 320 rows: more clusters than one wave holds, so the step
+    # runs as scan kernel + cluster select on the scores + split-K gather
+    sp = spec(batch=40, len_range=(300, 3000), seed=87)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_sparse(d)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = sp.group
+    stats = {}
+    for b in range(0, sp.batch, 3):
+        for g in range(sp.n_kv_heads):
+            compare_sparse_row(w, b, g, idx_h[b, g, :cnt_h[b, g]], out_h[b, g * G:(g + 1) * G], stats)
+    assert stats["swapped"] <= max(1, stats["rows"] // 10)
+
+
+def test_shared_index_step_many_rows_runs_three_stages():
+    sp = WorkloadSpec(name="shared_many", batch=24, n_q_heads=32, n_kv_heads=8, head_dim=128, theta=5e5,
+                      len_range=(500, 9000), n_layers=2, topk_shared=300, seed=88)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_shared(d, fused=True)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = sp.group
+    rows = [(b, g) for b in range(0, 24, 5) for g in range(8)]
+    ref = oracle.shared_index_step(f64(w.q), f64(w.q_layers), f64(w.k), f64(w.v), w.offsets.tolist(), 300, w.scale,
+                                   rows=rows)
+    for (b, g), r in ref.items():
+        sel = idx_h[b, g, :cnt_h[b, g]]
+        ok, msg = oracle.tie_band_check(sel, r["scores"], min(300, int(w.lengths[b])))
+        assert ok, msg
+        tol = OUT_ATOL
+        if not np.array_equal(sel, r["sel"]):
+            qg, keys, values = row_inputs(w, b, g)
+            for l in range(2):
+                tol = max(tol, OUT_ATOL + band_swap_bound(f64(w.q_layers[l, b, g * G:(g + 1) * G]), keys, values,
+                                                          r["scores"], len(sel), w.scale))
+        assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= tol

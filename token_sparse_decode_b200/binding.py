@@ -25,7 +25,7 @@ EXPORTS = (
     "aoh_status_string", "aoh_version", "aoh_last_cuda_error", "aoh_device_check", "aoh_pack_dominant", "aoh_tip_score",
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
-    "aoh_shared_index_step", "aoh_stream_decode_noalloc",
+    "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
 )
 
 
@@ -74,7 +74,8 @@ def lib() -> ctypes.CDLL:
             "aoh_stream_decode_workspace_size": (SZ, [KVP, I32, P, I32, I32]),
             "aoh_shared_index_decode": (ctypes.c_int, [P, I32, I32, KVP, P, P, I32, F32, P, P, SZ, P]),
             "aoh_shared_index_decode_workspace_size": (SZ, [KVP, I32, I32, I32]),
-            "aoh_shared_index_step": (ctypes.c_int, [P, P, I32, I32, KVP, I32, P, P, F32, P, P]),
+            "aoh_shared_index_step": (ctypes.c_int, [P, P, I32, I32, KVP, I32, P, P, F32, P, P, SZ, P]),
+            "aoh_shared_index_step_workspace_size": (SZ, [KVP, I32, I32, I32]),
             "aoh_stream_decode_noalloc": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P]),
         }
         for name, (res, args) in sig.items():
@@ -207,11 +208,15 @@ def shared_index_decode(q_layers: torch.Tensor, kv: KVCache, idx: torch.Tensor, 
         n_fac_cap, float(scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def shared_index_step_workspace_size(kv: KVCache, n_layers: int, n_q_heads: int, topk: int) -> int:
+    return int(lib().aoh_shared_index_step_workspace_size(ctypes.byref(kv), n_layers, n_q_heads, topk))
+
+
 def shared_index_step(q_index: torch.Tensor, q_layers: torch.Tensor, kv: KVCache, topk: int, idx: torch.Tensor,
-                      count: torch.Tensor, scale: float, out: torch.Tensor, stream=None) -> None:
+                      count: torch.Tensor, scale: float, out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
     _check("aoh_shared_index_step", lib().aoh_shared_index_step(
         _ptr(q_index), _ptr(q_layers), q_layers.shape[0], q_layers.shape[-2], ctypes.byref(kv), topk, _ptr(idx),
-        _ptr(count), float(scale), _ptr(out), _stream(stream)))
+        _ptr(count), float(scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def stream_decode_noalloc(q: torch.Tensor, kv: KVCache, roles, sink: int, window: int, scale: float,

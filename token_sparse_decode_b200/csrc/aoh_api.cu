@@ -83,7 +83,7 @@ FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
   // about two CTAs per SM; at least two pipeline stages per CTA; at most kFdMaxSplits splits a row
   const int64_t target = int64_t(kSmCount) * 2;
   int64_t chunk = ceil_div(std::max<int64_t>(work_tokens, 1), target);
-  chunk = std::max<int64_t>(chunk, 2 * kFdTS);
+  chunk = std::min<int64_t>(std::max<int64_t>(chunk, 2 * kFdTS), 1024);  // long CTAs are latency bound
   chunk = std::max<int64_t>(chunk, ceil_div(std::max<int64_t>(n_max, 1), kFdMaxSplits));
   chunk = ceil_div(chunk, kFdTS) * kFdTS;
   g.chunk = (int)chunk;
@@ -147,7 +147,7 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
   tp.d = kv->head_dim;
   tp.G = Hq / kv->n_kv_heads;
   tp.n_dom = n_dom;
-  if (kv->k_dom) {
+  if (kv->k_dom && idom) {
     if (2 * n_dom > kv->k_dom_cols) return AOH_ERR_INVALID_ARG;
     tp.src = static_cast<const uint16_t*>(kv->k_dom);
     tp.row_stride_tok = kv->k_dom_cols;
@@ -177,6 +177,12 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
     default: tip_score_kernel<16><<<grid, kTipThreads, 0, st>>>(tp); break;
   }
   return cuda_status(cudaGetLastError());
+}
+
+// Full-dimension scores (every chunk; the shared indexer's score), K read in place.
+aoh_status launch_tip_full(const void* q, int32_t Hq, const aoh_kv_cache* kv, float* scores, const uint8_t* heads,
+                           int n_listed, cudaStream_t st) {
+  return launch_tip(q, Hq, kv, nullptr, kv->head_dim / 2, scores, heads, n_listed, st);
 }
 
 // ------------------------------------------------------------------ top-k select
@@ -238,7 +244,7 @@ struct FusedPlan {
   size_t keys_bytes, ring_bytes, smem;
 };
 
-FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
+FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true) {
   FusedPlan f{};
   const int64_t L = std::max(kv->max_len, 1);
   const int64_t slice = (ceil_div(L, CL) + 3) & ~int64_t(3);
@@ -248,9 +254,10 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
   // 1 KB of slack: the kernel aligns its dynamic shared memory to 1024 bytes
   size_t budget = kTwoPerSm - 1024;
-  if (f.keys_bytes + kRingMin > budget) budget = kOnePerSm - 1024;
-  if (f.keys_bytes + kRingMin > budget) return f;
-  f.ring_bytes = std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage);
+  const size_t ring_min = need_ring ? kRingMin : 0;
+  if (f.keys_bytes + ring_min > budget) budget = kOnePerSm - 1024;
+  if (f.keys_bytes + ring_min > budget) return f;
+  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage) : 0;
   f.smem = f.keys_bytes + f.ring_bytes + 1024;
   f.ok = true;
   return f;
@@ -324,8 +331,49 @@ bool fused_feasible(const aoh_kv_cache* kv, int nq, bool packed) {
 int g_force_cluster = 0;  // diagnostic build: force the fused kernel's cluster size
 #endif
 
+template <typename K>
+int max_active_clusters(K kern, int CL, size_t smem) {
+  // (cluster size, dynamic shared memory) -> cudaOccupancyMaxActiveClusters, cached per process
+  static std::mutex mu;
+  static int keys[64][3];
+  static int n_keys = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const int kid = (int)(reinterpret_cast<uintptr_t>(reinterpret_cast<const void*>(kern)) & 0x7fffffff);
+  for (int i = 0; i < n_keys; ++i)
+    if (keys[i][0] == kid && keys[i][1] == CL && keys[i][2] >> 8 == (int)(smem >> 8)) return keys[i][2] & 0xff;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, 1, 1);
+  cfg.blockDim = dim3(kSrThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  n = std::min(n, 255);
+  if (n_keys < 64) {
+    keys[n_keys][0] = kid;
+    keys[n_keys][1] = CL;
+    keys[n_keys][2] = (int)((smem >> 8) << 8) | n;
+    ++n_keys;
+  }
+  return n;
+}
+
+// Launch the cluster row kernel with the cluster size that needs the fewest waves x slice
+// length (ties to the smaller cluster).  With max_waves > 0 nothing is launched when every
+// choice needs more waves; *launched says which happened.
 template <int D, int NT>
-aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st) {
+aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st, bool need_ring,
+                         int max_waves, bool* launched) {
+  *launched = false;
   auto kern = sparse_row_kernel<D, NT>;
   static bool configured = false;
   if (!configured) {
@@ -335,49 +383,29 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
     if (s != AOH_OK) return s;
     configured = true;
   }
-  // cluster size: fewest waves x slice length (the per-CTA work), ties to the smaller cluster
-  static int occ_cache[3][2] = {{-1, -1}, {-1, -1}, {-1, -1}};  // [CL 4/8/16][two-per-SM?]
   const int n_rows = n_listed * B;
   FusedPlan best{};
-  int64_t best_cost = INT64_MAX;
+  int64_t best_cost = INT64_MAX, best_waves = 0;
   const int cls[3] = {4, 8, 16};
   for (int i = 0; i < 3; ++i) {
-    const FusedPlan f = fused_candidate(kv, cls[i]);
+    const FusedPlan f = fused_candidate(kv, cls[i], need_ring);
     if (!f.ok) continue;
 #ifdef AOH_PHASE_TIMERS
     if (g_force_cluster && f.CL != g_force_cluster) continue;
 #endif
-    const int two = f.smem <= kTwoPerSm ? 1 : 0;  // the cache holds one entry per budget class
-    int& maxc = occ_cache[i][two];
-    if (maxc < 0) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(f.CL, 1, 1);
-      cfg.blockDim = dim3(kSrThreads);
-      cfg.dynamicSmemBytes = f.smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = f.CL;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        n = 0;
-      }
-      maxc = n;
-    }
+    const int maxc = max_active_clusters(kern, f.CL, f.smem);
     if (maxc <= 0) continue;
     const int64_t waves = ceil_div(n_rows, maxc);
     const int64_t cost = waves * f.slice;
     if (cost < best_cost) {
       best_cost = cost;
+      best_waves = waves;
       best = f;
     }
   }
   if (!best.ok) return AOH_ERR_UNSUPPORTED;
-  {
+  if (max_waves > 0 && best_waves > max_waves) return AOH_OK;
+  if (need_ring && !rp.scores_in) {
     const aoh_status ms = make_scan_map(rp, kv);
     if (ms != AOH_OK) return ms;
   }
@@ -395,21 +423,51 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, rp));
+  const aoh_status s = cuda_status(cudaLaunchKernelEx(&cfg, kern, rp));
+  *launched = (s == AOH_OK);
+  return s;
 }
 
-aoh_status launch_rows(const RowParams& rp, const aoh_kv_cache* kv, int nq, int n_listed, int B,
-                       cudaStream_t st) {
+aoh_status launch_rows(const RowParams& rp, const aoh_kv_cache* kv, int nq, int n_listed, int B, cudaStream_t st,
+                       bool need_ring, int max_waves, bool* launched) {
   const int nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
   if (kv->head_dim == 128) {
-    if (nqp == 8) return launch_rows_t<128, 1>(rp, kv, n_listed, B, st);
-    if (nqp == 16) return launch_rows_t<128, 2>(rp, kv, n_listed, B, st);
-    return launch_rows_t<128, 4>(rp, kv, n_listed, B, st);
+    if (nqp == 8) return launch_rows_t<128, 1>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
+    if (nqp == 16) return launch_rows_t<128, 2>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
+    return launch_rows_t<128, 4>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
   }
-  if (nqp == 8) return launch_rows_t<64, 1>(rp, kv, n_listed, B, st);
-  if (nqp == 16) return launch_rows_t<64, 2>(rp, kv, n_listed, B, st);
-  return launch_rows_t<64, 4>(rp, kv, n_listed, B, st);
+  if (nqp == 8) return launch_rows_t<64, 1>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
+  if (nqp == 16) return launch_rows_t<64, 2>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
+  return launch_rows_t<64, 4>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
 }
+
+// Select-only launch of the row kernel on precomputed scores: writes idx / count.
+aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
+                              int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
+                              cudaStream_t st) {
+  RowParams rp{};
+  rp.offsets = kv->offsets;
+  rp.scores_in = scores;
+  rp.select_only = 1;
+  rp.n_fac_per_seq = nfps;
+  rp.n_fac = n_fac;
+  rp.cap = cap;
+  rp.idx_out = idx;
+  rp.count_out = count;
+  rp.T = (int32_t)kv->total_tokens;
+  rp.B = kv->batch;
+  rp.Hkv = kv->n_kv_heads;
+  rp.G = 1;
+  rp.NQ = 1;
+  rp.srow_len = 16;
+  memcpy(rp.heads, heads, n_listed);
+  bool launched = false;
+  const aoh_status s = launch_rows(rp, kv, 1, n_listed, kv->batch, st, false, 0, &launched);
+  if (s == AOH_OK && !launched) return AOH_ERR_UNSUPPORTED;
+  return s;
+}
+
+bool select_rows_feasible(const aoh_kv_cache* kv) { return fused_candidate(kv, kSrMaxCluster, false).ok; }
 
 // Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,
 // or (idom == nullptr) K in place with every chunk.
@@ -576,6 +634,8 @@ aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t 
   if (!idx || !count || (!scores && kv->total_tokens > 0)) return AOH_ERR_INVALID_ARG;
   uint8_t heads[kMaxHeads];
   const int n = list_heads(kv, nullptr, true, heads);
+  if (select_rows_feasible(kv))
+    return launch_select_rows(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
   return launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
 }
 
@@ -641,15 +701,23 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
     rp.NQ = G;
     rp.scale_log2 = scale * 1.4426950408889634f;
     memcpy(rp.heads, heads, n_listed);
-    return launch_rows(rp, kv, G, n_listed, kv->batch, st);
+    // one launch when every row's cluster runs in a single wave
+    bool launched = false;
+    if ((s = launch_rows(rp, kv, G, n_listed, kv->batch, st, true, 1, &launched)) != AOH_OK) return s;
+    if (launched) return AOH_OK;
   }
 
-  // rows too long for one cluster: scan, select and attend as three kernels
+  // otherwise three kernels: the scan over all SMs, the cluster select on the (L2-resident)
+  // scores, and the split-K gather
   if (kv->total_tokens > 0) {
     if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st)) != AOH_OK) return s;
   }
-  if ((s = launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st)) != AOH_OK)
-    return s;
+  if (select_rows_feasible(kv)) {
+    s = launch_select_rows(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st);
+  } else {
+    s = launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st);
+  }
+  if (s != AOH_OK) return s;
 
   const FdGeom geo = sparse_geom(kv, n_q_heads, n_fac_cap);
   FdecParams fp{};
@@ -773,9 +841,21 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream));
 }
 
+size_t shared_step_ws_bytes(const aoh_kv_cache* kv, int32_t n_layers, int32_t Hq, int32_t topk) {
+  return fd_bytes(shared_geom(kv, n_layers, Hq, topk)) +
+         align256(sizeof(float) * (size_t)kv->n_kv_heads * (size_t)std::max<int64_t>(kv->total_tokens, 1));
+}
+
+size_t aoh_shared_index_step_workspace_size(const aoh_kv_cache* kv, int32_t n_layers, int32_t n_q_heads,
+                                            int32_t topk) {
+  if (check_kv(kv) != AOH_OK || check_heads(kv, n_q_heads) != AOH_OK || n_layers < 1 || topk < 1) return 0;
+  if (int64_t(n_layers) * (n_q_heads / kv->n_kv_heads) > kMaxQRows) return 0;
+  return shared_step_ws_bytes(kv, n_layers, n_q_heads, topk);
+}
+
 aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int32_t n_layers, int32_t n_q_heads,
                                  const aoh_kv_cache* kv, int32_t topk, int32_t* idx, int32_t* count, float scale,
-                                 float* out, void* stream) {
+                                 float* out, void* workspace, size_t workspace_bytes, void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
   if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
@@ -785,44 +865,74 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   if (kv->batch == 0) return AOH_OK;
   if (!q_index || !q_layers || !idx || !count || !out) return AOH_ERR_INVALID_ARG;
   if (!aligned16(q_index) || !aligned16(q_layers)) return AOH_ERR_ALIGNMENT;
+  const size_t need = shared_step_ws_bytes(kv, n_layers, n_q_heads, topk);
+  if (!ws_ok(workspace, workspace_bytes, need)) return AOH_ERR_WORKSPACE;
   uint8_t heads[kMaxHeads];
   const int n_listed = list_heads(kv, nullptr, true, heads);
-  if (!fused_feasible(kv, n_layers * G, false)) return AOH_ERR_UNSUPPORTED;
-  RowParams rp{};
-  rp.q_score = static_cast<const uint16_t*>(q_index);
-  rp.q_attn = static_cast<const uint16_t*>(q_layers);
-  rp.k = static_cast<const uint16_t*>(kv->k);
-  rp.v = static_cast<const uint16_t*>(kv->v);
-  rp.offsets = kv->offsets;
-  rows_score_source(rp, kv, nullptr, kv->head_dim / 2);
-  rp.n_fac_per_seq = nullptr;
-  rp.n_fac = topk;
-  rp.cap = topk;
-  rp.idx_out = idx;
-  rp.count_out = count;
-  rp.out = out;
-  rp.stride_tok = kv->stride_tok;
-  rp.stride_head = kv->stride_head;
-  rp.T = (int32_t)kv->total_tokens;
-  rp.B = kv->batch;
-  rp.Hq = n_q_heads;
-  rp.Hkv = kv->n_kv_heads;
-  rp.G = G;
-  rp.NQ = n_layers * G;
-  rp.scale_log2 = scale * 1.4426950408889634f;
-  memcpy(rp.heads, heads, n_listed);
-  return launch_rows(rp, kv, n_layers * G, n_listed, kv->batch, as_stream(stream));
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const FdGeom geo = shared_geom(kv, n_layers, n_q_heads, topk);
+  float* scores = reinterpret_cast<float*>(ws + fd_bytes(geo));
+  if (fused_feasible(kv, n_layers * G, false)) {
+    RowParams rp{};
+    rp.q_score = static_cast<const uint16_t*>(q_index);
+    rp.q_attn = static_cast<const uint16_t*>(q_layers);
+    rp.k = static_cast<const uint16_t*>(kv->k);
+    rp.v = static_cast<const uint16_t*>(kv->v);
+    rp.offsets = kv->offsets;
+    rows_score_source(rp, kv, nullptr, kv->head_dim / 2);
+    rp.n_fac_per_seq = nullptr;
+    rp.n_fac = topk;
+    rp.cap = topk;
+    rp.idx_out = idx;
+    rp.count_out = count;
+    rp.out = out;
+    rp.stride_tok = kv->stride_tok;
+    rp.stride_head = kv->stride_head;
+    rp.T = (int32_t)kv->total_tokens;
+    rp.B = kv->batch;
+    rp.Hq = n_q_heads;
+    rp.Hkv = kv->n_kv_heads;
+    rp.G = G;
+    rp.NQ = n_layers * G;
+    rp.scale_log2 = scale * 1.4426950408889634f;
+    memcpy(rp.heads, heads, n_listed);
+    bool launched = false;
+    if ((s = launch_rows(rp, kv, n_layers * G, n_listed, kv->batch, st, true, 1, &launched)) != AOH_OK) return s;
+    if (launched) return AOH_OK;
+  }
+  // three kernels: full-dimension scores, the cluster select, the shared-index gather
+  if (kv->total_tokens > 0) {
+    if ((s = launch_tip_full(q_index, n_q_heads, kv, scores, heads, n_listed, st)) != AOH_OK) return s;
+  }
+  if (select_rows_feasible(kv)) {
+    s = launch_select_rows(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, st);
+  } else {
+    s = launch_select(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, st);
+  }
+  if (s != AOH_OK) return s;
+  FdecParams fp{};
+  fp.q = static_cast<const uint16_t*>(q_layers);
+  fp.k = static_cast<const uint16_t*>(kv->k);
+  fp.v = static_cast<const uint16_t*>(kv->v);
+  fp.offsets = kv->offsets;
+  fp.idx = idx;
+  fp.count = count;
+  fp.out = out;
+  fp.stride_tok = kv->stride_tok;
+  fp.stride_head = kv->stride_head;
+  fp.B = kv->batch;
+  fp.Hq = n_q_heads;
+  fp.Hkv = kv->n_kv_heads;
+  fp.G = G;
+  fp.NQ = n_layers * G;
+  fp.cap = topk;
+  fp.list_mode = 1;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  memcpy(fp.heads, heads, n_listed);
+  fd_bind(fp, geo, ws);
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st);
 }
-
-#ifdef AOH_PHASE_TIMERS
-void aoh_debug_force_cluster(int32_t cl) { g_force_cluster = cl; }
-
-// Diagnostic build only: copy the phase stamps of the fused kernel to the host.
-int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
-  if (n_ctas > kPhaseCtas) n_ctas = kPhaseCtas;
-  return cudaMemcpyFromSymbol(host, g_phase_ns, sizeof(long long) * kPhaseSlots * n_ctas) == cudaSuccess ? 0 : 5;
-}
-#endif
 
 }  // extern "C"
 

@@ -66,6 +66,8 @@ struct RowParams {
   int32_t T, B, Hq, Hkv, G, NQ;
   int32_t keys_bytes;        // dynamic shared memory before the ring
   int32_t ring_bytes;        // ring region (scan stages, then attention stages); >= 64 KB
+  const float* scores_in;    // non-null: keys come from these fp32 scores [Hkv][T] (no scan)
+  int32_t select_only;       // 1: stop after writing the index (no attention)
   int32_t scan_box;          // scan tile: inner box (elements, <= 64) ...
   int32_t scan_rows;         // ... and rows per stage (<= 256); halves = srow_len / scan_box
   float scale_log2;
@@ -177,9 +179,15 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   int* plist = reinterpret_cast<int*>(smem);  // selected positions replace the keys
   int nloc;
 
+  if (n < L && p.scores_in) {
+    // scores already computed (the scan ran as its own kernel): load them as keys
+    const float* srow = p.scores_in + (int64_t)g * p.T + off + lo;
+    for (int i = tid; i < m; i += kSrThreads) keys[i] = score_key(__ldcg(srow + i));
+    __syncthreads();
+  }
   if (n < L) {
     // =============================================================== 1. scan
-    {
+    if (!p.scores_in) {
       // ring of tensor-map tiles: one elected thread issues halves x (box x rows) per stage
       const int box = p.scan_box, rows = p.scan_rows;
       const int halves = p.srow_len / box;
@@ -473,6 +481,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     nloc = m;
   }
   __syncthreads();
+  if (p.select_only) {  // index written; peers may still read this CTA's histograms
+    cluster.sync();
+    return;
+  }
 
   AOH_PHASE(3);
   // =============================================================== 3. attend

@@ -21,7 +21,7 @@ constexpr int kTipThreads = 256;
 struct TipParams {
   const uint16_t* q;        // [B][Hq][d]
   const uint16_t* src;      // packed k_dom or K
-  const int32_t* idom;      // [Hkv][n_dom]
+  const int32_t* idom;      // [Hkv][n_dom]; null: every chunk (K in place)
   const int32_t* offsets;   // [B + 1]
   float* scores;            // [Hkv][T]
   int64_t row_stride_tok;   // elements between token rows of one head
@@ -81,6 +81,8 @@ __global__ void __launch_bounds__(kTipThreads) tip_score_kernel(const TipParams 
           dim = tid < p.n_dom ? c : c + C;
         }
       }
+    } else if (p.idom == nullptr) {
+      dim = tid;  // every chunk: the full dot
     } else {
       const int c = tid < C ? tid : tid - C;
       for (int j = 0; j < p.n_dom; ++j) {

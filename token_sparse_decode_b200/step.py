@@ -75,7 +75,7 @@ class SparseDecodeStep:
 
 
 class SharedIndexStep:
-    """fused=True: one ``aoh_shared_index_step`` launch; False: score, select, decode as three calls."""
+    """fused=True: one ``aoh_shared_index_step`` call; False: score, select, decode as three calls."""
 
     def __init__(self, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
                  n_layers: int, n_q_heads: int, topk: int, scale: float, fused: bool = True):
@@ -91,6 +91,8 @@ class SharedIndexStep:
         self.idx = torch.empty((batch, Hkv, self.topk), dtype=torch.int32, device=self.dev)
         self.count = torch.empty((batch, Hkv), dtype=torch.int32, device=self.dev)
         self.ws = B.workspace(B.shared_index_decode_workspace_size(self.kv, n_layers, n_q_heads, self.topk), self.dev)
+        self.ws_step = B.workspace(B.shared_index_step_workspace_size(self.kv, n_layers, n_q_heads, self.topk),
+                                   self.dev) if fused else None
         self.out = torch.zeros((n_layers, batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
 
     def index(self, q_index: torch.Tensor) -> None:
@@ -99,7 +101,8 @@ class SharedIndexStep:
 
     def __call__(self, q_index: torch.Tensor, q_layers: torch.Tensor) -> torch.Tensor:
         if self.fused:
-            B.shared_index_step(q_index, q_layers, self.kv, self.topk, self.idx, self.count, self.scale, self.out)
+            B.shared_index_step(q_index, q_layers, self.kv, self.topk, self.idx, self.count, self.scale, self.out,
+                                self.ws_step)
             return self.out
         self.index(q_index)
         B.shared_index_decode(q_layers, self.kv, self.idx, self.count, self.topk, self.scale, self.out, self.ws)
