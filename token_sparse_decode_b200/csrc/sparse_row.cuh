@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   int32_t* idx_row = p.idx_out + ((int64_t)b * p.Hkv + g) * p.cap;
   for (int j = n + rk * kSrThreads + tid; j < p.cap; j += CL * kSrThreads) idx_row[j] = -1;
   if (rk == 0 && tid == 0) p.count_out[(int64_t)b * p.Hkv + g] = n;
-  if (n == 0) {  // uniform over the cluster: zero rows, no barrier taken
-    if (rk == 0) {
+  if (n == 0) {  // uniform over the cluster: zero rows (none in select-only mode), no barrier taken
+    if (rk == 0 && !p.select_only) {
       for (int e = tid; e < p.NQ * D; e += kSrThreads) {
         const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
         p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + e % D] = 0.f;
