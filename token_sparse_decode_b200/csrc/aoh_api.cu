@@ -244,6 +244,12 @@ struct FusedPlan {
   size_t keys_bytes, ring_bytes, smem;
 };
 
+#ifdef AOH_PHASE_TIMERS
+int g_force_cluster = 0;  // diagnostic build: force the fused kernel's cluster size ...
+int g_force_ring = 0;     // ... cap its ring (bytes) ...
+int g_force_one_per_sm = 0;  // ... or give one CTA per SM the whole budget
+#endif
+
 FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true) {
   FusedPlan f{};
   const int64_t L = std::max(kv->max_len, 1);
@@ -256,8 +262,14 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   size_t budget = kTwoPerSm - 1024;
   const size_t ring_min = need_ring ? kRingMin : 0;
   if (f.keys_bytes + ring_min > budget) budget = kOnePerSm - 1024;
+#ifdef AOH_PHASE_TIMERS
+  if (g_force_one_per_sm) budget = kOnePerSm - 1024;
+#endif
   if (f.keys_bytes + ring_min > budget) return f;
   f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage) : 0;
+#ifdef AOH_PHASE_TIMERS
+  if (need_ring && g_force_ring) f.ring_bytes = std::min(f.ring_bytes, (size_t)g_force_ring);
+#endif
   f.smem = f.keys_bytes + f.ring_bytes + 1024;
   f.ok = true;
   return f;
@@ -327,9 +339,6 @@ bool fused_feasible(const aoh_kv_cache* kv, int nq, bool packed) {
   return nq <= kMaxQRows && scan_layout_ok(kv, packed) && fused_candidate(kv, kSrMaxCluster).ok;
 }
 
-#ifdef AOH_PHASE_TIMERS
-int g_force_cluster = 0;  // diagnostic build: force the fused kernel's cluster size
-#endif
 
 template <typename K>
 int max_active_clusters(K kern, int CL, size_t smem) {
@@ -933,6 +942,26 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   fd_bind(fp, geo, ws);
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st);
 }
+
+#ifdef AOH_PHASE_TIMERS
+// Diagnostic build only: copy the phase stamps of the fused kernel to the host.
+int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
+  if (n_ctas > kPhaseCtas) n_ctas = kPhaseCtas;
+  return cudaMemcpyFromSymbol(host, g_phase_ns, sizeof(long long) * kPhaseSlots * n_ctas) == cudaSuccess ? 0 : 5;
+}
+void aoh_debug_force_cluster(int32_t cl) { g_force_cluster = cl; }
+void aoh_debug_force_ring(int32_t bytes, int32_t one_per_sm) {
+  g_force_ring = bytes;
+  g_force_one_per_sm = one_per_sm;
+}
+// cudaOccupancyMaxActiveClusters of the fused kernel (d 128, one n-tile).
+int32_t aoh_debug_max_clusters(int32_t cl, int32_t smem) {
+  auto kern = sparse_row_kernel<128, 1>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOnePerSm);
+  cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return max_active_clusters(kern, cl, (size_t)smem);
+}
+#endif
 
 }  // extern "C"
 
