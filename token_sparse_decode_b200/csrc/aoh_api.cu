@@ -260,13 +260,14 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
   // 1 KB of slack: the kernel aligns its dynamic shared memory to 1024 bytes
   size_t budget = kTwoPerSm - 1024;
-  const size_t ring_min = need_ring ? kRingMin : 0;
+  // select-only launches still need a region as large as the keys for the select's candidates
+  const size_t ring_min = need_ring ? kRingMin : f.keys_bytes;
   if (f.keys_bytes + ring_min > budget) budget = kOnePerSm - 1024;
 #ifdef AOH_PHASE_TIMERS
   if (g_force_one_per_sm) budget = kOnePerSm - 1024;
 #endif
   if (f.keys_bytes + ring_min > budget) return f;
-  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage) : 0;
+  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage) : f.keys_bytes;
 #ifdef AOH_PHASE_TIMERS
   if (need_ring && g_force_ring) f.ring_bytes = std::min(f.ring_bytes, (size_t)g_force_ring);
 #endif

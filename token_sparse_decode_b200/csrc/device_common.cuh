@@ -149,6 +149,14 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+// ------------------------------------------------------------------ split cluster barrier
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
 // ------------------------------------------------------------------ small reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -131,12 +131,12 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t mbar_s[kSrMaxStages];
-  __shared__ int hist[2][256];
+  __shared__ int lh[256];      // this CTA's histogram of the current digit
+  __shared__ int tot[2][256];  // cluster totals of digits 0-2 (every CTA adds its counts here)
   __shared__ int scan_scratch[33];
   __shared__ float qt[128];
-  __shared__ int s_bin, s_above, s_eq_before, s_sel_before;
+  __shared__ int s_bin, s_above, s_eq_before, s_sel_before, s_ncand, s_up;
   __shared__ int s_gt[kSrMaxCluster], s_eq[kSrMaxCluster], s_eq_all;
-  __shared__ int s_gt24[8];  // per warp: this CTA's keys whose first 24 bits exceed the prefix
 
   AOH_PHASE(0);
   cgs::cluster_group cluster = cgs::this_cluster();
@@ -179,10 +179,30 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   int* plist = reinterpret_cast<int*>(smem);  // selected positions replace the keys
   int nloc;
 
+  // The select's totals are filled by every CTA of the cluster: zero them, then arrive on a
+  // cluster barrier that is waited on only before the first remote add (the scan runs in between).
+  if (n < L) {
+    lh[tid] = 0;
+    tot[0][tid] = 0;
+    tot[1][tid] = 0;
+    if (tid == 0) s_up = 0;
+    __syncthreads();
+    cluster_arrive_release();
+  }
   if (n < L && p.scores_in) {
-    // scores already computed (the scan ran as its own kernel): load them as keys
+    // scores already computed (the scan ran as its own kernel): load them as keys and count
+    // their first digit
     const float* srow = p.scores_in + (int64_t)g * p.T + off + lo;
-    for (int i = tid; i < m; i += kSrThreads) keys[i] = score_key(__ldcg(srow + i));
+    for (int b0 = warp * 32; b0 < m; b0 += kSrThreads) {  // warp-uniform trip count
+      const int i = b0 + lane;
+      int bin = -1;
+      if (i < m) {
+        const uint32_t key = score_key(__ldcg(srow + i));
+        keys[i] = key;
+        bin = (int)(key >> 24);
+      }
+      hist_add(lh, bin);
+    }
     __syncthreads();
   }
   if (n < L) {
@@ -293,12 +313,23 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
               mma_16816(c4, a, bt[ks][0], bt[ks][1]);
             }
           }
+          int bin_a = -1, bin_b = -1;
           if ((lane & 3) == 0) {
             const int ri = lane >> 2;  // row within the 16-row tile; nv counts from the tile start
             const int r0 = st * rows + tile * 16 + ri;
-            if (ri < nv) keys[r0] = score_key(c4[0] + c4[1]);
-            if (ri + 8 < nv) keys[r0 + 8] = score_key(c4[2] + c4[3]);
+            if (ri < nv) {
+              const uint32_t key = score_key(c4[0] + c4[1]);
+              keys[r0] = key;
+              bin_a = (int)(key >> 24);
+            }
+            if (ri + 8 < nv) {
+              const uint32_t key = score_key(c4[2] + c4[3]);
+              keys[r0 + 8] = key;
+              bin_b = (int)(key >> 24);
+            }
           }
+          hist_add(lh, bin_a);  // first radix digit, counted as the keys are made
+          hist_add(lh, bin_b);
         }
         __syncthreads();  // the slot is free: refill it
         if (tid == 0 && st + ns < nst) issue(st + ns);
@@ -311,79 +342,73 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     }
     AOH_PHASE(1);
     // =============================================================== 2. select
-    // One cluster barrier and two block barriers per digit.  In the last digit every
-    // CTA also derives, from the histograms it reads anyway, how many keys of each
-    // peer lie above the threshold (s_gt) and equal it (s_eq): the compaction then
-    // needs no further exchange.
+    // 4-digit MSB radix select over the cluster.  Digits 0-2: every CTA adds its non-zero
+    // counts into each peer's total (remote atomics), one cluster barrier, then the digit is
+    // picked from the local total.  Digit 3: every CTA reads each peer's last histogram, which
+    // also gives each peer's number of keys above the threshold (s_gt) and equal to it (s_eq),
+    // so the compaction needs no further exchange.  After digit 0 the keys sharing the chosen
+    // first digit are compacted; digits 1-3 count only those.
+    cluster_wait_acquire();  // peers have zeroed their totals
+    uint32_t* cand = reinterpret_cast<uint32_t*>(smem + p.keys_bytes);  // free region during the select
     uint32_t prefix = 0u, pmask = 0u;
     int krem = n;
-    hist[0][tid] = 0;
-    if (tid < 8) s_gt24[tid] = 0;
-    __syncthreads();
+    int ncand = 0;
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
-      int* h = hist[pass & 1];
-      if (pass == 1) AOH_PHASE(12);
-      // count (four keys per lane, warp-uniform trip count); the first digit (sign and
-      // exponent) is shared by most keys, so it is counted with warp aggregation.  In the
-      // last digit, keys whose first 24 bits exceed the prefix are counted too.
-      int above24 = 0;
-      for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
-        const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the keys region
-        const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
-        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+      if (pass > 0) {
+        for (int b0 = warp * 128; b0 < ncand; b0 += 8 * 128) {
+          const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the candidate region
+          const uint4 k4 = *reinterpret_cast<const uint4*>(cand + i0);
+          const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool valid = i0 + j < m;
-          const bool in = valid && ((kk[j] & pmask) == prefix);
-          const int bin = in ? (int)((kk[j] >> shift) & 255u) : -1;
-          if (pass == 0) {
-            hist_add(h, bin);
-          } else if (in) {
-            atomicAdd(&h[bin], 1);
-          }
-          if (pass == 3) above24 += valid && ((kk[j] & pmask) > prefix);
+          for (int j = 0; j < 4; ++j)
+            if (i0 + j < ncand && (kk[j] & pmask) == prefix) atomicAdd(&lh[(kk[j] >> shift) & 255u], 1);
         }
       }
-      if (pass == 3) {
-        above24 = __reduce_add_sync(0xffffffffu, above24);
-        if (lane == 0) s_gt24[warp] = above24;
-      }
-      if (pass == 1) AOH_PHASE(8);
-      cluster.sync();
-      if (pass == 1) AOH_PHASE(9);
-      int* hn = hist[(pass + 1) & 1];  // peers finished reading it before this barrier
-      hn[tid] = 0;
-      const int bin = 255 - tid;       // scanned from the top bin down
+      __syncthreads();
+      const int bin = 255 - tid;  // the scan below runs from the top bin down
+      int total_bin;
       int v[kSrMaxCluster];
+      if (pass < 3) {
+        const int c = lh[tid];
+        if (c) {
+          for (int q = 0; q < CL; ++q) atomicAdd(cluster.map_shared_rank(&tot[pass & 1][tid], q), c);
+        }
+        tot[(pass + 1) & 1][tid] = 0;  // peers add into it only after the barrier below
+        cluster.sync();
+        total_bin = tot[pass & 1][bin];
+      } else {
+        cluster.sync();  // every peer's last-digit histogram is complete
 #pragma unroll
-      for (int q = 0; q < kSrMaxCluster; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
-      int tot = 0;
+        for (int q = 0; q < kSrMaxCluster; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(lh, q)[bin] : 0;
+        total_bin = 0;
 #pragma unroll
-      for (int q = 0; q < kSrMaxCluster; ++q) tot += v[q];
-      if (pass == 1) AOH_PHASE(10);
+        for (int q = 0; q < kSrMaxCluster; ++q) total_bin += v[q];
+      }
       // exclusive prefix over tid (bins from the top): warp scan, then the warp totals
-      int x = tot;
+      int x = total_bin;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
       if (lane == 31) scan_scratch[warp] = x;
+      if (tid == 0) s_ncand = 0;
       __syncthreads();
-      int above = x - tot;
+      int above = x - total_bin;
       for (int w2 = 0; w2 < warp; ++w2) above += scan_scratch[w2];
-      if (above < krem && krem <= above + tot) {
+      if (above < krem && krem <= above + total_bin) {
         s_bin = bin;
         s_above = above;
       }
       __syncthreads();
       const int sb = s_bin;
-      if (pass == 1) AOH_PHASE(11);
-      if (pass == 3) {
-        // peers' keys above the threshold: first 24 bits above the prefix, or equal
-        // there and in a higher last digit; equal to it: the chosen bin
+      if (pass < 3) {
+        // this CTA's keys above the threshold decided by this digit
+        const int w = __reduce_add_sync(0xffffffffu, bin > sb ? lh[bin] : 0);
+        if (lane == 0 && w) atomicAdd(&s_up, w);
+      } else {
 #pragma unroll
         for (int q = 0; q < kSrMaxCluster; ++q) {
           if (q < CL) {
@@ -396,19 +421,32 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
           for (int q = 0; q < kSrMaxCluster; ++q)
             if (q < CL) s_eq[q] = v[q];
         }
-        if (tid < CL) {
-          const int* g24 = cluster.map_shared_rank(s_gt24, tid);
-          int t = 0;
+        if (tid < CL) atomicAdd(&s_gt[tid], *cluster.map_shared_rank(&s_up, tid));
+      }
+      if (pass == 0) {
+        // candidates of digits 1-3: the keys whose first digit is the chosen one
+        for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
+          const int i0 = b0 + 4 * lane;
+          const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
+          const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-          for (int w2 = 0; w2 < 8; ++w2) t += g24[w2];
-          atomicAdd(&s_gt[tid], t);
+          for (int j = 0; j < 4; ++j) {
+            const bool hit = (i0 + j < m) && (int)(kk[j] >> 24) == sb;
+            const unsigned bal = __ballot_sync(0xffffffffu, hit);
+            int base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&s_ncand, __popc(bal));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (hit) cand[base + __popc(bal & ((1u << lane) - 1u))] = kk[j];
+          }
         }
       }
       prefix |= (uint32_t)sb << shift;
       pmask |= 255u << shift;
       krem -= s_above;
+      if (pass < 3) lh[tid] = 0;  // the last histogram stays: peers read it
+      __syncthreads();
+      if (pass == 0) ncand = s_ncand;
     }
-    __syncthreads();
     const uint32_t KT = prefix;
     const int need_eq = krem;
     AOH_PHASE(2);

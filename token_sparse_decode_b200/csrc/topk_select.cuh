@@ -36,12 +36,6 @@ struct SelectParams {
   uint8_t heads[kMaxHeads];
 };
 
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
 
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectParams p) {
   extern __shared__ __align__(16) uint32_t skeys[];
