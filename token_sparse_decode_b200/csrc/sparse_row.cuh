@@ -190,19 +190,9 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     cluster_arrive_release();
   }
   if (n < L && p.scores_in) {
-    // scores already computed (the scan ran as its own kernel): load them as keys and count
-    // their first digit
+    // scores already computed (the scan ran as its own kernel): load them as keys
     const float* srow = p.scores_in + (int64_t)g * p.T + off + lo;
-    for (int b0 = warp * 32; b0 < m; b0 += kSrThreads) {  // warp-uniform trip count
-      const int i = b0 + lane;
-      int bin = -1;
-      if (i < m) {
-        const uint32_t key = score_key(__ldcg(srow + i));
-        keys[i] = key;
-        bin = (int)(key >> 24);
-      }
-      hist_add(lh, bin);
-    }
+    for (int i = tid; i < m; i += kSrThreads) keys[i] = score_key(__ldcg(srow + i));
     __syncthreads();
   }
   if (n < L) {
@@ -313,23 +303,12 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
               mma_16816(c4, a, bt[ks][0], bt[ks][1]);
             }
           }
-          int bin_a = -1, bin_b = -1;
           if ((lane & 3) == 0) {
             const int ri = lane >> 2;  // row within the 16-row tile; nv counts from the tile start
             const int r0 = st * rows + tile * 16 + ri;
-            if (ri < nv) {
-              const uint32_t key = score_key(c4[0] + c4[1]);
-              keys[r0] = key;
-              bin_a = (int)(key >> 24);
-            }
-            if (ri + 8 < nv) {
-              const uint32_t key = score_key(c4[2] + c4[3]);
-              keys[r0 + 8] = key;
-              bin_b = (int)(key >> 24);
-            }
+            if (ri < nv) keys[r0] = score_key(c4[0] + c4[1]);
+            if (ri + 8 < nv) keys[r0 + 8] = score_key(c4[2] + c4[3]);
           }
-          hist_add(lh, bin_a);  // first radix digit, counted as the keys are made
-          hist_add(lh, bin_b);
         }
         __syncthreads();  // the slot is free: refill it
         if (tid == 0 && st + ns < nst) issue(st + ns);
@@ -356,7 +335,16 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
-      if (pass > 0) {
+      if (pass == 0) {
+        // the first digit (sign and exponent) is shared by most keys: warp-aggregated counts
+        for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
+          const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the keys region
+          const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
+          const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) hist_add(lh, i0 + j < m ? (int)(kk[j] >> 24) : -1);
+        }
+      } else {
         for (int b0 = warp * 128; b0 < ncand; b0 += 8 * 128) {
           const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the candidate region
           const uint4 k4 = *reinterpret_cast<const uint4*>(cand + i0);
