@@ -86,9 +86,15 @@ FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
   chunk = std::min<int64_t>(std::max<int64_t>(chunk, 2 * kFdTS), 1024);  // long CTAs are latency bound
   chunk = std::max<int64_t>(chunk, ceil_div(std::max<int64_t>(n_max, 1), kFdMaxSplits));
   chunk = ceil_div(chunk, kFdTS) * kFdTS;
+  g.nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
+  // partials grow with the query rows and the last CTA of a row reads them all: at most 16
+  // splits for 16 query rows, 8 for 32
+  if (g.nqp > 8) {
+    const int64_t max_sp = g.nqp == 16 ? 16 : 8;
+    chunk = std::max<int64_t>(chunk, ceil_div(ceil_div(std::max<int64_t>(n_max, 1), max_sp), kFdTS) * kFdTS);
+  }
   g.chunk = (int)chunk;
   g.max_splits = (int)std::max<int64_t>(1, ceil_div(std::max<int64_t>(n_max, 1), chunk));
-  g.nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
   g.rows = rows;
   g.ticket_bytes = align256(sizeof(int32_t) * (size_t)std::max(rows, 1));
   g.ml_bytes = align256(sizeof(float) * (size_t)rows * g.max_splits * g.nqp * 2);
@@ -186,9 +192,11 @@ aoh_status launch_tip_full(const void* q, int32_t Hq, const aoh_kv_cache* kv, fl
 }
 
 // ------------------------------------------------------------------ top-k select
+// The select kernel with `cl` CTAs per row (1: one CTA reads the row's scores from L2
+// and takes no cluster barrier; up to 8: a cluster shares the row).
 aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
                          int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
-                         cudaStream_t st) {
+                         cudaStream_t st, int cl = 0) {
   SelectParams sp{};
   sp.scores = scores;
   sp.offsets = kv->offsets;
@@ -200,7 +208,8 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
   sp.n_fac = n_fac;
   sp.cap = cap;
   memcpy(sp.heads, heads, n_listed);
-  const int CL = (int)std::min<int64_t>(kSelMaxCluster, std::max<int64_t>(1, ceil_div(kv->max_len, 256)));
+  const int CL = cl > 0 ? std::min(cl, kSelMaxCluster)
+                        : (int)std::min<int64_t>(kSelMaxCluster, std::max<int64_t>(1, ceil_div(kv->max_len, 256)));
   const int64_t chunk = std::max<int64_t>(4, ceil_div(ceil_div(std::max(kv->max_len, 1), CL), 4) * 4);
   sp.chunk = (int32_t)chunk;
   size_t smem = (size_t)chunk * 4;
@@ -479,6 +488,17 @@ aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32
 
 bool select_rows_feasible(const aoh_kv_cache* kv) { return fused_candidate(kv, kSrMaxCluster, false).ok; }
 
+// The select stage of the three-kernel step: one CTA per row (scores streamed from L2, no
+// cluster barrier) when there are enough rows to occupy the SMs, else a cluster per row.
+aoh_status select_stage(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
+                        int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
+                        cudaStream_t st) {
+  const int64_t rows = int64_t(kv->batch) * n_listed;
+  if (rows >= kSmCount / 2 || !select_rows_feasible(kv))
+    return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st, 1);
+  return launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
+}
+
 // Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,
 // or (idom == nullptr) K in place with every chunk.
 void rows_score_source(RowParams& rp, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom) {
@@ -722,11 +742,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   if (kv->total_tokens > 0) {
     if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st)) != AOH_OK) return s;
   }
-  if (select_rows_feasible(kv)) {
-    s = launch_select_rows(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st);
-  } else {
-    s = launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st);
-  }
+  s = select_stage(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st);
   if (s != AOH_OK) return s;
 
   const FdGeom geo = sparse_geom(kv, n_q_heads, n_fac_cap);
@@ -915,11 +931,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   if (kv->total_tokens > 0) {
     if ((s = launch_tip_full(q_index, n_q_heads, kv, scores, heads, n_listed, st)) != AOH_OK) return s;
   }
-  if (select_rows_feasible(kv)) {
-    s = launch_select_rows(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, st);
-  } else {
-    s = launch_select(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, st);
-  }
+  s = select_stage(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, st);
   if (s != AOH_OK) return s;
   FdecParams fp{};
   fp.q = static_cast<const uint16_t*>(q_layers);

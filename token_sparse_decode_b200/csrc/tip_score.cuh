@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kTipThreads) tip_score_kernel(const TipParams 
     active |= (qs[i] != 0.f);
   }
   constexpr int RPI = kTipThreads / S;  // rows per block iteration
-  constexpr int U = 4;                  // independent loads in flight per thread
+  constexpr int U = 8;                  // independent loads in flight per thread
   const uint16_t* base = p.src + (int64_t)g * p.row_stride_head + (int64_t)off * p.row_stride_tok + seg * 8;
   float* srow = p.scores + (int64_t)g * p.T + off;
   // Warp-uniform loop bounds: every lane of a warp takes the same trip count, so the
