@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
   constexpr int KS = D / 16;          // k-steps of QK
-  constexpr int KH = KS / 2;          // PV m-tiles per half of the head dimension
-  constexpr int WT = 4 / NT;          // token groups per (n-tile, half)
+  constexpr int DP = (NT == 4) ? 2 : 4;  // parts of the head dimension in the PV product
+  constexpr int TG = 8 / (NT * DP);      // token groups (warps sharing an n-tile and a part)
+  constexpr int KH = KS / DP;            // PV m-tiles per part
   constexpr int SUB = kSrTS / 16;     // 16-token sub-tiles per stage
   constexpr int NQP = NT * 8;
 
@@ -514,8 +515,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 
   AOH_PHASE(3);
   // =============================================================== 3. attend
-  const int half = warp >> 2, r4 = warp & 3;
-  const int nt = r4 % NT, tg = r4 / NT;
+  // warp = (token group, n-tile, part of the head dimension)
+  const int dp = warp % DP, nt = (warp / DP) % NT, tg = warp / (DP * NT);
   float acc[KH][4];
 #pragma unroll
   for (int i = 0; i < KH; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
@@ -572,7 +573,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     const uint32_t vt = kt + AttTile<D>::kTile;
 #pragma unroll
     for (int u = 0; u < SUB; ++u) {
-      if ((st * SUB + u) % WT != tg) continue;
+      if ((st * SUB + u) % TG != tg) continue;
       const int nv = nloc - (st * kSrTS + u * 16);
       if (nv <= 0) continue;
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -623,7 +624,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 #pragma unroll
         for (int mt = 0; mt < KH; ++mt) {
           uint32_t a[4];
-          ldsm_x4_trans(a, vt + r * AttTile<D>::kPitch + ((half * KH + mt) * 16 + dsel) * 2);
+          ldsm_x4_trans(a, vt + r * AttTile<D>::kPitch + ((dp * KH + mt) * 16 + dsel) * 2);
           mma_16816(acc[mt], a, pb0, pb1);
           mma_16816(acc[mt], a, pl0, pl1);
         }
@@ -639,10 +640,11 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   __syncthreads();  // stage buffers are free
 
   AOH_PHASE(4);
-  // ---- merge the warps of this CTA: red_ml [8][8][2], red_acc [8][8][D/2]; CTA state after
+  // ---- merge the warps of this CTA: red_ml [8][8][2], red_acc [8][8][D/DP]; CTA state after
+  constexpr int DW = D / DP;                   // dims per part
   float* red_ml = reinterpret_cast<float*>(stage_mem);
   float* red_acc = red_ml + 8 * 8 * 2;
-  float* cst_ml = red_acc + 8 * 8 * (D / 2);   // [NQP][2]   (read by the cluster peers)
+  float* cst_ml = red_acc + 8 * 8 * DW;        // [NQP][2]   (read by the cluster peers)
   float* cst_acc = cst_ml + NQP * 2;           // [NQP][D]
   {
     const int c0 = 2 * (lane & 3);
@@ -655,27 +657,27 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 #pragma unroll
     for (int mt = 0; mt < KH; ++mt) {
       const int d0 = mt * 16 + (lane >> 2);
-      red_acc[(warp * 8 + c0) * (D / 2) + d0] = acc[mt][0];
-      red_acc[(warp * 8 + c0 + 1) * (D / 2) + d0] = acc[mt][1];
-      red_acc[(warp * 8 + c0) * (D / 2) + d0 + 8] = acc[mt][2];
-      red_acc[(warp * 8 + c0 + 1) * (D / 2) + d0 + 8] = acc[mt][3];
+      red_acc[(warp * 8 + c0) * DW + d0] = acc[mt][0];
+      red_acc[(warp * 8 + c0 + 1) * DW + d0] = acc[mt][1];
+      red_acc[(warp * 8 + c0) * DW + d0 + 8] = acc[mt][2];
+      red_acc[(warp * 8 + c0 + 1) * DW + d0 + 8] = acc[mt][3];
     }
   }
   __syncthreads();
   for (int e = tid; e < NQP * D; e += kSrThreads) {
     const int qr = e / D, dd = e % D;
-    const int hf = dd / (D / 2), ntq = qr >> 3, cq = qr & 7;
+    const int pe = dd / DW, ntq = qr >> 3, cq = qr & 7;
     float M = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t + 4 * hf) * 8 + cq) * 2]);
+    for (int t = 0; t < TG; ++t) M = fmaxf(M, red_ml[((pe + DP * (ntq + NT * t)) * 8 + cq) * 2]);
     float Ls = 0.f, A = 0.f;
 #pragma unroll
-    for (int t = 0; t < WT; ++t) {
-      const int w = ntq + NT * t + 4 * hf;
+    for (int t = 0; t < TG; ++t) {
+      const int w = pe + DP * (ntq + NT * t);
       const float mw = red_ml[(w * 8 + cq) * 2];
       const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
       Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
-      A += f * red_acc[(w * 8 + cq) * (D / 2) + (dd % (D / 2))];
+      A += f * red_acc[(w * 8 + cq) * DW + (dd % DW)];
     }
     cst_acc[qr * D + dd] = A;
     if (dd == 0) {

@@ -88,24 +88,48 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
     int* h = hist[pass & 1];
     if (tid < 256) h[tid] = 0;
     __syncthreads();
-    // Warp-aggregated counting: keys of one row share few leading digits (the top
-    // digit is sign + exponent), so lanes with the same bin add once per warp.
-    for (int base = lo + (tid & ~31); base < hi; base += kSelThreads) {
-      const int i = base + (tid & 31);
-      int bin = -1;
-      if (i < hi) {
-        const uint32_t k = key_at(i);
-        if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
+    if (p.keys_in_smem) {
+      // four keys per lane from shared memory; the first digit (sign + exponent) is shared by
+      // most keys and counted with warp aggregation, later digits directly
+      for (int b0 = (tid & ~31) * 4; b0 < hi - lo; b0 += kSelThreads * 4) {  // warp-uniform
+        const int i0 = b0 + 4 * (tid & 31);  // i0 + 3 < chunk: inside the keys region
+        const uint4 k4 = *reinterpret_cast<const uint4*>(skeys + i0);
+        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const bool in = (i0 + j < hi - lo) && ((kk[j] & pmask) == prefix);
+          const int bin = in ? (int)((kk[j] >> shift) & 255u) : -1;
+          if (pass == 0) {
+            const unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+          } else if (in) {
+            atomicAdd(&h[bin], 1);
+          }
+        }
       }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+    } else {
+      // scores re-read from L2: warp-aggregated counts
+      for (int base = lo + (tid & ~31); base < hi; base += kSelThreads) {
+        const int i = base + (tid & 31);
+        int bin = -1;
+        if (i < hi) {
+          const uint32_t k = key_at(i);
+          if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+      }
     }
     cluster.sync();
     // cluster-wide total of the bin that this thread scans, bins taken from the top down
     int tot = 0;
     if (tid < 256) {
       const int bin = 255 - tid;
-      for (int q = 0; q < CL; ++q) tot += cluster.map_shared_rank(h, q)[bin];
+      int v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) tot += v[q];
     }
     int total;
     const int above = block_exclusive_scan(tot, scan_scratch, &total);
