@@ -488,18 +488,17 @@ aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32
 
 bool select_rows_feasible(const aoh_kv_cache* kv) { return fused_candidate(kv, kSrMaxCluster, false).ok; }
 
-// The select stage of the three-kernel step.  Many rows: the smallest cluster whose slices
-// keep the row's keys in shared memory (one CTA per row up to 40960 keys), so nearly every
-// row selects in the same wave with few or no cluster barriers.  Few rows: the row kernel's
-// wider clusters.
+// The select stage of the three-kernel step: the row kernel's cluster select on the scores;
+// rows longer than its clusters take the select kernel with the smallest cluster that keeps
+// each slice's keys in shared memory.
 aoh_status select_stage(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
                         int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
                         cudaStream_t st) {
   const int64_t rows = int64_t(kv->batch) * n_listed;
   int cl = 1;
   while (cl < kSelMaxCluster && ceil_div(std::max(kv->max_len, 1), cl) > 40960) cl *= 2;
-  if (rows >= kSmCount / 2 || !select_rows_feasible(kv))
-    return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st, cl);
+  (void)rows;
+  if (!select_rows_feasible(kv)) return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st, cl);
   return launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
 }
 
