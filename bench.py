@@ -62,15 +62,17 @@ def algorithmic_bytes(w) -> dict:
     d = sp.head_dim
     L = w.lengths.astype(np.int64)
     roles = w.roles.numpy()
-    out = {"tip": 0, "fac": 0, "window": 0, "indexer": 0, "gather": 0}
+    out = {"tip": 0, "fac": 0, "window": 0, "indexer": 0, "gather": 0, "select": 0}
     if sp.n_layers > 0:
         out["indexer"] = int(L.sum()) * sp.n_kv_heads * d * 2
         out["gather"] = int(np.minimum(L, sp.topk_shared).sum()) * sp.n_kv_heads * 4 * d
+        out["select"] = int(L.sum()) * sp.n_kv_heads * 4
     else:
         n_sparse = int((roles == ROLE_SPARSE).sum())
         nfac = w.n_fac_per_seq.numpy().astype(np.int64)
         out["tip"] = int(L.sum()) * n_sparse * 4 * sp.n_dom
         out["fac"] = int(np.minimum(L, nfac).sum()) * n_sparse * 4 * d
+        out["select"] = int(L.sum()) * n_sparse * 4
         for g, r in enumerate(roles):
             if r == 1:
                 out["window"] += int(L.sum()) * 4 * d
@@ -78,7 +80,8 @@ def algorithmic_bytes(w) -> dict:
                 a = np.minimum(L, sp.sink)
                 n = a + (L - np.maximum(a, L - sp.window))
                 out["window"] += int(n.sum()) * 4 * d
-    out["total"] = sum(v for k, v in out.items())
+    # the scores the select reads are an intermediate of the three-kernel form, not step traffic
+    out["total"] = sum(v for k, v in out.items() if k != "select")
     return out
 
 
@@ -177,33 +180,10 @@ def build_step(w, dev):
     return step, (w.q.to(dev),)
 
 
-KERNEL_OF_CALL = {"sparse_decode": "sparse_row_kernel", "shared_index_step": "sparse_row_kernel",
-                  "stream_decode": "flash_gather_kernel"}
-FUSED_MAX_LEN = 16 * 16384  # rows up to this length run as one cluster kernel (library rule)
-
-
-def launches_per_step(w) -> int:
-    if w.spec.n_layers > 0:
-        return 1  # fused shared-index step
-    roles = w.roles.numpy()
-    n = 0
-    if (roles == ROLE_SPARSE).any():
-        n += 1 if w.max_len <= FUSED_MAX_LEN else 3  # fused row kernel, or scan + select + attend
-    if (roles != ROLE_SPARSE).any():
-        n += 1    # window attention
-    return n
-
-
-def stage_timing(w, step, q, steps: int, flush) -> dict:
-    """Device time of each public call of the step (CUDA events on the launching stream).
-
-    Each sample runs behind a short device-side sleep so that the host has queued
-    the calls before the first one starts: the events then time the kernels, not the
-    host's launch latency.  L2 is flushed before every sample.
-    """
+def step_calls(w, step, q):
+    """The public calls one step makes, by name (the same arguments as the step)."""
     from token_sparse_decode_b200 import binding as B
 
-    st = torch.cuda.current_stream()
     calls = []
     if w.spec.n_layers > 0:
         calls.append(("shared_index_step", lambda: step(*q)))
@@ -215,22 +195,68 @@ def stage_timing(w, step, q, steps: int, flush) -> dict:
         if step.has_stream:
             calls.append(("stream_decode", lambda: B.stream_decode(
                 q[0], step.kv, step.roles, step.sink, step.window, step.scale, step.out, step.ws_stream)))
+    return calls
+
+
+def launches_per_step(step, q) -> dict:
+    """Kernels one eager step launches, by kernel name (the library's launch counters)."""
+    from token_sparse_decode_b200 import binding as B
+
+    c0 = B.launch_counts()
+    step(*q)
+    torch.cuda.synchronize()
+    c1 = B.launch_counts()
+    return {k: c1[k] - c0[k] for k in c0 if c1[k] != c0[k]}
+
+
+def kernel_timing(w, step, q, steps: int, flush) -> dict:
+    """Device time of every kernel of the step, per public call.
+
+    Each call runs with the library's launch-event recording armed, so every kernel is
+    bracketed by CUDA events recorded on its own stream right before and after it.  Each
+    sample runs behind a device-side sleep, so that the host has queued the calls before
+    the first one starts; L2 is flushed before every sample.
+    """
+    from token_sparse_decode_b200 import binding as B
+
+    calls = step_calls(w, step, q)
     for _, fn in calls:
         fn()
     torch.cuda.synchronize()
-    times = {n: [] for n, _ in calls}
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in calls]
+    per, call_ms, order = {}, {n: [] for n, _ in calls}, {}
     for _ in range(steps):
         flush()
-        torch.cuda._sleep(200000)
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-        evs[0].record(st)
-        for i, (_, fn) in enumerate(calls):
-            fn()
-            evs[i + 1].record(st)
+        torch.cuda._sleep(1000000)
+        recs = [(name, B.timed_launches(fn, evs)) for (name, fn), evs in zip(calls, evsets)]
         torch.cuda.synchronize()
-        for i, (n, _) in enumerate(calls):
-            times[n].append(evs[i].elapsed_time(evs[i + 1]))
-    return {n: float(np.mean(t)) for n, t in times.items()}
+        for name, r in recs:
+            order[name] = [k for k, _, _ in r]
+            for i, (kern, e0, e1) in enumerate(r):
+                per.setdefault((name, i, kern), []).append(e0.elapsed_time(e1))
+            if r:
+                call_ms[name].append(r[0][1].elapsed_time(r[-1][2]))
+    kernels = [{"call": n, "index": i, "kernel": k, "ms": float(np.mean(t))} for (n, i, k), t in sorted(per.items())]
+    return {"calls": {n: float(np.mean(t)) for n, t in call_ms.items() if t}, "kernels": kernels, "order": order}
+
+
+def kernel_bytes(w, ab: dict, call: str, kernel: str, order: list) -> int:
+    """Algorithmic bytes one launch of `kernel` moves inside `call` (see algorithmic_bytes).
+
+    A call that launches the row kernel alone runs the whole path in it; in the three-kernel
+    form the scan reads the score columns, the select reads the fp32 scores (4 bytes per token
+    and scored KV head) and the gather reads the selected K / V rows.
+    """
+    fused = order == ["sparse_row_kernel"]
+    if call == "stream_decode":
+        return ab["window"]
+    if call == "shared_index_step":
+        if fused:
+            return ab["indexer"] + ab["gather"]
+        return {"tip_score_kernel": ab["indexer"], "flash_gather_kernel": ab["gather"]}.get(kernel, ab["select"])
+    if fused:
+        return ab["tip"] + ab["fac"]
+    return {"tip_score_kernel": ab["tip"], "flash_gather_kernel": ab["fac"]}.get(kernel, ab["select"])
 
 
 def capture_graph(fn):
@@ -285,6 +311,7 @@ def run_ours(args, rank, world, local_rank):
 
     step(*q)  # first call outside capture (sets kernel attributes)
     torch.cuda.synchronize()
+    per_step = launches_per_step(step, q)
     if args.graph:
         g_step = capture_graph(lambda: step(*q))
         one = g_step.replay
@@ -347,7 +374,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_ms += e0.elapsed_time(e1)
         flush()
 
-    stages = stage_timing(w, step, q, args.steps if args.steps <= 200 else 200, flush)
+    kt = kernel_timing(w, step, q, args.steps if args.steps <= 200 else 200, flush)
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
@@ -357,11 +384,10 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = aggregate_throughput(tokens_step, world, e2e_ms / args.steps)
     ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_gbs()
-    call_bytes = {"shared_index_step": ab["indexer"] + ab["gather"], "sparse_decode": ab["tip"] + ab["fac"],
-                  "stream_decode": ab["window"]}
-    dom = max(stages, key=lambda k: stages[k]) if stages else None
-    dom_bytes = call_bytes.get(dom, 0)
-    dom_ms = stages.get(dom)
+    # the dominant kernel: the largest device time of one step
+    dom = max(kt["kernels"], key=lambda e: e["ms"]) if kt["kernels"] else None
+    dom_bytes = kernel_bytes(w, ab, dom["call"], dom["kernel"], kt["order"][dom["call"]]) if dom else 0
+    dom_ms = dom["ms"] if dom else None
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms else None
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     return {
@@ -388,13 +414,18 @@ def run_ours(args, rank, world, local_rank):
         },
         "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
                      "bytes_per_step": ab["total"]},
-        "roofline": {"kernel": KERNEL_OF_CALL.get(dom, dom), "call": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        "roofline": {"kernel": dom["kernel"] if dom else None, "call": dom["call"] if dom else None, "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "peak_source": peak_kind,
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
-                     "traffic": ncu_traffic(w.spec.name, dom)},
-        "stage_ms": stages,
+                     "traffic": ncu_traffic(w.spec.name, dom["kernel"]) if dom else None},
+        "call_ms": kt["calls"],
+        "kernel_ms": [{"call": e["call"], "kernel": e["kernel"], "ms": e["ms"],
+                       "bytes": kernel_bytes(w, ab, e["call"], e["kernel"], kt["order"][e["call"]])}
+                      for e in kt["kernels"]],
+        "launches_per_step": per_step,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step(w) * args.steps,
+        "gpu_launches": sum(per_step.values()) * args.steps,
         "clocks": clocks,
         "_w": w,
     }

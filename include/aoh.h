@@ -110,6 +110,39 @@ int32_t aoh_version(void);
  * host thread (0 if none); cudaGetErrorString() names it. */
 int32_t aoh_last_cuda_error(void);
 
+/* Kernels the library launches, one counter each (see aoh_launch_counts). */
+typedef enum {
+  AOH_KERNEL_TIP_SCORE = 0,     /* stand-alone importance scan                       */
+  AOH_KERNEL_TOPK_SELECT = 1,   /* stand-alone cluster select (rows beyond the row kernel) */
+  AOH_KERNEL_SPARSE_ROW = 2,    /* fused row kernel, or its select-only form         */
+  AOH_KERNEL_FLASH_GATHER = 3,  /* split-K gather / window attention                 */
+  AOH_KERNEL_PACK_DOMINANT = 4, /* dominant-column packing of K                      */
+  AOH_KERNEL_KINDS = 5
+} aoh_kernel_kind;
+
+/*
+ * aoh_launch_counts -- kernel launches this process has made through the
+ * library, by kernel.  Host-side counters, incremented at every launch the
+ * runtime accepted (a launch captured into a CUDA graph counts once, at
+ * capture; graph replays do not count).  Writes min(n, AOH_KERNEL_KINDS)
+ * host int64 to `counts` (may be NULL when n is 0); returns AOH_KERNEL_KINDS.
+ * Differences of two readings around a call give that call's launches.
+ */
+int32_t aoh_launch_counts(int64_t* counts, int32_t n);
+
+/*
+ * aoh_record_launch_events -- diagnostic timing of the kernels inside a call.
+ * While armed (events not NULL), the next launch records events[0] on its
+ * stream just before it, and launch i (1-based) records events[i] just after
+ * it and writes its aoh_kernel_kind to kinds[i - 1], for i < n; later
+ * launches record nothing.  cudaEventElapsedTime(events[i - 1], events[i])
+ * is then the device time of launch i.  `events`: host array of n
+ * cudaEvent_t created by the caller; `kinds`: host int32[n - 1] or NULL.
+ * Both must stay valid until the call is repeated with events = NULL, which
+ * disarms it.  Process-wide and not thread-safe: for measurement only.
+ */
+void aoh_record_launch_events(void** events, int32_t* kinds, int32_t n);
+
 /*
  * aoh_device_check -- synchronise `stream`, then read and clear this
  * device's error word.  Returns AOH_OK, AOH_ERR_DEVICE_CHECK (and, if

@@ -111,6 +111,21 @@ def compare_window_row(w, b, g, gpu_out, role, sink, window):
     return err
 
 
+def launches_of(fn) -> dict:
+    """Kernels fn() launched through the library, by name (the library's launch counters)."""
+    c0 = B.launch_counts()
+    fn()
+    torch.cuda.synchronize()
+    c1 = B.launch_counts()
+    return {k: c1[k] - c0[k] for k in c0 if c1[k] != c0[k]}
+
+
+def three_kernel_form(launches: dict) -> bool:
+    """scan + select (the row kernel's select-only form or the select kernel) + gather"""
+    sel = launches.get("sparse_row_kernel", 0) + launches.get("topk_select_kernel", 0)
+    return launches.get("tip_score_kernel") == 1 and sel == 1 and launches.get("flash_gather_kernel") == 1
+
+
 def run_sparse(d: Dev, pack=True):
     w = d.w
     step = SparseDecodeStep(d.k, d.v, d.offsets, d.max_len, d.T, w.spec.n_q_heads, w.roles.tolist(), w.scale,

@@ -45,6 +45,22 @@ def test_version_and_status_strings(lib):
     assert lib.aoh_status_string(99) == b"unknown status"
 
 
+def test_launch_counters_are_host_side(lib):
+    # the kernel-kind enum of the header and the binding's names agree, and the counters
+    # read without a device; host validation failures launch nothing
+    text = open(HEADER).read()
+    kinds = re.findall(r"AOH_KERNEL_([A-Z_]+) = (\d+)", text)
+    named = {k.lower(): int(v) for k, v in kinds if k != "KINDS"}
+    assert [f"{k}_kernel" for k, _ in sorted(named.items(), key=lambda kv: kv[1])] == list(B.KERNELS)
+    before = B.launch_counts()
+    assert set(before) == set(B.KERNELS) and all(v >= 0 for v in before.values())
+    assert lib.aoh_launch_counts(None, 0) == len(B.KERNELS)
+    kv = B.KVCache()
+    kv.batch, kv.n_kv_heads, kv.head_dim = 1, 1, 96  # unsupported head_dim: refused on the host
+    assert lib.aoh_tip_score(None, 1, ctypes.byref(kv), None, 1, None, None) == 2
+    assert B.launch_counts() == before
+
+
 def test_struct_layout_matches_header():
     src = r"""
     #include <stdio.h>

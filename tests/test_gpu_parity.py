@@ -12,7 +12,8 @@ import torch
 
 import oracle
 from gpu_helpers import (OUT_ATOL, SCORE_REL, Dev, check_device, compare_sparse_row, compare_window_row, f64,
-                         row_inputs, run_shared, run_sparse, score_bound, band_swap_bound)
+                         launches_of, row_inputs, run_shared, run_sparse, score_bound, band_swap_bound,
+                         three_kernel_form)
 from token_sparse_decode_b200 import binding as B
 from workloads import ROLE_DENSE, ROLE_SPARSE, ROLE_STREAM, WorkloadSpec, make_workload
 
@@ -157,6 +158,8 @@ def test_sparse_decode_matches_oracle(name, pack):
     w = make_workload(MEDIUM[name])
     d = Dev(w)
     step, out = run_sparse(d, pack=pack)
+    # a few rows: the whole path in one cluster launch
+    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
     G = w.spec.group
@@ -296,6 +299,7 @@ def test_sparse_decode_long_row_uses_three_kernels():
     w = make_workload(sp)
     d = Dev(w)
     step, out = run_sparse(d)
+    assert three_kernel_form(launches_of(lambda: step(d.q)))
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
     compare_sparse_row(w, 0, 0, idx_h[0, 0, :cnt_h[0, 0]], out_h[0, 0:2])
@@ -322,6 +326,15 @@ def test_sparse_decode_many_rows_runs_three_stages():
     w = make_workload(sp)
     d = Dev(w)
     step, out = run_sparse(d)
+    assert three_kernel_form(launches_of(lambda: step(d.q)))
+    # the same call with launch events armed: three kernels, in path order, each timed
+    rec = B.timed_launches(lambda: B.sparse_decode(d.q, step.kv, step.idom, step.n_dom, step.n_fac,
+                                                   step.n_fac_per_seq, step.n_fac_cap, step.roles, step.scale,
+                                                   step.out, step.ws_sparse, step.idx, step.count))
+    torch.cuda.synchronize()
+    names = [k for k, _, _ in rec]
+    assert names[0] == "tip_score_kernel" and names[-1] == "flash_gather_kernel" and len(names) == 3
+    assert all(e0.elapsed_time(e1) > 0 for _, e0, e1 in rec)
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
     G = sp.group
@@ -338,6 +351,7 @@ def test_shared_index_step_many_rows_runs_three_stages():
     w = make_workload(sp)
     d = Dev(w)
     step, out = run_shared(d, fused=True)
+    assert three_kernel_form(launches_of(lambda: step(d.q, d.q_layers)))
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
     G = sp.group

@@ -26,7 +26,12 @@ EXPORTS = (
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
     "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
+    "aoh_launch_counts", "aoh_record_launch_events",
 )
+
+# aoh_kernel_kind order
+KERNELS = ("tip_score_kernel", "topk_select_kernel", "sparse_row_kernel", "flash_gather_kernel",
+           "pack_dominant_kernel")
 
 
 class AohError(RuntimeError):
@@ -65,6 +70,8 @@ def lib() -> ctypes.CDLL:
             "aoh_version": (I32, []),
             "aoh_last_cuda_error": (I32, []),
             "aoh_device_check": (ctypes.c_int, [P, P]),
+            "aoh_launch_counts": (I32, [P, I32]),
+            "aoh_record_launch_events": (None, [P, P, I32]),
             "aoh_pack_dominant": (ctypes.c_int, [KVP, P, I32, P, I32, P]),
             "aoh_tip_score": (ctypes.c_int, [P, I32, KVP, P, I32, P, P]),
             "aoh_topk_select": (ctypes.c_int, [P, KVP, I32, P, I32, P, P, P]),
@@ -144,6 +151,47 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 
 # ---------------------------------------------------------------------------- entry points
+
+def launch_counts() -> dict:
+    """Kernel launches made through the library so far, by kernel name (host counters)."""
+    n = len(KERNELS)
+    buf = (ctypes.c_int64 * n)()
+    kinds = lib().aoh_launch_counts(ctypes.cast(buf, ctypes.c_void_p), n)
+    if kinds != n:
+        raise AohError("aoh_launch_counts", 1)
+    return {name: int(buf[i]) for i, name in enumerate(KERNELS)}
+
+
+def timed_launches(fn, events=None, max_launches: int = 8):
+    """Run fn() (one library call) with launch-event recording armed.
+
+    Returns [(kernel name, start event, end event)] for the kernels fn() launched, in
+    launch order; the events are recorded on each launch's stream, so elapsed_time of a
+    pair (after a synchronize) is that kernel's device time.  `events` (max_launches + 1
+    timing events) may be passed in to be reused.
+    """
+    n = max_launches + 1
+    evs = events if events is not None else [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    if len(evs) != n:
+        raise ValueError("timed_launches: need max_launches + 1 events")
+    for ev in evs:
+        if not ev.cuda_event:  # created on first record
+            ev.record()
+    handles = (ctypes.c_void_p * n)(*[ev.cuda_event for ev in evs])
+    kinds = (ctypes.c_int32 * max_launches)(*([-1] * max_launches))
+    L = lib()
+    L.aoh_record_launch_events(ctypes.cast(handles, ctypes.c_void_p), ctypes.cast(kinds, ctypes.c_void_p), n)
+    try:
+        fn()
+    finally:
+        L.aoh_record_launch_events(None, None, 0)
+    out = []
+    for i in range(max_launches):
+        if kinds[i] < 0:
+            break
+        out.append((KERNELS[kinds[i]], evs[i], evs[i + 1]))
+    return out
+
 
 def device_check(stream=None):
     detail = (ctypes.c_int32 * 4)()

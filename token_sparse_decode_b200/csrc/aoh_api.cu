@@ -1,12 +1,12 @@
 // C ABI of the token-sparse decode step: argument checks on the host, then
 // asynchronous launches on the caller's stream.  Declarations and the contract
 // of every entry point are in include/aoh.h.
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -23,8 +23,6 @@ namespace {
 
 constexpr int kSmCount = 148;        // B200
 constexpr int kMaxQRows = 32;        // query rows per KV head in one gather kernel (4 n-tiles)
-constexpr int kSelMaxCluster = 8;    // portable cluster size
-constexpr size_t kSelSmemCap = 200 * 1024;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -56,10 +54,41 @@ aoh_status check_heads(const aoh_kv_cache* kv, int32_t n_q_heads) {
 
 thread_local int t_last_cuda_error = 0;
 
+
 aoh_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return AOH_OK;
   t_last_cuda_error = (int)e;
   return AOH_ERR_CUDA;
+}
+
+std::atomic<int64_t> g_launches[AOH_KERNEL_KINDS];
+
+// aoh_record_launch_events state: events[0] before the first launch, events[i] after launch i
+struct LaunchEvents {
+  cudaEvent_t* ev = nullptr;
+  int32_t* kinds = nullptr;
+  int n = 0;
+  int next = 0;
+};
+LaunchEvents g_ev;
+
+void before_launch(cudaStream_t st) {
+  if (g_ev.ev && g_ev.next == 0 && g_ev.n > 1) {
+    cudaEventRecord(g_ev.ev[0], st);
+    g_ev.next = 1;
+  }
+}
+
+// status of the launch just made on `st`; counts it under `kind` when the runtime accepted it
+aoh_status count_launch(aoh_kernel_kind kind, cudaStream_t st) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e);
+  g_launches[kind].fetch_add(1, std::memory_order_relaxed);
+  if (g_ev.ev && g_ev.next > 0 && g_ev.next < g_ev.n) {
+    if (g_ev.kinds) g_ev.kinds[g_ev.next - 1] = kind;
+    cudaEventRecord(g_ev.ev[g_ev.next++], st);
+  }
+  return AOH_OK;
 }
 
 // Opt in to `bytes` of dynamic shared memory.  Always set: static shared memory
@@ -124,8 +153,9 @@ aoh_status launch_fd_t(const FdecParams& fp, int n_listed, int B, cudaStream_t s
     configured = true;
   }
   dim3 grid(fp.max_splits, n_listed, B);
+  before_launch(st);
   flash_gather_kernel<D, NT><<<grid, kFdThreads, smem, st>>>(fp);
-  return cuda_status(cudaGetLastError());
+  return count_launch(AOH_KERNEL_FLASH_GATHER, st);
 }
 
 aoh_status launch_fd(const FdecParams& fp, int d, int nqp, int n_listed, int B, cudaStream_t st) {
@@ -140,6 +170,24 @@ aoh_status launch_fd(const FdecParams& fp, int d, int nqp, int n_listed, int B, 
 }
 
 // ------------------------------------------------------------------ TIP scan
+template <int S>
+aoh_status launch_tip_t(TipParams& tp, cudaStream_t st) {
+  static int per_sm = 0;  // resident CTAs per SM (cached per process)
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tip_score_kernel<S>, kTipThreads, 0) != cudaSuccess ||
+        per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+  }
+  const int64_t resident = int64_t(kSmCount) * per_sm;
+  tp.per_cta = std::max<int64_t>(256, ceil_div(tp.total, resident));
+  const int64_t grid = ceil_div(tp.total, tp.per_cta);
+  before_launch(st);
+  tip_score_kernel<S><<<(unsigned)grid, kTipThreads, 0, st>>>(tp);
+  return count_launch(AOH_KERNEL_TIP_SCORE, st);
+}
+
 aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom,
                       float* scores, const uint8_t* heads, int n_listed, cudaStream_t st) {
   TipParams tp{};
@@ -153,8 +201,9 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
   tp.d = kv->head_dim;
   tp.G = Hq / kv->n_kv_heads;
   tp.n_dom = n_dom;
-  if (kv->k_dom && idom) {
-    if (2 * n_dom > kv->k_dom_cols) return AOH_ERR_INVALID_ARG;
+  const bool packed = kv->k_dom && idom;
+  if (packed && 2 * n_dom > kv->k_dom_cols) return AOH_ERR_INVALID_ARG;
+  if (packed) {
     tp.src = static_cast<const uint16_t*>(kv->k_dom);
     tp.row_stride_tok = kv->k_dom_cols;
     tp.row_stride_head = kv->total_tokens * kv->k_dom_cols;
@@ -168,21 +217,18 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
     tp.packed = 0;
   }
   memcpy(tp.heads, heads, n_listed);
-  const int64_t rows = int64_t(kv->batch) * n_listed;
-  int64_t tile = ceil_div(std::max<int64_t>(1, int64_t(kv->max_len) * rows), int64_t(kSmCount) * 6);
-  tile = std::min<int64_t>(std::max<int64_t>(ceil_div(tile, 256) * 256, 256), 8192);
-  tp.tile = (int32_t)tile;
-  dim3 grid((unsigned)std::max<int64_t>(1, ceil_div(kv->max_len, tile)), n_listed, kv->batch);
+  tp.B = kv->batch;
+  tp.total = int64_t(n_listed) * kv->total_tokens;
+  if (tp.total == 0) return AOH_OK;
   int lanes = 1;
   while (lanes * 8 < tp.row_len) lanes <<= 1;
   switch (lanes) {
-    case 1: tip_score_kernel<1><<<grid, kTipThreads, 0, st>>>(tp); break;
-    case 2: tip_score_kernel<2><<<grid, kTipThreads, 0, st>>>(tp); break;
-    case 4: tip_score_kernel<4><<<grid, kTipThreads, 0, st>>>(tp); break;
-    case 8: tip_score_kernel<8><<<grid, kTipThreads, 0, st>>>(tp); break;
-    default: tip_score_kernel<16><<<grid, kTipThreads, 0, st>>>(tp); break;
+    case 1: return launch_tip_t<1>(tp, st);
+    case 2: return launch_tip_t<2>(tp, st);
+    case 4: return launch_tip_t<4>(tp, st);
+    case 8: return launch_tip_t<8>(tp, st);
+    default: return launch_tip_t<16>(tp, st);
   }
-  return cuda_status(cudaGetLastError());
 }
 
 // Full-dimension scores (every chunk; the shared indexer's score), K read in place.
@@ -192,11 +238,10 @@ aoh_status launch_tip_full(const void* q, int32_t Hq, const aoh_kv_cache* kv, fl
 }
 
 // ------------------------------------------------------------------ top-k select
-// The select kernel with `cl` CTAs per row (1: one CTA reads the row's scores from L2
-// and takes no cluster barrier; up to 8: a cluster shares the row).
+// The streaming select kernel: one CTA per row, scores read from L2.
 aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
                          int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
-                         cudaStream_t st, int cl = 0) {
+                         cudaStream_t st) {
   SelectParams sp{};
   sp.scores = scores;
   sp.offsets = kv->offsets;
@@ -208,43 +253,29 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
   sp.n_fac = n_fac;
   sp.cap = cap;
   memcpy(sp.heads, heads, n_listed);
-  const int CL = cl > 0 ? std::min(cl, kSelMaxCluster)
-                        : (int)std::min<int64_t>(kSelMaxCluster, std::max<int64_t>(1, ceil_div(kv->max_len, 256)));
-  const int64_t chunk = std::max<int64_t>(4, ceil_div(ceil_div(std::max(kv->max_len, 1), CL), 4) * 4);
-  sp.chunk = (int32_t)chunk;
-  size_t smem = (size_t)chunk * 4;
-  sp.keys_in_smem = smem <= kSelSmemCap;
-  if (!sp.keys_in_smem) smem = 0;
-  static size_t configured = 0;
-  if (smem > configured) {
-    aoh_status s = set_smem(topk_select_kernel, kSelSmemCap);
+  const size_t smem = size_t(kSelCandCap) * 4;
+  static bool configured = false;
+  if (!configured) {
+    aoh_status s = set_smem(topk_select_kernel, smem);
     if (s != AOH_OK) return s;
-    configured = kSelSmemCap;
+    configured = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CL, n_listed, kv->batch);
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, topk_select_kernel, sp));
+  before_launch(st);
+  topk_select_kernel<<<dim3(n_listed, kv->batch), kSelThreads, smem, st>>>(sp);
+  return count_launch(AOH_KERNEL_TOPK_SELECT, st);
 }
 
 
 // ------------------------------------------------------------------ fused row kernel
-// Shared memory per CTA: keys of the slice, then a ring of 16 KB stages used by the
-// scan and then by the attention.  Two CTAs per SM when the keys leave room for a
-// ring of >= 64 KB in 108 KB, else one CTA per SM with up to 128 KB of ring.
+// Shared memory per CTA: keys of the slice, then a ring region used by the scan's
+// per-warp cp.async rings (64 KB) and then by the attention stages.  Two CTAs per SM
+// when the keys leave room for a ring of >= 64 KB in 108 KB, else one CTA per SM with
+// up to 128 KB of ring (sized in 16 KB steps).
 constexpr size_t kTwoPerSm = 108 * 1024;
 constexpr size_t kOnePerSm = 220 * 1024;
-constexpr size_t kRingMin = 4 * kSrRingStage;
-constexpr size_t kRingMax = kSrMaxStages * kSrRingStage;
+constexpr size_t kRingStep = 16 * 1024;
+constexpr size_t kRingMin = kSrRingMin;
+constexpr size_t kRingMax = 8 * kRingStep;
 
 struct FusedPlan {
   bool ok;
@@ -257,7 +288,17 @@ struct FusedPlan {
 int g_force_cluster = 0;  // diagnostic build: force the fused kernel's cluster size ...
 int g_force_ring = 0;     // ... cap its ring (bytes) ...
 int g_force_one_per_sm = 0;  // ... or give one CTA per SM the whole budget
+int g_force_three = 0;       // ... or take the three-kernel form
+int g_select_rows = 0;       // ... with the row kernel's cluster select
 #endif
+
+bool allow_fused() {
+#ifdef AOH_PHASE_TIMERS
+  return !g_force_three;
+#else
+  return true;
+#endif
+}
 
 FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true) {
   FusedPlan f{};
@@ -276,7 +317,7 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   if (g_force_one_per_sm) budget = kOnePerSm - 1024;
 #endif
   if (f.keys_bytes + ring_min > budget) return f;
-  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kSrRingStage * kSrRingStage) : f.keys_bytes;
+  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kRingStep * kRingStep) : f.keys_bytes;
 #ifdef AOH_PHASE_TIMERS
   if (need_ring && g_force_ring) f.ring_bytes = std::min(f.ring_bytes, (size_t)g_force_ring);
 #endif
@@ -285,68 +326,15 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   return f;
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// cuTensorMapEncodeTiled, resolved through the runtime (no link against the driver library)
-EncodeTiledFn encode_tiled() {
-  static const EncodeTiledFn fn = [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return (EncodeTiledFn) nullptr;
-    }
-    return reinterpret_cast<EncodeTiledFn>(ptr);
-  }();
-  return fn;
-}
-
-// The scan reads its rows through a 2-D tensor map: packed rows as [Hkv * T][cols]; K in
-// place as [T][stride_tok] with the head at column g * stride_head (needs every head's
-// row inside one token stride).
-bool scan_layout_ok(const aoh_kv_cache* kv, bool packed) {
-  if (packed) return true;
-  return int64_t(kv->n_kv_heads - 1) * kv->stride_head + kv->head_dim <= kv->stride_tok;
-}
-
-aoh_status make_scan_map(RowParams& rp, const aoh_kv_cache* kv) {
-  const EncodeTiledFn enc = encode_tiled();
-  if (!enc) return AOH_ERR_CUDA;
-  const int box = std::min(rp.srow_len, 64);
-  const int rows = std::min(256, kSrRingStage / (rp.srow_len * 2));
-  rp.scan_box = box;
-  rp.scan_rows = rows;
-  cuuint64_t dims[2], strides[1];
-  if (rp.packed) {
-    dims[0] = (cuuint64_t)kv->k_dom_cols;
-    dims[1] = (cuuint64_t)kv->n_kv_heads * (cuuint64_t)kv->total_tokens;
-    strides[0] = (cuuint64_t)kv->k_dom_cols * 2;
-  } else {
-    dims[0] = (cuuint64_t)kv->stride_tok;
-    dims[1] = (cuuint64_t)kv->total_tokens;
-    strides[0] = (cuuint64_t)kv->stride_tok * 2;
-  }
-  const cuuint32_t boxd[2] = {(cuuint32_t)box, (cuuint32_t)rows};
-  const cuuint32_t es[2] = {1, 1};
-  const CUtensorMapSwizzle sw = box * 2 == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                : box * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                : CU_TENSOR_MAP_SWIZZLE_128B;
-  const CUresult r = enc(&rp.tmap_scan, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(rp.score_src), dims,
-                         strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? AOH_OK : AOH_ERR_CUDA;
-}
-
+// The fused scan shares a row among cols / 8 lanes: a power of two from 16 columns.
 bool packed_scan(const aoh_kv_cache* kv, const int32_t* idom) {
-  return kv->k_dom && idom && (kv->k_dom_cols % 16) == 0;
+  const int c = kv->k_dom_cols;
+  return kv->k_dom && idom && c >= 16 && (c & (c - 1)) == 0;
 }
 
 // Whether some cluster size handles these rows in one fused launch.
-bool fused_feasible(const aoh_kv_cache* kv, int nq, bool packed) {
-  return nq <= kMaxQRows && scan_layout_ok(kv, packed) && fused_candidate(kv, kSrMaxCluster).ok;
+bool fused_feasible(const aoh_kv_cache* kv, int nq) {
+  return nq <= kMaxQRows && fused_candidate(kv, kSrMaxCluster).ok;
 }
 
 
@@ -424,10 +412,6 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   }
   if (!best.ok) return AOH_ERR_UNSUPPORTED;
   if (max_waves > 0 && best_waves > max_waves) return AOH_OK;
-  if (need_ring && !rp.scores_in) {
-    const aoh_status ms = make_scan_map(rp, kv);
-    if (ms != AOH_OK) return ms;
-  }
   rp.keys_bytes = (int32_t)best.keys_bytes;
   rp.ring_bytes = (int32_t)best.ring_bytes;
   cudaLaunchConfig_t cfg = {};
@@ -442,7 +426,9 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const aoh_status s = cuda_status(cudaLaunchKernelEx(&cfg, kern, rp));
+  before_launch(st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, rp);
+  const aoh_status s = e != cudaSuccess ? cuda_status(e) : count_launch(AOH_KERNEL_SPARSE_ROW, st);
   *launched = (s == AOH_OK);
   return s;
 }
@@ -494,12 +480,16 @@ bool select_rows_feasible(const aoh_kv_cache* kv) { return fused_candidate(kv, k
 aoh_status select_stage(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
                         int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
                         cudaStream_t st) {
+  // Rows enough to fill the SMs: one CTA per row.  Fewer, longer rows: the row kernel's
+  // cluster select, which spreads each row over a cluster's shared memory.
   const int64_t rows = int64_t(kv->batch) * n_listed;
-  int cl = 1;
-  while (cl < kSelMaxCluster && ceil_div(std::max(kv->max_len, 1), cl) > 40960) cl *= 2;
-  (void)rows;
-  if (!select_rows_feasible(kv)) return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st, cl);
-  return launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
+  bool rows_kernel = rows < kSmCount && select_rows_feasible(kv);
+#ifdef AOH_PHASE_TIMERS
+  if (g_select_rows == 1) rows_kernel = select_rows_feasible(kv);
+  if (g_select_rows == 2) rows_kernel = false;
+#endif
+  if (rows_kernel) return launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
+  return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
 }
 
 // Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,
@@ -606,6 +596,18 @@ int32_t aoh_version(void) { return 1; }
 
 int32_t aoh_last_cuda_error(void) { return t_last_cuda_error; }
 
+void aoh_record_launch_events(void** events, int32_t* kinds, int32_t n) {
+  g_ev.ev = reinterpret_cast<cudaEvent_t*>(events);
+  g_ev.kinds = kinds;
+  g_ev.n = events ? n : 0;
+  g_ev.next = 0;
+}
+
+int32_t aoh_launch_counts(int64_t* counts, int32_t n) {
+  for (int i = 0; i < n && i < AOH_KERNEL_KINDS && counts; ++i) counts[i] = g_launches[i].load(std::memory_order_relaxed);
+  return AOH_KERNEL_KINDS;
+}
+
 aoh_status aoh_device_check(void* stream, int32_t* detail) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return AOH_ERR_CUDA;
   int h[4] = {0, 0, 0, 0};
@@ -639,8 +641,9 @@ aoh_status aoh_pack_dominant(const aoh_kv_cache* kv, const int32_t* idom, int32_
   pp.cols = k_dom_cols;
   const int64_t total = int64_t(pp.Hkv) * pp.T * pp.cols;
   const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), int64_t(kSmCount) * 16);
+  before_launch(as_stream(stream));
   pack_dominant_kernel<<<blocks, 256, 0, as_stream(stream)>>>(pp);
-  return cuda_status(cudaGetLastError());
+  return count_launch(AOH_KERNEL_PACK_DOMINANT, as_stream(stream));
 }
 
 aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv, const int32_t* idom,
@@ -667,9 +670,7 @@ aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t 
   if (!idx || !count || (!scores && kv->total_tokens > 0)) return AOH_ERR_INVALID_ARG;
   uint8_t heads[kMaxHeads];
   const int n = list_heads(kv, nullptr, true, heads);
-  if (select_rows_feasible(kv))
-    return launch_select_rows(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
-  return launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
+  return select_stage(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
 }
 
 size_t aoh_sparse_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, int32_t n_fac_cap) {
@@ -710,7 +711,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + off_idx);
   int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + off_count);
 
-  if (fused_feasible(kv, G, packed_scan(kv, idom))) {
+  if (allow_fused() && fused_feasible(kv, G)) {
     RowParams rp{};
     rp.q_score = static_cast<const uint16_t*>(q);
     rp.q_attn = static_cast<const uint16_t*>(q);
@@ -902,7 +903,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const FdGeom geo = shared_geom(kv, n_layers, n_q_heads, topk);
   float* scores = reinterpret_cast<float*>(ws + fd_bytes(geo));
-  if (fused_feasible(kv, n_layers * G, false)) {
+  if (allow_fused() && fused_feasible(kv, n_layers * G)) {
     RowParams rp{};
     rp.q_score = static_cast<const uint16_t*>(q_index);
     rp.q_attn = static_cast<const uint16_t*>(q_layers);
@@ -966,6 +967,13 @@ int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
   return cudaMemcpyFromSymbol(host, g_phase_ns, sizeof(long long) * kPhaseSlots * n_ctas) == cudaSuccess ? 0 : 5;
 }
 void aoh_debug_force_cluster(int32_t cl) { g_force_cluster = cl; }
+void aoh_debug_force_three(int32_t on) { g_force_three = on; }
+void aoh_debug_select_rows(int32_t on) { g_select_rows = on; }
+// per-CTA record of the select kernel's last launch: [b, g, L, nf, n, cap, T, KT, need_eq, eq_total]
+int32_t aoh_debug_select_info(int32_t* host, int32_t rows) {
+  cudaDeviceSynchronize();
+  return cudaMemcpyFromSymbol(host, g_sel_dbg, size_t(std::min(rows, 4096)) * 10 * sizeof(int)) == cudaSuccess;
+}
 void aoh_debug_force_ring(int32_t bytes, int32_t one_per_sm) {
   g_force_ring = bytes;
   g_force_one_per_sm = one_per_sm;

@@ -47,6 +47,19 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// fp32 dot of 8 bf16 (one 16-byte segment) with 8 fp32 weights, in element order
+__device__ __forceinline__ float dot8(const uint4& w, const float (&qs)[8]) {
+  float s = bf16lo(w.x) * qs[0];
+  s = fmaf(bf16hi(w.x), qs[1], s);
+  s = fmaf(bf16lo(w.y), qs[2], s);
+  s = fmaf(bf16hi(w.y), qs[3], s);
+  s = fmaf(bf16lo(w.z), qs[4], s);
+  s = fmaf(bf16hi(w.z), qs[5], s);
+  s = fmaf(bf16lo(w.w), qs[6], s);
+  s = fmaf(bf16hi(w.w), qs[7], s);
+  return s;
+}
+
 // ------------------------------------------------------------------ async copies
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

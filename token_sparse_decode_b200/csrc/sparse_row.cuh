@@ -8,11 +8,11 @@
 //
 // The row's L positions are cut into CL contiguous slices, one per CTA.
 //  1. scan:    each CTA streams the score rows of its slice (packed dominant
-//              columns, or K in place) through a 4-stage cp.async ring and scores
-//              16 rows per tensor-core MMA: rows on M, the group-summed query split
-//              into hi + lo bf16 parts on N (score = C[:,0] + C[:,1], fp32-exact to
-//              ~2^-17 of the query); the scores stay in shared memory as
-//              order-preserving uint32 keys;
+//              columns, or K in place): every warp runs its own cp.async ring of
+//              16-byte row segments, 16 in flight per lane, and takes the fp32 dots
+//              with the group-summed query (the same arithmetic as the stand-alone
+//              scan kernel); the scores stay in shared memory as order-preserving
+//              uint32 keys;
 //  2. select:  4-digit MSB radix select of the n-th largest key over the cluster
 //              (histograms summed through distributed shared memory, one cluster
 //              barrier per digit); ties broken toward lower positions by an ordered
@@ -29,7 +29,6 @@
 #pragma once
 
 #include <cooperative_groups.h>
-#include <cuda.h>  // CUtensorMap (the map is encoded on the host through the runtime's driver entry point)
 
 #include "device_common.cuh"
 
@@ -42,10 +41,11 @@ constexpr int kSrTS = 32;        // tokens per attention stage
 constexpr int kSrMaxStages = 8;  // ring stages (run-time count, from the shared memory left)
 constexpr int kSrMaxCluster = 16;
 constexpr int kSrMaxRun = 64;    // keys per thread in the compaction: slice <= 256 * 64
-constexpr int kSrRingStage = 16384;  // bytes per stage of the scan ring
+constexpr int kScanU = 4;        // scan: rows per lane per cp.async group
+constexpr int kScanDepth = 4;    // scan: groups in flight per warp (ring = 8 warps x 8 KB)
+constexpr int kSrRingMin = 8 * kScanDepth * kScanU * 512;  // 64 KB
 
 struct RowParams {
-  CUtensorMap tmap_scan;     // 2-D view of the score rows: packed [Hkv*T][cols] or K [T][stride_tok]
   const uint16_t* q_score;   // [B][Hq][D]: the query that scores (group-summed)
   const uint16_t* q_attn;    // [n_layers][B][Hq][D]: query rows of the attention
   const uint16_t* k;
@@ -65,11 +65,9 @@ struct RowParams {
   int64_t stride_tok, stride_head;
   int32_t T, B, Hq, Hkv, G, NQ;
   int32_t keys_bytes;        // dynamic shared memory before the ring
-  int32_t ring_bytes;        // ring region (scan stages, then attention stages); >= 64 KB
+  int32_t ring_bytes;        // ring region (scan rings, then attention stages); >= kSrRingMin
   const float* scores_in;    // non-null: keys come from these fp32 scores [Hkv][T] (no scan)
   int32_t select_only;       // 1: stop after writing the index (no attention)
-  int32_t scan_box;          // scan tile: inner box (elements, <= 64) ...
-  int32_t scan_rows;         // ... and rows per stage (<= 256); halves = srow_len / scan_box
   float scale_log2;
   uint8_t heads[kMaxHeads];
 };
@@ -83,15 +81,6 @@ struct AttTile {
   static constexpr int kTile = kSrTS * kPitch;  // one of K or V per stage
   static constexpr int kStage = 2 * kTile;
 };
-
-// Scan tiles are written by the tensor map with the span-byte swizzle (span = 2 * box,
-// 32/64/128 bytes): 16-byte chunk bits XOR address bits 7.. (span/16 - 1 mask).
-__device__ __forceinline__ uint32_t scan_tile_off(int r, int c, int span_shift, int rows) {
-  const int cpb = 1 << (span_shift - 4);     // 16-byte chunks per box row
-  const int h = c >> (span_shift - 4);
-  const uint32_t off = (uint32_t)(h * rows + r) << span_shift | (uint32_t)(c & (cpb - 1)) << 4;
-  return off ^ (((off >> 7) & (uint32_t)(cpb - 1)) << 4);
-}
 
 #ifdef AOH_PHASE_TIMERS
 // Diagnostic build only: global-timer stamps at the phase boundaries of every CTA.
@@ -131,7 +120,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   constexpr int NQP = NT * 8;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t mbar_s[kSrMaxStages];
   __shared__ int lh[256];      // this CTA's histogram of the current digit
   __shared__ int tot[2][256];  // cluster totals of digits 0-2 (every CTA adds its counts here)
   __shared__ int scan_scratch[33];
@@ -171,7 +159,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     s_gt[tid] = 0;
     s_eq[tid] = 0;
   }
-  // swizzled tensor loads need 1024-byte aligned slots: the host adds 1 KB of slack
+  // the dynamic region is used from a 1 KB boundary (the host adds 1 KB of slack)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int slice = (((L + CL - 1) / CL) + 3) & ~3;
   const int lo = min(L, rk * slice), hi = min(L, lo + slice);
@@ -199,31 +187,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   if (n < L) {
     // =============================================================== 1. scan
     if (!p.scores_in) {
-      // ring of tensor-map tiles: one elected thread issues halves x (box x rows) per stage
-      const int box = p.scan_box, rows = p.scan_rows;
-      const int halves = p.srow_len / box;
-      const int span_shift = 31 - __clz(box * 2);        // box row bytes = 2^span_shift
-      const int stage_bytes = halves * rows * (box * 2);
-      const int nst = (m + rows - 1) / rows;
-      const int ns = min(kSrMaxStages, p.ring_bytes / kSrRingStage);
-      const uint32_t rbase = smem_u32(smem + p.keys_bytes);
-      const int y0 = (p.packed ? g * p.T : 0) + off + lo;
-      const int x0 = p.packed ? 0 : g * (int)p.srow_stride_head;
-      if (tid == 0) {
-        for (int i = 0; i < ns; ++i) mbar_init(smem_u32(&mbar_s[i]), 1);
-        fence_mbar_init();
-        fence_proxy_async();
-      }
-      __syncthreads();
-      auto issue = [&](int st) {  // called by thread 0 only
-        const uint32_t bar = smem_u32(&mbar_s[st % ns]);
-        const uint32_t sb = rbase + (st % ns) * kSrRingStage;
-        mbar_expect_tx(bar, stage_bytes);
-        for (int h2 = 0; h2 < halves; ++h2)
-          tma_tile_2d(sb + h2 * rows * (box * 2), &p.tmap_scan, x0 + h2 * box, y0 + st * rows, bar);
-      };
-      if (tid == 0)
-        for (int s0 = 0; s0 < min(ns, nst); ++s0) issue(s0);
     if (tid < p.srow_len) {
       const int C = D / 2;
       int dim = -1;
@@ -263,60 +226,53 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     }
     __syncthreads();
     {
-      // B fragments of [hi | lo | 0 ...] (k = score dims, n = 8 columns): lanes 0-3 carry
-      // column 0 (hi), lanes 4-7 column 1 (lo), the others zeros.
-      const int ksteps = p.srow_len >> 4;   // 1 .. 8
-      uint32_t bt[8][2];
+      // Each warp streams a contiguous run of the slice's rows through its own cp.async
+      // ring: S lanes share a row (16 bytes each), kScanU rows per lane per group,
+      // kScanDepth groups in flight.  A lane reads back only the bytes it copied, so the
+      // ring needs no barrier; the dot and its shuffle reduction match the stand-alone
+      // scan kernel term for term (same fp32 scores, same keys).
+      const int S = p.srow_len >> 3;  // 2, 4, 8 or 16
+      const int seg = lane & (S - 1);
+      const int rpw = 32 / S;
+      float qs[8];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        bt[ks][0] = bt[ks][1] = 0u;
-        if (ks < ksteps && lane < 8) {
-          const int d0 = ks * 16 + 2 * (lane & 3);
-          float v[4] = {qt[d0], qt[d0 + 1], qt[d0 + 8], qt[d0 + 9]};
-          if (lane >= 4) {  // lo = value - bf16(value)
+      for (int i = 0; i < 8; ++i) qs[i] = qt[seg * 8 + i];
+      const int per_warp = (m + 7) / 8;
+      const int wr0 = min(m, warp * per_warp), wr1 = min(m, wr0 + per_warp);
+      const int grows = rpw * kScanU;
+      const int nb = (wr1 - wr0 + grows - 1) / grows;
+      const uint32_t wring = smem_u32(smem + p.keys_bytes) + warp * (kScanDepth * kScanU * 512) + lane * 16;
+      const uint16_t* src0 = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)(off + lo) * p.srow_stride_tok + seg * 8;
+      auto issue = [&](int k) {
+        const uint32_t slot = wring + (k % kScanDepth) * (kScanU * 512);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] -= __bfloat162float(__float2bfloat16_rn(v[i]));
-          }
-          bt[ks][0] = pack_bf16x2(v[0], v[1]);
-          bt[ks][1] = pack_bf16x2(v[2], v[3]);
+        for (int u = 0; u < kScanU; ++u) {
+          const int r = wr0 + k * grows + u * rpw + lane / S;
+          const bool ok = r < wr1;
+          cp_async_16(slot + u * 512, src0 + (int64_t)(ok ? r : wr0) * p.srow_stride_tok, ok);
+        }
+      };
+#pragma unroll
+      for (int k = 0; k < kScanDepth - 1; ++k) {
+        if (k < nb) issue(k);
+        cp_async_commit();
+      }
+      for (int k = 0; k < nb; ++k) {
+        if (k + kScanDepth - 1 < nb) issue(k + kScanDepth - 1);
+        cp_async_commit();
+        cp_async_wait<kScanDepth - 1>();
+        const uint8_t* slot = smem + p.keys_bytes + warp * (kScanDepth * kScanU * 512) + lane * 16 +
+                              (k % kScanDepth) * (kScanU * 512);
+#pragma unroll
+        for (int u = 0; u < kScanU; ++u) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(slot + u * 512);
+          float sc = dot8(v4, qs);
+          for (int o = S >> 1; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+          const int r = wr0 + k * grows + u * rpw + lane / S;
+          if (seg == 0 && r < wr1) keys[r] = score_key(sc);
         }
       }
-      bool failed = false;
-      int st = 0;
-      for (; st < nst; ++st) {
-        const bool ok = mbar_wait(smem_u32(&mbar_s[st % ns]), (uint32_t)((st / ns) & 1));
-        if (__syncthreads_or(!ok)) {
-          if (tid == 0) record_error(kCheckTimeout, b, g, st);
-          failed = true;
-          break;
-        }
-        const uint32_t sb = rbase + (st % ns) * kSrRingStage;
-        for (int tile = warp; tile * 16 < rows; tile += 8) {
-          const int nv = m - (st * rows + tile * 16);
-          if (nv <= 0) break;
-          float c4[4] = {0.f, 0.f, 0.f, 0.f};
-          const int r = tile * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            if (ks < ksteps) {
-              uint32_t a[4];
-              ldsm_x4(a, sb + scan_tile_off(r, 2 * ks + (lane >> 4), span_shift, rows));
-              mma_16816(c4, a, bt[ks][0], bt[ks][1]);
-            }
-          }
-          if ((lane & 3) == 0) {
-            const int ri = lane >> 2;  // row within the 16-row tile; nv counts from the tile start
-            const int r0 = st * rows + tile * 16 + ri;
-            if (ri < nv) keys[r0] = score_key(c4[0] + c4[1]);
-            if (ri + 8 < nv) keys[r0 + 8] = score_key(c4[2] + c4[3]);
-          }
-        }
-        __syncthreads();  // the slot is free: refill it
-        if (tid == 0 && st + ns < nst) issue(st + ns);
-      }
-      if (failed && tid == 0) {  // drain the copies still in flight (bounded) before reuse
-        for (int s2 = st; s2 < min(nst, st + ns); ++s2) mbar_wait(smem_u32(&mbar_s[s2 % ns]), (uint32_t)((s2 / ns) & 1));
-      }
+      cp_async_wait<0>();
       __syncthreads();
     }
     }

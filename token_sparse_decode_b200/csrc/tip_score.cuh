@@ -29,8 +29,10 @@ struct TipParams {
   int32_t T, Hq, Hkv, d, G, n_dom;
   int32_t row_len;          // elements per row: k_dom cols (packed) or d (in place)
   int32_t packed;
-  int32_t tile;             // tokens per CTA
-  uint8_t heads[kMaxHeads]; // KV heads scored, one per blockIdx.y
+  int32_t B;
+  int64_t per_cta;          // flattened (listed head, token) rows per CTA
+  int64_t total;            // n_listed * T
+  uint8_t heads[kMaxHeads]; // KV heads scored
 };
 
 __device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
@@ -41,99 +43,140 @@ __device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
   return r;
 }
 
-__device__ __forceinline__ float dot8(const uint4& w, const float (&qs)[8]) {
-  float s = bf16lo(w.x) * qs[0];
-  s = fmaf(bf16hi(w.x), qs[1], s);
-  s = fmaf(bf16lo(w.y), qs[2], s);
-  s = fmaf(bf16hi(w.y), qs[3], s);
-  s = fmaf(bf16lo(w.z), qs[4], s);
-  s = fmaf(bf16hi(w.z), qs[5], s);
-  s = fmaf(bf16lo(w.w), qs[6], s);
-  s = fmaf(bf16hi(w.w), qs[7], s);
-  return s;
-}
 
 // S = lanes per row: row_len / 8 rounded up to a power of two (1 .. 16); lanes whose
 // 16-byte segment lies past the row end carry zero weights and load nothing.
+//
+// Persistent grid: CTA c owns rows [c * per_cta, (c + 1) * per_cta) of the flattened
+// (listed head j, token t) space, so every CTA streams the same number of rows.  A CTA walks
+// its share segment by segment (a segment = the rows of one head within one sequence); at a
+// segment start it issues the first batch of row loads, then finds the sequence and builds
+// q~ while those loads are in flight.
 template <int S>
-__global__ void __launch_bounds__(kTipThreads) tip_score_kernel(const TipParams p) {
+__global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipParams p) {
   __shared__ float qt[128];
-  const int b = blockIdx.z;
-  const int g = p.heads[blockIdx.y];
-  const int off = p.offsets[b];
-  const int L = p.offsets[b + 1] - off;
-  const int t0 = blockIdx.x * p.tile;
-  if (t0 >= L) return;
-  const int t1 = min(L, t0 + p.tile);
+  __shared__ int s_seg[2];  // sequence b of the segment (-1: none), its end token
+  const int tid = threadIdx.x, lane = tid & 31;
   const int C = p.d >> 1;
-  const int tid = threadIdx.x;
-
-  // q~ for this (b, g): fp32 group sum, restricted to the dominant dims.
-  if (tid < p.row_len) {
-    int dim = -1;
-    if (p.packed) {
-      if (tid < 2 * p.n_dom) {
-        const int j = tid < p.n_dom ? tid : tid - p.n_dom;
-        const int c = p.idom[g * p.n_dom + j];
-        if (c < 0 || c >= C) {
-          record_error(kCheckChunk, g, j, c);
-        } else {
-          dim = tid < p.n_dom ? c : c + C;
-        }
-      }
-    } else if (p.idom == nullptr) {
-      dim = tid;  // every chunk: the full dot
-    } else {
-      const int c = tid < C ? tid : tid - C;
-      for (int j = 0; j < p.n_dom; ++j) {
-        const int cj = p.idom[g * p.n_dom + j];
-        if (cj < 0 || cj >= C) record_error(kCheckChunk, g, j, cj);
-        if (cj == c) dim = tid;
-      }
-    }
-    float acc = 0.f;
-    if (dim >= 0) {
-      const uint16_t* qb = p.q + ((int64_t)b * p.Hq + (int64_t)g * p.G) * p.d + dim;
-      for (int h = 0; h < p.G; ++h) acc += __uint_as_float((uint32_t)qb[(int64_t)h * p.d] << 16);
-    }
-    qt[tid] = acc;
-  }
-  __syncthreads();
-
-  const int lane = tid & 31;
   const int seg = lane % S;
-  float qs[8];
-  bool active = false;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    qs[i] = (seg * 8 + i < p.row_len) ? qt[seg * 8 + i] : 0.f;
-    active |= (qs[i] != 0.f);
-  }
   constexpr int RPI = kTipThreads / S;  // rows per block iteration
   constexpr int U = 8;                  // independent loads in flight per thread
-  const uint16_t* base = p.src + (int64_t)g * p.row_stride_head + (int64_t)off * p.row_stride_tok + seg * 8;
-  float* srow = p.scores + (int64_t)g * p.T + off;
-  // Warp-uniform loop bounds: every lane of a warp takes the same trip count, so the
-  // shuffles below always run with the full mask; rows past the tile are masked.
-  const int warp_row0 = (tid >> 5) * (32 / S);
-  const int lrow = lane / S;
-
-  for (int tb = t0 + warp_row0; tb < t1; tb += U * RPI) {
-    uint4 w[U];
+  constexpr int BATCH = U * RPI;
+  const int prow = (tid >> 5) * (32 / S) + lane / S;
+  const int64_t w1 = min(p.total, (int64_t)(blockIdx.x + 1) * p.per_cta);
+  int64_t w = (int64_t)blockIdx.x * p.per_cta;
+  int bhint = 0;
+  int64_t cur_j = -1;
+  while (w < w1) {  // CTA-uniform
+    const int64_t j = w / p.T;
+    const int t = (int)(w - j * p.T);
+    const int g = p.heads[j];
+    const int lim = (int)min(w1 - w, (j + 1) * (int64_t)p.T - w);  // rows of this head in the share
+    // the rows' segment columns: in place with I_dom, segments without a dominant dim stay unread
+    bool active = true;
+    if (!p.packed && p.idom) {
+      active = false;
+      for (int jj = 0; jj < p.n_dom; ++jj) {
+        const int c = p.idom[g * p.n_dom + jj];
+        const int lo = seg * 8, hi = seg * 8 + 8;
+        if ((c >= lo && c < hi) || (c + C >= lo && c + C < hi)) active = true;
+      }
+    }
+    active = active && seg * 8 < p.row_len;
+    const uint16_t* base = p.src + (int64_t)g * p.row_stride_head + (int64_t)t * p.row_stride_tok + seg * 8;
+    uint4 v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int tt = tb + u * RPI + lrow;
-      w[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (tt < t1 && active) w[u] = ld_stream_v4(base + (int64_t)tt * p.row_stride_tok);
+      const int r = u * RPI + prow;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < lim && active) v[u] = ld_stream_v4(base + (int64_t)r * p.row_stride_tok);
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float s = dot8(w[u], qs);
-#pragma unroll
-      for (int o = S / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const int tt = tb + u * RPI + lrow;
-      if (seg == 0 && tt < t1) srow[tt] = s;
+    // the segment: sequence b holding token t (searched from the previous one within a head)
+    if (j != cur_j) bhint = 0;
+    cur_j = j;
+    if (tid < 32) {
+      int b = -1;
+      for (int b0 = bhint; b0 < p.B && b < 0; b0 += 32) {
+        const int i = b0 + lane;
+        const bool hit = i < p.B && p.offsets[i] <= t && t < p.offsets[i + 1];
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) b = b0 + __ffs(m) - 1;
+      }
+      if (lane == 0) {
+        int e = p.T;
+        if (b < 0) {
+          record_error(kCheckPosition, (int)j, t, -1);
+        } else {
+          e = p.offsets[b + 1];
+          if (e > p.T) {  // offsets past the cache: score no row beyond it
+            record_error(kCheckPosition, (int)j, e, p.T);
+            e = p.T;
+          }
+        }
+        s_seg[0] = b;
+        s_seg[1] = e;
+      }
     }
+    __syncthreads();
+    const int b = s_seg[0];
+    const int n = min(lim, s_seg[1] - t);  // rows of the segment (>= 1)
+    if (b >= 0) bhint = b;
+    // q~ for (b, g): fp32 group sum in head order, restricted to the dominant dims
+    if (tid < p.row_len) {
+      int dim = -1;
+      if (b < 0) {
+      } else if (p.packed) {
+        if (tid < 2 * p.n_dom) {
+          const int jj = tid < p.n_dom ? tid : tid - p.n_dom;
+          const int c = p.idom[g * p.n_dom + jj];
+          if (c < 0 || c >= C) {
+            record_error(kCheckChunk, g, jj, c);
+          } else {
+            dim = tid < p.n_dom ? c : c + C;
+          }
+        }
+      } else if (p.idom == nullptr) {
+        dim = tid;  // every chunk: the full dot
+      } else {
+        const int c = tid < C ? tid : tid - C;
+        for (int jj = 0; jj < p.n_dom; ++jj) {
+          const int cj = p.idom[g * p.n_dom + jj];
+          if (cj < 0 || cj >= C) record_error(kCheckChunk, g, jj, cj);
+          if (cj == c) dim = tid;
+        }
+      }
+      float acc = 0.f;
+      if (dim >= 0) {
+        const uint16_t* qb = p.q + ((int64_t)b * p.Hq + (int64_t)g * p.G) * p.d + dim;
+        for (int h = 0; h < p.G; ++h) acc += __uint_as_float((uint32_t)qb[(int64_t)h * p.d] << 16);
+      }
+      qt[tid] = acc;
+    }
+    __syncthreads();
+    float qs[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qs[i] = (seg * 8 + i < p.row_len) ? qt[seg * 8 + i] : 0.f;
+    __syncthreads();  // qt is rewritten by the next segment
+    float* srow = p.scores + (int64_t)g * p.T + t;
+    for (int r0 = 0; r0 < n; r0 += BATCH) {  // CTA-uniform trip count: full-mask shuffles
+      if (r0 > 0) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int r = r0 + u * RPI + prow;
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (r < n && active) v[u] = ld_stream_v4(base + (int64_t)r * p.row_stride_tok);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float sc = dot8(v[u], qs);
+#pragma unroll
+        for (int o = S / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+        const int r = r0 + u * RPI + prow;
+        if (seg == 0 && r < n) srow[r] = sc;
+      }
+    }
+    w += n;
   }
 }
 

@@ -1,28 +1,30 @@
-// Top-N_fac selection (FASA: Frequency-aware Sparse Attention, §2.B.1; the
-// shared index of "Cómo funciona CLSA" is the same operation with k fixed).
+// Top-N_fac selection over precomputed scores (FASA: Frequency-aware Sparse
+// Attention, §2.B.1; the shared index of "Cómo funciona CLSA" is the same
+// operation with k fixed).
 //
-// One thread-block cluster per (sequence b, KV head g).  The row's scores are
-// split into CL contiguous slices, one per CTA, cached in shared memory as
+// One CTA of 512 threads per (sequence b, KV head g) row; the row's fp32 scores
+// (written by the scan kernel just before, so resident in L2) are read as
 // order-preserving uint32 keys.  An MSB-first radix select (4 digits of 8 bits)
-// finds the n-th largest key K_T: each CTA builds a 256-bin histogram of the keys
-// that still match the prefix, every CTA sums the CL histograms through
-// distributed shared memory and picks the same digit.  Histograms are double
-// buffered so one cluster barrier per digit suffices.  The selection is then
-// {key > K_T} plus the first (n - #{key > K_T}) positions with key == K_T in
-// position order, which is exactly "score descending, lower position first".
-// An ordered compaction (block scans inside a CTA, a cluster-wide prefix over the
-// CTA totals) writes the positions in ascending order.  Deterministic.
+// finds the n-th largest key K_T:
+//   digit 0: a coalesced pass over the row builds its 256-bin histogram (warp-
+//            aggregated shared-memory counts);
+//   then the keys sharing the chosen first digit are compacted into shared
+//            memory by a second pass (when they fit; otherwise the later digits
+//            re-read the row), and digits 1-3 are counted over those candidates.
+// The selection is {key > K_T} plus the first (n - #{key > K_T}) positions with
+// key == K_T in position order, i.e. "score descending, lower position first".
+// A third pass writes it in ascending position order: tiles of 2048 positions,
+// four consecutive positions per thread, one block scan of the packed
+// (#greater, #equal) counts per tile gives each thread its output offset and
+// its rank among the equal keys.  Deterministic; no cluster, no global scratch.
 #pragma once
-
-#include <cooperative_groups.h>
 
 #include "device_common.cuh"
 
 namespace aoh {
 
-namespace cg = cooperative_groups;
-
 constexpr int kSelThreads = 512;
+constexpr int kSelCandCap = 24576;  // candidate keys kept in shared memory (96 KB)
 
 struct SelectParams {
   const float* scores;            // [Hkv][T]
@@ -31,184 +33,174 @@ struct SelectParams {
   int32_t* idx;                   // [B][Hkv][cap]
   int32_t* count;                 // [B][Hkv]
   int32_t T, Hkv, n_fac, cap;
-  int32_t chunk;                  // positions per CTA slice
-  int32_t keys_in_smem;           // 1: slice cached in dynamic shared memory
-  uint8_t heads[kMaxHeads];
+  uint8_t heads[kMaxHeads];       // KV head of blockIdx.x
 };
 
+// Warp-aggregated histogram increment (bin < 0: the lane does not count); every lane
+// of the warp must call it.
+__device__ __forceinline__ void sel_hist_add(int* h, int bin) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+}
+
+#ifdef AOH_PHASE_TIMERS
+__device__ int g_sel_dbg[4096][10];  // diagnostic build: each CTA's view of its row
+#define AOH_SEL_DBG(i, v) \
+  if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096) g_sel_dbg[blockIdx.y * gridDim.x + blockIdx.x][i] = (int)(v)
+#else
+#define AOH_SEL_DBG(i, v)
+#endif
 
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectParams p) {
-  extern __shared__ __align__(16) uint32_t skeys[];
-  __shared__ int hist[2][256];
+  extern __shared__ __align__(16) uint32_t cand[];  // kSelCandCap keys
+  __shared__ int hist[256];
   __shared__ int scan_scratch[33];
-  __shared__ int s_bin, s_above;
-  __shared__ int s_cnt[2];            // this CTA's (#eq, #gt)
-  __shared__ int s_eq_before, s_sel_before;
+  __shared__ int s_bin, s_above, s_in_bin, s_nc;
 
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CL = (int)cluster.num_blocks();
-  const int r = (int)cluster.block_rank();
-  const int tid = threadIdx.x;
-  const int b = blockIdx.z;
-  const int g = p.heads[blockIdx.y];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.y;
+  const int g = p.heads[blockIdx.x];
   const int off = p.offsets[b];
   const int L = p.offsets[b + 1] - off;
   int nf = p.n_fac_per_seq ? p.n_fac_per_seq[b] : p.n_fac;
   if (nf > p.cap) {
-    if (r == 0 && tid == 0) record_error(kCheckCount, b, nf, p.cap);
+    if (tid == 0) record_error(kCheckCount, b, nf, p.cap);
     nf = p.cap;
   }
   const int n = max(0, min(nf, L));
   int32_t* out = p.idx + ((int64_t)b * p.Hkv + g) * p.cap;
   const float* row = p.scores + (int64_t)g * p.T + off;
-  const int lo = min(L, r * p.chunk);
-  const int hi = min(L, lo + p.chunk);
+  AOH_SEL_DBG(0, b);
+  AOH_SEL_DBG(1, g);
+  AOH_SEL_DBG(2, L);
+  AOH_SEL_DBG(3, nf);
+  AOH_SEL_DBG(4, n);
+  AOH_SEL_DBG(5, p.cap);
+  AOH_SEL_DBG(6, p.T);
+  for (int j = n + tid; j < p.cap; j += kSelThreads) out[j] = -1;
+  if (tid == 0) p.count[(int64_t)b * p.Hkv + g] = n;
+  if (n == 0) return;  // before any barrier: uniform over the CTA
+  // N_fac >= L needs no special case: the threshold is then the smallest key and every
+  // key equal to it is taken, so the compaction below writes every position in order.
 
-  // padding of the unused tail of the row, spread over the cluster
-  for (int j = n + r * kSelThreads + tid; j < p.cap; j += CL * kSelThreads) out[j] = -1;
-  if (r == 0 && tid == 0) p.count[(int64_t)b * p.Hkv + g] = n;
-  if (n == 0) return;               // uniform over the cluster: no barrier taken
-  if (n == L) {                     // N_fac >= L: every position, in order
-    for (int j = lo + tid; j < hi; j += kSelThreads) out[j] = j;
-    return;
-  }
-
-  if (p.keys_in_smem) {
-    for (int i = lo + tid; i < hi; i += kSelThreads) skeys[i - lo] = score_key(row[i]);
-  }
-  auto key_at = [&](int i) -> uint32_t {  // i in [lo, hi)
-    return p.keys_in_smem ? skeys[i - lo] : score_key(__ldcg(row + i));
-  };
-
+  // ---- threshold K_T: 4 digits of 8 bits, most significant first
   uint32_t prefix = 0u, pmask = 0u;
-  int krem = n;  // rank of the threshold among keys matching the prefix (1-based from the top)
+  int krem = n;        // rank of the threshold among the keys matching the prefix (1 = largest)
+  int nc = -1;         // candidates in shared memory (-1: the row is re-read)
+  int eq_total = 0;    // keys equal to K_T (the chosen bin of the last digit)
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    int* h = hist[pass & 1];
-    if (tid < 256) h[tid] = 0;
+    if (tid < 256) hist[tid] = 0;
     __syncthreads();
-    if (p.keys_in_smem) {
-      // four keys per lane from shared memory; the first digit (sign + exponent) is shared by
-      // most keys and counted with warp aggregation, later digits directly
-      for (int b0 = (tid & ~31) * 4; b0 < hi - lo; b0 += kSelThreads * 4) {  // warp-uniform
-        const int i0 = b0 + 4 * (tid & 31);  // i0 + 3 < chunk: inside the keys region
-        const uint4 k4 = *reinterpret_cast<const uint4*>(skeys + i0);
-        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool in = (i0 + j < hi - lo) && ((kk[j] & pmask) == prefix);
-          const int bin = in ? (int)((kk[j] >> shift) & 255u) : -1;
-          if (pass == 0) {
-            const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
-          } else if (in) {
-            atomicAdd(&h[bin], 1);
-          }
-        }
+    if (nc >= 0) {
+      for (int i = tid; i < nc; i += kSelThreads) {
+        const uint32_t k = cand[i];
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
       }
     } else {
-      // scores re-read from L2: warp-aggregated counts
-      for (int base = lo + (tid & ~31); base < hi; base += kSelThreads) {
-        const int i = base + (tid & 31);
-        int bin = -1;
-        if (i < hi) {
-          const uint32_t k = key_at(i);
-          if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255u);
+      // coalesced pass over the row, four loads in flight per lane (warp-uniform trip count)
+      for (int base = warp * 32; base < L; base += 4 * kSelThreads) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + lane;
+          v[u] = i < L ? __ldcg(row + i) : 0.f;
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + lane;
+          const uint32_t k = score_key(v[u]);
+          sel_hist_add(hist, (i < L && (k & pmask) == prefix) ? (int)((k >> shift) & 255u) : -1);
+        }
       }
     }
-    cluster.sync();
-    // cluster-wide total of the bin that this thread scans, bins taken from the top down
-    int tot = 0;
-    if (tid < 256) {
-      const int bin = 255 - tid;
-      int v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = (q < CL) ? cluster.map_shared_rank(h, q)[bin] : 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) tot += v[q];
-    }
+    __syncthreads();
+    // bins from the top down: exclusive prefix, then the bin holding rank krem
+    const int tot = tid < 256 ? hist[255 - tid] : 0;
     int total;
     const int above = block_exclusive_scan(tot, scan_scratch, &total);
     if (tid < 256 && above < krem && krem <= above + tot) {
       s_bin = 255 - tid;
       s_above = above;
+      s_in_bin = tot;
     }
+    if (tid == 0) s_nc = 0;
     __syncthreads();
     prefix |= (uint32_t)s_bin << shift;
     pmask |= 255u << shift;
     krem -= s_above;
+    eq_total = s_in_bin;
+    // after the first digit: compact the keys sharing it (order irrelevant: only counted)
+    const bool compact = (pass == 0) && (s_in_bin <= kSelCandCap);
+    if (compact) {
+      for (int base = warp * 32; base < L; base += 4 * kSelThreads) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + lane;
+          v[u] = i < L ? __ldcg(row + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = base + u * kSelThreads + lane;
+          const uint32_t k = score_key(v[u]);
+          const bool hit = i < L && (k & pmask) == prefix;
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
+          int slot = 0;
+          if (lane == 0 && bal) slot = atomicAdd(&s_nc, __popc(bal));
+          slot = __shfl_sync(0xffffffffu, slot, 0);
+          if (hit) cand[slot + __popc(bal & ((1u << lane) - 1u))] = k;
+        }
+      }
+    }
     __syncthreads();
+    if (compact) nc = s_nc;
   }
   const uint32_t KT = prefix;
-  const int need_eq = krem;  // how many positions with key == KT are taken (lowest first)
+  const int need_eq = krem;    // keys equal to K_T that are taken, lowest positions first
+  AOH_SEL_DBG(7, KT);
+  AOH_SEL_DBG(8, need_eq);
+  AOH_SEL_DBG(9, eq_total);
 
-  // ---- ordered compaction
-  const int m = hi - lo;
-  const int run = (m + kSelThreads - 1) / kSelThreads;
-  const int a0 = lo + min(m, tid * run);
-  const int a1 = lo + min(m, (tid + 1) * run);
-  int n_eq = 0, n_gt = 0;
-  for (int i = a0; i < a1; ++i) {
-    const uint32_t k = key_at(i);
-    n_gt += k > KT;
-    n_eq += k == KT;
-  }
-  int eq_cta, gt_cta;
-  const int eq_excl = block_exclusive_scan(n_eq, scan_scratch, &eq_cta);
-  block_exclusive_scan(n_gt, scan_scratch, &gt_cta);
-  if (tid == 0) {
-    s_cnt[0] = eq_cta;
-    s_cnt[1] = gt_cta;
-  }
-  cluster.sync();
-  if (tid == 0) {
-    int eq_before = 0, sel_before = 0;
-    for (int q = 0; q < r; ++q) {
-      const int* c = cluster.map_shared_rank(s_cnt, q);
-      const int eqq = c[0], gtq = c[1];
-      sel_before += gtq + max(0, min(need_eq - eq_before, eqq));
-      eq_before += eqq;
+  // ---- ordered compaction: tiles of 4 * kSelThreads positions, 4 consecutive per thread
+  int sel_base = 0, eq_base = 0;
+  const bool all_eq = (eq_total == need_eq);  // every key equal to K_T is taken
+  for (int t0 = 0; t0 < L; t0 += 4 * kSelThreads) {
+    const int i0 = t0 + 4 * tid;
+    uint32_t k[4];
+    int ngt = 0, neq = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      k[j] = i0 + j < L ? score_key(__ldg(row + i0 + j)) : 0u;  // L1 merges the 4 strided loads
+      const bool in = i0 + j < L;
+      ngt += (in && k[j] > KT);
+      neq += (in && k[j] == KT);
     }
-    s_eq_before = eq_before;
-    s_sel_before = sel_before;
-  }
-  __syncthreads();
-  cluster_arrive_release();  // this CTA is done reading its peers' shared memory
-  const int eq_base = s_eq_before + eq_excl;
-  int n_sel = 0;
-  {
-    int seen = 0;
-    for (int i = a0; i < a1; ++i) {
-      const uint32_t k = key_at(i);
-      if (k > KT) {
-        ++n_sel;
-      } else if (k == KT) {
-        n_sel += (eq_base + seen < need_eq);
-        ++seen;
+    int packed_tot;
+    const int packed = block_exclusive_scan((ngt << 16) | neq, scan_scratch, &packed_tot);
+    const int gt_excl = packed >> 16, eq_excl = packed & 0xffff;
+    // equal keys before this thread (whole row), and how many of them are taken
+    const int eq_prev = eq_base + eq_excl;
+    int pos = sel_base + gt_excl + (all_eq ? eq_excl : min(need_eq, eq_prev) - min(need_eq, eq_base));
+    int eq_seen = eq_prev;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (i0 + j >= L) break;
+      bool take = k[j] > KT;
+      if (k[j] == KT) {
+        take = all_eq || eq_seen < need_eq;
+        ++eq_seen;
+      }
+      if (take) {
+        if (pos < n) out[pos] = i0 + j;  // pos < n by construction; kept as a guard
+        ++pos;
       }
     }
+    const int gt_t = packed_tot >> 16, eq_t = packed_tot & 0xffff;
+    sel_base += gt_t + (all_eq ? eq_t : min(need_eq, eq_base + eq_t) - min(need_eq, eq_base));
+    eq_base += eq_t;
   }
-  int sel_cta;
-  int pos = s_sel_before + block_exclusive_scan(n_sel, scan_scratch, &sel_cta);
-  {
-    int seen = 0;
-    for (int i = a0; i < a1; ++i) {
-      const uint32_t k = key_at(i);
-      bool take = false;
-      if (k > KT) {
-        take = true;
-      } else if (k == KT) {
-        take = (eq_base + seen < need_eq);
-        ++seen;
-      }
-      if (take && pos < n) out[pos++] = i;  // pos < n holds by construction; kept as a guard
-    }
-  }
-  cluster_wait_acquire();  // peers may still read s_cnt until they have all arrived
 }
 
 }  // namespace aoh
