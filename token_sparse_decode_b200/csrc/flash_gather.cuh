@@ -356,13 +356,22 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
   __threadfence();
   const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
   const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
-  // weights w[s][q] = 2^(m_sq - M_q) staged in shared memory (nsplit * NQP <= kFdMaxSplits * NQP fits)
+  // weights w[s][q] = 2^(m_sq - M_q) staged in shared memory (nsplit * NQP <= kFdMaxSplits * NQP fits).
+  // The partials sit in L2: every loop below keeps 8 independent loads in flight per thread.
   float* sw = reinterpret_cast<float*>(smem);        // [nsplit][NQP]
   float* sM = sw + nsplit * NQP;                     // [NQP]
   float* sL = sM + NQP;                              // [NQP]
   if (tid < NQP) {
     float M = -INFINITY;
-    for (int s2 = 0; s2 < nsplit; ++s2) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2));
+    int s2 = 0;
+    for (; s2 + 8 <= nsplit; s2 += 8) {
+      float mv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mv[u] = __ldcg(rml + ((int64_t)(s2 + u) * NQP + tid) * 2);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) M = fmaxf(M, mv[u]);
+    }
+    for (; s2 < nsplit; ++s2) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2));
     sM[tid] = M;
   }
   __syncthreads();
@@ -373,23 +382,52 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
   __syncthreads();
   if (tid < NQP) {
     float Ls = 0.f;
-    for (int s2 = 0; s2 < nsplit; ++s2) Ls += sw[s2 * NQP + tid] * __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2 + 1);
+    int s2 = 0;
+    for (; s2 + 8 <= nsplit; s2 += 8) {
+      float lv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) lv[u] = __ldcg(rml + ((int64_t)(s2 + u) * NQP + tid) * 2 + 1);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) Ls += sw[(s2 + u) * NQP + tid] * lv[u];
+    }
+    for (; s2 < nsplit; ++s2) Ls += sw[s2 * NQP + tid] * __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2 + 1);
     sL[tid] = Ls;
   }
   __syncthreads();
-  for (int e = tid; e < p.NQ * D; e += kFdThreads) {
-    const int qr = e / D, dd = e % D;
-    float A0 = 0.f, A1 = 0.f, A2 = 0.f, A3 = 0.f;
+  // four consecutive dimensions of one query row per thread
+  for (int e4 = tid; e4 < p.NQ * (D / 4); e4 += kFdThreads) {
+    const int qr = e4 / (D / 4), dd = (e4 % (D / 4)) * 4;
+    const float* col = racc + (int64_t)qr * D + dd;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
     int s2 = 0;
-    for (; s2 + 4 <= nsplit; s2 += 4) {
-      A0 += sw[(s2 + 0) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 0) * NQP + qr) * D + dd);
-      A1 += sw[(s2 + 1) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 1) * NQP + qr) * D + dd);
-      A2 += sw[(s2 + 2) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 2) * NQP + qr) * D + dd);
-      A3 += sw[(s2 + 3) * NQP + qr] * __ldcg(racc + ((int64_t)(s2 + 3) * NQP + qr) * D + dd);
+    for (; s2 + 8 <= nsplit; s2 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)(s2 + u) * NQP * D));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = sw[(s2 + u) * NQP + qr];
+        A.x += w * v[u].x;
+        A.y += w * v[u].y;
+        A.z += w * v[u].z;
+        A.w += w * v[u].w;
+      }
     }
-    for (; s2 < nsplit; ++s2) A0 += sw[s2 * NQP + qr] * __ldcg(racc + ((int64_t)s2 * NQP + qr) * D + dd);
+    for (; s2 < nsplit; ++s2) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)s2 * NQP * D));
+      const float w = sw[s2 * NQP + qr];
+      A.x += w * v.x;
+      A.y += w * v.y;
+      A.z += w * v.z;
+      A.w += w * v.w;
+    }
+    const float inv = 1.f / sL[qr];
     const int l = qr / p.G, h = g * p.G + qr % p.G;
-    p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = ((A0 + A1) + (A2 + A3)) / sL[qr];
+    float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
+    o[0] = A.x * inv;
+    o[1] = A.y * inv;
+    o[2] = A.z * inv;
+    o[3] = A.w * inv;
   }
   if (tid == 0) p.tickets[row_id] = 0;
 }

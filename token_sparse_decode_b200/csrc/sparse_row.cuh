@@ -413,33 +413,39 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     __syncthreads();
     const int run = (m + kSrThreads - 1) / kSrThreads;  // <= kSrMaxRun (host guarantees)
     const int a0 = min(m, tid * run), a1 = min(m, (tid + 1) * run);
+    const int len = a1 - a0;
+    // One pass over this thread's run of keys, in a lane-skewed order so that the 32 lanes
+    // of a warp read 32 different banks: bit i of gtm / eqm marks key a0 + i above / equal
+    // to the threshold.
+    uint64_t gtm = 0ull, eqm = 0ull;
+    if (len > 0) {
+      int e = lane % len;
+      for (int j = 0; j < len; ++j) {
+        const uint32_t k = keys[a0 + e];
+        gtm |= (uint64_t)(k > KT) << e;
+        eqm |= (uint64_t)(k == KT) << e;
+        if (++e == len) e = 0;
+      }
+    }
+    const int n_eq = __popcll(eqm);
     int eq_excl = 0;
     if (s_eq_all > need_eq) {  // more keys equal the threshold than are taken: rank them
-      int n_eq = 0;
-      for (int i = a0; i < a1; ++i) n_eq += keys[i] == KT;
       int eq_cta;
       eq_excl = block_exclusive_scan(n_eq, scan_scratch, &eq_cta);
     }
-    uint64_t take = 0ull;
-    int n_sel = 0;
-    {
-      const int eq_base = s_eq_before + eq_excl;
-      int seen = 0;
-      for (int i = a0; i < a1; ++i) {
-        const uint32_t k = keys[i];
-        bool t = false;
-        if (k > KT) {
-          t = true;
-        } else if (k == KT) {
-          t = (eq_base + seen < need_eq);
-          ++seen;
-        }
-        if (t) {
-          take |= 1ull << (i - a0);
-          ++n_sel;
-        }
+    // this thread takes the lowest max(0, need_eq - equal keys before it) of its equal keys
+    const int take_eq = min(n_eq, max(0, need_eq - (s_eq_before + eq_excl)));
+    uint64_t take = gtm;
+    if (take_eq == n_eq) {
+      take |= eqm;
+    } else {
+      uint64_t rest = eqm;
+      for (int i = 0; i < take_eq; ++i) {
+        take |= rest & (~rest + 1ull);
+        rest &= rest - 1ull;
       }
     }
+    const int n_sel = __popcll(take);
     int sel_cta;
     const int my = block_exclusive_scan(n_sel, scan_scratch, &sel_cta);  // ends with a barrier
     {
