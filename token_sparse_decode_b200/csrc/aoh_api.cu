@@ -310,14 +310,15 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
   // 1 KB of slack: the kernel aligns its dynamic shared memory to 1024 bytes
   size_t budget = kTwoPerSm - 1024;
-  // select-only launches still need a region as large as the keys for the select's candidates
-  const size_t ring_min = need_ring ? kRingMin : f.keys_bytes;
+  // select-only launches need only a region for the select's candidates (a quarter of the
+  // keys; a CTA whose candidates do not fit counts its later digits over all its keys)
+  const size_t ring_min = need_ring ? kRingMin : (size_t)ceil_div(f.keys_bytes / 4, 1024) * 1024;
   if (f.keys_bytes + ring_min > budget) budget = kOnePerSm - 1024;
 #ifdef AOH_PHASE_TIMERS
   if (g_force_one_per_sm) budget = kOnePerSm - 1024;
 #endif
   if (f.keys_bytes + ring_min > budget) return f;
-  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kRingStep * kRingStep) : f.keys_bytes;
+  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kRingStep * kRingStep) : ring_min;
 #ifdef AOH_PHASE_TIMERS
   if (need_ring && g_force_ring) f.ring_bytes = std::min(f.ring_bytes, (size_t)g_force_ring);
 #endif

@@ -302,13 +302,16 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
           for (int j = 0; j < 4; ++j) hist_add(lh, i0 + j < m ? (int)(kk[j] >> 24) : -1);
         }
       } else {
-        for (int b0 = warp * 128; b0 < ncand; b0 += 8 * 128) {
-          const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the candidate region
-          const uint4 k4 = *reinterpret_cast<const uint4*>(cand + i0);
+        // digits 1-3: over the compacted candidates, or over all keys when they did not fit
+        const uint32_t* src = ncand >= 0 ? cand : keys;
+        const int cnt = ncand >= 0 ? ncand : m;
+        for (int b0 = warp * 128; b0 < cnt; b0 += 8 * 128) {
+          const int i0 = b0 + 4 * lane;  // i0 + 3 inside the region (4 entries of slack)
+          const uint4 k4 = *reinterpret_cast<const uint4*>(src + i0);
           const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            if (i0 + j < ncand && (kk[j] & pmask) == prefix) atomicAdd(&lh[(kk[j] >> shift) & 255u], 1);
+            if (i0 + j < cnt && (kk[j] & pmask) == prefix) atomicAdd(&lh[(kk[j] >> shift) & 255u], 1);
         }
       }
       __syncthreads();
@@ -368,8 +371,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
         }
         if (tid < CL) atomicAdd(&s_gt[tid], *cluster.map_shared_rank(&s_up, tid));
       }
-      if (pass == 0) {
-        // candidates of digits 1-3: the keys whose first digit is the chosen one
+      // candidates of digits 1-3: the keys whose first digit is the chosen one, when they fit
+      // the candidate region (this CTA's count of them is its own histogram's bin)
+      const bool compact = pass == 0 && lh[sb] <= p.ring_bytes / 4 - 4;
+      if (compact) {
         for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
           const int i0 = b0 + 4 * lane;
           const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
@@ -390,7 +395,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       krem -= s_above;
       if (pass < 3) lh[tid] = 0;  // the last histogram stays: peers read it
       __syncthreads();
-      if (pass == 0) ncand = s_ncand;
+      if (pass == 0) ncand = compact ? s_ncand : -1;
     }
     const uint32_t KT = prefix;
     const int need_eq = krem;
