@@ -102,12 +102,6 @@ __device__ __forceinline__ void phase_stamp(int slot) {
 #define AOH_PHASE(i)
 #endif
 
-// Warp-aggregated histogram increment (bin < 0: lane does not count).
-__device__ __forceinline__ void hist_add(int* h, int bin) {
-  const unsigned peers = __match_any_sync(0xffffffffu, bin);
-  if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
-}
-
 template <int D, int NT>
 __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_constant__ RowParams p) {
   static_assert(D == 64 || D == 128, "head_dim");
@@ -120,11 +114,11 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   constexpr int NQP = NT * 8;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ int lh[256];      // this CTA's histogram of the current digit
+  __shared__ int lhb[2][256];  // this CTA's histogram of digit p in lhb[p & 1] (one cleared per digit)
   __shared__ int tot[2][256];  // cluster totals of digits 0-2 (every CTA adds its counts here)
   __shared__ int scan_scratch[33];
   __shared__ float qt[128];
-  __shared__ int s_bin, s_above, s_eq_before, s_sel_before, s_ncand, s_up;
+  __shared__ int s_bin, s_above, s_eq_before, s_sel_before, s_up;
   __shared__ int s_gt[kSrMaxCluster], s_eq[kSrMaxCluster], s_eq_all;
 
   AOH_PHASE(0);
@@ -171,7 +165,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   // The select's totals are filled by every CTA of the cluster: zero them, then arrive on a
   // cluster barrier that is waited on only before the first remote add (the scan runs in between).
   if (n < L) {
-    lh[tid] = 0;
+    lhb[0][tid] = 0;
+    lhb[1][tid] = 0;
     tot[0][tid] = 0;
     tot[1][tid] = 0;
     if (tid == 0) s_up = 0;
@@ -292,14 +287,21 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
+      int* lh = lhb[pass & 1];
+      // the buffer of the next digit held digit pass - 1, whose readers passed the barrier
+      // that ended that digit
+      if (pass == 1 || pass == 2) lhb[(pass + 1) & 1][tid] = 0;
       if (pass == 0) {
-        // the first digit (sign and exponent) is shared by most keys: warp-aggregated counts
+        // the first digit (sign and exponent): plain shared-memory atomics (same-address
+        // updates of one warp are combined by the hardware; faster here than aggregating
+        // them with match.any)
         for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
           const int i0 = b0 + 4 * lane;  // i0 + 3 < slice: inside the keys region
           const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
           const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) hist_add(lh, i0 + j < m ? (int)(kk[j] >> 24) : -1);
+          for (int j = 0; j < 4; ++j)
+            if (i0 + j < m) atomicAdd(&lh[kk[j] >> 24], 1);
         }
       } else {
         // digits 1-3: over the compacted candidates, or over all keys when they did not fit
@@ -342,7 +344,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
         if (lane >= o) x += y;
       }
       if (lane == 31) scan_scratch[warp] = x;
-      if (tid == 0) s_ncand = 0;
       __syncthreads();
       int above = x - total_bin;
       for (int w2 = 0; w2 < warp; ++w2) above += scan_scratch[w2];
@@ -373,8 +374,23 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       }
       // candidates of digits 1-3: the keys whose first digit is the chosen one, when they fit
       // the candidate region (this CTA's count of them is its own histogram's bin)
-      const bool compact = pass == 0 && lh[sb] <= p.ring_bytes / 4 - 4;
+      const int n_sb = lh[sb];  // this CTA's keys in the chosen bin
+      const bool compact = pass == 0 && n_sb <= p.ring_bytes / 4 - 4;
       if (compact) {
+        // every warp counts its candidates (ballots), then writes them from its own offset
+        // (the counts of the lower warps): no shared counter
+        int wcnt = 0;
+        for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
+          const int i0 = b0 + 4 * lane;
+          const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
+          const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) wcnt += __popc(__ballot_sync(0xffffffffu, (i0 + j < m) && (int)(kk[j] >> 24) == sb));
+        }
+        if (lane == 0) scan_scratch[warp] = wcnt;
+        __syncthreads();
+        int wbase = 0;
+        for (int w2 = 0; w2 < warp; ++w2) wbase += scan_scratch[w2];
         for (int b0 = warp * 128; b0 < m; b0 += 8 * 128) {
           const int i0 = b0 + 4 * lane;
           const uint4 k4 = *reinterpret_cast<const uint4*>(keys + i0);
@@ -383,19 +399,16 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
           for (int j = 0; j < 4; ++j) {
             const bool hit = (i0 + j < m) && (int)(kk[j] >> 24) == sb;
             const unsigned bal = __ballot_sync(0xffffffffu, hit);
-            int base = 0;
-            if (lane == 0 && bal) base = atomicAdd(&s_ncand, __popc(bal));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (hit) cand[base + __popc(bal & ((1u << lane) - 1u))] = kk[j];
+            if (hit) cand[wbase + __popc(bal & ((1u << lane) - 1u))] = kk[j];
+            wbase += __popc(bal);
           }
         }
       }
       prefix |= (uint32_t)sb << shift;
       pmask |= 255u << shift;
       krem -= s_above;
-      if (pass < 3) lh[tid] = 0;  // the last histogram stays: peers read it
       __syncthreads();
-      if (pass == 0) ncand = compact ? s_ncand : -1;
+      if (pass == 0) ncand = compact ? n_sb : -1;
     }
     const uint32_t KT = prefix;
     const int need_eq = krem;

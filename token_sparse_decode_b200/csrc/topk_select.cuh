@@ -24,7 +24,8 @@
 namespace aoh {
 
 constexpr int kSelThreads = 512;
-constexpr int kSelCandCap = 24576;  // candidate keys kept in shared memory (96 KB)
+constexpr int kSelCandCap = 20480;  // candidate keys kept in shared memory (80 KB: two CTAs an SM)
+constexpr int kSelU = 8;            // row loads in flight per lane in the streaming passes
 
 struct SelectParams {
   const float* scores;            // [Hkv][T]
@@ -35,13 +36,6 @@ struct SelectParams {
   int32_t T, Hkv, n_fac, cap;
   uint8_t heads[kMaxHeads];       // KV head of blockIdx.x
 };
-
-// Warp-aggregated histogram increment (bin < 0: the lane does not count); every lane
-// of the warp must call it.
-__device__ __forceinline__ void sel_hist_add(int* h, int bin) {
-  const unsigned peers = __match_any_sync(0xffffffffu, bin);
-  if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
-}
 
 #ifdef AOH_PHASE_TIMERS
 __device__ int g_sel_dbg[4096][10];  // diagnostic build: each CTA's view of its row
@@ -54,8 +48,9 @@ __device__ int g_sel_dbg[4096][10];  // diagnostic build: each CTA's view of its
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectParams p) {
   extern __shared__ __align__(16) uint32_t cand[];  // kSelCandCap keys
   __shared__ int hist[256];
+  __shared__ int whist[kSelThreads / 32][256];  // per-warp first-digit counts (and candidate offsets)
   __shared__ int scan_scratch[33];
-  __shared__ int s_bin, s_above, s_in_bin, s_nc;
+  __shared__ int s_bin, s_above, s_in_bin;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.y;
@@ -92,6 +87,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     if (tid < 256) hist[tid] = 0;
+    if (pass == 0)
+      for (int i = tid; i < (kSelThreads / 32) * 256; i += kSelThreads) (&whist[0][0])[i] = 0;
     __syncthreads();
     if (nc >= 0) {
       for (int i = tid; i < nc; i += kSelThreads) {
@@ -99,19 +96,30 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
         if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
       }
     } else {
-      // coalesced pass over the row, four loads in flight per lane (warp-uniform trip count)
-      for (int base = warp * 32; base < L; base += 4 * kSelThreads) {
-        float v[4];
+      // coalesced pass over the row, eight loads in flight per lane; plain shared-memory
+      // atomics (the first digit into this warp's histogram)
+      int* h = pass == 0 ? whist[warp] : hist;
+      for (int base = warp * 32; base < L; base += kSelU * kSelThreads) {
+        float v[kSelU];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kSelU; ++u) {
           const int i = base + u * kSelThreads + lane;
           v[u] = i < L ? __ldcg(row + i) : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kSelU; ++u) {
           const int i = base + u * kSelThreads + lane;
           const uint32_t k = score_key(v[u]);
-          sel_hist_add(hist, (i < L && (k & pmask) == prefix) ? (int)((k >> shift) & 255u) : -1);
+          if (i < L && (k & pmask) == prefix) atomicAdd(&h[(k >> shift) & 255u], 1);
+        }
+      }
+      if (pass == 0) {
+        __syncthreads();
+        if (tid < 256) {
+          int c = 0;
+#pragma unroll
+          for (int w2 = 0; w2 < kSelThreads / 32; ++w2) c += whist[w2][tid];
+          hist[tid] = c;
         }
       }
     }
@@ -125,37 +133,38 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
       s_above = above;
       s_in_bin = tot;
     }
-    if (tid == 0) s_nc = 0;
     __syncthreads();
     prefix |= (uint32_t)s_bin << shift;
     pmask |= 255u << shift;
     krem -= s_above;
     eq_total = s_in_bin;
-    // after the first digit: compact the keys sharing it (order irrelevant: only counted)
+    // after the first digit: compact the keys sharing it (order irrelevant: only counted).
+    // Every warp writes from its own offset: the counts of the chosen bin in the lower warps.
     const bool compact = (pass == 0) && (s_in_bin <= kSelCandCap);
     if (compact) {
-      for (int base = warp * 32; base < L; base += 4 * kSelThreads) {
-        float v[4];
+      int wbase = 0;
+      for (int w2 = 0; w2 < warp; ++w2) wbase += whist[w2][s_bin];
+      for (int base = warp * 32; base < L; base += kSelU * kSelThreads) {
+        float v[kSelU];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kSelU; ++u) {
           const int i = base + u * kSelThreads + lane;
           v[u] = i < L ? __ldcg(row + i) : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kSelU; ++u) {
           const int i = base + u * kSelThreads + lane;
           const uint32_t k = score_key(v[u]);
           const bool hit = i < L && (k & pmask) == prefix;
           const unsigned bal = __ballot_sync(0xffffffffu, hit);
-          int slot = 0;
-          if (lane == 0 && bal) slot = atomicAdd(&s_nc, __popc(bal));
-          slot = __shfl_sync(0xffffffffu, slot, 0);
-          if (hit) cand[slot + __popc(bal & ((1u << lane) - 1u))] = k;
+          if (hit) cand[wbase + __popc(bal & ((1u << lane) - 1u))] = k;
+          wbase += __popc(bal);
         }
       }
     }
+    const int n_in = s_in_bin;
     __syncthreads();
-    if (compact) nc = s_nc;
+    if (compact) nc = n_in;
   }
   const uint32_t KT = prefix;
   const int need_eq = krem;    // keys equal to K_T that are taken, lowest positions first
@@ -166,13 +175,21 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
   // ---- ordered compaction: tiles of 4 * kSelThreads positions, 4 consecutive per thread
   int sel_base = 0, eq_base = 0;
   const bool all_eq = (eq_total == need_eq);  // every key equal to K_T is taken
+  // the next tile's scores are loaded while this tile is scanned
+  float vn[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) vn[j] = 4 * tid + j < L ? __ldg(row + 4 * tid + j) : 0.f;
   for (int t0 = 0; t0 < L; t0 += 4 * kSelThreads) {
     const int i0 = t0 + 4 * tid;
     uint32_t k[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) k[j] = score_key(vn[j]);
+    const int i1 = i0 + 4 * kSelThreads;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vn[j] = i1 + j < L ? __ldg(row + i1 + j) : 0.f;  // L1 merges the 4 strided loads
     int ngt = 0, neq = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      k[j] = i0 + j < L ? score_key(__ldg(row + i0 + j)) : 0u;  // L1 merges the 4 strided loads
       const bool in = i0 + j < L;
       ngt += (in && k[j] > KT);
       neq += (in && k[j] == KT);
