@@ -143,30 +143,93 @@ void fd_bind(FdecParams& fp, const FdGeom& g, uint8_t* ws) {
   fp.max_splits = g.max_splits;
 }
 
+template <typename K>
+int max_active_clusters(K kern, int CL, size_t smem, int threads = kSrThreads) {
+  // (cluster size, dynamic shared memory) -> cudaOccupancyMaxActiveClusters, cached per process
+  static std::mutex mu;
+  static int keys[64][3];  // kernel id, CL, smem / 256 << 8 | clusters (threads fixed per kernel)
+  static int n_keys = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const int kid = (int)(reinterpret_cast<uintptr_t>(reinterpret_cast<const void*>(kern)) & 0x7fffffff);
+  for (int i = 0; i < n_keys; ++i)
+    if (keys[i][0] == kid && keys[i][1] == CL && keys[i][2] >> 8 == (int)(smem >> 8)) return keys[i][2] & 0xff;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, 1, 1);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  n = std::min(n, 255);
+  if (n_keys < 64) {
+    keys[n_keys][0] = kid;
+    keys[n_keys][1] = CL;
+    keys[n_keys][2] = (int)((smem >> 8) << 8) | n;
+    ++n_keys;
+  }
+  return n;
+}
+
 template <int D, int NT>
-aoh_status launch_fd_t(const FdecParams& fp, int n_listed, int B, cudaStream_t st) {
+aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStream_t st) {
   const size_t smem = FdTile<D>::kSmem;
-  static bool configured = false;  // attribute is per function and process-wide
+  auto kern = flash_gather_kernel<D, NT>;
+  static bool configured = false;  // attributes are per function and process-wide
   if (!configured) {
-    aoh_status s = set_smem(flash_gather_kernel<D, NT>, smem);
+    aoh_status s = set_smem(kern, smem);
+    if (s != AOH_OK) return s;
+    s = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     if (s != AOH_OK) return s;
     configured = true;
   }
   dim3 grid(fp.max_splits, n_listed, B);
+  // rows of about equal length with 2..16 splits: one cluster per row, merged on chip
+  const int CL = fp.max_splits;
+  if (uniform && CL >= 2 && CL <= kFdMaxCluster && max_active_clusters(kern, CL, smem, kFdThreads) > 0) {
+    fp.cluster_combine = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kFdThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    before_launch(st);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, fp);
+    if (e != cudaSuccess) return cuda_status(e);
+    return count_launch(AOH_KERNEL_FLASH_GATHER, st);
+  }
+  fp.cluster_combine = 0;
   before_launch(st);
-  flash_gather_kernel<D, NT><<<grid, kFdThreads, smem, st>>>(fp);
+  kern<<<grid, kFdThreads, smem, st>>>(fp);
   return count_launch(AOH_KERNEL_FLASH_GATHER, st);
 }
 
-aoh_status launch_fd(const FdecParams& fp, int d, int nqp, int n_listed, int B, cudaStream_t st) {
+// `uniform`: every row attends to about the same number of positions (a fixed N_fac or k)
+aoh_status launch_fd(const FdecParams& fp, int d, int nqp, int n_listed, int B, cudaStream_t st,
+                     bool uniform = false) {
   if (d == 128) {
-    if (nqp == 8) return launch_fd_t<128, 1>(fp, n_listed, B, st);
-    if (nqp == 16) return launch_fd_t<128, 2>(fp, n_listed, B, st);
-    return launch_fd_t<128, 4>(fp, n_listed, B, st);
+    if (nqp == 8) return launch_fd_t<128, 1>(fp, n_listed, B, uniform, st);
+    if (nqp == 16) return launch_fd_t<128, 2>(fp, n_listed, B, uniform, st);
+    return launch_fd_t<128, 4>(fp, n_listed, B, uniform, st);
   }
-  if (nqp == 8) return launch_fd_t<64, 1>(fp, n_listed, B, st);
-  if (nqp == 16) return launch_fd_t<64, 2>(fp, n_listed, B, st);
-  return launch_fd_t<64, 4>(fp, n_listed, B, st);
+  if (nqp == 8) return launch_fd_t<64, 1>(fp, n_listed, B, uniform, st);
+  if (nqp == 16) return launch_fd_t<64, 2>(fp, n_listed, B, uniform, st);
+  return launch_fd_t<64, 4>(fp, n_listed, B, uniform, st);
 }
 
 // ------------------------------------------------------------------ TIP scan
@@ -339,41 +402,6 @@ bool fused_feasible(const aoh_kv_cache* kv, int nq) {
 }
 
 
-template <typename K>
-int max_active_clusters(K kern, int CL, size_t smem) {
-  // (cluster size, dynamic shared memory) -> cudaOccupancyMaxActiveClusters, cached per process
-  static std::mutex mu;
-  static int keys[64][3];
-  static int n_keys = 0;
-  std::lock_guard<std::mutex> lock(mu);
-  const int kid = (int)(reinterpret_cast<uintptr_t>(reinterpret_cast<const void*>(kern)) & 0x7fffffff);
-  for (int i = 0; i < n_keys; ++i)
-    if (keys[i][0] == kid && keys[i][1] == CL && keys[i][2] >> 8 == (int)(smem >> 8)) return keys[i][2] & 0xff;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CL, 1, 1);
-  cfg.blockDim = dim3(kSrThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    n = 0;
-  }
-  n = std::min(n, 255);
-  if (n_keys < 64) {
-    keys[n_keys][0] = kid;
-    keys[n_keys][1] = CL;
-    keys[n_keys][2] = (int)((smem >> 8) << 8) | n;
-    ++n_keys;
-  }
-  return n;
-}
 
 // Launch the cluster row kernel with the cluster size that needs the fewest waves x slice
 // length (ties to the smaller cluster).  With max_waves > 0 nothing is launched when every
@@ -771,7 +799,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   fp.scale_log2 = scale * 1.4426950408889634f;
   memcpy(fp.heads, heads, n_listed);
   fd_bind(fp, geo, ws);
-  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st);
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st, n_fac_per_seq == nullptr);
 }
 
 size_t aoh_stream_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, const uint8_t* roles,
@@ -869,7 +897,7 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
   fp.scale_log2 = scale * 1.4426950408889634f;
   memcpy(fp.heads, heads, n_listed);
   fd_bind(fp, geo, static_cast<uint8_t*>(workspace));
-  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream));
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream), true);
 }
 
 size_t shared_step_ws_bytes(const aoh_kv_cache* kv, int32_t n_layers, int32_t Hq, int32_t topk) {
@@ -958,7 +986,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   fp.scale_log2 = scale * 1.4426950408889634f;
   memcpy(fp.heads, heads, n_listed);
   fd_bind(fp, geo, ws);
-  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st);
+  return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st, true);
 }
 
 #ifdef AOH_PHASE_TIMERS

@@ -9,7 +9,9 @@
 //   * the shared-index cross-decoder layers ("Cómo funciona CLSA"): one index,
 //     NQ = n_layers * G query rows read every gathered K/V row once.
 //
-// Work split: blockIdx = (split, listed KV head, sequence).  A CTA owns `chunk`
+// Work split: blockIdx = (split, listed KV head, sequence).  When every row has about
+// the same list length and at most 16 splits, the splits of a row run as one thread-
+// block cluster and merge through distributed shared memory instead (cluster_combine).  A CTA owns `chunk`
 // consecutive list entries, streams their K and V rows through a 3-stage
 // cp.async pipeline into 128-byte-swizzled shared tiles (the layout a TMA
 // 128B-swizzle load produces), and runs the contraction on tensor cores with the
@@ -23,6 +25,8 @@
 // the partials and writes the fp32 output, then re-arms the ticket to zero.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "device_common.cuh"
 
 namespace aoh {
@@ -32,6 +36,8 @@ constexpr int kFdTS = 64;        // tokens per pipeline stage
 constexpr int kFdStages = 3;
 constexpr int kFdPosCap = 1024;  // list positions staged in shared memory per CTA
 constexpr int kFdMaxSplits = 256; // splits per row (the combine stages their weights in shared memory)
+constexpr int kFdMaxCluster = 16;  // splits of a row merged through distributed shared memory
+constexpr int kFdMergeOff = 32768; // cluster merge buffers, past the warp partials (<= 16.5 KB)
 
 struct FdecParams {
   const uint16_t* q;         // row (layer l, b, h) at q + ((l * B + b) * Hq + h) * D
@@ -49,6 +55,7 @@ struct FdecParams {
   int32_t chunk;             // list entries per CTA, multiple of kFdTS
   int32_t max_splits;
   int32_t list_mode;         // 1: positions from idx/count; 0: role ranges
+  int32_t cluster_combine;   // 1: launched with clusters of max_splits CTAs (one row each)
   int32_t sink, window;
   float scale_log2;          // softmax scale * log2(e)
   uint8_t heads[kMaxHeads];  // listed KV heads (blockIdx.y)
@@ -124,9 +131,10 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
     }
     return;
   }
-  if (split >= nsplit) return;
+  const bool clus = p.cluster_combine != 0;
+  if (split >= nsplit && !clus) return;  // in a cluster an idle split still takes part in the merge
   const int j0 = split * p.chunk;
-  const int ntok = min(n, j0 + p.chunk) - j0;
+  const int ntok = max(0, min(n, j0 + p.chunk) - j0);
   const int nstages = (ntok + kFdTS - 1) / kFdTS;
 
   // list mode: stage this CTA's positions once (one round trip instead of one per stage)
@@ -311,6 +319,62 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
   __syncthreads();
 
   // CTA result for padded query row qr: warps {nt + NT * t : t < WT} hold it.
+  if (clus) {
+    // ---- cluster merge: every CTA leaves (M, L, A) of its split in shared memory (past the
+    // warp partials), then CTA r combines outputs r, r + CL, ... over the CL splits
+    namespace cgs = cooperative_groups;
+    cgs::cluster_group cluster = cgs::this_cluster();
+    const int CLn = (int)cluster.num_blocks(), rk = (int)cluster.block_rank();
+    float* cm = reinterpret_cast<float*>(smem + kFdMergeOff);  // [NQP]
+    float* cls = cm + NQP;                                      // [NQP]
+    float* ca = cls + NQP;                                      // [NQP][D]
+    float* cw = ca + NQP * D;                                   // [16][NQP] merge weights
+    float* cinv = cw + 16 * NQP;                                // [NQP]
+    for (int e = tid; e < NQP * D; e += kFdThreads) {
+      const int qr = e / D, dd = e % D;
+      const int ntq = qr >> 3, cq = qr & 7;
+      float M = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t) * 8 + cq) * 2]);
+      float Ls = 0.f, A = 0.f;
+#pragma unroll
+      for (int t = 0; t < WT; ++t) {
+        const int w = ntq + NT * t;
+        const float mw = red_ml[(w * 8 + cq) * 2];
+        const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
+        A += f * red_acc[(w * 8 + cq) * D + dd];
+      }
+      ca[e] = A;
+      if (dd == 0) {
+        cm[qr] = M;
+        cls[qr] = Ls;
+      }
+    }
+    cluster.sync();
+    if (tid < NQP) {
+      float Mx = -INFINITY;
+      for (int q = 0; q < CLn; ++q) Mx = fmaxf(Mx, cluster.map_shared_rank(cm, q)[tid]);
+      float Ls = 0.f;
+      for (int q = 0; q < CLn; ++q) {
+        const float mq = cluster.map_shared_rank(cm, q)[tid];
+        const float w = (mq == -INFINITY) ? 0.f : exp2f(mq - Mx);
+        cw[q * NQP + tid] = w;
+        Ls += w * cluster.map_shared_rank(cls, q)[tid];
+      }
+      cinv[tid] = 1.f / Ls;
+    }
+    __syncthreads();
+    for (int e = rk * kFdThreads + tid; e < p.NQ * D; e += CLn * kFdThreads) {
+      const int qr = e / D, dd = e % D;
+      float A = 0.f;
+      for (int q = 0; q < CLn; ++q) A += cw[q * NQP + qr] * cluster.map_shared_rank(ca, q)[e];
+      const int l = qr / p.G, h = g * p.G + qr % p.G;
+      p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A * cinv[qr];
+    }
+    cluster.sync();  // peers read this CTA's shared memory until here
+    return;
+  }
   const bool single = (nsplit == 1);
   float* pml = p.part_ml + ((int64_t)row_id * p.max_splits + split) * NQP * 2;
   float* pacc = p.part_acc + ((int64_t)row_id * p.max_splits + split) * NQP * D;
