@@ -194,11 +194,12 @@ aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStr
   dim3 grid(fp.max_splits, n_listed, B);
   // rows of about equal length with 2..16 splits: one cluster per row, merged on chip
   const int CL = fp.max_splits;
-  if (uniform && CL >= 2 && CL <= kFdMaxCluster && max_active_clusters(kern, CL, smem, kFdThreads) > 0) {
+  constexpr int threads = fd_threads(NT);
+  if (uniform && CL >= 2 && CL <= kFdMaxCluster && max_active_clusters(kern, CL, smem, threads) > 0) {
     fp.cluster_combine = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(kFdThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -215,7 +216,7 @@ aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStr
   }
   fp.cluster_combine = 0;
   before_launch(st);
-  kern<<<grid, kFdThreads, smem, st>>>(fp);
+  kern<<<grid, threads, smem, st>>>(fp);
   return count_launch(AOH_KERNEL_FLASH_GATHER, st);
 }
 

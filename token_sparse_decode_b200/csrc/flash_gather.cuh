@@ -31,13 +31,17 @@
 
 namespace aoh {
 
-constexpr int kFdThreads = 128;  // 4 warps
+// token-group warps for every n-tile of 8 query rows: 4 (one or two n-tiles) or 2 (four n-tiles),
+// so a CTA has 128 or 256 threads and two fit an SM
+__host__ __device__ constexpr int fd_groups(int nt) { return nt == 4 ? 2 : 4; }
+__host__ __device__ constexpr int fd_threads(int nt) { return 32 * nt * fd_groups(nt); }
 constexpr int kFdTS = 64;        // tokens per pipeline stage
 constexpr int kFdStages = 3;
 constexpr int kFdPosCap = 1024;  // list positions staged in shared memory per CTA
 constexpr int kFdMaxSplits = 256; // splits per row (the combine stages their weights in shared memory)
 constexpr int kFdMaxCluster = 16;  // splits of a row merged through distributed shared memory
-constexpr int kFdMergeOff = 32768; // cluster merge buffers, past the warp partials (<= 16.5 KB)
+// cluster merge buffers start past the warps' partials [warps][8][2 + D] floats
+__host__ __device__ constexpr int fd_merge_off(int nt, int d) { return ((nt * fd_groups(nt) * 8 * (2 + d) * 4) + 255) & ~255; }
 
 struct FdecParams {
   const uint16_t* q;         // row (layer l, b, h) at q + ((l * B + b) * Hq + h) * D
@@ -78,11 +82,14 @@ __device__ __forceinline__ uint32_t fd_tile_off(int r, int dd) {
 }
 
 template <int D, int NT>
-__global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecParams p) {
+__global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const FdecParams p) {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
   constexpr int KS = D / 16;         // k-steps of QK, m-tiles of PV
-  constexpr int WT = 4 / NT;         // token groups (warps sharing one n-tile)
+  constexpr int WT = fd_groups(NT);  // token groups (warps sharing one n-tile)
+  constexpr int kFdThreads = fd_threads(NT);
+  constexpr int NW = kFdThreads / 32;
+  constexpr int kFdMergeOff = fd_merge_off(NT, D);
   constexpr int SUB = kFdTS / 16;    // 16-token sub-tiles per stage
   constexpr int NQP = NT * 8;        // padded query rows
   constexpr int CPR = D / 8;         // 16-byte chunks per row
@@ -297,8 +304,8 @@ __global__ void __launch_bounds__(kFdThreads) flash_gather_kernel(const FdecPara
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
   __syncthreads();  // every warp is done with the stage buffers
-  float* red_ml = reinterpret_cast<float*>(smem);             // [4 warps][8][2]
-  float* red_acc = red_ml + 4 * 8 * 2;                        // [4 warps][8][D]
+  float* red_ml = reinterpret_cast<float*>(smem);             // [NW warps][8][2]
+  float* red_acc = red_ml + NW * 8 * 2;                       // [NW warps][8][D]
   {
     const int c0 = 2 * (lane & 3);
     if (lane < 4) {
