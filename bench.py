@@ -12,9 +12,11 @@ together), and the algorithmic HBM bytes per second of the step and of its
 dominant kernel against the measured copy bandwidth.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
-the launching stream; L2 is flushed (a 2 x L2 buffer is rewritten) between
-steps, outside the events.  Barrier + synchronize on both sides, max over
-ranks.  Multi-GPU: every rank decodes its own independent batch (weak scaling,
+the launching stream.  Every step starts with its inputs out of L2: the steps
+rotate over R device copies of the inputs, R chosen so that the other copies'
+traffic between two uses of a copy is at least twice the L2 size (a step too
+small for that at R <= 8 flushes L2 instead, by rewriting a 2 x L2 buffer
+outside the events).  Barrier + synchronize on both sides, max over ranks.  Multi-GPU: every rank decodes its own independent batch (weak scaling,
 no collective on the data path); NCCL is used only for the barrier and the
 max-reduction of the timings.
 
@@ -209,25 +211,28 @@ def launches_per_step(step, q) -> dict:
     return {k: c1[k] - c0[k] for k in c0 if c1[k] != c0[k]}
 
 
-def kernel_timing(w, step, q, steps: int, flush) -> dict:
+def kernel_timing(w, copies, steps: int, between) -> dict:
     """Device time of every kernel of the step, per public call.
 
     Each call runs with the library's launch-event recording armed, so every kernel is
-    bracketed by CUDA events recorded on its own stream right before and after it.  Each
-    sample runs behind a device-side sleep, so that the host has queued the calls before
-    the first one starts; L2 is flushed before every sample.
+    bracketed by CUDA events recorded on its own stream right before and after it.  Sample i
+    runs on input copy i mod R (see cold_copies) behind a device-side sleep, so that the host
+    has queued the calls before the first one starts; `between()` runs before every sample.
     """
     from token_sparse_decode_b200 import binding as B
 
-    calls = step_calls(w, step, q)
-    for _, fn in calls:
-        fn()
+    per_copy = [step_calls(w, step, q) for step, q in copies]
+    for calls in per_copy:
+        for _, fn in calls:
+            fn()
     torch.cuda.synchronize()
-    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in calls]
-    per, call_ms, order = {}, {n: [] for n, _ in calls}, {}
-    for _ in range(steps):
-        flush()
+    names = [n for n, _ in per_copy[0]]
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in names]
+    per, call_ms, order = {}, {n: [] for n in names}, {}
+    for it in range(steps):
+        between()
         torch.cuda._sleep(1000000)
+        calls = per_copy[it % len(per_copy)]
         recs = [(name, B.timed_launches(fn, evs)) for (name, fn), evs in zip(calls, evsets)]
         torch.cuda.synchronize()
         for name, r in recs:
@@ -238,6 +243,24 @@ def kernel_timing(w, step, q, steps: int, flush) -> dict:
                 call_ms[name].append(r[0][1].elapsed_time(r[-1][2]))
     kernels = [{"call": n, "index": i, "kernel": k, "ms": float(np.mean(t))} for (n, i, k), t in sorted(per.items())]
     return {"calls": {n: float(np.mean(t)) for n, t in call_ms.items() if t}, "kernels": kernels, "order": order}
+
+
+MAX_COPIES = 8
+
+
+def cold_copies(step_bytes: int, l2_bytes: int) -> int:
+    """Input copies R to rotate over so that every step starts with its inputs out of L2.
+
+    Copy i is reused R steps later, after R - 1 other steps have moved (R - 1) * step_bytes
+    through L2; R is the smallest count (at least 2) for which that is at least twice the L2
+    size.  Returns 0 when more than MAX_COPIES would be needed (then L2 is flushed instead).
+    """
+    r = 2
+    while (r - 1) * step_bytes < 2 * l2_bytes:
+        r += 1
+        if r > MAX_COPIES:
+            return 0
+    return r
 
 
 def kernel_bytes(w, ab: dict, call: str, kernel: str, order: list) -> int:
@@ -302,79 +325,105 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     spec = shard_spec(preset(args.workload), rank, world)
     w = make_workload(spec)
-    step, q = build_step(w, dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    ab = algorithmic_bytes(w)
+    # Cold inputs every step: rotate over R device copies of the inputs (each step's traffic
+    # pushes the other copies out of L2), or, for steps too small for that, flush L2 by
+    # rewriting a buffer of twice its size between steps (outside the events).
+    R = cold_copies(ab["total"], l2) if args.copies == 0 else (args.copies if args.copies > 1 else 0)
+    copies = [build_step(w, dev) for _ in range(max(R, 1))]
+    step, q = copies[0]
+    if R:
+        def between():
+            pass
+        l2_note = (f"inputs rotated over {R} device copies ({R - 1} x {ab['total']} B of step traffic "
+                   f"between reuses of a copy, >= 2 x L2); no flush")
+    else:
+        flush_buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
-    def flush():
-        flush_buf.fill_(1)
+        def between():
+            flush_buf.fill_(1)
+        l2_note = "flushed between timed steps (2 x L2 buffer rewritten, outside the events)"
 
-    step(*q)  # first call outside capture (sets kernel attributes)
+    for s_, q_ in copies:
+        s_(*q_)  # first call outside capture (sets kernel attributes)
     torch.cuda.synchronize()
     per_step = launches_per_step(step, q)
     if args.graph:
-        g_step = capture_graph(lambda: step(*q))
-        one = g_step.replay
+        graphs = [capture_graph(lambda s_=s_, q_=q_: s_(*q_)) for s_, q_ in copies]
+
+        def one(i):
+            graphs[i % len(graphs)].replay()
     else:
-        def one():
-            return step(*q)
+        def one(i):
+            s_, q_ = copies[i % len(copies)]
+            return s_(*q_)
 
     st = torch.cuda.current_stream()
     sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
     t_wall0 = time.time()
-    for _ in range(args.warmup):
-        one()
-        flush()
+    for i in range(args.warmup):
+        one(i)
+        between()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for e0, e1 in evs:
+    for i, (e0, e1) in enumerate(evs):
         e0.record(st)
-        one()
+        one(args.warmup + i)
         e1.record(st)
-        flush()
+        between()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
     # keep the GPU loaded until the clock sampler has seen a few samples
+    i = 0
     while time.time() - t_wall0 < 1.5:
-        one()
-        flush()
+        one(i)
+        between()
+        i += 1
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
 
     # end-to-end through the public API with host buffers: H2D of q, the step, D2H of the output
     q_host = [t.cpu().pin_memory() for t in q]
-    q_dev = [t.clone() for t in q]
     out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in q_host)
     d2h = out_host.numel() * out_host.element_size()
-    def host_step():
-        for a, b_ in zip(q_dev, q_host):
+
+    def host_step(s_, q_):
+        for a, b_ in zip(q_, q_host):
             a.copy_(b_, non_blocking=True)
-        out = step(*q_dev)
+        out = s_(*q_)
         out_host.copy_(out, non_blocking=True)
 
-    e2e_one = capture_graph(host_step).replay if args.graph else host_step
-    for _ in range(max(1, args.warmup)):
-        e2e_one()
-        flush()
+    if args.graph:
+        e2e_graphs = [capture_graph(lambda s_=s_, q_=q_: host_step(s_, q_)) for s_, q_ in copies]
+
+        def e2e_one(i):
+            e2e_graphs[i % len(e2e_graphs)].replay()
+    else:
+        def e2e_one(i):
+            host_step(*copies[i % len(copies)])
+    for i in range(max(1, args.warmup)):
+        e2e_one(i)
+        between()
     torch.cuda.synchronize()
     e2e_ms = 0.0
-    for _ in range(args.steps):
+    for i in range(args.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(st)
-        e2e_one()
+        e2e_one(i)
         e1.record(st)
         torch.cuda.synchronize()
         e2e_ms += e0.elapsed_time(e1)
-        flush()
+        between()
 
-    kt = kernel_timing(w, step, q, args.steps if args.steps <= 200 else 200, flush)
+    kt = kernel_timing(w, copies, args.steps if args.steps <= 200 else 200, between)
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
@@ -382,7 +431,6 @@ def run_ours(args, rank, world, local_rank):
     ms_step = ms / args.steps
     value = aggregate_throughput(tokens_step, world, ms_step)
     e2e_value = aggregate_throughput(tokens_step, world, e2e_ms / args.steps)
-    ab = algorithmic_bytes(w)
     peak, peak_kind = measured_peak_gbs()
     # the dominant kernel: the largest device time of one step
     dom = max(kt["kernels"], key=lambda e: e["ms"]) if kt["kernels"] else None
@@ -408,7 +456,7 @@ def run_ours(args, rank, world, local_rank):
             "tokens_per_step_per_gpu": tokens_step, "q_heads": w.spec.n_q_heads, "kv_heads": w.spec.n_kv_heads,
             "head_dim": w.spec.head_dim, "n_dom": w.spec.n_dom, "n_fac": int(w.n_fac_per_seq.max()),
             "n_layers": w.spec.n_layers, "parallelism": f"independent sequences per rank x{world}",
-            "l2": "flushed between timed steps (2 x L2 buffer rewritten, outside the events)",
+            "l2": l2_note,
             "launch": "CUDA graph replay" if args.graph else "direct launches",
             "algorithmic_bytes_per_step": ab["total"],
         },
@@ -517,6 +565,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", type=int, default=1, help="replay each step from a CUDA graph (1) or launch (0)")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="input copies to rotate over (0: enough for cold inputs; 1: one copy, L2 flushed)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
