@@ -147,7 +147,9 @@ void aoh_record_launch_events(void** events, int32_t* kinds, int32_t n);
  * aoh_device_check -- synchronise `stream`, then read and clear this
  * device's error word.  Returns AOH_OK, AOH_ERR_DEVICE_CHECK (and, if
  * `detail` is not NULL, writes 4 host int32: check id, then three values of
- * the first failing access), or AOH_ERR_CUDA.
+ * the first failing access), or AOH_ERR_CUDA.  Check ids: 1 a position
+ * outside [0, L_b) or offsets past the cache, 2 a count or per-sequence
+ * N_fac above the capacity, 3 a chunk id outside [0, d/2).
  */
 aoh_status aoh_device_check(void* stream, int32_t* detail);
 

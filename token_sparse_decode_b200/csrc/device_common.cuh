@@ -17,7 +17,6 @@ enum DeviceCheck : int {
   kCheckPosition = 1,    // a stored position outside [0, L_b)
   kCheckCount = 2,       // a count or per-sequence N_fac above the row capacity
   kCheckChunk = 3,       // a chunk id outside [0, d/2)
-  kCheckTimeout = 4,     // a bounded wait for an asynchronous copy gave up
 };
 
 __device__ int g_device_error[4];
@@ -91,51 +90,6 @@ __device__ __forceinline__ void cp_async_wait_n(int n) {
   }
 }
 
-// ------------------------------------------------------------------ TMA and mbarriers
-// Bulk / tensor copies complete on an mbarrier (transaction count).  No multicast.
-constexpr int kWaitLimit = 1 << 24;  // try_wait rounds before a wait is given up as failed
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false if the phase did not complete within kWaitLimit rounds.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (int i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
-}
-// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-// 2-D tensor tile global -> shared through a tensor map (kernel-parameter address).
-__device__ __forceinline__ void tma_tile_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
-      "l"(tmap), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
 // ------------------------------------------------------------------ tensor-core fragments
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -171,11 +125,6 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 }
 
 // ------------------------------------------------------------------ small reductions
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // Block-wide exclusive scan of one int per thread (blockDim.x <= 1024, multiple of 32).
 // `scratch` holds >= 33 ints of shared memory.  Returns the exclusive prefix; *total

@@ -428,21 +428,24 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
   const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
   // weights w[s][q] = 2^(m_sq - M_q) staged in shared memory (nsplit * NQP <= kFdMaxSplits * NQP fits).
-  // The partials sit in L2: every loop below keeps 8 independent loads in flight per thread.
+  // The partials sit in L2: the max and sum run over all threads, the weighted sum keeps 16
+  // independent loads in flight per thread.
   float* sw = reinterpret_cast<float*>(smem);        // [nsplit][NQP]
   float* sM = sw + nsplit * NQP;                     // [NQP]
   float* sL = sM + NQP;                              // [NQP]
+  float* sred = sL + NQP;                            // [kFdThreads]: per-thread partial max / sum
+  // every thread takes query row tid % NQP over the splits j, j + SP, ... (SP = threads / NQP)
+  constexpr int SP = kFdThreads / NQP;
+  const int rq = tid % NQP, sj = tid / NQP;
+  {
+    float M = -INFINITY;
+    for (int s2 = sj; s2 < nsplit; s2 += SP) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + rq) * 2));
+    sred[tid] = M;
+  }
+  __syncthreads();
   if (tid < NQP) {
     float M = -INFINITY;
-    int s2 = 0;
-    for (; s2 + 8 <= nsplit; s2 += 8) {
-      float mv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mv[u] = __ldcg(rml + ((int64_t)(s2 + u) * NQP + tid) * 2);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) M = fmaxf(M, mv[u]);
-    }
-    for (; s2 < nsplit; ++s2) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2));
+    for (int j = 0; j < SP; ++j) M = fmaxf(M, sred[j * NQP + tid]);
     sM[tid] = M;
   }
   __syncthreads();
@@ -451,17 +454,15 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     sw[e] = exp2f(__ldcg(rml + (int64_t)e * 2) - sM[qr]);
   }
   __syncthreads();
+  {
+    float Ls = 0.f;
+    for (int s2 = sj; s2 < nsplit; s2 += SP) Ls += sw[s2 * NQP + rq] * __ldcg(rml + ((int64_t)s2 * NQP + rq) * 2 + 1);
+    sred[tid] = Ls;
+  }
+  __syncthreads();
   if (tid < NQP) {
     float Ls = 0.f;
-    int s2 = 0;
-    for (; s2 + 8 <= nsplit; s2 += 8) {
-      float lv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) lv[u] = __ldcg(rml + ((int64_t)(s2 + u) * NQP + tid) * 2 + 1);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) Ls += sw[(s2 + u) * NQP + tid] * lv[u];
-    }
-    for (; s2 < nsplit; ++s2) Ls += sw[s2 * NQP + tid] * __ldcg(rml + ((int64_t)s2 * NQP + tid) * 2 + 1);
+    for (int j = 0; j < SP; ++j) Ls += sred[j * NQP + tid];
     sL[tid] = Ls;
   }
   __syncthreads();
@@ -471,12 +472,12 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     const float* col = racc + (int64_t)qr * D + dd;
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
     int s2 = 0;
-    for (; s2 + 8 <= nsplit; s2 += 8) {
-      float4 v[8];
+    for (; s2 + 16 <= nsplit; s2 += 16) {
+      float4 v[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)(s2 + u) * NQP * D));
+      for (int u = 0; u < 16; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)(s2 + u) * NQP * D));
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const float w = sw[(s2 + u) * NQP + qr];
         A.x += w * v[u].x;
         A.y += w * v[u].y;
