@@ -127,6 +127,37 @@ def test_topk_bit_exact_on_given_scores(kind):
             assert np.all(idx_h[b, g, n:] == -1)
 
 
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
+def test_topk_many_rows_one_cta_per_row(kind):
+    # 54 sequences x 3 KV heads = 162 rows, more than the SMs: the one-CTA-per-row select.
+    # Lengths mix empty, one-token, N_fac >= L and long rows; the ties / zeros kinds put more
+    # keys in the first digit's bin than its shared-memory candidate region holds (re-read path).
+    rng = np.random.default_rng(15)
+    lengths = [0, 1, 3, 700, 24000, 60000] + [int(x) for x in rng.integers(50, 9000, 48)]
+    Hkv = 3
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = given_scores(rng, lengths, Hkv, kind)
+    nfps = np.array([4, 1, 9, 700, 2048, 1500] + [int(x) for x in rng.integers(1, 2049, 48)], dtype=np.int32)
+    cap = 2048
+    dev = torch.device("cuda")
+    k = torch.zeros((int(offs[-1]), Hkv, 64), dtype=torch.bfloat16, device=dev)
+    kv = B.make_kv(k, k, torch.from_numpy(offs).to(dev), max(lengths), int(offs[-1]))
+    idx = torch.full((len(lengths), Hkv, cap), 12345, dtype=torch.int32, device=dev)
+    cnt = torch.full((len(lengths), Hkv), -7, dtype=torch.int32, device=dev)
+    sd, nd = torch.from_numpy(s).to(dev), torch.from_numpy(nfps).to(dev)
+    launched = launches_of(lambda: B.topk_select(sd, kv, 0, nd, cap, idx, cnt))
+    assert launched == {"topk_select_kernel": 1}
+    check_device()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b, L in enumerate(lengths):
+        for g in range(Hkv):
+            ref = oracle.select_top(s[g, offs[b]:offs[b + 1]], int(nfps[b]))
+            n = len(ref)
+            assert cnt_h[b, g] == n, (kind, b, g)
+            assert np.array_equal(idx_h[b, g, :n], ref), (kind, b, g)
+            assert np.all(idx_h[b, g, n:] == -1), (kind, b, g)
+
+
 def test_topk_fixed_nfac_and_determinism():
     rng = np.random.default_rng(6)
     lengths = [131072, 4096, 777]
