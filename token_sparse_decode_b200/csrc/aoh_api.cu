@@ -98,6 +98,26 @@ aoh_status set_smem(F* kernel, size_t bytes) {
   return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
 }
 
+// One-time set-up per device: function attributes apply to the current device only, so a
+// process that drives several GPUs sets them once on each.  `done` is a per-call-site mask
+// of device ordinals (devices 0..63).
+inline bool set_up_on_this_device(std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
+  }
+  return (done.load(std::memory_order_acquire) >> (dev & 63)) & 1ull;
+}
+inline void mark_set_up(std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
+  }
+  done.fetch_or(1ull << (dev & 63), std::memory_order_release);
+}
+
 // ------------------------------------------------------------------ gather-kernel geometry
 struct FdGeom {
   int chunk;
@@ -183,13 +203,13 @@ template <int D, int NT>
 aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStream_t st) {
   const size_t smem = FdTile<D>::kSmem;
   auto kern = flash_gather_kernel<D, NT>;
-  static bool configured = false;  // attributes are per function and process-wide
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  if (!set_up_on_this_device(configured)) {
     aoh_status s = set_smem(kern, smem);
     if (s != AOH_OK) return s;
     s = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     if (s != AOH_OK) return s;
-    configured = true;
+    mark_set_up(configured);
   }
   dim3 grid(fp.max_splits, n_listed, B);
   // rows of about equal length with 2..16 splits: one cluster per row, merged on chip
@@ -318,11 +338,11 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
   sp.cap = cap;
   memcpy(sp.heads, heads, n_listed);
   const size_t smem = size_t(kSelCandCap) * 4;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  if (!set_up_on_this_device(configured)) {
     aoh_status s = set_smem(topk_select_kernel, smem);
     if (s != AOH_OK) return s;
-    configured = true;
+    mark_set_up(configured);
   }
   before_launch(st);
   topk_select_kernel<<<dim3(n_listed, kv->batch), kSelThreads, smem, st>>>(sp);
@@ -412,13 +432,13 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
                          int max_waves, bool* launched) {
   *launched = false;
   auto kern = sparse_row_kernel<D, NT>;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  if (!set_up_on_this_device(configured)) {
     aoh_status s = set_smem(kern, kOnePerSm);
     if (s != AOH_OK) return s;
     s = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     if (s != AOH_OK) return s;
-    configured = true;
+    mark_set_up(configured);
   }
   const int n_rows = n_listed * B;
   FusedPlan best{};
