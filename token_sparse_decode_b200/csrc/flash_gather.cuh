@@ -9,20 +9,20 @@
 //   * the shared-index cross-decoder layers ("Cómo funciona CLSA"): one index,
 //     NQ = n_layers * G query rows read every gathered K/V row once.
 //
-// Work split: blockIdx = (split, listed KV head, sequence).  When every row has about
-// the same list length and at most 16 splits, the splits of a row run as one thread-
-// block cluster and merge through distributed shared memory instead (cluster_combine).  A CTA owns `chunk`
-// consecutive list entries, streams their K and V rows through a 3-stage
-// cp.async pipeline into 128-byte-swizzled shared tiles (the layout a TMA
-// 128B-swizzle load produces), and runs the contraction on tensor cores with the
-// tokens on the M side:
+// Work split: blockIdx = (split, listed KV head, sequence).  A CTA owns `chunk`
+// consecutive list entries, streams their K and V rows through a 3-stage cp.async
+// pipeline into 128-byte-swizzled shared tiles, and runs the contraction on tensor
+// cores with the tokens on the M side:
 //     S^T[16 tok x 8 q] = K[16 tok x d] . Q^T[d x 8 q]          (m16n8k16, bf16)
 //     O^T[d x 8 q]     += V^T[d x 16 tok] . P^T[16 tok x 8 q]
 // so G <= 8 query rows fill the N = 8 side of one MMA (G = 7: 7/8 useful) instead
-// of padding 16 rows.  P goes from the accumulator layout to the B-operand layout
-// with movmatrix.trans.  Softmax is online in fp32 (exp2 domain).  Each CTA
-// writes (m, l, acc) for its chunk; the last CTA of a row (atomic ticket) merges
-// the partials and writes the fp32 output, then re-arms the ticket to zero.
+// of padding 16 rows.  NT n-tiles of 8 query rows, each with 4 (NT <= 2) or 2
+// (NT = 4) warps over the stage's 16-token sub-tiles.  P goes from the accumulator
+// layout to the B-operand layout with movmatrix.trans.  Softmax is online in fp32
+// (exp2 domain).  Each CTA leaves (m, l, acc) for its chunk; they are merged either
+// in a thread-block cluster of the row's splits (rows of about equal length with
+// 2-16 splits: distributed shared memory, each CTA writes 1/CL of the outputs) or by
+// the last CTA of the row through the workspace (atomic ticket, re-armed to zero).
 #pragma once
 
 #include <cooperative_groups.h>

@@ -16,12 +16,15 @@
 //  2. select:  4-digit MSB radix select of the n-th largest key over the cluster
 //              (histograms summed through distributed shared memory, one cluster
 //              barrier per digit); ties broken toward lower positions by an ordered
-//              compaction that also writes the index (ascending) to global memory;
+//              compaction that also writes the index (ascending) to global memory.
+//              Select-only mode (three-kernel form) loads the keys from given
+//              scores and stops here;
 //  3. attend:  every CTA gathers the K / V rows of the positions it selected from
-//              its own slice (cp.async into 128B-swizzled tiles) and runs the
-//              online-softmax contraction on tensor cores (tokens on M, query rows
-//              on N, P as hi + lo bf16 parts), 8 warps = 4 token/row groups x 2
-//              halves of the head dimension for the PV product;
+//              its own slice (cp.async into tiles at a 2*d+16-byte row pitch) and
+//              runs the online-softmax contraction on tensor cores (tokens on M,
+//              query rows on N, P as hi + lo bf16 parts); the 8 warps split the
+//              tokens, the query n-tiles and 2-4 parts of the head dimension of
+//              the PV product;
 //  4. combine: the CL partial (m, l, acc) states are merged through distributed
 //              shared memory, each CTA writing 1/CL of the outputs.
 // Nothing but the index and the outputs goes to global memory; no global

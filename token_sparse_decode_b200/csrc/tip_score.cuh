@@ -4,9 +4,10 @@
 //   q~_g = sum over the group's q heads of q_h, restricted to the dominant dims
 //          {c, c + d/2 : c in I_dom[g]} (zero elsewhere)
 // with the key row.  By linearity this is the per-head chunk sum of the method
-// aggregated over the GQA group.  The kernel is a streaming GEMV: every key row
-// is read once with 16-byte vector loads, S = row_bytes/16 lanes share a row and
-// reduce with shuffles.  Two row sources:
+// aggregated over the GQA group.  The kernel is a persistent streaming GEMV: every
+// CTA streams an equal share of the (head, token) rows, every key row is read once
+// with 16-byte vector loads, S = row_bytes/16 lanes share a row and reduce with
+// shuffles.  Two row sources:
 //   packed   k_dom[g][t][0 .. cols)  (dominant columns only: 4*n_dom bytes a row)
 //   in place K[t][g][0 .. d)         (16-byte segments holding no dominant dim
 //                                     are not loaded)
