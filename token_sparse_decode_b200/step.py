@@ -6,9 +6,11 @@ attention (one ``aoh_sparse_decode`` call); DENSE / STREAM heads run
 ``aoh_stream_decode``.  Both write into one fp32 output.
 
 ``SharedIndexStep``: the shared-index cross-decoder stack.  The indexer scores
-every cached token with the full-dimension q.k (``aoh_tip_score`` with every
-chunk), takes one top-k (``aoh_topk_select``) and every layer attends over that
-index (``aoh_shared_index_decode``).
+every cached token with the full-dimension q.k, takes one top-k and every layer
+attends over that index.  By default that is one ``aoh_shared_index_step`` call
+(the library runs it as one cluster kernel or as scan, select and gather kernels);
+``fused=False`` makes the three public calls instead (``aoh_tip_score`` with every
+chunk, ``aoh_topk_select``, ``aoh_shared_index_decode``).
 
 Every call is asynchronous on the current torch stream; nothing is computed in
 Python.
@@ -87,15 +89,22 @@ class SharedIndexStep:
         batch = offsets.numel() - 1
         self.n_layers, self.n_q_heads, self.topk, self.scale = n_layers, n_q_heads, int(topk), float(scale)
         self.all_chunks = torch.arange(d // 2, dtype=torch.int32, device=self.dev).repeat(Hkv, 1).contiguous()
-        self.scores = torch.empty((Hkv, max(total_tokens, 1)), dtype=torch.float32, device=self.dev)
         self.idx = torch.empty((batch, Hkv, self.topk), dtype=torch.int32, device=self.dev)
         self.count = torch.empty((batch, Hkv), dtype=torch.int32, device=self.dev)
-        self.ws = B.workspace(B.shared_index_decode_workspace_size(self.kv, n_layers, n_q_heads, self.topk), self.dev)
-        self.ws_step = B.workspace(B.shared_index_step_workspace_size(self.kv, n_layers, n_q_heads, self.topk),
-                                   self.dev) if fused else None
+        if fused:  # the step's workspace holds its own scores
+            self.scores = self.ws = None
+            self.ws_step = B.workspace(B.shared_index_step_workspace_size(self.kv, n_layers, n_q_heads, self.topk),
+                                       self.dev)
+        else:
+            self.scores = torch.empty((Hkv, max(total_tokens, 1)), dtype=torch.float32, device=self.dev)
+            self.ws = B.workspace(B.shared_index_decode_workspace_size(self.kv, n_layers, n_q_heads, self.topk),
+                                  self.dev)
+            self.ws_step = None
         self.out = torch.zeros((n_layers, batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
 
     def index(self, q_index: torch.Tensor) -> None:
+        if self.scores is None:
+            raise RuntimeError("SharedIndexStep.index needs fused=False (the fused step keeps its scores inside)")
         B.tip_score(q_index, self.kv, self.all_chunks, self.all_chunks.shape[1], self.scores)
         B.topk_select(self.scores, self.kv, self.topk, None, self.topk, self.idx, self.count)
 
