@@ -1,0 +1,164 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in the oracle (on the CPU, through monkeypatch: the
+oracle package and its module both see the mutant) and runs every pin of
+test_oracle_pins.py; at least one pin must fail.  The mutants are the mistakes a
+restatement of the method could plausibly make: a RoPE rotation of the wrong
+sense, the wrong pairing of dims or a wrong frequency; a TIP that drops the
+c + d/2 term or scores one head of the group; a select that breaks ties toward
+the higher position or returns positions in score order; attention without the
+scale or with keys where values belong; a streaming window one token short.
+"""
+
+import inspect
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.reference as ref
+import test_oracle_pins as pins
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_example.json")
+
+
+def rope_wrong_sense(x, positions, theta):
+    x = np.asarray(x, dtype=np.float64)
+    n, d = x.shape
+    C = d // 2
+    out = np.empty_like(x)
+    for c in range(C):
+        w = theta ** (-2.0 * c / d)
+        for i in range(n):
+            a = float(positions[i]) * w
+            ca, sa = math.cos(a), math.sin(a)
+            u, v = x[i, c], x[i, c + C]
+            out[i, c] = ca * u + sa * v
+            out[i, c + C] = -sa * u + ca * v
+    return out
+
+
+def rope_interleaved(x, positions, theta):
+    x = np.asarray(x, dtype=np.float64)
+    n, d = x.shape
+    out = np.empty_like(x)
+    for c in range(d // 2):
+        w = theta ** (-2.0 * c / d)
+        for i in range(n):
+            a = float(positions[i]) * w
+            ca, sa = math.cos(a), math.sin(a)
+            u, v = x[i, 2 * c], x[i, 2 * c + 1]
+            out[i, 2 * c] = ca * u - sa * v
+            out[i, 2 * c + 1] = sa * u + ca * v
+    return out
+
+
+def rope_half_frequency(x, positions, theta):
+    x = np.asarray(x, dtype=np.float64)
+    n, d = x.shape
+    C = d // 2
+    out = np.empty_like(x)
+    for c in range(C):
+        w = theta ** (-1.0 * c / d)
+        for i in range(n):
+            a = float(positions[i]) * w
+            ca, sa = math.cos(a), math.sin(a)
+            u, v = x[i, c], x[i, c + C]
+            out[i, c] = ca * u - sa * v
+            out[i, c + C] = sa * u + ca * v
+    return out
+
+
+def tip_first_half_only(q_group, keys, idom):
+    q_group = np.asarray(q_group, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    s = np.zeros(keys.shape[0])
+    for h in range(q_group.shape[0]):
+        for c in idom:
+            s += q_group[h, int(c)] * keys[:, int(c)]
+    return s
+
+
+def tip_one_head(q_group, keys, idom):
+    return ref.__wrapped_tip(np.asarray(q_group)[:1], keys, idom)
+
+
+def select_ties_high(scores, n):
+    scores = np.asarray(scores)
+    L = scores.shape[0]
+    n = min(int(n), L)
+    if n <= 0:
+        return np.zeros(0, dtype=np.int64)
+    order = np.lexsort((-np.arange(L), -scores.astype(np.float64)))
+    return np.sort(order[:n]).astype(np.int64)
+
+
+def select_score_order(scores, n):
+    scores = np.asarray(scores)
+    L = scores.shape[0]
+    n = min(int(n), L)
+    if n <= 0:
+        return np.zeros(0, dtype=np.int64)
+    return np.lexsort((np.arange(L), -scores.astype(np.float64)))[:n].astype(np.int64)
+
+
+def attend_no_scale(q, keys, values, scale):
+    return ref.__wrapped_attend(q, keys, values, 1.0)
+
+
+def attend_keys_for_values(q, keys, values, scale):
+    return ref.__wrapped_attend(q, keys, keys, scale)
+
+
+def stream_window_short(L, sink, window):
+    keep = set(range(0, min(sink, L))) | set(range(max(0, L - window + 1), L))
+    return np.array(sorted(keep), dtype=np.int64)
+
+
+MUTANTS = {
+    "rope_wrong_sense": ("rope", rope_wrong_sense),
+    "rope_interleaved_pairs": ("rope", rope_interleaved),
+    "rope_half_frequency": ("rope", rope_half_frequency),
+    "tip_drops_c_plus_half": ("tip_scores", tip_first_half_only),
+    "tip_scores_one_head": ("tip_scores", tip_one_head),
+    "select_ties_to_higher_position": ("select_top", select_ties_high),
+    "select_in_score_order": ("select_top", select_score_order),
+    "attend_without_scale": ("attend", attend_no_scale),
+    "attend_keys_as_values": ("attend", attend_keys_for_values),
+    "stream_window_one_short": ("stream_positions", stream_window_short),
+}
+
+
+def run_pins():
+    """Names of the pins that fail (any exception) with the oracle as it is now."""
+    with open(GOLDEN) as f:
+        hand = json.load(f)
+    failed = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        args = [hand if p == "hand" else None for p in inspect.signature(fn).parameters]
+        try:
+            fn(*args)
+        except Exception:  # an assertion, or a shape error the mistake causes
+            failed.append(name)
+    return failed
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert run_pins() == []
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_mutant_is_caught(mutant, monkeypatch):
+    attr, fn = MUTANTS[mutant]
+    # helpers some mutants call: the original functions
+    monkeypatch.setattr(ref, "__wrapped_tip", ref.tip_scores, raising=False)
+    monkeypatch.setattr(ref, "__wrapped_attend", ref.attend, raising=False)
+    monkeypatch.setattr(ref, attr, fn)
+    monkeypatch.setattr(oracle, attr, fn)
+    failed = run_pins()
+    assert failed, f"no pin catches the mutant {mutant}"
