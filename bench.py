@@ -461,15 +461,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; bf16 N(0,1) post-RoPE q/K, V; planted salient keys where the workload has them)",
-        "config": {
-            "workload": w.spec.name, "batch": w.spec.batch, "seq_len": int(w.max_len),
-            "tokens_per_step_per_gpu": tokens_step, "q_heads": w.spec.n_q_heads, "kv_heads": w.spec.n_kv_heads,
-            "head_dim": w.spec.head_dim, "n_dom": w.spec.n_dom, "n_fac": int(w.n_fac_per_seq.max()),
-            "n_layers": w.spec.n_layers, "parallelism": f"independent sequences per rank x{world}",
-            "l2": l2_note,
-            "launch": "CUDA graph replay" if args.graph else "direct launches",
-            "algorithmic_bytes_per_step": ab["total"],
-        },
+        "config": dict(workload_config(w, world), l2=l2_note,
+                       launch="CUDA graph replay" if args.graph else "direct launches"),
         "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
                      "bytes_per_step": ab["total"]},
         "roofline": {"kernel": dom["kernel"] if dom else None, "call": dom["call"] if dom else None, "bound": "hbm",
@@ -537,6 +530,18 @@ def cpu_baseline(w, seconds: float = 15.0) -> dict:
                       f"BLAS limited to 1 thread, {dt:.1f} s"}
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` of the JSON line: the workload, its shape and the step's algorithmic bytes."""
+    return {
+        "workload": w.spec.name, "batch": w.spec.batch, "seq_len": int(w.max_len),
+        "tokens_per_step_per_gpu": int(w.lengths.sum()), "q_heads": w.spec.n_q_heads,
+        "kv_heads": w.spec.n_kv_heads, "head_dim": w.spec.head_dim, "n_dom": w.spec.n_dom,
+        "n_fac": int(w.n_fac_per_seq.max()), "n_layers": w.spec.n_layers,
+        "parallelism": f"independent sequences per rank x{world}",
+        "algorithmic_bytes_per_step": algorithmic_bytes(w)["total"],
+    }
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -557,7 +562,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same inputs)",
-        "config": {"workload": w.spec.name, "batch": w.spec.batch, "seq_len": int(w.max_len)},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"{per_step_rows} of {rows_total} (sequence, KV head) rows per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -19,7 +19,7 @@ def lite(name):
     spec = preset(name)
     lengths = _draw_lengths(spec)
     return SimpleNamespace(spec=spec, lengths=lengths, roles=torch.from_numpy(_draw_roles(spec)),
-                           n_fac_per_seq=torch.from_numpy(_n_fac(spec, lengths)))
+                           n_fac_per_seq=torch.from_numpy(_n_fac(spec, lengths)), max_len=int(lengths.max()))
 
 
 def test_algorithmic_bytes_of_the_fixed_shape_workloads():
@@ -78,3 +78,12 @@ def test_kernel_bytes_follow_the_path_taken():
     assert bench.kernel_bytes(c, abc, "shared_index_step", "sparse_row_kernel", fused) == abc["total"]
     assert bench.kernel_bytes(c, abc, "shared_index_step", "topk_select_kernel", three) == abc["select"]
     assert bench.kernel_bytes(c, abc, "shared_index_step", "flash_gather_kernel", three) == abc["gather"]
+
+
+def test_both_arms_report_the_same_config():
+    # the reference arm and ours describe the workload with the same keys and values
+    w = lite("clsa_shared_L128k")
+    cfg = bench.workload_config(w, 1)
+    assert cfg["workload"] == "clsa_shared_L128k" and cfg["algorithmic_bytes_per_step"] == 553648128
+    assert cfg["tokens_per_step_per_gpu"] == 2 * 131072 and cfg["n_layers"] == 8
+    assert cfg["parallelism"] == "independent sequences per rank x1"
