@@ -2,12 +2,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-A step is one pass of the whole decode path over one batch: for the default
-Llama-3-8B-shaped layer (batch 4, 32 q / 8 KV heads, d 128, L 32768, 16 of 64
-dominant chunks, N_fac 2048) that is the importance scan, the top-N_fac select
-and focused attention of every KV head (``aoh_sparse_decode``), plus the
-window attention of DENSE / STREAM heads when the workload has any.  The metric
-is KV tokens scanned per second (sum over sequences of L_b per step, all ranks
+A step is one pass of the whole decode path over one batch.  For the default
+workload, the 128K shared-index cross-decoder stack (batch 2, one shared cache of
+131072 tokens x 8 KV heads, d 128; an indexer scores every token with the
+full-dimension q.k, takes one top-2048 per (sequence, KV head), and 8 layers of 32
+q heads attend over that index), that is one ``aoh_shared_index_step`` call.  For
+the sparse workloads it is the importance scan, the top-N_fac select and focused
+attention of every SPARSE KV head (``aoh_sparse_decode``), plus the window
+attention of DENSE / STREAM heads when the workload has any.  The metric is KV
+tokens scanned per second (sum over sequences of L_b per step, all ranks
 together), and the algorithmic HBM bytes per second of the step and of its
 dominant kernel against the measured copy bandwidth.
 
@@ -21,7 +24,12 @@ no collective on the data path); NCCL is used only for the barrier and the
 max-reduction of the timings.
 
 ``--impl reference`` times the float64 CPU oracle on the host cores instead
-(same metric and workload, each step a bounded sample of rows).
+(same metric and workload, each step a bounded sample of rows), once with one
+worker process per core of the process affinity (each limited to one BLAS
+thread) and once on a single thread.
+
+``--gpus N`` outside torchrun re-launches this script under
+``torch.distributed.run`` with N ranks on this node.
 """
 
 from __future__ import annotations
@@ -46,7 +54,8 @@ import torch  # noqa: E402
 from workloads import ROLE_SPARSE, make_workload, preset  # noqa: E402
 
 METRIC = "sparse decode: KV tokens scanned/s/GPU; achieved HBM GB/s vs B200 peak"
-DEFAULT_WORKLOAD = "llama8b_gqa4_L32k"
+DEFAULT_WORKLOAD = "clsa_shared_L128k"
+MAX_POOL = 32  # oracle worker processes at most (each holds one float64 row: up to ~0.3 GB)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -446,6 +455,11 @@ def run_ours(args, rank, world, local_rank):
     dom = max(kt["kernels"], key=lambda e: e["ms"]) if kt["kernels"] else None
     dom_bytes = kernel_bytes(w, ab, dom["call"], dom["kernel"], kt["order"][dom["call"]]) if dom else 0
     dom_ms = dom["ms"] if dom else None
+    one_kernel_step = dom is not None and len(kt["kernels"]) == 1
+    if one_kernel_step:
+        # the step is that one kernel: its graph-replayed time per step is the kernel's time
+        # (the per-launch events add the event records' own overhead around an eager launch)
+        dom_ms = ms_step
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms else None
     step_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     return {
@@ -469,6 +483,8 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "peak_source": peak_kind,
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
+                     "timing": "graph-replayed step (one-kernel step)" if one_kernel_step
+                     else "CUDA events around the kernel inside the call",
                      "traffic": ncu_traffic(w.spec.name, dom["kernel"]) if dom else None},
         "call_ms": kt["calls"],
         "kernel_ms": [{"call": e["call"], "kernel": e["kernel"], "ms": e["ms"],
@@ -483,51 +499,156 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------------------ oracle (CPU) arms
+#
+# The oracle runs on whole (sequence, KV head) rows: the select needs every score of a row.
+# A row task carries that row's bf16 inputs (compact copies), so a worker process needs
+# nothing else; every run keeps BLAS to one thread per process, and the all-cores run uses
+# one spawned worker process per core of this process's affinity (at most MAX_POOL).
 
-def oracle_rows_per_sec(w, max_seconds: float, max_rows: int = 10 ** 9):
-    """Time the float64 oracle on whole (sequence, KV head) rows of the workload, in order."""
+def host_cores() -> dict:
+    """Logical CPUs of the host and of this process's affinity mask."""
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        aff = os.cpu_count() or 1
+    return {"host_cpu_count": os.cpu_count(), "affinity_cores": aff}
+
+
+def row_task(w, b: int, g: int):
+    """The inputs of oracle row (b, g) as compact bf16 tensors, and its token count."""
+    sp = w.spec
+    G = sp.group
+    o0, o1 = int(w.offsets[b]), int(w.offsets[b + 1])
+    keys = w.k[o0:o1, g].clone()
+    vals = w.v[o0:o1, g].clone()
+    if sp.n_layers > 0:
+        return ("shared", w.q[b, g * G:(g + 1) * G].clone(), w.q_layers[:, b, g * G:(g + 1) * G].clone(),
+                keys, vals, sp.topk_shared, w.scale), o1 - o0
+    return ("row", w.q[b, g * G:(g + 1) * G].clone(), keys, vals, int(w.roles[g]), w.scale,
+            None if w.idom is None else w.idom[g].tolist(), int(w.n_fac_per_seq[b]), sp.sink, sp.window), o1 - o0
+
+
+def oracle_row(task) -> float:
+    """Run the oracle on one row task; returns its wall time in seconds (one BLAS thread)."""
     import oracle
     from threadpoolctl import threadpool_limits
 
-    sp = w.spec
-    G = sp.group
-    rows = [(b, g) for b in range(sp.batch) for g in range(sp.n_kv_heads)]
-    done, t0 = 0, time.perf_counter()
-    tokens = 0
     with threadpool_limits(limits=1):
-        while done < max_rows:
-            b, g = rows[done % len(rows)]
-            o0, o1 = int(w.offsets[b]), int(w.offsets[b + 1])
-            keys = w.k[o0:o1, g].double().numpy()
-            vals = w.v[o0:o1, g].double().numpy()
-            if sp.n_layers > 0:
-                qi = w.q[b:b + 1].double().numpy()
-                ql = w.q_layers[:, b:b + 1].double().numpy()
-                kk = np.ascontiguousarray(keys[:, None, :])
-                vv = np.ascontiguousarray(vals[:, None, :])
-                oracle.shared_index_step(qi[:, g * G:(g + 1) * G], ql[:, :, g * G:(g + 1) * G], kk, vv,
-                                         [0, o1 - o0], sp.topk_shared, w.scale)
-            else:
-                oracle.decode_row(w.q[b, g * G:(g + 1) * G].double().numpy(), keys, vals, int(w.roles[g]), w.scale,
-                                  None if w.idom is None else w.idom[g].tolist(), int(w.n_fac_per_seq[b]),
-                                  sp.sink, sp.window)
-            done += 1
-            tokens += o1 - o0
-            if time.perf_counter() - t0 > max_seconds:
-                break
-    dt = time.perf_counter() - t0
-    return done, tokens, dt
+        t0 = time.perf_counter()
+        if task[0] == "shared":
+            _, qi, ql, keys, vals, topk, scale = task
+            kk = np.ascontiguousarray(keys.double().numpy()[:, None, :])
+            vv = np.ascontiguousarray(vals.double().numpy()[:, None, :])
+            oracle.shared_index_step(qi.double().numpy()[None], ql.double().numpy()[:, None], kk, vv,
+                                     [0, kk.shape[0]], topk, scale)
+        else:
+            _, qg, keys, vals, role, scale, idom, n_fac, sink, window = task
+            oracle.decode_row(qg.double().numpy(), keys.double().numpy(), vals.double().numpy(), role, scale, idom,
+                              n_fac, sink, window)
+        return time.perf_counter() - t0
 
 
-def cpu_baseline(w, seconds: float = 15.0) -> dict:
-    done, tokens, dt = oracle_rows_per_sec(w, seconds)
-    rows_total = w.spec.batch * w.spec.n_kv_heads
-    step_tokens = int(w.lengths.sum())
-    # tokens/s: the fraction of a step done, times the tokens a step scans, per second
-    value = (done / rows_total) * step_tokens / dt
-    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} (sequence, KV head) rows ({rows_total} make one step), float64 numpy, "
-                      f"BLAS limited to 1 thread, {dt:.1f} s"}
+def _oracle_repeat(arg) -> float:
+    """Worker body: one row task run `repeat` times; returns the busy time."""
+    task, repeat = arg
+    return sum(oracle_row(task) for _ in range(repeat))
+
+
+def _pool_ready(_):
+    import oracle  # noqa: F401  (the workers' imports happen before any timing)
+    from threadpoolctl import threadpool_limits  # noqa: F401
+
+    return os.getpid()
+
+
+class OraclePool:
+    """Spawned worker processes (never forked: the parent may hold a CUDA context)."""
+
+    def __init__(self, workers: int):
+        import multiprocessing
+        from concurrent.futures import ProcessPoolExecutor
+
+        self.workers = workers
+        self.ex = ProcessPoolExecutor(max_workers=workers, mp_context=multiprocessing.get_context("spawn"))
+        list(self.ex.map(_pool_ready, range(workers)))
+
+    def run(self, tasks, repeat: int) -> float:
+        """Wall time of every worker running its task `repeat` times (one task per worker)."""
+        t0 = time.perf_counter()
+        list(self.ex.map(_oracle_repeat, [(t, repeat) for t in tasks]))
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.ex.shutdown(wait=True)
+
+
+def all_rows(w):
+    return [(b, g) for b in range(w.spec.batch) for g in range(w.spec.n_kv_heads)]
+
+
+def oracle_single_thread(w, seconds: float) -> dict:
+    """Rows of the workload in order, one thread, until `seconds` have passed (at least one row)."""
+    rows = all_rows(w)
+    done, tokens, busy = 0, 0, 0.0
+    while busy < seconds:
+        b, g = rows[done % len(rows)]
+        task, n_tok = row_task(w, b, g)
+        busy += oracle_row(task)
+        done += 1
+        tokens += n_tok
+    return {"value": tokens / busy, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (sequence, KV head) rows ({len(rows)} make one step), float64 numpy, "
+                      f"one process, BLAS limited to 1 thread, {busy:.1f} s",
+            "s_per_row": busy / done}
+
+
+def pool_size(w) -> int:
+    return max(1, min(host_cores()["affinity_cores"], MAX_POOL))
+
+
+def repeats_for(s_per_row: float, target_s: float = 1.0) -> int:
+    """Times a worker repeats its row so that one batch is about target_s of work per worker."""
+    return max(1, int(round(target_s / max(s_per_row, 1e-6))))
+
+
+class PoolSteps:
+    """Batches of the pool: worker j runs row (i * workers + j) mod rows, `repeat` times."""
+
+    def __init__(self, w, pool: OraclePool, repeat: int):
+        self.w, self.pool, self.repeat = w, pool, repeat
+        self.rows = all_rows(w)
+        self.i = 0
+
+    def batch(self):
+        tasks = [row_task(self.w, *self.rows[(self.i * self.pool.workers + j) % len(self.rows)])
+                 for j in range(self.pool.workers)]
+        self.i += 1
+        wall = self.pool.run([t for t, _ in tasks], self.repeat)
+        return wall, sum(n for _, n in tasks) * self.repeat
+
+    def describe(self, rows_done: int, wall: float) -> str:
+        return (f"{rows_done} (sequence, KV head) row runs ({len(self.rows)} rows make one step) in batches of "
+                f"{self.pool.workers} rows x {self.repeat} repeats, float64 numpy, {self.pool.workers} spawned "
+                f"worker processes with 1 BLAS thread each, {wall:.1f} s of wall time")
+
+
+def cpu_baseline(w, seconds: float = 10.0) -> dict:
+    """The oracle on all cores of this process's affinity and on one thread (both reported)."""
+    single = oracle_single_thread(w, seconds)
+    pool = OraclePool(pool_size(w))
+    try:
+        ps = PoolSteps(w, pool, repeats_for(single["s_per_row"]))
+        wall, tokens, runs = 0.0, 0, 0
+        while wall < seconds:
+            dt, n = ps.batch()
+            wall += dt
+            tokens += n
+            runs += pool.workers * ps.repeat
+        multi = {"value": tokens / wall, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
+                 "sample": ps.describe(runs, wall)}
+    finally:
+        pool.close()
+    return dict(multi, **host_cores(), single_thread=single)
 
 
 def workload_config(w, world: int) -> dict:
@@ -543,33 +664,53 @@ def workload_config(w, world: int) -> dict:
 
 
 def run_reference(args, rank, world):
+    """The oracle on the host cores: each step is one batch of rows on the worker pool."""
     if rank != 0:
         return None
     w = make_workload(preset(args.workload))
-    rows_total = w.spec.batch * w.spec.n_kv_heads
-    # size one step's sample so that warm-up + timed steps end within about two minutes
-    _, _, dt1 = oracle_rows_per_sec(w, 1e9, max_rows=1)
-    per_step_rows = max(1, min(rows_total, int(100.0 / max(1, args.steps + args.warmup) / max(dt1, 1e-3))))
-    for _ in range(args.warmup):
-        oracle_rows_per_sec(w, 1e9, max_rows=per_step_rows)
-    t = 0.0
-    for _ in range(args.steps):
-        _, _, dt = oracle_rows_per_sec(w, 1e9, max_rows=per_step_rows)
-        t += dt
+    single = oracle_single_thread(w, 5.0)
+    pool = OraclePool(pool_size(w))
+    try:
+        ps = PoolSteps(w, pool, repeats_for(single["s_per_row"], 2.0))
+        for _ in range(args.warmup):
+            ps.batch()
+        t, tokens = 0.0, 0
+        for _ in range(args.steps):
+            dt, n = ps.batch()
+            t += dt
+            tokens += n
+    finally:
+        pool.close()
     ms_step = t / args.steps * 1e3
-    value = (per_step_rows / rows_total) * int(w.lengths.sum()) / (ms_step * 1e-3)
+    value = tokens / t
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same inputs)",
         "config": workload_config(w, world),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step_rows} of {rows_total} (sequence, KV head) rows per step"},
+        "cpu_baseline": dict({"value": value, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
+                              "sample": ps.describe(args.steps * pool.workers * ps.repeat, t)},
+                             **host_cores(), single_thread=single),
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
 # ------------------------------------------------------------------------------ main
+
+def torchrun_command(n: int, port: int, argv) -> list:
+    """The command that runs this script with the same arguments as n ranks on this node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def relaunch_under_torchrun(n: int) -> int:
+    import socket
+
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    return subprocess.call(torchrun_command(n, port, sys.argv[1:]))
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -585,9 +726,14 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: run this same command under torchrun with N ranks
+        sys.exit(relaunch_under_torchrun(args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and rank == 0:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; measuring {world} ranks", file=sys.stderr)
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)

@@ -87,3 +87,31 @@ def test_both_arms_report_the_same_config():
     assert cfg["workload"] == "clsa_shared_L128k" and cfg["algorithmic_bytes_per_step"] == 553648128
     assert cfg["tokens_per_step_per_gpu"] == 2 * 131072 and cfg["n_layers"] == 8
     assert cfg["parallelism"] == "independent sequences per rank x1"
+
+
+def test_gpus_flag_relaunches_under_torchrun():
+    cmd = bench.torchrun_command(4, 29555, ["--gpus", "4", "--steps", "7"])
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd and "--master-port=29555" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "7"] and cmd[-5].endswith("bench.py")
+
+
+def test_oracle_pool_sizing_and_core_report():
+    cores = bench.host_cores()
+    assert cores["affinity_cores"] >= 1 and cores["host_cpu_count"] >= cores["affinity_cores"]
+    assert 1 <= bench.pool_size(None) <= min(bench.MAX_POOL, cores["affinity_cores"])
+    assert bench.repeats_for(5.0) == 1          # a long row runs once per batch
+    assert bench.repeats_for(0.01, 1.0) == 100  # short rows repeat to about a second of work
+    assert bench.repeats_for(0.0) >= 1
+
+
+def test_row_tasks_carry_compact_copies():
+    from workloads import make_workload
+
+    w = make_workload(preset("tiny_mixed_d64_L512"))
+    task, n = bench.row_task(w, 0, 3)
+    assert n == 512 and task[0] == "row" and task[4] == int(w.roles[3])
+    keys = task[2]
+    assert keys.is_contiguous() and keys.shape == (512, 64) and keys.untyped_storage().nbytes() == 512 * 64 * 2
+    assert bench.oracle_row(task) > 0
