@@ -113,7 +113,7 @@ int32_t aoh_last_cuda_error(void);
 /* Kernels the library launches, one counter each (see aoh_launch_counts). */
 typedef enum {
   AOH_KERNEL_TIP_SCORE = 0,     /* stand-alone importance scan                       */
-  AOH_KERNEL_TOPK_SELECT = 1,   /* stand-alone cluster select (rows beyond the row kernel) */
+  AOH_KERNEL_TOPK_SELECT = 1,   /* stand-alone select, one CTA per row (many rows)   */
   AOH_KERNEL_SPARSE_ROW = 2,    /* fused row kernel, or its select-only form         */
   AOH_KERNEL_FLASH_GATHER = 3,  /* split-K gather / window attention                 */
   AOH_KERNEL_PACK_DOMINANT = 4, /* dominant-column packing of K                      */
@@ -266,9 +266,15 @@ size_t aoh_stream_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_head
  * allocates nothing.  Arguments and results are those of aoh_stream_decode.
  *   - Returns AOH_ERR_WORKSPACE, without launching, when the step needs more
  *     than 16 MiB of scratch (aoh_stream_decode_workspace_size gives the need).
- *   - The first call on a device sets the array up (looks up its address with
- *     that device current, zeroes it and synchronises the device), so make that
- *     first call before any stream capture.
+ *   - Every call looks the array's address up with the current device (a host
+ *     query).  The first call on a device sets the array up: it zeroes it and
+ *     synchronises the device, so make that first call before any stream
+ *     capture.  A cudaDeviceReset destroys the array with its context; the next
+ *     call finds the new address and sets the array up again (so, again, not
+ *     during a capture).
+ *   - Arguments are validated before the array is touched; a refused call
+ *     leaves it as it was.  A kernel that was aborted (a lost context) can
+ *     leave its split counters set; only a reset clears them.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents; calls that can overlap on the GPU (different streams without
  *     ordering) race on it.  Serialise them on one stream.

@@ -4,11 +4,14 @@
 
 The library is one translation unit (csrc/aoh_api.cu includes the kernels) linked
 against the shared CUDA runtime, so that it shares the runtime instance (current
-device, streams) of the PyTorch process that loads it.
+device, streams) of the PyTorch process that loads it.  A rebuild happens whenever
+the sha256 of the sources and flags differs from the one recorded beside the
+library (libaoh.so.srchash), whatever the files' times.
 """
 
 from __future__ import annotations
 
+import hashlib
 import os
 import shutil
 import subprocess
@@ -18,6 +21,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "aoh_api.cu")
 OUT = os.path.join(HERE, "libaoh.so")
+HASH = OUT + ".srchash"  # source hash the library was built from
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -30,22 +34,39 @@ def _nvcc() -> str:
 
 def _sources():
     d = os.path.join(HERE, "csrc")
-    return [os.path.join(d, f) for f in os.listdir(d)] + [os.path.join(ROOT, "include", "aoh.h")]
+    return sorted(os.path.join(d, f) for f in os.listdir(d)) + [os.path.join(ROOT, "include", "aoh.h")]
+
+
+def _command(out: str) -> list:
+    return [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+            "-cudart", "shared", "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"),
+            "-o", out, SRC]
+
+
+def source_hash() -> str:
+    """sha256 of every source file (name and bytes) and of the compile flags."""
+    h = hashlib.sha256()
+    for path in _sources():
+        h.update(os.path.basename(path).encode() + b"\0")
+        with open(path, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(_command("libaoh.so")[1:]).encode())
+    return h.hexdigest()
 
 
 def up_to_date() -> bool:
-    if not os.path.exists(OUT):
+    """The library exists and was built from exactly the current sources and flags."""
+    if not (os.path.exists(OUT) and os.path.exists(HASH)):
         return False
-    t = os.path.getmtime(OUT)
-    return all(os.path.getmtime(s) <= t for s in _sources())
+    with open(HASH) as f:
+        return f.read().strip() == source_hash()
 
 
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if not force and up_to_date():
         return OUT
-    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-cudart", "shared", "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"),
-           "-o", OUT + ".tmp", SRC]
+    digest = source_hash()
+    cmd = _command(OUT + ".tmp")
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -54,6 +75,8 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if ptxas_verbose:
         sys.stderr.write(res.stdout + res.stderr)
     os.replace(OUT + ".tmp", OUT)
+    with open(HASH, "w") as f:
+        f.write(digest + "\n")
     return OUT
 
 

@@ -21,7 +21,6 @@ using namespace aoh;
 
 namespace {
 
-constexpr int kSmCount = 148;        // B200
 constexpr int kMaxQRows = 32;        // query rows per KV head in one gather kernel (4 n-tiles)
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -53,6 +52,26 @@ aoh_status check_heads(const aoh_kv_cache* kv, int32_t n_q_heads) {
 }
 
 thread_local int t_last_cuda_error = 0;
+
+// Streaming multiprocessors of the current device (148 on a B200), read once per device.
+// Grids of the persistent and split-K kernels are sized from it.
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = 0;
+  }
+  std::atomic<int>& slot = cached[dev & 63];
+  int n = slot.load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 148;
+  }
+  slot.store(n, std::memory_order_relaxed);
+  return n;
+}
 
 
 aoh_status cuda_status(cudaError_t e) {
@@ -130,7 +149,7 @@ struct FdGeom {
 FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
   FdGeom g{};
   // about two CTAs per SM; at least two pipeline stages per CTA; at most kFdMaxSplits splits a row
-  const int64_t target = int64_t(kSmCount) * 2;
+  const int64_t target = int64_t(sm_count()) * 2;
   int64_t chunk = ceil_div(std::max<int64_t>(work_tokens, 1), target);
   chunk = std::min<int64_t>(std::max<int64_t>(chunk, 2 * kFdTS), 1024);  // long CTAs are latency bound
   chunk = std::max<int64_t>(chunk, ceil_div(std::max<int64_t>(n_max, 1), kFdMaxSplits));
@@ -264,7 +283,7 @@ aoh_status launch_tip_t(TipParams& tp, cudaStream_t st) {
       per_sm = 1;
     }
   }
-  const int64_t resident = int64_t(kSmCount) * per_sm;
+  const int64_t resident = int64_t(sm_count()) * per_sm;
   tp.per_cta = std::max<int64_t>(256, ceil_div(tp.total, resident));
   const int64_t grid = ceil_div(tp.total, tp.per_cta);
   before_launch(st);
@@ -368,22 +387,6 @@ struct FusedPlan {
   size_t keys_bytes, ring_bytes, smem;
 };
 
-#ifdef AOH_PHASE_TIMERS
-int g_force_cluster = 0;  // diagnostic build: force the fused kernel's cluster size ...
-int g_force_ring = 0;     // ... cap its ring (bytes) ...
-int g_force_one_per_sm = 0;  // ... or give one CTA per SM the whole budget
-int g_force_three = 0;       // ... or take the three-kernel form
-int g_select_rows = 0;       // ... with the row kernel's cluster select
-#endif
-
-bool allow_fused() {
-#ifdef AOH_PHASE_TIMERS
-  return !g_force_three;
-#else
-  return true;
-#endif
-}
-
 FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true) {
   FusedPlan f{};
   const int64_t L = std::max(kv->max_len, 1);
@@ -398,14 +401,8 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   // keys; a CTA whose candidates do not fit counts its later digits over all its keys)
   const size_t ring_min = need_ring ? kRingMin : (size_t)ceil_div(f.keys_bytes / 4, 1024) * 1024;
   if (f.keys_bytes + ring_min > budget) budget = kOnePerSm - 1024;
-#ifdef AOH_PHASE_TIMERS
-  if (g_force_one_per_sm) budget = kOnePerSm - 1024;
-#endif
   if (f.keys_bytes + ring_min > budget) return f;
   f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kRingStep * kRingStep) : ring_min;
-#ifdef AOH_PHASE_TIMERS
-  if (need_ring && g_force_ring) f.ring_bytes = std::min(f.ring_bytes, (size_t)g_force_ring);
-#endif
   f.smem = f.keys_bytes + f.ring_bytes + 1024;
   f.ok = true;
   return f;
@@ -447,9 +444,6 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   for (int i = 0; i < 3; ++i) {
     const FusedPlan f = fused_candidate(kv, cls[i], need_ring);
     if (!f.ok) continue;
-#ifdef AOH_PHASE_TIMERS
-    if (g_force_cluster && f.CL != g_force_cluster) continue;
-#endif
     const int maxc = max_active_clusters(kern, f.CL, f.smem);
     if (maxc <= 0) continue;
     const int64_t waves = ceil_div(n_rows, maxc);
@@ -533,11 +527,7 @@ aoh_status select_stage(const float* scores, const aoh_kv_cache* kv, int32_t n_f
   // Rows enough to fill the SMs: one CTA per row.  Fewer, longer rows: the row kernel's
   // cluster select, which spreads each row over a cluster's shared memory.
   const int64_t rows = int64_t(kv->batch) * n_listed;
-  bool rows_kernel = rows < kSmCount && select_rows_feasible(kv);
-#ifdef AOH_PHASE_TIMERS
-  if (g_select_rows == 1) rows_kernel = select_rows_feasible(kv);
-  if (g_select_rows == 2) rows_kernel = false;
-#endif
+  const bool rows_kernel = rows < sm_count() && select_rows_feasible(kv);
   if (rows_kernel) return launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
   return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
 }
@@ -690,7 +680,7 @@ aoh_status aoh_pack_dominant(const aoh_kv_cache* kv, const int32_t* idom, int32_
   pp.n_dom = n_dom;
   pp.cols = k_dom_cols;
   const int64_t total = int64_t(pp.Hkv) * pp.T * pp.cols;
-  const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), int64_t(kSmCount) * 16);
+  const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), int64_t(sm_count()) * 16);
   before_launch(as_stream(stream));
   pack_dominant_kernel<<<blocks, 256, 0, as_stream(stream)>>>(pp);
   return count_launch(AOH_KERNEL_PACK_DOMINANT, as_stream(stream));
@@ -761,7 +751,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + off_idx);
   int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + off_count);
 
-  if (allow_fused() && fused_feasible(kv, G)) {
+  if (fused_feasible(kv, G)) {
     RowParams rp{};
     rp.q_score = static_cast<const uint16_t*>(q);
     rp.q_attn = static_cast<const uint16_t*>(q);
@@ -953,7 +943,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const FdGeom geo = shared_geom(kv, n_layers, n_q_heads, topk);
   float* scores = reinterpret_cast<float*>(ws + fd_bytes(geo));
-  if (allow_fused() && fused_feasible(kv, n_layers * G)) {
+  if (fused_feasible(kv, n_layers * G)) {
     RowParams rp{};
     rp.q_score = static_cast<const uint16_t*>(q_index);
     rp.q_attn = static_cast<const uint16_t*>(q_layers);
@@ -1010,33 +1000,6 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st, true);
 }
 
-#ifdef AOH_PHASE_TIMERS
-// Diagnostic build only: copy the phase stamps of the fused kernel to the host.
-int32_t aoh_debug_phase_ns(long long* host, int32_t n_ctas) {
-  if (n_ctas > kPhaseCtas) n_ctas = kPhaseCtas;
-  return cudaMemcpyFromSymbol(host, g_phase_ns, sizeof(long long) * kPhaseSlots * n_ctas) == cudaSuccess ? 0 : 5;
-}
-void aoh_debug_force_cluster(int32_t cl) { g_force_cluster = cl; }
-void aoh_debug_force_three(int32_t on) { g_force_three = on; }
-void aoh_debug_select_rows(int32_t on) { g_select_rows = on; }
-// per-CTA record of the select kernel's last launch: [b, g, L, nf, n, cap, T, KT, need_eq, eq_total]
-int32_t aoh_debug_select_info(int32_t* host, int32_t rows) {
-  cudaDeviceSynchronize();
-  return cudaMemcpyFromSymbol(host, g_sel_dbg, size_t(std::min(rows, 4096)) * 10 * sizeof(int)) == cudaSuccess;
-}
-void aoh_debug_force_ring(int32_t bytes, int32_t one_per_sm) {
-  g_force_ring = bytes;
-  g_force_one_per_sm = one_per_sm;
-}
-// cudaOccupancyMaxActiveClusters of the fused kernel (d 128, one n-tile).
-int32_t aoh_debug_max_clusters(int32_t cl, int32_t smem) {
-  auto kern = sparse_row_kernel<128, 1>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOnePerSm);
-  cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  return max_active_clusters(kern, cl, (size_t)smem);
-}
-#endif
-
 }  // extern "C"
 
 // ===================================================================== no-allocation variant
@@ -1047,26 +1010,28 @@ static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBy
 
 namespace {
 std::mutex g_static_mu;
-void* g_static_addr[256];  // device address of the array, per device ordinal (host-side)
+void* g_static_addr[256];  // device address of the array last set up, per device ordinal (host-side)
 
-// The array's device address on the current device.  First use on a device: look the
-// address up with that device current and zero the array (the split counters at its head
-// must start at zero; every later call leaves them at zero).  This set-up synchronises
-// the device, so the first call on a device must not happen during a stream capture.
+// The array's device address on the current device, looked up on every call (a host-side
+// query, no synchronisation), so that a context created after cudaDeviceReset, which loads
+// the module again, is never handed a stale address.  When the address is new for this
+// device the array is zeroed (the split counters at its head must start at zero; every
+// later call leaves them at zero) and the device synchronised: the first call on a device,
+// and the first after a reset, must therefore not happen during a stream capture.
 aoh_status static_scratch_address(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return AOH_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaGetLastError());
   if (dev < 0 || dev >= 256) return AOH_ERR_UNSUPPORTED;
+  void* ptr = nullptr;
+  aoh_status s = cuda_status(cudaGetSymbolAddress(&ptr, g_static_scratch));
+  if (s != AOH_OK) return s;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_addr[dev]) {
-    void* ptr = nullptr;
-    aoh_status s = cuda_status(cudaGetSymbolAddress(&ptr, g_static_scratch));
-    if (s != AOH_OK) return s;
+  if (g_static_addr[dev] != ptr) {
     if ((s = cuda_status(cudaMemset(ptr, 0, kStaticScratchBytes))) != AOH_OK) return s;
     if ((s = cuda_status(cudaDeviceSynchronize())) != AOH_OK) return s;
     g_static_addr[dev] = ptr;
   }
-  *out = g_static_addr[dev];
+  *out = ptr;
   return AOH_OK;
 }
 }  // namespace
@@ -1074,6 +1039,7 @@ aoh_status static_scratch_address(void** out) {
 extern "C" aoh_status aoh_stream_decode_noalloc(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
                                                 const uint8_t* roles, int32_t sink, int32_t window, float scale,
                                                 float* out, void* stream) {
+  // every argument check of aoh_stream_decode runs before the scratch is touched
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
   if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
@@ -1082,6 +1048,8 @@ extern "C" aoh_status aoh_stream_decode_noalloc(const void* q, int32_t n_q_heads
   if (n_q_heads / kv->n_kv_heads > kMaxQRows) return AOH_ERR_UNSUPPORTED;
   if (sink < 0 || window < 0 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
   if (kv->batch == 0) return AOH_OK;
+  if (!q || !out) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(q)) return AOH_ERR_ALIGNMENT;
   if (fd_bytes(stream_geom(kv, n_q_heads, roles, sink, window)) > kStaticScratchBytes) return AOH_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((s = static_scratch_address(&scratch)) != AOH_OK) return s;

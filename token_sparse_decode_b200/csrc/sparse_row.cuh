@@ -75,35 +75,15 @@ struct RowParams {
   uint8_t heads[kMaxHeads];
 };
 
-// Attention tiles: gathered K / V rows land whole (one 1-D bulk copy each) at a row
-// pitch of 2*D + 16 bytes, so the 8 rows an ldmatrix reads sit in 8 different
-// 16-byte bank groups.
+// Attention tiles: gathered K / V rows are copied as 16-byte cp.async segments into rows
+// of pitch 2*D + 16 bytes, so the 8 rows an ldmatrix reads sit in 8 different 16-byte
+// bank groups.
 template <int D>
 struct AttTile {
   static constexpr int kPitch = 2 * D + 16;
   static constexpr int kTile = kSrTS * kPitch;  // one of K or V per stage
   static constexpr int kStage = 2 * kTile;
 };
-
-#ifdef AOH_PHASE_TIMERS
-// Diagnostic build only: global-timer stamps at the phase boundaries of every CTA.
-constexpr int kPhaseSlots = 16;
-constexpr int kPhaseCtas = 8192;
-__device__ long long g_phase_ns[kPhaseCtas][kPhaseSlots];
-__device__ __forceinline__ void phase_stamp(int slot) {
-  if (threadIdx.x == 0) {
-    const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-    if (cta < kPhaseCtas) {
-      long long t;
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      g_phase_ns[cta][slot] = t;
-    }
-  }
-}
-#define AOH_PHASE(i) phase_stamp(i)
-#else
-#define AOH_PHASE(i)
-#endif
 
 template <int D, int NT>
 __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_constant__ RowParams p) {
@@ -124,7 +104,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   __shared__ int s_bin, s_above, s_eq_before, s_sel_before, s_up;
   __shared__ int s_gt[kSrMaxCluster], s_eq[kSrMaxCluster], s_eq_all;
 
-  AOH_PHASE(0);
   cgs::cluster_group cluster = cgs::this_cluster();
   const int CL = (int)cluster.num_blocks();
   const int rk = (int)cluster.block_rank();
@@ -274,7 +253,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       __syncthreads();
     }
     }
-    AOH_PHASE(1);
     // =============================================================== 2. select
     // 4-digit MSB radix select over the cluster.  Digits 0-2: every CTA adds its non-zero
     // counts into each peer's total (remote atomics), one cluster barrier, then the digit is
@@ -415,7 +393,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     }
     const uint32_t KT = prefix;
     const int need_eq = krem;
-    AOH_PHASE(2);
 
     // ---- ordered compaction: positions in ascending order, lower position first among equals
     if (tid == 0) {
@@ -496,7 +473,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     return;
   }
 
-  AOH_PHASE(3);
   // =============================================================== 3. attend
   // warp = (token group, n-tile, part of the head dimension)
   const int dp = warp % DP, nt = (warp / DP) % NT, tg = warp / (DP * NT);
@@ -622,7 +598,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   }
   __syncthreads();  // stage buffers are free
 
-  AOH_PHASE(4);
   // ---- merge the warps of this CTA: red_ml [8][8][2], red_acc [8][8][D/DP]; CTA state after
   constexpr int DW = D / DP;                   // dims per part
   float* red_ml = reinterpret_cast<float*>(stage_mem);
@@ -670,9 +645,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   }
 
   // =============================================================== 4. combine over the cluster
-  AOH_PHASE(5);
   cluster.sync();
-  AOH_PHASE(6);
   float* wsm = red_ml;  // [CL][NQP] weights, then [NQP] totals (local scratch; red_* are dead)
   float* Lsm = wsm + 16 * NQP;
   if (tid < NQP) {
@@ -717,7 +690,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     }
   }
   cluster.sync();  // peers may read this CTA's state until every CTA is done
-  AOH_PHASE(7);
 }
 
 }  // namespace aoh

@@ -6,8 +6,9 @@
 // (written by the scan kernel just before, so resident in L2) are read as
 // order-preserving uint32 keys.  An MSB-first radix select (4 digits of 8 bits)
 // finds the n-th largest key K_T:
-//   digit 0: a coalesced pass over the row builds its 256-bin histogram (warp-
-//            aggregated shared-memory counts);
+//   digit 0: a coalesced pass over the row builds per-warp 256-bin histograms
+//            (plain shared-memory atomics), which also give every warp its offset
+//            for the compaction below;
 //   then the keys sharing the chosen first digit are compacted into shared
 //            memory by a second pass (when they fit; otherwise the later digits
 //            re-read the row), and digits 1-3 are counted over those candidates.
@@ -37,14 +38,6 @@ struct SelectParams {
   uint8_t heads[kMaxHeads];       // KV head of blockIdx.x
 };
 
-#ifdef AOH_PHASE_TIMERS
-__device__ int g_sel_dbg[4096][10];  // diagnostic build: each CTA's view of its row
-#define AOH_SEL_DBG(i, v) \
-  if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096) g_sel_dbg[blockIdx.y * gridDim.x + blockIdx.x][i] = (int)(v)
-#else
-#define AOH_SEL_DBG(i, v)
-#endif
-
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectParams p) {
   extern __shared__ __align__(16) uint32_t cand[];  // kSelCandCap keys
   __shared__ int hist[256];
@@ -65,13 +58,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
   const int n = max(0, min(nf, L));
   int32_t* out = p.idx + ((int64_t)b * p.Hkv + g) * p.cap;
   const float* row = p.scores + (int64_t)g * p.T + off;
-  AOH_SEL_DBG(0, b);
-  AOH_SEL_DBG(1, g);
-  AOH_SEL_DBG(2, L);
-  AOH_SEL_DBG(3, nf);
-  AOH_SEL_DBG(4, n);
-  AOH_SEL_DBG(5, p.cap);
-  AOH_SEL_DBG(6, p.T);
   for (int j = n + tid; j < p.cap; j += kSelThreads) out[j] = -1;
   if (tid == 0) p.count[(int64_t)b * p.Hkv + g] = n;
   if (n == 0) return;  // before any barrier: uniform over the CTA
@@ -168,9 +154,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
   }
   const uint32_t KT = prefix;
   const int need_eq = krem;    // keys equal to K_T that are taken, lowest positions first
-  AOH_SEL_DBG(7, KT);
-  AOH_SEL_DBG(8, need_eq);
-  AOH_SEL_DBG(9, eq_total);
 
   // ---- ordered compaction: tiles of 4 * kSelThreads positions, 4 consecutive per thread
   int sel_base = 0, eq_base = 0;
