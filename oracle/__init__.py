@@ -17,5 +17,6 @@ from .reference import (  # noqa: F401
     decode_row,
     decode_step,
     shared_index_step,
+    tie_band,
     tie_band_check,
 )

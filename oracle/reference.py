@@ -121,10 +121,27 @@ def select_top(scores: np.ndarray, n: int) -> np.ndarray:
     return np.sort(order[:n]).astype(np.int64)
 
 
-def tie_band_check(gpu_sel: np.ndarray, ref_scores: np.ndarray, n: int, rel: float = 1e-4) -> Tuple[bool, str]:
+def tie_band(ref_scores: np.ndarray, n: int, rel: float = 1e-4, floor: float = 0.0) -> float:
+    """Half-width beta of the score band around the n-th largest score s_n.
+
+    beta = max(rel * |s_n|, floor).  The relative part is the band the selection may
+    disagree within; `floor` is an absolute width a caller derives from the rounding
+    bound of the scores it compares (an fp32 score cannot be closer than that to the
+    exact one, so near s_n = 0 the relative band alone would demand the impossible).
+    """
+    s = np.asarray(ref_scores, dtype=np.float64)
+    n = min(int(n), s.shape[0])
+    if n <= 0:
+        return float(floor)
+    s_n = np.sort(s)[::-1][n - 1]
+    return max(rel * abs(float(s_n)), float(floor))
+
+
+def tie_band_check(gpu_sel: np.ndarray, ref_scores: np.ndarray, n: int, rel: float = 1e-4,
+                   floor: float = 0.0) -> Tuple[bool, str]:
     """Is ``gpu_sel`` a valid top-n of ``ref_scores`` up to the score band around the n-th score?
 
-    With s_n the n-th largest oracle score and beta = rel * max(|s_n|, mean|s|):
+    With s_n the n-th largest oracle score and beta = tie_band(ref_scores, n, rel, floor):
     every token with s > s_n + beta must be selected, none with s < s_n - beta,
     and exactly n tokens must be selected (each at most once).
     """
@@ -143,7 +160,7 @@ def tie_band_check(gpu_sel: np.ndarray, ref_scores: np.ndarray, n: int, rel: flo
     if n == L:
         return True, ""
     s_n = np.sort(s)[::-1][n - 1]
-    beta = rel * max(abs(s_n), float(np.mean(np.abs(s))))
+    beta = tie_band(s, n, rel, floor)
     chosen = np.zeros(L, dtype=bool)
     chosen[sel] = True
     must = s > s_n + beta

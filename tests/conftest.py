@@ -23,3 +23,15 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """How the GPU parity tests used the top-k tie band (rows checked, swaps, widening)."""
+    helpers = sys.modules.get("gpu_helpers")
+    if helpers is None or not helpers.BAND_STATS["rows"]:
+        return
+    st = helpers.BAND_STATS
+    terminalreporter.write_line(
+        f"tie band: {st['rows']} selections checked, {st['floor_binding']} where the fp32 floor exceeded "
+        f"1e-4 |s_n|, {st['swapped']} (row, layer) outputs compared with a set that differs inside the band, "
+        f"largest tolerance widening {st['max_widening']:.3g}")

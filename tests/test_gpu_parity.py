@@ -11,8 +11,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import (OUT_ATOL, SCORE_REL, Dev, check_device, compare_sparse_row, compare_window_row, f64,
-                         launches_of, row_inputs, run_shared, run_sparse, score_bound, band_swap_bound,
+from gpu_helpers import (OUT_ATOL, SCORE_REL, Dev, check_device, compare_shared_row, compare_sparse_row,
+                         compare_window_row, f64, launches_of, row_inputs, run_shared, run_sparse, score_bound,
                          three_kernel_form)
 from token_sparse_decode_b200 import binding as B
 from workloads import ROLE_DENSE, ROLE_SPARSE, ROLE_STREAM, WorkloadSpec, make_workload
@@ -269,18 +269,10 @@ def test_shared_index_decode_matches_oracle(n_layers, hq, hkv, fused):
     ref = oracle.shared_index_step(f64(w.q), f64(w.q_layers), f64(w.k), f64(w.v), w.offsets.tolist(), 700,
                                    w.scale)
     for (b, g), r in ref.items():
-        n = cnt_h[b, g]
-        sel = idx_h[b, g, :n]
-        ok, msg = oracle.tie_band_check(sel, r["scores"], min(700, int(w.lengths[b])))
-        assert ok, msg
-        tol = OUT_ATOL
-        if not np.array_equal(sel, r["sel"]):
-            qg, keys, values = row_inputs(w, b, g)
-            for l in range(n_layers):
-                tol = max(tol, OUT_ATOL + band_swap_bound(f64(w.q_layers[l, b, g * G:(g + 1) * G]), keys, values,
-                                                          r["scores"], n, w.scale))
-        err = np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max()
-        assert err <= tol, (b, g, err)
+        sel = idx_h[b, g, :cnt_h[b, g]]
+        compare_shared_row(w, b, g, sel, out_h[:, b, g * G:(g + 1) * G], 700)
+        if np.array_equal(sel, r["sel"]):  # the stack's own oracle on the same index
+            assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= OUT_ATOL
 
 
 def test_shared_index_reports_out_of_range_positions():
@@ -391,12 +383,6 @@ def test_shared_index_step_many_rows_runs_three_stages():
                                    rows=rows)
     for (b, g), r in ref.items():
         sel = idx_h[b, g, :cnt_h[b, g]]
-        ok, msg = oracle.tie_band_check(sel, r["scores"], min(300, int(w.lengths[b])))
-        assert ok, msg
-        tol = OUT_ATOL
-        if not np.array_equal(sel, r["sel"]):
-            qg, keys, values = row_inputs(w, b, g)
-            for l in range(2):
-                tol = max(tol, OUT_ATOL + band_swap_bound(f64(w.q_layers[l, b, g * G:(g + 1) * G]), keys, values,
-                                                          r["scores"], len(sel), w.scale))
-        assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= tol
+        compare_shared_row(w, b, g, sel, out_h[:, b, g * G:(g + 1) * G], 300)
+        if np.array_equal(sel, r["sel"]):
+            assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= OUT_ATOL

@@ -191,6 +191,22 @@ def test_tie_band_check_accepts_and_rejects():
     assert not oracle.tie_band_check(np.array([0, 0]), s, 2)[0]   # duplicate
 
 
+def test_tie_band_is_relative_to_the_nth_score_with_a_floor():
+    # n = 3, s_n = 5: beta = 1e-4 * 5 = 5e-4 (the far-off scores do not enter it)
+    s = np.array([1000.0, 10.0, 5.0, 4.9996, -1000.0])
+    assert oracle.tie_band(s, 3) == pytest.approx(5e-4)
+    assert oracle.tie_band_check(np.array([0, 1, 2]), s, 3)[0]
+    assert oracle.tie_band_check(np.array([0, 1, 3]), s, 3)[0]       # 4.9996 is inside the band
+    s2 = np.array([1000.0, 10.0, 5.0, 4.9994, -1000.0])
+    assert not oracle.tie_band_check(np.array([0, 1, 3]), s2, 3)[0]  # 4.9994 < 5 - 5e-4: below it
+    # s_n = 0: the relative band is empty, only the caller's rounding floor remains
+    z = np.array([3.0, 1e-9, 0.0, -1e-9, -2.0])
+    assert oracle.tie_band(z, 3) == 0.0
+    assert not oracle.tie_band_check(np.array([0, 1, 3]), z, 3)[0]
+    assert oracle.tie_band_check(np.array([0, 1, 3]), z, 3, floor=1e-8)[0]
+    assert oracle.tie_band(z, 3, floor=1e-8) == 1e-8
+
+
 # ---------------------------------------------------------------------------- attention
 
 def test_attend_hand_example(hand):
