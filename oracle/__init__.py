@@ -18,5 +18,11 @@ from .reference import (  # noqa: F401
     decode_step,
     shared_index_step,
     tie_band,
+    ring_slot,
+    ring_contents,
+    to_bf16_bits,
+    bf16_bits_to_f64,
+    append_token_rows,
+    pack_dominant_row,
     tie_band_check,
 )

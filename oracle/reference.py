@@ -211,6 +211,74 @@ def dense_positions(L: int) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# cache maintenance: appending the decoded token (AoH §4: retrieval heads keep the whole
+# cache, streaming heads keep only a fixed sink and a recent window; FASA §2.C: the
+# dominant part of K is kept apart)
+# --------------------------------------------------------------------------------------
+
+def ring_slot(p: int, sink: int, window: int) -> int:
+    """Slot of position p in a streaming head's cache of sink + window slots.
+
+    Positions below the sink keep their own slot; later positions take the window
+    slots in turn, each overwriting the position `window` places before it.
+    Returns -1 when the head keeps no window (window = 0) and p >= sink.
+    """
+    if p < sink:
+        return p
+    if window == 0:
+        return -1
+    return sink + (p - sink) % window
+
+
+def ring_contents(L: int, sink: int, window: int) -> np.ndarray:
+    """Position held by every slot after positions 0 .. L-1 were written in order (-1: empty)."""
+    slots = np.full(sink + window, -1, dtype=np.int64)
+    for p in range(L):
+        s = ring_slot(p, sink, window)
+        if s >= 0:
+            slots[s] = p
+    return slots
+
+
+def to_bf16_bits(x) -> np.ndarray:
+    """Round float64 values to bf16 storage: to float32 (nearest), then to 8 significant
+    bits, nearest with ties to even.  Returns the uint16 bit patterns (finite inputs)."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact float64 value of bf16 bit patterns."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def append_token_rows(q_raw: np.ndarray, k_raw: np.ndarray, v_raw: np.ndarray, position: int,
+                      theta: float) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Rows a decoded token adds: its query and key rotated to `position` (FASA §2.A
+    chunks), its value as given; all rounded to bf16 (bit patterns).
+
+    q_raw: [Hq, d]; k_raw, v_raw: [Hkv, d] (pre-rotation values).  The key is stored at
+    `position` = the number of tokens the sequence held before; the query sits at the
+    same position.
+    """
+    q = rope(np.asarray(q_raw, dtype=np.float64), [position] * len(q_raw), theta)
+    k = rope(np.asarray(k_raw, dtype=np.float64), [position] * len(k_raw), theta)
+    return to_bf16_bits(q), to_bf16_bits(k), to_bf16_bits(np.asarray(v_raw, dtype=np.float64))
+
+
+def pack_dominant_row(k_row: np.ndarray, idom: Sequence[int], cols: int) -> np.ndarray:
+    """The dominant columns of one key row: dims I_dom, then dims I_dom + d/2, zero-padded to cols."""
+    k_row = np.asarray(k_row)
+    dims = dominant_dims(idom, k_row.shape[0])
+    out = np.zeros(cols, dtype=k_row.dtype)
+    out[:len(dims)] = k_row[dims]
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # one decode step
 # --------------------------------------------------------------------------------------
 

@@ -7,7 +7,9 @@ restatement of the method could plausibly make: a RoPE rotation of the wrong
 sense, the wrong pairing of dims or a wrong frequency; a TIP that drops the
 c + d/2 term or scores one head of the group; a select that breaks ties toward
 the higher position or returns positions in score order; attention without the
-scale or with keys where values belong; a streaming window one token short.
+scale or with keys where values belong; a streaming window one token short; a ring
+slot one place off, bf16 storage by truncation, a token appended one position
+late, dominant columns packed in the wrong half order.
 """
 
 import inspect
@@ -118,6 +120,32 @@ def stream_window_short(L, sink, window):
     return np.array(sorted(keep), dtype=np.int64)
 
 
+def ring_slot_off_by_one(p, sink, window):
+    if p < sink:
+        return p
+    if window == 0:
+        return -1
+    return sink + (p - sink + 1) % window
+
+
+def bf16_truncate(x):
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def append_one_late(q_raw, k_raw, v_raw, position, theta):
+    return ref.__wrapped_append(q_raw, k_raw, v_raw, position + 1, theta)
+
+
+def pack_second_half_first(k_row, idom, cols):
+    k_row = np.asarray(k_row)
+    C = k_row.shape[0] // 2
+    dims = [int(c) + C for c in idom] + [int(c) for c in idom]
+    out = np.zeros(cols, dtype=k_row.dtype)
+    out[:len(dims)] = k_row[dims]
+    return out
+
+
 MUTANTS = {
     "rope_wrong_sense": ("rope", rope_wrong_sense),
     "rope_interleaved_pairs": ("rope", rope_interleaved),
@@ -129,6 +157,10 @@ MUTANTS = {
     "attend_without_scale": ("attend", attend_no_scale),
     "attend_keys_as_values": ("attend", attend_keys_for_values),
     "stream_window_one_short": ("stream_positions", stream_window_short),
+    "ring_slot_off_by_one": ("ring_slot", ring_slot_off_by_one),
+    "bf16_truncates": ("to_bf16_bits", bf16_truncate),
+    "append_one_position_late": ("append_token_rows", append_one_late),
+    "pack_second_half_first": ("pack_dominant_row", pack_second_half_first),
 }
 
 
@@ -158,6 +190,7 @@ def test_mutant_is_caught(mutant, monkeypatch):
     # helpers some mutants call: the original functions
     monkeypatch.setattr(ref, "__wrapped_tip", ref.tip_scores, raising=False)
     monkeypatch.setattr(ref, "__wrapped_attend", ref.attend, raising=False)
+    monkeypatch.setattr(ref, "__wrapped_append", ref.append_token_rows, raising=False)
     monkeypatch.setattr(ref, attr, fn)
     monkeypatch.setattr(oracle, attr, fn)
     failed = run_pins()

@@ -348,3 +348,74 @@ def test_shared_index_scores_are_full_dot_and_one_index_per_group():
             for j in range(2):
                 want = oracle.attend(ql[l, 0, 2 * g + j], k[r["sel"], g], v[r["sel"], g], 0.25)
                 assert np.allclose(r["out"][l, j], want, rtol=1e-14, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------- appending a token
+
+def test_ring_holds_exactly_the_streaming_positions():
+    # the ring of sink + window slots, written position by position, holds the sink plus the
+    # recent window: the set the streaming head attends to (brute force over small sizes)
+    for sink in range(0, 5):
+        for window in range(0, 7):
+            for L in range(0, 40):
+                held = oracle.ring_contents(L, sink, window)
+                kept = held[held >= 0]
+                assert len(set(kept.tolist())) == len(kept)  # a slot holds one position, none twice
+                assert sorted(kept.tolist()) == oracle.stream_positions(L, sink, window).tolist(), (L, sink, window)
+    # hand example: sink 2, window 3, ten tokens: slots hold 0 1 | 8 9 7
+    assert oracle.ring_contents(10, 2, 3).tolist() == [0, 1, 8, 9, 7]
+    assert oracle.ring_slot(1, 2, 3) == 1 and oracle.ring_slot(2, 2, 3) == 2 and oracle.ring_slot(5, 2, 3) == 2
+    assert oracle.ring_slot(7, 4, 0) == -1
+
+
+def test_bf16_rounding_hand_values_and_library():
+    one = 1.0
+    assert oracle.to_bf16_bits([one])[0] == 0x3F80
+    assert oracle.to_bf16_bits([-2.0])[0] == 0xC000
+    assert oracle.to_bf16_bits([1 + 2 ** -8])[0] == 0x3F80       # halfway: ties to the even code
+    assert oracle.to_bf16_bits([1 + 3 * 2 ** -8])[0] == 0x3F82   # halfway: ties to the even code
+    assert oracle.to_bf16_bits([1 + 2 ** -8 + 2 ** -20])[0] == 0x3F81  # above halfway: up
+    assert oracle.to_bf16_bits([0.0])[0] == 0 and oracle.to_bf16_bits([-0.0])[0] == 0x8000
+    # the same codes as the library's float32 -> bfloat16 conversion
+    import torch
+
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))).astype(np.float32)
+    lib = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.to_bf16_bits(x.astype(np.float64)), lib)
+    assert np.array_equal(oracle.bf16_bits_to_f64(lib), torch.from_numpy(lib.view(np.int16)).view(torch.bfloat16)
+                          .double().numpy())
+
+
+def test_append_one_at_a_time_equals_rotating_the_whole_sequence():
+    # a key appended when the sequence held p tokens sits at position p: appending L tokens
+    # one by one gives the cache that rotating the raw keys at 0 .. L-1 gives
+    rng = np.random.default_rng(11)
+    d, Hkv, Hq, L, theta = 16, 2, 4, 9, 1e4
+    raw_k = rng.standard_normal((L, Hkv, d))
+    raw_v = rng.standard_normal((L, Hkv, d))
+    raw_q = rng.standard_normal((L, Hq, d))
+    for p in range(L):
+        qb, kb, vb = oracle.append_token_rows(raw_q[p], raw_k[p], raw_v[p], p, theta)
+        for g in range(Hkv):
+            whole = oracle.to_bf16_bits(oracle.rope(raw_k[:, g], range(L), theta))
+            assert np.array_equal(kb[g], whole[p])
+        assert np.array_equal(vb, oracle.to_bf16_bits(raw_v[p]))
+        assert np.array_equal(qb, oracle.to_bf16_bits(oracle.rope(raw_q[p], [p] * Hq, theta)))
+
+
+def test_query_and_key_of_one_token_keep_their_raw_dot():
+    # rotated to the same position, a token's q and k have the raw q.k (closed form)
+    rng = np.random.default_rng(12)
+    q, k = rng.standard_normal((1, 8)), rng.standard_normal((1, 8))
+    for p in (0, 1, 17, 4096):
+        a = oracle.rope(q, [p], 500.0)[0] @ oracle.rope(k, [p], 500.0)[0]
+        assert abs(a - float(q[0] @ k[0])) < 1e-12
+        b = oracle.rope(q, [p + 1], 500.0)[0] @ oracle.rope(k, [p], 500.0)[0]
+        assert abs(b - float(q[0] @ k[0])) > 1e-6
+
+
+def test_pack_dominant_row_hand_example():
+    k = np.arange(8.0)  # d = 8, chunks 0..3 pair dims (c, c + 4)
+    assert oracle.pack_dominant_row(k, [1, 3], 8).tolist() == [1.0, 3.0, 5.0, 7.0, 0, 0, 0, 0]
+    assert oracle.pack_dominant_row(k, [0], 2).tolist() == [0.0, 4.0]
