@@ -79,11 +79,35 @@ enum {
  * multiples of 8 elements (every row starts on a 16-byte boundary).
  *
  * k_dom (optional) is a packed copy of the dominant columns of K, laid out
- * [n_kv_heads][total_tokens][k_dom_cols]: in row (h, t), column j < n_dom
- * holds K dim I_dom[h][j], column n_dom + j holds dim I_dom[h][j] + d/2, the
- * rest (up to k_dom_cols, a multiple of 8) are zero.  aoh_pack_dominant
- * writes it.  With it the importance scan reads 4 * n_dom bytes per token
- * and head instead of the sectors of K that the chunks touch.
+ * [head slots][total_tokens][k_dom_cols]: in row (slot of h, t), column
+ * j < n_dom holds K dim I_dom[h][j], column n_dom + j holds dim I_dom[h][j] +
+ * d/2, the rest (up to k_dom_cols, a multiple of 8) are zero.
+ * aoh_pack_dominant writes it, aoh_kv_append extends it.  With it the
+ * importance scan reads 4 * n_dom bytes per token and head instead of the
+ * sectors of K that the chunks touch.
+ *
+ * Lengths and capacity (ABI 2).  With lengths == NULL sequence b fills its
+ * region [offsets[b], offsets[b+1]): L_b = offsets[b+1] - offsets[b].  With
+ * lengths, sequence b holds positions 0 .. lengths[b] - 1 and its region is
+ * its capacity; tokens of the region past the length are never read.
+ *
+ * Head slots (ABI 2).  KV head g's rows are stored in head slot s =
+ * head_slot[g] (identity when head_slot is NULL): element i of position p is at
+ * k[t * stride_tok + s * stride_head + i] with t the position's token.  A
+ * cache need not store every head: AOH_NO_SLOT marks a head it does not store,
+ * and every call on that cache skips such heads.  So the retrieval heads of the
+ * AoH split can live in one cache (the whole history) and the streaming heads in
+ * a ring (below), each sized for the heads it holds.
+ *
+ * Layouts.  ring_sink = ring_window = 0: the linear layout, position p is
+ * token offsets[b] + p (lengths[b] <= offsets[b+1] - offsets[b], else device
+ * check 4 and the length is clamped).  Otherwise the ring layout of a streaming
+ * head's cache (AoH summary, Metodologia section 4: a fixed sink plus a recent
+ * window): the region holds ring_sink + ring_window slots, position p < sink
+ * is slot p and a later position is slot sink + (p - sink) mod window, so
+ * after L tokens the ring holds exactly positions [0, min(sink, L)) and
+ * [max(sink, L - window), L).  Only aoh_stream_decode (STREAM heads) and
+ * aoh_kv_append use a ring; the other calls refuse it.
  */
 typedef struct aoh_kv_cache {
   const void* k;               /* device, bf16                                         */
@@ -96,14 +120,22 @@ typedef struct aoh_kv_cache {
   int64_t total_tokens;        /* host copy of offsets[batch], < 2^31                  */
   int64_t stride_tok;          /* elements between tokens t and t+1 of one head        */
   int64_t stride_head;         /* elements between heads h and h+1 of one token        */
-  const void* k_dom;           /* device bf16 [Hkv][total_tokens][k_dom_cols], or NULL */
+  const void* k_dom;           /* device bf16 [slots][total_tokens][k_dom_cols], or NULL */
   int32_t k_dom_cols;          /* row length of k_dom in elements (0 when k_dom NULL)  */
+  /* ABI 2 (zero-filled: the ABI 1 meaning) */
+  const int32_t* lengths;      /* device int32 [batch] or NULL: positions held per sequence */
+  const uint8_t* head_slot;    /* host uint8 [n_kv_heads] or NULL (identity); read per call */
+  int32_t ring_sink;           /* ring layout: sink slots (0 and 0: linear layout)      */
+  int32_t ring_window;         /* ring layout: window slots                            */
 } aoh_kv_cache;
+
+#define AOH_NO_SLOT 255        /* head_slot entry of a head the cache does not store    */
 
 /* Human-readable name of a status code (static string). */
 const char* aoh_status_string(aoh_status s);
 
-/* Library ABI version: 1. */
+/* Library ABI version: 2 (1 plus lengths, head slots and rings in aoh_kv_cache,
+ * and aoh_kv_append). */
 int32_t aoh_version(void);
 
 /* The cudaError_t code behind the last AOH_ERR_CUDA returned on the calling
@@ -117,7 +149,8 @@ typedef enum {
   AOH_KERNEL_SPARSE_ROW = 2,    /* fused row kernel, or its select-only form         */
   AOH_KERNEL_FLASH_GATHER = 3,  /* split-K gather / window attention                 */
   AOH_KERNEL_PACK_DOMINANT = 4, /* dominant-column packing of K                      */
-  AOH_KERNEL_KINDS = 5
+  AOH_KERNEL_KV_APPEND = 5,     /* rotation and append of a decoded token            */
+  AOH_KERNEL_KINDS = 6
 } aoh_kernel_kind;
 
 /*
@@ -149,7 +182,9 @@ void aoh_record_launch_events(void** events, int32_t* kinds, int32_t n);
  * `detail` is not NULL, writes 4 host int32: check id, then three values of
  * the first failing access), or AOH_ERR_CUDA.  Check ids: 1 a position
  * outside [0, L_b) or offsets past the cache, 2 a count or per-sequence
- * N_fac above the capacity, 3 a chunk id outside [0, d/2).
+ * N_fac above the capacity, 3 a chunk id outside [0, d/2), 4 a sequence
+ * length or appended position past its region's capacity (or a ring region
+ * smaller than its slots).
  */
 aoh_status aoh_device_check(void* stream, int32_t* detail);
 
@@ -332,6 +367,37 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
 
 size_t aoh_shared_index_step_workspace_size(const aoh_kv_cache* kv, int32_t n_layers,
                                             int32_t n_q_heads, int32_t topk);
+
+/*
+ * aoh_kv_append -- add the decoded token of every sequence to the caches.
+ * The token's key and query are rotated by RoPE to its absolute position p
+ * (FASA section 2.A: chunk c = dims (c, c + d/2) turned by p * theta^(-2c/d);
+ * angles and rotation in double precision, stored as bf16 rounded to nearest,
+ * ties to even); its key and value rows go to every cache that stores the
+ * head: the linear cache for retrieval heads (the whole history) and the ring
+ * for streaming heads (sink plus recent window), as the AoH summary's
+ * Metodologia section 4 deploys them; the packed dominant row of each head the
+ * linear cache stores is written when it has k_dom (FASA section 2.C).
+ *   q_new      device bf16 [B][n_q_heads][d], before rotation, or NULL
+ *   k_new, v_new  device bf16 [B][Hkv][d]: the key before rotation, the value
+ *   theta      RoPE base (> 0)
+ *   kv         the linear cache (ring_sink = ring_window = 0), or NULL
+ *   ring       a ring-layout cache with the same batch / heads / head_dim, or
+ *              NULL.  Every KV head must be stored by kv or ring (or both).
+ *              The descriptors' own lengths fields are not used here.
+ *   idom, n_dom  I_dom of every KV head, required when kv->k_dom is set
+ *   lengths    device int32 [B]: p = lengths[b] is the new token's position;
+ *              after the rows are written lengths[b] = p + 1
+ *   q_out      device bf16 [B][n_q_heads][d]: q rotated to p (NULL iff q_new is)
+ * A sequence whose linear region is full (p >= offsets[b+1] - offsets[b]), or
+ * whose ring region has fewer than ring_sink + ring_window tokens, is left
+ * unchanged (lengths included) and device check 4 is recorded.  Decoding after
+ * the append attends over positions 0 .. p: the new token included.
+ */
+aoh_status aoh_kv_append(const void* q_new, int32_t n_q_heads, const void* k_new, const void* v_new,
+                         double theta, const aoh_kv_cache* kv, const aoh_kv_cache* ring,
+                         const int32_t* idom, int32_t n_dom, int32_t* lengths, void* q_out,
+                         void* stream);
 
 #ifdef __cplusplus
 }

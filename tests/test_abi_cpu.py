@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.aoh_version() == 1
+    assert lib.aoh_version() == 2
     assert lib.aoh_status_string(0) == b"ok"
     assert lib.aoh_status_string(4).startswith(b"workspace")
     assert lib.aoh_status_string(99) == b"unknown status"
@@ -67,9 +67,11 @@ def test_struct_layout_matches_header():
     #include <stddef.h>
     #include "aoh.h"
     int main(void) {
-      printf("%zu %zu %zu %zu %zu %zu\n", sizeof(aoh_kv_cache), offsetof(aoh_kv_cache, batch),
+      printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(aoh_kv_cache), offsetof(aoh_kv_cache, batch),
              offsetof(aoh_kv_cache, total_tokens), offsetof(aoh_kv_cache, stride_head),
-             offsetof(aoh_kv_cache, k_dom), offsetof(aoh_kv_cache, k_dom_cols));
+             offsetof(aoh_kv_cache, k_dom), offsetof(aoh_kv_cache, k_dom_cols),
+             offsetof(aoh_kv_cache, lengths), offsetof(aoh_kv_cache, head_slot),
+             offsetof(aoh_kv_cache, ring_sink), offsetof(aoh_kv_cache, ring_window));
       return 0;
     }
     """
@@ -81,7 +83,8 @@ def test_struct_layout_matches_header():
         vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()]
     K = B.KVCache
     assert vals == [ctypes.sizeof(K), K.batch.offset, K.total_tokens.offset, K.stride_head.offset,
-                    K.k_dom.offset, K.k_dom_cols.offset]
+                    K.k_dom.offset, K.k_dom_cols.offset, K.lengths.offset, K.head_slot.offset,
+                    K.ring_sink.offset, K.ring_window.offset]
 
 
 def fake_kv(**kw):
@@ -148,3 +151,49 @@ def test_workspace_sizes_are_host_computations(lib):
     assert lib.aoh_shared_index_decode_workspace_size(ctypes.byref(kv), 8, 32, 2048) > 0
     assert lib.aoh_shared_index_decode_workspace_size(ctypes.byref(kv), 9, 32, 2048) == 0
     assert lib.aoh_sparse_decode_workspace_size(ctypes.byref(fake_kv(head_dim=96)), 32, 64) == 0
+
+
+def test_ring_and_append_rules_are_checked_on_the_host(lib):
+    INVALID = 1
+    ring = fake_kv(ring_sink=16, ring_window=64)
+    roles = (ctypes.c_uint8 * 8)(*([2] * 8))            # every head STREAM
+    r = ctypes.cast(roles, ctypes.c_void_p)
+    # a ring serves streaming heads within its sink and window, and nothing else
+    assert call_sparse(lib, ring) == INVALID
+    assert lib.aoh_tip_score(0x40000, 32, ctypes.byref(ring), 0x50000, 16, 0x60000, None) == INVALID
+    assert lib.aoh_pack_dominant(ctypes.byref(ring), 0x50000, 16, 0x60000, 32, None) == INVALID
+    assert lib.aoh_stream_decode(0x40000, 32, ctypes.byref(ring), r, 17, 64, 0.1, 0x60000, 0x70000,
+                                 1 << 40, None) == INVALID  # sink beyond the ring's
+    assert lib.aoh_stream_decode(0x40000, 32, ctypes.byref(ring), r, 16, 65, 0.1, 0x60000, 0x70000,
+                                 1 << 40, None) == INVALID  # window beyond the ring's
+    dense = (ctypes.c_uint8 * 8)(1, 2, 2, 2, 2, 2, 2, 2)
+    assert lib.aoh_stream_decode(0x40000, 32, ctypes.byref(ring), ctypes.cast(dense, ctypes.c_void_p), 16, 64, 0.1,
+                                 0x60000, 0x70000, 1 << 40, None) == INVALID  # a DENSE head stored in a ring
+    # ... unless the ring does not store that head
+    slots = (ctypes.c_uint8 * 8)(255, 0, 1, 2, 3, 4, 5, 6)
+    ring2 = fake_kv(ring_sink=16, ring_window=64, head_slot=ctypes.cast(slots, ctypes.c_void_p).value)
+    assert lib.aoh_stream_decode_workspace_size(ctypes.byref(ring2), 32, ctypes.cast(dense, ctypes.c_void_p),
+                                                16, 64) > 0
+    # append: a linear cache and a ring, every head kept somewhere, lengths required
+    lin = fake_kv()
+    app = lib.aoh_kv_append
+    assert app(0x40000, 32, 0x50000, 0x58000, 5e5, None, None, None, 0, 0x60000, 0x68000, None) == INVALID
+    assert app(0x40000, 32, 0x50000, 0x58000, 5e5, ctypes.byref(ring), None, None, 0, 0x60000, 0x68000,
+               None) == INVALID                       # a ring given as the linear cache
+    assert app(0x40000, 32, 0x50000, 0x58000, 5e5, None, ctypes.byref(lin), None, 0, 0x60000, 0x68000,
+               None) == INVALID                       # a linear cache given as the ring
+    only_two = (ctypes.c_uint8 * 8)(0, 1, 255, 255, 255, 255, 255, 255)
+    part = fake_kv(head_slot=ctypes.cast(only_two, ctypes.c_void_p).value)
+    assert app(0x40000, 32, 0x50000, 0x58000, 5e5, ctypes.byref(part), None, None, 0, 0x60000, 0x68000,
+               None) == INVALID                       # heads 2..7 kept nowhere
+    assert app(0x40000, 32, 0x50000, 0x58000, 5e5, ctypes.byref(lin), None, None, 0, None, 0x68000,
+               None) == INVALID                       # no lengths
+    assert app(0x40000, 32, 0x50000, 0x58000, -1.0, ctypes.byref(lin), None, None, 0, 0x60000, 0x68000,
+               None) == INVALID                       # theta <= 0
+    assert app(0x40000, 32, 0x50000, 0x58000, 5e5, ctypes.byref(lin), None, None, 0, 0x60000, None,
+               None) == INVALID                       # q without q_out
+    packed = fake_kv(k_dom=0x80000, k_dom_cols=32)
+    assert app(None, 0, 0x50000, 0x58000, 5e5, ctypes.byref(packed), None, None, 0, 0x60000, None,
+               None) == INVALID                       # k_dom without I_dom
+    assert app(None, 0, 0x50000, 0x58000, 5e5, ctypes.byref(fake_kv(batch=0)), None, None, 0, None, None,
+               None) == 0                             # empty batch: nothing to do

@@ -26,12 +26,13 @@ EXPORTS = (
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
     "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
-    "aoh_launch_counts", "aoh_record_launch_events",
+    "aoh_launch_counts", "aoh_record_launch_events", "aoh_kv_append",
 )
+NO_SLOT = 255  # head_slot entry of a KV head a cache does not store
 
 # aoh_kernel_kind order
 KERNELS = ("tip_score_kernel", "topk_select_kernel", "sparse_row_kernel", "flash_gather_kernel",
-           "pack_dominant_kernel")
+           "pack_dominant_kernel", "kv_append_kernel")
 
 
 class AohError(RuntimeError):
@@ -50,6 +51,8 @@ class KVCache(ctypes.Structure):
         ("batch", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("max_len", ctypes.c_int32), ("total_tokens", ctypes.c_int64), ("stride_tok", ctypes.c_int64),
         ("stride_head", ctypes.c_int64), ("k_dom", ctypes.c_void_p), ("k_dom_cols", ctypes.c_int32),
+        ("lengths", ctypes.c_void_p), ("head_slot", ctypes.c_void_p), ("ring_sink", ctypes.c_int32),
+        ("ring_window", ctypes.c_int32),
     ]
 
 
@@ -84,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "aoh_shared_index_step": (ctypes.c_int, [P, P, I32, I32, KVP, I32, P, P, F32, P, P, SZ, P]),
             "aoh_shared_index_step_workspace_size": (SZ, [KVP, I32, I32, I32]),
             "aoh_stream_decode_noalloc": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P]),
+            "aoh_kv_append": (ctypes.c_int, [P, I32, P, P, ctypes.c_double, KVP, KVP, P, I32, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -115,17 +119,32 @@ def _host_u8(arr) -> Optional[ctypes.Array]:
 
 
 def make_kv(k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
-            k_dom: Optional[torch.Tensor] = None) -> KVCache:
-    """Describe a cache held in torch tensors k, v of shape [T, Hkv, d] (bf16, last dim contiguous)."""
+            k_dom: Optional[torch.Tensor] = None, lengths: Optional[torch.Tensor] = None, head_slot=None,
+            n_kv_heads: Optional[int] = None, ring: Optional[tuple] = None) -> KVCache:
+    """Describe a cache held in torch tensors k, v of shape [T, slots, d] (bf16, last dim contiguous).
+
+    lengths: device int32 [B] (positions held per sequence) or None (sequences fill their regions);
+    head_slot: per KV head its slot in k / v (NO_SLOT: not stored here), or None (identity, slots = heads);
+    n_kv_heads: the model's KV heads (default: k.shape[1]); ring: (sink, window) for a ring layout.
+    """
     assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16 and k.is_cuda and v.is_cuda
     assert k.shape == v.shape and k.stride() == v.stride() and k.stride(2) == 1
     assert offsets.dtype == torch.int32 and offsets.is_cuda
+    assert lengths is None or (lengths.dtype == torch.int32 and lengths.is_cuda)
     kv = KVCache()
-    kv._keep = (k, v, offsets, k_dom)  # the descriptor holds raw pointers: keep the tensors alive with it
+    slots = None if head_slot is None else (ctypes.c_uint8 * len(head_slot))(*[int(x) for x in head_slot])
+    kv._keep = (k, v, offsets, k_dom, lengths, slots)  # raw pointers: keep their owners alive with the descriptor
     kv.k, kv.v, kv.offsets = k.data_ptr(), v.data_ptr(), offsets.data_ptr()
     kv.batch = offsets.numel() - 1
-    kv.n_kv_heads = k.shape[1]
+    kv.n_kv_heads = n_kv_heads if n_kv_heads is not None else k.shape[1]
     kv.head_dim = k.shape[2]
+    if lengths is not None:
+        kv.lengths = lengths.data_ptr()
+    if slots is not None:
+        assert len(head_slot) == kv.n_kv_heads
+        kv.head_slot = ctypes.cast(slots, ctypes.c_void_p).value
+    if ring is not None:
+        kv.ring_sink, kv.ring_window = int(ring[0]), int(ring[1])
     kv.max_len = int(max_len)
     kv.total_tokens = int(total_tokens)
     kv.stride_tok = k.stride(0)
@@ -274,3 +293,13 @@ def stream_decode_noalloc(q: torch.Tensor, kv: KVCache, roles, sink: int, window
     _check("aoh_stream_decode_noalloc", lib().aoh_stream_decode_noalloc(
         _ptr(q), q.shape[-2], ctypes.byref(kv), ctypes.cast(r, ctypes.c_void_p), sink, window, float(scale),
         _ptr(out), _stream(stream)))
+
+
+def kv_append(q_new: Optional[torch.Tensor], k_new: torch.Tensor, v_new: torch.Tensor, theta: float,
+              kv: Optional[KVCache], ring: Optional[KVCache], idom: Optional[torch.Tensor], n_dom: int,
+              lengths: torch.Tensor, q_out: Optional[torch.Tensor], stream=None) -> None:
+    """Rotate and append every sequence's decoded token (aoh_kv_append); lengths[b] += 1."""
+    _check("aoh_kv_append", lib().aoh_kv_append(
+        _ptr(q_new), 0 if q_new is None else q_new.shape[-2], _ptr(k_new), _ptr(v_new), float(theta),
+        None if kv is None else ctypes.byref(kv), None if ring is None else ctypes.byref(ring), _ptr(idom),
+        int(n_dom), _ptr(lengths), _ptr(q_out), _stream(stream)))

@@ -13,6 +13,7 @@
 #include "aoh.h"
 #include "device_common.cuh"
 #include "flash_gather.cuh"
+#include "kv_append.cuh"
 #include "sparse_row.cuh"
 #include "tip_score.cuh"
 #include "topk_select.cuh"
@@ -43,7 +44,20 @@ aoh_status check_kv(const aoh_kv_cache* kv) {
     if (kv->k_dom_cols < 8 || kv->k_dom_cols > 128 || (kv->k_dom_cols % 8)) return AOH_ERR_INVALID_ARG;
     if (!aligned16(kv->k_dom)) return AOH_ERR_ALIGNMENT;
   }
+  if (kv->ring_sink < 0 || kv->ring_window < 0) return AOH_ERR_INVALID_ARG;
   return AOH_OK;
+}
+
+bool is_ring(const aoh_kv_cache* kv) { return kv->ring_sink + kv->ring_window > 0; }
+
+// KV head g's slot in this cache's K / V (and k_dom), or kNoSlot when the cache does not store it
+uint8_t slot_of(const aoh_kv_cache* kv, int g) { return kv->head_slot ? kv->head_slot[g] : (uint8_t)g; }
+
+// per-sequence lengths and head slots of the cache, into any kernel's parameters
+template <typename P>
+void bind_cache(P& prm, const aoh_kv_cache* kv) {
+  prm.lengths = kv->lengths;
+  for (int g = 0; g < kv->n_kv_heads; ++g) prm.slot[g] = slot_of(kv, g);
 }
 
 aoh_status check_heads(const aoh_kv_cache* kv, int32_t n_q_heads) {
@@ -297,6 +311,7 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
   tp.q = static_cast<const uint16_t*>(q);
   tp.idom = idom;
   tp.offsets = kv->offsets;
+  bind_cache(tp, kv);
   tp.scores = scores;
   tp.T = (int32_t)kv->total_tokens;
   tp.Hq = Hq;
@@ -348,6 +363,7 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
   SelectParams sp{};
   sp.scores = scores;
   sp.offsets = kv->offsets;
+  bind_cache(sp, kv);
   sp.n_fac_per_seq = nfps;
   sp.idx = idx;
   sp.count = count;
@@ -496,6 +512,7 @@ aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32
                               cudaStream_t st) {
   RowParams rp{};
   rp.offsets = kv->offsets;
+  bind_cache(rp, kv);
   rp.scores_in = scores;
   rp.select_only = 1;
   rp.n_fac_per_seq = nfps;
@@ -552,12 +569,13 @@ void rows_score_source(RowParams& rp, const aoh_kv_cache* kv, const int32_t* ido
   }
 }
 
+// The KV heads a call computes: those of its roles that this cache stores.
 int list_heads(const aoh_kv_cache* kv, const uint8_t* roles, bool want_sparse, uint8_t* out) {
   int n = 0;
   for (int g = 0; g < kv->n_kv_heads; ++g) {
     const uint8_t r = roles ? roles[g] : (uint8_t)AOH_ROLE_SPARSE;
     const bool sparse = (r == AOH_ROLE_SPARSE);
-    if (sparse == want_sparse) out[n++] = (uint8_t)g;
+    if (sparse == want_sparse && slot_of(kv, g) != kNoSlot) out[n++] = (uint8_t)g;
   }
   return n;
 }
@@ -593,7 +611,7 @@ FdGeom stream_geom(const aoh_kv_cache* kv, int32_t Hq, const uint8_t* roles, int
   int64_t n_max = 0, work = 0;
   for (int g = 0; g < kv->n_kv_heads; ++g) {
     const uint8_t r = roles[g];
-    if (r == AOH_ROLE_SPARSE) continue;
+    if (r == AOH_ROLE_SPARSE || slot_of(kv, g) == kNoSlot) continue;
     const int64_t L = kv->max_len;
     const int64_t n = (r == AOH_ROLE_DENSE) ? L : std::min<int64_t>(L, int64_t(sink) + window);
     n_max = std::max(n_max, n);
@@ -607,6 +625,16 @@ FdGeom shared_geom(const aoh_kv_cache* kv, int32_t n_layers, int32_t Hq, int32_t
   const int G = Hq / kv->n_kv_heads;
   const int rows = kv->batch * kv->n_kv_heads;
   return fd_geom(int64_t(rows) * cap, cap, rows, n_layers * G, kv->head_dim);
+}
+
+// A ring keeps only streaming heads' sink and window: it serves STREAM heads whose sink and
+// window lie within its own, and stores no DENSE head.
+aoh_status check_ring_roles(const aoh_kv_cache* kv, const uint8_t* roles, int32_t sink, int32_t window) {
+  if (!is_ring(kv)) return AOH_OK;
+  if (sink > kv->ring_sink || window > kv->ring_window) return AOH_ERR_INVALID_ARG;
+  for (int g = 0; g < kv->n_kv_heads; ++g)
+    if (roles[g] == AOH_ROLE_DENSE && slot_of(kv, g) != kNoSlot) return AOH_ERR_INVALID_ARG;
+  return AOH_OK;
 }
 
 bool ws_ok(const void* ws, size_t have, size_t need) {
@@ -632,7 +660,7 @@ const char* aoh_status_string(aoh_status s) {
   return "unknown status";
 }
 
-int32_t aoh_version(void) { return 1; }
+int32_t aoh_version(void) { return 2; }
 
 int32_t aoh_last_cuda_error(void) { return t_last_cuda_error; }
 
@@ -668,6 +696,7 @@ aoh_status aoh_pack_dominant(const aoh_kv_cache* kv, const int32_t* idom, int32_
   if (kv->batch == 0 || kv->total_tokens == 0) return AOH_OK;
   if (!idom || !k_dom) return AOH_ERR_INVALID_ARG;
   if (!aligned16(k_dom)) return AOH_ERR_ALIGNMENT;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;
   PackParams pp{};
   pp.k = static_cast<const uint16_t*>(kv->k);
   pp.idom = idom;
@@ -675,11 +704,13 @@ aoh_status aoh_pack_dominant(const aoh_kv_cache* kv, const int32_t* idom, int32_
   pp.stride_tok = kv->stride_tok;
   pp.stride_head = kv->stride_head;
   pp.T = (int32_t)kv->total_tokens;
-  pp.Hkv = kv->n_kv_heads;
   pp.d = kv->head_dim;
   pp.n_dom = n_dom;
   pp.cols = k_dom_cols;
-  const int64_t total = int64_t(pp.Hkv) * pp.T * pp.cols;
+  pp.n_listed = list_heads(kv, nullptr, true, pp.heads);  // every stored head (roles NULL: all SPARSE)
+  for (int g = 0; g < kv->n_kv_heads; ++g) pp.slot[g] = slot_of(kv, g);
+  if (pp.n_listed == 0) return AOH_OK;
+  const int64_t total = int64_t(pp.n_listed) * pp.T * pp.cols;
   const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), int64_t(sm_count()) * 16);
   before_launch(as_stream(stream));
   pack_dominant_kernel<<<blocks, 256, 0, as_stream(stream)>>>(pp);
@@ -690,6 +721,7 @@ aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* k
                          int32_t n_dom, float* scores, void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;  // a ring holds streaming heads only
   if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
   if (n_dom < 1 || n_dom > kv->head_dim / 2) return AOH_ERR_INVALID_ARG;
   if (kv->batch == 0 || kv->total_tokens == 0) return AOH_OK;
@@ -704,6 +736,7 @@ aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t 
                            void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;  // a ring holds streaming heads only
   if (n_fac_cap < 1) return AOH_ERR_INVALID_ARG;
   if (!n_fac_per_seq && (n_fac < 0 || n_fac > n_fac_cap)) return AOH_ERR_INVALID_ARG;
   if (kv->batch == 0) return AOH_OK;
@@ -726,6 +759,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
                              int32_t* count_out, void* workspace, size_t workspace_bytes, void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;  // a ring holds streaming heads only
   if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
   if ((s = check_roles(kv, roles)) != AOH_OK) return s;
   const int G = n_q_heads / kv->n_kv_heads;
@@ -758,6 +792,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
     rp.k = static_cast<const uint16_t*>(kv->k);
     rp.v = static_cast<const uint16_t*>(kv->v);
     rp.offsets = kv->offsets;
+    bind_cache(rp, kv);
     rows_score_source(rp, kv, idom, n_dom);
     rp.n_fac_per_seq = n_fac_per_seq;
     rp.n_fac = n_fac;
@@ -795,6 +830,7 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   fp.k = static_cast<const uint16_t*>(kv->k);
   fp.v = static_cast<const uint16_t*>(kv->v);
   fp.offsets = kv->offsets;
+  bind_cache(fp, kv);
   fp.idx = idx;
   fp.count = cnt;
   fp.out = out;
@@ -832,6 +868,7 @@ aoh_status aoh_stream_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   const int G = n_q_heads / kv->n_kv_heads;
   if (G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
   if (sink < 0 || window < 0 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  if ((s = check_ring_roles(kv, roles, sink, window)) != AOH_OK) return s;
   if (kv->batch == 0) return AOH_OK;
   if (!q || !out) return AOH_ERR_INVALID_ARG;
   if (!aligned16(q)) return AOH_ERR_ALIGNMENT;
@@ -845,6 +882,7 @@ aoh_status aoh_stream_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   fp.k = static_cast<const uint16_t*>(kv->k);
   fp.v = static_cast<const uint16_t*>(kv->v);
   fp.offsets = kv->offsets;
+  bind_cache(fp, kv);
   fp.out = out;
   fp.stride_tok = kv->stride_tok;
   fp.stride_head = kv->stride_head;
@@ -857,6 +895,8 @@ aoh_status aoh_stream_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   fp.list_mode = 0;
   fp.sink = sink;
   fp.window = window;
+  fp.ring_sink = kv->ring_sink;
+  fp.ring_window = kv->ring_window;
   fp.scale_log2 = scale * 1.4426950408889634f;
   memcpy(fp.heads, heads, n_listed);
   memcpy(fp.roles, roles, kv->n_kv_heads);
@@ -877,6 +917,7 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
                                    size_t workspace_bytes, void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;  // a ring holds streaming heads only
   if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
   if (n_layers < 1 || n_fac_cap < 1 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
   const int G = n_q_heads / kv->n_kv_heads;
@@ -893,6 +934,7 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
   fp.k = static_cast<const uint16_t*>(kv->k);
   fp.v = static_cast<const uint16_t*>(kv->v);
   fp.offsets = kv->offsets;
+  bind_cache(fp, kv);
   fp.idx = idx;
   fp.count = count;
   fp.out = out;
@@ -928,6 +970,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
                                  float* out, void* workspace, size_t workspace_bytes, void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;  // a ring holds streaming heads only
   if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
   if (n_layers < 1 || topk < 1 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
   const int G = n_q_heads / kv->n_kv_heads;
@@ -950,6 +993,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
     rp.k = static_cast<const uint16_t*>(kv->k);
     rp.v = static_cast<const uint16_t*>(kv->v);
     rp.offsets = kv->offsets;
+    bind_cache(rp, kv);
     rows_score_source(rp, kv, nullptr, kv->head_dim / 2);
     rp.n_fac_per_seq = nullptr;
     rp.n_fac = topk;
@@ -982,6 +1026,7 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   fp.k = static_cast<const uint16_t*>(kv->k);
   fp.v = static_cast<const uint16_t*>(kv->v);
   fp.offsets = kv->offsets;
+  bind_cache(fp, kv);
   fp.idx = idx;
   fp.count = count;
   fp.out = out;
@@ -998,6 +1043,80 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
   memcpy(fp.heads, heads, n_listed);
   fd_bind(fp, geo, ws);
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, st, true);
+}
+
+aoh_status aoh_kv_append(const void* q_new, int32_t n_q_heads, const void* k_new, const void* v_new, double theta,
+                         const aoh_kv_cache* kv, const aoh_kv_cache* ring, const int32_t* idom, int32_t n_dom,
+                         int32_t* lengths, void* q_out, void* stream) {
+  if (!kv && !ring) return AOH_ERR_INVALID_ARG;
+  aoh_status s;
+  if (kv) {
+    if ((s = check_kv(kv)) != AOH_OK) return s;
+    if (is_ring(kv)) return AOH_ERR_INVALID_ARG;
+  }
+  if (ring) {
+    if ((s = check_kv(ring)) != AOH_OK) return s;
+    if (!is_ring(ring)) return AOH_ERR_INVALID_ARG;
+    if (ring->k_dom) return AOH_ERR_INVALID_ARG;
+  }
+  const aoh_kv_cache* any = kv ? kv : ring;
+  if (kv && ring && (kv->batch != ring->batch || kv->n_kv_heads != ring->n_kv_heads ||
+                     kv->head_dim != ring->head_dim))
+    return AOH_ERR_INVALID_ARG;
+  for (int g = 0; g < any->n_kv_heads; ++g) {  // every head is kept somewhere
+    const bool in_kv = kv && slot_of(kv, g) != kNoSlot, in_ring = ring && slot_of(ring, g) != kNoSlot;
+    if (!in_kv && !in_ring) return AOH_ERR_INVALID_ARG;
+  }
+  if ((q_new == nullptr) != (q_out == nullptr)) return AOH_ERR_INVALID_ARG;
+  if (q_new && (n_q_heads < 1 || n_q_heads % any->n_kv_heads)) return AOH_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return AOH_ERR_INVALID_ARG;
+  const bool pack = kv && kv->k_dom;
+  if (pack && (!idom || n_dom < 1 || n_dom > kv->head_dim / 2 || 2 * n_dom > kv->k_dom_cols))
+    return AOH_ERR_INVALID_ARG;
+  if (any->batch == 0) return AOH_OK;
+  if (!k_new || !v_new || !lengths) return AOH_ERR_INVALID_ARG;
+  AppendParams ap{};
+  ap.q_new = static_cast<const uint16_t*>(q_new);
+  ap.k_new = static_cast<const uint16_t*>(k_new);
+  ap.v_new = static_cast<const uint16_t*>(v_new);
+  ap.q_out = static_cast<uint16_t*>(q_out);
+  ap.lengths = lengths;
+  ap.B = any->batch;
+  ap.Hq = q_new ? n_q_heads : 0;
+  ap.Hkv = any->n_kv_heads;
+  ap.d = any->head_dim;
+  ap.theta = theta;
+  for (int g = 0; g < any->n_kv_heads; ++g) {
+    ap.slot[g] = kv ? slot_of(kv, g) : kNoSlot;
+    ap.rslot[g] = ring ? slot_of(ring, g) : kNoSlot;
+  }
+  if (kv) {
+    ap.k = static_cast<uint16_t*>(const_cast<void*>(kv->k));
+    ap.v = static_cast<uint16_t*>(const_cast<void*>(kv->v));
+    ap.offsets = kv->offsets;
+    ap.stride_tok = kv->stride_tok;
+    ap.stride_head = kv->stride_head;
+    ap.T = kv->total_tokens;
+    if (pack) {
+      ap.k_dom = static_cast<uint16_t*>(const_cast<void*>(kv->k_dom));
+      ap.k_dom_cols = kv->k_dom_cols;
+      ap.idom = idom;
+      ap.n_dom = n_dom;
+    }
+  }
+  if (ring) {
+    ap.rk = static_cast<uint16_t*>(const_cast<void*>(ring->k));
+    ap.rv = static_cast<uint16_t*>(const_cast<void*>(ring->v));
+    ap.roffsets = ring->offsets;
+    ap.rstride_tok = ring->stride_tok;
+    ap.rstride_head = ring->stride_head;
+    ap.ring_sink = ring->ring_sink;
+    ap.ring_window = ring->ring_window;
+  }
+  cudaStream_t st = as_stream(stream);
+  before_launch(st);
+  kv_append_kernel<<<ap.B, kAppendThreads, 0, st>>>(ap);
+  return count_launch(AOH_KERNEL_KV_APPEND, st);
 }
 
 }  // extern "C"
@@ -1047,6 +1166,7 @@ extern "C" aoh_status aoh_stream_decode_noalloc(const void* q, int32_t n_q_heads
   if ((s = check_roles(kv, roles)) != AOH_OK) return s;
   if (n_q_heads / kv->n_kv_heads > kMaxQRows) return AOH_ERR_UNSUPPORTED;
   if (sink < 0 || window < 0 || !std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  if ((s = check_ring_roles(kv, roles, sink, window)) != AOH_OK) return s;
   if (kv->batch == 0) return AOH_OK;
   if (!q || !out) return AOH_ERR_INVALID_ARG;
   if (!aligned16(q)) return AOH_ERR_ALIGNMENT;

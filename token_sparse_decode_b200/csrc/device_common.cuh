@@ -17,7 +17,10 @@ enum DeviceCheck : int {
   kCheckPosition = 1,    // a stored position outside [0, L_b)
   kCheckCount = 2,       // a count or per-sequence N_fac above the row capacity
   kCheckChunk = 3,       // a chunk id outside [0, d/2)
+  kCheckCapacity = 4,    // a sequence length (or an appended position) past its region's capacity
 };
+
+constexpr uint8_t kNoSlot = 255;  // head_slot entry of a KV head that a cache does not store
 
 __device__ int g_device_error[4];
 
@@ -27,6 +30,33 @@ __device__ __forceinline__ void record_error(int id, int a, int b, int c) {
     g_device_error[2] = b;
     g_device_error[3] = c;
   }
+}
+
+// ------------------------------------------------------------------ sequences of a cache
+// Sequence b owns the tokens [offsets[b], offsets[b + 1]) of the cache (its region).
+// Without per-sequence lengths it fills the region; with them it holds positions
+// 0 .. lengths[b] - 1.  In the linear layout position p is token offsets[b] + p, so a
+// length beyond the region is recorded (check 4) and clamped to it; a ring keeps only
+// some positions (see ring_slot) and its length is not bounded by the region.
+__device__ __forceinline__ int seq_length(const int32_t* offsets, const int32_t* lengths, int b, bool ring,
+                                          int* off_out) {
+  const int off = offsets[b];
+  const int cap = offsets[b + 1] - off;
+  *off_out = off;
+  if (!lengths) return cap;
+  int L = lengths[b];
+  if (L < 0 || (!ring && L > cap)) {
+    record_error(kCheckCapacity, b, L, cap);
+    L = L < 0 ? 0 : cap;
+  }
+  return L;
+}
+
+// Slot of position p in a ring of `sink` + `window` slots: positions below the sink keep
+// their own slot, later ones take the window slots in turn (the caller reads only
+// positions the ring still holds: [0, min(sink, L)) and [max(sink, L - window), L)).
+__device__ __forceinline__ int ring_slot(int p, int sink, int window) {
+  return (p < sink || window <= 0) ? p : sink + (p - sink) % window;
 }
 
 // ------------------------------------------------------------------ bf16 unpacking

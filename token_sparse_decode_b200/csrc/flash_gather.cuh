@@ -5,7 +5,9 @@
 //   * focused attention over the selected tokens (FASA: Frequency-aware Sparse
 //     Attention, §2.B.2): positions come from the top-N_fac index, NQ = G;
 //   * retrieval / streaming heads (AoH summary, Metodología §4): positions are
-//     [0, L) or [0, min(S, L)) U [max(S, L - W), L), NQ = G;
+//     [0, L) or [0, min(S, L)) U [max(S, L - W), L), NQ = G; a streaming head may
+//     keep its rows in a ring of sink + window slots (then position p is read
+//     from slot ring_slot(p));
 //   * the shared-index cross-decoder layers ("Cómo funciona CLSA"): one index,
 //     NQ = n_layers * G query rows read every gathered K/V row once.
 //
@@ -48,6 +50,7 @@ struct FdecParams {
   const uint16_t* k;
   const uint16_t* v;
   const int32_t* offsets;    // [B + 1]
+  const int32_t* lengths;    // [B] or null (sequences fill their regions)
   const int32_t* idx;        // list mode: [B][Hkv][cap]
   const int32_t* count;      // list mode: [B][Hkv]
   float* out;                // row (l, b, h) at out + ((l * B + b) * Hq + h) * D
@@ -61,9 +64,12 @@ struct FdecParams {
   int32_t list_mode;         // 1: positions from idx/count; 0: role ranges
   int32_t cluster_combine;   // 1: launched with clusters of max_splits CTAs (one row each)
   int32_t sink, window;
+  int32_t ring_sink, ring_window;  // range mode on a ring cache (> 0 sum): position p is kept in
+                                   // slot ring_slot(p); 0, 0: position p is token p of the region
   float scale_log2;          // softmax scale * log2(e)
   uint8_t heads[kMaxHeads];  // listed KV heads (blockIdx.y)
   uint8_t roles[kMaxHeads];  // role of every KV head (range mode)
+  uint8_t slot[kMaxHeads];   // head slot of every KV head in K / V
 };
 
 template <int D>
@@ -103,8 +109,9 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   const int g = p.heads[y];
   const int split = blockIdx.x;
   const int row_id = b * gridDim.y + y;
-  const int off = p.offsets[b];
-  const int L = p.offsets[b + 1] - off;
+  const bool ring = (p.ring_sink + p.ring_window) > 0;
+  int off;
+  const int L = seq_length(p.offsets, p.lengths, b, ring, &off);
 
   // ---- the row's list of positions
   int n, ra = 0, rb = 0;
@@ -117,6 +124,9 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     }
     n = max(n, 0);
     lst = p.idx + ((int64_t)b * p.Hkv + g) * p.cap;
+  } else if (ring && p.offsets[b + 1] - off < p.ring_sink + p.ring_window) {
+    // a ring region too small for its slots: nothing is read (recorded once, below)
+    n = 0;
   } else {
     if (p.roles[g] == 1) {  // DENSE
       ra = L;
@@ -130,6 +140,8 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   const int nsplit = (n + p.chunk - 1) / p.chunk;
 
   if (n == 0) {  // nothing to attend to: zero rows
+    if (ring && split == 0 && tid == 0 && p.offsets[b + 1] - off < p.ring_sink + p.ring_window)
+      record_error(kCheckCapacity, b, p.offsets[b + 1] - off, p.ring_sink + p.ring_window);
     if (split == 0) {
       for (int e = tid; e < p.NQ * D; e += kFdThreads) {
         const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
@@ -158,8 +170,8 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     __syncthreads();
   }
 
-  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
-  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)p.slot[g] * p.stride_head;
+  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)p.slot[g] * p.stride_head;
   const uint32_t sbase = smem_u32(smem);
 
   auto issue_stage = [&](int st) {
@@ -189,6 +201,7 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
             }
           } else {
             pos = j < ra ? j : rb + (j - ra);
+            if (ring) pos = ring_slot(pos, p.ring_sink, p.ring_window);
           }
         }
         const int64_t eo = (int64_t)pos * p.stride_tok + ch * 8;

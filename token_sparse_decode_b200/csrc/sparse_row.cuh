@@ -54,6 +54,7 @@ struct RowParams {
   const uint16_t* k;
   const uint16_t* v;
   const int32_t* offsets;    // [B + 1]
+  const int32_t* lengths;    // [B] or null (sequences fill their regions)
   const uint16_t* score_src; // packed k_dom or K
   int64_t srow_stride_tok, srow_stride_head;
   int32_t srow_len;          // elements per score row: 16, 32, 64 or 128 (k_dom cols, or D in place)
@@ -73,6 +74,7 @@ struct RowParams {
   int32_t select_only;       // 1: stop after writing the index (no attention)
   float scale_log2;
   uint8_t heads[kMaxHeads];
+  uint8_t slot[kMaxHeads];   // head slot of every KV head in K / V and in the score rows
 };
 
 // Attention tiles: gathered K / V rows are copied as 16-byte cp.async segments into rows
@@ -110,8 +112,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.z;
   const int g = p.heads[blockIdx.y];
-  const int off = p.offsets[b];
-  const int L = p.offsets[b + 1] - off;
+  int off;
+  const int L = seq_length(p.offsets, p.lengths, b, false, &off);
   int nf = p.n_fac_per_seq ? p.n_fac_per_seq[b] : p.n_fac;
   if (nf > p.cap) {
     if (rk == 0 && tid == 0) record_error(kCheckCount, b, nf, p.cap);
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       const int grows = rpw * kScanU;
       const int nb = (wr1 - wr0 + grows - 1) / grows;
       const uint32_t wring = smem_u32(smem + p.keys_bytes) + warp * (kScanDepth * kScanU * 512) + lane * 16;
-      const uint16_t* src0 = p.score_src + (int64_t)g * p.srow_stride_head + (int64_t)(off + lo) * p.srow_stride_tok + seg * 8;
+      const uint16_t* src0 = p.score_src + (int64_t)p.slot[g] * p.srow_stride_head + (int64_t)(off + lo) * p.srow_stride_tok + seg * 8;
       auto issue = [&](int k) {
         const uint32_t slot = wring + (k % kScanDepth) * (kScanU * 512);
 #pragma unroll
@@ -483,8 +485,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 
   uint8_t* stage_mem = smem + p.keys_bytes;
   const uint32_t sbase = smem_u32(stage_mem);
-  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
-  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)g * p.stride_head;
+  const uint16_t* kbase = p.k + (int64_t)off * p.stride_tok + (int64_t)p.slot[g] * p.stride_head;
+  const uint16_t* vbase = p.v + (int64_t)off * p.stride_tok + (int64_t)p.slot[g] * p.stride_head;
   const int nstages = (nloc + kSrTS - 1) / kSrTS;
   const int nsa = min(kSrMaxStages, p.ring_bytes / AttTile<D>::kStage);
   // every thread copies 16-byte chunks of the stage's K and V rows (cp.async); entries past

@@ -1,4 +1,6 @@
 // Token Importance Predictor scan (FASA: Frequency-aware Sparse Attention, §2.B.1).
+// (Rows are addressed through each KV head's slot in the cache; the unused tail of a
+// sequence's region, when the cache carries per-sequence lengths, is not scored.)
 //
 // For KV head g of sequence b the score of cached token t is the fp32 dot of
 //   q~_g = sum over the group's q heads of q_h, restricted to the dominant dims
@@ -24,6 +26,7 @@ struct TipParams {
   const uint16_t* src;      // packed k_dom or K
   const int32_t* idom;      // [Hkv][n_dom]; null: every chunk (K in place)
   const int32_t* offsets;   // [B + 1]
+  const int32_t* lengths;   // [B] or null (sequences fill their regions)
   float* scores;            // [Hkv][T]
   int64_t row_stride_tok;   // elements between token rows of one head
   int64_t row_stride_head;  // elements between heads
@@ -34,6 +37,7 @@ struct TipParams {
   int64_t per_cta;          // flattened (listed head, token) rows per CTA
   int64_t total;            // n_listed * T
   uint8_t heads[kMaxHeads]; // KV heads scored
+  uint8_t slot[kMaxHeads];  // head slot of every KV head in the row source
 };
 
 __device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
@@ -56,7 +60,7 @@ __device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
 template <int S>
 __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipParams p) {
   __shared__ float qt[128];
-  __shared__ int s_seg[2];  // sequence b of the segment (-1: none), its end token
+  __shared__ int s_seg[3];  // sequence b of the segment (-1: none), its region's end, its last token + 1
   const int tid = threadIdx.x, lane = tid & 31;
   const int C = p.d >> 1;
   const int seg = lane % S;
@@ -84,7 +88,7 @@ __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipPara
       }
     }
     active = active && seg * 8 < p.row_len;
-    const uint16_t* base = p.src + (int64_t)g * p.row_stride_head + (int64_t)t * p.row_stride_tok + seg * 8;
+    const uint16_t* base = p.src + (int64_t)p.slot[g] * p.row_stride_head + (int64_t)t * p.row_stride_tok + seg * 8;
     uint4 v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -104,7 +108,7 @@ __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipPara
         if (m) b = b0 + __ffs(m) - 1;
       }
       if (lane == 0) {
-        int e = p.T;
+        int e = p.T, ve = p.T;
         if (b < 0) {
           record_error(kCheckPosition, (int)j, t, -1);
         } else {
@@ -113,14 +117,22 @@ __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipPara
             record_error(kCheckPosition, (int)j, e, p.T);
             e = p.T;
           }
+          int off;
+          ve = p.lengths ? min(e, p.offsets[b] + seq_length(p.offsets, p.lengths, b, false, &off)) : e;
         }
         s_seg[0] = b;
         s_seg[1] = e;
+        s_seg[2] = ve;
       }
     }
     __syncthreads();
     const int b = s_seg[0];
-    const int n = min(lim, s_seg[1] - t);  // rows of the segment (>= 1)
+    if (t >= s_seg[2]) {  // the unused tail of a sequence's region: nothing to score
+      w += min(lim, s_seg[1] - t);
+      __syncthreads();    // s_seg is rewritten by the next segment
+      continue;
+    }
+    const int n = min(lim, s_seg[2] - t);  // rows of the segment (>= 1)
     if (b >= 0) bhint = b;
     // q~ for (b, g): fp32 group sum in head order, restricted to the dominant dims
     if (tid < p.row_len) {
@@ -185,20 +197,23 @@ __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipPara
 struct PackParams {
   const uint16_t* k;
   const int32_t* idom;
-  uint16_t* k_dom;          // [Hkv][T][cols]
+  uint16_t* k_dom;          // [head slots][T][cols]
   int64_t stride_tok, stride_head;
-  int32_t T, Hkv, d, n_dom, cols;
+  int32_t T, n_listed, d, n_dom, cols;
+  uint8_t heads[kMaxHeads]; // KV heads the cache stores
+  uint8_t slot[kMaxHeads];  // their head slots (in K and in k_dom)
 };
 
 __global__ void __launch_bounds__(256) pack_dominant_kernel(const PackParams p) {
   const int C = p.d >> 1;
-  const int64_t n_rows = (int64_t)p.Hkv * p.T;
+  const int64_t n_rows = (int64_t)p.n_listed * p.T;
   const int64_t total = n_rows * p.cols;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
     const int j = (int)(e % p.cols);
     const int64_t row = e / p.cols;
-    const int g = (int)(row / p.T);
+    const int g = p.heads[row / p.T];
+    const int s = p.slot[g];
     const int64_t t = row % p.T;
     uint16_t val = 0;
     if (j < 2 * p.n_dom) {
@@ -207,10 +222,10 @@ __global__ void __launch_bounds__(256) pack_dominant_kernel(const PackParams p) 
         record_error(kCheckChunk, g, j, c);
       } else {
         const int dim = j < p.n_dom ? c : c + C;
-        val = p.k[t * p.stride_tok + (int64_t)g * p.stride_head + dim];
+        val = p.k[t * p.stride_tok + (int64_t)s * p.stride_head + dim];
       }
     }
-    p.k_dom[e] = val;
+    p.k_dom[((int64_t)s * p.T + t) * p.cols + j] = val;
   }
 }
 

@@ -31,11 +31,13 @@ constexpr int kSelU = 8;            // row loads in flight per lane in the strea
 struct SelectParams {
   const float* scores;            // [Hkv][T]
   const int32_t* offsets;         // [B + 1]
+  const int32_t* lengths;         // [B] or null (sequences fill their regions)
   const int32_t* n_fac_per_seq;   // [B] or null
   int32_t* idx;                   // [B][Hkv][cap]
   int32_t* count;                 // [B][Hkv]
   int32_t T, Hkv, n_fac, cap;
   uint8_t heads[kMaxHeads];       // KV head of blockIdx.x
+  uint8_t slot[kMaxHeads];        // head slots of the cache (the scores are indexed by KV head)
 };
 
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectParams p) {
@@ -48,8 +50,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const SelectPa
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.y;
   const int g = p.heads[blockIdx.x];
-  const int off = p.offsets[b];
-  const int L = p.offsets[b + 1] - off;
+  int off;
+  const int L = seq_length(p.offsets, p.lengths, b, false, &off);
   int nf = p.n_fac_per_seq ? p.n_fac_per_seq[b] : p.n_fac;
   if (nf > p.cap) {
     if (tid == 0) record_error(kCheckCount, b, nf, p.cap);

@@ -116,3 +116,99 @@ class SharedIndexStep:
         self.index(q_index)
         B.shared_index_decode(q_layers, self.kv, self.idx, self.count, self.topk, self.scale, self.out, self.ws)
         return self.out
+
+
+class AppendDecodeStep:
+    """Decode steps that first append their token (``aoh_kv_append``), then attend.
+
+    The AoH deployment of the head roles: SPARSE and DENSE KV heads keep their whole
+    history in a linear cache with a fixed capacity per sequence; STREAM heads keep only
+    a ring of ``sink + window`` slots per sequence.  Each cache holds only its own heads
+    (head slots), so a streaming head costs sink + window rows, not its sequence length.
+    ``lengths`` (device int32 [B]) is the one position counter both caches share.
+
+    One call: rotate the new q and k to position lengths[b], write the K / V rows (and the
+    packed dominant row of each linear-cache head), lengths += 1; then the SPARSE heads'
+    importance scan / top-N_fac / focused attention and the DENSE heads' full attention on
+    the linear cache, and the STREAM heads' sink + window attention on the ring.  The
+    query attends over positions 0 .. p, its own token included.
+    """
+
+    def __init__(self, batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, theta: float,
+                 roles: Sequence[int], capacity: Sequence[int], sink: int, window: int, scale: float,
+                 idom: Optional[torch.Tensor] = None, n_fac: int = 0, device="cuda"):
+        self.dev = torch.device(device)
+        self.B, self.Hq, self.Hkv, self.d = batch, n_q_heads, n_kv_heads, head_dim
+        self.theta, self.scale = float(theta), float(scale)
+        self.roles = [int(r) for r in roles]
+        self.sink, self.window = int(sink), int(window)
+        self.idom = idom
+        self.n_dom = 0 if idom is None else idom.shape[1]
+        self.n_fac = int(n_fac)
+        lin = [g for g in range(n_kv_heads) if self.roles[g] != B.ROLE_STREAM]
+        rng = [g for g in range(n_kv_heads) if self.roles[g] == B.ROLE_STREAM]
+        self.lin_slot = [lin.index(g) if g in lin else B.NO_SLOT for g in range(n_kv_heads)]
+        self.ring_slot = [rng.index(g) if g in rng else B.NO_SLOT for g in range(n_kv_heads)]
+        self.has_sparse = any(r == B.ROLE_SPARSE for r in self.roles)
+        self.has_dense = any(r == B.ROLE_DENSE for r in self.roles)
+        self.has_stream = bool(rng)
+        cap = [int(c) for c in capacity]
+        assert len(cap) == batch
+        self.capacity = cap
+        offs = [0]
+        for c in cap:
+            offs.append(offs[-1] + c)
+        self.offsets = torch.tensor(offs, dtype=torch.int32, device=self.dev)
+        self.lengths = torch.zeros(batch, dtype=torch.int32, device=self.dev)
+        T, max_len = offs[-1], max(cap) if cap else 0
+        self.k = torch.zeros((max(T, 1), max(len(lin), 1), head_dim), dtype=torch.bfloat16, device=self.dev)
+        self.v = torch.zeros_like(self.k)
+        self.k_dom = None
+        if self.has_sparse:
+            assert idom is not None and idom.shape[0] == n_kv_heads
+            self.k_dom = torch.zeros((max(len(lin), 1), max(T, 1), B.k_dom_cols(self.n_dom)), dtype=torch.bfloat16,
+                                     device=self.dev)
+        self.kv = None
+        if lin:
+            self.kv = B.make_kv(self.k, self.v, self.offsets, max_len, T, self.k_dom, self.lengths, self.lin_slot,
+                                n_kv_heads)
+        self.ring = None
+        if rng:
+            slots = self.sink + self.window
+            self.ring_offsets = torch.arange(0, (batch + 1) * slots, slots, dtype=torch.int32, device=self.dev)
+            self.rk = torch.zeros((max(batch * slots, 1), len(rng), head_dim), dtype=torch.bfloat16, device=self.dev)
+            self.rv = torch.zeros_like(self.rk)
+            self.ring = B.make_kv(self.rk, self.rv, self.ring_offsets, max_len, batch * slots, None, self.lengths,
+                                  self.ring_slot, n_kv_heads, ring=(self.sink, self.window))
+        self.q_rot = torch.zeros((batch, n_q_heads, head_dim), dtype=torch.bfloat16, device=self.dev)
+        self.out = torch.zeros((batch, n_q_heads, head_dim), dtype=torch.float32, device=self.dev)
+        self.idx = self.count = self.ws_sparse = self.ws_dense = self.ws_ring = None
+        if self.has_sparse:
+            self.idx = torch.empty((batch, n_kv_heads, max(self.n_fac, 1)), dtype=torch.int32, device=self.dev)
+            self.count = torch.empty((batch, n_kv_heads), dtype=torch.int32, device=self.dev)
+            self.ws_sparse = B.workspace(B.sparse_decode_workspace_size(self.kv, n_q_heads, max(self.n_fac, 1)),
+                                         self.dev)
+        if self.has_dense:
+            self.ws_dense = B.workspace(B.stream_decode_workspace_size(self.kv, n_q_heads, self.roles, 0, 0), self.dev)
+        if self.has_stream:
+            self.ws_ring = B.workspace(B.stream_decode_workspace_size(self.ring, n_q_heads, self.roles, self.sink,
+                                                                      self.window), self.dev)
+
+    def append(self, q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor) -> None:
+        B.kv_append(q_new, k_new, v_new, self.theta, self.kv, self.ring, self.idom, self.n_dom, self.lengths,
+                    self.q_rot)
+
+    def decode(self) -> torch.Tensor:
+        if self.has_sparse:
+            B.sparse_decode(self.q_rot, self.kv, self.idom, self.n_dom, self.n_fac, None, max(self.n_fac, 1),
+                            self.roles, self.scale, self.out, self.ws_sparse, self.idx, self.count)
+        if self.has_dense:
+            B.stream_decode(self.q_rot, self.kv, self.roles, 0, 0, self.scale, self.out, self.ws_dense)
+        if self.has_stream:
+            B.stream_decode(self.q_rot, self.ring, self.roles, self.sink, self.window, self.scale, self.out,
+                            self.ws_ring)
+        return self.out
+
+    def __call__(self, q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor) -> torch.Tensor:
+        self.append(q_new, k_new, v_new)
+        return self.decode()

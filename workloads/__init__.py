@@ -17,4 +17,5 @@ from .synth import (  # noqa: F401
     preset,
     make_workload,
     rope_rotate_f32,
+    token_draws,
 )

@@ -341,3 +341,21 @@ def make_workload(spec: WorkloadSpec, threads: Optional[int] = None) -> Workload
         scale=1.0 / math.sqrt(d),
         planted=planted,
     )
+
+
+# --------------------------------------------------------------------------------------
+# decoded tokens (appended one step at a time): raw rows, before any rotation
+# --------------------------------------------------------------------------------------
+
+_TAG_STEP = 10
+
+
+def token_draws(seed: int, step: int, batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int):
+    """The new token of every sequence at decode step `step`: bf16 N(0,1) rows of its query
+    [B, Hq, d], key [B, Hkv, d] and value [B, Hkv, d], as a model's projections would give
+    them (before RoPE)."""
+    r = _rng(seed, _TAG_STEP, step)
+    q = r.standard_normal((batch, n_q_heads, head_dim), dtype=np.float32)
+    k = r.standard_normal((batch, n_kv_heads, head_dim), dtype=np.float32)
+    v = r.standard_normal((batch, n_kv_heads, head_dim), dtype=np.float32)
+    return _to_bf16(q), _to_bf16(k), _to_bf16(v)
