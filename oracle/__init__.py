@@ -6,6 +6,9 @@ reference legs may import it; the product path never does.
 """
 
 from .reference import (  # noqa: F401
+    ROLE_SPARSE,
+    ROLE_DENSE,
+    ROLE_STREAM,
     rope,
     dominant_dims,
     tip_scores,
@@ -24,5 +27,13 @@ from .reference import (  # noqa: F401
     bf16_bits_to_f64,
     append_token_rows,
     pack_dominant_row,
+    head_rows,
+    qk_kernel,
+    proxy_matrix,
+    proxy_singular_values,
+    effective_rank,
+    head_effective_ranks,
+    group_effective_ranks,
+    classify_heads,
     tie_band_check,
 )

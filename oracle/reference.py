@@ -279,6 +279,80 @@ def pack_dominant_row(k_row: np.ndarray, idom: Sequence[int], cols: int) -> np.n
 
 
 # --------------------------------------------------------------------------------------
+# AoH head classifier (AoH summary, Metodología §1-§4): the effective rank of every head's
+# frozen query-key kernel, computed from its d_head x d_head proxy, aggregated per GQA
+# group; the lowest become retrieval heads
+# --------------------------------------------------------------------------------------
+
+def head_rows(W: np.ndarray, h: int, head_dim: int) -> np.ndarray:
+    """Head h's block of a projection weight [H * d_head, d_model]: rows h*d_head .. (h+1)*d_head."""
+    return np.asarray(W, dtype=np.float64)[h * head_dim:(h + 1) * head_dim]
+
+
+def qk_kernel(wq: np.ndarray, wk: np.ndarray) -> np.ndarray:
+    """M_h = W_K^T W_Q (d_model x d_model) for head blocks wq, wk [d_head, d_model] (§1)."""
+    return np.asarray(wk, dtype=np.float64).T @ np.asarray(wq, dtype=np.float64)
+
+
+def proxy_matrix(wq: np.ndarray, wk: np.ndarray) -> np.ndarray:
+    """C_h = (W_Q W_Q^T)(W_K W_K^T), d_head x d_head (§3)."""
+    wq = np.asarray(wq, dtype=np.float64)
+    wk = np.asarray(wk, dtype=np.float64)
+    return (wq @ wq.T) @ (wk @ wk.T)
+
+
+def proxy_singular_values(wq: np.ndarray, wk: np.ndarray) -> np.ndarray:
+    """Singular values of M_h from the proxy (§3, Sylvester): sigma_k = sqrt(eig_k(C_h)).
+
+    C_h is a product of two positive semi-definite matrices, so its eigenvalues are real
+    and non-negative; rounding leaves tiny imaginary parts and negatives, dropped here.
+    Returned in descending order.
+    """
+    lam = np.linalg.eigvals(proxy_matrix(wq, wk)).real
+    return np.sort(np.sqrt(np.maximum(lam, 0.0)))[::-1]
+
+
+def effective_rank(sigma: np.ndarray, rel_zero: float = 1e-12) -> float:
+    """exp of the Shannon entropy of the normalised non-zero singular values (§2).
+
+    sigma_hat_k = sigma_k / sum sigma over the r_h non-zero values (those above
+    rel_zero * max sigma), ER = exp(-sum sigma_hat_k log sigma_hat_k).
+    """
+    s = np.asarray(sigma, dtype=np.float64)
+    if s.size == 0 or s.max() <= 0:
+        return 0.0
+    s = s[s > rel_zero * s.max()]
+    p = s / s.sum()
+    return float(np.exp(-np.sum(p * np.log(p))))
+
+
+def head_effective_ranks(W_Q: np.ndarray, W_K: np.ndarray, n_q_heads: int, n_kv_heads: int,
+                         head_dim: int) -> np.ndarray:
+    """ER of every q head h, whose key block is KV head h // G (GQA): float64 [n_q_heads]."""
+    G = n_q_heads // n_kv_heads
+    return np.array([effective_rank(proxy_singular_values(head_rows(W_Q, h, head_dim),
+                                                          head_rows(W_K, h // G, head_dim)))
+                     for h in range(n_q_heads)])
+
+
+def group_effective_ranks(er_heads: np.ndarray, n_kv_heads: int) -> np.ndarray:
+    """GQA aggregation by the mean (§4): the mean ER of each group's q heads, float64 [n_kv_heads]."""
+    er = np.asarray(er_heads, dtype=np.float64)
+    G = er.shape[0] // n_kv_heads
+    return np.array([er[g * G:(g + 1) * G].mean() for g in range(n_kv_heads)])
+
+
+def classify_heads(er_groups: np.ndarray, n_retrieval: int) -> np.ndarray:
+    """Roles per KV head (§4): the n_retrieval lowest-ER groups are retrieval heads (DENSE,
+    the whole cache), the rest streaming heads (STREAM); equal ER: the lower index first."""
+    er = np.asarray(er_groups, dtype=np.float64)
+    order = np.lexsort((np.arange(er.shape[0]), er))
+    roles = np.full(er.shape[0], ROLE_STREAM, dtype=np.uint8)
+    roles[order[:max(0, int(n_retrieval))]] = ROLE_DENSE
+    return roles
+
+
+# --------------------------------------------------------------------------------------
 # one decode step
 # --------------------------------------------------------------------------------------
 

@@ -9,7 +9,9 @@ c + d/2 term or scores one head of the group; a select that breaks ties toward
 the higher position or returns positions in score order; attention without the
 scale or with keys where values belong; a streaming window one token short; a ring
 slot one place off, bf16 storage by truncation, a token appended one position
-late, dominant columns packed in the wrong half order.
+late, dominant columns packed in the wrong half order; a head classifier that takes
+the proxy's eigenvalues for singular values, a base-2 entropy, the group maximum for
+the mean, or the highest ranks for retrieval heads.
 """
 
 import inspect
@@ -146,6 +148,34 @@ def pack_second_half_first(k_row, idom, cols):
     return out
 
 
+def proxy_eigenvalues_not_roots(wq, wk):
+    lam = np.linalg.eigvals(ref.proxy_matrix(wq, wk)).real
+    return np.sort(np.maximum(lam, 0.0))[::-1]
+
+
+def effective_rank_log2(sigma, rel_zero=1e-12):
+    s = np.asarray(sigma, dtype=np.float64)
+    if s.size == 0 or s.max() <= 0:
+        return 0.0
+    s = s[s > rel_zero * s.max()]
+    p = s / s.sum()
+    return float(np.exp(-np.sum(p * np.log2(p))))
+
+
+def group_max(er_heads, n_kv_heads):
+    er = np.asarray(er_heads, dtype=np.float64)
+    G = er.shape[0] // n_kv_heads
+    return np.array([er[g * G:(g + 1) * G].max() for g in range(n_kv_heads)])
+
+
+def classify_highest(er_groups, n_retrieval):
+    er = np.asarray(er_groups, dtype=np.float64)
+    order = np.lexsort((np.arange(er.shape[0]), -er))
+    roles = np.full(er.shape[0], ref.ROLE_STREAM, dtype=np.uint8)
+    roles[order[:max(0, int(n_retrieval))]] = ref.ROLE_DENSE
+    return roles
+
+
 MUTANTS = {
     "rope_wrong_sense": ("rope", rope_wrong_sense),
     "rope_interleaved_pairs": ("rope", rope_interleaved),
@@ -161,6 +191,10 @@ MUTANTS = {
     "bf16_truncates": ("to_bf16_bits", bf16_truncate),
     "append_one_position_late": ("append_token_rows", append_one_late),
     "pack_second_half_first": ("pack_dominant_row", pack_second_half_first),
+    "proxy_eigenvalues_as_singular_values": ("proxy_singular_values", proxy_eigenvalues_not_roots),
+    "effective_rank_base_two": ("effective_rank", effective_rank_log2),
+    "group_by_max": ("group_effective_ranks", group_max),
+    "retrieval_is_highest_rank": ("classify_heads", classify_highest),
 }
 
 

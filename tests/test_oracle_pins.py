@@ -419,3 +419,78 @@ def test_pack_dominant_row_hand_example():
     k = np.arange(8.0)  # d = 8, chunks 0..3 pair dims (c, c + 4)
     assert oracle.pack_dominant_row(k, [1, 3], 8).tolist() == [1.0, 3.0, 5.0, 7.0, 0, 0, 0, 0]
     assert oracle.pack_dominant_row(k, [0], 2).tolist() == [0.0, 4.0]
+
+
+# ---------------------------------------------------------------------------- head classifier
+
+def test_proxy_gives_the_singular_values_of_the_full_kernel():
+    # Sylvester: the non-zero singular values of M_h = W_K^T W_Q (d_model x d_model) are the
+    # square roots of the eigenvalues of the d_head x d_head proxy; checked against a direct
+    # SVD of M_h, for square, wide and nearly rank-deficient heads
+    rng = np.random.default_rng(21)
+    for d_head, d_model in [(6, 40), (8, 8), (3, 50)]:
+        for scale in (1.0, 1e-3):
+            wq = rng.standard_normal((d_head, d_model))
+            wk = rng.standard_normal((d_head, d_model))
+            wk[-1] = wk[0] + scale * rng.standard_normal(d_model)  # two close rows when scale is small
+            direct = np.linalg.svd(oracle.qk_kernel(wq, wk), compute_uv=False)[:d_head]
+            proxy = oracle.proxy_singular_values(wq, wk)
+            assert np.allclose(proxy, direct, rtol=1e-7, atol=1e-9 * direct[0]), (d_head, d_model, scale)
+            assert oracle.qk_kernel(wq, wk).shape == (d_model, d_model)
+
+
+def test_effective_rank_hand_examples_and_closed_forms():
+    # W_Q = diag(2, 1), W_K = I: M = W_Q, sigma = (2, 1), sigma_hat = (2/3, 1/3)
+    wq, wk = np.diag([2.0, 1.0]), np.eye(2)
+    assert np.allclose(oracle.proxy_singular_values(wq, wk), [2.0, 1.0])
+    er = oracle.effective_rank(oracle.proxy_singular_values(wq, wk))
+    assert er == pytest.approx(math.exp(-(2 / 3) * math.log(2 / 3) - (1 / 3) * math.log(1 / 3)), rel=1e-12)
+    assert er == pytest.approx(1.8898815748423097, rel=1e-12)
+    # one row each: M = k^T q has rank one, sigma = |q| |k| = 5
+    assert np.allclose(oracle.proxy_singular_values(np.array([[3.0, 4.0]]), np.array([[1.0, 0.0]])), [5.0])
+    assert oracle.effective_rank([5.0]) == 1.0
+    # r equal values: ER = r; scale does not matter; zero values are not counted
+    for r in (1, 2, 7, 128):
+        assert oracle.effective_rank(np.full(r, 3.5)) == pytest.approx(r, rel=1e-12)
+    s = np.array([4.0, 2.0, 1.0, 1.0])
+    assert oracle.effective_rank(s) == pytest.approx(oracle.effective_rank(1e6 * s), rel=1e-12)
+    assert oracle.effective_rank(np.array([4.0, 2.0, 0.0, 0.0])) == pytest.approx(oracle.effective_rank([4.0, 2.0]))
+    assert 1.0 < oracle.effective_rank(s) < 4.0
+
+
+def test_effective_rank_is_blind_to_a_shared_rotation_of_the_model_space():
+    # W_Q R and W_K R with R orthogonal (d_model x d_model): M becomes R^T M R, same spectrum
+    rng = np.random.default_rng(22)
+    wq, wk = rng.standard_normal((5, 30)), rng.standard_normal((5, 30))
+    R, _ = np.linalg.qr(rng.standard_normal((30, 30)))
+    a = oracle.effective_rank(oracle.proxy_singular_values(wq, wk))
+    b = oracle.effective_rank(oracle.proxy_singular_values(wq @ R, wk @ R))
+    assert a == pytest.approx(b, rel=1e-10)
+    # a head whose query block is low rank has a concentrated spectrum: lower ER
+    low = rng.standard_normal((5, 2)) @ rng.standard_normal((2, 30))
+    assert oracle.effective_rank(oracle.proxy_singular_values(low, wk)) < a
+
+
+def test_heads_grouped_by_mean_and_lowest_become_retrieval():
+    # two KV groups of two q heads: group 0 = heads 0-1, group 1 = heads 2-3
+    rng = np.random.default_rng(23)
+    d, dm = 4, 24
+    W_Q = rng.standard_normal((4 * d, dm))
+    W_K = rng.standard_normal((2 * d, dm))
+    er = oracle.head_effective_ranks(W_Q, W_K, 4, 2, d)
+    for h in range(4):
+        g = h // 2
+        assert er[h] == pytest.approx(oracle.effective_rank(np.linalg.svd(
+            oracle.qk_kernel(W_Q[h * d:(h + 1) * d], W_K[g * d:(g + 1) * d]), compute_uv=False)[:d]), rel=1e-9)
+    grp = oracle.group_effective_ranks(er, 2)
+    assert grp.tolist() == pytest.approx([(er[0] + er[1]) / 2, (er[2] + er[3]) / 2])
+    assert oracle.group_effective_ranks([1.0, 2.0, 3.0, 6.0, 5.0, 7.0], 2).tolist() == [2.0, 6.0]
+    # brute force: the retrieval set is the n lowest, equal values to the lower index
+    vals = np.array([3.0, 1.0, 2.0, 1.0, 5.0, 2.0])
+    for n in range(0, 7):
+        roles = oracle.classify_heads(vals, n)
+        chosen = sorted(np.flatnonzero(roles == oracle.ROLE_DENSE).tolist())
+        ranked = sorted(range(6), key=lambda g: (vals[g], g))[:n]
+        assert chosen == sorted(ranked), n
+        assert np.all(roles[roles != oracle.ROLE_DENSE] == oracle.ROLE_STREAM)
+    assert oracle.classify_heads(vals, 2).tolist() == [2, 1, 2, 1, 2, 2]
