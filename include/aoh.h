@@ -150,7 +150,11 @@ typedef enum {
   AOH_KERNEL_FLASH_GATHER = 3,  /* split-K gather / window attention                 */
   AOH_KERNEL_PACK_DOMINANT = 4, /* dominant-column packing of K                      */
   AOH_KERNEL_KV_APPEND = 5,     /* rotation and append of a decoded token            */
-  AOH_KERNEL_KINDS = 6
+  AOH_KERNEL_GRAM = 6,          /* head classifier: W W^T of every head (tensor cores) */
+  AOH_KERNEL_GRAM_REDUCE = 7,   /* head classifier: fp64 sum of the split partials   */
+  AOH_KERNEL_SPECTRUM = 8,      /* head classifier: Cholesky, congruence, Jacobi, ER */
+  AOH_KERNEL_GROUP_ROLES = 9,   /* head classifier: group means and roles            */
+  AOH_KERNEL_KINDS = 10
 } aoh_kernel_kind;
 
 /*
@@ -184,7 +188,8 @@ void aoh_record_launch_events(void** events, int32_t* kinds, int32_t n);
  * outside [0, L_b) or offsets past the cache, 2 a count or per-sequence
  * N_fac above the capacity, 3 a chunk id outside [0, d/2), 4 a sequence
  * length or appended position past its region's capacity (or a ring region
- * smaller than its slots).
+ * smaller than its slots), 5 a key Gram matrix without a Cholesky factor
+ * (aoh_head_classify: a key block without full row rank).
  */
 aoh_status aoh_device_check(void* stream, int32_t* detail);
 
@@ -398,6 +403,40 @@ aoh_status aoh_kv_append(const void* q_new, int32_t n_q_heads, const void* k_new
                          double theta, const aoh_kv_cache* kv, const aoh_kv_cache* ring,
                          const int32_t* idom, int32_t n_dom, int32_t* lengths, void* q_out,
                          void* stream);
+
+/*
+ * aoh_head_classify -- the AoH offline head classifier on frozen projection
+ * weights (AoH summary, Metodologia sections 1-4).  For q head h, whose keys
+ * are KV head g = h / G, with W^h its d_head x d_model block of rows:
+ *   M_h = W_K^g^T W_Q^h (section 1); its non-zero singular values are the
+ *   square roots of the eigenvalues of C_h = (W_Q^h W_Q^h^T)(W_K^g W_K^g^T)
+ *   (section 3); ER(h) = exp(-sum sigma_hat log sigma_hat) with sigma_hat =
+ *   sigma / sum sigma over the values above 1e-12 of the largest (section 2);
+ *   the group's ER is the mean over its q heads (GQA aggregation, section 4)
+ *   and the n_retrieval lowest groups are retrieval heads (AOH_ROLE_DENSE),
+ *   the rest streaming heads (AOH_ROLE_STREAM); equal ER: lower KV head first.
+ * The Gram matrices run on tensor cores (bf16 products, fp32 sums of at most
+ * 512 terms, summed over d_model in fp64); the spectrum is computed in fp64
+ * (Cholesky of the key Gram B = L L^T, S = L^T A L whose eigenvalues are
+ * those of C_h, cyclic Jacobi).  An offline step: run once per model.
+ *   w_q        device bf16 [n_q_heads * head_dim][d_model], row-major (the
+ *              q projection weight, one head's block of rows after another)
+ *   w_k        device bf16 [n_kv_heads * head_dim][d_model], row-major
+ *   d_model    multiple of 64, >= head_dim; head_dim 64 or 128
+ *   n_retrieval  0 .. n_kv_heads
+ *   er_heads   device float64 [n_q_heads]; er_groups device float64 [n_kv_heads]
+ *   roles      device uint8 [n_kv_heads]: AOH_ROLE_DENSE or AOH_ROLE_STREAM
+ *   workspace  device, 256-byte aligned, >= aoh_head_classify_workspace_size
+ * A key block without full row rank has no Cholesky factor: the ER of its
+ * q heads is NaN and device check 5 is recorded.
+ */
+aoh_status aoh_head_classify(const void* w_q, const void* w_k, int32_t d_model, int32_t n_q_heads,
+                             int32_t n_kv_heads, int32_t head_dim, int32_t n_retrieval,
+                             double* er_heads, double* er_groups, uint8_t* roles, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+size_t aoh_head_classify_workspace_size(int32_t d_model, int32_t n_q_heads, int32_t n_kv_heads,
+                                        int32_t head_dim);
 
 #ifdef __cplusplus
 }

@@ -197,3 +197,29 @@ def test_ring_and_append_rules_are_checked_on_the_host(lib):
                None) == INVALID                       # k_dom without I_dom
     assert app(None, 0, 0x50000, 0x58000, 5e5, ctypes.byref(fake_kv(batch=0)), None, None, 0, None, None,
                None) == 0                             # empty batch: nothing to do
+
+
+def test_head_classifier_arguments_are_checked_on_the_host(lib):
+    INVALID, UNSUP, ALIGN, WS = 1, 2, 3, 4
+    cls = lib.aoh_head_classify
+    ok = dict(wq=0x10000, wk=0x20000, dm=4096, hq=32, hkv=8, d=128, nr=4, eh=0x30000, eg=0x38000, r=0x40000,
+              ws=0x50000, wsb=1 << 40)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return cls(a["wq"], a["wk"], a["dm"], a["hq"], a["hkv"], a["d"], a["nr"], a["eh"], a["eg"], a["r"], a["ws"],
+                   a["wsb"], None)
+
+    assert call(d=96) == UNSUP
+    assert call(hq=30) == INVALID            # q heads not a multiple of the KV heads
+    assert call(dm=4000) == INVALID          # d_model not a multiple of 64
+    assert call(dm=64) == INVALID            # d_model below head_dim
+    assert call(nr=9) == INVALID and call(nr=-1) == INVALID
+    assert call(wq=0x10008) == ALIGN
+    assert call(eh=None) == INVALID
+    assert call(ws=None) == WS and call(wsb=1000) == WS
+    size = lib.aoh_head_classify_workspace_size
+    need = size(4096, 32, 8, 128)
+    # fp32 partials of 8 splits of 512 columns, fp64 Gram matrices of 40 heads, fp64 scratch of 32
+    assert need == 40 * 8 * 128 * 128 * 4 + 40 * 128 * 128 * 8 + 32 * 128 * 128 * 8
+    assert size(4096, 30, 8, 128) == 0 and size(192, 4, 2, 64) > 0

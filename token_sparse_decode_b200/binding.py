@@ -26,13 +26,15 @@ EXPORTS = (
     "aoh_topk_select", "aoh_sparse_decode", "aoh_sparse_decode_workspace_size", "aoh_stream_decode",
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
     "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
-    "aoh_launch_counts", "aoh_record_launch_events", "aoh_kv_append",
+    "aoh_launch_counts", "aoh_record_launch_events", "aoh_kv_append", "aoh_head_classify",
+    "aoh_head_classify_workspace_size",
 )
 NO_SLOT = 255  # head_slot entry of a KV head a cache does not store
 
 # aoh_kernel_kind order
 KERNELS = ("tip_score_kernel", "topk_select_kernel", "sparse_row_kernel", "flash_gather_kernel",
-           "pack_dominant_kernel", "kv_append_kernel")
+           "pack_dominant_kernel", "kv_append_kernel", "gram_kernel", "gram_reduce_kernel", "spectrum_kernel",
+           "group_roles_kernel")
 
 
 class AohError(RuntimeError):
@@ -88,6 +90,8 @@ def lib() -> ctypes.CDLL:
             "aoh_shared_index_step_workspace_size": (SZ, [KVP, I32, I32, I32]),
             "aoh_stream_decode_noalloc": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P]),
             "aoh_kv_append": (ctypes.c_int, [P, I32, P, P, ctypes.c_double, KVP, KVP, P, I32, P, P, P]),
+            "aoh_head_classify": (ctypes.c_int, [P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
+            "aoh_head_classify_workspace_size": (SZ, [I32, I32, I32, I32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -303,3 +307,18 @@ def kv_append(q_new: Optional[torch.Tensor], k_new: torch.Tensor, v_new: torch.T
         _ptr(q_new), 0 if q_new is None else q_new.shape[-2], _ptr(k_new), _ptr(v_new), float(theta),
         None if kv is None else ctypes.byref(kv), None if ring is None else ctypes.byref(ring), _ptr(idom),
         int(n_dom), _ptr(lengths), _ptr(q_out), _stream(stream)))
+
+
+def head_classify_workspace_size(d_model: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
+    return int(lib().aoh_head_classify_workspace_size(d_model, n_q_heads, n_kv_heads, head_dim))
+
+
+def head_classify(w_q: torch.Tensor, w_k: torch.Tensor, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                  n_retrieval: int, er_heads: torch.Tensor, er_groups: torch.Tensor, roles: torch.Tensor,
+                  ws: torch.Tensor, stream=None) -> None:
+    """AoH head classification from bf16 projection weights w_q [Hq*d, d_model], w_k [Hkv*d, d_model]."""
+    assert w_q.dtype == torch.bfloat16 and w_k.dtype == torch.bfloat16 and w_q.is_contiguous() and w_k.is_contiguous()
+    assert er_heads.dtype == torch.float64 and er_groups.dtype == torch.float64 and roles.dtype == torch.uint8
+    _check("aoh_head_classify", lib().aoh_head_classify(
+        _ptr(w_q), _ptr(w_k), w_q.shape[1], n_q_heads, n_kv_heads, head_dim, n_retrieval, _ptr(er_heads),
+        _ptr(er_groups), _ptr(roles), _ptr(ws), ws.numel(), _stream(stream)))

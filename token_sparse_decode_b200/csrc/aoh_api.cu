@@ -13,6 +13,7 @@
 #include "aoh.h"
 #include "device_common.cuh"
 #include "flash_gather.cuh"
+#include "head_classify.cuh"
 #include "kv_append.cuh"
 #include "sparse_row.cuh"
 #include "tip_score.cuh"
@@ -1120,6 +1121,119 @@ aoh_status aoh_kv_append(const void* q_new, int32_t n_q_heads, const void* k_new
 }
 
 }  // extern "C"
+
+// ===================================================================== AoH head classifier
+namespace {
+
+struct ClassifyGeom {
+  int splits, k_per_split;
+  size_t partial_bytes, gram_bytes, work_bytes;
+};
+
+// d_model split into CTAs of at most 512 columns (a multiple of 64 that divides d_model)
+ClassifyGeom classify_geom(int32_t d_model, int32_t Hq, int32_t Hkv, int32_t D) {
+  ClassifyGeom g{};
+  int kps = 512;
+  while (kps > 64 && d_model % kps) kps -= 64;
+  g.k_per_split = kps;
+  g.splits = d_model / kps;
+  const size_t heads = (size_t)Hq + Hkv, dd = (size_t)D * D;
+  g.partial_bytes = align256(heads * g.splits * dd * sizeof(float));
+  g.gram_bytes = align256(heads * dd * sizeof(double));
+  g.work_bytes = align256((size_t)Hq * dd * sizeof(double));
+  return g;
+}
+
+aoh_status check_classify(int32_t d_model, int32_t Hq, int32_t Hkv, int32_t D, int32_t n_retrieval) {
+  if (D != 64 && D != 128) return AOH_ERR_UNSUPPORTED;
+  if (Hkv < 1 || Hkv > kMaxHeads || Hq < 1 || Hq % Hkv) return AOH_ERR_INVALID_ARG;
+  if (d_model < D || d_model % 64) return AOH_ERR_INVALID_ARG;
+  if (n_retrieval < 0 || n_retrieval > Hkv) return AOH_ERR_INVALID_ARG;
+  return AOH_OK;
+}
+
+template <int D>
+aoh_status launch_classify(const void* w_q, const void* w_k, int32_t d_model, int32_t Hq, int32_t Hkv,
+                           int32_t n_retrieval, double* er_heads, double* er_groups, uint8_t* roles, uint8_t* ws,
+                           const ClassifyGeom& geo, cudaStream_t st) {
+  static std::atomic<uint64_t> configured{0};
+  const size_t gram_smem = size_t(kGramStages) * D * kGramPitch * 2;
+  const size_t spec_smem = (size_t(D) * (D + 1) + size_t(D) * 8) * sizeof(double);
+  if (!set_up_on_this_device(configured)) {
+    aoh_status s = set_smem(gram_kernel<D>, gram_smem);
+    if (s != AOH_OK) return s;
+    if ((s = set_smem(spectrum_kernel<D>, spec_smem)) != AOH_OK) return s;
+    mark_set_up(configured);
+  }
+  float* partial = reinterpret_cast<float*>(ws);
+  double* gram = reinterpret_cast<double*>(ws + geo.partial_bytes);
+  double* work = reinterpret_cast<double*>(ws + geo.partial_bytes + geo.gram_bytes);
+  GramParams gp{};
+  gp.wq = static_cast<const uint16_t*>(w_q);
+  gp.wk = static_cast<const uint16_t*>(w_k);
+  gp.partial = partial;
+  gp.d_model = d_model;
+  gp.Hq = Hq;
+  gp.Hkv = Hkv;
+  gp.splits = geo.splits;
+  gp.k_per_split = geo.k_per_split;
+  before_launch(st);
+  gram_kernel<D><<<dim3(geo.splits, Hq + Hkv), kGramThreads, gram_smem, st>>>(gp);
+  aoh_status s = count_launch(AOH_KERNEL_GRAM, st);
+  if (s != AOH_OK) return s;
+  const int64_t n = int64_t(Hq + Hkv) * D * D;
+  before_launch(st);
+  gram_reduce_kernel<<<(unsigned)std::min<int64_t>(ceil_div(n, 256), int64_t(sm_count()) * 8), 256, 0, st>>>(
+      partial, gram, Hq + Hkv, geo.splits, D * D);
+  if ((s = count_launch(AOH_KERNEL_GRAM_REDUCE, st)) != AOH_OK) return s;
+  SpectrumParams sp{};
+  sp.gram = gram;
+  sp.work = work;
+  sp.er_heads = er_heads;
+  sp.Hq = Hq;
+  sp.Hkv = Hkv;
+  sp.G = Hq / Hkv;
+  before_launch(st);
+  spectrum_kernel<D><<<Hq, kSpecThreads, spec_smem, st>>>(sp);
+  if ((s = count_launch(AOH_KERNEL_SPECTRUM, st)) != AOH_OK) return s;
+  RolesParams rp{};
+  rp.er_heads = er_heads;
+  rp.er_groups = er_groups;
+  rp.roles = roles;
+  rp.Hkv = Hkv;
+  rp.G = Hq / Hkv;
+  rp.n_retrieval = n_retrieval;
+  before_launch(st);
+  group_roles_kernel<<<1, 128, 0, st>>>(rp);
+  return count_launch(AOH_KERNEL_GROUP_ROLES, st);
+}
+
+}  // namespace
+
+extern "C" size_t aoh_head_classify_workspace_size(int32_t d_model, int32_t n_q_heads, int32_t n_kv_heads,
+                                                  int32_t head_dim) {
+  if (check_classify(d_model, n_q_heads, n_kv_heads, head_dim, 0) != AOH_OK) return 0;
+  const ClassifyGeom g = classify_geom(d_model, n_q_heads, n_kv_heads, head_dim);
+  return g.partial_bytes + g.gram_bytes + g.work_bytes;
+}
+
+extern "C" aoh_status aoh_head_classify(const void* w_q, const void* w_k, int32_t d_model, int32_t n_q_heads,
+                                        int32_t n_kv_heads, int32_t head_dim, int32_t n_retrieval, double* er_heads,
+                                        double* er_groups, uint8_t* roles, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  aoh_status s = check_classify(d_model, n_q_heads, n_kv_heads, head_dim, n_retrieval);
+  if (s != AOH_OK) return s;
+  if (!w_q || !w_k || !er_heads || !er_groups || !roles) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(w_q) || !aligned16(w_k)) return AOH_ERR_ALIGNMENT;
+  const ClassifyGeom geo = classify_geom(d_model, n_q_heads, n_kv_heads, head_dim);
+  if (!ws_ok(workspace, workspace_bytes, geo.partial_bytes + geo.gram_bytes + geo.work_bytes)) return AOH_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (head_dim == 128)
+    return launch_classify<128>(w_q, w_k, d_model, n_q_heads, n_kv_heads, n_retrieval, er_heads, er_groups, roles, ws,
+                                geo, as_stream(stream));
+  return launch_classify<64>(w_q, w_k, d_model, n_q_heads, n_kv_heads, n_retrieval, er_heads, er_groups, roles, ws,
+                             geo, as_stream(stream));
+}
 
 // ===================================================================== no-allocation variant
 // Scratch for aoh_stream_decode_noalloc: a file-scope device array, so the call needs no

@@ -18,4 +18,7 @@ from .synth import (  # noqa: F401
     make_workload,
     rope_rotate_f32,
     token_draws,
+    HeadWeightSpec,
+    HEAD_WEIGHT_PRESETS,
+    head_weights,
 )

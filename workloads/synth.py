@@ -359,3 +359,63 @@ def token_draws(seed: int, step: int, batch: int, n_q_heads: int, n_kv_heads: in
     k = r.standard_normal((batch, n_kv_heads, head_dim), dtype=np.float32)
     v = r.standard_normal((batch, n_kv_heads, head_dim), dtype=np.float32)
     return _to_bf16(q), _to_bf16(k), _to_bf16(v)
+
+
+# --------------------------------------------------------------------------------------
+# frozen projection weights for the head classifier (no trained checkpoint is used)
+# --------------------------------------------------------------------------------------
+
+_TAG_WQ, _TAG_WK, _TAG_BASIS, _TAG_RANKS = 11, 12, 13, 14
+
+
+@dataclass(frozen=True)
+class HeadWeightSpec:
+    """Shape and recipe of synthetic q / k projection weights.
+
+    Every KV group g gets a rank r_g (drawn from `ranks` by a seeded permutation; 0 means
+    none): its key block and each of its q heads' blocks are `strength` times a rank-r_g
+    product P R_g (P per head, R_g shared by the group, both N(0, 1)) plus unit N(0, 1)
+    noise, all scaled by 1/sqrt(d_model) and rounded to bf16.  A small r_g concentrates
+    the group's query-key spectrum; r_g = 0 leaves it as diffuse as noise.
+    """
+
+    name: str
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    d_model: int
+    ranks: Tuple[int, ...]
+    strength: float = 3.0
+    n_retrieval: int = 0
+    seed: int = 1
+
+
+HEAD_WEIGHT_PRESETS = {
+    # Llama-3-8B-shaped attention projections: 32 q / 8 KV heads of 128, d_model 4096; half the
+    # KV groups retrieval heads (the pages' 50 % sparsity)
+    "llama8b_heads": HeadWeightSpec(name="llama8b_heads", n_q_heads=32, n_kv_heads=8, head_dim=128, d_model=4096,
+                                    ranks=(2, 4, 8, 16, 0, 0, 0, 0), n_retrieval=4, seed=606),
+    # a small model: 8 q / 4 KV heads of 64, d_model 512
+    "small_heads_d64": HeadWeightSpec(name="small_heads_d64", n_q_heads=8, n_kv_heads=4, head_dim=64, d_model=512,
+                                      ranks=(3, 0, 12, 0), n_retrieval=2, seed=607),
+}
+
+
+def head_weights(spec: HeadWeightSpec):
+    """(W_Q bf16 [Hq*d, d_model], W_K bf16 [Hkv*d, d_model], group ranks int64 [Hkv])."""
+    Hq, Hkv, d, dm = spec.n_q_heads, spec.n_kv_heads, spec.head_dim, spec.d_model
+    G = Hq // Hkv
+    ranks = np.asarray(spec.ranks, dtype=np.int64)[_rng(spec.seed, _TAG_RANKS).permutation(Hkv)]
+    scale = np.float32(1.0 / math.sqrt(dm))
+
+    def block(tag, idx, g):
+        r = _rng(spec.seed, tag, idx)
+        w = r.standard_normal((d, dm), dtype=np.float32)
+        if ranks[g] > 0:
+            basis = _rng(spec.seed, _TAG_BASIS, g).standard_normal((int(ranks[g]), dm), dtype=np.float32)
+            w += np.float32(spec.strength) * (r.standard_normal((d, int(ranks[g])), dtype=np.float32) @ basis)
+        return w * scale
+
+    wq = np.concatenate([block(_TAG_WQ, h, h // G) for h in range(Hq)])
+    wk = np.concatenate([block(_TAG_WK, g, g) for g in range(Hkv)])
+    return _to_bf16(wq), _to_bf16(wk), ranks
