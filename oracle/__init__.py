@@ -27,6 +27,7 @@ from .reference import (  # noqa: F401
     bf16_bits_to_f64,
     append_token_rows,
     pack_dominant_row,
+    rest_dims,
     head_rows,
     qk_kernel,
     proxy_matrix,

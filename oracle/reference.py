@@ -269,6 +269,13 @@ def append_token_rows(q_raw: np.ndarray, k_raw: np.ndarray, v_raw: np.ndarray, p
     return to_bf16_bits(q), to_bf16_bits(k), to_bf16_bits(np.asarray(v_raw, dtype=np.float64))
 
 
+def rest_dims(idom: Sequence[int], head_dim: int) -> List[int]:
+    """The dims outside the dominant chunks, ascending: what FASA-M (§2.C) moves to host memory
+    together with V, while the dominant components of K stay on the GPU."""
+    dom = set(dominant_dims(idom, head_dim))
+    return [i for i in range(head_dim) if i not in dom]
+
+
 def pack_dominant_row(k_row: np.ndarray, idom: Sequence[int], cols: int) -> np.ndarray:
     """The dominant columns of one key row: dims I_dom, then dims I_dom + d/2, zero-padded to cols."""
     k_row = np.asarray(k_row)

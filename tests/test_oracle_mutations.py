@@ -176,6 +176,10 @@ def classify_highest(er_groups, n_retrieval):
     return roles
 
 
+def rest_dims_drops_last(idom, head_dim):
+    return ref.__wrapped_rest(idom, head_dim)[:-1]
+
+
 MUTANTS = {
     "rope_wrong_sense": ("rope", rope_wrong_sense),
     "rope_interleaved_pairs": ("rope", rope_interleaved),
@@ -195,6 +199,7 @@ MUTANTS = {
     "effective_rank_base_two": ("effective_rank", effective_rank_log2),
     "group_by_max": ("group_effective_ranks", group_max),
     "retrieval_is_highest_rank": ("classify_heads", classify_highest),
+    "rest_dims_drops_one": ("rest_dims", rest_dims_drops_last),
 }
 
 
@@ -225,6 +230,7 @@ def test_mutant_is_caught(mutant, monkeypatch):
     monkeypatch.setattr(ref, "__wrapped_tip", ref.tip_scores, raising=False)
     monkeypatch.setattr(ref, "__wrapped_attend", ref.attend, raising=False)
     monkeypatch.setattr(ref, "__wrapped_append", ref.append_token_rows, raising=False)
+    monkeypatch.setattr(ref, "__wrapped_rest", ref.rest_dims, raising=False)
     monkeypatch.setattr(ref, attr, fn)
     monkeypatch.setattr(oracle, attr, fn)
     failed = run_pins()

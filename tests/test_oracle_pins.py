@@ -494,3 +494,16 @@ def test_heads_grouped_by_mean_and_lowest_become_retrieval():
         assert chosen == sorted(ranked), n
         assert np.all(roles[roles != oracle.ROLE_DENSE] == oracle.ROLE_STREAM)
     assert oracle.classify_heads(vals, 2).tolist() == [2, 1, 2, 1, 2, 2]
+
+
+def test_dominant_and_rest_dims_split_every_key():
+    # FASA-M keeps the dominant components on the GPU and the rest (with V) on the host: the
+    # two sets partition the dims, and a dot product taken part by part is the whole one
+    rng = np.random.default_rng(24)
+    for d, idom in [(8, [1, 3]), (16, [0, 2, 7]), (128, sorted(rng.choice(64, 16, replace=False)))]:
+        dom, rest = oracle.dominant_dims(idom, d), oracle.rest_dims(idom, d)
+        assert sorted(dom + rest) == list(range(d)) and not set(dom) & set(rest)
+        assert rest == sorted(rest)
+        q, k = rng.standard_normal(d), rng.standard_normal(d)
+        assert abs(q[dom] @ k[dom] + q[rest] @ k[rest] - q @ k) < 1e-12
+    assert oracle.rest_dims([1, 3], 8) == [0, 2, 4, 6]
