@@ -154,7 +154,9 @@ typedef enum {
   AOH_KERNEL_GRAM_REDUCE = 7,   /* head classifier: fp64 sum of the split partials   */
   AOH_KERNEL_SPECTRUM = 8,      /* head classifier: Cholesky, congruence, Jacobi, ER */
   AOH_KERNEL_GROUP_ROLES = 9,   /* head classifier: group means and roles            */
-  AOH_KERNEL_KINDS = 10
+  AOH_KERNEL_OFFLOAD_STAGE = 10,  /* host offload: selected rows across the host link */
+  AOH_KERNEL_OFFLOAD_SPLIT = 11,  /* host offload: a device cache split to host parts */
+  AOH_KERNEL_KINDS = 12
 } aoh_kernel_kind;
 
 /*
@@ -437,6 +439,64 @@ aoh_status aoh_head_classify(const void* w_q, const void* w_k, int32_t d_model, 
 
 size_t aoh_head_classify_workspace_size(int32_t d_model, int32_t n_q_heads, int32_t n_kv_heads,
                                         int32_t head_dim);
+
+/*
+ * FASA-M, the memory-saving variant (FASA section 2.C): the value cache and
+ * the non-dominant parts of the keys live in host memory; only the dominant
+ * components of K stay on the GPU.  The importance scan and the top-N_fac
+ * select run on the GPU part; only the selected tokens' rows cross the host
+ * link.  Head-major layouts, token t of KV head g:
+ *   k_dom   device bf16 [n_kv_heads][total_tokens][k_dom_cols]: the packed
+ *           dominant columns of aoh_kv_cache (dims I_dom, then I_dom + d/2)
+ *   k_rest  host bf16 [n_kv_heads][total_tokens][rest_cols]: the other
+ *           d - 2 n_dom dims in ascending order, zero-padded to rest_cols
+ *   v       host bf16 [n_kv_heads][total_tokens][head_dim]
+ * Host buffers must be pinned (page-locked, e.g. cudaHostAlloc) so the GPU can
+ * read them in place; pageable memory is refused (AOH_ERR_INVALID_ARG).
+ * offsets / lengths: as in aoh_kv_cache.  Every KV head is SPARSE here.
+ * I_dom sizes must be multiples of 4 (whole 16-byte dominant segments).
+ */
+typedef struct aoh_offload_cache {
+  const int32_t* offsets;      /* device int32 [batch + 1]                             */
+  const int32_t* lengths;      /* device int32 [batch] or NULL                         */
+  int32_t batch;
+  int32_t n_kv_heads;          /* 1..128                                               */
+  int32_t head_dim;            /* 64 or 128                                            */
+  int32_t max_len;             /* host upper bound of the lengths                      */
+  int64_t total_tokens;        /* host copy of offsets[batch], < 2^31                  */
+  const void* k_dom;           /* device, 16-byte aligned                              */
+  int32_t k_dom_cols;          /* multiple of 8, >= 2 n_dom                            */
+  int32_t rest_cols;           /* multiple of 8, >= head_dim - 2 n_dom, <= head_dim     */
+  const void* k_rest;          /* pinned host, 16-byte aligned                         */
+  const void* v;               /* pinned host, 16-byte aligned                         */
+} aoh_offload_cache;
+
+/*
+ * aoh_offload_split -- write the host parts (k_rest, v) of every head from a
+ * linear device cache `kv` (every head stored), with I_dom of n_dom chunks per
+ * head; rows are written over the host link.  Cache maintenance, not a decode
+ * step.  k_dom is written by aoh_pack_dominant.
+ */
+aoh_status aoh_offload_split(const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom,
+                             void* k_rest, int32_t rest_cols, void* v, void* stream);
+
+/*
+ * aoh_offload_decode -- aoh_sparse_decode on a FASA-M cache: the scan of k_dom
+ * and the select on the GPU, then the K rows (dominant part from k_dom, the
+ * rest from the host) and V rows of the selected tokens are brought across
+ * the link into the workspace, and focused attention runs on them.  The K rows
+ * and q are taken in each head's dominant-first dim order, which leaves every
+ * q.k unchanged.  Arguments as for aoh_sparse_decode (every head SPARSE);
+ * workspace >= aoh_offload_decode_workspace_size, zero-filled before first use.
+ */
+aoh_status aoh_offload_decode(const void* q, int32_t n_q_heads, const aoh_offload_cache* oc,
+                              const int32_t* idom, int32_t n_dom, int32_t n_fac,
+                              const int32_t* n_fac_per_seq, int32_t n_fac_cap, float scale,
+                              float* out, int32_t* idx_out, int32_t* count_out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+size_t aoh_offload_decode_workspace_size(const aoh_offload_cache* oc, int32_t n_q_heads,
+                                         int32_t n_fac_cap);
 
 #ifdef __cplusplus
 }

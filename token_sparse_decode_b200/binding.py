@@ -27,14 +27,14 @@ EXPORTS = (
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
     "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
     "aoh_launch_counts", "aoh_record_launch_events", "aoh_kv_append", "aoh_head_classify",
-    "aoh_head_classify_workspace_size",
+    "aoh_head_classify_workspace_size", "aoh_offload_split", "aoh_offload_decode", "aoh_offload_decode_workspace_size",
 )
 NO_SLOT = 255  # head_slot entry of a KV head a cache does not store
 
 # aoh_kernel_kind order
 KERNELS = ("tip_score_kernel", "topk_select_kernel", "sparse_row_kernel", "flash_gather_kernel",
            "pack_dominant_kernel", "kv_append_kernel", "gram_kernel", "gram_reduce_kernel", "spectrum_kernel",
-           "group_roles_kernel")
+           "group_roles_kernel", "offload_stage_kernel", "offload_split_kernel")
 
 
 class AohError(RuntimeError):
@@ -55,6 +55,17 @@ class KVCache(ctypes.Structure):
         ("stride_head", ctypes.c_int64), ("k_dom", ctypes.c_void_p), ("k_dom_cols", ctypes.c_int32),
         ("lengths", ctypes.c_void_p), ("head_slot", ctypes.c_void_p), ("ring_sink", ctypes.c_int32),
         ("ring_window", ctypes.c_int32),
+    ]
+
+
+class OffloadCache(ctypes.Structure):
+    """Mirror of ``aoh_offload_cache`` (include/aoh.h)."""
+
+    _fields_ = [
+        ("offsets", ctypes.c_void_p), ("lengths", ctypes.c_void_p), ("batch", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("max_len", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int64), ("k_dom", ctypes.c_void_p), ("k_dom_cols", ctypes.c_int32),
+        ("rest_cols", ctypes.c_int32), ("k_rest", ctypes.c_void_p), ("v", ctypes.c_void_p),
     ]
 
 
@@ -92,6 +103,10 @@ def lib() -> ctypes.CDLL:
             "aoh_kv_append": (ctypes.c_int, [P, I32, P, P, ctypes.c_double, KVP, KVP, P, I32, P, P, P]),
             "aoh_head_classify": (ctypes.c_int, [P, P, I32, I32, I32, I32, I32, P, P, P, P, SZ, P]),
             "aoh_head_classify_workspace_size": (SZ, [I32, I32, I32, I32]),
+            "aoh_offload_split": (ctypes.c_int, [KVP, P, I32, P, I32, P, P]),
+            "aoh_offload_decode": (ctypes.c_int, [P, I32, ctypes.POINTER(OffloadCache), P, I32, I32, P, I32, F32, P, P, P,
+                                                  P, SZ, P]),
+            "aoh_offload_decode_workspace_size": (SZ, [ctypes.POINTER(OffloadCache), I32, I32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -322,3 +337,46 @@ def head_classify(w_q: torch.Tensor, w_k: torch.Tensor, n_q_heads: int, n_kv_hea
     _check("aoh_head_classify", lib().aoh_head_classify(
         _ptr(w_q), _ptr(w_k), w_q.shape[1], n_q_heads, n_kv_heads, head_dim, n_retrieval, _ptr(er_heads),
         _ptr(er_groups), _ptr(roles), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def rest_cols(head_dim: int, n_dom: int) -> int:
+    """Row length of the host copy of the non-dominant key dims: d - 2 n_dom rounded up to 8."""
+    return (head_dim - 2 * n_dom + 7) // 8 * 8
+
+
+def make_offload(offsets: torch.Tensor, max_len: int, total_tokens: int, n_kv_heads: int, head_dim: int,
+                 k_dom: torch.Tensor, k_rest: torch.Tensor, v: torch.Tensor,
+                 lengths: Optional[torch.Tensor] = None) -> OffloadCache:
+    """Describe a FASA-M cache: k_dom on the device, k_rest and v in pinned host memory."""
+    assert k_dom.is_cuda and not k_rest.is_cuda and not v.is_cuda
+    assert k_rest.is_pinned() and v.is_pinned(), "host parts must be pinned"
+    oc = OffloadCache()
+    oc._keep = (offsets, k_dom, k_rest, v, lengths)
+    oc.offsets = offsets.data_ptr()
+    if lengths is not None:
+        oc.lengths = lengths.data_ptr()
+    oc.batch = offsets.numel() - 1
+    oc.n_kv_heads, oc.head_dim, oc.max_len, oc.total_tokens = n_kv_heads, head_dim, int(max_len), int(total_tokens)
+    oc.k_dom, oc.k_dom_cols = k_dom.data_ptr(), k_dom.shape[-1]
+    oc.k_rest, oc.rest_cols = k_rest.data_ptr(), k_rest.shape[-1]
+    oc.v = v.data_ptr()
+    return oc
+
+
+def offload_split(kv: KVCache, idom: torch.Tensor, n_dom: int, k_rest: torch.Tensor, v_host: torch.Tensor,
+                  stream=None) -> None:
+    _check("aoh_offload_split", lib().aoh_offload_split(ctypes.byref(kv), _ptr(idom), n_dom, _ptr(k_rest),
+                                                         k_rest.shape[-1], _ptr(v_host), _stream(stream)))
+
+
+def offload_decode_workspace_size(oc: OffloadCache, n_q_heads: int, n_fac_cap: int) -> int:
+    return int(lib().aoh_offload_decode_workspace_size(ctypes.byref(oc), n_q_heads, n_fac_cap))
+
+
+def offload_decode(q: torch.Tensor, oc: OffloadCache, idom: torch.Tensor, n_dom: int, n_fac: int,
+                   n_fac_per_seq: Optional[torch.Tensor], n_fac_cap: int, scale: float, out: torch.Tensor,
+                   ws: torch.Tensor, idx_out: Optional[torch.Tensor] = None, count_out: Optional[torch.Tensor] = None,
+                   stream=None) -> None:
+    _check("aoh_offload_decode", lib().aoh_offload_decode(
+        _ptr(q), q.shape[-2], ctypes.byref(oc), _ptr(idom), n_dom, n_fac, _ptr(n_fac_per_seq), n_fac_cap,
+        float(scale), _ptr(out), _ptr(idx_out), _ptr(count_out), _ptr(ws), ws.numel(), _stream(stream)))

@@ -15,6 +15,7 @@
 #include "flash_gather.cuh"
 #include "head_classify.cuh"
 #include "kv_append.cuh"
+#include "offload.cuh"
 #include "sparse_row.cuh"
 #include "tip_score.cuh"
 #include "topk_select.cuh"
@@ -1233,6 +1234,226 @@ extern "C" aoh_status aoh_head_classify(const void* w_q, const void* w_k, int32_
                                 geo, as_stream(stream));
   return launch_classify<64>(w_q, w_k, d_model, n_q_heads, n_kv_heads, n_retrieval, er_heads, er_groups, roles, ws,
                              geo, as_stream(stream));
+}
+
+// ===================================================================== FASA-M host offload
+namespace {
+
+// The device-side address of a buffer the GPU can reach (device memory, or pinned host memory
+// mapped into the device's address space); pageable host memory is refused.
+aoh_status device_view(const void* p, const void** out) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return AOH_ERR_INVALID_ARG;
+  }
+  if (a.type == cudaMemoryTypeUnregistered || a.devicePointer == nullptr) return AOH_ERR_INVALID_ARG;
+  *out = a.devicePointer;
+  return AOH_OK;
+}
+
+aoh_status check_offload(const aoh_offload_cache* oc, int32_t n_dom) {
+  if (!oc) return AOH_ERR_INVALID_ARG;
+  if (oc->batch < 0 || oc->n_kv_heads < 1 || oc->n_kv_heads > kMaxHeads) return AOH_ERR_INVALID_ARG;
+  if (oc->head_dim != 64 && oc->head_dim != 128) return AOH_ERR_UNSUPPORTED;
+  if (oc->max_len < 0 || oc->total_tokens < 0 || oc->total_tokens >= (int64_t(1) << 31)) return AOH_ERR_INVALID_ARG;
+  if (n_dom < 1 || n_dom > oc->head_dim / 2) return AOH_ERR_INVALID_ARG;
+  if (n_dom % 4) return AOH_ERR_UNSUPPORTED;  // the dominant part of a row is whole 16-byte segments
+  if (oc->k_dom_cols < 2 * n_dom || oc->k_dom_cols > 128 || oc->k_dom_cols % 8) return AOH_ERR_INVALID_ARG;
+  if (oc->rest_cols < oc->head_dim - 2 * n_dom || oc->rest_cols % 8 || oc->rest_cols > oc->head_dim)
+    return AOH_ERR_INVALID_ARG;
+  if (oc->batch == 0) return AOH_OK;
+  if (!oc->offsets || !oc->k_dom || !oc->k_rest || !oc->v) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(oc->k_dom) || !aligned16(oc->k_rest) || !aligned16(oc->v)) return AOH_ERR_ALIGNMENT;
+  return AOH_OK;
+}
+
+// A cache descriptor over the device part only (the packed dominant columns): what the scan
+// and the select read.  Its k / v point at k_dom as well but are never read.
+aoh_kv_cache offload_device_part(const aoh_offload_cache* oc) {
+  aoh_kv_cache kv{};
+  kv.k = kv.v = oc->k_dom;
+  kv.offsets = oc->offsets;
+  kv.lengths = oc->lengths;
+  kv.batch = oc->batch;
+  kv.n_kv_heads = oc->n_kv_heads;
+  kv.head_dim = oc->head_dim;
+  kv.max_len = oc->max_len;
+  kv.total_tokens = oc->total_tokens;
+  kv.stride_tok = oc->k_dom_cols;
+  kv.stride_head = std::max<int64_t>(oc->total_tokens, 1) * oc->k_dom_cols;
+  kv.k_dom = oc->k_dom;
+  kv.k_dom_cols = oc->k_dom_cols;
+  return kv;
+}
+
+struct OffloadWs {
+  size_t fd, scores, idx, count, sidx, soff, sk, sv, sq, total;
+};
+
+OffloadWs offload_ws(const aoh_offload_cache* oc, int32_t Hq, int32_t cap) {
+  const aoh_kv_cache kv = offload_device_part(oc);
+  OffloadWs w{};
+  const size_t B = (size_t)oc->batch, H = (size_t)oc->n_kv_heads, d = (size_t)oc->head_dim;
+  size_t o = 0;
+  w.fd = o;
+  o += fd_bytes(sparse_geom(&kv, Hq, cap));
+  w.scores = o;
+  o += align256(sizeof(float) * H * (size_t)std::max<int64_t>(oc->total_tokens, 1));
+  w.idx = o;
+  o += align256(sizeof(int32_t) * B * H * cap);
+  w.count = o;
+  o += align256(sizeof(int32_t) * B * H);
+  w.sidx = o;
+  o += align256(sizeof(int32_t) * B * H * cap);
+  w.soff = o;
+  o += align256(sizeof(int32_t) * (B + 1));
+  w.sk = o;
+  o += align256(2 * B * cap * H * d);
+  w.sv = o;
+  o += align256(2 * B * cap * H * d);
+  w.sq = o;
+  o += align256(2 * B * (size_t)Hq * d);
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+
+extern "C" aoh_status aoh_offload_split(const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom, void* k_rest,
+                                        int32_t rest_cols, void* v_host, void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if (is_ring(kv)) return AOH_ERR_INVALID_ARG;
+  if (n_dom < 1 || n_dom > kv->head_dim / 2) return AOH_ERR_INVALID_ARG;
+  if (n_dom % 4) return AOH_ERR_UNSUPPORTED;
+  if (rest_cols < kv->head_dim - 2 * n_dom || rest_cols % 8 || rest_cols > kv->head_dim) return AOH_ERR_INVALID_ARG;
+  for (int g = 0; g < kv->n_kv_heads; ++g)
+    if (slot_of(kv, g) == kNoSlot) return AOH_ERR_INVALID_ARG;  // every head is split
+  if (kv->batch == 0 || kv->total_tokens == 0) return AOH_OK;
+  if (!idom || !k_rest || !v_host) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(k_rest) || !aligned16(v_host)) return AOH_ERR_ALIGNMENT;
+  const void *kr = nullptr, *vh = nullptr;
+  if ((s = device_view(k_rest, &kr)) != AOH_OK) return s;
+  if ((s = device_view(v_host, &vh)) != AOH_OK) return s;
+  SplitParams sp{};
+  sp.k = static_cast<const uint16_t*>(kv->k);
+  sp.v = static_cast<const uint16_t*>(kv->v);
+  sp.stride_tok = kv->stride_tok;
+  sp.stride_head = kv->stride_head;
+  sp.idom = idom;
+  sp.k_rest = static_cast<uint16_t*>(const_cast<void*>(kr));
+  sp.v_host = static_cast<uint16_t*>(const_cast<void*>(vh));
+  sp.T = (int32_t)kv->total_tokens;
+  sp.d = kv->head_dim;
+  sp.n_dom = n_dom;
+  sp.rest_cols = rest_cols;
+  for (int g = 0; g < kv->n_kv_heads; ++g) sp.slot[g] = slot_of(kv, g);
+  const int slabs = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(kv->total_tokens, 64),
+                                                                 ceil_div(int64_t(sm_count()) * 4, kv->n_kv_heads)));
+  cudaStream_t st = as_stream(stream);
+  before_launch(st);
+  offload_split_kernel<<<dim3(slabs, kv->n_kv_heads), kStageThreads, 0, st>>>(sp);
+  return count_launch(AOH_KERNEL_OFFLOAD_SPLIT, st);
+}
+
+extern "C" size_t aoh_offload_decode_workspace_size(const aoh_offload_cache* oc, int32_t n_q_heads,
+                                                   int32_t n_fac_cap) {
+  if (!oc || oc->n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % oc->n_kv_heads || n_fac_cap < 1) return 0;
+  if (oc->head_dim != 64 && oc->head_dim != 128) return 0;
+  if (n_q_heads / oc->n_kv_heads > kMaxQRows) return 0;
+  return offload_ws(oc, n_q_heads, n_fac_cap).total;
+}
+
+extern "C" aoh_status aoh_offload_decode(const void* q, int32_t n_q_heads, const aoh_offload_cache* oc,
+                                         const int32_t* idom, int32_t n_dom, int32_t n_fac,
+                                         const int32_t* n_fac_per_seq, int32_t n_fac_cap, float scale, float* out,
+                                         int32_t* idx_out, int32_t* count_out, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  aoh_status s = check_offload(oc, n_dom);
+  if (s != AOH_OK) return s;
+  if (n_q_heads < 1 || n_q_heads % oc->n_kv_heads) return AOH_ERR_INVALID_ARG;
+  const int G = n_q_heads / oc->n_kv_heads;
+  if (G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (n_fac_cap < 1 || (!n_fac_per_seq && (n_fac < 0 || n_fac > n_fac_cap))) return AOH_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return AOH_ERR_INVALID_ARG;
+  if ((idx_out == nullptr) != (count_out == nullptr)) return AOH_ERR_INVALID_ARG;
+  if (oc->batch == 0) return AOH_OK;
+  if (!q || !idom || !out) return AOH_ERR_INVALID_ARG;
+  if (!aligned16(q)) return AOH_ERR_ALIGNMENT;
+  const OffloadWs wl = offload_ws(oc, n_q_heads, n_fac_cap);
+  if (!ws_ok(workspace, workspace_bytes, wl.total)) return AOH_ERR_WORKSPACE;
+  const void *kr = nullptr, *vh = nullptr;
+  if ((s = device_view(oc->k_rest, &kr)) != AOH_OK) return s;
+  if ((s = device_view(oc->v, &vh)) != AOH_OK) return s;
+  const aoh_kv_cache kv = offload_device_part(oc);
+  uint8_t heads[kMaxHeads];
+  const int Hkv = oc->n_kv_heads, d = oc->head_dim;
+  for (int g = 0; g < Hkv; ++g) heads[g] = (uint8_t)g;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* scores = reinterpret_cast<float*>(ws + wl.scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + wl.idx);
+  int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + wl.count);
+  cudaStream_t st = as_stream(stream);
+  // 1-2. importance scan of the dominant columns (on the GPU) and the top-N_fac select
+  if (kv.total_tokens > 0 && (s = launch_tip(q, n_q_heads, &kv, idom, n_dom, scores, heads, Hkv, st)) != AOH_OK)
+    return s;
+  if ((s = select_stage(scores, &kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, Hkv, st)) != AOH_OK) return s;
+  // 3. the selected rows across the host link, into HBM
+  StageParams sp{};
+  sp.q = static_cast<const uint16_t*>(q);
+  sp.k_dom = static_cast<const uint16_t*>(oc->k_dom);
+  sp.k_rest = static_cast<const uint16_t*>(kr);
+  sp.v_host = static_cast<const uint16_t*>(vh);
+  sp.idom = idom;
+  sp.offsets = oc->offsets;
+  sp.lengths = oc->lengths;
+  sp.idx = idx;
+  sp.count = cnt;
+  sp.sk = reinterpret_cast<uint16_t*>(ws + wl.sk);
+  sp.sv = reinterpret_cast<uint16_t*>(ws + wl.sv);
+  sp.sq = reinterpret_cast<uint16_t*>(ws + wl.sq);
+  sp.sidx = reinterpret_cast<int32_t*>(ws + wl.sidx);
+  sp.soffsets = reinterpret_cast<int32_t*>(ws + wl.soff);
+  sp.T = oc->total_tokens;
+  sp.B = oc->batch;
+  sp.Hq = n_q_heads;
+  sp.Hkv = Hkv;
+  sp.G = G;
+  sp.d = d;
+  sp.n_dom = n_dom;
+  sp.k_dom_cols = oc->k_dom_cols;
+  sp.rest_cols = oc->rest_cols;
+  sp.cap = n_fac_cap;
+  memcpy(sp.heads, heads, Hkv);
+  before_launch(st);
+  offload_stage_kernel<<<dim3(Hkv, oc->batch), kStageThreads, 0, st>>>(sp);
+  if ((s = count_launch(AOH_KERNEL_OFFLOAD_STAGE, st)) != AOH_OK) return s;
+  // 4. focused attention over the staged rows (identity index, dominant-first dim order)
+  const FdGeom geo = sparse_geom(&kv, n_q_heads, n_fac_cap);
+  FdecParams fp{};
+  fp.q = sp.sq;
+  fp.k = sp.sk;
+  fp.v = sp.sv;
+  fp.offsets = sp.soffsets;
+  fp.lengths = nullptr;
+  fp.idx = sp.sidx;
+  fp.count = cnt;
+  fp.out = out;
+  fp.stride_tok = int64_t(Hkv) * d;
+  fp.stride_head = d;
+  fp.B = oc->batch;
+  fp.Hq = n_q_heads;
+  fp.Hkv = Hkv;
+  fp.G = G;
+  fp.NQ = G;
+  fp.cap = n_fac_cap;
+  fp.list_mode = 1;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  memcpy(fp.heads, heads, Hkv);
+  for (int g = 0; g < Hkv; ++g) fp.slot[g] = (uint8_t)g;
+  fd_bind(fp, geo, ws + wl.fd);
+  return launch_fd(fp, d, geo.nqp, Hkv, oc->batch, st, n_fac_per_seq == nullptr);
 }
 
 // ===================================================================== no-allocation variant

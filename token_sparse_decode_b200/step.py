@@ -212,3 +212,48 @@ class AppendDecodeStep:
     def __call__(self, q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor) -> torch.Tensor:
         self.append(q_new, k_new, v_new)
         return self.decode()
+
+
+class OffloadDecodeStep:
+    """FASA-M decode step: V and the non-dominant key dims in pinned host memory.
+
+    Built from a device cache: the dominant columns are packed into device memory
+    (``aoh_pack_dominant``) and the rest of K and all of V are written to pinned host
+    buffers (``aoh_offload_split``); the device K / V are not kept.  A call is one
+    ``aoh_offload_decode``: scan and select on the GPU, the selected rows across the host
+    link, focused attention.  Every KV head is SPARSE.
+    """
+
+    def __init__(self, k: torch.Tensor, v: torch.Tensor, offsets: torch.Tensor, max_len: int, total_tokens: int,
+                 n_q_heads: int, idom: torch.Tensor, scale: float, n_fac: int = 0,
+                 n_fac_per_seq: Optional[torch.Tensor] = None, n_fac_cap: int = 0,
+                 lengths: Optional[torch.Tensor] = None):
+        self.dev = k.device
+        Hkv, d = k.shape[1], k.shape[2]
+        self.idom, self.n_dom = idom, idom.shape[1]
+        self.scale, self.n_fac, self.n_fac_per_seq, self.n_fac_cap = float(scale), int(n_fac), n_fac_per_seq, int(n_fac_cap)
+        kv = B.make_kv(k, v, offsets, max_len, total_tokens, lengths=lengths)
+        self.k_dom = torch.empty((Hkv, max(total_tokens, 1), B.k_dom_cols(self.n_dom)), dtype=torch.bfloat16,
+                                 device=self.dev)
+        B.pack_dominant(kv, idom, self.n_dom, self.k_dom)
+        self.k_rest = torch.empty((Hkv, max(total_tokens, 1), B.rest_cols(d, self.n_dom)), dtype=torch.bfloat16,
+                                  pin_memory=True)
+        self.v_host = torch.empty((Hkv, max(total_tokens, 1), d), dtype=torch.bfloat16, pin_memory=True)
+        B.offload_split(kv, idom, self.n_dom, self.k_rest, self.v_host)
+        torch.cuda.current_stream().synchronize()  # the host parts are complete before k, v may go
+        self.oc = B.make_offload(offsets, max_len, total_tokens, Hkv, d, self.k_dom, self.k_rest, self.v_host, lengths)
+        batch = offsets.numel() - 1
+        self.idx = torch.empty((batch, Hkv, self.n_fac_cap), dtype=torch.int32, device=self.dev)
+        self.count = torch.empty((batch, Hkv), dtype=torch.int32, device=self.dev)
+        self.ws = B.workspace(B.offload_decode_workspace_size(self.oc, n_q_heads, self.n_fac_cap), self.dev)
+        self.out = torch.zeros((batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
+
+    def link_bytes_per_step(self) -> int:
+        """Bytes that cross the host link per step: the selected rows' rest-of-K and V."""
+        n = self.count.to(torch.int64).sum().item()
+        return int(n) * 2 * (self.k_rest.shape[-1] + self.v_host.shape[-1])
+
+    def __call__(self, q: torch.Tensor) -> torch.Tensor:
+        B.offload_decode(q, self.oc, self.idom, self.n_dom, self.n_fac, self.n_fac_per_seq, self.n_fac_cap,
+                         self.scale, self.out, self.ws, self.idx, self.count)
+        return self.out
