@@ -498,6 +498,100 @@ def run_ours(args, rank, world, local_rank):
     }
 
 
+# ------------------------------------------------------------------------------ the other rows of the path
+
+def _event_ms(fn, steps: int, warmup: int) -> float:
+    """Mean device time of fn() over `steps` calls (CUDA events on the current stream)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def measure_append(dev, steps: int = 200, warmup: int = 5) -> dict:
+    """aoh_kv_append for a serving batch: 64 sequences, 32 q / 8 KV heads of 128, AoH split
+    (2 retrieval, 2 sparse, 4 streaming heads with sink 128 + window 4096)."""
+    from token_sparse_decode_b200 import binding as B
+    from token_sparse_decode_b200.step import AppendDecodeStep
+    from workloads import ROLE_DENSE, ROLE_STREAM, token_draws
+
+    Bn, Hq, Hkv, d = 64, 32, 8, 128
+    roles = [ROLE_DENSE, ROLE_SPARSE, ROLE_STREAM, ROLE_STREAM, ROLE_DENSE, ROLE_SPARSE, ROLE_STREAM, ROLE_STREAM]
+    idom = torch.stack([torch.randperm(64, generator=torch.Generator().manual_seed(g))[:16].sort().values
+                        for g in range(Hkv)]).to(torch.int32).to(dev)
+    step = AppendDecodeStep(Bn, Hq, Hkv, d, 5e5, roles, [steps + warmup + 8] * Bn, 128, 4096, d ** -0.5,
+                            idom=idom, n_fac=64)
+    q, k, v = (t.to(dev) for t in token_draws(1, 0, Bn, Hq, Hkv, d))
+    ms = _event_ms(lambda: step.append(q, k, v), steps, warmup)
+    st, _ = B.device_check()
+    n_lin = sum(1 for r in roles if r != ROLE_STREAM)
+    moved = Bn * (2 * Hq * d * 2 + Hkv * d * 2 * 2 + Hkv * d * 2 * 2 + 2 * n_lin * B.k_dom_cols(16))
+    return {"us_per_call": ms * 1e3, "tokens_per_call": Bn, "us_per_token": ms * 1e3 / Bn,
+            "bytes_per_call": moved, "device_check": st,
+            "workload": "64 sequences x (32 q, 8 KV heads, d 128): 2 retrieval + 2 sparse heads to the linear "
+                        "cache, 4 streaming heads to a 128 + 4096 ring"}
+
+
+def measure_offload(dev, steps: int = 20, warmup: int = 3) -> dict:
+    """FASA-M on the 8B-shaped layer: V and the non-dominant K dims in pinned host memory."""
+    from token_sparse_decode_b200.step import OffloadDecodeStep
+
+    w = make_workload(preset("llama8b_gqa4_L32k"))
+    k, v = w.k.to(dev), w.v.to(dev)
+    offs, idom = w.offsets.to(dev), w.idom.to(dev)
+    nfac = int(w.n_fac_per_seq.max())
+    step = OffloadDecodeStep(k, v, offs, w.max_len, w.total_tokens, w.spec.n_q_heads, idom, w.scale, n_fac=nfac,
+                             n_fac_cap=nfac)
+    del k, v
+    torch.cuda.empty_cache()
+    q = w.q.to(dev)
+    ms = _event_ms(lambda: step(q), steps, warmup)
+    link = step.link_bytes_per_step()
+    # the host link's measured copy bandwidth: 256 MB pinned host -> device
+    src = torch.empty(256 << 20, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    copy_ms = _event_ms(lambda: dst.copy_(src, non_blocking=True), 5, 2)
+    peak = src.numel() / (copy_ms * 1e-3) / 1e9
+    achieved = link / (ms * 1e-3) / 1e9
+    return {"ms_per_step": ms, "tokens_per_step": int(w.lengths.sum()),
+            "value": int(w.lengths.sum()) / (ms * 1e-3), "unit": "tokens/s",
+            "link_bytes_per_step": link, "link_achieved_gbs": achieved, "link_peak_gbs": peak,
+            "link_frac": achieved / peak, "peak_source": "measured pinned host-to-device copy of 256 MB",
+            "device_bytes": int(step.k_dom.numel() * 2),
+            "host_bytes": int((step.k_rest.numel() + step.v_host.numel()) * 2),
+            "workload": "llama8b_gqa4_L32k with V and the non-dominant K dims in pinned host memory"}
+
+
+def measure_classify(dev, steps: int = 5, warmup: int = 1) -> dict:
+    """The AoH head classifier on 8B-shaped projection weights (32 q / 8 KV heads, d_model 4096)."""
+    from token_sparse_decode_b200 import binding as B
+    from workloads import HEAD_WEIGHT_PRESETS, head_weights
+
+    sp = HEAD_WEIGHT_PRESETS["llama8b_heads"]
+    wq, wk, _ = head_weights(sp)
+    wq, wk = wq.to(dev), wk.to(dev)
+    er_h = torch.empty(sp.n_q_heads, dtype=torch.float64, device=dev)
+    er_g = torch.empty(sp.n_kv_heads, dtype=torch.float64, device=dev)
+    roles = torch.empty(sp.n_kv_heads, dtype=torch.uint8, device=dev)
+    ws = B.workspace(B.head_classify_workspace_size(sp.d_model, sp.n_q_heads, sp.n_kv_heads, sp.head_dim), dev)
+    fn = lambda: B.head_classify(wq, wk, sp.n_q_heads, sp.n_kv_heads, sp.head_dim, sp.n_retrieval, er_h, er_g,  # noqa: E731
+                                 roles, ws)
+    ms = _event_ms(fn, steps, warmup)
+    gram_flops = 2 * (sp.n_q_heads + sp.n_kv_heads) * sp.head_dim ** 2 * sp.d_model
+    rec = B.timed_launches(fn)
+    torch.cuda.synchronize()
+    per = {n: e0.elapsed_time(e1) for n, e0, e1 in rec}
+    return {"ms_per_call": ms, "kernel_ms": per, "gram_flops": gram_flops,
+            "weight_bytes": int((wq.numel() + wk.numel()) * 2), "roles": roles.cpu().tolist(),
+            "workload": "llama8b_heads: W_Q [4096, 4096], W_K [1024, 4096] bf16, 4 of 8 groups retrieval"}
+
+
 # ------------------------------------------------------------------------------ oracle (CPU) arms
 #
 # The oracle runs on whole (sequence, KV head) rows: the select needs every score of a row.
@@ -720,6 +814,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the append, host-offload and head-classifier measurements")
     ap.add_argument("--graph", type=int, default=1, help="replay each step from a CUDA graph (1) or launch (0)")
     ap.add_argument("--copies", type=int, default=0,
                     help="input copies to rotate over (0: enough for cold inputs; 1: one copy, L2 flushed)")
@@ -750,6 +846,11 @@ def main():
     res = run_ours(args, rank, world, local_rank)
     w = res.pop("_w")
     if rank == 0:
+        if not args.no_extras:
+            dev = torch.device("cuda", local_rank)
+            res["append"] = measure_append(dev)
+            res["offload"] = measure_offload(dev)
+            res["classify"] = measure_classify(dev)
         if not args.no_cpu_baseline and world == 1:
             res["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(res), flush=True)

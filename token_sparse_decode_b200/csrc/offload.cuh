@@ -64,7 +64,8 @@ struct SplitParams {
   uint8_t slot[kMaxHeads];
 };
 
-// One CTA per (KV head, slab of tokens): writes the head's host rows.
+// One CTA per (KV head, slab of tokens): writes the head's host rows, one 16-byte store per
+// 8 elements (each store crosses the host link).
 __global__ void __launch_bounds__(kStageThreads) offload_split_kernel(const SplitParams p) {
   __shared__ uint8_t perm[128];
   __shared__ int s_scan[33];
@@ -73,17 +74,30 @@ __global__ void __launch_bounds__(kStageThreads) offload_split_kernel(const Spli
   const int nrest = p.d - 2 * p.n_dom;
   const int64_t per = (p.T + gridDim.x - 1) / gridDim.x;
   const int64_t t0 = blockIdx.x * per, t1 = min((int64_t)p.T, t0 + per);
-  const int64_t row_elems = (int64_t)p.rest_cols + p.d;
-  for (int64_t e = t0 * row_elems + threadIdx.x; e < t1 * row_elems; e += kStageThreads) {
-    const int64_t t = e / row_elems;
-    const int i = (int)(e % row_elems);
+  const int rc = p.rest_cols / 8, vc = p.d / 8;  // 16-byte chunks of a rest row and of a value row
+  const int64_t row_chunks = rc + vc;
+  for (int64_t e = t0 * row_chunks + threadIdx.x; e < t1 * row_chunks; e += kStageThreads) {
+    const int64_t t = e / row_chunks;
+    const int c = (int)(e % row_chunks);
     const uint16_t* kr = p.k + t * p.stride_tok + (int64_t)p.slot[g] * p.stride_head;
     const uint16_t* vr = p.v + t * p.stride_tok + (int64_t)p.slot[g] * p.stride_head;
-    if (i < p.rest_cols) {
-      p.k_rest[((int64_t)g * p.T + t) * p.rest_cols + i] = i < nrest ? kr[perm[2 * p.n_dom + i]] : (uint16_t)0;
+    if (c < rc) {
+      uint16_t x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = c * 8 + u;
+        x[u] = i < nrest ? kr[perm[2 * p.n_dom + i]] : (uint16_t)0;
+      }
+      uint4 w;
+      w.x = (uint32_t)x[0] | ((uint32_t)x[1] << 16);
+      w.y = (uint32_t)x[2] | ((uint32_t)x[3] << 16);
+      w.z = (uint32_t)x[4] | ((uint32_t)x[5] << 16);
+      w.w = (uint32_t)x[6] | ((uint32_t)x[7] << 16);
+      *reinterpret_cast<uint4*>(p.k_rest + ((int64_t)g * p.T + t) * p.rest_cols + c * 8) = w;
     } else {
-      const int j = i - p.rest_cols;
-      p.v_host[((int64_t)g * p.T + t) * p.d + j] = vr[j];
+      const int j = c - rc;
+      *reinterpret_cast<uint4*>(p.v_host + ((int64_t)g * p.T + t) * p.d + j * 8) =
+          *reinterpret_cast<const uint4*>(vr + j * 8);
     }
   }
 }
