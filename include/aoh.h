@@ -145,7 +145,7 @@ int32_t aoh_last_cuda_error(void);
 /* Kernels the library launches, one counter each (see aoh_launch_counts). */
 typedef enum {
   AOH_KERNEL_TIP_SCORE = 0,     /* stand-alone importance scan                       */
-  AOH_KERNEL_TOPK_SELECT = 1,   /* stand-alone select, one CTA per row (many rows)   */
+  AOH_KERNEL_SELECT_HIST = 1,   /* select: first-digit histograms of given scores    */
   AOH_KERNEL_SPARSE_ROW = 2,    /* fused row kernel, or its select-only form         */
   AOH_KERNEL_FLASH_GATHER = 3,  /* split-K gather / window attention                 */
   AOH_KERNEL_PACK_DOMINANT = 4, /* dominant-column packing of K                      */
@@ -156,7 +156,9 @@ typedef enum {
   AOH_KERNEL_GROUP_ROLES = 9,   /* head classifier: group means and roles            */
   AOH_KERNEL_OFFLOAD_STAGE = 10,  /* host offload: selected rows across the host link */
   AOH_KERNEL_OFFLOAD_SPLIT = 11,  /* host offload: a device cache split to host parts */
-  AOH_KERNEL_KINDS = 12
+  AOH_KERNEL_SELECT_CHUNK = 12, /* select: threshold bin, candidates, exact threshold */
+  AOH_KERNEL_SELECT_WRITE = 13, /* select: ordered write of the chosen positions     */
+  AOH_KERNEL_KINDS = 14
 } aoh_kernel_kind;
 
 /*
@@ -241,11 +243,21 @@ aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* k
  *   n_fac_cap       capacity per row; n_fac (or every n_fac_per_seq entry) <= cap
  *   idx             device int32 [B][Hkv][n_fac_cap]; entries >= n are set to -1
  *   count           device int32 [B][Hkv]: n
- * Deterministic: the same input gives the same bits.
+ *   workspace       device, 256-byte aligned, >= aoh_topk_select_workspace_size
+ *                   bytes, zero-filled once before its first use (every call
+ *                   leaves its counters at zero again)
+ * Rows up to 4 M positions (AOH_ERR_UNSUPPORTED beyond).  Deterministic: the
+ * same input gives the same bits.  Mechanism: per row, a histogram of the top
+ * 11 bits of the order-preserving keys, then chunks of 4096 keys in parallel
+ * (keys above the threshold bin counted, keys in it collected, the exact
+ * threshold resolved once per row, every chunk's picks written in order).
  */
 aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
                            const int32_t* n_fac_per_seq, int32_t n_fac_cap,
-                           int32_t* idx, int32_t* count, void* stream);
+                           int32_t* idx, int32_t* count, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+size_t aoh_topk_select_workspace_size(const aoh_kv_cache* kv);
 
 /*
  * aoh_sparse_decode -- the whole sparse step for the heads whose role is

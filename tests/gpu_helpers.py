@@ -184,9 +184,10 @@ def launches_of(fn) -> dict:
 
 
 def three_kernel_form(launches: dict) -> bool:
-    """scan + select (the row kernel's select-only form or the select kernel) + gather"""
-    sel = launches.get("sparse_row_kernel", 0) + launches.get("topk_select_kernel", 0)
-    return launches.get("tip_score_kernel") == 1 and sel == 1 and launches.get("flash_gather_kernel") == 1
+    """scan (which also builds the select's histograms) + chunked select + gather"""
+    return (launches.get("tip_score_kernel") == 1 and launches.get("select_chunk_kernel") == 1
+            and launches.get("select_write_kernel") == 1 and "select_hist_kernel" not in launches
+            and launches.get("flash_gather_kernel", 0) >= 1)
 
 
 def run_sparse(d: Dev, pack=True):

@@ -136,7 +136,11 @@ def test_host_validation_rejects_before_launch(lib):
     # shared index: more than 32 query rows per KV head
     assert lib.aoh_shared_index_decode(0x40000, 9, 32, ctypes.byref(fake_kv()), 0x50000, 0x58000, 64, 0.1,
                                        0x60000, 0x70000, 1 << 40, None) == UNSUP
-    assert lib.aoh_topk_select(0x40000, ctypes.byref(fake_kv()), 10, None, 0, 0x50000, 0x58000, None) == INVALID
+    assert lib.aoh_topk_select(0x40000, ctypes.byref(fake_kv()), 10, None, 0, 0x50000, 0x58000, 0x70000, 1 << 40,
+                               None) == INVALID
+    assert lib.aoh_topk_select(0x40000, ctypes.byref(fake_kv()), 10, None, 64, 0x50000, 0x58000, None, 0,
+                               None) == WS
+    assert lib.aoh_topk_select_workspace_size(ctypes.byref(fake_kv())) >= 8 * 2000 * 8  # the candidate lists
     assert lib.aoh_pack_dominant(ctypes.byref(fake_kv()), 0x50000, 16, 0x60000, 36, None) == INVALID
 
 

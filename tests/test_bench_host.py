@@ -68,15 +68,15 @@ def test_kernel_bytes_follow_the_path_taken():
     w = lite("llama8b_gqa4_L32k")
     ab = bench.algorithmic_bytes(w)
     fused = ["sparse_row_kernel"]
-    three = ["tip_score_kernel", "sparse_row_kernel", "flash_gather_kernel"]
+    three = ["tip_score_kernel", "select_chunk_kernel", "select_write_kernel", "flash_gather_kernel"]
     assert bench.kernel_bytes(w, ab, "sparse_decode", "sparse_row_kernel", fused) == ab["tip"] + ab["fac"]
     assert bench.kernel_bytes(w, ab, "sparse_decode", "tip_score_kernel", three) == ab["tip"]
-    assert bench.kernel_bytes(w, ab, "sparse_decode", "sparse_row_kernel", three) == ab["select"]
+    assert bench.kernel_bytes(w, ab, "sparse_decode", "select_chunk_kernel", three) == ab["select"]
     assert bench.kernel_bytes(w, ab, "sparse_decode", "flash_gather_kernel", three) == ab["fac"]
     c = lite("clsa_shared_L128k")
     abc = bench.algorithmic_bytes(c)
     assert bench.kernel_bytes(c, abc, "shared_index_step", "sparse_row_kernel", fused) == abc["total"]
-    assert bench.kernel_bytes(c, abc, "shared_index_step", "topk_select_kernel", three) == abc["select"]
+    assert bench.kernel_bytes(c, abc, "shared_index_step", "select_write_kernel", three) == abc["select"]
     assert bench.kernel_bytes(c, abc, "shared_index_step", "flash_gather_kernel", three) == abc["gather"]
 
 

@@ -128,10 +128,10 @@ def test_topk_bit_exact_on_given_scores(kind):
 
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
-def test_topk_many_rows_one_cta_per_row(kind):
-    # 54 sequences x 3 KV heads = 162 rows, more than the SMs: the one-CTA-per-row select.
-    # Lengths mix empty, one-token, N_fac >= L and long rows; the ties / zeros kinds put more
-    # keys in the first digit's bin than its shared-memory candidate region holds (re-read path).
+def test_topk_many_rows(kind):
+    # 54 sequences x 3 KV heads = 162 rows of many chunks.  Lengths mix empty, one-token,
+    # N_fac >= L and long rows; the ties / zeros kinds put more candidates in the threshold
+    # bin than the resolving CTA keeps in shared memory (it then reads them from the list).
     rng = np.random.default_rng(15)
     lengths = [0, 1, 3, 700, 24000, 60000] + [int(x) for x in rng.integers(50, 9000, 48)]
     Hkv = 3
@@ -146,7 +146,7 @@ def test_topk_many_rows_one_cta_per_row(kind):
     cnt = torch.full((len(lengths), Hkv), -7, dtype=torch.int32, device=dev)
     sd, nd = torch.from_numpy(s).to(dev), torch.from_numpy(nfps).to(dev)
     launched = launches_of(lambda: B.topk_select(sd, kv, 0, nd, cap, idx, cnt))
-    assert launched == {"topk_select_kernel": 1}
+    assert launched == {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_write_kernel": 1}
     check_device()
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
     for b, L in enumerate(lengths):
@@ -344,7 +344,7 @@ def test_sparse_decode_every_token_selected():
 
 def test_sparse_decode_many_rows_runs_three_stages():
     # 40 sequences x 8 KV heads = 320 rows: more clusters than one wave holds, so the step
-    # runs as scan kernel + cluster select on the scores + split-K gather
+    # runs as scan kernel (with the select's histograms) + chunked select + split-K gather
     sp = spec(batch=40, len_range=(300, 3000), seed=87)
     w = make_workload(sp)
     d = Dev(w)
@@ -356,7 +356,7 @@ def test_sparse_decode_many_rows_runs_three_stages():
                                                    step.out, step.ws_sparse, step.idx, step.count))
     torch.cuda.synchronize()
     names = [k for k, _, _ in rec]
-    assert names[0] == "tip_score_kernel" and names[-1] == "flash_gather_kernel" and len(names) == 3
+    assert names == ["tip_score_kernel", "select_chunk_kernel", "select_write_kernel", "flash_gather_kernel"]
     assert all(e0.elapsed_time(e1) > 0 for _, e0, e1 in rec)
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()

@@ -27,14 +27,15 @@ EXPORTS = (
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
     "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
     "aoh_launch_counts", "aoh_record_launch_events", "aoh_kv_append", "aoh_head_classify",
-    "aoh_head_classify_workspace_size", "aoh_offload_split", "aoh_offload_decode", "aoh_offload_decode_workspace_size",
+    "aoh_head_classify_workspace_size", "aoh_topk_select_workspace_size", "aoh_offload_split", "aoh_offload_decode", "aoh_offload_decode_workspace_size",
 )
 NO_SLOT = 255  # head_slot entry of a KV head a cache does not store
 
 # aoh_kernel_kind order
-KERNELS = ("tip_score_kernel", "topk_select_kernel", "sparse_row_kernel", "flash_gather_kernel",
+KERNELS = ("tip_score_kernel", "select_hist_kernel", "sparse_row_kernel", "flash_gather_kernel",
            "pack_dominant_kernel", "kv_append_kernel", "gram_kernel", "gram_reduce_kernel", "spectrum_kernel",
-           "group_roles_kernel", "offload_stage_kernel", "offload_split_kernel")
+           "group_roles_kernel", "offload_stage_kernel", "offload_split_kernel", "select_chunk_kernel",
+           "select_write_kernel")
 
 
 class AohError(RuntimeError):
@@ -90,7 +91,8 @@ def lib() -> ctypes.CDLL:
             "aoh_record_launch_events": (None, [P, P, I32]),
             "aoh_pack_dominant": (ctypes.c_int, [KVP, P, I32, P, I32, P]),
             "aoh_tip_score": (ctypes.c_int, [P, I32, KVP, P, I32, P, P]),
-            "aoh_topk_select": (ctypes.c_int, [P, KVP, I32, P, I32, P, P, P]),
+            "aoh_topk_select": (ctypes.c_int, [P, KVP, I32, P, I32, P, P, P, SZ, P]),
+            "aoh_topk_select_workspace_size": (SZ, [KVP]),
             "aoh_sparse_decode": (ctypes.c_int, [P, I32, KVP, P, I32, I32, P, I32, P, F32, P, P, P, P, SZ, P]),
             "aoh_sparse_decode_workspace_size": (SZ, [KVP, I32, I32]),
             "aoh_stream_decode": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P, SZ, P]),
@@ -248,10 +250,19 @@ def tip_score(q: torch.Tensor, kv: KVCache, idom: torch.Tensor, n_dom: int, scor
                                                  _ptr(scores), _stream(stream)))
 
 
+def topk_select_workspace_size(kv: KVCache) -> int:
+    return int(lib().aoh_topk_select_workspace_size(ctypes.byref(kv)))
+
+
 def topk_select(scores: torch.Tensor, kv: KVCache, n_fac: int, n_fac_per_seq: Optional[torch.Tensor],
-                n_fac_cap: int, idx: torch.Tensor, count: torch.Tensor, stream=None) -> None:
+                n_fac_cap: int, idx: torch.Tensor, count: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                stream=None) -> None:
+    """aoh_topk_select; without `ws` a zero-filled workspace of the required size is made here."""
+    if ws is None:
+        ws = workspace(topk_select_workspace_size(kv), scores.device)
     _check("aoh_topk_select", lib().aoh_topk_select(_ptr(scores), ctypes.byref(kv), n_fac, _ptr(n_fac_per_seq),
-                                                     n_fac_cap, _ptr(idx), _ptr(count), _stream(stream)))
+                                                     n_fac_cap, _ptr(idx), _ptr(count), _ptr(ws), ws.numel(),
+                                                     _stream(stream)))
 
 
 def sparse_decode_workspace_size(kv: KVCache, n_q_heads: int, n_fac_cap: int) -> int:

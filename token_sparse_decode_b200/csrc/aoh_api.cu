@@ -16,9 +16,9 @@
 #include "head_classify.cuh"
 #include "kv_append.cuh"
 #include "offload.cuh"
+#include "select_hist.cuh"
 #include "sparse_row.cuh"
 #include "tip_score.cuh"
-#include "topk_select.cuh"
 
 using namespace aoh;
 
@@ -308,8 +308,9 @@ aoh_status launch_tip_t(TipParams& tp, cudaStream_t st) {
 }
 
 aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom,
-                      float* scores, const uint8_t* heads, int n_listed, cudaStream_t st) {
+                      float* scores, const uint8_t* heads, int n_listed, cudaStream_t st, uint32_t* hist = nullptr) {
   TipParams tp{};
+  tp.hist = hist;
   tp.q = static_cast<const uint16_t*>(q);
   tp.idom = idom;
   tp.offsets = kv->offsets;
@@ -353,39 +354,86 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
 
 // Full-dimension scores (every chunk; the shared indexer's score), K read in place.
 aoh_status launch_tip_full(const void* q, int32_t Hq, const aoh_kv_cache* kv, float* scores, const uint8_t* heads,
-                           int n_listed, cudaStream_t st) {
-  return launch_tip(q, Hq, kv, nullptr, kv->head_dim / 2, scores, heads, n_listed, st);
+                           int n_listed, cudaStream_t st, uint32_t* hist = nullptr) {
+  return launch_tip(q, Hq, kv, nullptr, kv->head_dim / 2, scores, heads, n_listed, st, hist);
 }
 
-// ------------------------------------------------------------------ top-k select
-// The streaming select kernel: one CTA per row, scores read from L2.
-aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
-                         int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
-                         cudaStream_t st) {
-  SelectParams sp{};
-  sp.scores = scores;
-  sp.offsets = kv->offsets;
-  bind_cache(sp, kv);
-  sp.n_fac_per_seq = nfps;
-  sp.idx = idx;
-  sp.count = count;
-  sp.T = (int32_t)kv->total_tokens;
-  sp.Hkv = kv->n_kv_heads;
-  sp.n_fac = n_fac;
-  sp.cap = cap;
-  memcpy(sp.heads, heads, n_listed);
-  const size_t smem = size_t(kSelCandCap) * 4;
-  static std::atomic<uint64_t> configured{0};
-  if (!set_up_on_this_device(configured)) {
-    aoh_status s = set_smem(topk_select_kernel, smem);
-    if (s != AOH_OK) return s;
-    mark_set_up(configured);
+// ------------------------------------------------------------------ chunked select
+// Workspace of the select (after the scores): [hist][cand_count][tickets] first (these must
+// start at zero and every select leaves them at zero), then the candidate list, the chunk
+// counts and offsets, and the row results.
+struct SelectWs {
+  size_t hist, cand_count, tickets, cand, chunk_above, chunk_info, row_info, total;
+  int max_chunks;
+};
+
+SelectWs select_ws(const aoh_kv_cache* kv) {
+  SelectWs w{};
+  const size_t rows = (size_t)kv->n_kv_heads * (size_t)std::max(kv->batch, 1);
+  w.max_chunks = (int)std::max<int64_t>(1, ceil_div(std::max(kv->max_len, 1), kSelChunk));
+  size_t o = 0;
+  w.hist = o;
+  o += align256(rows * kSelHistBins * sizeof(uint32_t));
+  w.cand_count = o;
+  o += align256(rows * sizeof(int32_t));
+  w.tickets = o;
+  o += align256(rows * sizeof(int32_t));
+  w.cand = o;
+  o += align256((size_t)kv->n_kv_heads * (size_t)std::max<int64_t>(kv->total_tokens, 1) * sizeof(unsigned long long));
+  w.chunk_above = o;
+  o += align256(rows * w.max_chunks * sizeof(int32_t));
+  w.chunk_info = o;
+  o += align256(rows * w.max_chunks * 2 * sizeof(int32_t));
+  w.row_info = o;
+  o += align256(rows * 2 * sizeof(int32_t));
+  w.total = o;
+  return w;
+}
+
+bool select_fits(const aoh_kv_cache* kv) { return ceil_div(std::max(kv->max_len, 1), kSelChunk) <= kSelMaxChunks; }
+
+// The select on the scores: the first-digit histograms (unless the scan built them), the chunk
+// pass and the ordered write.  `ws` is the select's region (layout of select_ws).
+aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
+                               int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
+                               uint8_t* ws, bool hist_ready, cudaStream_t st) {
+  if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
+  const SelectWs w = select_ws(kv);
+  HistSelectParams hp{};
+  hp.scores = scores;
+  hp.offsets = kv->offsets;
+  hp.lengths = kv->lengths;
+  hp.n_fac_per_seq = nfps;
+  hp.hist = reinterpret_cast<uint32_t*>(ws + w.hist);
+  hp.cand = reinterpret_cast<unsigned long long*>(ws + w.cand);
+  hp.cand_count = reinterpret_cast<int32_t*>(ws + w.cand_count);
+  hp.tickets = reinterpret_cast<int32_t*>(ws + w.tickets);
+  hp.chunk_above = reinterpret_cast<int32_t*>(ws + w.chunk_above);
+  hp.chunk_info = reinterpret_cast<int32_t*>(ws + w.chunk_info);
+  hp.row_info = reinterpret_cast<int32_t*>(ws + w.row_info);
+  hp.idx = idx;
+  hp.count = count;
+  hp.T = (int32_t)kv->total_tokens;
+  hp.B = kv->batch;
+  hp.Hkv = kv->n_kv_heads;
+  hp.n_fac = n_fac;
+  hp.cap = cap;
+  hp.max_chunks = w.max_chunks;
+  memcpy(hp.heads, heads, n_listed);
+  const dim3 grid(w.max_chunks, n_listed, kv->batch);
+  aoh_status s;
+  if (!hist_ready && kv->total_tokens > 0) {
+    before_launch(st);
+    select_hist_kernel<<<grid, kSelCtaThreads, 0, st>>>(hp);
+    if ((s = count_launch(AOH_KERNEL_SELECT_HIST, st)) != AOH_OK) return s;
   }
   before_launch(st);
-  topk_select_kernel<<<dim3(n_listed, kv->batch), kSelThreads, smem, st>>>(sp);
-  return count_launch(AOH_KERNEL_TOPK_SELECT, st);
+  select_chunk_kernel<<<grid, kSelCtaThreads, 0, st>>>(hp);
+  if ((s = count_launch(AOH_KERNEL_SELECT_CHUNK, st)) != AOH_OK) return s;
+  before_launch(st);
+  select_write_kernel<<<grid, kSelCtaThreads, 0, st>>>(hp);
+  return count_launch(AOH_KERNEL_SELECT_WRITE, st);
 }
-
 
 // ------------------------------------------------------------------ fused row kernel
 // Shared memory per CTA: keys of the slice, then a ring region used by the scan's
@@ -405,7 +453,7 @@ struct FusedPlan {
   size_t keys_bytes, ring_bytes, smem;
 };
 
-FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true) {
+FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
   FusedPlan f{};
   const int64_t L = std::max(kv->max_len, 1);
   const int64_t slice = (ceil_div(L, CL) + 3) & ~int64_t(3);
@@ -415,12 +463,10 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool need_ring = true)
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
   // 1 KB of slack: the kernel aligns its dynamic shared memory to 1024 bytes
   size_t budget = kTwoPerSm - 1024;
-  // select-only launches need only a region for the select's candidates (a quarter of the
-  // keys; a CTA whose candidates do not fit counts its later digits over all its keys)
-  const size_t ring_min = need_ring ? kRingMin : (size_t)ceil_div(f.keys_bytes / 4, 1024) * 1024;
+  const size_t ring_min = kRingMin;
   if (f.keys_bytes + ring_min > budget) budget = kOnePerSm - 1024;
   if (f.keys_bytes + ring_min > budget) return f;
-  f.ring_bytes = need_ring ? std::min(kRingMax, (budget - f.keys_bytes) / kRingStep * kRingStep) : ring_min;
+  f.ring_bytes = std::min(kRingMax, (budget - f.keys_bytes) / kRingStep * kRingStep);
   f.smem = f.keys_bytes + f.ring_bytes + 1024;
   f.ok = true;
   return f;
@@ -443,8 +489,8 @@ bool fused_feasible(const aoh_kv_cache* kv, int nq) {
 // length (ties to the smaller cluster).  With max_waves > 0 nothing is launched when every
 // choice needs more waves; *launched says which happened.
 template <int D, int NT>
-aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st, bool need_ring,
-                         int max_waves, bool* launched) {
+aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st, int max_waves,
+                         bool* launched) {
   *launched = false;
   auto kern = sparse_row_kernel<D, NT>;
   static std::atomic<uint64_t> configured{0};
@@ -460,7 +506,7 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   int64_t best_cost = INT64_MAX, best_waves = 0;
   const int cls[3] = {4, 8, 16};
   for (int i = 0; i < 3; ++i) {
-    const FusedPlan f = fused_candidate(kv, cls[i], need_ring);
+    const FusedPlan f = fused_candidate(kv, cls[i]);
     if (!f.ok) continue;
     const int maxc = max_active_clusters(kern, f.CL, f.smem);
     if (maxc <= 0) continue;
@@ -496,59 +542,16 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
 }
 
 aoh_status launch_rows(const RowParams& rp, const aoh_kv_cache* kv, int nq, int n_listed, int B, cudaStream_t st,
-                       bool need_ring, int max_waves, bool* launched) {
+                       int max_waves, bool* launched) {
   const int nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
   if (kv->head_dim == 128) {
-    if (nqp == 8) return launch_rows_t<128, 1>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
-    if (nqp == 16) return launch_rows_t<128, 2>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
-    return launch_rows_t<128, 4>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
+    if (nqp == 8) return launch_rows_t<128, 1>(rp, kv, n_listed, B, st, max_waves, launched);
+    if (nqp == 16) return launch_rows_t<128, 2>(rp, kv, n_listed, B, st, max_waves, launched);
+    return launch_rows_t<128, 4>(rp, kv, n_listed, B, st, max_waves, launched);
   }
-  if (nqp == 8) return launch_rows_t<64, 1>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
-  if (nqp == 16) return launch_rows_t<64, 2>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
-  return launch_rows_t<64, 4>(rp, kv, n_listed, B, st, need_ring, max_waves, launched);
-}
-
-// Select-only launch of the row kernel on precomputed scores: writes idx / count.
-aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
-                              int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
-                              cudaStream_t st) {
-  RowParams rp{};
-  rp.offsets = kv->offsets;
-  bind_cache(rp, kv);
-  rp.scores_in = scores;
-  rp.select_only = 1;
-  rp.n_fac_per_seq = nfps;
-  rp.n_fac = n_fac;
-  rp.cap = cap;
-  rp.idx_out = idx;
-  rp.count_out = count;
-  rp.T = (int32_t)kv->total_tokens;
-  rp.B = kv->batch;
-  rp.Hkv = kv->n_kv_heads;
-  rp.G = 1;
-  rp.NQ = 1;
-  rp.srow_len = 16;
-  memcpy(rp.heads, heads, n_listed);
-  bool launched = false;
-  const aoh_status s = launch_rows(rp, kv, 1, n_listed, kv->batch, st, false, 0, &launched);
-  if (s == AOH_OK && !launched) return AOH_ERR_UNSUPPORTED;
-  return s;
-}
-
-bool select_rows_feasible(const aoh_kv_cache* kv) { return fused_candidate(kv, kSrMaxCluster, false).ok; }
-
-// The select stage of the three-kernel step: the row kernel's cluster select on the scores;
-// rows longer than its clusters take the select kernel with the smallest cluster that keeps
-// each slice's keys in shared memory.
-aoh_status select_stage(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
-                        int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
-                        cudaStream_t st) {
-  // Rows enough to fill the SMs: one CTA per row.  Fewer, longer rows: the row kernel's
-  // cluster select, which spreads each row over a cluster's shared memory.
-  const int64_t rows = int64_t(kv->batch) * n_listed;
-  const bool rows_kernel = rows < sm_count() && select_rows_feasible(kv);
-  if (rows_kernel) return launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
-  return launch_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st);
+  if (nqp == 8) return launch_rows_t<64, 1>(rp, kv, n_listed, B, st, max_waves, launched);
+  if (nqp == 16) return launch_rows_t<64, 2>(rp, kv, n_listed, B, st, max_waves, launched);
+  return launch_rows_t<64, 4>(rp, kv, n_listed, B, st, max_waves, launched);
 }
 
 // Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,
@@ -606,7 +609,7 @@ size_t sparse_ws_bytes(const aoh_kv_cache* kv, int32_t Hq, int32_t cap, size_t* 
   o += align256(sizeof(int32_t) * (size_t)kv->batch * kv->n_kv_heads * (size_t)cap);
   *off_count = o;
   o += align256(sizeof(int32_t) * (size_t)kv->batch * kv->n_kv_heads);
-  return o;
+  return o + select_ws(kv).total;  // the select's region last
 }
 
 FdGeom stream_geom(const aoh_kv_cache* kv, int32_t Hq, const uint8_t* roles, int32_t sink, int32_t window) {
@@ -733,9 +736,14 @@ aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* k
   return launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n, as_stream(stream));
 }
 
+size_t aoh_topk_select_workspace_size(const aoh_kv_cache* kv) {
+  if (check_kv(kv) != AOH_OK || is_ring(kv)) return 0;
+  return select_ws(kv).total;
+}
+
 aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
                            const int32_t* n_fac_per_seq, int32_t n_fac_cap, int32_t* idx, int32_t* count,
-                           void* stream) {
+                           void* workspace, size_t workspace_bytes, void* stream) {
   aoh_status s = check_kv(kv);
   if (s != AOH_OK) return s;
   if (is_ring(kv)) return AOH_ERR_INVALID_ARG;  // a ring holds streaming heads only
@@ -743,9 +751,12 @@ aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t 
   if (!n_fac_per_seq && (n_fac < 0 || n_fac > n_fac_cap)) return AOH_ERR_INVALID_ARG;
   if (kv->batch == 0) return AOH_OK;
   if (!idx || !count || (!scores && kv->total_tokens > 0)) return AOH_ERR_INVALID_ARG;
+  if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
+  if (!ws_ok(workspace, workspace_bytes, select_ws(kv).total)) return AOH_ERR_WORKSPACE;
   uint8_t heads[kMaxHeads];
   const int n = list_heads(kv, nullptr, true, heads);
-  return select_stage(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n, as_stream(stream));
+  return launch_chunk_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n,
+                             static_cast<uint8_t*>(workspace), false, as_stream(stream));
 }
 
 size_t aoh_sparse_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, int32_t n_fac_cap) {
@@ -814,16 +825,19 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
     memcpy(rp.heads, heads, n_listed);
     // one launch when every row's cluster runs in a single wave
     bool launched = false;
-    if ((s = launch_rows(rp, kv, G, n_listed, kv->batch, st, true, 1, &launched)) != AOH_OK) return s;
+    if ((s = launch_rows(rp, kv, G, n_listed, kv->batch, st, 1, &launched)) != AOH_OK) return s;
     if (launched) return AOH_OK;
   }
 
-  // otherwise three kernels: the scan over all SMs, the cluster select on the (L2-resident)
-  // scores, and the split-K gather
+  // otherwise: the scan over all SMs (with the rows' first-digit histograms), the chunked
+  // select on the (L2-resident) scores, and the split-K gather
+  if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
+  uint8_t* sel_ws = ws + off_count + align256(sizeof(int32_t) * (size_t)kv->batch * kv->n_kv_heads);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sel_ws + select_ws(kv).hist);
   if (kv->total_tokens > 0) {
-    if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st)) != AOH_OK) return s;
+    if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st, hist)) != AOH_OK) return s;
   }
-  s = select_stage(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, st);
+  s = launch_chunk_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, sel_ws, true, st);
   if (s != AOH_OK) return s;
 
   const FdGeom geo = sparse_geom(kv, n_q_heads, n_fac_cap);
@@ -955,9 +969,13 @@ aoh_status aoh_shared_index_decode(const void* q_layers, int32_t n_layers, int32
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream), true);
 }
 
+size_t shared_step_scores_bytes(const aoh_kv_cache* kv) {
+  return align256(sizeof(float) * (size_t)kv->n_kv_heads * (size_t)std::max<int64_t>(kv->total_tokens, 1));
+}
+
+// [gather partials][scores][select region]
 size_t shared_step_ws_bytes(const aoh_kv_cache* kv, int32_t n_layers, int32_t Hq, int32_t topk) {
-  return fd_bytes(shared_geom(kv, n_layers, Hq, topk)) +
-         align256(sizeof(float) * (size_t)kv->n_kv_heads * (size_t)std::max<int64_t>(kv->total_tokens, 1));
+  return fd_bytes(shared_geom(kv, n_layers, Hq, topk)) + shared_step_scores_bytes(kv) + select_ws(kv).total;
 }
 
 size_t aoh_shared_index_step_workspace_size(const aoh_kv_cache* kv, int32_t n_layers, int32_t n_q_heads,
@@ -1014,14 +1032,18 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
     rp.scale_log2 = scale * 1.4426950408889634f;
     memcpy(rp.heads, heads, n_listed);
     bool launched = false;
-    if ((s = launch_rows(rp, kv, n_layers * G, n_listed, kv->batch, st, true, 1, &launched)) != AOH_OK) return s;
+    if ((s = launch_rows(rp, kv, n_layers * G, n_listed, kv->batch, st, 1, &launched)) != AOH_OK) return s;
     if (launched) return AOH_OK;
   }
-  // three kernels: full-dimension scores, the cluster select, the shared-index gather
+  // otherwise: full-dimension scores (with the first-digit histograms), the chunked select,
+  // the shared-index gather
+  if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
+  uint8_t* sel_ws = ws + fd_bytes(geo) + shared_step_scores_bytes(kv);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sel_ws + select_ws(kv).hist);
   if (kv->total_tokens > 0) {
-    if ((s = launch_tip_full(q_index, n_q_heads, kv, scores, heads, n_listed, st)) != AOH_OK) return s;
+    if ((s = launch_tip_full(q_index, n_q_heads, kv, scores, heads, n_listed, st, hist)) != AOH_OK) return s;
   }
-  s = select_stage(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, st);
+  s = launch_chunk_select(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, sel_ws, true, st);
   if (s != AOH_OK) return s;
   FdecParams fp{};
   fp.q = static_cast<const uint16_t*>(q_layers);
@@ -1288,7 +1310,7 @@ aoh_kv_cache offload_device_part(const aoh_offload_cache* oc) {
 }
 
 struct OffloadWs {
-  size_t fd, scores, idx, count, sidx, soff, sk, sv, sq, total;
+  size_t fd, scores, idx, count, sidx, soff, sk, sv, sq, sel, total;
 };
 
 OffloadWs offload_ws(const aoh_offload_cache* oc, int32_t Hq, int32_t cap) {
@@ -1314,6 +1336,8 @@ OffloadWs offload_ws(const aoh_offload_cache* oc, int32_t Hq, int32_t cap) {
   o += align256(2 * B * cap * H * d);
   w.sq = o;
   o += align256(2 * B * (size_t)Hq * d);
+  w.sel = o;
+  o += select_ws(&kv).total;
   w.total = o;
   return w;
 }
@@ -1396,9 +1420,13 @@ extern "C" aoh_status aoh_offload_decode(const void* q, int32_t n_q_heads, const
   int32_t* cnt = count_out ? count_out : reinterpret_cast<int32_t*>(ws + wl.count);
   cudaStream_t st = as_stream(stream);
   // 1-2. importance scan of the dominant columns (on the GPU) and the top-N_fac select
-  if (kv.total_tokens > 0 && (s = launch_tip(q, n_q_heads, &kv, idom, n_dom, scores, heads, Hkv, st)) != AOH_OK)
+  if (!select_fits(&kv)) return AOH_ERR_UNSUPPORTED;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + wl.sel + select_ws(&kv).hist);
+  if (kv.total_tokens > 0 && (s = launch_tip(q, n_q_heads, &kv, idom, n_dom, scores, heads, Hkv, st, hist)) != AOH_OK)
     return s;
-  if ((s = select_stage(scores, &kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, Hkv, st)) != AOH_OK) return s;
+  if ((s = launch_chunk_select(scores, &kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, Hkv, ws + wl.sel, true,
+                               st)) != AOH_OK)
+    return s;
   // 3. the selected rows across the host link, into HBM
   StageParams sp{};
   sp.q = static_cast<const uint16_t*>(q);

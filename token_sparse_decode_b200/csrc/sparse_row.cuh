@@ -16,9 +16,7 @@
 //  2. select:  4-digit MSB radix select of the n-th largest key over the cluster
 //              (histograms summed through distributed shared memory, one cluster
 //              barrier per digit); ties broken toward lower positions by an ordered
-//              compaction that also writes the index (ascending) to global memory.
-//              Select-only mode (three-kernel form) loads the keys from given
-//              scores and stops here;
+//              compaction that also writes the index (ascending) to global memory;
 //  3. attend:  every CTA gathers the K / V rows of the positions it selected from
 //              its own slice (cp.async into tiles at a 2*d+16-byte row pitch) and
 //              runs the online-softmax contraction on tensor cores (tokens on M,
@@ -70,8 +68,6 @@ struct RowParams {
   int32_t T, B, Hq, Hkv, G, NQ;
   int32_t keys_bytes;        // dynamic shared memory before the ring
   int32_t ring_bytes;        // ring region (scan rings, then attention stages); >= kSrRingMin
-  const float* scores_in;    // non-null: keys come from these fp32 scores [Hkv][T] (no scan)
-  int32_t select_only;       // 1: stop after writing the index (no attention)
   float scale_log2;
   uint8_t heads[kMaxHeads];
   uint8_t slot[kMaxHeads];   // head slot of every KV head in K / V and in the score rows
@@ -123,8 +119,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   int32_t* idx_row = p.idx_out + ((int64_t)b * p.Hkv + g) * p.cap;
   for (int j = n + rk * kSrThreads + tid; j < p.cap; j += CL * kSrThreads) idx_row[j] = -1;
   if (rk == 0 && tid == 0) p.count_out[(int64_t)b * p.Hkv + g] = n;
-  if (n == 0) {  // uniform over the cluster: zero rows (none in select-only mode), no barrier taken
-    if (rk == 0 && !p.select_only) {
+  if (n == 0) {  // uniform over the cluster: zero rows, no barrier taken
+    if (rk == 0) {
       for (int e = tid; e < p.NQ * D; e += kSrThreads) {
         const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
         p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + e % D] = 0.f;
@@ -157,15 +153,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     __syncthreads();
     cluster_arrive_release();
   }
-  if (n < L && p.scores_in) {
-    // scores already computed (the scan ran as its own kernel): load them as keys
-    const float* srow = p.scores_in + (int64_t)g * p.T + off + lo;
-    for (int i = tid; i < m; i += kSrThreads) keys[i] = score_key(__ldcg(srow + i));
-    __syncthreads();
-  }
   if (n < L) {
     // =============================================================== 1. scan
-    if (!p.scores_in) {
     if (tid < p.srow_len) {
       const int C = D / 2;
       int dim = -1;
@@ -253,7 +242,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       }
       cp_async_wait<0>();
       __syncthreads();
-    }
     }
     // =============================================================== 2. select
     // 4-digit MSB radix select over the cluster.  Digits 0-2: every CTA adds its non-zero
@@ -470,10 +458,6 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     nloc = m;
   }
   __syncthreads();
-  if (p.select_only) {  // index written; peers may still read this CTA's histograms
-    cluster.sync();
-    return;
-  }
 
   // =============================================================== 3. attend
   // warp = (token group, n-tile, part of the head dimension)

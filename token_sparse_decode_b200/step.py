@@ -99,6 +99,7 @@ class SharedIndexStep:
             self.scores = torch.empty((Hkv, max(total_tokens, 1)), dtype=torch.float32, device=self.dev)
             self.ws = B.workspace(B.shared_index_decode_workspace_size(self.kv, n_layers, n_q_heads, self.topk),
                                   self.dev)
+            self.ws_select = B.workspace(B.topk_select_workspace_size(self.kv), self.dev)
             self.ws_step = None
         self.out = torch.zeros((n_layers, batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
 
@@ -106,7 +107,7 @@ class SharedIndexStep:
         if self.scores is None:
             raise RuntimeError("SharedIndexStep.index needs fused=False (the fused step keeps its scores inside)")
         B.tip_score(q_index, self.kv, self.all_chunks, self.all_chunks.shape[1], self.scores)
-        B.topk_select(self.scores, self.kv, self.topk, None, self.topk, self.idx, self.count)
+        B.topk_select(self.scores, self.kv, self.topk, None, self.topk, self.idx, self.count, self.ws_select)
 
     def __call__(self, q_index: torch.Tensor, q_layers: torch.Tensor) -> torch.Tensor:
         if self.fused:
