@@ -445,6 +445,7 @@ constexpr size_t kOnePerSm = 220 * 1024;
 constexpr size_t kRingStep = 16 * 1024;
 constexpr size_t kRingMin = kSrRingMin;
 constexpr size_t kRingMax = 8 * kRingStep;
+constexpr int kShortRow = 2048;  // rows this short run as one CTA each (no cluster exchange)
 
 struct FusedPlan {
   bool ok;
@@ -504,8 +505,21 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   const int n_rows = n_listed * B;
   FusedPlan best{};
   int64_t best_cost = INT64_MAX, best_waves = 0;
+  // Short rows (<= kShortRow positions) take one CTA per row when that fits one wave: their
+  // time is the fixed cost of the phases, and a one-CTA cluster's barriers are block barriers.
+  if (kv->max_len <= kShortRow) {
+    const FusedPlan f = fused_candidate(kv, 1);
+    if (f.ok) {
+      const int maxc = max_active_clusters(kern, 1, f.smem);
+      if (maxc > 0 && n_rows <= maxc) {
+        best = f;
+        best_waves = 1;
+        best_cost = 0;
+      }
+    }
+  }
   const int cls[3] = {4, 8, 16};
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < 3 && best_cost > 0; ++i) {
     const FusedPlan f = fused_candidate(kv, cls[i]);
     if (!f.ok) continue;
     const int maxc = max_active_clusters(kern, f.CL, f.smem);
