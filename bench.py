@@ -205,18 +205,11 @@ def step_calls(w, step, q):
     """The public calls one step makes, by name (the same arguments as the step)."""
     from token_sparse_decode_b200 import binding as B
 
-    calls = []
     if w.spec.n_layers > 0:
-        calls.append(("shared_index_step", lambda: step(*q)))
-    else:
-        if step.has_sparse:
-            calls.append(("sparse_decode", lambda: B.sparse_decode(
-                q[0], step.kv, step.idom, step.n_dom, step.n_fac, step.n_fac_per_seq, step.n_fac_cap, step.roles,
-                step.scale, step.out, step.ws_sparse, step.idx, step.count)))
-        if step.has_stream:
-            calls.append(("stream_decode", lambda: B.stream_decode(
-                q[0], step.kv, step.roles, step.sink, step.window, step.scale, step.out, step.ws_stream)))
-    return calls
+        return [("shared_index_step", lambda: step(*q))]
+    return [("decode_step", lambda: B.decode_step(
+        q[0], step.kv, step.idom, step.n_dom, step.n_fac, step.n_fac_per_seq, step.n_fac_cap, step.roles, step.sink,
+        step.window, step.scale, step.out, step.ws, step.idx, step.count))]
 
 
 def launches_per_step(step, q) -> dict:
@@ -282,12 +275,14 @@ def cold_copies(step_bytes: int, l2_bytes: int) -> int:
     return r
 
 
-def kernel_bytes(w, ab: dict, call: str, kernel: str, order: list) -> int:
-    """Algorithmic bytes one launch of `kernel` moves inside `call` (see algorithmic_bytes).
+def kernel_bytes(w, ab: dict, call: str, kernel: str, order: list, index: int = -1) -> int:
+    """Algorithmic bytes one launch of `kernel` (launch `index` of `order`) moves inside `call`
+    (see algorithmic_bytes).
 
-    A call that launches the row kernel alone runs the whole path in it; in the three-kernel
-    form the scan reads the score columns, the select reads the fp32 scores (4 bytes per token
-    and scored KV head) and the gather reads the selected K / V rows.
+    A call that launches the row kernel alone runs the whole path in it (window heads
+    included); in the three-kernel form the scan reads the score columns, the select kernels
+    read the fp32 scores (4 bytes per token and scored KV head) and the gather reads the
+    selected K / V rows; a later gather of the same call attends the window heads.
     """
     fused = order == ["sparse_row_kernel"]
     if call == "stream_decode":
@@ -297,8 +292,12 @@ def kernel_bytes(w, ab: dict, call: str, kernel: str, order: list) -> int:
             return ab["indexer"] + ab["gather"]
         return {"tip_score_kernel": ab["indexer"], "flash_gather_kernel": ab["gather"]}.get(kernel, ab["select"])
     if fused:
-        return ab["tip"] + ab["fac"]
-    return {"tip_score_kernel": ab["tip"], "flash_gather_kernel": ab["fac"]}.get(kernel, ab["select"])
+        return ab["tip"] + ab["fac"] + ab["window"]
+    if kernel == "flash_gather_kernel":
+        first = order.index("flash_gather_kernel")
+        sparse_gather = "tip_score_kernel" in order and (index < 0 or index == first)
+        return ab["fac"] if sparse_gather else ab["window"]
+    return {"tip_score_kernel": ab["tip"], "sparse_row_kernel": ab["tip"] + ab["fac"]}.get(kernel, ab["select"])
 
 
 def capture_graph(fn):
@@ -453,7 +452,7 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = measured_peak_gbs()
     # the dominant kernel: the largest device time of one step
     dom = max(kt["kernels"], key=lambda e: e["ms"]) if kt["kernels"] else None
-    dom_bytes = kernel_bytes(w, ab, dom["call"], dom["kernel"], kt["order"][dom["call"]]) if dom else 0
+    dom_bytes = kernel_bytes(w, ab, dom["call"], dom["kernel"], kt["order"][dom["call"]], dom["index"]) if dom else 0
     dom_ms = dom["ms"] if dom else None
     one_kernel_step = dom is not None and len(kt["kernels"]) == 1
     if one_kernel_step:
@@ -488,7 +487,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": ncu_traffic(w.spec.name, dom["kernel"]) if dom else None},
         "call_ms": kt["calls"],
         "kernel_ms": [{"call": e["call"], "kernel": e["kernel"], "ms": e["ms"],
-                       "bytes": kernel_bytes(w, ab, e["call"], e["kernel"], kt["order"][e["call"]])}
+                       "bytes": kernel_bytes(w, ab, e["call"], e["kernel"], kt["order"][e["call"]], e["index"])}
                       for e in kt["kernels"]],
         "launches_per_step": per_step,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

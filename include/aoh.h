@@ -338,6 +338,28 @@ aoh_status aoh_stream_decode_noalloc(const void* q, int32_t n_q_heads, const aoh
                                      float scale, float* out, void* stream);
 
 /*
+ * aoh_decode_step -- the whole head-role-split step in one call: the SPARSE
+ * heads as aoh_sparse_decode, the DENSE / STREAM heads as aoh_stream_decode,
+ * on the same `out`.  When the fused row kernel holds every row in one wave
+ * and no window head's list exceeds 4 * n_fac_cap positions, DENSE / STREAM
+ * heads ride in the same launch as the SPARSE ones (their clusters attend over
+ * their ranges without scan or select): one launch for the whole step.
+ * Otherwise it runs the two calls in turn.  Arguments as for those two calls;
+ * roles may be NULL (every head SPARSE); a ring cache takes window heads only.
+ *   workspace  >= aoh_decode_step_workspace_size bytes, 256-byte aligned,
+ *              zero-filled once before its first use
+ */
+aoh_status aoh_decode_step(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv,
+                           const int32_t* idom, int32_t n_dom, int32_t n_fac,
+                           const int32_t* n_fac_per_seq, int32_t n_fac_cap, const uint8_t* roles,
+                           int32_t sink, int32_t window, float scale, float* out,
+                           int32_t* idx_out, int32_t* count_out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+size_t aoh_decode_step_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, int32_t n_fac_cap,
+                                      const uint8_t* roles, int32_t sink, int32_t window);
+
+/*
  * aoh_shared_index_decode -- the cross-decoder layers of a shared-cache
  * stack reuse one index ("Como funciona CLSA"): for every layer l, every
  * q head h of group g and sequence b,

@@ -69,10 +69,18 @@ def test_kernel_bytes_follow_the_path_taken():
     ab = bench.algorithmic_bytes(w)
     fused = ["sparse_row_kernel"]
     three = ["tip_score_kernel", "select_chunk_kernel", "select_write_kernel", "flash_gather_kernel"]
-    assert bench.kernel_bytes(w, ab, "sparse_decode", "sparse_row_kernel", fused) == ab["tip"] + ab["fac"]
-    assert bench.kernel_bytes(w, ab, "sparse_decode", "tip_score_kernel", three) == ab["tip"]
-    assert bench.kernel_bytes(w, ab, "sparse_decode", "select_chunk_kernel", three) == ab["select"]
-    assert bench.kernel_bytes(w, ab, "sparse_decode", "flash_gather_kernel", three) == ab["fac"]
+    assert bench.kernel_bytes(w, ab, "decode_step", "sparse_row_kernel", fused) == ab["tip"] + ab["fac"]
+    assert bench.kernel_bytes(w, ab, "decode_step", "tip_score_kernel", three) == ab["tip"]
+    assert bench.kernel_bytes(w, ab, "decode_step", "select_chunk_kernel", three) == ab["select"]
+    assert bench.kernel_bytes(w, ab, "decode_step", "flash_gather_kernel", three, 3) == ab["fac"]
+    # a second gather in the same call attends the window heads; without a scan every gather does
+    t = lite("tiny_mixed_d64_L512")
+    abt = bench.algorithmic_bytes(t)
+    assert bench.kernel_bytes(t, abt, "decode_step", "sparse_row_kernel", fused) == abt["tip"] + abt["fac"] + abt["window"]
+    assert bench.kernel_bytes(t, abt, "decode_step", "flash_gather_kernel", three + ["flash_gather_kernel"], 4) == abt["window"]
+    a = lite("aoh_roles_L128k")
+    aba = bench.algorithmic_bytes(a)
+    assert bench.kernel_bytes(a, aba, "decode_step", "flash_gather_kernel", ["flash_gather_kernel"], 0) == aba["window"]
     c = lite("clsa_shared_L128k")
     abc = bench.algorithmic_bytes(c)
     assert bench.kernel_bytes(c, abc, "shared_index_step", "sparse_row_kernel", fused) == abc["total"]

@@ -237,10 +237,13 @@ def test_stream_decode_matches_oracle(sink, window):
 
 
 def test_full_role_split_step_mixed_heads():
+    # every row in one wave and window lists no longer than 4 x N_fac: the whole step, window
+    # heads included, is one launch of the row kernel
     roles = (ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_SPARSE)
     w = make_workload(spec(n_q_heads=16, n_kv_heads=4, roles=roles, sink=16, window=200, n_fac_div=4, seed=82))
     d = Dev(w)
     step, out = run_sparse(d)
+    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
     G = w.spec.group
@@ -353,7 +356,7 @@ def test_sparse_decode_many_rows_runs_three_stages():
     # the same call with launch events armed: three kernels, in path order, each timed
     rec = B.timed_launches(lambda: B.sparse_decode(d.q, step.kv, step.idom, step.n_dom, step.n_fac,
                                                    step.n_fac_per_seq, step.n_fac_cap, step.roles, step.scale,
-                                                   step.out, step.ws_sparse, step.idx, step.count))
+                                                   step.out, step.ws, step.idx, step.count))
     torch.cuda.synchronize()
     names = [k for k, _, _ in rec]
     assert names == ["tip_score_kernel", "select_chunk_kernel", "select_write_kernel", "flash_gather_kernel"]
@@ -386,3 +389,24 @@ def test_shared_index_step_many_rows_runs_three_stages():
         compare_shared_row(w, b, g, sel, out_h[:, b, g * G:(g + 1) * G], 300)
         if np.array_equal(sel, r["sel"]):
             assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= OUT_ATOL
+
+
+def test_role_split_step_with_long_dense_rows_takes_two_calls():
+    # a dense row far longer than a selection keeps the split-K gather: the sparse step, then the window gather
+    roles = (ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_SPARSE)
+    w = make_workload(spec(n_q_heads=16, n_kv_heads=4, roles=roles, sink=16, window=200, n_fac_div=0, n_fac=48,
+                           len_range=(2000, 6000), seed=83))
+    d = Dev(w)
+    step, out = run_sparse(d)
+    launched = launches_of(lambda: step(d.q))
+    assert launched.get("flash_gather_kernel", 0) >= 1
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = w.spec.group
+    for b in range(w.spec.batch):
+        for g, role in enumerate(roles):
+            rows = out_h[b, g * G:(g + 1) * G]
+            if role == ROLE_SPARSE:
+                compare_sparse_row(w, b, g, idx_h[b, g, :cnt_h[b, g]], rows)
+            else:
+                compare_window_row(w, b, g, rows, role, w.spec.sink, w.spec.window)

@@ -6,7 +6,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import Dev, compare_shared_row, compare_sparse_row, compare_window_row, f64, run_shared, run_sparse
+from gpu_helpers import (Dev, compare_shared_row, compare_sparse_row, compare_window_row, f64, launches_of, run_shared,
+                         run_sparse)
 from workloads import ROLE_SPARSE, make_workload, preset
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -44,6 +45,14 @@ def check_role_split(name, n_rows, pack=True):
 
 def test_tiny_mixed_d64_L512_all_rows():
     check_role_split("tiny_mixed_d64_L512", 10 ** 9)
+
+
+def test_tiny_mixed_step_is_one_launch():
+    # 2 sparse + 2 streaming heads of a 512-token sequence: one row-kernel launch, one CTA a row
+    w = make_workload(preset("tiny_mixed_d64_L512"))
+    d = Dev(w)
+    step, _ = run_sparse(d)
+    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
 
 
 def test_llama8b_gqa4_L32k_all_rows():

@@ -27,7 +27,8 @@ EXPORTS = (
     "aoh_stream_decode_workspace_size", "aoh_shared_index_decode", "aoh_shared_index_decode_workspace_size",
     "aoh_shared_index_step", "aoh_shared_index_step_workspace_size", "aoh_stream_decode_noalloc",
     "aoh_launch_counts", "aoh_record_launch_events", "aoh_kv_append", "aoh_head_classify",
-    "aoh_head_classify_workspace_size", "aoh_topk_select_workspace_size", "aoh_offload_split", "aoh_offload_decode", "aoh_offload_decode_workspace_size",
+    "aoh_head_classify_workspace_size", "aoh_topk_select_workspace_size", "aoh_decode_step",
+    "aoh_decode_step_workspace_size", "aoh_offload_split", "aoh_offload_decode", "aoh_offload_decode_workspace_size",
 )
 NO_SLOT = 255  # head_slot entry of a KV head a cache does not store
 
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
             "aoh_tip_score": (ctypes.c_int, [P, I32, KVP, P, I32, P, P]),
             "aoh_topk_select": (ctypes.c_int, [P, KVP, I32, P, I32, P, P, P, SZ, P]),
             "aoh_topk_select_workspace_size": (SZ, [KVP]),
+            "aoh_decode_step": (ctypes.c_int, [P, I32, KVP, P, I32, I32, P, I32, P, I32, I32, F32, P, P, P, P, SZ, P]),
+            "aoh_decode_step_workspace_size": (SZ, [KVP, I32, I32, P, I32, I32]),
             "aoh_sparse_decode": (ctypes.c_int, [P, I32, KVP, P, I32, I32, P, I32, P, F32, P, P, P, P, SZ, P]),
             "aoh_sparse_decode_workspace_size": (SZ, [KVP, I32, I32]),
             "aoh_stream_decode": (ctypes.c_int, [P, I32, KVP, P, I32, I32, F32, P, P, SZ, P]),
@@ -292,6 +295,25 @@ def stream_decode(q: torch.Tensor, kv: KVCache, roles, sink: int, window: int, s
     _check("aoh_stream_decode", lib().aoh_stream_decode(
         _ptr(q), q.shape[-2], ctypes.byref(kv), ctypes.cast(r, ctypes.c_void_p), sink, window, float(scale),
         _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def decode_step_workspace_size(kv: KVCache, n_q_heads: int, n_fac_cap: int, roles, sink: int, window: int) -> int:
+    r = _host_u8(roles)
+    return int(lib().aoh_decode_step_workspace_size(ctypes.byref(kv), n_q_heads, n_fac_cap,
+                                                    None if r is None else ctypes.cast(r, ctypes.c_void_p), sink,
+                                                    window))
+
+
+def decode_step(q: torch.Tensor, kv: KVCache, idom: Optional[torch.Tensor], n_dom: int, n_fac: int,
+                n_fac_per_seq: Optional[torch.Tensor], n_fac_cap: int, roles, sink: int, window: int, scale: float,
+                out: torch.Tensor, ws: torch.Tensor, idx_out: Optional[torch.Tensor] = None,
+                count_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Every head of the step, by role (aoh_decode_step)."""
+    r = _host_u8(roles)
+    _check("aoh_decode_step", lib().aoh_decode_step(
+        _ptr(q), q.shape[-2], ctypes.byref(kv), _ptr(idom), n_dom, n_fac, _ptr(n_fac_per_seq), n_fac_cap,
+        None if r is None else ctypes.cast(r, ctypes.c_void_p), sink, window, float(scale), _ptr(out), _ptr(idx_out),
+        _ptr(count_out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def shared_index_decode_workspace_size(kv: KVCache, n_layers: int, n_q_heads: int, n_fac_cap: int) -> int:

@@ -934,6 +934,94 @@ aoh_status aoh_stream_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
   return launch_fd(fp, kv->head_dim, geo.nqp, n_listed, kv->batch, as_stream(stream));
 }
 
+size_t aoh_decode_step_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, int32_t n_fac_cap,
+                                      const uint8_t* roles, int32_t sink, int32_t window) {
+  if (check_kv(kv) != AOH_OK || check_heads(kv, n_q_heads) != AOH_OK || n_fac_cap < 1 || sink < 0 || window < 0)
+    return 0;
+  if (check_roles(kv, roles) != AOH_OK || n_q_heads / kv->n_kv_heads > kMaxQRows) return 0;
+  size_t a, b, c;
+  const size_t sparse = is_ring(kv) ? 0 : sparse_ws_bytes(kv, n_q_heads, n_fac_cap, &a, &b, &c);
+  return sparse + (roles ? fd_bytes(stream_geom(kv, n_q_heads, roles, sink, window)) : 0);
+}
+
+aoh_status aoh_decode_step(const void* q, int32_t n_q_heads, const aoh_kv_cache* kv, const int32_t* idom,
+                           int32_t n_dom, int32_t n_fac, const int32_t* n_fac_per_seq, int32_t n_fac_cap,
+                           const uint8_t* roles, int32_t sink, int32_t window, float scale, float* out,
+                           int32_t* idx_out, int32_t* count_out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  aoh_status s = check_kv(kv);
+  if (s != AOH_OK) return s;
+  if ((s = check_heads(kv, n_q_heads)) != AOH_OK) return s;
+  if ((s = check_roles(kv, roles)) != AOH_OK) return s;
+  const int G = n_q_heads / kv->n_kv_heads;
+  if (G > kMaxQRows) return AOH_ERR_UNSUPPORTED;
+  if (sink < 0 || window < 0 || !std::isfinite(scale) || n_fac_cap < 1) return AOH_ERR_INVALID_ARG;
+  uint8_t sparse_heads[kMaxHeads], win_heads[kMaxHeads];
+  const int n_sparse = list_heads(kv, roles, true, sparse_heads);
+  const int n_win = roles ? list_heads(kv, roles, false, win_heads) : 0;
+  if (is_ring(kv) && n_sparse) return AOH_ERR_INVALID_ARG;
+  size_t a, b, c;
+  const size_t sparse_need = is_ring(kv) ? 0 : sparse_ws_bytes(kv, n_q_heads, n_fac_cap, &a, &b, &c);
+  const size_t win_need = roles ? fd_bytes(stream_geom(kv, n_q_heads, roles, sink, window)) : 0;
+  if (kv->batch == 0) return AOH_OK;
+  if (!ws_ok(workspace, workspace_bytes, sparse_need + win_need)) return AOH_ERR_WORKSPACE;
+  // one launch for every head when the fused row kernel holds all rows in one wave and the
+  // window heads' lists are about as long as a selection (long dense rows keep the split-K gather)
+  int64_t win_max = 0;
+  for (int i = 0; i < n_win; ++i)
+    win_max = std::max<int64_t>(win_max, roles[win_heads[i]] == AOH_ROLE_DENSE
+                                             ? kv->max_len : std::min<int64_t>(kv->max_len, int64_t(sink) + window));
+  if (n_sparse > 0 && n_win > 0 && !is_ring(kv) && win_max <= 4 * int64_t(n_fac_cap) && fused_feasible(kv, G) && q &&
+      idom && out && aligned16(q) && n_dom >= 1 && n_dom <= kv->head_dim / 2 &&
+      (n_fac_per_seq || (n_fac >= 0 && n_fac <= n_fac_cap)) && (idx_out == nullptr) == (count_out == nullptr) &&
+      !(kv->k_dom && 2 * n_dom > kv->k_dom_cols)) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    RowParams rp{};
+    rp.q_score = static_cast<const uint16_t*>(q);
+    rp.q_attn = static_cast<const uint16_t*>(q);
+    rp.k = static_cast<const uint16_t*>(kv->k);
+    rp.v = static_cast<const uint16_t*>(kv->v);
+    rp.offsets = kv->offsets;
+    bind_cache(rp, kv);
+    rows_score_source(rp, kv, idom, n_dom);
+    rp.n_fac_per_seq = n_fac_per_seq;
+    rp.n_fac = n_fac;
+    rp.cap = n_fac_cap;
+    rp.idx_out = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + b);
+    rp.count_out = count_out ? count_out : reinterpret_cast<int32_t*>(ws + c);
+    rp.out = out;
+    rp.stride_tok = kv->stride_tok;
+    rp.stride_head = kv->stride_head;
+    rp.T = (int32_t)kv->total_tokens;
+    rp.B = kv->batch;
+    rp.Hq = n_q_heads;
+    rp.Hkv = kv->n_kv_heads;
+    rp.G = G;
+    rp.NQ = G;
+    rp.scale_log2 = scale * 1.4426950408889634f;
+    rp.sink = sink;
+    rp.window = window;
+    memcpy(rp.roles, roles, kv->n_kv_heads);
+    uint8_t heads[kMaxHeads];
+    memcpy(heads, sparse_heads, n_sparse);
+    memcpy(heads + n_sparse, win_heads, n_win);
+    memcpy(rp.heads, heads, n_sparse + n_win);
+    bool launched = false;
+    if ((s = launch_rows(rp, kv, G, n_sparse + n_win, kv->batch, as_stream(stream), 1, &launched)) != AOH_OK) return s;
+    if (launched) return AOH_OK;
+  }
+  // otherwise the SPARSE heads' step, then the window heads' attention
+  if (n_sparse > 0) {
+    s = aoh_sparse_decode(q, n_q_heads, kv, idom, n_dom, n_fac, n_fac_per_seq, n_fac_cap, roles, scale, out, idx_out,
+                          count_out, workspace, sparse_need, stream);
+    if (s != AOH_OK) return s;
+  }
+  if (n_win > 0)
+    return aoh_stream_decode(q, n_q_heads, kv, roles, sink, window, scale, out,
+                             static_cast<uint8_t*>(workspace) + sparse_need, win_need, stream);
+  return AOH_OK;
+}
+
 size_t aoh_shared_index_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_layers, int32_t n_q_heads,
                                               int32_t n_fac_cap) {
   if (check_kv(kv) != AOH_OK || check_heads(kv, n_q_heads) != AOH_OK || n_layers < 1 || n_fac_cap < 1) return 0;

@@ -26,7 +26,8 @@
 //  4. combine: the CL partial (m, l, acc) states are merged through distributed
 //              shared memory, each CTA writing 1/CL of the outputs.
 // Nothing but the index and the outputs goes to global memory; no global
-// scratch, no second launch.
+// scratch, no second launch.  DENSE / STREAM heads may ride in the same launch: their
+// clusters skip 1-2 and attend over their range (the whole AoH step in one launch).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -71,6 +72,8 @@ struct RowParams {
   float scale_log2;
   uint8_t heads[kMaxHeads];
   uint8_t slot[kMaxHeads];   // head slot of every KV head in K / V and in the score rows
+  uint8_t roles[kMaxHeads];  // 0 SPARSE (scan, select, attend); 1 DENSE / 2 STREAM: attend over the range
+  int32_t sink, window;      // the STREAM range: [0, min(sink, L)) U [max(sink, L - window), L)
 };
 
 // Attention tiles: gathered K / V rows are copied as 16-byte cp.async segments into rows
@@ -116,10 +119,24 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     nf = p.cap;
   }
   const int n = max(0, min(nf, L));
+  // a window head (DENSE or STREAM role, AoH summary Metodología §4) attends over its range,
+  // split evenly across the cluster: no scan, no select, no index written
+  const int role = p.roles[g];
+  int wra = 0, wrb = 0;
+  if (role == 1) {
+    wra = L;
+    wrb = L;
+  } else if (role == 2) {
+    wra = min(p.sink, L);
+    wrb = max(wra, L - p.window);
+  }
+  const int nwin = wra + (L - wrb);
   int32_t* idx_row = p.idx_out + ((int64_t)b * p.Hkv + g) * p.cap;
-  for (int j = n + rk * kSrThreads + tid; j < p.cap; j += CL * kSrThreads) idx_row[j] = -1;
-  if (rk == 0 && tid == 0) p.count_out[(int64_t)b * p.Hkv + g] = n;
-  if (n == 0) {  // uniform over the cluster: zero rows, no barrier taken
+  if (role == 0) {
+    for (int j = n + rk * kSrThreads + tid; j < p.cap; j += CL * kSrThreads) idx_row[j] = -1;
+    if (rk == 0 && tid == 0) p.count_out[(int64_t)b * p.Hkv + g] = n;
+  }
+  if ((role == 0 ? n : nwin) == 0) {  // uniform over the cluster: zero rows, no barrier taken
     if (rk == 0) {
       for (int e = tid; e < p.NQ * D; e += kSrThreads) {
         const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
@@ -144,7 +161,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
 
   // The select's totals are filled by every CTA of the cluster: zero them, then arrive on a
   // cluster barrier that is waited on only before the first remote add (the scan runs in between).
-  if (n < L) {
+  if (role == 0 && n < L) {
     lhb[0][tid] = 0;
     lhb[1][tid] = 0;
     tot[0][tid] = 0;
@@ -153,7 +170,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     __syncthreads();
     cluster_arrive_release();
   }
-  if (n < L) {
+  if (role == 0 && n < L) {
     // =============================================================== 1. scan
     if (tid < p.srow_len) {
       const int C = D / 2;
@@ -449,13 +466,22 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       }
     }
     nloc = sel_cta;
-  } else {
+  } else if (role == 0) {
     // N_fac >= L: every position of the slice, in order
     for (int i = tid; i < m; i += kSrThreads) {
       plist[i] = lo + i;
       idx_row[lo + i] = lo + i;
     }
     nloc = m;
+  } else {
+    // a window head: this CTA's share of the range (at most ceil(L / CL) <= slice entries)
+    const int per = (nwin + CL - 1) / CL;
+    const int j0 = min(nwin, rk * per), j1 = min(nwin, j0 + per);
+    for (int i = tid; i < j1 - j0; i += kSrThreads) {
+      const int j = j0 + i;
+      plist[i] = j < wra ? j : wrb + (j - wra);
+    }
+    nloc = j1 - j0;
   }
   __syncthreads();
 

@@ -1,9 +1,9 @@
 """Decode steps composed from the C-ABI entry points (device buffers held by torch).
 
-``SparseDecodeStep``: the head-role-split step.  KV heads with role SPARSE run the
-importance scan over their dominant chunks, the top-N_fac select and focused
-attention (one ``aoh_sparse_decode`` call); DENSE / STREAM heads run
-``aoh_stream_decode``.  Both write into one fp32 output.
+``SparseDecodeStep``: the head-role-split step in one ``aoh_decode_step`` call.  KV
+heads with role SPARSE run the importance scan over their dominant chunks, the
+top-N_fac select and focused attention; DENSE / STREAM heads attend over the whole
+cache or the sink + window.  All write into one fp32 output.
 
 ``SharedIndexStep``: the shared-index cross-decoder stack.  The indexer scores
 every cached token with the full-dimension q.k, takes one top-k and every layer
@@ -50,23 +50,20 @@ class SparseDecodeStep:
             kv0 = B.make_kv(k, v, offsets, max_len, total_tokens)
             B.pack_dominant(kv0, idom, self.n_dom, self.k_dom)
         self.kv = B.make_kv(k, v, offsets, max_len, total_tokens, self.k_dom)
-        self.ws_sparse = self.ws_stream = None
+        self.n_fac_cap = max(self.n_fac_cap, 1)
+        self.idx = self.count = None
         if self.has_sparse:
-            self.ws_sparse = B.workspace(B.sparse_decode_workspace_size(self.kv, n_q_heads, self.n_fac_cap), self.dev)
             self.idx = torch.empty((batch, k.shape[1], self.n_fac_cap), dtype=torch.int32, device=self.dev)
             self.count = torch.empty((batch, k.shape[1]), dtype=torch.int32, device=self.dev)
-        if self.has_stream:
-            self.ws_stream = B.workspace(
-                B.stream_decode_workspace_size(self.kv, n_q_heads, self.roles, self.sink, self.window), self.dev)
+        self.ws = B.workspace(B.decode_step_workspace_size(self.kv, n_q_heads, self.n_fac_cap, self.roles, self.sink,
+                                                           self.window), self.dev)
         self.out = torch.zeros((batch, n_q_heads, d), dtype=torch.float32, device=self.dev)
 
     def __call__(self, q: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Every head of the step in one ``aoh_decode_step`` call (one launch when the rows allow)."""
         out = self.out if out is None else out
-        if self.has_sparse:
-            B.sparse_decode(q, self.kv, self.idom, self.n_dom, self.n_fac, self.n_fac_per_seq, self.n_fac_cap,
-                            self.roles, self.scale, out, self.ws_sparse, self.idx, self.count)
-        if self.has_stream:
-            B.stream_decode(q, self.kv, self.roles, self.sink, self.window, self.scale, out, self.ws_stream)
+        B.decode_step(q, self.kv, self.idom, self.n_dom, self.n_fac, self.n_fac_per_seq, self.n_fac_cap, self.roles,
+                      self.sink, self.window, self.scale, out, self.ws, self.idx, self.count)
         return out
 
     def run_host(self, q_host: torch.Tensor, out_host: torch.Tensor, q_dev: torch.Tensor) -> None:
