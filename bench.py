@@ -183,7 +183,8 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ our arm
 
-def build_step(w, dev):
+def build_step(w, dev, pack: bool = True):
+    """The workload's step on `dev`; pack=False keeps no packed dominant columns (the scan reads K in place)."""
     from token_sparse_decode_b200.step import SharedIndexStep, SparseDecodeStep
 
     k, v = w.k.to(dev), w.v.to(dev)
@@ -197,7 +198,7 @@ def build_step(w, dev):
     step = SparseDecodeStep(k, v, offsets, w.max_len, w.total_tokens, w.spec.n_q_heads, w.roles.tolist(),
                             w.scale, idom=idom, n_fac=int(w.n_fac_per_seq.max()),
                             n_fac_per_seq=w.n_fac_per_seq.to(dev), n_fac_cap=int(w.n_fac_per_seq.max()),
-                            sink=w.spec.sink, window=w.spec.window)
+                            sink=w.spec.sink, window=w.spec.window, pack_dominant=pack)
     return step, (w.q.to(dev),)
 
 
@@ -349,7 +350,7 @@ def run_ours(args, rank, world, local_rank):
     # pushes the other copies out of L2), or, for steps too small for that, flush L2 by
     # rewriting a buffer of twice its size between steps (outside the events).
     R = cold_copies(ab["total"], l2) if args.copies == 0 else (args.copies if args.copies > 1 else 0)
-    copies = [build_step(w, dev) for _ in range(max(R, 1))]
+    copies = [build_step(w, dev, not args.in_place_scan) for _ in range(max(R, 1))]
     step, q = copies[0]
     if R:
         def between():
@@ -475,7 +476,8 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic (seeded; bf16 N(0,1) post-RoPE q/K, V; planted salient keys where the workload has them)",
         "config": dict(workload_config(w, world), l2=l2_note,
-                       launch="CUDA graph replay" if args.graph else "direct launches"),
+                       launch="CUDA graph replay" if args.graph else "direct launches",
+                       **({"scan": "K read in place (no packed dominant columns)"} if args.in_place_scan else {})),
         "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
                      "bytes_per_step": ab["total"]},
         "roofline": {"kernel": dom["kernel"] if dom else None, "call": dom["call"] if dom else None, "bound": "hbm",
@@ -813,6 +815,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--in-place-scan", action="store_true",
+                    help="keep no packed dominant columns: the importance scan reads the 16-byte segments of K")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the append, host-offload and head-classifier measurements")
     ap.add_argument("--graph", type=int, default=1, help="replay each step from a CUDA graph (1) or launch (0)")
