@@ -66,25 +66,25 @@ class OracleCaches:
 def prefix(step: AppendDecodeStep, orc: OracleCaches, L0, seed):
     """Positions 0 .. L0_b - 1 of every sequence, written into both sides' caches by the test."""
     d, theta = step.d, step.theta
-    for b, L0 in enumerate(L0):
+    for b, Lb in enumerate(L0):
         r = np.random.default_rng([seed, b])
-        raw_k = r.standard_normal((L0, step.Hkv, d))
-        raw_v = r.standard_normal((L0, step.Hkv, d))
+        raw_k = r.standard_normal((Lb, step.Hkv, d))
+        raw_v = r.standard_normal((Lb, step.Hkv, d))
         o = int(step.offsets[b])
         for g in range(step.Hkv):
-            kb = oracle.to_bf16_bits(oracle.rope(raw_k[:, g], range(L0), theta)) if L0 else np.zeros((0, d), np.uint16)
-            vb = oracle.to_bf16_bits(raw_v[:, g]) if L0 else np.zeros((0, d), np.uint16)
+            kb = oracle.to_bf16_bits(oracle.rope(raw_k[:, g], range(Lb), theta)) if Lb else np.zeros((0, d), np.uint16)
+            vb = oracle.to_bf16_bits(raw_v[:, g]) if Lb else np.zeros((0, d), np.uint16)
             orc.k[(b, g)] = list(kb)
             orc.v[(b, g)] = list(vb)
-            if L0 == 0:
+            if Lb == 0:
                 continue
             if step.lin_slot[g] != B.NO_SLOT:
                 s = step.lin_slot[g]
-                step.k[o:o + L0, s] = to_dev_bf16(kb)
-                step.v[o:o + L0, s] = to_dev_bf16(vb)
+                step.k[o:o + Lb, s] = to_dev_bf16(kb)
+                step.v[o:o + Lb, s] = to_dev_bf16(vb)
             if step.ring_slot[g] != B.NO_SLOT:
                 s, ro = step.ring_slot[g], b * (step.sink + step.window)
-                for j, pos in enumerate(oracle.ring_contents(L0, step.sink, step.window)):
+                for j, pos in enumerate(oracle.ring_contents(Lb, step.sink, step.window)):
                     if pos >= 0:
                         step.rk[ro + j, s] = to_dev_bf16(kb[pos])
                         step.rv[ro + j, s] = to_dev_bf16(vb[pos])

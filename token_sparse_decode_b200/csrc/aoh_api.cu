@@ -172,9 +172,10 @@ FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
   chunk = ceil_div(chunk, kFdTS) * kFdTS;
   g.nqp = nq <= 8 ? 8 : (nq <= 16 ? 16 : 32);
   // partials grow with the query rows and the last CTA of a row reads them all: at most 16
-  // splits for 16 or 32 query rows (rows of equal length merge them on chip, in a cluster)
+  // splits for 16 query rows, 8 for 32 (measured: 16 splits of the 32-row shared-index gather,
+  // merged in 16-CTA clusters, took 32.9 us against 24.9 us for 8)
   if (g.nqp > 8) {
-    const int64_t max_sp = 16;
+    const int64_t max_sp = g.nqp == 16 ? 16 : 8;
     chunk = std::max<int64_t>(chunk, ceil_div(ceil_div(std::max<int64_t>(n_max, 1), max_sp), kFdTS) * kFdTS);
   }
   g.chunk = (int)chunk;
