@@ -224,6 +224,6 @@ def test_head_classifier_arguments_are_checked_on_the_host(lib):
     assert call(ws=None) == WS and call(wsb=1000) == WS
     size = lib.aoh_head_classify_workspace_size
     need = size(4096, 32, 8, 128)
-    # fp32 partials of 8 splits of 512 columns, fp64 Gram matrices of 40 heads, fp64 scratch of 32
-    assert need == 40 * 8 * 128 * 128 * 4 + 40 * 128 * 128 * 8 + 32 * 128 * 128 * 8
+    # fp64 partials of 8 splits of 512 columns, fp64 Gram matrices of 40 heads, fp64 scratch of 32
+    assert need == 40 * 8 * 128 * 128 * 8 + 40 * 128 * 128 * 8 + 32 * 128 * 128 * 8
     assert size(4096, 30, 8, 128) == 0 and size(192, 4, 2, 64) > 0

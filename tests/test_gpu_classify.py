@@ -1,12 +1,14 @@
 """The AoH head classifier on the GPU against the float64 oracle.
 
-Tolerance: effective ranks within 1e-5 relative.  The GPU forms each Gram matrix
-from bf16 products (exact in fp32) summed in fp32 over at most 512 columns per
-split, the splits summed in fp64; everything after is fp64.  A CPU simulation of
-that summation on the 8B-shaped weights moves ER by at most 1.3e-7 relative, so
-1e-5 leaves a wide margin for the tensor cores' own summation order.  Roles must
-match exactly wherever the oracle's group ranks are separated by more than twice
-that tolerance at the retrieval boundary (else either order is a valid answer).
+Tolerance: effective ranks within 1e-8 relative.  The GPU forms each Gram matrix on
+the fp64 tensor-core path from bf16 weights (exact in fp64, so every product is
+exact) and everything after is fp64; it differs from the oracle only in summation
+order and in how the eigenvalues are found (Cholesky, congruence and Jacobi against
+numpy's eig of C_h), both at the 1e-13 level for these well-conditioned Gram
+matrices (numpy's eig of the non-symmetric C_h being the looser of the two), so 1e-8 leaves a wide margin.  (With fp32 accumulation on the bf16 path,
+the same tests measured errors up to 2.6e-4 relative on concentrated spectra.)
+Roles must match exactly wherever the oracle's group ranks are separated by more
+than twice that tolerance at the retrieval boundary (else either order is valid).
 """
 
 import numpy as np
@@ -20,7 +22,7 @@ from workloads import HEAD_WEIGHT_PRESETS, HeadWeightSpec, head_weights
 
 pytestmark = pytest.mark.gpu
 
-ER_REL = 1e-5
+ER_REL = 1e-8
 
 
 def classify_on_gpu(wq, wk, spec, n_retrieval):

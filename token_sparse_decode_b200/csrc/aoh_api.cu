@@ -1264,7 +1264,7 @@ ClassifyGeom classify_geom(int32_t d_model, int32_t Hq, int32_t Hkv, int32_t D) 
   g.k_per_split = kps;
   g.splits = d_model / kps;
   const size_t heads = (size_t)Hq + Hkv, dd = (size_t)D * D;
-  g.partial_bytes = align256(heads * g.splits * dd * sizeof(float));
+  g.partial_bytes = align256(heads * g.splits * dd * sizeof(double));
   g.gram_bytes = align256(heads * dd * sizeof(double));
   g.work_bytes = align256((size_t)Hq * dd * sizeof(double));
   return g;
@@ -1291,7 +1291,7 @@ aoh_status launch_classify(const void* w_q, const void* w_k, int32_t d_model, in
     if ((s = set_smem(spectrum_kernel<D>, spec_smem)) != AOH_OK) return s;
     mark_set_up(configured);
   }
-  float* partial = reinterpret_cast<float*>(ws);
+  double* partial = reinterpret_cast<double*>(ws);
   double* gram = reinterpret_cast<double*>(ws + geo.partial_bytes);
   double* work = reinterpret_cast<double*>(ws + geo.partial_bytes + geo.gram_bytes);
   GramParams gp{};
@@ -1304,7 +1304,7 @@ aoh_status launch_classify(const void* w_q, const void* w_k, int32_t d_model, in
   gp.splits = geo.splits;
   gp.k_per_split = geo.k_per_split;
   before_launch(st);
-  gram_kernel<D><<<dim3(geo.splits, Hq + Hkv), kGramThreads, gram_smem, st>>>(gp);
+  gram_kernel<D><<<dim3(geo.splits, Hq + Hkv, 2), kGramThreads, gram_smem, st>>>(gp);
   aoh_status s = count_launch(AOH_KERNEL_GRAM, st);
   if (s != AOH_OK) return s;
   const int64_t n = int64_t(Hq + Hkv) * D * D;

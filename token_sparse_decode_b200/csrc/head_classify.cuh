@@ -11,10 +11,11 @@
 //       are retrieval heads (DENSE), the others streaming heads (STREAM).
 //
 // Kernels:
-//   gram_kernel      A_h and B_g for every head: [d x d_model] x [d_model x d] on tensor
-//                    cores (mma.sync m16n8k16 bf16, fp32 accumulation), d_model split over
-//                    CTAs; each CTA writes its fp32 partial (bf16 products are exact in
-//                    fp32, a split sums <= 512 of them);
+//   gram_kernel      A_h and B_g for every head: [d x d_model] x [d_model x d] on the fp64
+//                    tensor-core path (mma.sync m8n8k4 f64): the bf16 weights are exact in
+//                    fp64, so products are exact and sums round in fp64 (the fp32
+//                    accumulation of the bf16 path moved ER by up to 2.6e-4 on
+//                    concentrated spectra); d_model split over CTAs, fp64 partials;
 //   gram_reduce      the partials summed in a fixed order in fp64 (deterministic);
 //   spectrum_kernel  one CTA per q head, fp64 in shared memory: Cholesky B = L L^T, then
 //                    S = L^T A L (symmetric, eig(S) = eig(A B) = eig(C_h)), its eigenvalues
@@ -41,18 +42,32 @@ constexpr int kCheckFactor = 5;       // device check id: a key Gram matrix with
 struct GramParams {
   const uint16_t* wq;   // [Hq * D][d_model]
   const uint16_t* wk;   // [Hkv * D][d_model]
-  float* partial;       // [Hq + Hkv][splits][D][D]
+  double* partial;      // [Hq + Hkv][splits][D][D]
   int32_t d_model, Hq, Hkv, splits, k_per_split;
 };
 
+// D = A(8x4, row) * B(4x8, col) + C on the fp64 tensor-core path
+__device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};\n"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ double bf16_at(const uint16_t* t, int r, int c) {
+  return (double)__uint_as_float((uint32_t)t[r * kGramPitch + c] << 16);
+}
+
+// One CTA: half of the columns (blockIdx.z) of a head's W W^T over one split of d_model, on the
+// fp64 tensor-core path: bf16 weights are exact in fp64, so every product is exact and the sums
+// carry fp64 rounding only.  8 warps as 4 (rows) x 2 (columns) of 8 x 8 tiles.
 template <int D>
 __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramParams p) {
-  constexpr int WM = D / 4, WN = D / 2;  // warp tile: 4 x 2 warps cover D x D
-  constexpr int MT = WM / 16, NT = WN / 8;
+  constexpr int WM = D / 4, WN = D / 4;  // warp tile; the CTA covers D rows x D/2 columns
+  constexpr int MT = WM / 8, NT = WN / 8;
   constexpr int kStageElems = D * kGramPitch;
   extern __shared__ __align__(16) uint16_t gsm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int head = blockIdx.y, split = blockIdx.x;
+  const int head = blockIdx.y, split = blockIdx.x, half = blockIdx.z;
   const uint16_t* w = head < p.Hq ? p.wq + (int64_t)head * D * p.d_model
                                   : p.wk + (int64_t)(head - p.Hq) * D * p.d_model;
   const int k0 = split * p.k_per_split;
@@ -71,12 +86,14 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramParams p) 
     cp_async_commit();
   };
 
-  const int wm = warp & 3, wn = warp >> 2;  // rows wm*WM.., columns wn*WN..
-  float acc[MT][NT][4];
+  const int wm = warp & 3, wn = warp >> 2;
+  const int row0 = wm * WM, col0 = half * (D / 2) + wn * WN;
+  const int gr = lane >> 2, gc = lane & 3;  // fragment row (A) / column (B), and k within the step
+  double acc[MT][NT][2];
 #pragma unroll
   for (int i = 0; i < MT; ++i)
 #pragma unroll
-    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
 
 #pragma unroll
   for (int s = 0; s < kGramStages - 1; ++s) issue(s);
@@ -84,54 +101,40 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramParams p) 
     cp_async_wait<kGramStages - 2>();
     __syncthreads();
     issue(st + kGramStages - 1);
-    const uint32_t tile = sbase + (uint32_t)((st % kGramStages) * kStageElems) * 2;
+    const uint16_t* tile = gsm + (st % kGramStages) * kStageElems;
+#pragma unroll 4
+    for (int kk = 0; kk < kGramK; kk += 4) {
+      double a[MT], b[NT];
 #pragma unroll
-    for (int kk = 0; kk < kGramK; kk += 16) {
-      uint32_t a[MT][4];
+      for (int i = 0; i < MT; ++i) a[i] = bf16_at(tile, row0 + i * 8 + gr, kk + gc);  // A[i][k] = W[i][k]
 #pragma unroll
-      for (int i = 0; i < MT; ++i) {
-        const int r = wm * WM + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int c = kk + (lane >> 4) * 8;
-        ldsm_x4(a[i], tile + (uint32_t)(r * kGramPitch + c) * 2);
-      }
+      for (int j = 0; j < NT; ++j) b[j] = bf16_at(tile, col0 + j * 8 + gr, kk + gc);  // B[k][j] = W[j][k]
 #pragma unroll
-      for (int j = 0; j < NT; j += 2) {
-        // two n-tiles of B at once: B[k][n] = W[n][k], the rows of the same tile
-        uint32_t b[4];
-        const int r = wn * WN + j * 8 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = kk + ((lane >> 3) & 1) * 8;
-        ldsm_x4(b, tile + (uint32_t)(r * kGramPitch + c) * 2);
+      for (int i = 0; i < MT; ++i)
 #pragma unroll
-        for (int i = 0; i < MT; ++i) {
-          mma_16816(acc[i][j], a[i], b[0], b[1]);
-          mma_16816(acc[i][j + 1], a[i], b[2], b[3]);
-        }
-      }
+        for (int j = 0; j < NT; ++j) dmma_884(acc[i][j], a[i], b[j]);
     }
   }
   cp_async_wait<0>();
-  float* out = p.partial + ((int64_t)head * p.splits + split) * D * D;
+  double* out = p.partial + ((int64_t)head * p.splits + split) * D * D;
 #pragma unroll
   for (int i = 0; i < MT; ++i)
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-      const int r = wm * WM + i * 16 + (lane >> 2);
-      const int c = wn * WN + j * 8 + 2 * (lane & 3);
+      const int r = row0 + i * 8 + gr, c = col0 + j * 8 + 2 * gc;
       out[r * D + c] = acc[i][j][0];
       out[r * D + c + 1] = acc[i][j][1];
-      out[(r + 8) * D + c] = acc[i][j][2];
-      out[(r + 8) * D + c + 1] = acc[i][j][3];
     }
 }
 
 // gram[h][i][j] = sum over splits s (in order) of partial[h][s][i][j], in fp64
-__global__ void __launch_bounds__(256) gram_reduce_kernel(const float* partial, double* gram, int64_t n_heads,
+__global__ void __launch_bounds__(256) gram_reduce_kernel(const double* partial, double* gram, int64_t n_heads,
                                                           int splits, int dd) {
   const int64_t total = n_heads * dd;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
     const int64_t h = e / dd, ij = e % dd;
     double s = 0.0;
-    for (int t = 0; t < splits; ++t) s += (double)partial[(h * splits + t) * dd + ij];
+    for (int t = 0; t < splits; ++t) s += partial[(h * splits + t) * dd + ij];
     gram[e] = s;
   }
 }
