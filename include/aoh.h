@@ -146,7 +146,7 @@ int32_t aoh_last_cuda_error(void);
 typedef enum {
   AOH_KERNEL_TIP_SCORE = 0,     /* stand-alone importance scan                       */
   AOH_KERNEL_SELECT_HIST = 1,   /* select: first-digit histograms of given scores    */
-  AOH_KERNEL_SPARSE_ROW = 2,    /* fused row kernel, or its select-only form         */
+  AOH_KERNEL_SPARSE_ROW = 2,    /* fused row kernel                                  */
   AOH_KERNEL_FLASH_GATHER = 3,  /* split-K gather / window attention                 */
   AOH_KERNEL_PACK_DOMINANT = 4, /* dominant-column packing of K                      */
   AOH_KERNEL_KV_APPEND = 5,     /* rotation and append of a decoded token            */
@@ -158,7 +158,8 @@ typedef enum {
   AOH_KERNEL_OFFLOAD_SPLIT = 11,  /* host offload: a device cache split to host parts */
   AOH_KERNEL_SELECT_CHUNK = 12, /* select: threshold bin, candidates, exact threshold */
   AOH_KERNEL_SELECT_WRITE = 13, /* select: ordered write of the chosen positions     */
-  AOH_KERNEL_KINDS = 14
+  AOH_KERNEL_SELECT_CLUSTER = 14, /* select: one cluster per row, keys on chip      */
+  AOH_KERNEL_KINDS = 15
 } aoh_kernel_kind;
 
 /*
@@ -247,10 +248,14 @@ aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* k
  *                   bytes, zero-filled once before its first use (every call
  *                   leaves its counters at zero again)
  * Rows up to 4 M positions (AOH_ERR_UNSUPPORTED beyond).  Deterministic: the
- * same input gives the same bits.  Mechanism: per row, a histogram of the top
- * 11 bits of the order-preserving keys, then chunks of 4096 keys in parallel
- * (keys above the threshold bin counted, keys in it collected, the exact
- * threshold resolved once per row, every chunk's picks written in order).
+ * same input gives the same bits.  Mechanism, on order-preserving uint32 keys:
+ * rows of at most 128 K positions take one launch, one thread-block cluster
+ * per row with the row's keys on chip (MSB radix select with 11-, 11- and
+ * 10-bit digits, histograms summed across the cluster through distributed
+ * shared memory, picks written in order); longer rows take three launches (a
+ * histogram of the top 11 bits, then chunks of 4096 keys in parallel: keys
+ * above the threshold bin counted, keys in it collected, the exact threshold
+ * resolved once per row, every chunk's picks written in order).
  */
 aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
                            const int32_t* n_fac_per_seq, int32_t n_fac_cap,

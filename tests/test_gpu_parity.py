@@ -127,18 +127,8 @@ def test_topk_bit_exact_on_given_scores(kind):
             assert np.all(idx_h[b, g, n:] == -1)
 
 
-@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
-def test_topk_many_rows(kind):
-    # 54 sequences x 3 KV heads = 162 rows of many chunks.  Lengths mix empty, one-token,
-    # N_fac >= L and long rows; the ties / zeros kinds put more candidates in the threshold
-    # bin than the resolving CTA keeps in shared memory (it then reads them from the list).
-    rng = np.random.default_rng(15)
-    lengths = [0, 1, 3, 700, 24000, 60000] + [int(x) for x in rng.integers(50, 9000, 48)]
-    Hkv = 3
-    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
-    s = given_scores(rng, lengths, Hkv, kind)
-    nfps = np.array([4, 1, 9, 700, 2048, 1500] + [int(x) for x in rng.integers(1, 2049, 48)], dtype=np.int32)
-    cap = 2048
+def check_topk(s, offs, lengths, nfps, cap, expect_launches, kind):
+    Hkv = s.shape[0]
     dev = torch.device("cuda")
     k = torch.zeros((int(offs[-1]), Hkv, 64), dtype=torch.bfloat16, device=dev)
     kv = B.make_kv(k, k, torch.from_numpy(offs).to(dev), max(lengths), int(offs[-1]))
@@ -146,7 +136,7 @@ def test_topk_many_rows(kind):
     cnt = torch.full((len(lengths), Hkv), -7, dtype=torch.int32, device=dev)
     sd, nd = torch.from_numpy(s).to(dev), torch.from_numpy(nfps).to(dev)
     launched = launches_of(lambda: B.topk_select(sd, kv, 0, nd, cap, idx, cnt))
-    assert launched == {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_write_kernel": 1}
+    assert launched == expect_launches
     check_device()
     idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
     for b, L in enumerate(lengths):
@@ -158,164 +148,60 @@ def test_topk_many_rows(kind):
             assert np.all(idx_h[b, g, n:] == -1), (kind, b, g)
 
 
-def test_topk_fixed_nfac_and_determinism():
-    rng = np.random.default_rng(6)
-    lengths = [131072, 4096, 777]
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
+def test_topk_many_rows(kind):
+    # 54 sequences x 3 KV heads = 162 rows, up to 60000 positions: more 8-CTA clusters than
+    # one wave holds, so the chunked select runs.  Lengths mix empty, one-token, N_fac >= L
+    # and long rows; the ties / zeros kinds leave many keys equal to the threshold, so the
+    # lowest positions among them decide.
+    rng = np.random.default_rng(15)
+    lengths = [0, 1, 3, 700, 24000, 60000] + [int(x) for x in rng.integers(50, 9000, 48)]
+    Hkv = 3
     offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
-    s = (np.round(rng.standard_normal((2, int(offs[-1]))) * 8) / 8).astype(np.float32)
-    dev = torch.device("cuda")
-    k = torch.zeros((int(offs[-1]), 2, 64), dtype=torch.bfloat16, device=dev)
-    kv = B.make_kv(k, k, torch.from_numpy(offs).to(dev), max(lengths), int(offs[-1]))
-    sd = torch.from_numpy(s).to(dev)
-    outs = []
-    for _ in range(2):
-        idx = torch.empty((3, 2, 2048), dtype=torch.int32, device=dev)
-        cnt = torch.empty((3, 2), dtype=torch.int32, device=dev)
-        B.topk_select(sd, kv, 2048, None, 2048, idx, cnt)
-        torch.cuda.synchronize()
-        outs.append((idx.cpu().numpy(), cnt.cpu().numpy()))
-    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
-    for b in range(3):
-        for g in range(2):
-            ref = oracle.select_top(s[g, offs[b]:offs[b + 1]], 2048)
-            assert np.array_equal(outs[0][0][b, g, :len(ref)], ref)
+    s = given_scores(rng, lengths, Hkv, kind)
+    nfps = np.array([4, 1, 9, 700, 2048, 1500] + [int(x) for x in rng.integers(1, 2049, 48)], dtype=np.int32)
+    check_topk(s, offs, lengths, nfps, 2048,
+               {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_write_kernel": 1}, kind)
 
 
-# ------------------------------------------------------------------------------ sparse decode
-
-@pytest.mark.parametrize("name", list(MEDIUM))
-@pytest.mark.parametrize("pack", [True, False])
-def test_sparse_decode_matches_oracle(name, pack):
-    w = make_workload(MEDIUM[name])
-    d = Dev(w)
-    step, out = run_sparse(d, pack=pack)
-    # a few rows: the whole path in one cluster launch
-    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
-    out_h = f64(out)
-    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
-    G = w.spec.group
-    stats = {}
-    for b in range(w.spec.batch):
-        for g in range(w.spec.n_kv_heads):
-            n = cnt_h[b, g]
-            compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G], stats)
-    assert stats["swapped"] <= max(1, stats["rows"] // 10)
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
+def test_topk_rows_in_clusters(kind):
+    # 6 sequences x 3 KV heads = 18 rows up to 60000 positions: one wave of 8-CTA clusters,
+    # the on-chip select (same score kinds as above)
+    rng = np.random.default_rng(18)
+    lengths = [0, 3, 700, 24000, 60000, 51234]
+    Hkv = 3
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = given_scores(rng, lengths, Hkv, kind)
+    nfps = np.array([4, 9, 700, 2048, 1500, 1], dtype=np.int32)
+    check_topk(s, offs, lengths, nfps, 2048, {"select_cluster_kernel": 1}, kind)
 
 
-def test_sparse_decode_is_deterministic():
-    w = make_workload(MEDIUM["gqa4_d128"])
-    d = Dev(w)
-    step, out = run_sparse(d)
-    first = out.clone()
-    step(d.q)
-    torch.cuda.synchronize()
-    assert torch.equal(first, step.out)
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
+def test_topk_long_rows_chunked(kind):
+    # rows beyond one cluster's 128 K positions take the chunked select (histogram, chunk pass,
+    # ordered write); the ties / zeros kinds put more candidates in the threshold bin than
+    # the resolving CTA keeps in shared memory (it then reads them from the list)
+    rng = np.random.default_rng(16)
+    lengths = [131073, 0, 5, 200000, 2000, 140000]
+    Hkv = 2
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = given_scores(rng, lengths, Hkv, kind)
+    nfps = np.array([3000, 4, 9, 2048, 2500, 1], dtype=np.int32)
+    check_topk(s, offs, lengths, nfps, 3000,
+               {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_write_kernel": 1}, kind)
 
 
-# ------------------------------------------------------------------------------ retrieval / streaming heads
-
-@pytest.mark.parametrize("sink,window", [(4, 60), (128, 512), (0, 100), (3000, 4000), (0, 0)])
-def test_stream_decode_matches_oracle(sink, window):
-    roles = (ROLE_DENSE, ROLE_STREAM, ROLE_STREAM, ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_STREAM, ROLE_STREAM)
-    w = make_workload(spec(roles=roles, sink=sink, window=window, len_range=(0, 7000), seed=81))
-    d = Dev(w)
-    kv = d.kv()
-    out = torch.full((w.spec.batch, w.spec.n_q_heads, w.spec.head_dim), 777.0, device="cuda")
-    ws = B.workspace(B.stream_decode_workspace_size(kv, w.spec.n_q_heads, roles, sink, window), "cuda")
-    B.stream_decode(d.q, kv, roles, sink, window, w.scale, out, ws)
-    torch.cuda.synchronize()
-    check_device()
-    out_h = f64(out)
-    G = w.spec.group
-    for b in range(w.spec.batch):
-        for g, role in enumerate(roles):
-            rows = out_h[b, g * G:(g + 1) * G]
-            if role == ROLE_SPARSE:
-                assert np.all(rows == 777.0)   # not this call's heads: untouched
-            else:
-                compare_window_row(w, b, g, rows, role, sink, window)
-
-
-def test_full_role_split_step_mixed_heads():
-    # every row in one wave and window lists no longer than 4 x N_fac: the whole step, window
-    # heads included, is one launch of the row kernel
-    roles = (ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_SPARSE)
-    w = make_workload(spec(n_q_heads=16, n_kv_heads=4, roles=roles, sink=16, window=200, n_fac_div=4, seed=82))
-    d = Dev(w)
-    step, out = run_sparse(d)
-    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
-    out_h = f64(out)
-    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
-    G = w.spec.group
-    for b in range(w.spec.batch):
-        for g, role in enumerate(roles):
-            rows = out_h[b, g * G:(g + 1) * G]
-            if role == ROLE_SPARSE:
-                compare_sparse_row(w, b, g, idx_h[b, g, :cnt_h[b, g]], rows)
-            else:
-                compare_window_row(w, b, g, rows, role, w.spec.sink, w.spec.window)
-
-
-# ------------------------------------------------------------------------------ shared index
-
-@pytest.mark.parametrize("fused", [True, False])
-@pytest.mark.parametrize("n_layers,hq,hkv", [(8, 32, 8), (2, 16, 4), (3, 16, 4), (1, 8, 8)])
-def test_shared_index_decode_matches_oracle(n_layers, hq, hkv, fused):
-    sp = WorkloadSpec(name="shared", batch=2, n_q_heads=hq, n_kv_heads=hkv, head_dim=128, theta=5e5,
-                      len_range=(500, 9000), n_layers=n_layers, topk_shared=700, seed=90 + n_layers)
-    w = make_workload(sp)
-    d = Dev(w)
-    step, out = run_shared(d, fused=fused)
-    out_h = f64(out)
-    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
-    G = sp.group
-    ref = oracle.shared_index_step(f64(w.q), f64(w.q_layers), f64(w.k), f64(w.v), w.offsets.tolist(), 700,
-                                   w.scale)
-    for (b, g), r in ref.items():
-        sel = idx_h[b, g, :cnt_h[b, g]]
-        compare_shared_row(w, b, g, sel, out_h[:, b, g * G:(g + 1) * G], 700)
-        if np.array_equal(sel, r["sel"]):  # the stack's own oracle on the same index
-            assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= OUT_ATOL
-
-
-def test_shared_index_reports_out_of_range_positions():
-    sp = WorkloadSpec(name="shared", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, theta=1e4,
-                      lengths=(300,), n_layers=2, topk_shared=16, seed=3)
-    w = make_workload(sp)
-    d = Dev(w)
-    kv = d.kv()
-    idx = torch.arange(16, dtype=torch.int32, device="cuda").repeat(1, 2, 1).contiguous()
-    idx[0, 1, 5] = 300            # one past the end of the sequence
-    cnt = torch.full((1, 2), 16, dtype=torch.int32, device="cuda")
-    out = torch.empty((2, 1, 8, 64), device="cuda")
-    ws = B.workspace(B.shared_index_decode_workspace_size(kv, 2, 8, 16), "cuda")
-    B.shared_index_decode(d.q_layers, kv, idx, cnt, 16, w.scale, out, ws)
-    st, detail = B.device_check()
-    assert st == 6 and detail[0] == 1 and detail[3] == 300
-    assert B.device_check()[0] == 0   # reading clears the word
-    assert torch.isfinite(out).all()
-
-
-# ------------------------------------------------------------------------------ edge cases
-
-def test_edge_cases_empty_and_short_sequences():
-    sp = spec(batch=5, lengths=(0, 1, 2, 64, 65), len_range=None, n_fac_div=0, n_fac=64, n_dom=3,
-              planted_frac=0.0, seed=84)
-    w = make_workload(sp)
-    d = Dev(w)
-    step, out = run_sparse(d)
-    out_h = f64(out)
-    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
-    G = sp.group
-    for b in range(sp.batch):
-        for g in range(sp.n_kv_heads):
-            n = cnt_h[b, g]
-            assert n == min(64, int(w.lengths[b]))
-            if w.lengths[b] == 0:
-                assert np.all(out_h[b, g * G:(g + 1) * G] == 0.0)
-            else:
-                compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G])
-            assert np.all(idx_h[b, g, n:] == -1)
+@pytest.mark.parametrize("L", [1, 8191, 8192, 8193, 65536, 131072])
+def test_topk_cluster_slice_edges(L):
+    # row lengths at the edges of the cluster sizes (8192 positions per CTA): a slice that is
+    # full, one position over (the next cluster size), and the largest row one cluster takes
+    rng = np.random.default_rng(17 + L)
+    lengths = [L, max(1, L // 3)]
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = given_scores(rng, lengths, 2, "normal")
+    nfps = np.array([min(2048, max(1, L - 1)), min(2048, max(1, L // 5))], dtype=np.int32)
+    check_topk(s, offs, lengths, nfps, 2048, {"select_cluster_kernel": 1}, "normal")
 
 
 def test_sparse_decode_long_row_uses_three_kernels():
@@ -347,7 +233,7 @@ def test_sparse_decode_every_token_selected():
 
 def test_sparse_decode_many_rows_runs_three_stages():
     # 40 sequences x 8 KV heads = 320 rows: more clusters than one wave holds, so the step
-    # runs as scan kernel (with the select's histograms) + chunked select + split-K gather
+    # runs as scan kernel + select (cluster or chunked) + split-K gather
     sp = spec(batch=40, len_range=(300, 3000), seed=87)
     w = make_workload(sp)
     d = Dev(w)
@@ -359,7 +245,9 @@ def test_sparse_decode_many_rows_runs_three_stages():
                                                    step.out, step.ws, step.idx, step.count))
     torch.cuda.synchronize()
     names = [k for k, _, _ in rec]
-    assert names == ["tip_score_kernel", "select_chunk_kernel", "select_write_kernel", "flash_gather_kernel"]
+    assert names in (["tip_score_kernel", "select_cluster_kernel", "flash_gather_kernel"],
+                     ["tip_score_kernel", "select_hist_kernel", "select_chunk_kernel", "select_write_kernel",
+                      "flash_gather_kernel"])
     assert all(e0.elapsed_time(e1) > 0 for _, e0, e1 in rec)
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()

@@ -16,6 +16,7 @@
 #include "head_classify.cuh"
 #include "kv_append.cuh"
 #include "offload.cuh"
+#include "select_cluster.cuh"
 #include "select_hist.cuh"
 #include "sparse_row.cuh"
 #include "tip_score.cuh"
@@ -199,6 +200,36 @@ void fd_bind(FdecParams& fp, const FdGeom& g, uint8_t* ws) {
   fp.max_splits = g.max_splits;
 }
 
+// Launch of a kernel that follows another one of the same call on the stream: programmatic
+// dependent launch lets it be scheduled while that kernel drains (the kernel itself waits for
+// it with griddepcontrol.wait before touching memory); cl > 0 adds a cluster dimension.
+constexpr int kDependentLaunch = 1;
+
+template <typename K, typename P>
+aoh_status launch_dependent(K kern, dim3 grid, int threads, size_t smem, int cl, cudaStream_t st, const P& params) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (cl > 0) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cl;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = kDependentLaunch;
+  ++na;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  before_launch(st);
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, params));
+}
+
 template <typename K>
 int max_active_clusters(K kern, int CL, size_t smem, int threads = kSrThreads) {
   // (cluster size, dynamic shared memory) -> cudaOccupancyMaxActiveClusters, cached per process
@@ -251,28 +282,11 @@ aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStr
   // rows of about equal length with 2..16 splits: one cluster per row, merged on chip
   const int CL = fp.max_splits;
   constexpr int threads = fd_threads(NT);
-  if (uniform && CL >= 2 && CL <= kFdMaxCluster && max_active_clusters(kern, CL, smem, threads) > 0) {
-    fp.cluster_combine = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    before_launch(st);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, fp);
-    if (e != cudaSuccess) return cuda_status(e);
-    return count_launch(AOH_KERNEL_FLASH_GATHER, st);
-  }
-  fp.cluster_combine = 0;
-  before_launch(st);
-  kern<<<grid, threads, smem, st>>>(fp);
+  const bool merge_on_chip =
+      uniform && CL >= 2 && CL <= kFdMaxCluster && max_active_clusters(kern, CL, smem, threads) > 0;
+  fp.cluster_combine = merge_on_chip ? 1 : 0;
+  const aoh_status s = launch_dependent(kern, grid, threads, smem, merge_on_chip ? CL : 0, st, fp);
+  if (s != AOH_OK) return s;
   return count_launch(AOH_KERNEL_FLASH_GATHER, st);
 }
 
@@ -309,9 +323,8 @@ aoh_status launch_tip_t(TipParams& tp, cudaStream_t st) {
 }
 
 aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const int32_t* idom, int32_t n_dom,
-                      float* scores, const uint8_t* heads, int n_listed, cudaStream_t st, uint32_t* hist = nullptr) {
+                      float* scores, const uint8_t* heads, int n_listed, cudaStream_t st) {
   TipParams tp{};
-  tp.hist = hist;
   tp.q = static_cast<const uint16_t*>(q);
   tp.idom = idom;
   tp.offsets = kv->offsets;
@@ -355,16 +368,16 @@ aoh_status launch_tip(const void* q, int32_t Hq, const aoh_kv_cache* kv, const i
 
 // Full-dimension scores (every chunk; the shared indexer's score), K read in place.
 aoh_status launch_tip_full(const void* q, int32_t Hq, const aoh_kv_cache* kv, float* scores, const uint8_t* heads,
-                           int n_listed, cudaStream_t st, uint32_t* hist = nullptr) {
-  return launch_tip(q, Hq, kv, nullptr, kv->head_dim / 2, scores, heads, n_listed, st, hist);
+                           int n_listed, cudaStream_t st) {
+  return launch_tip(q, Hq, kv, nullptr, kv->head_dim / 2, scores, heads, n_listed, st);
 }
 
 // ------------------------------------------------------------------ chunked select
-// Workspace of the select (after the scores): [hist][cand_count][tickets] first (these must
-// start at zero and every select leaves them at zero), then the candidate list, the chunk
-// counts and offsets, and the row results.
+// Workspace of the select (after the scores): the histograms first (they must start at zero
+// and every select leaves them at zero), then the candidate counts and list, the chunk counts
+// and the row results.
 struct SelectWs {
-  size_t hist, cand_count, tickets, cand, chunk_above, chunk_info, row_info, total;
+  size_t hist, cand_count, cand, chunk_above, row_info, total;
   int max_chunks;
 };
 
@@ -377,14 +390,10 @@ SelectWs select_ws(const aoh_kv_cache* kv) {
   o += align256(rows * kSelHistBins * sizeof(uint32_t));
   w.cand_count = o;
   o += align256(rows * sizeof(int32_t));
-  w.tickets = o;
-  o += align256(rows * sizeof(int32_t));
   w.cand = o;
   o += align256((size_t)kv->n_kv_heads * (size_t)std::max<int64_t>(kv->total_tokens, 1) * sizeof(unsigned long long));
   w.chunk_above = o;
   o += align256(rows * w.max_chunks * sizeof(int32_t));
-  w.chunk_info = o;
-  o += align256(rows * w.max_chunks * 2 * sizeof(int32_t));
   w.row_info = o;
   o += align256(rows * 2 * sizeof(int32_t));
   w.total = o;
@@ -393,11 +402,11 @@ SelectWs select_ws(const aoh_kv_cache* kv) {
 
 bool select_fits(const aoh_kv_cache* kv) { return ceil_div(std::max(kv->max_len, 1), kSelChunk) <= kSelMaxChunks; }
 
-// The select on the scores: the first-digit histograms (unless the scan built them), the chunk
-// pass and the ordered write.  `ws` is the select's region (layout of select_ws).
+// The chunked select on the scores: the first-digit histograms, the chunk pass and the
+// ordered write.  `ws` is the select's region (layout of select_ws).
 aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
                                int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
-                               uint8_t* ws, bool hist_ready, cudaStream_t st) {
+                               uint8_t* ws, cudaStream_t st) {
   if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
   const SelectWs w = select_ws(kv);
   HistSelectParams hp{};
@@ -408,9 +417,7 @@ aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int3
   hp.hist = reinterpret_cast<uint32_t*>(ws + w.hist);
   hp.cand = reinterpret_cast<unsigned long long*>(ws + w.cand);
   hp.cand_count = reinterpret_cast<int32_t*>(ws + w.cand_count);
-  hp.tickets = reinterpret_cast<int32_t*>(ws + w.tickets);
   hp.chunk_above = reinterpret_cast<int32_t*>(ws + w.chunk_above);
-  hp.chunk_info = reinterpret_cast<int32_t*>(ws + w.chunk_info);
   hp.row_info = reinterpret_cast<int32_t*>(ws + w.row_info);
   hp.idx = idx;
   hp.count = count;
@@ -423,17 +430,62 @@ aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int3
   memcpy(hp.heads, heads, n_listed);
   const dim3 grid(w.max_chunks, n_listed, kv->batch);
   aoh_status s;
-  if (!hist_ready && kv->total_tokens > 0) {
-    before_launch(st);
-    select_hist_kernel<<<grid, kSelCtaThreads, 0, st>>>(hp);
+  if (kv->total_tokens > 0) {
+    if ((s = launch_dependent(select_hist_kernel, grid, kSelCtaThreads, 0, 0, st, hp)) != AOH_OK) return s;
     if ((s = count_launch(AOH_KERNEL_SELECT_HIST, st)) != AOH_OK) return s;
   }
-  before_launch(st);
-  select_chunk_kernel<<<grid, kSelCtaThreads, 0, st>>>(hp);
+  if ((s = launch_dependent(select_chunk_kernel, grid, kSelCtaThreads, 0, 0, st, hp)) != AOH_OK) return s;
   if ((s = count_launch(AOH_KERNEL_SELECT_CHUNK, st)) != AOH_OK) return s;
-  before_launch(st);
-  select_write_kernel<<<grid, kSelCtaThreads, 0, st>>>(hp);
+  if ((s = launch_dependent(select_write_kernel, grid, kSelCtaThreads, 0, 0, st, hp)) != AOH_OK) return s;
   return count_launch(AOH_KERNEL_SELECT_WRITE, st);
+}
+
+// Cluster size of the on-chip select: the smallest power of two whose slices of
+// kScSlice positions hold the longest row; 0 when none does.
+int select_cluster_size(const aoh_kv_cache* kv) {
+  const int64_t L = std::max(kv->max_len, 1);
+  for (int cl = 1; cl <= kScMaxCluster; cl *= 2)
+    if (L <= int64_t(cl) * kScSlice) return cl;
+  return 0;
+}
+
+// The select on the scores: one cluster per row, on chip, when every row's cluster runs in
+// one wave; else the chunked select, which spreads every row over all SMs (measured: the
+// 128K shared-index rows, whose 16 clusters of 16 CTAs need two waves, and the 256 serving
+// rows select faster chunked; 32 rows of 32K faster in clusters).  Both take the same
+// workspace region.
+aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps, int32_t cap,
+                         int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed, uint8_t* ws,
+                         cudaStream_t st) {
+  const int CL = select_cluster_size(kv);
+  if (CL > 0) {
+    auto kern = select_cluster_kernel;
+    static std::atomic<uint64_t> configured{0};
+    if (!set_up_on_this_device(configured)) {
+      const aoh_status s = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+      if (s != AOH_OK) return s;
+      mark_set_up(configured);
+    }
+    const int maxc = max_active_clusters(kern, CL, 0, kScThreads);
+    if (maxc > 0 && int64_t(n_listed) * kv->batch <= maxc) {
+      ClusterSelectParams cp{};
+      cp.scores = scores;
+      cp.offsets = kv->offsets;
+      cp.lengths = kv->lengths;
+      cp.n_fac_per_seq = nfps;
+      cp.idx = idx;
+      cp.count = count;
+      cp.T = (int32_t)kv->total_tokens;
+      cp.Hkv = kv->n_kv_heads;
+      cp.n_fac = n_fac;
+      cp.cap = cap;
+      memcpy(cp.heads, heads, n_listed);
+      const aoh_status s = launch_dependent(kern, dim3(CL, n_listed, kv->batch), kScThreads, 0, CL, st, cp);
+      if (s != AOH_OK) return s;
+      return count_launch(AOH_KERNEL_SELECT_CLUSTER, st);
+    }
+  }
+  return launch_chunk_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, ws, st);
 }
 
 // ------------------------------------------------------------------ fused row kernel
@@ -770,8 +822,8 @@ aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t 
   if (!ws_ok(workspace, workspace_bytes, select_ws(kv).total)) return AOH_ERR_WORKSPACE;
   uint8_t heads[kMaxHeads];
   const int n = list_heads(kv, nullptr, true, heads);
-  return launch_chunk_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n,
-                             static_cast<uint8_t*>(workspace), false, as_stream(stream));
+  return launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, count, heads, n,
+                       static_cast<uint8_t*>(workspace), as_stream(stream));
 }
 
 size_t aoh_sparse_decode_workspace_size(const aoh_kv_cache* kv, int32_t n_q_heads, int32_t n_fac_cap) {
@@ -844,15 +896,14 @@ aoh_status aoh_sparse_decode(const void* q, int32_t n_q_heads, const aoh_kv_cach
     if (launched) return AOH_OK;
   }
 
-  // otherwise: the scan over all SMs (with the rows' first-digit histograms), the chunked
-  // select on the (L2-resident) scores, and the split-K gather
+  // otherwise: the scan over all SMs, the select on the (L2-resident) scores, and the
+  // split-K gather
   if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
   uint8_t* sel_ws = ws + off_count + align256(sizeof(int32_t) * (size_t)kv->batch * kv->n_kv_heads);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sel_ws + select_ws(kv).hist);
   if (kv->total_tokens > 0) {
-    if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st, hist)) != AOH_OK) return s;
+    if ((s = launch_tip(q, n_q_heads, kv, idom, n_dom, scores, heads, n_listed, st)) != AOH_OK) return s;
   }
-  s = launch_chunk_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, sel_ws, true, st);
+  s = launch_select(scores, kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, n_listed, sel_ws, st);
   if (s != AOH_OK) return s;
 
   const FdGeom geo = sparse_geom(kv, n_q_heads, n_fac_cap);
@@ -1138,15 +1189,13 @@ aoh_status aoh_shared_index_step(const void* q_index, const void* q_layers, int3
     if ((s = launch_rows(rp, kv, n_layers * G, n_listed, kv->batch, st, 1, &launched)) != AOH_OK) return s;
     if (launched) return AOH_OK;
   }
-  // otherwise: full-dimension scores (with the first-digit histograms), the chunked select,
-  // the shared-index gather
+  // otherwise: full-dimension scores, the select, the shared-index gather
   if (!select_fits(kv)) return AOH_ERR_UNSUPPORTED;
   uint8_t* sel_ws = ws + fd_bytes(geo) + shared_step_scores_bytes(kv);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(sel_ws + select_ws(kv).hist);
   if (kv->total_tokens > 0) {
-    if ((s = launch_tip_full(q_index, n_q_heads, kv, scores, heads, n_listed, st, hist)) != AOH_OK) return s;
+    if ((s = launch_tip_full(q_index, n_q_heads, kv, scores, heads, n_listed, st)) != AOH_OK) return s;
   }
-  s = launch_chunk_select(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, sel_ws, true, st);
+  s = launch_select(scores, kv, topk, nullptr, topk, idx, count, heads, n_listed, sel_ws, st);
   if (s != AOH_OK) return s;
   FdecParams fp{};
   fp.q = static_cast<const uint16_t*>(q_layers);
@@ -1524,11 +1573,10 @@ extern "C" aoh_status aoh_offload_decode(const void* q, int32_t n_q_heads, const
   cudaStream_t st = as_stream(stream);
   // 1-2. importance scan of the dominant columns (on the GPU) and the top-N_fac select
   if (!select_fits(&kv)) return AOH_ERR_UNSUPPORTED;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(ws + wl.sel + select_ws(&kv).hist);
-  if (kv.total_tokens > 0 && (s = launch_tip(q, n_q_heads, &kv, idom, n_dom, scores, heads, Hkv, st, hist)) != AOH_OK)
+  if (kv.total_tokens > 0 && (s = launch_tip(q, n_q_heads, &kv, idom, n_dom, scores, heads, Hkv, st)) != AOH_OK)
     return s;
-  if ((s = launch_chunk_select(scores, &kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, Hkv, ws + wl.sel, true,
-                               st)) != AOH_OK)
+  if ((s = launch_select(scores, &kv, n_fac, n_fac_per_seq, n_fac_cap, idx, cnt, heads, Hkv, ws + wl.sel, st)) !=
+      AOH_OK)
     return s;
   // 3. the selected rows across the host link, into HBM
   StageParams sp{};

@@ -146,6 +146,15 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may be scheduled while the kernel
+// before it on the stream is still running.  grid_dep_wait() blocks until that kernel has
+// completed and its writes are visible (a no-op when the launch has no such dependency);
+// every kernel launched that way calls it before it reads or writes global memory.
+// grid_dep_launch() lets the next such launch begin scheduling its CTAs.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ------------------------------------------------------------------ split cluster barrier
 __device__ __forceinline__ void cluster_arrive_release() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");

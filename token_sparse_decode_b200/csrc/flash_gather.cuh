@@ -89,6 +89,8 @@ __device__ __forceinline__ uint32_t fd_tile_off(int r, int dd) {
 
 template <int D, int NT>
 __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const FdecParams p) {
+  grid_dep_wait();  // the selection comes from the kernel before this one
+  grid_dep_launch();
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
   constexpr int KS = D / 16;         // k-steps of QK, m-tiles of PV
@@ -372,25 +374,58 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
       }
     }
     cluster.sync();
+    // every peer's (M, L) of a query row: all remote loads issued before any is used
     if (tid < NQP) {
+      float mv[kFdMaxCluster], lv[kFdMaxCluster];
+#pragma unroll
+      for (int q = 0; q < kFdMaxCluster; ++q) {
+        mv[q] = q < CLn ? cluster.map_shared_rank(cm, q)[tid] : -INFINITY;
+        lv[q] = q < CLn ? cluster.map_shared_rank(cls, q)[tid] : 0.f;
+      }
       float Mx = -INFINITY;
-      for (int q = 0; q < CLn; ++q) Mx = fmaxf(Mx, cluster.map_shared_rank(cm, q)[tid]);
+#pragma unroll
+      for (int q = 0; q < kFdMaxCluster; ++q) Mx = fmaxf(Mx, mv[q]);
       float Ls = 0.f;
-      for (int q = 0; q < CLn; ++q) {
-        const float mq = cluster.map_shared_rank(cm, q)[tid];
-        const float w = (mq == -INFINITY) ? 0.f : exp2f(mq - Mx);
-        cw[q * NQP + tid] = w;
-        Ls += w * cluster.map_shared_rank(cls, q)[tid];
+#pragma unroll
+      for (int q = 0; q < kFdMaxCluster; ++q) {
+        if (q < CLn) {
+          const float w = (mv[q] == -INFINITY) ? 0.f : exp2f(mv[q] - Mx);
+          cw[q * NQP + tid] = w;
+          Ls += w * lv[q];
+        }
       }
       cinv[tid] = 1.f / Ls;
     }
     __syncthreads();
-    for (int e = rk * kFdThreads + tid; e < p.NQ * D; e += CLn * kFdThreads) {
-      const int qr = e / D, dd = e % D;
-      float A = 0.f;
-      for (int q = 0; q < CLn; ++q) A += cw[q * NQP + qr] * cluster.map_shared_rank(ca, q)[e];
+    // outputs 4 consecutive dims at a time, 16-byte reads of the peers' partials, 4 peers' reads
+    // in flight together; the peers are summed in rank order
+    for (int e4 = rk * kFdThreads + tid; e4 < p.NQ * D / 4; e4 += CLn * kFdThreads) {
+      const int e = 4 * e4, qr = e / D, dd = e % D;
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q0 = 0; q0 < CLn; q0 += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          v[u] = q0 + u < CLn ? *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, q0 + u) + e)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (q0 + u < CLn) {
+            const float w = cw[(q0 + u) * NQP + qr];
+            A.x += w * v[u].x;
+            A.y += w * v[u].y;
+            A.z += w * v[u].z;
+            A.w += w * v[u].w;
+          }
+        }
+      }
+      const float sc = cinv[qr];
       const int l = qr / p.G, h = g * p.G + qr % p.G;
-      p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A * cinv[qr];
+      float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
+      o[0] = A.x * sc;
+      o[1] = A.y * sc;
+      o[2] = A.z * sc;
+      o[3] = A.w * sc;
     }
     cluster.sync();  // peers read this CTA's shared memory until here
     return;

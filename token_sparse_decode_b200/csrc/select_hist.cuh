@@ -6,23 +6,28 @@
 // The selection of a (sequence b, KV head g) row is {key > K_T} plus the lowest
 // positions among {key == K_T}, n in all, written in ascending position order.
 //
-// First digit: the top 11 bits of a key (sign, exponent, two mantissa bits).  The row's
-// histogram of it comes from the importance scan (which counts each score as it writes
-// it) or, on caller-given scores, from select_hist_kernel.  Then, with chunks of
-// kSelChunk keys of a row, one CTA each:
-//   select_chunk_kernel  finds the bin T1 holding the n-th key from the histogram, counts
-//                        the chunk's keys above T1 and appends the chunk's keys in T1
-//                        (key, position) to the row's candidate list.  The last CTA of the
-//                        row (atomic ticket) resolves K_T among the candidates with the
-//                        remaining 21 bits (digits of 8, 8 and 5 bits), counts per chunk the
-//                        candidates above and equal to K_T, and turns all counts into every
-//                        chunk's output offset and number of equal keys before it; it then
-//                        re-arms the histogram, the candidate count and the ticket to zero;
-//   select_write_kernel  every chunk writes its selected positions at its offset, in order:
-//                        warps own runs of 32 x kWriteK consecutive keys, ballots rank the
-//                        picks inside a warp, one block scan ranks the warps.
-// A row with n >= L_b takes every position without a select.  Deterministic: the
-// candidate list's order varies between runs, the counts drawn from it do not.
+// First digit: the top 11 bits of a key (sign, exponent, two mantissa bits).  With chunks
+// of kSelChunk keys of a row, one CTA each, three launches:
+//   select_hist_kernel   counts the chunk's first digits in shared memory and adds the
+//                        non-empty bins into the row's histogram (chunk 0 also clears the
+//                        row's candidate count);
+//   select_chunk_kernel  finds the bin T1 holding the n-th key from the histogram (chunk 0
+//                        records T1 and the keys above it for the row), counts the chunk's
+//                        keys above T1 and appends the chunk's keys in T1 (key, position) to
+//                        the row's candidate list (one atomic per CTA reserves the chunk's
+//                        run of the list);
+//   select_write_kernel  every chunk resolves K_T from the row's candidates on its own (the
+//                        remaining 21 bits, digits of 8, 8 and 5, over the candidates in
+//                        shared memory), counts the keys the chunks before it take (their
+//                        keys above T1 plus their candidates above or equal to K_T), and
+//                        writes its selected positions at that offset, in order: warps own
+//                        runs of 32 x kWriteK consecutive keys, ballots rank the picks inside
+//                        a warp, one block scan ranks the warps.  Chunk 0 re-arms the row's
+//                        histogram to zero.
+// No CTA waits for another and no CTA resolves for the others: every dependency is a kernel
+// boundary.  Every kernel issues all of its key loads before it uses any.  A row with
+// n >= L_b takes every position without a select.  Deterministic: the candidate list's order
+// varies between runs, the counts drawn from it do not.
 #pragma once
 
 #include "device_common.cuh"
@@ -33,9 +38,9 @@ constexpr int kSelChunk = 4096;        // keys of a row per CTA
 constexpr int kSelHistBins = 2048;     // first digit: the top 11 bits of a key
 constexpr int kSelHistShift = 21;
 constexpr int kSelCtaThreads = 256;
-constexpr int kWriteK = kSelChunk / kSelCtaThreads;  // keys per lane in the write pass (16)
+constexpr int kWriteK = kSelChunk / kSelCtaThreads;  // keys per lane (16)
 constexpr int kSelMaxChunks = 1024;    // chunks per row: rows up to 4 M keys
-constexpr int kSelResolveCap = 8192;   // candidates the last CTA keeps in shared memory
+constexpr int kSelResolveCap = 4096;   // candidates a CTA keeps in shared memory (more: read from L2)
 
 struct HistSelectParams {
   const float* scores;          // [Hkv][T]
@@ -44,11 +49,9 @@ struct HistSelectParams {
   const int32_t* n_fac_per_seq; // [B] or null
   uint32_t* hist;               // [Hkv][B][2048], zero between calls
   unsigned long long* cand;     // [Hkv][T]: (key << 32 | position) of the row at offset offsets[b]
-  int32_t* cand_count;          // [Hkv][B], zero between calls
-  int32_t* tickets;             // [Hkv][B], zero between calls
-  int32_t* chunk_above;         // [Hkv][B][max_chunks]
-  int32_t* chunk_info;          // [Hkv][B][max_chunks][2]: selected before the chunk, equal keys before it
-  int32_t* row_info;            // [Hkv][B][2]: K_T, equal keys taken
+  int32_t* cand_count;          // [Hkv][B]
+  int32_t* chunk_above;         // [Hkv][B][max_chunks]: keys of the chunk above T1
+  int32_t* row_info;            // [Hkv][B][2]: T1, keys of the row above T1
   int32_t* idx;                 // [B][Hkv][cap]
   int32_t* count;               // [B][Hkv]
   int32_t T, B, Hkv, n_fac, cap, max_chunks;
@@ -68,17 +71,28 @@ __device__ __forceinline__ int sel_n(const HistSelectParams& p, int b, int L, bo
 // The first-digit histogram of the chunk's keys, added into the row's global histogram
 // (non-empty bins only).
 __global__ void __launch_bounds__(kSelCtaThreads) select_hist_kernel(const HistSelectParams p) {
+  grid_dep_wait();  // inputs come from the kernel before this one
+  grid_dep_launch();
   __shared__ uint32_t h[kSelHistBins];
   const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
   int off;
   const int L = seq_length(p.offsets, p.lengths, b, false, &off);
   const int n = sel_n(p, b, L, false);
-  if (n >= L || c * kSelChunk >= L) return;  // nothing to select here
+  if (n == 0 || n >= L || c * kSelChunk >= L) return;  // nothing to select here
+  const float* row = p.scores + (int64_t)g * p.T + off;
+  const int i0 = c * kSelChunk, i1 = min(L, i0 + kSelChunk);
+  float f[kWriteK];
+#pragma unroll
+  for (int r = 0; r < kWriteK; ++r) {  // every load in flight before any is used
+    const int i = i0 + r * kSelCtaThreads + tid;
+    f[r] = i < i1 ? __ldcg(row + i) : 0.f;
+  }
+  if (c == 0 && tid == 0) p.cand_count[(int64_t)g * p.B + b] = 0;  // read after this kernel only
   for (int i = tid; i < kSelHistBins; i += kSelCtaThreads) h[i] = 0u;
   __syncthreads();
-  const float* row = p.scores + (int64_t)g * p.T + off;
-  const int i1 = min(L, (c + 1) * kSelChunk);
-  for (int i = c * kSelChunk + tid; i < i1; i += kSelCtaThreads) atomicAdd(&h[score_key(__ldcg(row + i)) >> kSelHistShift], 1u);
+#pragma unroll
+  for (int r = 0; r < kWriteK; ++r)
+    if (i0 + r * kSelCtaThreads + tid < i1) atomicAdd(&h[score_key(f[r]) >> kSelHistShift], 1u);
   __syncthreads();
   uint32_t* gh = p.hist + ((int64_t)g * p.B + b) * kSelHistBins;
   for (int i = tid; i < kSelHistBins; i += kSelCtaThreads)
@@ -120,13 +134,13 @@ __device__ __forceinline__ int threshold_bin(const uint32_t* gh, int n, int* abo
 
 // ---------------------------------------------------------------------------- chunk pass
 __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const HistSelectParams p) {
+  grid_dep_wait();  // inputs come from the kernel before this one
+  grid_dep_launch();
   __shared__ int scratch[33];
   __shared__ int s_out[2];
-  __shared__ int s_last;
   __shared__ int s_warp[kSelCtaThreads / 32];
-  __shared__ uint32_t s_key[kSelResolveCap];
-  __shared__ int s_hist[256];
-  __shared__ int s_gt[kSelMaxChunks], s_eq[kSelMaxChunks];  // per-chunk counts
+  __shared__ int s_whit[kSelCtaThreads / 32];
+  __shared__ int s_base;
   const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   int off;
@@ -134,135 +148,73 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const Hist
   const int n = sel_n(p, b, L, c == 0 && tid == 0);
   const int nch = (L + kSelChunk - 1) / kSelChunk;
   const int64_t rid = (int64_t)g * p.B + b;
-  uint32_t* gh = p.hist + rid * kSelHistBins;
-  if (n >= L) {  // every position taken: the write pass alone; the scan's counts are cleared
-    if (c == 0)
-      for (int i = tid; i < kSelHistBins; i += kSelCtaThreads) gh[i] = 0u;
-    return;
-  }
-  if (c >= nch) return;
-  int above1;
-  const int T1 = threshold_bin(gh, n, &above1, scratch, s_out);
-
-  // this chunk: keys above the bin (counted), keys in the bin (to the candidate list)
+  if (n == 0 || n >= L || c >= nch) return;  // nothing to select (the write pass alone), or past the row
+  // this chunk's keys first: their loads fly while the row's histogram is read
   const float* row = p.scores + (int64_t)g * p.T + off;
   unsigned long long* cand = p.cand + (int64_t)g * p.T + off;
   const int i0 = c * kSelChunk, i1 = min(L, i0 + kSelChunk);
-  int n_above = 0;
   uint32_t kk[kWriteK];
-#pragma unroll
-  for (int r = 0; r < kWriteK; ++r) {  // every load in flight before any is used
-    const int i = i0 + r * kSelCtaThreads + tid;
-    kk[r] = i < i1 ? score_key(__ldcg(row + i)) : 0u;
-  }
 #pragma unroll
   for (int r = 0; r < kWriteK; ++r) {
     const int i = i0 + r * kSelCtaThreads + tid;
-    const uint32_t k = kk[r];
-    const int bin = (int)(k >> kSelHistShift);
+    kk[r] = i < i1 ? score_key(__ldcg(row + i)) : 0u;
+  }
+  int above1;
+  const int T1 = threshold_bin(p.hist + rid * kSelHistBins, n, &above1, scratch, s_out);
+  if (c == 0 && tid == 0) {
+    p.row_info[rid * 2] = T1;
+    p.row_info[rid * 2 + 1] = above1;
+  }
+  // keys above the bin (counted) and keys in the bin (to the candidate list: one atomic per
+  // CTA reserves the chunk's run, warps and lanes take consecutive places in it)
+  int n_above = 0, n_hit = 0;
+  unsigned hits[kWriteK];
+#pragma unroll
+  for (int r = 0; r < kWriteK; ++r) {
+    const int i = i0 + r * kSelCtaThreads + tid;
+    const int bin = (int)(kk[r] >> kSelHistShift);
     n_above += (i < i1 && bin > T1);
-    const bool hit = i < i1 && bin == T1;
-    const unsigned bal = __ballot_sync(0xffffffffu, hit);
-    int wbase = 0;
-    if (lane == 0 && bal) wbase = atomicAdd(p.cand_count + rid, __popc(bal));
-    wbase = __shfl_sync(0xffffffffu, wbase, 0);
-    if (hit) cand[wbase + __popc(bal & ((1u << lane) - 1u))] = ((unsigned long long)k << 32) | (uint32_t)i;
+    hits[r] = __ballot_sync(0xffffffffu, i < i1 && bin == T1);
+    n_hit += __popc(hits[r]);
   }
   n_above = __reduce_add_sync(0xffffffffu, n_above);
-  if (lane == 0) s_warp[warp] = n_above;
+  if (lane == 0) {
+    s_warp[warp] = n_above;
+    s_whit[warp] = n_hit;
+  }
   __syncthreads();
   if (tid == 0) {
-    int t = 0;
-    for (int w = 0; w < kSelCtaThreads / 32; ++w) t += s_warp[w];
+    int t = 0, hsum = 0;
+    for (int w = 0; w < kSelCtaThreads / 32; ++w) {
+      t += s_warp[w];
+      const int x = s_whit[w];
+      s_whit[w] = hsum;  // exclusive offsets of the warps' candidates
+      hsum += x;
+    }
     p.chunk_above[rid * p.max_chunks + c] = t;
-  }
-  // ---- the last CTA of the row resolves K_T
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(p.tickets + rid, 1) == nch - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const int m = atomicAdd(p.cand_count + rid, 0);  // every candidate of the row is written
-  const bool in_smem = m <= kSelResolveCap;
-  if (in_smem) {
-    for (int j = tid; j < m; j += kSelCtaThreads) s_key[j] = (uint32_t)(__ldcg(cand + j) >> 32);
-    __syncthreads();
-  }
-  // rank krem (1 = largest) among the candidates, digits of the low 21 bits
-  uint32_t prefix = (uint32_t)T1 << kSelHistShift, pmask = 0xffffffffu << kSelHistShift;
-  int krem = n - above1;
-  const int shifts[3] = {13, 5, 0};
-  const int widths[3] = {8, 8, 5};
-#pragma unroll 1
-  for (int d = 0; d < 3; ++d) {
-    const int sh = shifts[d], nb = 1 << widths[d];
-    if (tid < 256) s_hist[tid] = 0;
-    __syncthreads();
-    for (int j = tid; j < m; j += kSelCtaThreads) {
-      const uint32_t k = in_smem ? s_key[j] : (uint32_t)(__ldcg(cand + j) >> 32);
-      if ((k & pmask) == prefix) atomicAdd(&s_hist[(k >> sh) & (nb - 1)], 1);
-    }
-    __syncthreads();
-    // bins from the top: thread t takes bin nb - 1 - t
-    const int cnt = tid < nb ? s_hist[nb - 1 - tid] : 0;
-    int total;
-    const int excl = block_exclusive_scan(cnt, scratch, &total);
-    if (tid < nb && excl < krem && krem <= excl + cnt) {
-      s_out[0] = nb - 1 - tid;
-      s_out[1] = excl;
-    }
-    __syncthreads();
-    prefix |= (uint32_t)s_out[0] << sh;
-    pmask |= (uint32_t)(nb - 1) << sh;
-    krem -= s_out[1];
-    __syncthreads();
-  }
-  const uint32_t KT = prefix;
-  const int need_eq = krem;  // keys equal to K_T that are taken (>= 1), lowest positions first
-  // candidates above / equal to K_T, per chunk
-  for (int q = tid; q < nch; q += kSelCtaThreads) {
-    s_gt[q] = 0;
-    s_eq[q] = 0;
+    s_base = hsum ? atomicAdd(p.cand_count + rid, hsum) : 0;
   }
   __syncthreads();
-  for (int j = tid; j < m; j += kSelCtaThreads) {
-    const unsigned long long e = __ldcg(cand + j);
-    const uint32_t k = (uint32_t)(e >> 32);
-    const int q = (int)(uint32_t)e / kSelChunk;
-    if (k > KT) atomicAdd(&s_gt[q], 1);
-    else if (k == KT) atomicAdd(&s_eq[q], 1);
+  int wbase = s_base + s_whit[warp];
+#pragma unroll
+  for (int r = 0; r < kWriteK; ++r) {
+    if ((hits[r] >> lane) & 1u)
+      cand[wbase + __popc(hits[r] & ((1u << lane) - 1u))] =
+          ((unsigned long long)kk[r] << 32) | (uint32_t)(i0 + r * kSelCtaThreads + tid);
+    wbase += __popc(hits[r]);
   }
-  __syncthreads();
-  // offsets: thread t owns chunks [t * per, (t + 1) * per)
-  const int per = (nch + kSelCtaThreads - 1) / kSelCtaThreads;
-  int sel_t = 0, eq_t = 0;
-  for (int q = tid * per; q < min(nch, (tid + 1) * per); ++q) {
-    sel_t += __ldcg(p.chunk_above + rid * p.max_chunks + q) + s_gt[q];
-    eq_t += s_eq[q];
-  }
-  int tot_sel, tot_eq;
-  int sel_before = block_exclusive_scan(sel_t, scratch, &tot_sel);
-  int eq_before = block_exclusive_scan(eq_t, scratch, &tot_eq);
-  for (int q = tid * per; q < min(nch, (tid + 1) * per); ++q) {
-    // selected before chunk q: keys above K_T before it plus the equal keys taken before it
-    p.chunk_info[(rid * p.max_chunks + q) * 2] = sel_before + min(need_eq, eq_before);
-    p.chunk_info[(rid * p.max_chunks + q) * 2 + 1] = eq_before;
-    sel_before += __ldcg(p.chunk_above + rid * p.max_chunks + q) + s_gt[q];
-    eq_before += s_eq[q];
-  }
-  if (tid == 0) {
-    p.row_info[rid * 2] = (int)KT;
-    p.row_info[rid * 2 + 1] = need_eq;
-    p.cand_count[rid] = 0;
-    p.tickets[rid] = 0;
-  }
-  for (int i = tid; i < kSelHistBins; i += kSelCtaThreads) gh[i] = 0u;
 }
 
 // ---------------------------------------------------------------------------- ordered write
 __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const HistSelectParams p) {
+  grid_dep_wait();  // inputs come from the kernels before this one
+  grid_dep_launch();
   __shared__ int scratch[33];
+  __shared__ int s_out[2];
+  __shared__ int s_hist[256];
+  __shared__ int s_red[2][kSelCtaThreads / 32];
+  __shared__ uint32_t s_key[kSelResolveCap];
+  __shared__ uint32_t s_pos[kSelResolveCap];
   const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   int off;
@@ -281,19 +233,99 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const Hist
     return;
   }
   const int64_t rid = (int64_t)g * p.B + b;
-  const uint32_t KT = (uint32_t)__ldcg(p.row_info + rid * 2);
-  const int need_eq = __ldcg(p.row_info + rid * 2 + 1);
-  const int sel_chunk = __ldcg(p.chunk_info + (rid * p.max_chunks + c) * 2);
-  const int eq_chunk = __ldcg(p.chunk_info + (rid * p.max_chunks + c) * 2 + 1);
   const float* row = p.scores + (int64_t)g * p.T + off;
-  // warp w owns keys [i0 + w * 32 * kWriteK, ...): lane-consecutive loads, kWriteK rounds
+  const unsigned long long* cand = p.cand + (int64_t)g * p.T + off;
+  // the chunk's keys (warp w owns keys [i0 + w * 32 * kWriteK, ...), lane-consecutive loads),
+  // the row's threshold bin and candidate count: all loads in flight together
   const int w0 = i0 + warp * 32 * kWriteK;
   uint32_t k[kWriteK];
-  int ngt = 0, neq = 0;
 #pragma unroll
   for (int r = 0; r < kWriteK; ++r) {
     const int i = w0 + r * 32 + lane;
     k[r] = i < i1 ? score_key(__ldcg(row + i)) : 0u;
+  }
+  const int T1 = __ldcg(p.row_info + rid * 2), above1 = __ldcg(p.row_info + rid * 2 + 1);
+  const int m = __ldcg(p.cand_count + rid);
+  // keys above T1 in the chunks before this one
+  int ab = 0;
+  for (int q = tid; q < c; q += kSelCtaThreads) ab += __ldcg(p.chunk_above + rid * p.max_chunks + q);
+  const bool in_smem = m <= kSelResolveCap;
+  if (in_smem) {
+    for (int j = tid; j < m; j += kSelCtaThreads) {
+      const unsigned long long e = __ldcg(cand + j);
+      s_key[j] = (uint32_t)(e >> 32);
+      s_pos[j] = (uint32_t)e;
+    }
+  }
+  if (c == 0)  // the histogram's last reader was the chunk pass: re-arm it for the next call
+    for (int i = tid; i < kSelHistBins; i += kSelCtaThreads) p.hist[rid * kSelHistBins + i] = 0u;
+  __syncthreads();
+  // K_T: rank krem (1 = largest) among the candidates, digits of the low 21 bits
+  uint32_t prefix = (uint32_t)T1 << kSelHistShift, pmask = 0xffffffffu << kSelHistShift;
+  int krem = n - above1;
+#pragma unroll 1
+  for (int d = 0; d < 3; ++d) {
+    const int sh = d == 0 ? 13 : (d == 1 ? 5 : 0);
+    const int nb = d < 2 ? 256 : 32;
+    s_hist[tid] = 0;
+    __syncthreads();
+    for (int j = tid; j < m; j += kSelCtaThreads) {
+      const uint32_t kj = in_smem ? s_key[j] : (uint32_t)(__ldcg(cand + j) >> 32);
+      if ((kj & pmask) == prefix) atomicAdd(&s_hist[(kj >> sh) & (nb - 1)], 1);
+    }
+    __syncthreads();
+    // bins from the top: thread t takes bin nb - 1 - t
+    const int cnt = tid < nb ? s_hist[nb - 1 - tid] : 0;
+    int total;
+    const int excl = block_exclusive_scan(cnt, scratch, &total);
+    if (tid < nb && excl < krem && krem <= excl + cnt) {
+      s_out[0] = nb - 1 - tid;
+      s_out[1] = excl;
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_out[0] << sh;
+    pmask |= (uint32_t)(nb - 1) << sh;
+    krem -= s_out[1];
+    __syncthreads();
+  }
+  const uint32_t KT = prefix;
+  const int need_eq = krem;  // keys equal to K_T that are taken (>= 1), lowest positions first
+  // candidates of the chunks before this one above / equal to K_T
+  int gtb = 0, eqb = 0;
+  for (int j = tid; j < m; j += kSelCtaThreads) {
+    uint32_t kj, pj;
+    if (in_smem) {
+      kj = s_key[j];
+      pj = s_pos[j];
+    } else {
+      const unsigned long long e = __ldcg(cand + j);
+      kj = (uint32_t)(e >> 32);
+      pj = (uint32_t)e;
+    }
+    if ((int)pj < i0) {
+      gtb += kj > KT;
+      eqb += kj == KT;
+    }
+  }
+  ab = __reduce_add_sync(0xffffffffu, ab + gtb);
+  eqb = __reduce_add_sync(0xffffffffu, eqb);
+  if (lane == 0) {
+    s_red[0][warp] = ab;
+    s_red[1][warp] = eqb;
+  }
+  __syncthreads();
+  int sel_chunk = 0, eq_chunk = 0;
+#pragma unroll
+  for (int w = 0; w < kSelCtaThreads / 32; ++w) {
+    sel_chunk += s_red[0][w];
+    eq_chunk += s_red[1][w];
+  }
+  sel_chunk += min(need_eq, eq_chunk);  // equal keys taken before the chunk
+  // this chunk's picks, in order
+  int ngt = 0, neq = 0;
+#pragma unroll
+  for (int r = 0; r < kWriteK; ++r) {
+    const int i = w0 + r * 32 + lane;
     ngt += (i < i1 && k[r] > KT);
     neq += (i < i1 && k[r] == KT);
   }

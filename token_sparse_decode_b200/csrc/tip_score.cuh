@@ -1,8 +1,6 @@
 // Token Importance Predictor scan (FASA: Frequency-aware Sparse Attention, §2.B.1).
 // (Rows are addressed through each KV head's slot in the cache; the unused tail of a
-// sequence's region, when the cache carries per-sequence lengths, is not scored.  With a
-// histogram buffer the scan also counts the top 11 bits of every key it writes, per
-// (KV head, sequence) row, for the select that follows.)
+// sequence's region, when the cache carries per-sequence lengths, is not scored.)
 //
 // For KV head g of sequence b the score of cached token t is the fp32 dot of
 //   q~_g = sum over the group's q heads of q_h, restricted to the dominant dims
@@ -38,7 +36,6 @@ struct TipParams {
   int32_t B;
   int64_t per_cta;          // flattened (listed head, token) rows per CTA
   int64_t total;            // n_listed * T
-  uint32_t* hist;           // [Hkv][B][2048] first-digit histograms of the rows' keys, or null
   uint8_t heads[kMaxHeads]; // KV heads scored
   uint8_t slot[kMaxHeads];  // head slot of every KV head in the row source
 };
@@ -62,9 +59,9 @@ __device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
 // q~ while those loads are in flight.
 template <int S>
 __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipParams p) {
+  grid_dep_launch();  // the select that follows may begin scheduling
   __shared__ float qt[128];
   __shared__ int s_seg[3];  // sequence b of the segment (-1: none), its region's end, its last token + 1
-  __shared__ uint32_t s_hist[2048];  // the segment's first-digit counts (top 11 bits of the keys)
   const int tid = threadIdx.x, lane = tid & 31;
   const int C = p.d >> 1;
   const int seg = lane % S;
@@ -76,8 +73,6 @@ __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipPara
   int64_t w = (int64_t)blockIdx.x * p.per_cta;
   int bhint = 0;
   int64_t cur_j = -1;
-  if (p.hist)
-    for (int i = tid; i < 2048; i += kTipThreads) s_hist[i] = 0u;  // read after the first barrier below
   while (w < w1) {  // CTA-uniform
     const int64_t j = w / p.T;
     const int t = (int)(w - j * p.T);
@@ -192,27 +187,8 @@ __global__ void __launch_bounds__(kTipThreads, 4) tip_score_kernel(const TipPara
 #pragma unroll
         for (int o = S / 2; o > 0; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
         const int r = r0 + u * RPI + prow;
-        if (seg == 0 && r < n) {
-          srow[r] = sc;
-          if (p.hist) atomicAdd(&s_hist[score_key(sc) >> 21], 1u);
-        }
+        if (seg == 0 && r < n) srow[r] = sc;
       }
-    }
-    if (p.hist) {  // CTA-uniform: the segment's counts into its row's histogram
-      __syncthreads();
-      if (b >= 0) {
-        uint32_t* gh = p.hist + ((int64_t)g * p.B + b) * 2048;
-        for (int i = tid; i < 2048; i += kTipThreads) {
-          const uint32_t c = s_hist[i];
-          if (c) {
-            atomicAdd(gh + i, c);
-            s_hist[i] = 0u;
-          }
-        }
-      } else {
-        for (int i = tid; i < 2048; i += kTipThreads) s_hist[i] = 0u;
-      }
-      __syncthreads();
     }
     w += n;
   }
