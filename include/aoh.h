@@ -156,10 +156,11 @@ typedef enum {
   AOH_KERNEL_GROUP_ROLES = 9,   /* head classifier: group means and roles            */
   AOH_KERNEL_OFFLOAD_STAGE = 10,  /* host offload: selected rows across the host link */
   AOH_KERNEL_OFFLOAD_SPLIT = 11,  /* host offload: a device cache split to host parts */
-  AOH_KERNEL_SELECT_CHUNK = 12, /* select: threshold bin, candidates, exact threshold */
+  AOH_KERNEL_SELECT_CHUNK = 12, /* select: threshold bin, counts above it, candidates */
   AOH_KERNEL_SELECT_WRITE = 13, /* select: ordered write of the chosen positions     */
   AOH_KERNEL_SELECT_CLUSTER = 14, /* select: one cluster per row, keys on chip      */
-  AOH_KERNEL_KINDS = 15
+  AOH_KERNEL_SELECT_RESOLVE = 15, /* select: exact threshold and chunk offsets per row */
+  AOH_KERNEL_KINDS = 16
 } aoh_kernel_kind;
 
 /*
@@ -254,8 +255,9 @@ aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* k
  * 10-bit digits, histograms summed across the cluster through distributed
  * shared memory, picks written in order); longer rows take three launches (a
  * histogram of the top 11 bits, then chunks of 4096 keys in parallel: keys
- * above the threshold bin counted, keys in it collected, the exact threshold
- * resolved once per row, every chunk's picks written in order).
+ * above the threshold bin counted, keys in it collected; one CTA per row
+ * resolves the exact threshold and every chunk's offset; every chunk's picks
+ * written in order).
  */
 aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
                            const int32_t* n_fac_per_seq, int32_t n_fac_cap,

@@ -161,7 +161,7 @@ def test_topk_many_rows(kind):
     s = given_scores(rng, lengths, Hkv, kind)
     nfps = np.array([4, 1, 9, 700, 2048, 1500] + [int(x) for x in rng.integers(1, 2049, 48)], dtype=np.int32)
     check_topk(s, offs, lengths, nfps, 2048,
-               {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_write_kernel": 1}, kind)
+               {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_resolve_kernel": 1, "select_write_kernel": 1}, kind)
 
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
@@ -189,7 +189,7 @@ def test_topk_long_rows_chunked(kind):
     s = given_scores(rng, lengths, Hkv, kind)
     nfps = np.array([3000, 4, 9, 2048, 2500, 1], dtype=np.int32)
     check_topk(s, offs, lengths, nfps, 3000,
-               {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_write_kernel": 1}, kind)
+               {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_resolve_kernel": 1, "select_write_kernel": 1}, kind)
 
 
 @pytest.mark.parametrize("L", [1, 8191, 8192, 8193, 65536, 131072])
@@ -246,8 +246,8 @@ def test_sparse_decode_many_rows_runs_three_stages():
     torch.cuda.synchronize()
     names = [k for k, _, _ in rec]
     assert names in (["tip_score_kernel", "select_cluster_kernel", "flash_gather_kernel"],
-                     ["tip_score_kernel", "select_hist_kernel", "select_chunk_kernel", "select_write_kernel",
-                      "flash_gather_kernel"])
+                     ["tip_score_kernel", "select_hist_kernel", "select_chunk_kernel", "select_resolve_kernel",
+                      "select_write_kernel", "flash_gather_kernel"])
     assert all(e0.elapsed_time(e1) > 0 for _, e0, e1 in rec)
     out_h = f64(out)
     idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()

@@ -36,7 +36,8 @@ NO_SLOT = 255  # head_slot entry of a KV head a cache does not store
 KERNELS = ("tip_score_kernel", "select_hist_kernel", "sparse_row_kernel", "flash_gather_kernel",
            "pack_dominant_kernel", "kv_append_kernel", "gram_kernel", "gram_reduce_kernel", "spectrum_kernel",
            "group_roles_kernel", "offload_stage_kernel", "offload_split_kernel", "select_chunk_kernel",
-           "select_write_kernel", "select_cluster_kernel")
+           "select_write_kernel", "select_cluster_kernel",
+           "select_resolve_kernel")
 
 
 class AohError(RuntimeError):

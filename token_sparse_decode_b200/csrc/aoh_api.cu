@@ -377,7 +377,7 @@ aoh_status launch_tip_full(const void* q, int32_t Hq, const aoh_kv_cache* kv, fl
 // and every select leaves them at zero), then the candidate counts and list, the chunk counts
 // and the row results.
 struct SelectWs {
-  size_t hist, cand_count, cand, chunk_above, row_info, total;
+  size_t hist, cand_count, cand, chunk_above, chunk_info, row_info, total;
   int max_chunks;
 };
 
@@ -394,8 +394,10 @@ SelectWs select_ws(const aoh_kv_cache* kv) {
   o += align256((size_t)kv->n_kv_heads * (size_t)std::max<int64_t>(kv->total_tokens, 1) * sizeof(unsigned long long));
   w.chunk_above = o;
   o += align256(rows * w.max_chunks * sizeof(int32_t));
+  w.chunk_info = o;
+  o += align256(rows * w.max_chunks * 2 * sizeof(int32_t));
   w.row_info = o;
-  o += align256(rows * 2 * sizeof(int32_t));
+  o += align256(rows * kRowInfo * sizeof(int32_t));
   w.total = o;
   return w;
 }
@@ -418,6 +420,7 @@ aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int3
   hp.cand = reinterpret_cast<unsigned long long*>(ws + w.cand);
   hp.cand_count = reinterpret_cast<int32_t*>(ws + w.cand_count);
   hp.chunk_above = reinterpret_cast<int32_t*>(ws + w.chunk_above);
+  hp.chunk_info = reinterpret_cast<int32_t*>(ws + w.chunk_info);
   hp.row_info = reinterpret_cast<int32_t*>(ws + w.row_info);
   hp.idx = idx;
   hp.count = count;
@@ -436,6 +439,10 @@ aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int3
   }
   if ((s = launch_dependent(select_chunk_kernel, grid, kSelCtaThreads, 0, 0, st, hp)) != AOH_OK) return s;
   if ((s = count_launch(AOH_KERNEL_SELECT_CHUNK, st)) != AOH_OK) return s;
+  if ((s = launch_dependent(select_resolve_kernel, dim3(1, n_listed, kv->batch), kSelResolveThreads, 0, 0, st, hp)) !=
+      AOH_OK)
+    return s;
+  if ((s = count_launch(AOH_KERNEL_SELECT_RESOLVE, st)) != AOH_OK) return s;
   if ((s = launch_dependent(select_write_kernel, grid, kSelCtaThreads, 0, 0, st, hp)) != AOH_OK) return s;
   return count_launch(AOH_KERNEL_SELECT_WRITE, st);
 }

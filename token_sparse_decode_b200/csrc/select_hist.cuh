@@ -7,7 +7,7 @@
 // positions among {key == K_T}, n in all, written in ascending position order.
 //
 // First digit: the top 11 bits of a key (sign, exponent, two mantissa bits).  With chunks
-// of kSelChunk keys of a row, one CTA each, three launches:
+// of kSelChunk keys of a row, one CTA each (the resolve: one CTA per row), four launches:
 //   select_hist_kernel   counts the chunk's first digits in shared memory and adds the
 //                        non-empty bins into the row's histogram (chunk 0 also clears the
 //                        row's candidate count);
@@ -16,17 +16,18 @@
 //                        keys above T1 and appends the chunk's keys in T1 (key, position) to
 //                        the row's candidate list (one atomic per CTA reserves the chunk's
 //                        run of the list);
-//   select_write_kernel  every chunk resolves K_T from the row's candidates on its own (the
-//                        remaining 21 bits, digits of 8, 8 and 5, over the candidates in
-//                        shared memory), counts the keys the chunks before it take (their
-//                        keys above T1 plus their candidates above or equal to K_T), and
-//                        writes its selected positions at that offset, in order: warps own
-//                        runs of 32 x kWriteK consecutive keys, ballots rank the picks inside
-//                        a warp, one block scan ranks the warps.  Chunk 0 re-arms the row's
-//                        histogram to zero.
-// No CTA waits for another and no CTA resolves for the others: every dependency is a kernel
-// boundary.  Every kernel issues all of its key loads before it uses any.  A row with
-// n >= L_b takes every position without a select.  Deterministic: the candidate list's order
+//   select_resolve_kernel one CTA per row resolves K_T from the row's candidates (the
+//                        remaining 21 bits, digits of 11 and 10, candidates in shared memory;
+//                        it stops early when the chosen bin is exactly what is left, and keys
+//                        are then compared masked), turns the per-chunk counts into every
+//                        chunk's output offset and number of equal keys before it, and
+//                        re-arms the row's histogram to zero;
+//   select_write_kernel  every chunk writes its selected positions at that offset, in order:
+//                        warps own runs of 32 x kWriteK consecutive keys, ballots rank the
+//                        picks inside a warp, one block scan ranks the warps.
+// No CTA waits for another: every dependency is a kernel boundary.  Every kernel issues all
+// of its key loads before it uses any.  A row with n >= L_b takes every position without a
+// select.  Deterministic: the candidate list's order
 // varies between runs, the counts drawn from it do not.
 #pragma once
 
@@ -40,7 +41,9 @@ constexpr int kSelHistShift = 21;
 constexpr int kSelCtaThreads = 256;
 constexpr int kWriteK = kSelChunk / kSelCtaThreads;  // keys per lane (16)
 constexpr int kSelMaxChunks = 1024;    // chunks per row: rows up to 4 M keys
-constexpr int kSelResolveCap = 4096;   // candidates a CTA keeps in shared memory (more: read from L2)
+constexpr int kSelResolveCap = 4096;   // candidates the resolve keeps in shared memory (more: read from L2)
+constexpr int kSelResolveThreads = 512;
+constexpr int kRowInfo = 8;            // ints per row in row_info
 
 struct HistSelectParams {
   const float* scores;          // [Hkv][T]
@@ -51,7 +54,8 @@ struct HistSelectParams {
   unsigned long long* cand;     // [Hkv][T]: (key << 32 | position) of the row at offset offsets[b]
   int32_t* cand_count;          // [Hkv][B]
   int32_t* chunk_above;         // [Hkv][B][max_chunks]: keys of the chunk above T1
-  int32_t* row_info;            // [Hkv][B][2]: T1, keys of the row above T1
+  int32_t* chunk_info;          // [Hkv][B][max_chunks][2]: keys selected before the chunk, equal keys before it
+  int32_t* row_info;            // [Hkv][B][kRowInfo]: T1, keys above T1, threshold prefix, its mask, equal keys taken
   int32_t* idx;                 // [B][Hkv][cap]
   int32_t* count;               // [B][Hkv]
   int32_t T, B, Hkv, n_fac, cap, max_chunks;
@@ -162,8 +166,8 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const Hist
   int above1;
   const int T1 = threshold_bin(p.hist + rid * kSelHistBins, n, &above1, scratch, s_out);
   if (c == 0 && tid == 0) {
-    p.row_info[rid * 2] = T1;
-    p.row_info[rid * 2 + 1] = above1;
+    p.row_info[rid * kRowInfo] = T1;
+    p.row_info[rid * kRowInfo + 1] = above1;
   }
   // keys above the bin (counted) and keys in the bin (to the candidate list: one atomic per
   // CTA reserves the chunk's run, warps and lanes take consecutive places in it)
@@ -205,16 +209,137 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const Hist
   }
 }
 
+// ---------------------------------------------------------------------------- resolve
+// One CTA per row: the exact threshold among the row's candidates (the remaining 21 bits in
+// digits of 11 and 10 bits; when the chosen bin holds exactly the keys still needed its low
+// bits do not matter, the bin is taken whole and keys are compared masked), then every chunk's
+// output offset: the keys above T1 in the chunks before it, their candidates above the
+// threshold and the equal keys taken before it.  Re-arms the row's histogram (its last reader
+// was the chunk pass).
+__global__ void __launch_bounds__(kSelResolveThreads) select_resolve_kernel(const HistSelectParams p) {
+  grid_dep_wait();  // inputs come from the kernels before this one
+  grid_dep_launch();
+  __shared__ int scratch[33];
+  __shared__ int s_out[3];
+  __shared__ int s_hist[2048];
+  __shared__ uint32_t s_key[kSelResolveCap];
+  __shared__ uint16_t s_chk[kSelResolveCap];  // chunk of every candidate
+  __shared__ int s_gt[kSelMaxChunks], s_eq[kSelMaxChunks];
+  const int g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
+  int off;
+  const int L = seq_length(p.offsets, p.lengths, b, false, &off);
+  const int n = sel_n(p, b, L, false);
+  if (n == 0 || n >= L) return;  // nothing to select: the write pass alone
+  const int64_t rid = (int64_t)g * p.B + b;
+  const int nch = (L + kSelChunk - 1) / kSelChunk;
+  const unsigned long long* cand = p.cand + (int64_t)g * p.T + off;
+  const int T1 = __ldcg(p.row_info + rid * kRowInfo), above1 = __ldcg(p.row_info + rid * kRowInfo + 1);
+  const int m = __ldcg(p.cand_count + rid);
+  const bool in_smem = m <= kSelResolveCap;
+  if (in_smem) {
+    for (int j = tid; j < m; j += kSelResolveThreads) {
+      const unsigned long long e = __ldcg(cand + j);
+      s_key[j] = (uint32_t)(e >> 32);
+      s_chk[j] = (uint16_t)((uint32_t)e / kSelChunk);
+    }
+  }
+  for (int q = tid; q < nch; q += kSelResolveThreads) {
+    s_gt[q] = 0;
+    s_eq[q] = 0;
+  }
+  for (int i = tid; i < kSelHistBins; i += kSelResolveThreads) p.hist[rid * kSelHistBins + i] = 0u;
+  uint32_t prefix = (uint32_t)T1 << kSelHistShift, pmask = 0xffffffffu << kSelHistShift;
+  int krem = n - above1;
+#pragma unroll 1
+  for (int d = 0; d < 2; ++d) {
+    const int sh = d == 0 ? 10 : 0;
+    const int nb = d == 0 ? 2048 : 1024;
+    for (int i = tid; i < nb; i += kSelResolveThreads) s_hist[i] = 0;
+    __syncthreads();
+    for (int j = tid; j < m; j += kSelResolveThreads) {
+      const uint32_t kj = in_smem ? s_key[j] : (uint32_t)(__ldcg(cand + j) >> 32);
+      if ((kj & pmask) == prefix) atomicAdd(&s_hist[(kj >> sh) & (nb - 1)], 1);
+    }
+    __syncthreads();
+    // bins from the top: thread t takes per = nb / 512 consecutive bins
+    const int per = nb / kSelResolveThreads;
+    int cnt[4], sum = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      cnt[u] = u < per ? s_hist[nb - 1 - (tid * per + u)] : 0;
+      sum += cnt[u];
+    }
+    int total;
+    int excl = block_exclusive_scan(sum, scratch, &total);
+    if (excl < krem && krem <= excl + sum) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (u < per && excl < krem && krem <= excl + cnt[u]) {
+          s_out[0] = nb - 1 - (tid * per + u);
+          s_out[1] = excl;
+          s_out[2] = cnt[u];
+        }
+        excl += cnt[u];
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_out[0] << sh;
+    pmask |= (uint32_t)(nb - 1) << sh;
+    krem -= s_out[1];
+    const bool whole_bin = s_out[2] == krem;  // the same in every thread
+    __syncthreads();
+    if (whole_bin) break;
+  }
+  const int need_eq = krem;  // keys equal (masked) to the prefix that are taken, lowest positions first
+  // candidates above / equal to the threshold, per chunk
+  for (int j = tid; j < m; j += kSelResolveThreads) {
+    uint32_t kj;
+    int q;
+    if (in_smem) {
+      kj = s_key[j];
+      q = s_chk[j];
+    } else {
+      const unsigned long long e = __ldcg(cand + j);
+      kj = (uint32_t)(e >> 32);
+      q = (int)((uint32_t)e / kSelChunk);
+    }
+    const uint32_t mk = kj & pmask;
+    if (mk > prefix) atomicAdd(&s_gt[q], 1);
+    else if (mk == prefix) atomicAdd(&s_eq[q], 1);
+  }
+  __syncthreads();
+  // offsets: thread t owns chunks [t * per, (t + 1) * per)
+  const int per = (nch + kSelResolveThreads - 1) / kSelResolveThreads;
+  const int q0 = min(nch, tid * per), q1 = min(nch, q0 + per);
+  int sel_t = 0, eq_t = 0;
+  for (int q = q0; q < q1; ++q) {
+    sel_t += __ldcg(p.chunk_above + rid * p.max_chunks + q) + s_gt[q];
+    eq_t += s_eq[q];
+  }
+  int tot_sel, tot_eq;
+  int sel_before = block_exclusive_scan(sel_t, scratch, &tot_sel);
+  int eq_before = block_exclusive_scan(eq_t, scratch, &tot_eq);
+  for (int q = q0; q < q1; ++q) {
+    p.chunk_info[(rid * p.max_chunks + q) * 2] = sel_before + min(need_eq, eq_before);
+    p.chunk_info[(rid * p.max_chunks + q) * 2 + 1] = eq_before;
+    sel_before += __ldcg(p.chunk_above + rid * p.max_chunks + q) + s_gt[q];
+    eq_before += s_eq[q];
+  }
+  if (tid == 0) {
+    p.row_info[rid * kRowInfo + 2] = (int)prefix;
+    p.row_info[rid * kRowInfo + 3] = (int)pmask;
+    p.row_info[rid * kRowInfo + 4] = need_eq;
+  }
+}
+
 // ---------------------------------------------------------------------------- ordered write
+// Every chunk writes its selected positions at the offset the resolve gave it, in order: warps
+// own runs of 32 x kWriteK consecutive keys, one block scan ranks the warps, ballots rank the
+// picks inside a warp.
 __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const HistSelectParams p) {
   grid_dep_wait();  // inputs come from the kernels before this one
   grid_dep_launch();
   __shared__ int scratch[33];
-  __shared__ int s_out[2];
-  __shared__ int s_hist[256];
-  __shared__ int s_red[2][kSelCtaThreads / 32];
-  __shared__ uint32_t s_key[kSelResolveCap];
-  __shared__ uint32_t s_pos[kSelResolveCap];
   const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   int off;
@@ -234,9 +359,8 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const Hist
   }
   const int64_t rid = (int64_t)g * p.B + b;
   const float* row = p.scores + (int64_t)g * p.T + off;
-  const unsigned long long* cand = p.cand + (int64_t)g * p.T + off;
-  // the chunk's keys (warp w owns keys [i0 + w * 32 * kWriteK, ...), lane-consecutive loads),
-  // the row's threshold bin and candidate count: all loads in flight together
+  // the chunk's keys (warp w owns keys [i0 + w * 32 * kWriteK, ...), lane-consecutive loads)
+  // and the row's threshold: all loads in flight together
   const int w0 = i0 + warp * 32 * kWriteK;
   uint32_t k[kWriteK];
 #pragma unroll
@@ -244,90 +368,17 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const Hist
     const int i = w0 + r * 32 + lane;
     k[r] = i < i1 ? score_key(__ldcg(row + i)) : 0u;
   }
-  const int T1 = __ldcg(p.row_info + rid * 2), above1 = __ldcg(p.row_info + rid * 2 + 1);
-  const int m = __ldcg(p.cand_count + rid);
-  // keys above T1 in the chunks before this one
-  int ab = 0;
-  for (int q = tid; q < c; q += kSelCtaThreads) ab += __ldcg(p.chunk_above + rid * p.max_chunks + q);
-  const bool in_smem = m <= kSelResolveCap;
-  if (in_smem) {
-    for (int j = tid; j < m; j += kSelCtaThreads) {
-      const unsigned long long e = __ldcg(cand + j);
-      s_key[j] = (uint32_t)(e >> 32);
-      s_pos[j] = (uint32_t)e;
-    }
-  }
-  if (c == 0)  // the histogram's last reader was the chunk pass: re-arm it for the next call
-    for (int i = tid; i < kSelHistBins; i += kSelCtaThreads) p.hist[rid * kSelHistBins + i] = 0u;
-  __syncthreads();
-  // K_T: rank krem (1 = largest) among the candidates, digits of the low 21 bits
-  uint32_t prefix = (uint32_t)T1 << kSelHistShift, pmask = 0xffffffffu << kSelHistShift;
-  int krem = n - above1;
-#pragma unroll 1
-  for (int d = 0; d < 3; ++d) {
-    const int sh = d == 0 ? 13 : (d == 1 ? 5 : 0);
-    const int nb = d < 2 ? 256 : 32;
-    s_hist[tid] = 0;
-    __syncthreads();
-    for (int j = tid; j < m; j += kSelCtaThreads) {
-      const uint32_t kj = in_smem ? s_key[j] : (uint32_t)(__ldcg(cand + j) >> 32);
-      if ((kj & pmask) == prefix) atomicAdd(&s_hist[(kj >> sh) & (nb - 1)], 1);
-    }
-    __syncthreads();
-    // bins from the top: thread t takes bin nb - 1 - t
-    const int cnt = tid < nb ? s_hist[nb - 1 - tid] : 0;
-    int total;
-    const int excl = block_exclusive_scan(cnt, scratch, &total);
-    if (tid < nb && excl < krem && krem <= excl + cnt) {
-      s_out[0] = nb - 1 - tid;
-      s_out[1] = excl;
-    }
-    __syncthreads();
-    prefix |= (uint32_t)s_out[0] << sh;
-    pmask |= (uint32_t)(nb - 1) << sh;
-    krem -= s_out[1];
-    __syncthreads();
-  }
-  const uint32_t KT = prefix;
-  const int need_eq = krem;  // keys equal to K_T that are taken (>= 1), lowest positions first
-  // candidates of the chunks before this one above / equal to K_T
-  int gtb = 0, eqb = 0;
-  for (int j = tid; j < m; j += kSelCtaThreads) {
-    uint32_t kj, pj;
-    if (in_smem) {
-      kj = s_key[j];
-      pj = s_pos[j];
-    } else {
-      const unsigned long long e = __ldcg(cand + j);
-      kj = (uint32_t)(e >> 32);
-      pj = (uint32_t)e;
-    }
-    if ((int)pj < i0) {
-      gtb += kj > KT;
-      eqb += kj == KT;
-    }
-  }
-  ab = __reduce_add_sync(0xffffffffu, ab + gtb);
-  eqb = __reduce_add_sync(0xffffffffu, eqb);
-  if (lane == 0) {
-    s_red[0][warp] = ab;
-    s_red[1][warp] = eqb;
-  }
-  __syncthreads();
-  int sel_chunk = 0, eq_chunk = 0;
-#pragma unroll
-  for (int w = 0; w < kSelCtaThreads / 32; ++w) {
-    sel_chunk += s_red[0][w];
-    eq_chunk += s_red[1][w];
-  }
-  sel_chunk += min(need_eq, eq_chunk);  // equal keys taken before the chunk
-  // this chunk's picks, in order
+  const uint32_t KT = (uint32_t)__ldcg(p.row_info + rid * kRowInfo + 2);
+  const uint32_t pmask = (uint32_t)__ldcg(p.row_info + rid * kRowInfo + 3);
+  const int need_eq = __ldcg(p.row_info + rid * kRowInfo + 4);
+  const int sel_chunk = __ldcg(p.chunk_info + (rid * p.max_chunks + c) * 2);
+  const int eq_chunk = __ldcg(p.chunk_info + (rid * p.max_chunks + c) * 2 + 1);
   int ngt = 0, neq = 0;
 #pragma unroll
   for (int r = 0; r < kWriteK; ++r) {
     const int i = w0 + r * 32 + lane;
-    ngt += (i < i1 && k[r] > KT);
-    neq += (i < i1 && k[r] == KT);
+    ngt += (i < i1 && (k[r] & pmask) > KT);
+    neq += (i < i1 && (k[r] & pmask) == KT);
   }
   ngt = __reduce_add_sync(0xffffffffu, ngt);
   neq = __reduce_add_sync(0xffffffffu, neq);
@@ -342,8 +393,8 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const Hist
   for (int r = 0; r < kWriteK; ++r) {
     const int i = w0 + r * 32 + lane;
     const bool in = i < i1;
-    const bool gt = in && k[r] > KT;
-    const bool eq = in && k[r] == KT;
+    const bool gt = in && (k[r] & pmask) > KT;
+    const bool eq = in && (k[r] & pmask) == KT;
     const unsigned beq = __ballot_sync(0xffffffffu, eq);
     const int eq_rank = eq_before + __popc(beq & ((1u << lane) - 1u));
     const bool take = gt || (eq && eq_rank < need_eq);
