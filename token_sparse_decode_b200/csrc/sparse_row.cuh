@@ -13,10 +13,11 @@
 //              with the group-summed query (the same arithmetic as the stand-alone
 //              scan kernel); the scores stay in shared memory as order-preserving
 //              uint32 keys;
-//  2. select:  4-digit MSB radix select of the n-th largest key over the cluster
-//              (histograms summed through distributed shared memory, one cluster
-//              barrier per digit); ties broken toward lower positions by an ordered
-//              compaction that also writes the index (ascending) to global memory;
+//  2. select:  MSB radix select of the n-th largest key over the cluster, up to 4
+//              digits of 8 bits (histograms summed through distributed shared memory,
+//              one cluster barrier per digit; it stops at the first digit whose chosen
+//              bin is exactly what is left); ties broken toward lower positions by an
+//              ordered compaction that also writes the index (ascending) to global memory;
 //  3. attend:  every CTA gathers the K / V rows of the positions it selected from
 //              its own slice (cp.async into tiles at a 2*d+16-byte row pitch) and
 //              runs the online-softmax contraction on tensor cores (tokens on M,
@@ -266,7 +267,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     // picked from the local total.  Digit 3: every CTA reads each peer's last histogram, which
     // also gives each peer's number of keys above the threshold (s_gt) and equal to it (s_eq),
     // so the compaction needs no further exchange.  After digit 0 the keys sharing the chosen
-    // first digit are compacted; digits 1-3 count only those.
+    // first digit are compacted; digits 1-3 count only those.  When a digit's chosen bin holds
+    // exactly the keys still needed, the remaining digits are skipped.
     cluster_wait_acquire();  // peers have zeroed their totals
     uint32_t* cand = reinterpret_cast<uint32_t*>(smem + p.keys_bytes);  // free region during the select
     uint32_t prefix = 0u, pmask = 0u;
@@ -397,8 +399,21 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       krem -= s_above;
       __syncthreads();
       if (pass == 0) ncand = compact ? n_sb : -1;
+      // The chosen bin holds exactly the keys still needed (the same decision in every CTA):
+      // it is taken whole, whatever its lower digits, and keys are compared masked.  Every
+      // CTA's count above (s_up, final once the barrier below is passed) and its count in the
+      // bin are what the compaction needs; neither is written again.
+      if (pass < 3 && tot[pass & 1][sb] == krem) {
+        cluster.sync();
+        if (tid < CL) {
+          s_gt[tid] = *cluster.map_shared_rank(&s_up, tid);
+          s_eq[tid] = cluster.map_shared_rank(lhb[pass & 1], tid)[sb];
+        }
+        __syncthreads();
+        break;
+      }
     }
-    const uint32_t KT = prefix;
+    const uint32_t KT = prefix;  // with pmask: keys are taken when (key & pmask) is above KT
     const int need_eq = krem;
 
     // ---- ordered compaction: positions in ascending order, lower position first among equals
@@ -427,8 +442,8 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
       int e = lane % len;
       for (int j = 0; j < len; ++j) {
         const uint32_t k = keys[a0 + e];
-        gtm |= (uint64_t)(k > KT) << e;
-        eqm |= (uint64_t)(k == KT) << e;
+        gtm |= (uint64_t)((k & pmask) > KT) << e;
+        eqm |= (uint64_t)((k & pmask) == KT) << e;
         if (++e == len) e = 0;
       }
     }
