@@ -186,12 +186,9 @@ def launches_of(fn) -> dict:
 def three_kernel_form(launches: dict) -> bool:
     """scan + select + gather: the select is one cluster launch when every row's cluster fits
     one wave, else the chunked select's four launches"""
-    on_chip = launches.get("select_cluster_kernel") == 1 and not any(
-        k in launches
-        for k in ("select_hist_kernel", "select_chunk_kernel", "select_resolve_kernel", "select_write_kernel"))
-    chunked = (launches.get("select_hist_kernel") == 1 and launches.get("select_chunk_kernel") == 1
-               and launches.get("select_resolve_kernel") == 1 and launches.get("select_write_kernel") == 1
-               and "select_cluster_kernel" not in launches)
+    per_phase = ("select_hist_kernel", "select_chunk_kernel", "select_resolve_kernel", "select_write_kernel")
+    on_chip = launches.get("select_cluster_kernel") == 1 and not any(k in launches for k in per_phase)
+    chunked = all(launches.get(k) == 1 for k in per_phase) and "select_cluster_kernel" not in launches
     return (launches.get("tip_score_kernel") == 1 and (on_chip or chunked)
             and launches.get("flash_gather_kernel", 0) >= 1)
 

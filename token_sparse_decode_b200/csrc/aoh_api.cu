@@ -404,8 +404,8 @@ SelectWs select_ws(const aoh_kv_cache* kv) {
 
 bool select_fits(const aoh_kv_cache* kv) { return ceil_div(std::max(kv->max_len, 1), kSelChunk) <= kSelMaxChunks; }
 
-// The chunked select on the scores: the first-digit histograms, the chunk pass and the
-// ordered write.  `ws` is the select's region (layout of select_ws).
+// The chunked select on the scores: histograms, chunk pass, resolve, ordered write (one
+// launch per phase).  `ws` is the select's region (layout of select_ws).
 aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
                                int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
                                uint8_t* ws, cudaStream_t st) {
@@ -439,7 +439,7 @@ aoh_status launch_chunk_select(const float* scores, const aoh_kv_cache* kv, int3
   }
   if ((s = launch_dependent(select_chunk_kernel, grid, kSelCtaThreads, 0, 0, st, hp)) != AOH_OK) return s;
   if ((s = count_launch(AOH_KERNEL_SELECT_CHUNK, st)) != AOH_OK) return s;
-  if ((s = launch_dependent(select_resolve_kernel, dim3(1, n_listed, kv->batch), kSelResolveThreads, 0, 0, st, hp)) !=
+  if ((s = launch_dependent(select_resolve_kernel, dim3(1, n_listed, kv->batch), kSelCtaThreads, 0, 0, st, hp)) !=
       AOH_OK)
     return s;
   if ((s = count_launch(AOH_KERNEL_SELECT_RESOLVE, st)) != AOH_OK) return s;

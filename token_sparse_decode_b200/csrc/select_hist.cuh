@@ -6,44 +6,43 @@
 // The selection of a (sequence b, KV head g) row is {key > K_T} plus the lowest
 // positions among {key == K_T}, n in all, written in ascending position order.
 //
-// First digit: the top 11 bits of a key (sign, exponent, two mantissa bits).  With chunks
-// of kSelChunk keys of a row, one CTA each (the resolve: one CTA per row), four launches:
-//   select_hist_kernel   counts the chunk's first digits in shared memory and adds the
-//                        non-empty bins into the row's histogram (chunk 0 also clears the
-//                        row's candidate count);
-//   select_chunk_kernel  finds the bin T1 holding the n-th key from the histogram (chunk 0
-//                        records T1 and the keys above it for the row), counts the chunk's
-//                        keys above T1 and appends the chunk's keys in T1 (key, position) to
-//                        the row's candidate list (one atomic per CTA reserves the chunk's
-//                        run of the list);
-//   select_resolve_kernel one CTA per row resolves K_T from the row's candidates (the
-//                        remaining 21 bits, digits of 11 and 10, candidates in shared memory;
-//                        it stops early when the chosen bin is exactly what is left, and keys
-//                        are then compared masked), turns the per-chunk counts into every
-//                        chunk's output offset and number of equal keys before it, and
-//                        re-arms the row's histogram to zero;
-//   select_write_kernel  every chunk writes its selected positions at that offset, in order:
-//                        warps own runs of 32 x kWriteK consecutive keys, ballots rank the
-//                        picks inside a warp, one block scan ranks the warps.
-// No CTA waits for another: every dependency is a kernel boundary.  Every kernel issues all
-// of its key loads before it uses any.  A row with n >= L_b takes every position without a
-// select.  Deterministic: the candidate list's order
-// varies between runs, the counts drawn from it do not.
+// First digit: the top 11 bits of a key (sign, exponent, two mantissa bits).  Four phases
+// over chunks of kSelChunk keys of every row (the resolve over rows):
+//   hist     counts a chunk's first digits in shared memory and adds the non-empty bins
+//            into the row's histogram (chunk 0 also clears the row's candidate count);
+//   chunk    finds the bin T1 holding the n-th key from the histogram (chunk 0 records T1
+//            and the keys above it for the row), counts the chunk's keys above T1 and
+//            appends its keys in T1 (key, position) to the row's candidate list (one
+//            atomic per CTA reserves the chunk's run of the list);
+//   resolve  per row: the exact threshold among the candidates (the remaining 21 bits in
+//            digits of 11 and 10; when the chosen bin holds exactly the keys still needed
+//            its low bits do not matter, the bin is taken whole and keys are compared
+//            masked), every chunk's output offset and number of equal keys before it;
+//            re-arms the row's histogram to zero;
+//   write    a chunk's selected positions at its offset, in order: warps own runs of
+//            32 x kWriteK consecutive keys, ballots rank the picks inside a warp, one
+//            block scan ranks the warps.
+// One kernel per phase (four launches, each dependency a kernel boundary); the phase bodies
+// are item functions over one shared scratch buffer.  Every phase issues all of its key
+// loads before it uses any.  A row with n >= L_b takes every position
+// without a select.  Deterministic: the candidate list's order varies between runs, the
+// counts drawn from it do not.
 #pragma once
 
 #include "device_common.cuh"
 
 namespace aoh {
 
-constexpr int kSelChunk = 4096;        // keys of a row per CTA
+constexpr int kSelChunk = 4096;        // keys of a row per chunk
 constexpr int kSelHistBins = 2048;     // first digit: the top 11 bits of a key
 constexpr int kSelHistShift = 21;
 constexpr int kSelCtaThreads = 256;
 constexpr int kWriteK = kSelChunk / kSelCtaThreads;  // keys per lane (16)
 constexpr int kSelMaxChunks = 1024;    // chunks per row: rows up to 4 M keys
 constexpr int kSelResolveCap = 4096;   // candidates the resolve keeps in shared memory (more: read from L2)
-constexpr int kSelResolveThreads = 512;
 constexpr int kRowInfo = 8;            // ints per row in row_info
+// shared scratch of the resolve phase
+constexpr int kSelSmem = 144 + 4 * kSelHistBins + 4 * kSelResolveCap + 2 * kSelResolveCap + 8 * kSelMaxChunks;
 
 struct HistSelectParams {
   const float* scores;          // [Hkv][T]
@@ -59,7 +58,7 @@ struct HistSelectParams {
   int32_t* idx;                 // [B][Hkv][cap]
   int32_t* count;               // [B][Hkv]
   int32_t T, B, Hkv, n_fac, cap, max_chunks;
-  uint8_t heads[kMaxHeads];     // KV head of blockIdx.y
+  uint8_t heads[kMaxHeads];     // listed KV heads
 };
 
 __device__ __forceinline__ int sel_n(const HistSelectParams& p, int b, int L, bool report) {
@@ -71,14 +70,12 @@ __device__ __forceinline__ int sel_n(const HistSelectParams& p, int b, int L, bo
   return max(0, min(nf, L));
 }
 
-// ---------------------------------------------------------------------------- histogram
-// The first-digit histogram of the chunk's keys, added into the row's global histogram
-// (non-empty bins only).
-__global__ void __launch_bounds__(kSelCtaThreads) select_hist_kernel(const HistSelectParams p) {
-  grid_dep_wait();  // inputs come from the kernel before this one
-  grid_dep_launch();
-  __shared__ uint32_t h[kSelHistBins];
-  const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
+// ---------------------------------------------------------------------------- hist phase
+// The first-digit histogram of chunk c of row (listed head y, sequence b), added into the
+// row's global histogram (non-empty bins only).
+__device__ __forceinline__ void sel_hist_item(const HistSelectParams& p, uint8_t* sm, int c, int y, int b) {
+  uint32_t* h = reinterpret_cast<uint32_t*>(sm);
+  const int g = p.heads[y], tid = threadIdx.x;
   int off;
   const int L = seq_length(p.offsets, p.lengths, b, false, &off);
   const int n = sel_n(p, b, L, false);
@@ -91,7 +88,8 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_hist_kernel(const HistS
     const int i = i0 + r * kSelCtaThreads + tid;
     f[r] = i < i1 ? __ldcg(row + i) : 0.f;
   }
-  if (c == 0 && tid == 0) p.cand_count[(int64_t)g * p.B + b] = 0;  // read after this kernel only
+  if (c == 0 && tid == 0) p.cand_count[(int64_t)g * p.B + b] = 0;  // read after this phase only
+  __syncthreads();  // the scratch may still be read for the previous item
   for (int i = tid; i < kSelHistBins; i += kSelCtaThreads) h[i] = 0u;
   __syncthreads();
 #pragma unroll
@@ -136,23 +134,21 @@ __device__ __forceinline__ int threshold_bin(const uint32_t* gh, int n, int* abo
   return s_out[0];
 }
 
-// ---------------------------------------------------------------------------- chunk pass
-__global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const HistSelectParams p) {
-  grid_dep_wait();  // inputs come from the kernel before this one
-  grid_dep_launch();
-  __shared__ int scratch[33];
-  __shared__ int s_out[2];
-  __shared__ int s_warp[kSelCtaThreads / 32];
-  __shared__ int s_whit[kSelCtaThreads / 32];
-  __shared__ int s_base;
-  const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
+// ---------------------------------------------------------------------------- chunk phase
+__device__ __forceinline__ void sel_chunk_item(const HistSelectParams& p, uint8_t* sm, int c, int y, int b) {
+  int* scratch = reinterpret_cast<int*>(sm);  // [33]
+  int* s_out = scratch + 33;                  // [2]
+  int* s_warp = s_out + 2;                    // [8]
+  int* s_whit = s_warp + 8;                   // [8]
+  int* s_base = s_whit + 8;                   // [1]
+  const int g = p.heads[y], tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   int off;
   const int L = seq_length(p.offsets, p.lengths, b, false, &off);
   const int n = sel_n(p, b, L, c == 0 && tid == 0);
   const int nch = (L + kSelChunk - 1) / kSelChunk;
   const int64_t rid = (int64_t)g * p.B + b;
-  if (n == 0 || n >= L || c >= nch) return;  // nothing to select (the write pass alone), or past the row
+  if (n == 0 || n >= L || c >= nch) return;  // nothing to select (the write phase alone), or past the row
   // this chunk's keys first: their loads fly while the row's histogram is read
   const float* row = p.scores + (int64_t)g * p.T + off;
   unsigned long long* cand = p.cand + (int64_t)g * p.T + off;
@@ -163,6 +159,7 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const Hist
     const int i = i0 + r * kSelCtaThreads + tid;
     kk[r] = i < i1 ? score_key(__ldcg(row + i)) : 0u;
   }
+  __syncthreads();  // the scratch may still be read for the previous item
   int above1;
   const int T1 = threshold_bin(p.hist + rid * kSelHistBins, n, &above1, scratch, s_out);
   if (c == 0 && tid == 0) {
@@ -196,10 +193,10 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const Hist
       hsum += x;
     }
     p.chunk_above[rid * p.max_chunks + c] = t;
-    s_base = hsum ? atomicAdd(p.cand_count + rid, hsum) : 0;
+    s_base[0] = hsum ? atomicAdd(p.cand_count + rid, hsum) : 0;
   }
   __syncthreads();
-  int wbase = s_base + s_whit[warp];
+  int wbase = s_base[0] + s_whit[warp];
 #pragma unroll
   for (int r = 0; r < kWriteK; ++r) {
     if ((hits[r] >> lane) & 1u)
@@ -209,63 +206,62 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const Hist
   }
 }
 
-// ---------------------------------------------------------------------------- resolve
-// One CTA per row: the exact threshold among the row's candidates (the remaining 21 bits in
-// digits of 11 and 10 bits; when the chosen bin holds exactly the keys still needed its low
-// bits do not matter, the bin is taken whole and keys are compared masked), then every chunk's
-// output offset: the keys above T1 in the chunks before it, their candidates above the
-// threshold and the equal keys taken before it.  Re-arms the row's histogram (its last reader
-// was the chunk pass).
-__global__ void __launch_bounds__(kSelResolveThreads) select_resolve_kernel(const HistSelectParams p) {
-  grid_dep_wait();  // inputs come from the kernels before this one
-  grid_dep_launch();
-  __shared__ int scratch[33];
-  __shared__ int s_out[3];
-  __shared__ int s_hist[2048];
-  __shared__ uint32_t s_key[kSelResolveCap];
-  __shared__ uint16_t s_chk[kSelResolveCap];  // chunk of every candidate
-  __shared__ int s_gt[kSelMaxChunks], s_eq[kSelMaxChunks];
-  const int g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
+// ---------------------------------------------------------------------------- resolve phase
+// Row (listed head y, sequence b): the exact threshold among the row's candidates, then every
+// chunk's output offset: the keys above T1 in the chunks before it, their candidates above
+// the threshold and the equal keys taken before it.  Re-arms the row's histogram (its last
+// reader was the chunk phase).
+__device__ __forceinline__ void sel_resolve_row(const HistSelectParams& p, uint8_t* sm, int y, int b) {
+  int* scratch = reinterpret_cast<int*>(sm);                             // [33]
+  int* s_out = scratch + 33;                                             // [3]
+  int* s_hist = reinterpret_cast<int*>(sm + 144);                        // [2048]
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(sm + 144 + 4 * kSelHistBins);  // [kSelResolveCap]
+  uint16_t* s_chk = reinterpret_cast<uint16_t*>(s_key + kSelResolveCap);        // [kSelResolveCap]
+  int* s_gt = reinterpret_cast<int*>(s_chk + kSelResolveCap);                   // [kSelMaxChunks]
+  int* s_eq = s_gt + kSelMaxChunks;                                             // [kSelMaxChunks]
+  constexpr int NT = kSelCtaThreads;
+  const int g = p.heads[y], tid = threadIdx.x;
   int off;
   const int L = seq_length(p.offsets, p.lengths, b, false, &off);
   const int n = sel_n(p, b, L, false);
-  if (n == 0 || n >= L) return;  // nothing to select: the write pass alone
+  if (n == 0 || n >= L) return;  // nothing to select: the write phase alone
   const int64_t rid = (int64_t)g * p.B + b;
   const int nch = (L + kSelChunk - 1) / kSelChunk;
   const unsigned long long* cand = p.cand + (int64_t)g * p.T + off;
   const int T1 = __ldcg(p.row_info + rid * kRowInfo), above1 = __ldcg(p.row_info + rid * kRowInfo + 1);
   const int m = __ldcg(p.cand_count + rid);
   const bool in_smem = m <= kSelResolveCap;
+  __syncthreads();  // the scratch may still be read for the previous item
   if (in_smem) {
-    for (int j = tid; j < m; j += kSelResolveThreads) {
+    for (int j = tid; j < m; j += NT) {
       const unsigned long long e = __ldcg(cand + j);
       s_key[j] = (uint32_t)(e >> 32);
       s_chk[j] = (uint16_t)((uint32_t)e / kSelChunk);
     }
   }
-  for (int q = tid; q < nch; q += kSelResolveThreads) {
+  for (int q = tid; q < nch; q += NT) {
     s_gt[q] = 0;
     s_eq[q] = 0;
   }
-  for (int i = tid; i < kSelHistBins; i += kSelResolveThreads) p.hist[rid * kSelHistBins + i] = 0u;
+  for (int i = tid; i < kSelHistBins; i += NT) p.hist[rid * kSelHistBins + i] = 0u;
   uint32_t prefix = (uint32_t)T1 << kSelHistShift, pmask = 0xffffffffu << kSelHistShift;
   int krem = n - above1;
 #pragma unroll 1
   for (int d = 0; d < 2; ++d) {
     const int sh = d == 0 ? 10 : 0;
     const int nb = d == 0 ? 2048 : 1024;
-    for (int i = tid; i < nb; i += kSelResolveThreads) s_hist[i] = 0;
+    for (int i = tid; i < nb; i += NT) s_hist[i] = 0;
     __syncthreads();
-    for (int j = tid; j < m; j += kSelResolveThreads) {
+    for (int j = tid; j < m; j += NT) {
       const uint32_t kj = in_smem ? s_key[j] : (uint32_t)(__ldcg(cand + j) >> 32);
       if ((kj & pmask) == prefix) atomicAdd(&s_hist[(kj >> sh) & (nb - 1)], 1);
     }
     __syncthreads();
-    // bins from the top: thread t takes per = nb / 512 consecutive bins
-    const int per = nb / kSelResolveThreads;
-    int cnt[4], sum = 0;
+    // bins from the top: thread t takes per = nb / NT consecutive bins
+    const int per = nb / NT;
+    int cnt[8], sum = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       cnt[u] = u < per ? s_hist[nb - 1 - (tid * per + u)] : 0;
       sum += cnt[u];
     }
@@ -273,7 +269,7 @@ __global__ void __launch_bounds__(kSelResolveThreads) select_resolve_kernel(cons
     int excl = block_exclusive_scan(sum, scratch, &total);
     if (excl < krem && krem <= excl + sum) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         if (u < per && excl < krem && krem <= excl + cnt[u]) {
           s_out[0] = nb - 1 - (tid * per + u);
           s_out[1] = excl;
@@ -292,7 +288,7 @@ __global__ void __launch_bounds__(kSelResolveThreads) select_resolve_kernel(cons
   }
   const int need_eq = krem;  // keys equal (masked) to the prefix that are taken, lowest positions first
   // candidates above / equal to the threshold, per chunk
-  for (int j = tid; j < m; j += kSelResolveThreads) {
+  for (int j = tid; j < m; j += NT) {
     uint32_t kj;
     int q;
     if (in_smem) {
@@ -309,7 +305,7 @@ __global__ void __launch_bounds__(kSelResolveThreads) select_resolve_kernel(cons
   }
   __syncthreads();
   // offsets: thread t owns chunks [t * per, (t + 1) * per)
-  const int per = (nch + kSelResolveThreads - 1) / kSelResolveThreads;
+  const int per = (nch + NT - 1) / NT;
   const int q0 = min(nch, tid * per), q1 = min(nch, q0 + per);
   int sel_t = 0, eq_t = 0;
   for (int q = q0; q < q1; ++q) {
@@ -332,15 +328,10 @@ __global__ void __launch_bounds__(kSelResolveThreads) select_resolve_kernel(cons
   }
 }
 
-// ---------------------------------------------------------------------------- ordered write
-// Every chunk writes its selected positions at the offset the resolve gave it, in order: warps
-// own runs of 32 x kWriteK consecutive keys, one block scan ranks the warps, ballots rank the
-// picks inside a warp.
-__global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const HistSelectParams p) {
-  grid_dep_wait();  // inputs come from the kernels before this one
-  grid_dep_launch();
-  __shared__ int scratch[33];
-  const int c = blockIdx.x, g = p.heads[blockIdx.y], b = blockIdx.z, tid = threadIdx.x;
+// ---------------------------------------------------------------------------- write phase
+__device__ __forceinline__ void sel_write_item(const HistSelectParams& p, uint8_t* sm, int c, int y, int b) {
+  int* scratch = reinterpret_cast<int*>(sm);  // [33]
+  const int g = p.heads[y], tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   int off;
   const int L = seq_length(p.offsets, p.lengths, b, false, &off);
@@ -382,6 +373,7 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const Hist
   }
   ngt = __reduce_add_sync(0xffffffffu, ngt);
   neq = __reduce_add_sync(0xffffffffu, neq);
+  __syncthreads();  // the scratch may still be read for the previous item
   int tot;
   // warp offsets inside the chunk (lane 0 of each warp contributes its warp's counts)
   const int packed = block_exclusive_scan(lane == 0 ? ((ngt << 16) | neq) : 0, scratch, &tot);
@@ -406,6 +398,36 @@ __global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const Hist
     sel_before += __popc(bt);
     eq_before += __popc(beq);
   }
+}
+
+// ---------------------------------------------------------------------------- kernels
+// One kernel per phase: grid (max_chunks, listed heads, sequences); the resolve (1, heads, sequences).
+__global__ void __launch_bounds__(kSelCtaThreads) select_hist_kernel(const HistSelectParams p) {
+  grid_dep_wait();  // inputs come from the kernel before this one
+  grid_dep_launch();
+  __shared__ __align__(16) uint8_t sm[4 * kSelHistBins];
+  sel_hist_item(p, sm, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+__global__ void __launch_bounds__(kSelCtaThreads) select_chunk_kernel(const HistSelectParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  __shared__ __align__(16) uint8_t sm[256];
+  sel_chunk_item(p, sm, blockIdx.x, blockIdx.y, blockIdx.z);
+}
+
+__global__ void __launch_bounds__(kSelCtaThreads) select_resolve_kernel(const HistSelectParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  __shared__ __align__(16) uint8_t sm[kSelSmem];
+  sel_resolve_row(p, sm, blockIdx.y, blockIdx.z);
+}
+
+__global__ void __launch_bounds__(kSelCtaThreads) select_write_kernel(const HistSelectParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  __shared__ __align__(16) uint8_t sm[256];
+  sel_write_item(p, sm, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 }  // namespace aoh
