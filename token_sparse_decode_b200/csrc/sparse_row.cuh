@@ -173,56 +173,16 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   }
   if (role == 0 && n < L) {
     // =============================================================== 1. scan
-    if (tid < p.srow_len) {
-      const int C = D / 2;
-      int dim = -1;
-      if (p.packed) {
-        if (tid < 2 * p.n_dom) {
-          const int j = tid < p.n_dom ? tid : tid - p.n_dom;
-          const int c = p.idom[g * p.n_dom + j];
-          if (c < 0 || c >= C) {
-            record_error(kCheckChunk, g, j, c);
-          } else {
-            dim = tid < p.n_dom ? c : c + C;
-          }
-        }
-      } else if (p.idom == nullptr) {
-        dim = tid;  // every chunk: the full dot
-      } else {
-        const int c = tid < C ? tid : tid - C;
-        for (int j = 0; j < p.n_dom; ++j) {
-          const int cj = p.idom[g * p.n_dom + j];
-          if (cj < 0 || cj >= C) record_error(kCheckChunk, g, j, cj);
-          if (cj == c) dim = tid;
-        }
-      }
-      float acc = 0.f;
-      if (dim >= 0) {
-        const uint16_t* qb = p.q_score + ((int64_t)b * p.Hq + (int64_t)g * p.G) * D + dim;
-        for (int h0 = 0; h0 < p.G; h0 += 8) {  // eight loads in flight, summed in head order
-          float qv[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            qv[u] = (h0 + u < p.G) ? __uint_as_float((uint32_t)qb[(int64_t)(h0 + u) * D] << 16) : 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) acc += qv[u];
-        }
-      }
-      qt[tid] = acc;
-    }
-    __syncthreads();
     {
       // Each warp streams a contiguous run of the slice's rows through its own cp.async
       // ring: S lanes share a row (16 bytes each), kScanU rows per lane per group,
-      // kScanDepth groups in flight.  A lane reads back only the bytes it copied, so the
-      // ring needs no barrier; the dot and its shuffle reduction match the stand-alone
-      // scan kernel term for term (same fp32 scores, same keys).
+      // kScanDepth groups in flight; the first groups are issued before the group-summed
+      // query is built (its loads then overlap theirs).  A lane reads back only the bytes it
+      // copied, so the ring needs no barrier; the dot and its shuffle reduction match the
+      // stand-alone scan kernel term for term (same fp32 scores, same keys).
       const int S = p.srow_len >> 3;  // 2, 4, 8 or 16
       const int seg = lane & (S - 1);
       const int rpw = 32 / S;
-      float qs[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) qs[i] = qt[seg * 8 + i];
       const int per_warp = (m + 7) / 8;
       const int wr0 = min(m, warp * per_warp), wr1 = min(m, wr0 + per_warp);
       const int grows = rpw * kScanU;
@@ -243,6 +203,47 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
         if (k < nb) issue(k);
         cp_async_commit();
       }
+      if (tid < p.srow_len) {
+        const int C = D / 2;
+        int dim = -1;
+        if (p.packed) {
+          if (tid < 2 * p.n_dom) {
+            const int j = tid < p.n_dom ? tid : tid - p.n_dom;
+            const int c = p.idom[g * p.n_dom + j];
+            if (c < 0 || c >= C) {
+              record_error(kCheckChunk, g, j, c);
+            } else {
+              dim = tid < p.n_dom ? c : c + C;
+            }
+          }
+        } else if (p.idom == nullptr) {
+          dim = tid;  // every chunk: the full dot
+        } else {
+          const int c = tid < C ? tid : tid - C;
+          for (int j = 0; j < p.n_dom; ++j) {
+            const int cj = p.idom[g * p.n_dom + j];
+            if (cj < 0 || cj >= C) record_error(kCheckChunk, g, j, cj);
+            if (cj == c) dim = tid;
+          }
+        }
+        float acc = 0.f;
+        if (dim >= 0) {
+          const uint16_t* qb = p.q_score + ((int64_t)b * p.Hq + (int64_t)g * p.G) * D + dim;
+          for (int h0 = 0; h0 < p.G; h0 += 8) {  // eight loads in flight, summed in head order
+            float qv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              qv[u] = (h0 + u < p.G) ? __uint_as_float((uint32_t)qb[(int64_t)(h0 + u) * D] << 16) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc += qv[u];
+          }
+        }
+        qt[tid] = acc;
+      }
+      __syncthreads();
+      float qs[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qs[i] = qt[seg * 8 + i];
       for (int k = 0; k < nb; ++k) {
         if (k + kScanDepth - 1 < nb) issue(k + kScanDepth - 1);
         cp_async_commit();
