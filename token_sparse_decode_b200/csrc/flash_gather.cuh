@@ -13,8 +13,8 @@
 //
 // Work split: blockIdx = (split, listed KV head, sequence).  A CTA owns `chunk`
 // consecutive list entries, streams their K and V rows through a 3-stage cp.async
-// pipeline into 128-byte-swizzled shared tiles, and runs the contraction on tensor
-// cores with the tokens on the M side:
+// pipeline into 128-byte-swizzled shared tiles, and runs the contraction on tensor cores
+// with the tokens on the M side:
 //     S^T[16 tok x 8 q] = K[16 tok x d] . Q^T[d x 8 q]          (m16n8k16, bf16)
 //     O^T[d x 8 q]     += V^T[d x 16 tok] . P^T[16 tok x 8 q]
 // so G <= 8 query rows fill the N = 8 side of one MMA (G = 7: 7/8 useful) instead
@@ -23,8 +23,10 @@
 // layout to the B-operand layout with movmatrix.trans.  Softmax is online in fp32
 // (exp2 domain).  Each CTA leaves (m, l, acc) for its chunk; they are merged either
 // in a thread-block cluster of the row's splits (rows of about equal length with
-// 2-16 splits: distributed shared memory, each CTA writes 1/CL of the outputs) or by
-// the last CTA of the row through the workspace (atomic ticket, re-armed to zero).
+// 2-16 splits: distributed shared memory, each CTA writes 1/CL of the outputs, every
+// thread fetching its row's (m, l) and the peers' partials in one round of remote loads
+// per 8 peers) or by the last CTA of the row through the workspace (atomic ticket,
+// re-armed to zero).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -89,6 +91,7 @@ __device__ __forceinline__ uint32_t fd_tile_off(int r, int dd) {
 
 template <int D, int NT>
 __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const FdecParams p) {
+  constexpr int ST = kFdStages;
   grid_dep_wait();  // the selection comes from the kernel before this one
   grid_dep_launch();
   static_assert(D == 64 || D == 128, "head_dim");
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
 
   auto issue_stage = [&](int st) {
     if (st < nstages) {
-      const uint32_t kt = sbase + (st % kFdStages) * FdTile<D>::kStageBytes;
+      const uint32_t kt = sbase + (st % ST) * FdTile<D>::kStageBytes;
       const uint32_t vt = kt + FdTile<D>::kTileBytes;
 #pragma unroll
       for (int c = tid; c < kFdTS * CPR; c += kFdThreads) {
@@ -240,13 +243,13 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // q rows 2*(lane%4) and +1
 
 #pragma unroll
-  for (int s = 0; s < kFdStages - 1; ++s) issue_stage(s);
+  for (int s = 0; s < ST - 1; ++s) issue_stage(s);
 
   for (int st = 0; st < nstages; ++st) {
-    cp_async_wait<kFdStages - 2>();
+    cp_async_wait<ST - 2>();
     __syncthreads();
-    issue_stage(st + kFdStages - 1);
-    const uint32_t kt = sbase + (st % kFdStages) * FdTile<D>::kStageBytes;
+    issue_stage(st + ST - 1);
+    const uint32_t kt = sbase + (st % ST) * FdTile<D>::kStageBytes;
     const uint32_t vt = kt + FdTile<D>::kTileBytes;
 #pragma unroll
     for (int i = 0; i < SUB / WT; ++i) {
@@ -350,8 +353,6 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     float* cm = reinterpret_cast<float*>(smem + kFdMergeOff);  // [NQP]
     float* cls = cm + NQP;                                      // [NQP]
     float* ca = cls + NQP;                                      // [NQP][D]
-    float* cw = ca + NQP * D;                                   // [16][NQP] merge weights
-    float* cinv = cw + 16 * NQP;                                // [NQP]
     for (int e = tid; e < NQP * D; e += kFdThreads) {
       const int qr = e / D, dd = e % D;
       const int ntq = qr >> 3, cq = qr & 7;
@@ -374,58 +375,55 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
       }
     }
     cluster.sync();
-    // every peer's (M, L) of a query row: all remote loads issued before any is used
-    if (tid < NQP) {
-      float mv[kFdMaxCluster], lv[kFdMaxCluster];
-#pragma unroll
-      for (int q = 0; q < kFdMaxCluster; ++q) {
-        mv[q] = q < CLn ? cluster.map_shared_rank(cm, q)[tid] : -INFINITY;
-        lv[q] = q < CLn ? cluster.map_shared_rank(cls, q)[tid] : 0.f;
-      }
-      float Mx = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < kFdMaxCluster; ++q) Mx = fmaxf(Mx, mv[q]);
-      float Ls = 0.f;
-#pragma unroll
-      for (int q = 0; q < kFdMaxCluster; ++q) {
-        if (q < CLn) {
-          const float w = (mv[q] == -INFINITY) ? 0.f : exp2f(mv[q] - Mx);
-          cw[q * NQP + tid] = w;
-          Ls += w * lv[q];
-        }
-      }
-      cinv[tid] = 1.f / Ls;
-    }
-    __syncthreads();
-    // outputs 4 consecutive dims at a time, 16-byte reads of the peers' partials, 4 peers' reads
-    // in flight together; the peers are summed in rank order
+    // outputs 4 consecutive dims at a time: each thread fetches its row's (M, L) from every
+    // peer together with the peers' 16-byte partials (batches of 8 peers, all of a batch's
+    // remote loads in flight together; a running rescale joins the batches)
     for (int e4 = rk * kFdThreads + tid; e4 < p.NQ * D / 4; e4 += CLn * kFdThreads) {
       const int e = 4 * e4, qr = e / D, dd = e % D;
+      float Mx = -INFINITY, Ls = 0.f;
       float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q0 = 0; q0 < CLn; q0 += 4) {
-        float4 v[4];
+      for (int q0 = 0; q0 < CLn; q0 += 8) {
+        float mv[8], lv[8];
+        float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          v[u] = q0 + u < CLn ? *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, q0 + u) + e)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           if (q0 + u < CLn) {
-            const float w = cw[(q0 + u) * NQP + qr];
-            A.x += w * v[u].x;
-            A.y += w * v[u].y;
-            A.z += w * v[u].z;
-            A.w += w * v[u].w;
+            mv[u] = cluster.map_shared_rank(cm, q0 + u)[qr];
+            lv[u] = cluster.map_shared_rank(cls, q0 + u)[qr];
+            v[u] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, q0 + u) + e);
+          } else {
+            mv[u] = -INFINITY;
+            lv[u] = 0.f;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
+        float Mb = Mx;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) Mb = fmaxf(Mb, mv[u]);
+        const float sc = (Mx == -INFINITY) ? 0.f : exp2f(Mx - Mb);
+        Ls *= sc;
+        A.x *= sc;
+        A.y *= sc;
+        A.z *= sc;
+        A.w *= sc;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float w = (mv[u] == -INFINITY) ? 0.f : exp2f(mv[u] - Mb);
+          Ls += w * lv[u];
+          A.x += w * v[u].x;
+          A.y += w * v[u].y;
+          A.z += w * v[u].z;
+          A.w += w * v[u].w;
+        }
+        Mx = Mb;
       }
-      const float sc = cinv[qr];
+      const float inv = 1.f / Ls;
       const int l = qr / p.G, h = g * p.G + qr % p.G;
       float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
-      o[0] = A.x * sc;
-      o[1] = A.y * sc;
-      o[2] = A.z * sc;
-      o[3] = A.w * sc;
+      o[0] = A.x * inv;
+      o[1] = A.y * inv;
+      o[2] = A.z * inv;
+      o[3] = A.w * inv;
     }
     cluster.sync();  // peers read this CTA's shared memory until here
     return;
