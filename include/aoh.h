@@ -160,7 +160,8 @@ typedef enum {
   AOH_KERNEL_SELECT_WRITE = 13, /* select: ordered write of the chosen positions     */
   AOH_KERNEL_SELECT_CLUSTER = 14, /* select: one cluster per row, keys on chip      */
   AOH_KERNEL_SELECT_RESOLVE = 15, /* select: exact threshold and chunk offsets per row */
-  AOH_KERNEL_KINDS = 16
+  AOH_KERNEL_FLASH_MERGE = 16,  /* split-K combine of rows with many splits           */
+  AOH_KERNEL_KINDS = 17
 } aoh_kernel_kind;
 
 /*

@@ -204,6 +204,191 @@ def test_topk_cluster_slice_edges(L):
     check_topk(s, offs, lengths, nfps, 2048, {"select_cluster_kernel": 1}, "normal")
 
 
+def test_topk_fixed_nfac_and_determinism():
+    rng = np.random.default_rng(6)
+    lengths = [131072, 4096, 777]
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = (np.round(rng.standard_normal((2, int(offs[-1]))) * 8) / 8).astype(np.float32)
+    dev = torch.device("cuda")
+    k = torch.zeros((int(offs[-1]), 2, 64), dtype=torch.bfloat16, device=dev)
+    kv = B.make_kv(k, k, torch.from_numpy(offs).to(dev), max(lengths), int(offs[-1]))
+    sd = torch.from_numpy(s).to(dev)
+    outs = []
+    for _ in range(2):
+        idx = torch.empty((3, 2, 2048), dtype=torch.int32, device=dev)
+        cnt = torch.empty((3, 2), dtype=torch.int32, device=dev)
+        B.topk_select(sd, kv, 2048, None, 2048, idx, cnt)
+        torch.cuda.synchronize()
+        outs.append((idx.cpu().numpy(), cnt.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    for b in range(3):
+        for g in range(2):
+            ref = oracle.select_top(s[g, offs[b]:offs[b + 1]], 2048)
+            assert np.array_equal(outs[0][0][b, g, :len(ref)], ref)
+
+
+# ------------------------------------------------------------------------------ sparse decode
+
+
+@pytest.mark.parametrize("name", list(MEDIUM))
+@pytest.mark.parametrize("pack", [True, False])
+def test_sparse_decode_matches_oracle(name, pack):
+    w = make_workload(MEDIUM[name])
+    d = Dev(w)
+    step, out = run_sparse(d, pack=pack)
+    # a few rows: the whole path in one cluster launch
+    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = w.spec.group
+    stats = {}
+    for b in range(w.spec.batch):
+        for g in range(w.spec.n_kv_heads):
+            n = cnt_h[b, g]
+            compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G], stats)
+    assert stats["swapped"] <= max(1, stats["rows"] // 10)
+
+
+def test_sparse_decode_is_deterministic():
+    w = make_workload(MEDIUM["gqa4_d128"])
+    d = Dev(w)
+    step, out = run_sparse(d)
+    first = out.clone()
+    step(d.q)
+    torch.cuda.synchronize()
+    assert torch.equal(first, step.out)
+
+
+# ------------------------------------------------------------------------------ retrieval / streaming heads
+
+
+@pytest.mark.parametrize("sink,window", [(4, 60), (128, 512), (0, 100), (3000, 4000), (0, 0)])
+def test_stream_decode_matches_oracle(sink, window):
+    roles = (ROLE_DENSE, ROLE_STREAM, ROLE_STREAM, ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_STREAM, ROLE_STREAM)
+    w = make_workload(spec(roles=roles, sink=sink, window=window, len_range=(0, 7000), seed=81))
+    d = Dev(w)
+    kv = d.kv()
+    out = torch.full((w.spec.batch, w.spec.n_q_heads, w.spec.head_dim), 777.0, device="cuda")
+    ws = B.workspace(B.stream_decode_workspace_size(kv, w.spec.n_q_heads, roles, sink, window), "cuda")
+    B.stream_decode(d.q, kv, roles, sink, window, w.scale, out, ws)
+    torch.cuda.synchronize()
+    check_device()
+    out_h = f64(out)
+    G = w.spec.group
+    for b in range(w.spec.batch):
+        for g, role in enumerate(roles):
+            rows = out_h[b, g * G:(g + 1) * G]
+            if role == ROLE_SPARSE:
+                assert np.all(rows == 777.0)   # not this call's heads: untouched
+            else:
+                compare_window_row(w, b, g, rows, role, sink, window)
+
+
+def test_long_dense_rows_merge_in_a_second_launch():
+    # DENSE rows of 60-90 K positions split into more than 16 parts: the gather leaves its
+    # partials and flash_merge_kernel combines them over many CTAs; the short STREAM rows of
+    # the same launch (one or a few splits) go through the same merge
+    roles = (ROLE_DENSE, ROLE_STREAM, ROLE_DENSE, ROLE_STREAM)
+    w = make_workload(spec(n_q_heads=16, n_kv_heads=4, roles=roles, sink=64, window=512, len_range=(60000, 90000),
+                           batch=2, seed=89))
+    d = Dev(w)
+    kv = d.kv()
+    out = torch.full((w.spec.batch, w.spec.n_q_heads, w.spec.head_dim), 777.0, device="cuda")
+    ws = B.workspace(B.stream_decode_workspace_size(kv, w.spec.n_q_heads, roles, 64, 512), "cuda")
+    launched = launches_of(lambda: B.stream_decode(d.q, kv, roles, 64, 512, w.scale, out, ws))
+    assert launched == {"flash_gather_kernel": 1, "flash_merge_kernel": 1}
+    check_device()
+    out_h = f64(out)
+    G = w.spec.group
+    for b in range(w.spec.batch):
+        for g, role in enumerate(roles):
+            compare_window_row(w, b, g, out_h[b, g * G:(g + 1) * G], role, 64, 512)
+
+
+def test_full_role_split_step_mixed_heads():
+    # every row in one wave and window lists no longer than 4 x N_fac: the whole step, window
+    # heads included, is one launch of the row kernel
+    roles = (ROLE_SPARSE, ROLE_DENSE, ROLE_STREAM, ROLE_SPARSE)
+    w = make_workload(spec(n_q_heads=16, n_kv_heads=4, roles=roles, sink=16, window=200, n_fac_div=4, seed=82))
+    d = Dev(w)
+    step, out = run_sparse(d)
+    assert launches_of(lambda: step(d.q)) == {"sparse_row_kernel": 1}
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = w.spec.group
+    for b in range(w.spec.batch):
+        for g, role in enumerate(roles):
+            rows = out_h[b, g * G:(g + 1) * G]
+            if role == ROLE_SPARSE:
+                compare_sparse_row(w, b, g, idx_h[b, g, :cnt_h[b, g]], rows)
+            else:
+                compare_window_row(w, b, g, rows, role, w.spec.sink, w.spec.window)
+
+
+# ------------------------------------------------------------------------------ shared index
+
+
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("n_layers,hq,hkv", [(8, 32, 8), (2, 16, 4), (3, 16, 4), (1, 8, 8)])
+def test_shared_index_decode_matches_oracle(n_layers, hq, hkv, fused):
+    sp = WorkloadSpec(name="shared", batch=2, n_q_heads=hq, n_kv_heads=hkv, head_dim=128, theta=5e5,
+                      len_range=(500, 9000), n_layers=n_layers, topk_shared=700, seed=90 + n_layers)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_shared(d, fused=fused)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = sp.group
+    ref = oracle.shared_index_step(f64(w.q), f64(w.q_layers), f64(w.k), f64(w.v), w.offsets.tolist(), 700,
+                                   w.scale)
+    for (b, g), r in ref.items():
+        sel = idx_h[b, g, :cnt_h[b, g]]
+        compare_shared_row(w, b, g, sel, out_h[:, b, g * G:(g + 1) * G], 700)
+        if np.array_equal(sel, r["sel"]):  # the stack's own oracle on the same index
+            assert np.abs(out_h[:, b, g * G:(g + 1) * G] - r["out"]).max() <= OUT_ATOL
+
+
+def test_shared_index_reports_out_of_range_positions():
+    sp = WorkloadSpec(name="shared", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, theta=1e4,
+                      lengths=(300,), n_layers=2, topk_shared=16, seed=3)
+    w = make_workload(sp)
+    d = Dev(w)
+    kv = d.kv()
+    idx = torch.arange(16, dtype=torch.int32, device="cuda").repeat(1, 2, 1).contiguous()
+    idx[0, 1, 5] = 300            # one past the end of the sequence
+    cnt = torch.full((1, 2), 16, dtype=torch.int32, device="cuda")
+    out = torch.empty((2, 1, 8, 64), device="cuda")
+    ws = B.workspace(B.shared_index_decode_workspace_size(kv, 2, 8, 16), "cuda")
+    B.shared_index_decode(d.q_layers, kv, idx, cnt, 16, w.scale, out, ws)
+    st, detail = B.device_check()
+    assert st == 6 and detail[0] == 1 and detail[3] == 300
+    assert B.device_check()[0] == 0   # reading clears the word
+    assert torch.isfinite(out).all()
+
+
+# ------------------------------------------------------------------------------ edge cases
+
+
+def test_edge_cases_empty_and_short_sequences():
+    sp = spec(batch=5, lengths=(0, 1, 2, 64, 65), len_range=None, n_fac_div=0, n_fac=64, n_dom=3,
+              planted_frac=0.0, seed=84)
+    w = make_workload(sp)
+    d = Dev(w)
+    step, out = run_sparse(d)
+    out_h = f64(out)
+    idx_h, cnt_h = step.idx.cpu().numpy(), step.count.cpu().numpy()
+    G = sp.group
+    for b in range(sp.batch):
+        for g in range(sp.n_kv_heads):
+            n = cnt_h[b, g]
+            assert n == min(64, int(w.lengths[b]))
+            if w.lengths[b] == 0:
+                assert np.all(out_h[b, g * G:(g + 1) * G] == 0.0)
+            else:
+                compare_sparse_row(w, b, g, idx_h[b, g, :n], out_h[b, g * G:(g + 1) * G])
+            assert np.all(idx_h[b, g, n:] == -1)
+
+
 def test_sparse_decode_long_row_uses_three_kernels():
     # a row longer than one cluster handles (262144 positions) takes the scan / select / attend path
     sp = WorkloadSpec(name="long", batch=1, n_q_heads=2, n_kv_heads=1, head_dim=64, theta=1e4, lengths=(300001,),

@@ -37,7 +37,7 @@ KERNELS = ("tip_score_kernel", "select_hist_kernel", "sparse_row_kernel", "flash
            "pack_dominant_kernel", "kv_append_kernel", "gram_kernel", "gram_reduce_kernel", "spectrum_kernel",
            "group_roles_kernel", "offload_stage_kernel", "offload_split_kernel", "select_chunk_kernel",
            "select_write_kernel", "select_cluster_kernel",
-           "select_resolve_kernel")
+           "select_resolve_kernel", "flash_merge_kernel")
 
 
 class AohError(RuntimeError):

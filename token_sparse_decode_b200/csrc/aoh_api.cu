@@ -285,9 +285,22 @@ aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStr
   const bool merge_on_chip =
       uniform && CL >= 2 && CL <= kFdMaxCluster && max_active_clusters(kern, CL, smem, threads) > 0;
   fp.cluster_combine = merge_on_chip ? 1 : 0;
-  const aoh_status s = launch_dependent(kern, grid, threads, smem, merge_on_chip ? CL : 0, st, fp);
+  // rows with many splits and no cluster merge: the gather leaves partials and a second launch
+  // combines them over many CTAs (one CTA merging up to 256 splits is latency-bound)
+  fp.defer_merge = (!merge_on_chip && fp.max_splits > kFdMaxCluster) ? 1 : 0;
+  aoh_status s = launch_dependent(kern, grid, threads, smem, merge_on_chip ? CL : 0, st, fp);
   if (s != AOH_OK) return s;
-  return count_launch(AOH_KERNEL_FLASH_GATHER, st);
+  if ((s = count_launch(AOH_KERNEL_FLASH_GATHER, st)) != AOH_OK || !fp.defer_merge) return s;
+  constexpr int NQP = NT * 8;
+  const dim3 mgrid((unsigned)ceil_div(int64_t(fp.NQ) * (D / 4), kFmOut), n_listed, B);
+  const size_t msmem = sizeof(float) * 2 * (size_t)fp.max_splits * NQP;  // <= 2 x 256 x 32 floats
+  static std::atomic<uint64_t> merge_configured{0};
+  if (!set_up_on_this_device(merge_configured)) {
+    if ((s = set_smem(flash_merge_kernel<D, NT>, sizeof(float) * 2 * kFdMaxSplits * NQP)) != AOH_OK) return s;
+    mark_set_up(merge_configured);
+  }
+  if ((s = launch_dependent(flash_merge_kernel<D, NT>, mgrid, kFmThreads, msmem, 0, st, fp)) != AOH_OK) return s;
+  return count_launch(AOH_KERNEL_FLASH_MERGE, st);
 }
 
 // `uniform`: every row attends to about the same number of positions (a fixed N_fac or k)

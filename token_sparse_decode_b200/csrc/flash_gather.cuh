@@ -65,6 +65,8 @@ struct FdecParams {
   int32_t max_splits;
   int32_t list_mode;         // 1: positions from idx/count; 0: role ranges
   int32_t cluster_combine;   // 1: launched with clusters of max_splits CTAs (one row each)
+  int32_t defer_merge;       // 1: the CTAs of a row with several splits only leave their partials
+                             //    (flash_merge_kernel combines them)
   int32_t sink, window;
   int32_t ring_sink, ring_window;  // range mode on a ring cache (> 0 sum): position p is kept in
                                    // slot ring_slot(p); 0, 0: position p is token p of the region
@@ -87,6 +89,25 @@ __device__ __forceinline__ uint32_t fd_tile_off(int r, int dd) {
   const int half = dd >> 6;
   const int cc = (dd & 63) >> 3;
   return (uint32_t)(half * (kFdTS * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+}
+
+// The number of positions row (b, g) attends to, and for a role range the split [0, ra) U
+// [rb, L): list mode takes the selection's count (clamped to [0, cap]); a ring region too small
+// for its slots attends to nothing.
+__device__ __forceinline__ int fd_row_count(const FdecParams& p, int b, int g, int L, int off, bool ring, int* ra,
+                                            int* rb) {
+  *ra = 0;
+  *rb = 0;
+  if (p.list_mode) return max(0, min(p.count[b * p.Hkv + g], p.cap));
+  if (ring && p.offsets[b + 1] - off < p.ring_sink + p.ring_window) return 0;
+  if (p.roles[g] == 1) {  // DENSE
+    *ra = L;
+    *rb = L;
+  } else {                // STREAM
+    *ra = min(p.sink, L);
+    *rb = max(*ra, L - p.window);
+  }
+  return *ra + (L - *rb);
 }
 
 template <int D, int NT>
@@ -119,29 +140,11 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   const int L = seq_length(p.offsets, p.lengths, b, ring, &off);
 
   // ---- the row's list of positions
-  int n, ra = 0, rb = 0;
-  const int32_t* lst = nullptr;
-  if (p.list_mode) {
-    n = p.count[b * p.Hkv + g];
-    if (n > p.cap) {
-      if (split == 0 && tid == 0) record_error(kCheckCount, b, g, n);
-      n = p.cap;
-    }
-    n = max(n, 0);
-    lst = p.idx + ((int64_t)b * p.Hkv + g) * p.cap;
-  } else if (ring && p.offsets[b + 1] - off < p.ring_sink + p.ring_window) {
-    // a ring region too small for its slots: nothing is read (recorded once, below)
-    n = 0;
-  } else {
-    if (p.roles[g] == 1) {  // DENSE
-      ra = L;
-      rb = L;
-    } else {                // STREAM
-      ra = min(p.sink, L);
-      rb = max(ra, L - p.window);
-    }
-    n = ra + (L - rb);
-  }
+  int ra, rb;
+  const int n = fd_row_count(p, b, g, L, off, ring, &ra, &rb);
+  if (p.list_mode && split == 0 && tid == 0 && p.count[b * p.Hkv + g] > p.cap)
+    record_error(kCheckCount, b, g, p.count[b * p.Hkv + g]);
+  const int32_t* lst = p.list_mode ? p.idx + ((int64_t)b * p.Hkv + g) * p.cap : nullptr;
   const int nsplit = (n + p.chunk - 1) / p.chunk;
 
   if (n == 0) {  // nothing to attend to: zero rows
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
       }
     }
   }
-  if (single) return;
+  if (single || p.defer_merge) return;
 
   // ---- split-K combine by the last CTA of the row
   __threadfence();
@@ -548,6 +551,123 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     o[3] = A.w * inv;
   }
   if (tid == 0) p.tickets[row_id] = 0;
+}
+
+// Split-K combine of rows with many splits, spread over CTAs: grid (slices of 16 float4
+// outputs, listed heads, sequences), 128 threads.  Every CTA stages the row's (m, l) pairs in
+// shared memory and weighs the splits itself (w[s][q] = 2^(m_sq - M_q), L_q = sum of w l, in
+// split order), then thread (o, s0) sums splits s0, s0 + 8, ...
+// of output float4 o with all of its loads in flight, and the 8 split groups are added in a
+// fixed order.  Rows with one split were written by the gather.
+constexpr int kFmThreads = 128;
+constexpr int kFmOut = 16;                    // float4 outputs per CTA
+constexpr int kFmGroups = kFmThreads / kFmOut;  // 8 split groups
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kFmThreads) flash_merge_kernel(const FdecParams p) {
+  grid_dep_wait();  // the partials come from the gather before this launch
+  constexpr int NQP = NT * 8;
+  extern __shared__ __align__(16) uint8_t fm_smem[];
+  float* sml = reinterpret_cast<float*>(fm_smem);  // [nsplit][NQP][2]: (m, l), then (w, l)
+  __shared__ float sL[NQP];
+  __shared__ float4 sred[kFmGroups][kFmOut];
+  const int tid = threadIdx.x;
+  const int b = blockIdx.z, y = blockIdx.y, g = p.heads[y];
+  const int row_id = b * gridDim.y + y;
+  const bool ring = (p.ring_sink + p.ring_window) > 0;
+  int off, ra, rb;
+  const int L = seq_length(p.offsets, p.lengths, b, ring, &off);
+  const int n = fd_row_count(p, b, g, L, off, ring, &ra, &rb);
+  const int nsplit = (n + p.chunk - 1) / p.chunk;
+  const int n_out = p.NQ * (D / 4);
+  const int o0 = blockIdx.x * kFmOut;
+  if (nsplit <= 1 || o0 >= n_out) return;
+  const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
+  const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
+  // weights: the row's (m, l) pairs staged in shared memory with one pass of independent
+  // loads, then per query row M_q = max m, w[s][q] = 2^(m_sq - M_q), L_q = sum of w l
+  for (int e = tid; e < nsplit * NQP * 2; e += kFmThreads) sml[e] = __ldcg(rml + e);
+  __syncthreads();
+  // thread t takes query row t % NQP over the splits t / NQP, + SP, ...; the partial maxima
+  // and sums are combined in a fixed order
+  constexpr int SP = kFmThreads / NQP;
+  __shared__ float s_part[kFmThreads], sM[NQP];
+  const int rq = tid % NQP, sj = tid / NQP;
+  {
+    float M = -INFINITY;
+    for (int s2 = sj; s2 < nsplit; s2 += SP) M = fmaxf(M, sml[(s2 * NQP + rq) * 2]);
+    s_part[tid] = M;
+  }
+  __syncthreads();
+  if (tid < NQP) {
+    float M = -INFINITY;
+    for (int j2 = 0; j2 < SP; ++j2) M = fmaxf(M, s_part[j2 * NQP + tid]);
+    sM[tid] = M;
+  }
+  __syncthreads();
+  {
+    float Ls = 0.f;
+    for (int s2 = sj; s2 < nsplit; s2 += SP) {
+      const float m = sml[(s2 * NQP + rq) * 2];
+      const float w = (m == -INFINITY) ? 0.f : exp2f(m - sM[rq]);
+      sml[(s2 * NQP + rq) * 2] = w;  // the weight replaces m
+      Ls += w * sml[(s2 * NQP + rq) * 2 + 1];
+    }
+    s_part[tid] = Ls;
+  }
+  __syncthreads();
+  if (tid < NQP) {
+    float Ls = 0.f;
+    for (int j2 = 0; j2 < SP; ++j2) Ls += s_part[j2 * NQP + tid];
+    sL[tid] = Ls;
+  }
+  __syncthreads();
+  // the weighted sums
+  const int ol = tid % kFmOut, s0 = tid / kFmOut;
+  const int o = o0 + ol;
+  float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (o < n_out) {
+    const int qr = o / (D / 4), dd = (o % (D / 4)) * 4;
+    const float* col = racc + (int64_t)qr * D + dd;
+    for (int sb = s0; sb < nsplit; sb += kFmGroups * 16) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int s2 = sb + u * kFmGroups;
+        v[u] = s2 < nsplit ? __ldcg(reinterpret_cast<const float4*>(col + (int64_t)s2 * NQP * D))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int s2 = sb + u * kFmGroups;
+        const float w = s2 < nsplit ? sml[(s2 * NQP + qr) * 2] : 0.f;
+        A.x += w * v[u].x;
+        A.y += w * v[u].y;
+        A.z += w * v[u].z;
+        A.w += w * v[u].w;
+      }
+    }
+  }
+  sred[s0][ol] = A;
+  __syncthreads();
+  if (s0 == 0 && o < n_out) {
+    float4 T = sred[0][ol];
+#pragma unroll
+    for (int j = 1; j < kFmGroups; ++j) {
+      T.x += sred[j][ol].x;
+      T.y += sred[j][ol].y;
+      T.z += sred[j][ol].z;
+      T.w += sred[j][ol].w;
+    }
+    const int qr = o / (D / 4), dd = (o % (D / 4)) * 4;
+    const float inv = 1.f / sL[qr];
+    const int l = qr / p.G, h = g * p.G + qr % p.G;
+    float* out = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
+    out[0] = T.x * inv;
+    out[1] = T.y * inv;
+    out[2] = T.z * inv;
+    out[3] = T.w * inv;
+  }
 }
 
 }  // namespace aoh
