@@ -250,15 +250,19 @@ aoh_status aoh_tip_score(const void* q, int32_t n_q_heads, const aoh_kv_cache* k
  *                   bytes, zero-filled once before its first use (every call
  *                   leaves its counters at zero again)
  * Rows up to 4 M positions (AOH_ERR_UNSUPPORTED beyond).  Deterministic: the
- * same input gives the same bits.  Mechanism, on order-preserving uint32 keys:
- * rows of at most 128 K positions take one launch, one thread-block cluster
- * per row with the row's keys on chip (MSB radix select with 11-, 11- and
- * 10-bit digits, histograms summed across the cluster through distributed
- * shared memory, picks written in order); longer rows take three launches (a
- * histogram of the top 11 bits, then chunks of 4096 keys in parallel: keys
- * above the threshold bin counted, keys in it collected; one CTA per row
- * resolves the exact threshold and every chunk's offset; every chunk's picks
- * written in order).
+ * same input gives the same bits.  Mechanism, on order-preserving uint32 keys,
+ * in one of three forms:
+ *  - rows of at most 128 K positions whose clusters fit one wave: one launch,
+ *    one thread-block cluster per row with the row's keys in registers (MSB
+ *    radix select with 11-, 11- and 10-bit digits, histograms summed across
+ *    the cluster through distributed shared memory, picks written in order);
+ *  - else, fewer rows than SMs of at most 256 K positions that fit one wave of
+ *    the fused row kernel's clusters: that kernel in its select-only mode (keys
+ *    in shared memory, 8-bit digits), one launch;
+ *  - else four launches: a histogram of the top 11 bits; chunks of 4096 keys
+ *    in parallel (keys above the threshold bin counted, keys in it collected);
+ *    one CTA per row resolving the exact threshold and every chunk's offset;
+ *    every chunk's picks written in order.
  */
 aoh_status aoh_topk_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac,
                            const int32_t* n_fac_per_seq, int32_t n_fac_cap,

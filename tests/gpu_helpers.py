@@ -185,11 +185,15 @@ def launches_of(fn) -> dict:
 
 def three_kernel_form(launches: dict) -> bool:
     """scan + select + gather: the select is one cluster launch when every row's cluster fits
-    one wave, else the chunked select's four launches"""
+    one wave, else the row kernel's select-only launch for fewer rows than SMs, else the
+    chunked select's four launches"""
     per_phase = ("select_hist_kernel", "select_chunk_kernel", "select_resolve_kernel", "select_write_kernel")
-    on_chip = launches.get("select_cluster_kernel") == 1 and not any(k in launches for k in per_phase)
-    chunked = all(launches.get(k) == 1 for k in per_phase) and "select_cluster_kernel" not in launches
-    return (launches.get("tip_score_kernel") == 1 and (on_chip or chunked)
+    others = lambda *ks: not any(k in launches for k in per_phase + ("select_cluster_kernel", "sparse_row_kernel")
+                                 if k not in ks)
+    on_chip = launches.get("select_cluster_kernel") == 1 and others("select_cluster_kernel")
+    rows = launches.get("sparse_row_kernel") == 1 and others("sparse_row_kernel")
+    chunked = all(launches.get(k) == 1 for k in per_phase) and others(*per_phase)
+    return (launches.get("tip_score_kernel") == 1 and (on_chip or rows or chunked)
             and launches.get("flash_gather_kernel", 0) >= 1)
 
 

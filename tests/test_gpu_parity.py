@@ -179,17 +179,31 @@ def test_topk_rows_in_clusters(kind):
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
 def test_topk_long_rows_chunked(kind):
-    # rows beyond one cluster's 128 K positions take the chunked select (histogram, chunk pass,
-    # ordered write); the ties / zeros kinds put more candidates in the threshold bin than
-    # the resolving CTA keeps in shared memory (it then reads them from the list)
+    # a row beyond the row kernel's 256 K positions sends the call to the chunked select
+    # (histogram, chunk pass, resolve, ordered write); the ties / zeros kinds put more
+    # candidates in the threshold bin than the resolving CTA keeps in shared memory (it then
+    # reads them from the list)
     rng = np.random.default_rng(16)
-    lengths = [131073, 0, 5, 200000, 2000, 140000]
+    lengths = [131073, 0, 5, 300000, 2000, 140000]
     Hkv = 2
     offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
     s = given_scores(rng, lengths, Hkv, kind)
     nfps = np.array([3000, 4, 9, 2048, 2500, 1], dtype=np.int32)
     check_topk(s, offs, lengths, nfps, 3000,
                {"select_hist_kernel": 1, "select_chunk_kernel": 1, "select_resolve_kernel": 1, "select_write_kernel": 1}, kind)
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "zeros", "wide"])
+def test_topk_rows_select_only(kind):
+    # rows past the cluster select's 128 K positions, fewer than the SMs: the fused row
+    # kernel's select-only mode (keys from the given scores, 16-CTA clusters, 8-bit digits)
+    rng = np.random.default_rng(18)
+    lengths = [140000, 0, 5, 131073, 131073]
+    Hkv = 2
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    s = given_scores(rng, lengths, Hkv, kind)
+    nfps = np.array([2048, 4, 9, 139999, 131072], dtype=np.int32)
+    check_topk(s, offs, lengths, nfps, 139999, {"sparse_row_kernel": 1}, kind)
 
 
 @pytest.mark.parametrize("L", [1, 8191, 8192, 8193, 65536, 131072])

@@ -474,10 +474,16 @@ int select_cluster_size(const aoh_kv_cache* kv) {
 // 128K shared-index rows, whose 16 clusters of 16 CTAs need two waves, and the 256 serving
 // rows select faster chunked; 32 rows of 32K faster in clusters).  Both take the same
 // workspace region.
+aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
+                              int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
+                              cudaStream_t st, bool* launched);
+
 aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps, int32_t cap,
                          int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed, uint8_t* ws,
                          cudaStream_t st) {
   const int CL = select_cluster_size(kv);
+  const int64_t n_rows = int64_t(n_listed) * kv->batch;
+  bool one_wave = false;
   if (CL > 0) {
     auto kern = select_cluster_kernel;
     static std::atomic<uint64_t> configured{0};
@@ -487,7 +493,8 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
       mark_set_up(configured);
     }
     const int maxc = max_active_clusters(kern, CL, 0, kScThreads);
-    if (maxc > 0 && int64_t(n_listed) * kv->batch <= maxc) {
+    one_wave = maxc > 0 && n_rows <= maxc;
+    if (one_wave) {
       ClusterSelectParams cp{};
       cp.scores = scores;
       cp.offsets = kv->offsets;
@@ -504,6 +511,13 @@ aoh_status launch_select(const float* scores, const aoh_kv_cache* kv, int32_t n_
       if (s != AOH_OK) return s;
       return count_launch(AOH_KERNEL_SELECT_CLUSTER, st);
     }
+  }
+  // Fewer rows than SMs that the cluster select cannot take in one wave: the row kernel's
+  // select over a cluster's shared memory (one launch, 8-bit digits), when its clusters fit.
+  if (n_rows < sm_count()) {
+    bool launched = false;
+    const aoh_status s = launch_select_rows(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, st, &launched);
+    if (s != AOH_OK || launched) return s;
   }
   return launch_chunk_select(scores, kv, n_fac, nfps, cap, idx, count, heads, n_listed, ws, st);
 }
@@ -527,7 +541,7 @@ struct FusedPlan {
   size_t keys_bytes, ring_bytes, smem;
 };
 
-FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
+FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL, bool select_only = false) {
   FusedPlan f{};
   const int64_t L = std::max(kv->max_len, 1);
   const int64_t slice = (ceil_div(L, CL) + 3) & ~int64_t(3);
@@ -535,6 +549,14 @@ FusedPlan fused_candidate(const aoh_kv_cache* kv, int CL) {
   f.CL = CL;
   f.slice = (int)slice;
   f.keys_bytes = (size_t)ceil_div(slice * 4, 1024) * 1024;
+  if (select_only) {
+    // no scan ring and no attention stages: the ring region only holds the candidates of the
+    // first digit (more than fit are re-read from the keys), so CTAs stay small and many fit an SM
+    f.ring_bytes = kRingStep;
+    f.smem = f.keys_bytes + f.ring_bytes + 1024;
+    f.ok = true;
+    return f;
+  }
   // 1 KB of slack: the kernel aligns its dynamic shared memory to 1024 bytes
   size_t budget = kTwoPerSm - 1024;
   const size_t ring_min = kRingMin;
@@ -562,11 +584,11 @@ bool fused_feasible(const aoh_kv_cache* kv, int nq) {
 // Launch the cluster row kernel with the cluster size that needs the fewest waves x slice
 // length (ties to the smaller cluster).  With max_waves > 0 nothing is launched when every
 // choice needs more waves; *launched says which happened.
-template <int D, int NT>
+template <int D, int NT, bool SO = false>
 aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int B, cudaStream_t st, int max_waves,
                          bool* launched) {
   *launched = false;
-  auto kern = sparse_row_kernel<D, NT>;
+  auto kern = sparse_row_kernel<D, NT, SO>;
   static std::atomic<uint64_t> configured{0};
   if (!set_up_on_this_device(configured)) {
     aoh_status s = set_smem(kern, kOnePerSm);
@@ -581,7 +603,7 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   // Short rows (<= kShortRow positions) take one CTA per row when that fits one wave: their
   // time is the fixed cost of the phases, and a one-CTA cluster's barriers are block barriers.
   if (kv->max_len <= kShortRow) {
-    const FusedPlan f = fused_candidate(kv, 1);
+    const FusedPlan f = fused_candidate(kv, 1, SO);
     if (f.ok) {
       const int maxc = max_active_clusters(kern, 1, f.smem);
       if (maxc > 0 && n_rows <= maxc) {
@@ -593,7 +615,7 @@ aoh_status launch_rows_t(RowParams rp, const aoh_kv_cache* kv, int n_listed, int
   }
   const int cls[3] = {4, 8, 16};
   for (int i = 0; i < 3 && best_cost > 0; ++i) {
-    const FusedPlan f = fused_candidate(kv, cls[i]);
+    const FusedPlan f = fused_candidate(kv, cls[i], SO);
     if (!f.ok) continue;
     const int maxc = max_active_clusters(kern, f.CL, f.smem);
     if (maxc <= 0) continue;
@@ -639,6 +661,31 @@ aoh_status launch_rows(const RowParams& rp, const aoh_kv_cache* kv, int nq, int 
   if (nqp == 8) return launch_rows_t<64, 1>(rp, kv, n_listed, B, st, max_waves, launched);
   if (nqp == 16) return launch_rows_t<64, 2>(rp, kv, n_listed, B, st, max_waves, launched);
   return launch_rows_t<64, 4>(rp, kv, n_listed, B, st, max_waves, launched);
+}
+
+// Select-only launch of the row kernel on the stand-alone scan's scores: writes idx / count.
+// Nothing is launched (*launched false) when no cluster size takes the rows in one wave.
+aoh_status launch_select_rows(const float* scores, const aoh_kv_cache* kv, int32_t n_fac, const int32_t* nfps,
+                              int32_t cap, int32_t* idx, int32_t* count, const uint8_t* heads, int n_listed,
+                              cudaStream_t st, bool* launched) {
+  *launched = false;
+  if (!fused_candidate(kv, kSrMaxCluster, true).ok) return AOH_OK;
+  RowParams rp{};
+  rp.offsets = kv->offsets;
+  rp.lengths = kv->lengths;
+  rp.scores_in = scores;
+  rp.n_fac_per_seq = nfps;
+  rp.n_fac = n_fac;
+  rp.cap = cap;
+  rp.idx_out = idx;
+  rp.count_out = count;
+  rp.T = (int32_t)kv->total_tokens;
+  rp.B = kv->batch;
+  rp.Hkv = kv->n_kv_heads;
+  rp.G = 1;
+  rp.NQ = 1;
+  memcpy(rp.heads, heads, n_listed);
+  return launch_rows_t<128, 1, true>(rp, kv, n_listed, kv->batch, st, 1, launched);
 }
 
 // Score source of the fused kernel: packed dominant columns, K in place masked to I_dom,

@@ -27,7 +27,9 @@
 //  4. combine: the CL partial (m, l, acc) states are merged through distributed
 //              shared memory, each CTA writing 1/CL of the outputs.
 // Nothing but the index and the outputs goes to global memory; no global
-// scratch, no second launch.  DENSE / STREAM heads may ride in the same launch: their
+// scratch, no second launch.  Select-only mode takes the keys from scores that the
+// stand-alone scan wrote and stops after 2 (fewer rows than SMs, each spread over a
+// cluster's shared memory).  DENSE / STREAM heads may ride in the same launch: their
 // clusters skip 1-2 and attend over their range (the whole AoH step in one launch).
 #pragma once
 
@@ -75,6 +77,7 @@ struct RowParams {
   uint8_t slot[kMaxHeads];   // head slot of every KV head in K / V and in the score rows
   uint8_t roles[kMaxHeads];  // 0 SPARSE (scan, select, attend); 1 DENSE / 2 STREAM: attend over the range
   int32_t sink, window;      // the STREAM range: [0, min(sink, L)) U [max(sink, L - window), L)
+  const float* scores_in;    // select-only form: the keys come from these fp32 scores [Hkv][T]
 };
 
 // Attention tiles: gathered K / V rows are copied as 16-byte cp.async segments into rows
@@ -87,7 +90,9 @@ struct AttTile {
   static constexpr int kStage = 2 * kTile;
 };
 
-template <int D, int NT>
+// SO: the select-only form (keys loaded from p.scores_in, no scan, stops once the index is
+// written: no attention, no outputs).
+template <int D, int NT, bool SO>
 __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_constant__ RowParams p) {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(NT == 1 || NT == 2 || NT == 4, "n-tiles");
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     if (rk == 0 && tid == 0) p.count_out[(int64_t)b * p.Hkv + g] = n;
   }
   if ((role == 0 ? n : nwin) == 0) {  // uniform over the cluster: zero rows, no barrier taken
-    if (rk == 0) {
+    if (rk == 0 && !SO) {
       for (int e = tid; e < p.NQ * D; e += kSrThreads) {
         const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
         p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + e % D] = 0.f;
@@ -173,7 +178,25 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
   }
   if (role == 0 && n < L) {
     // =============================================================== 1. scan
-    {
+    if constexpr (SO) {
+      // the scores were computed by the stand-alone scan: load them as keys, eight loads
+      // in flight per thread
+      const float* srow = p.scores_in + (int64_t)g * p.T + off + lo;
+      for (int i0 = 0; i0 < m; i0 += 8 * kSrThreads) {
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kSrThreads + tid;
+          f[u] = i < m ? __ldcg(srow + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kSrThreads + tid;
+          if (i < m) keys[i] = score_key(f[u]);
+        }
+      }
+      __syncthreads();
+    } else {
       // Each warp streams a contiguous run of the slice's rows through its own cp.async
       // ring: S lanes share a row (16 bytes each), kScanU rows per lane per group,
       // kScanDepth groups in flight; the first groups are issued before the group-summed
@@ -500,6 +523,10 @@ __global__ void __launch_bounds__(kSrThreads) sparse_row_kernel(const __grid_con
     nloc = j1 - j0;
   }
   __syncthreads();
+  if constexpr (SO) {  // the index is written; peers may still read this CTA's counts
+    cluster.sync();
+    return;
+  }
 
   // =============================================================== 3. attend
   // warp = (token group, n-tile, part of the head dimension)
