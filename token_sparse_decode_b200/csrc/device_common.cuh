@@ -120,6 +120,15 @@ __device__ __forceinline__ void cp_async_wait_n(int n) {
   }
 }
 
+// 16 bytes of read-only data that is used once: not kept in L1
+__device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
 // ------------------------------------------------------------------ tensor-core fragments
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"

@@ -110,6 +110,227 @@ __device__ __forceinline__ int fd_row_count(const FdecParams& p, int b, int g, i
   return *ra + (L - *rb);
 }
 
+// The end of a gather CTA, shared by both gather kernels: red_ml [NT * WT][8][2] and red_acc
+// [NT * WT][8][D] (floats at the start of the dynamic shared memory) hold the partial (m, l, acc)
+// of each (n-tile nt, token group t) at index nt + NT * t; the groups are merged, then the
+// row's splits (cluster merge, the row's last CTA through the workspace, or partials left for
+// flash_merge_kernel).  MERGE_OFF: where the cluster merge buffers start.
+template <int D, int NT, int WT, int THREADS, int MERGE_OFF>
+__device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, int* s_last_p, int tid, int b, int g,
+                                          int row_id, int split, int nsplit, bool clus) {
+  constexpr int kFdThreads = THREADS;
+  constexpr int kFdMergeOff = MERGE_OFF;
+  constexpr int NQP = NT * 8;
+  constexpr int NW = NT * WT;
+  int& s_last = *s_last_p;
+  const float* red_ml = reinterpret_cast<const float*>(smem);  // [NW][8][2]
+  const float* red_acc = red_ml + NW * 8 * 2;                  // [NW][8][D]
+  if (clus) {
+    // ---- cluster merge: every CTA leaves (M, L, A) of its split in shared memory (past the
+    // warp partials), then CTA r combines outputs r, r + CL, ... over the CL splits
+    namespace cgs = cooperative_groups;
+    cgs::cluster_group cluster = cgs::this_cluster();
+    const int CLn = (int)cluster.num_blocks(), rk = (int)cluster.block_rank();
+    float* cm = reinterpret_cast<float*>(smem + kFdMergeOff);  // [NQP]
+    float* cls = cm + NQP;                                      // [NQP]
+    float* ca = cls + NQP;                                      // [NQP][D]
+    for (int e = tid; e < NQP * D; e += kFdThreads) {
+      const int qr = e / D, dd = e % D;
+      const int ntq = qr >> 3, cq = qr & 7;
+      float M = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t) * 8 + cq) * 2]);
+      float Ls = 0.f, A = 0.f;
+#pragma unroll
+      for (int t = 0; t < WT; ++t) {
+        const int w = ntq + NT * t;
+        const float mw = red_ml[(w * 8 + cq) * 2];
+        const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
+        A += f * red_acc[(w * 8 + cq) * D + dd];
+      }
+      ca[e] = A;
+      if (dd == 0) {
+        cm[qr] = M;
+        cls[qr] = Ls;
+      }
+    }
+    cluster.sync();
+    // outputs 4 consecutive dims at a time: each thread fetches its row's (M, L) from every
+    // peer together with the peers' 16-byte partials (batches of 8 peers, all of a batch's
+    // remote loads in flight together; a running rescale joins the batches)
+    for (int e4 = rk * kFdThreads + tid; e4 < p.NQ * D / 4; e4 += CLn * kFdThreads) {
+      const int e = 4 * e4, qr = e / D, dd = e % D;
+      float Mx = -INFINITY, Ls = 0.f;
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q0 = 0; q0 < CLn; q0 += 8) {
+        float mv[8], lv[8];
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (q0 + u < CLn) {
+            mv[u] = cluster.map_shared_rank(cm, q0 + u)[qr];
+            lv[u] = cluster.map_shared_rank(cls, q0 + u)[qr];
+            v[u] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, q0 + u) + e);
+          } else {
+            mv[u] = -INFINITY;
+            lv[u] = 0.f;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float Mb = Mx;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) Mb = fmaxf(Mb, mv[u]);
+        const float sc = (Mx == -INFINITY) ? 0.f : exp2f(Mx - Mb);
+        Ls *= sc;
+        A.x *= sc;
+        A.y *= sc;
+        A.z *= sc;
+        A.w *= sc;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float w = (mv[u] == -INFINITY) ? 0.f : exp2f(mv[u] - Mb);
+          Ls += w * lv[u];
+          A.x += w * v[u].x;
+          A.y += w * v[u].y;
+          A.z += w * v[u].z;
+          A.w += w * v[u].w;
+        }
+        Mx = Mb;
+      }
+      const float inv = 1.f / Ls;
+      const int l = qr / p.G, h = g * p.G + qr % p.G;
+      float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
+      o[0] = A.x * inv;
+      o[1] = A.y * inv;
+      o[2] = A.z * inv;
+      o[3] = A.w * inv;
+    }
+    cluster.sync();  // peers read this CTA's shared memory until here
+    return;
+  }
+  const bool single = (nsplit == 1);
+  float* pml = p.part_ml + ((int64_t)row_id * p.max_splits + split) * NQP * 2;
+  float* pacc = p.part_acc + ((int64_t)row_id * p.max_splits + split) * NQP * D;
+  for (int e = tid; e < NQP * D; e += kFdThreads) {
+    const int qr = e / D, dd = e % D;
+    const int ntq = qr >> 3, cq = qr & 7;
+    float M = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t) * 8 + cq) * 2]);
+    float Ls = 0.f, A = 0.f;
+#pragma unroll
+    for (int t = 0; t < WT; ++t) {
+      const int w = ntq + NT * t;
+      const float mw = red_ml[(w * 8 + cq) * 2];
+      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
+      A += f * red_acc[(w * 8 + cq) * D + dd];
+    }
+    if (single) {
+      if (qr < p.NQ) {
+        const int l = qr / p.G, h = g * p.G + qr % p.G;
+        p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Ls;
+      }
+    } else {
+      pacc[qr * D + dd] = A;
+      if (dd == 0) {
+        pml[qr * 2] = M;
+        pml[qr * 2 + 1] = Ls;
+      }
+    }
+  }
+  if (single || p.defer_merge) return;
+
+  // ---- split-K combine by the last CTA of the row
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int ticket = atomicAdd(p.tickets + row_id, 1);
+    s_last = (ticket == nsplit - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
+  const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
+  // weights w[s][q] = 2^(m_sq - M_q) staged in shared memory (nsplit * NQP <= kFdMaxSplits * NQP fits).
+  // The partials sit in L2: the max and sum run over all threads, the weighted sum keeps 16
+  // independent loads in flight per thread.
+  float* sw = reinterpret_cast<float*>(smem);        // [nsplit][NQP]
+  float* sM = sw + nsplit * NQP;                     // [NQP]
+  float* sL = sM + NQP;                              // [NQP]
+  float* sred = sL + NQP;                            // [kFdThreads]: per-thread partial max / sum
+  // every thread takes query row tid % NQP over the splits j, j + SP, ... (SP = threads / NQP)
+  constexpr int SP = kFdThreads / NQP;
+  const int rq = tid % NQP, sj = tid / NQP;
+  {
+    float M = -INFINITY;
+    for (int s2 = sj; s2 < nsplit; s2 += SP) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + rq) * 2));
+    sred[tid] = M;
+  }
+  __syncthreads();
+  if (tid < NQP) {
+    float M = -INFINITY;
+    for (int j = 0; j < SP; ++j) M = fmaxf(M, sred[j * NQP + tid]);
+    sM[tid] = M;
+  }
+  __syncthreads();
+  for (int e = tid; e < nsplit * NQP; e += kFdThreads) {
+    const int qr = e % NQP;
+    sw[e] = exp2f(__ldcg(rml + (int64_t)e * 2) - sM[qr]);
+  }
+  __syncthreads();
+  {
+    float Ls = 0.f;
+    for (int s2 = sj; s2 < nsplit; s2 += SP) Ls += sw[s2 * NQP + rq] * __ldcg(rml + ((int64_t)s2 * NQP + rq) * 2 + 1);
+    sred[tid] = Ls;
+  }
+  __syncthreads();
+  if (tid < NQP) {
+    float Ls = 0.f;
+    for (int j = 0; j < SP; ++j) Ls += sred[j * NQP + tid];
+    sL[tid] = Ls;
+  }
+  __syncthreads();
+  // four consecutive dimensions of one query row per thread
+  for (int e4 = tid; e4 < p.NQ * (D / 4); e4 += kFdThreads) {
+    const int qr = e4 / (D / 4), dd = (e4 % (D / 4)) * 4;
+    const float* col = racc + (int64_t)qr * D + dd;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s2 = 0;
+    for (; s2 + 16 <= nsplit; s2 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)(s2 + u) * NQP * D));
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float w = sw[(s2 + u) * NQP + qr];
+        A.x += w * v[u].x;
+        A.y += w * v[u].y;
+        A.z += w * v[u].z;
+        A.w += w * v[u].w;
+      }
+    }
+    for (; s2 < nsplit; ++s2) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)s2 * NQP * D));
+      const float w = sw[s2 * NQP + qr];
+      A.x += w * v.x;
+      A.y += w * v.y;
+      A.z += w * v.z;
+      A.w += w * v.w;
+    }
+    const float inv = 1.f / sL[qr];
+    const int l = qr / p.G, h = g * p.G + qr % p.G;
+    float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
+    o[0] = A.x * inv;
+    o[1] = A.y * inv;
+    o[2] = A.z * inv;
+    o[3] = A.w * inv;
+  }
+  if (tid == 0) p.tickets[row_id] = 0;
+}
+
 template <int D, int NT>
 __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const FdecParams p) {
   constexpr int ST = kFdStages;
@@ -123,7 +344,6 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   constexpr int NW = kFdThreads / 32;
   constexpr int kFdMergeOff = fd_merge_off(NT, D);
   constexpr int SUB = kFdTS / 16;    // 16-token sub-tiles per stage
-  constexpr int NQP = NT * 8;        // padded query rows
   constexpr int CPR = D / 8;         // 16-byte chunks per row
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ int s_last;
@@ -346,211 +566,7 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   }
   __syncthreads();
 
-  // CTA result for padded query row qr: warps {nt + NT * t : t < WT} hold it.
-  if (clus) {
-    // ---- cluster merge: every CTA leaves (M, L, A) of its split in shared memory (past the
-    // warp partials), then CTA r combines outputs r, r + CL, ... over the CL splits
-    namespace cgs = cooperative_groups;
-    cgs::cluster_group cluster = cgs::this_cluster();
-    const int CLn = (int)cluster.num_blocks(), rk = (int)cluster.block_rank();
-    float* cm = reinterpret_cast<float*>(smem + kFdMergeOff);  // [NQP]
-    float* cls = cm + NQP;                                      // [NQP]
-    float* ca = cls + NQP;                                      // [NQP][D]
-    for (int e = tid; e < NQP * D; e += kFdThreads) {
-      const int qr = e / D, dd = e % D;
-      const int ntq = qr >> 3, cq = qr & 7;
-      float M = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t) * 8 + cq) * 2]);
-      float Ls = 0.f, A = 0.f;
-#pragma unroll
-      for (int t = 0; t < WT; ++t) {
-        const int w = ntq + NT * t;
-        const float mw = red_ml[(w * 8 + cq) * 2];
-        const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-        Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
-        A += f * red_acc[(w * 8 + cq) * D + dd];
-      }
-      ca[e] = A;
-      if (dd == 0) {
-        cm[qr] = M;
-        cls[qr] = Ls;
-      }
-    }
-    cluster.sync();
-    // outputs 4 consecutive dims at a time: each thread fetches its row's (M, L) from every
-    // peer together with the peers' 16-byte partials (batches of 8 peers, all of a batch's
-    // remote loads in flight together; a running rescale joins the batches)
-    for (int e4 = rk * kFdThreads + tid; e4 < p.NQ * D / 4; e4 += CLn * kFdThreads) {
-      const int e = 4 * e4, qr = e / D, dd = e % D;
-      float Mx = -INFINITY, Ls = 0.f;
-      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q0 = 0; q0 < CLn; q0 += 8) {
-        float mv[8], lv[8];
-        float4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (q0 + u < CLn) {
-            mv[u] = cluster.map_shared_rank(cm, q0 + u)[qr];
-            lv[u] = cluster.map_shared_rank(cls, q0 + u)[qr];
-            v[u] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, q0 + u) + e);
-          } else {
-            mv[u] = -INFINITY;
-            lv[u] = 0.f;
-            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-        float Mb = Mx;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) Mb = fmaxf(Mb, mv[u]);
-        const float sc = (Mx == -INFINITY) ? 0.f : exp2f(Mx - Mb);
-        Ls *= sc;
-        A.x *= sc;
-        A.y *= sc;
-        A.z *= sc;
-        A.w *= sc;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float w = (mv[u] == -INFINITY) ? 0.f : exp2f(mv[u] - Mb);
-          Ls += w * lv[u];
-          A.x += w * v[u].x;
-          A.y += w * v[u].y;
-          A.z += w * v[u].z;
-          A.w += w * v[u].w;
-        }
-        Mx = Mb;
-      }
-      const float inv = 1.f / Ls;
-      const int l = qr / p.G, h = g * p.G + qr % p.G;
-      float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
-      o[0] = A.x * inv;
-      o[1] = A.y * inv;
-      o[2] = A.z * inv;
-      o[3] = A.w * inv;
-    }
-    cluster.sync();  // peers read this CTA's shared memory until here
-    return;
-  }
-  const bool single = (nsplit == 1);
-  float* pml = p.part_ml + ((int64_t)row_id * p.max_splits + split) * NQP * 2;
-  float* pacc = p.part_acc + ((int64_t)row_id * p.max_splits + split) * NQP * D;
-  for (int e = tid; e < NQP * D; e += kFdThreads) {
-    const int qr = e / D, dd = e % D;
-    const int ntq = qr >> 3, cq = qr & 7;
-    float M = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < WT; ++t) M = fmaxf(M, red_ml[((ntq + NT * t) * 8 + cq) * 2]);
-    float Ls = 0.f, A = 0.f;
-#pragma unroll
-    for (int t = 0; t < WT; ++t) {
-      const int w = ntq + NT * t;
-      const float mw = red_ml[(w * 8 + cq) * 2];
-      const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-      Ls += f * red_ml[(w * 8 + cq) * 2 + 1];
-      A += f * red_acc[(w * 8 + cq) * D + dd];
-    }
-    if (single) {
-      if (qr < p.NQ) {
-        const int l = qr / p.G, h = g * p.G + qr % p.G;
-        p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Ls;
-      }
-    } else {
-      pacc[qr * D + dd] = A;
-      if (dd == 0) {
-        pml[qr * 2] = M;
-        pml[qr * 2 + 1] = Ls;
-      }
-    }
-  }
-  if (single || p.defer_merge) return;
-
-  // ---- split-K combine by the last CTA of the row
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int ticket = atomicAdd(p.tickets + row_id, 1);
-    s_last = (ticket == nsplit - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
-  const float* racc = p.part_acc + (int64_t)row_id * p.max_splits * NQP * D;
-  // weights w[s][q] = 2^(m_sq - M_q) staged in shared memory (nsplit * NQP <= kFdMaxSplits * NQP fits).
-  // The partials sit in L2: the max and sum run over all threads, the weighted sum keeps 16
-  // independent loads in flight per thread.
-  float* sw = reinterpret_cast<float*>(smem);        // [nsplit][NQP]
-  float* sM = sw + nsplit * NQP;                     // [NQP]
-  float* sL = sM + NQP;                              // [NQP]
-  float* sred = sL + NQP;                            // [kFdThreads]: per-thread partial max / sum
-  // every thread takes query row tid % NQP over the splits j, j + SP, ... (SP = threads / NQP)
-  constexpr int SP = kFdThreads / NQP;
-  const int rq = tid % NQP, sj = tid / NQP;
-  {
-    float M = -INFINITY;
-    for (int s2 = sj; s2 < nsplit; s2 += SP) M = fmaxf(M, __ldcg(rml + ((int64_t)s2 * NQP + rq) * 2));
-    sred[tid] = M;
-  }
-  __syncthreads();
-  if (tid < NQP) {
-    float M = -INFINITY;
-    for (int j = 0; j < SP; ++j) M = fmaxf(M, sred[j * NQP + tid]);
-    sM[tid] = M;
-  }
-  __syncthreads();
-  for (int e = tid; e < nsplit * NQP; e += kFdThreads) {
-    const int qr = e % NQP;
-    sw[e] = exp2f(__ldcg(rml + (int64_t)e * 2) - sM[qr]);
-  }
-  __syncthreads();
-  {
-    float Ls = 0.f;
-    for (int s2 = sj; s2 < nsplit; s2 += SP) Ls += sw[s2 * NQP + rq] * __ldcg(rml + ((int64_t)s2 * NQP + rq) * 2 + 1);
-    sred[tid] = Ls;
-  }
-  __syncthreads();
-  if (tid < NQP) {
-    float Ls = 0.f;
-    for (int j = 0; j < SP; ++j) Ls += sred[j * NQP + tid];
-    sL[tid] = Ls;
-  }
-  __syncthreads();
-  // four consecutive dimensions of one query row per thread
-  for (int e4 = tid; e4 < p.NQ * (D / 4); e4 += kFdThreads) {
-    const int qr = e4 / (D / 4), dd = (e4 % (D / 4)) * 4;
-    const float* col = racc + (int64_t)qr * D + dd;
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    int s2 = 0;
-    for (; s2 + 16 <= nsplit; s2 += 16) {
-      float4 v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)(s2 + u) * NQP * D));
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const float w = sw[(s2 + u) * NQP + qr];
-        A.x += w * v[u].x;
-        A.y += w * v[u].y;
-        A.z += w * v[u].z;
-        A.w += w * v[u].w;
-      }
-    }
-    for (; s2 < nsplit; ++s2) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (int64_t)s2 * NQP * D));
-      const float w = sw[s2 * NQP + qr];
-      A.x += w * v.x;
-      A.y += w * v.y;
-      A.z += w * v.z;
-      A.w += w * v.w;
-    }
-    const float inv = 1.f / sL[qr];
-    const int l = qr / p.G, h = g * p.G + qr % p.G;
-    float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
-    o[0] = A.x * inv;
-    o[1] = A.y * inv;
-    o[2] = A.z * inv;
-    o[3] = A.w * inv;
-  }
-  if (tid == 0) p.tickets[row_id] = 0;
+  fd_finish<D, NT, WT, kFdThreads, kFdMergeOff>(p, smem, &s_last, tid, b, g, row_id, split, nsplit, clus);
 }
 
 // Split-K combine of rows with many splits, spread over CTAs: grid (slices of 16 float4

@@ -40,15 +40,6 @@ struct TipParams {
   uint8_t slot[kMaxHeads];  // head slot of every KV head in the row source
 };
 
-__device__ __forceinline__ uint4 ld_stream_v4(const uint16_t* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-
 // S = lanes per row: row_len / 8 rounded up to a power of two (1 .. 16); lanes whose
 // 16-byte segment lies past the row end carry zero weights and load nothing.
 //
