@@ -343,7 +343,9 @@ def test_full_role_split_step_mixed_heads():
 
 
 @pytest.mark.parametrize("fused", [True, False])
-@pytest.mark.parametrize("n_layers,hq,hkv", [(8, 32, 8), (2, 16, 4), (3, 16, 4), (1, 8, 8)])
+# query rows n_layers * G: 32 and 20 and 18 take two CTAs per row in the three-kernel form (16 rows
+# each; the second holds 16, 4 and 2, with a group split across the two for 18), 12 / 8 / 1 one
+@pytest.mark.parametrize("n_layers,hq,hkv", [(8, 32, 8), (2, 16, 4), (3, 16, 4), (1, 8, 8), (5, 16, 4), (3, 24, 4)])
 def test_shared_index_decode_matches_oracle(n_layers, hq, hkv, fused):
     sp = WorkloadSpec(name="shared", batch=2, n_q_heads=hq, n_kv_heads=hkv, head_dim=128, theta=5e5,
                       len_range=(500, 9000), n_layers=n_layers, topk_shared=700, seed=90 + n_layers)

@@ -159,7 +159,8 @@ struct FdGeom {
   int chunk;
   int max_splits;
   int nqp;
-  int rows;
+  int rows;     // partial-state rows: sequences x KV heads x q_split
+  int q_split;  // CTAs sharing a row's positions, each with nqp of its query rows
   size_t ticket_bytes, ml_bytes, acc_bytes;
 };
 
@@ -182,6 +183,7 @@ FdGeom fd_geom(int64_t work_tokens, int64_t n_max, int rows, int nq, int d) {
   g.chunk = (int)chunk;
   g.max_splits = (int)std::max<int64_t>(1, ceil_div(std::max<int64_t>(n_max, 1), chunk));
   g.rows = rows;
+  g.q_split = 1;
   g.ticket_bytes = align256(sizeof(int32_t) * (size_t)std::max(rows, 1));
   g.ml_bytes = align256(sizeof(float) * (size_t)rows * g.max_splits * g.nqp * 2);
   g.acc_bytes = align256(sizeof(float) * (size_t)rows * g.max_splits * g.nqp * d);
@@ -198,6 +200,7 @@ void fd_bind(FdecParams& fp, const FdGeom& g, uint8_t* ws) {
   fp.part_acc = reinterpret_cast<float*>(ws + g.ticket_bytes + g.ml_bytes);
   fp.chunk = g.chunk;
   fp.max_splits = g.max_splits;
+  fp.q_split = g.q_split;
 }
 
 // Launch of a kernel that follows another one of the same call on the stream: programmatic
@@ -278,7 +281,8 @@ aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStr
     if (s != AOH_OK) return s;
     mark_set_up(configured);
   }
-  dim3 grid(fp.max_splits, n_listed, B);
+  const int QS = std::max(1, fp.q_split);
+  dim3 grid(fp.max_splits, n_listed * QS, B);
   // rows of about equal length with 2..16 splits: one cluster per row, merged on chip
   const int CL = fp.max_splits;
   constexpr int threads = fd_threads(NT);
@@ -292,7 +296,7 @@ aoh_status launch_fd_t(FdecParams fp, int n_listed, int B, bool uniform, cudaStr
   if (s != AOH_OK) return s;
   if ((s = count_launch(AOH_KERNEL_FLASH_GATHER, st)) != AOH_OK || !fp.defer_merge) return s;
   constexpr int NQP = NT * 8;
-  const dim3 mgrid((unsigned)ceil_div(int64_t(fp.NQ) * (D / 4), kFmOut), n_listed, B);
+  const dim3 mgrid((unsigned)ceil_div(int64_t(std::min(fp.NQ, NQP)) * (D / 4), kFmOut), n_listed * QS, B);
   const size_t msmem = sizeof(float) * 2 * (size_t)fp.max_splits * NQP;  // <= 2 x 256 x 32 floats
   static std::atomic<uint64_t> merge_configured{0};
   if (!set_up_on_this_device(merge_configured)) {
@@ -760,10 +764,17 @@ FdGeom stream_geom(const aoh_kv_cache* kv, int32_t Hq, const uint8_t* roles, int
   return fd_geom(work, n_max, kv->batch * kv->n_kv_heads, G, kv->head_dim);
 }
 
+// More than 16 query rows (the layers x group of a shared index) are split over two CTAs that
+// read the same positions: twice the CTAs, each with half the contraction and half the partials
+// (measured on the 128K shared-index step's 32 rows: see the gather's notes).
 FdGeom shared_geom(const aoh_kv_cache* kv, int32_t n_layers, int32_t Hq, int32_t cap) {
   const int G = Hq / kv->n_kv_heads;
-  const int rows = kv->batch * kv->n_kv_heads;
-  return fd_geom(int64_t(rows) * cap, cap, rows, n_layers * G, kv->head_dim);
+  const int nq = n_layers * G;
+  const int qs = nq > 16 ? 2 : 1;
+  const int rows = kv->batch * kv->n_kv_heads * qs;
+  FdGeom g = fd_geom(int64_t(rows) * cap, cap, rows, (nq + qs - 1) / qs, kv->head_dim);
+  g.q_split = qs;
+  return g;
 }
 
 // A ring keeps only streaming heads' sink and window: it serves STREAM heads whose sink and

@@ -67,6 +67,8 @@ struct FdecParams {
   int32_t cluster_combine;   // 1: launched with clusters of max_splits CTAs (one row each)
   int32_t defer_merge;       // 1: the CTAs of a row with several splits only leave their partials
                              //    (flash_merge_kernel combines them)
+  int32_t q_split;           // CTAs sharing a row's positions, each with NQP of its query rows (0 or 1:
+                             //    one); blockIdx.y = listed head * q_split + part
   int32_t sink, window;
   int32_t ring_sink, ring_window;  // range mode on a ring cache (> 0 sum): position p is kept in
                                    // slot ring_slot(p); 0, 0: position p is token p of the region
@@ -117,7 +119,7 @@ __device__ __forceinline__ int fd_row_count(const FdecParams& p, int b, int g, i
 // flash_merge_kernel).  MERGE_OFF: where the cluster merge buffers start.
 template <int D, int NT, int WT, int THREADS, int MERGE_OFF>
 __device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, int* s_last_p, int tid, int b, int g,
-                                          int row_id, int split, int nsplit, bool clus) {
+                                          int q0, int nq, int row_id, int split, int nsplit, bool clus) {
   constexpr int kFdThreads = THREADS;
   constexpr int kFdMergeOff = MERGE_OFF;
   constexpr int NQP = NT * 8;
@@ -159,19 +161,19 @@ __device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, in
     // outputs 4 consecutive dims at a time: each thread fetches its row's (M, L) from every
     // peer together with the peers' 16-byte partials (batches of 8 peers, all of a batch's
     // remote loads in flight together; a running rescale joins the batches)
-    for (int e4 = rk * kFdThreads + tid; e4 < p.NQ * D / 4; e4 += CLn * kFdThreads) {
+    for (int e4 = rk * kFdThreads + tid; e4 < nq * D / 4; e4 += CLn * kFdThreads) {
       const int e = 4 * e4, qr = e / D, dd = e % D;
       float Mx = -INFINITY, Ls = 0.f;
       float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q0 = 0; q0 < CLn; q0 += 8) {
+      for (int pq = 0; pq < CLn; pq += 8) {
         float mv[8], lv[8];
         float4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          if (q0 + u < CLn) {
-            mv[u] = cluster.map_shared_rank(cm, q0 + u)[qr];
-            lv[u] = cluster.map_shared_rank(cls, q0 + u)[qr];
-            v[u] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, q0 + u) + e);
+          if (pq + u < CLn) {
+            mv[u] = cluster.map_shared_rank(cm, pq + u)[qr];
+            lv[u] = cluster.map_shared_rank(cls, pq + u)[qr];
+            v[u] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ca, pq + u) + e);
           } else {
             mv[u] = -INFINITY;
             lv[u] = 0.f;
@@ -199,7 +201,7 @@ __device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, in
         Mx = Mb;
       }
       const float inv = 1.f / Ls;
-      const int l = qr / p.G, h = g * p.G + qr % p.G;
+      const int l = (q0 + qr) / p.G, h = g * p.G + (q0 + qr) % p.G;
       float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
       o[0] = A.x * inv;
       o[1] = A.y * inv;
@@ -228,8 +230,8 @@ __device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, in
       A += f * red_acc[(w * 8 + cq) * D + dd];
     }
     if (single) {
-      if (qr < p.NQ) {
-        const int l = qr / p.G, h = g * p.G + qr % p.G;
+      if (qr < nq) {
+        const int l = (q0 + qr) / p.G, h = g * p.G + (q0 + qr) % p.G;
         p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + dd] = A / Ls;
       }
     } else {
@@ -294,7 +296,7 @@ __device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, in
   }
   __syncthreads();
   // four consecutive dimensions of one query row per thread
-  for (int e4 = tid; e4 < p.NQ * (D / 4); e4 += kFdThreads) {
+  for (int e4 = tid; e4 < nq * (D / 4); e4 += kFdThreads) {
     const int qr = e4 / (D / 4), dd = (e4 % (D / 4)) * 4;
     const float* col = racc + (int64_t)qr * D + dd;
     float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -321,7 +323,7 @@ __device__ __forceinline__ void fd_finish(const FdecParams& p, uint8_t* smem, in
       A.w += w * v.w;
     }
     const float inv = 1.f / sL[qr];
-    const int l = qr / p.G, h = g * p.G + qr % p.G;
+    const int l = (q0 + qr) / p.G, h = g * p.G + (q0 + qr) % p.G;
     float* o = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
     o[0] = A.x * inv;
     o[1] = A.y * inv;
@@ -344,6 +346,7 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   constexpr int NW = kFdThreads / 32;
   constexpr int kFdMergeOff = fd_merge_off(NT, D);
   constexpr int SUB = kFdTS / 16;    // 16-token sub-tiles per stage
+  constexpr int NQP = NT * 8;        // padded query rows
   constexpr int CPR = D / 8;         // 16-byte chunks per row
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ int s_last;
@@ -352,7 +355,10 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.z;
   const int y = blockIdx.y;
-  const int g = p.heads[y];
+  const int QS = max(1, p.q_split);
+  const int g = p.heads[y / QS];
+  const int q0 = (y % QS) * NQP;               // this CTA's first query row
+  const int nq = max(0, min(NQP, p.NQ - q0));  // and its number of query rows
   const int split = blockIdx.x;
   const int row_id = b * gridDim.y + y;
   const bool ring = (p.ring_sink + p.ring_window) > 0;
@@ -371,8 +377,8 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
     if (ring && split == 0 && tid == 0 && p.offsets[b + 1] - off < p.ring_sink + p.ring_window)
       record_error(kCheckCapacity, b, p.offsets[b + 1] - off, p.ring_sink + p.ring_window);
     if (split == 0) {
-      for (int e = tid; e < p.NQ * D; e += kFdThreads) {
-        const int qr = e / D, l = qr / p.G, h = g * p.G + qr % p.G;
+      for (int e = tid; e < nq * D; e += kFdThreads) {
+        const int qr = q0 + e / D, l = qr / p.G, h = g * p.G + qr % p.G;
         p.out[(((int64_t)l * p.B + b) * p.Hq + h) * D + e % D] = 0.f;
       }
     }
@@ -446,8 +452,8 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   uint32_t bq[KS][2];
   {
     const int qr = nt * 8 + (lane >> 2);
-    if (qr < p.NQ) {
-      const int l = qr / p.G, h = g * p.G + qr % p.G;
+    if (qr < nq) {
+      const int l = (q0 + qr) / p.G, h = g * p.G + (q0 + qr) % p.G;
       const uint16_t* qp = p.q + (((int64_t)l * p.B + b) * p.Hq + h) * D + 2 * (lane & 3);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
@@ -566,7 +572,7 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   }
   __syncthreads();
 
-  fd_finish<D, NT, WT, kFdThreads, kFdMergeOff>(p, smem, &s_last, tid, b, g, row_id, split, nsplit, clus);
+  fd_finish<D, NT, WT, kFdThreads, kFdMergeOff>(p, smem, &s_last, tid, b, g, q0, nq, row_id, split, nsplit, clus);
 }
 
 // Split-K combine of rows with many splits, spread over CTAs: grid (slices of 16 float4
@@ -588,14 +594,16 @@ __global__ void __launch_bounds__(kFmThreads) flash_merge_kernel(const FdecParam
   __shared__ float sL[NQP];
   __shared__ float4 sred[kFmGroups][kFmOut];
   const int tid = threadIdx.x;
-  const int b = blockIdx.z, y = blockIdx.y, g = p.heads[y];
+  const int QS = max(1, p.q_split);
+  const int b = blockIdx.z, y = blockIdx.y, g = p.heads[y / QS];
+  const int q0 = (y % QS) * NQP, nq = max(0, min(NQP, p.NQ - q0));
   const int row_id = b * gridDim.y + y;
   const bool ring = (p.ring_sink + p.ring_window) > 0;
   int off, ra, rb;
   const int L = seq_length(p.offsets, p.lengths, b, ring, &off);
   const int n = fd_row_count(p, b, g, L, off, ring, &ra, &rb);
   const int nsplit = (n + p.chunk - 1) / p.chunk;
-  const int n_out = p.NQ * (D / 4);
+  const int n_out = nq * (D / 4);
   const int o0 = blockIdx.x * kFmOut;
   if (nsplit <= 1 || o0 >= n_out) return;
   const float* rml = p.part_ml + (int64_t)row_id * p.max_splits * NQP * 2;
@@ -677,7 +685,7 @@ __global__ void __launch_bounds__(kFmThreads) flash_merge_kernel(const FdecParam
     }
     const int qr = o / (D / 4), dd = (o % (D / 4)) * 4;
     const float inv = 1.f / sL[qr];
-    const int l = qr / p.G, h = g * p.G + qr % p.G;
+    const int l = (q0 + qr) / p.G, h = g * p.G + (q0 + qr) % p.G;
     float* out = p.out + (((int64_t)l * p.B + b) * p.Hq + h) * D + dd;
     out[0] = T.x * inv;
     out[1] = T.y * inv;
