@@ -61,10 +61,11 @@ FALLBACK_HBM_GBS = 6650.0
 
 # ------------------------------------------------------------------------------ bookkeeping
 
-def algorithmic_bytes(w) -> dict:
+def algorithmic_bytes(w, in_place: bool = False) -> dict:
     """Bytes the method must move per step (inputs' K / V columns and rows; q and outputs excluded).
 
-    importance scan: 4 * n_dom bytes per (token, SPARSE KV head) with the packed dominant columns;
+    importance scan: 4 * n_dom bytes per (token, SPARSE KV head) with the packed dominant columns,
+    2 * d (the K row) when the scan reads K in place (`in_place`);
     focused attention: 4 * d bytes (a K row and a V row) per selected token and KV head;
     DENSE / STREAM heads: 4 * d bytes per attended token; shared index: the indexer's full K rows
     (2 * d bytes per token and head) plus 4 * d per indexed token and head.
@@ -81,7 +82,7 @@ def algorithmic_bytes(w) -> dict:
     else:
         n_sparse = int((roles == ROLE_SPARSE).sum())
         nfac = w.n_fac_per_seq.numpy().astype(np.int64)
-        out["tip"] = int(L.sum()) * n_sparse * 4 * sp.n_dom
+        out["tip"] = int(L.sum()) * n_sparse * (2 * d if in_place else 4 * sp.n_dom)
         out["fac"] = int(np.minimum(L, nfac).sum()) * n_sparse * 4 * d
         out["select"] = int(L.sum()) * n_sparse * 4
         for g, r in enumerate(roles):
@@ -125,7 +126,8 @@ def kernel_source_hash() -> str:
 
 
 def ncu_traffic(workload: str, kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source
+    (`workload` carries the suffix ":in_place" for the step whose scan reads K in place)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
@@ -345,7 +347,7 @@ def run_ours(args, rank, world, local_rank):
     spec = shard_spec(preset(args.workload), rank, world)
     w = make_workload(spec)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    ab = algorithmic_bytes(w)
+    ab = algorithmic_bytes(w, args.in_place_scan)
     # Cold inputs every step: rotate over R device copies of the inputs (each step's traffic
     # pushes the other copies out of L2), or, for steps too small for that, flush L2 by
     # rewriting a buffer of twice its size between steps (outside the events).
@@ -486,7 +488,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; bf16 N(0,1) post-RoPE q/K, V; planted salient keys where the workload has them)",
-        "config": dict(workload_config(w, world), l2=l2_note, timing=timing_note,
+        "config": dict(workload_config(w, world), l2=l2_note, timing=timing_note, algorithmic_bytes_per_step=ab["total"],
                        launch="CUDA graph replay" if args.graph else "direct launches",
                        **({"scan": "K read in place (no packed dominant columns)"} if args.in_place_scan else {})),
         "step_hbm": {"achieved": step_gbs, "peak": peak, "unit": "GB/s", "frac": step_gbs / peak,
@@ -497,7 +499,8 @@ def run_ours(args, rank, world, local_rank):
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
                      "timing": "graph-replayed step (one-kernel step)" if one_kernel_step
                      else "CUDA events around the kernel inside the call",
-                     "traffic": ncu_traffic(w.spec.name, dom["kernel"]) if dom else None},
+                     "traffic": ncu_traffic(w.spec.name + (":in_place" if args.in_place_scan else ""),
+                                            dom["kernel"]) if dom else None},
         "call_ms": kt["calls"],
         "kernel_ms": [{"call": e["call"], "kernel": e["kernel"], "ms": e["ms"],
                        "bytes": kernel_bytes(w, ab, e["call"], e["kernel"], kt["order"][e["call"]], e["index"])}

@@ -27,6 +27,9 @@ def test_algorithmic_bytes_of_the_fixed_shape_workloads():
     ab = bench.algorithmic_bytes(lite("llama8b_gqa4_L32k"))
     assert ab["tip"] == 32 * 32768 * 64 and ab["fac"] == 32 * 2048 * 512
     assert ab["total"] == 100663296
+    # the same step with the scan reading K in place: the whole 256-byte K row of every token
+    ab = bench.algorithmic_bytes(lite("llama8b_gqa4_L32k"), in_place=True)
+    assert ab["tip"] == 32 * 32768 * 256 and ab["total"] == 32 * 32768 * 256 + 32 * 2048 * 512
     # AoH roles: 2 dense groups x 131072 tokens + 6 streaming groups x (128 + 4096) tokens, K+V rows of 512 B
     ab = bench.algorithmic_bytes(lite("aoh_roles_L128k"))
     assert ab["window"] == (2 * 131072 + 6 * 4224) * 512 == 147193856
