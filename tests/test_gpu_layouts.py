@@ -6,7 +6,9 @@ the float64 oracle:
   * padded rows: each (token, head) row is d + 8 elements long, the last 8 unused
     (stride_head = d + 8, stride_tok = Hkv * (d + 8));
   * head-major: all tokens of head 0, then of head 1, ... (stride_tok = d,
-    stride_head = T * d).
+    stride_head = T * d);
+  * interleaved: the K row and the V row of a (token, head) side by side in one buffer
+    [T, Hkv, 2, d] (v = k + d, stride_head = 2 * d, stride_tok = Hkv * 2 * d).
 Both the fused one-launch form (few rows) and the three-kernel form (more rows
 than one wave of clusters) are run, with the dominant columns packed and read in
 place, at d = 64 and d = 128.
@@ -40,11 +42,24 @@ def strided(t: torch.Tensor, layout: str) -> torch.Tensor:
     return view
 
 
+def interleaved(k: torch.Tensor, v: torch.Tensor):
+    """[T, Hkv, d] views of one [T, Hkv, 2, d] buffer holding copies of k and v."""
+    T, H, d = k.shape
+    buf = torch.stack([k, v], dim=2).contiguous()
+    kv, vv = buf[:, :, 0, :], buf[:, :, 1, :]
+    assert kv.stride() == vv.stride() == (H * 2 * d, 2 * d, 1)
+    assert vv.data_ptr() - kv.data_ptr() == 2 * d
+    return kv, vv
+
+
 class StridedDev(Dev):
     def __init__(self, w, layout):
         super().__init__(w)
-        self.k = strided(self.k, layout)
-        self.v = strided(self.v, layout)
+        if layout == "interleaved":
+            self.k, self.v = interleaved(self.k, self.v)
+        else:
+            self.k = strided(self.k, layout)
+            self.v = strided(self.v, layout)
 
 
 def sparse_spec(d, batch, roles, seed):
@@ -54,7 +69,7 @@ def sparse_spec(d, batch, roles, seed):
                         n_fac_div=8, roles=roles, sink=32, window=300, planted_frac=0.01, seed=seed)
 
 
-@pytest.mark.parametrize("layout", ["padded", "head_major"])
+@pytest.mark.parametrize("layout", ["padded", "head_major", "interleaved"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("rows", ["few", "many"])
 def test_role_split_step_on_strided_cache(layout, d, rows):
@@ -85,7 +100,7 @@ def test_role_split_step_on_strided_cache(layout, d, rows):
                     compare_window_row(w, b, g, o, role, w.spec.sink, w.spec.window)
 
 
-@pytest.mark.parametrize("layout", ["padded", "head_major"])
+@pytest.mark.parametrize("layout", ["padded", "head_major", "interleaved"])
 @pytest.mark.parametrize("batch", [2, 24])
 def test_shared_index_step_on_strided_cache(layout, batch):
     sp = WorkloadSpec(name="strided_shared", batch=batch, n_q_heads=32, n_kv_heads=8, head_dim=128, theta=5e5,
@@ -111,7 +126,7 @@ def test_strided_and_contiguous_caches_give_the_same_bits():
     roles = (ROLE_SPARSE,) * 4 + (ROLE_DENSE, ROLE_STREAM)
     w = make_workload(sparse_spec(128, 3, roles, 733))
     outs = []
-    for dv in (Dev(w), StridedDev(w, "padded"), StridedDev(w, "head_major")):
+    for dv in (Dev(w), StridedDev(w, "padded"), StridedDev(w, "head_major"), StridedDev(w, "interleaved")):
         step = SparseDecodeStep(dv.k, dv.v, dv.offsets, dv.max_len, dv.T, w.spec.n_q_heads, w.roles.tolist(),
                                 w.scale, idom=dv.idom, n_fac=int(w.n_fac_per_seq.max()),
                                 n_fac_per_seq=dv.n_fac_per_seq, n_fac_cap=int(w.n_fac_per_seq.max()),
