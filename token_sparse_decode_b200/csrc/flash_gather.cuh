@@ -41,6 +41,7 @@ __host__ __device__ constexpr int fd_groups(int nt) { return nt == 4 ? 2 : 4; }
 __host__ __device__ constexpr int fd_threads(int nt) { return 32 * nt * fd_groups(nt); }
 constexpr int kFdTS = 64;        // tokens per pipeline stage
 constexpr int kFdStages = 3;
+constexpr bool kFdWarpRing = true;  // role ranges, up to 8 query rows: warp-private rings (no block barrier per stage)
 constexpr int kFdPosCap = 1024;  // list positions staged in shared memory per CTA
 constexpr int kFdMaxSplits = 256; // splits per row (the combine stages their weights in shared memory)
 constexpr int kFdMaxCluster = 16;  // splits of a row merged through distributed shared memory
@@ -471,74 +472,149 @@ __global__ void __launch_bounds__(fd_threads(NT)) flash_gather_kernel(const Fdec
   for (int i = 0; i < KS; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // q rows 2*(lane%4) and +1
 
+  // (row r, dim dd) of a tile of `rows` rows stored as D/64 column halves of [rows x 128 B],
+  // 16-byte chunks XOR-swizzled by (r mod 8) (fd_tile_off for rows = kFdTS)
+  auto tile_off = [](int rows, int r, int dd) -> uint32_t {
+    const int half = dd >> 6;
+    const int cc = (dd & 63) >> 3;
+    return (uint32_t)(half * (rows * 128) + r * 128 + ((cc ^ (r & 7)) << 4));
+  };
+  // one 16-token sub-tile: rows r0 .. r0 + 15 of the K / V tiles at kt / vt, nv >= 1 of them valid
+  auto sub_tile = [&](uint32_t kt, uint32_t vt, int rows, int r0, int nv) {
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int r = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int dsel = (lane >> 4) * 8;
 #pragma unroll
-  for (int s = 0; s < ST - 1; ++s) issue_stage(s);
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(a, kt + tile_off(rows, r, ks * 16 + dsel));
+        mma_16816(s4, a, bq[ks][0], bq[ks][1]);
+      }
+    }
+    const int ta = lane >> 2, tb = ta + 8;
+    const float x0 = ta < nv ? s4[0] * p.scale_log2 : -INFINITY;
+    const float x1 = ta < nv ? s4[1] * p.scale_log2 : -INFINITY;
+    const float x2 = tb < nv ? s4[2] * p.scale_log2 : -INFINITY;
+    const float x3 = tb < nv ? s4[3] * p.scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: nv >= 1
+    const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+    const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+    const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+    l0 = l0 * al0 + p0 + p2;
+    l1 = l1 * al1 + p1 + p3;
+    m0 = mn0;
+    m1 = mn1;
+#pragma unroll
+    for (int i2 = 0; i2 < KS; ++i2) {
+      acc[i2][0] *= al0;
+      acc[i2][1] *= al1;
+      acc[i2][2] *= al0;
+      acc[i2][3] *= al1;
+    }
+    // P enters the PV product as hi + lo bf16 parts (p = hi + lo to ~2^-17), so the
+    // weights are not rounded to 8 bits: with few tokens that rounding alone reaches 2e-3.
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    const uint32_t l01 = pack_bf16x2(p0 - bf16lo(h01), p1 - bf16hi(h01));
+    const uint32_t l23 = pack_bf16x2(p2 - bf16lo(h23), p3 - bf16hi(h23));
+    const uint32_t pb0 = movmatrix_trans(h01), pb1 = movmatrix_trans(h23);
+    const uint32_t pl0 = movmatrix_trans(l01), pl1 = movmatrix_trans(l23);
+    {
+      const int r = r0 + (lane & 7) + (lane >> 4) * 8;
+      const int dsel = ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_trans(a, vt + tile_off(rows, r, mt * 16 + dsel));
+        mma_16816(acc[mt], a, pb0, pb1);
+        mma_16816(acc[mt], a, pl0, pl1);
+      }
+    }
+  };
 
-  for (int st = 0; st < nstages; ++st) {
-    cp_async_wait<ST - 2>();
-    __syncthreads();
-    issue_stage(st + ST - 1);
-    const uint32_t kt = sbase + (st % ST) * FdTile<D>::kStageBytes;
-    const uint32_t vt = kt + FdTile<D>::kTileBytes;
+  if (NT == 1 && kFdWarpRing && !p.list_mode) {
+    // Warp-private rings (role ranges, up to 8 query rows): warp tg owns the sub-tiles u = tg,
+    // tg + WT, ... of the chunk (16 tokens each; the same split as the block ring), copies their
+    // K / V rows itself into its own ring of ST slots and waits only for its own copies (a warp
+    // barrier, no block barrier): a warp goes on as soon as its rows have landed instead of
+    // waiting for the slowest copy of the stage.  Measured faster on the contiguous role ranges
+    // and not on scattered selections, which keep the block ring.
+    constexpr int kSubBytes = 16 * D * 2;  // one 16-row tile of K or V
+    const uint32_t wbase = sbase + warp * (ST * 2 * kSubBytes);
+    const int nsub = (ntok + 15) / 16;
+    const int my_n = nsub > tg ? (nsub - tg + WT - 1) / WT : 0;
+    auto issue_w = [&](int k) {
+      if (k < my_n) {
+        const int u = tg + WT * k;
+        const uint32_t kt = wbase + (k % ST) * 2 * kSubBytes;
+        const uint32_t vt = kt + kSubBytes;
 #pragma unroll
-    for (int i = 0; i < SUB / WT; ++i) {
-      const int u = tg + WT * i;
-      const int nv = ntok - (st * kFdTS + u * 16);  // valid tokens in this sub-tile
-      if (nv <= 0) break;                           // warp-uniform
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const int r = u * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int dsel = (lane >> 4) * 8;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t a[4];
-          ldsm_x4(a, kt + fd_tile_off(r, ks * 16 + dsel));
-          mma_16816(s4, a, bq[ks][0], bq[ks][1]);
+        for (int c = lane; c < 16 * CPR; c += 32) {
+          const int r = c / CPR, ch = c % CPR;
+          const int jj = u * 16 + r;  // entry within this CTA's chunk
+          bool ok = jj < ntok;
+          int pos = 0;
+          if (ok) {
+            const int j = j0 + jj;
+            if (pos_in_smem) {
+              pos = s_pos[jj];
+              if (pos < 0) {
+                ok = false;
+                pos = 0;
+              }
+            } else if (p.list_mode) {
+              pos = __ldg(lst + j);
+              if (pos < 0 || pos >= L) {
+                if (ch == 0) record_error(kCheckPosition, b, g, pos);
+                ok = false;
+                pos = 0;
+              }
+            } else {
+              pos = j < ra ? j : rb + (j - ra);
+              if (ring) pos = ring_slot(pos, p.ring_sink, p.ring_window);
+            }
+          }
+          const int64_t eo = (int64_t)pos * p.stride_tok + ch * 8;
+          const uint32_t so = tile_off(16, r, ch * 8);
+          cp_async_16(kt + so, kbase + eo, ok);
+          cp_async_16(vt + so, vbase + eo, ok);
         }
       }
-      const int ta = lane >> 2, tb = ta + 8;
-      const float x0 = ta < nv ? s4[0] * p.scale_log2 : -INFINITY;
-      const float x1 = ta < nv ? s4[1] * p.scale_log2 : -INFINITY;
-      const float x2 = tb < nv ? s4[2] * p.scale_log2 : -INFINITY;
-      const float x3 = tb < nv ? s4[3] * p.scale_log2 : -INFINITY;
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+      cp_async_commit();
+    };
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: nv >= 1
-      const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-      const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-      const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-      l0 = l0 * al0 + p0 + p2;
-      l1 = l1 * al1 + p1 + p3;
-      m0 = mn0;
-      m1 = mn1;
+    for (int k = 0; k < ST - 1; ++k) issue_w(k);
+    for (int k = 0; k < my_n; ++k) {
+      issue_w(k + ST - 1);     // into the slot this warp read at k - 1
+      cp_async_wait<ST - 1>();  // this lane's copies of sub-tile k have landed
+      __syncwarp();             // and so have the other lanes' (the tile mixes them)
+      const int u = tg + WT * k;
+      const uint32_t kt = wbase + (k % ST) * 2 * kSubBytes;
+      sub_tile(kt, kt + kSubBytes, 16, 0, ntok - u * 16);
+      __syncwarp();             // every lane is done with the slot before it is refilled
+    }
+  } else {
 #pragma unroll
-      for (int i2 = 0; i2 < KS; ++i2) {
-        acc[i2][0] *= al0;
-        acc[i2][1] *= al1;
-        acc[i2][2] *= al0;
-        acc[i2][3] *= al1;
-      }
-      // P enters the PV product as hi + lo bf16 parts (p = hi + lo to ~2^-17), so the
-      // weights are not rounded to 8 bits: with few tokens that rounding alone reaches 2e-3.
-      const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-      const uint32_t l01 = pack_bf16x2(p0 - bf16lo(h01), p1 - bf16hi(h01));
-      const uint32_t l23 = pack_bf16x2(p2 - bf16lo(h23), p3 - bf16hi(h23));
-      const uint32_t pb0 = movmatrix_trans(h01), pb1 = movmatrix_trans(h23);
-      const uint32_t pl0 = movmatrix_trans(l01), pl1 = movmatrix_trans(l23);
-      {
-        const int r = u * 16 + (lane & 7) + (lane >> 4) * 8;
-        const int dsel = ((lane >> 3) & 1) * 8;
+    for (int s = 0; s < ST - 1; ++s) issue_stage(s);
+
+    for (int st = 0; st < nstages; ++st) {
+      cp_async_wait<ST - 2>();
+      __syncthreads();
+      issue_stage(st + ST - 1);
+      const uint32_t kt = sbase + (st % ST) * FdTile<D>::kStageBytes;
+      const uint32_t vt = kt + FdTile<D>::kTileBytes;
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          uint32_t a[4];
-          ldsm_x4_trans(a, vt + fd_tile_off(r, mt * 16 + dsel));
-          mma_16816(acc[mt], a, pb0, pb1);
-          mma_16816(acc[mt], a, pl0, pl1);
-        }
+      for (int i = 0; i < SUB / WT; ++i) {
+        const int u = tg + WT * i;
+        const int nv = ntok - (st * kFdTS + u * 16);  // valid tokens in this sub-tile
+        if (nv <= 0) break;                           // warp-uniform
+        sub_tile(kt, vt, kFdTS, u * 16, nv);
       }
     }
   }
